@@ -1,0 +1,241 @@
+"""Oracle for SureLock's lock test, active-set bookkeeping and sampler.
+Test infrastructure (see the package docstring).
+
+Sources (the pages on "Stopping Computation for Converged Tokens in Masked
+Diffusion-LM Decoding"):
+  * Two disjoint sets per step: the active set A_t, which is computed, and the
+    locked set L_t, which is skipped but whose K/V stay cached; the active set
+    only shrinks (Paper-Notes, "Method: overall framework" and "permanent
+    locking", design motivation; "Key findings": M_t decreases monotonically).
+  * Lock criterion D_t^(i) = KL(p_t^(i) || p_{t-1}^(i)) <= eps (Paper-Notes,
+    "lock criterion: step-to-step KL"; gist.science/it section 2 "Criterio di
+    Blocco"), tested at unmasked positions (Abstract: "when the posterior at an
+    unmasked position has stabilized across steps").
+  * Optional confidence gate u_t^(i) = 1 - max_v p_t^(i)(v) <= q_m(u_t)
+    (Paper-Notes, "optional confidence gate"), q_m a percentile of u among the
+    active tokens (gist.science/it section 2, "Filtro di Confidenza").
+  * After the lock step t*, the posterior stays frozen: p_hat_t = p_{t*}
+    (Paper-Notes, "permanent locking", core idea).
+  * The comparison sampler is "the same sampler without locking" (Abstract).
+
+Readings where the pages are silent (listed in the design doc):
+  R4  "unmasked" means not [MASK] in the step's input x_t; prompt positions count.
+  R5  no previous posterior at t = 0, so nothing locks at t = 0.
+  R6  eps <= 0 disables locking (the pages' test D <= eps would fire at D = 0).
+  R7  D is clamped at 0 (rounding can make it slightly negative).
+  R8  q_m is the lower order statistic: sorted(u over A_t)[floor(q (|A_t|-1))],
+      over all active rows of the sequence, masked or not; comparison <=.
+  R9  ties: argmax takes the lowest vocab id, unmasking takes the lowest
+      position, compaction keeps ascending position order.
+  R11 semi-autoregressive blocks over the generated region; each step unmasks
+      the k highest-confidence masked positions of the current block, where
+      confidence and prediction are taken over v != [MASK].
+  Scripted mode: instead of the KL test, lock the eligible (unmasked, with a
+  previous posterior) active rows in ascending (D, position) order until the
+  active count reaches a target.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import numpy as np
+
+from . import model as om
+
+
+def log_softmax(z: np.ndarray) -> np.ndarray:
+    """log p = z - logsumexp(z) over the last axis."""
+    m = np.max(z, axis=-1, keepdims=True)
+    return z - (m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True)))
+
+
+def kl_rows(lp_cur: np.ndarray, lp_prev: np.ndarray) -> np.ndarray:
+    """D = max(0, sum_v p_cur(v) (log p_cur(v) - log p_prev(v))) per row."""
+    p = np.exp(lp_cur)
+    return np.maximum(0.0, np.sum(p * (lp_cur - lp_prev), axis=-1))
+
+
+def uncertainty(lp_cur: np.ndarray) -> np.ndarray:
+    """u = 1 - max_v p(v) per row (all vocab entries, [MASK] included)."""
+    return 1.0 - np.exp(np.max(lp_cur, axis=-1))
+
+
+def prediction(lp_cur: np.ndarray, mask_id: int):
+    """(conf, pred): the largest probability over v != mask_id and its lowest
+    index; this is what the sampler unmasks with."""
+    lp = np.array(lp_cur, copy=True)
+    lp[..., mask_id] = -np.inf
+    pred = np.argmax(lp, axis=-1)           # first occurrence = lowest id
+    conf = np.exp(np.take_along_axis(lp, pred[..., None], axis=-1)[..., 0])
+    return conf, pred.astype(np.int32)
+
+
+def gate_threshold(u_active: np.ndarray, q: float) -> float:
+    """q-quantile of u over the active rows, lower order statistic."""
+    m = u_active.shape[0]
+    if m == 0:
+        return np.inf
+    r = int(np.floor(q * (m - 1)))
+    return np.sort(u_active, kind="stable")[r]
+
+
+def lock_decision(D, u, masked, has_prev, eps: float, gate_q: float, thr):
+    """lock_j = eps>0 and not masked_j and has_prev_j and D_j<=eps and
+    (gate off or u_j <= thr)."""
+    if eps <= 0:
+        return np.zeros(D.shape, dtype=bool)
+    ok = (~masked.astype(bool)) & has_prev.astype(bool) & (D <= eps)
+    if gate_q >= 0:
+        ok &= (u <= thr)
+    return ok
+
+
+def scripted_locks(D, masked, has_prev, pos, n_lock: int):
+    """Lock the n_lock eligible rows with the smallest (D, position)."""
+    elig = (~masked.astype(bool)) & has_prev.astype(bool)
+    idx = np.nonzero(elig)[0]
+    order = idx[np.lexsort((pos[idx], D[idx]))]
+    lock = np.zeros(D.shape, dtype=bool)
+    lock[order[:max(0, n_lock)]] = True
+    return lock
+
+
+def compact(act: np.ndarray, lock: np.ndarray) -> np.ndarray:
+    """Stable removal of the locked rows from the active list."""
+    return act[~lock]
+
+
+def unmask_select(pos: np.ndarray, conf: np.ndarray, masked_rows: np.ndarray,
+                  lo: int, hi: int, k: int) -> np.ndarray:
+    """Indices (into the active rows) of the k masked rows in [lo, hi) with the
+    highest confidence, ties to the lower position."""
+    cand = np.nonzero(masked_rows.astype(bool) & (pos >= lo) & (pos < hi))[0]
+    order = cand[np.lexsort((pos[cand], -conf[cand]))]
+    return order[:k]
+
+
+@dataclasses.dataclass
+class State:
+    """Sampler state for a batch of sequences."""
+    tokens: np.ndarray        # [B, N] int32
+    masked: np.ndarray        # [B, N] bool
+    act: List[np.ndarray]     # per sequence: ascending active positions
+    locked: np.ndarray        # [B, N] bool
+    lock_t: np.ndarray        # [B, N] int32, -1 if never locked
+    has_prev: np.ndarray      # [B, N] bool
+    ck: np.ndarray            # [B, L, N, d]
+    cv: np.ndarray            # [B, L, N, d]
+    lp_prev: np.ndarray       # [B, N, V]  last posterior (frozen p_hat for locked rows)
+
+    def copy(self) -> "State":
+        return State(self.tokens.copy(), self.masked.copy(), [a.copy() for a in self.act],
+                     self.locked.copy(), self.lock_t.copy(), self.has_prev.copy(),
+                     self.ck.copy(), self.cv.copy(), self.lp_prev.copy())
+
+
+def init_state(shape, tokens: np.ndarray, masked: np.ndarray, dtype=np.float64) -> State:
+    B, N = tokens.shape
+    L, d, V = shape.n_layers, shape.d_model, shape.vocab
+    return State(tokens=tokens.astype(np.int32).copy(), masked=masked.astype(bool).copy(),
+                 act=[np.arange(N, dtype=np.int32) for _ in range(B)],
+                 locked=np.zeros((B, N), dtype=bool),
+                 lock_t=np.full((B, N), -1, dtype=np.int32),
+                 has_prev=np.zeros((B, N), dtype=bool),
+                 ck=np.zeros((B, L, N, d), dtype=dtype), cv=np.zeros((B, L, N, d), dtype=dtype),
+                 lp_prev=np.zeros((B, N, V), dtype=dtype))
+
+
+def lock_test(lp: np.ndarray, lp_prev: np.ndarray, has_prev: np.ndarray,
+              masked: np.ndarray, pos: np.ndarray, shape, setup, t: int,
+              n_active_target: Optional[int] = None):
+    """The sure test of one sequence's active rows.  Returns a dict with D, u,
+    conf, pred, thr and the lock flags."""
+    D = np.full(lp.shape[0], np.inf, dtype=lp.dtype)
+    hp = has_prev.astype(bool)
+    if np.any(hp):
+        D[hp] = kl_rows(lp[hp], lp_prev[hp])
+    u = uncertainty(lp)
+    conf, pred = prediction(lp, shape.mask_id)
+    thr = gate_threshold(u, setup.gate_q) if setup.gate_q >= 0 else np.inf
+    if setup.scripted:
+        target = setup.scripted_target(t) if n_active_target is None else n_active_target
+        lock = scripted_locks(D, masked, hp, pos, lp.shape[0] - target)
+    else:
+        lock = lock_decision(D, u, masked, hp, setup.eps, setup.gate_q, thr)
+    return {"D": D, "u": u, "conf": conf, "pred": pred, "thr": thr, "lock": lock}
+
+
+def step(shape, w: dict, st: State, setup, t: int, record_block_inputs: bool = False):
+    """One SureLock denoising step t on every sequence, updating `st` in place.
+
+    Order: forward on A_t (fresh K/V scattered into C) -> log-softmax -> sure
+    test on the mask flags at the start of the step -> unmask the top-k of the
+    current block -> record p_t for the active rows (frozen for those that lock)
+    -> remove the locked rows from A_t.  Returns one record per sequence."""
+    out = []
+    lo, hi = setup.block_bounds(t)
+    for b in range(st.tokens.shape[0]):
+        A = st.act[b]
+        blk = [] if record_block_inputs else None
+        z = om.forward_active(shape, w, st.tokens[b], A, st.ck[b], st.cv[b], blk)
+        lp = log_softmax(z)
+        masked_rows = st.masked[b, A].copy()
+        rec = lock_test(lp, st.lp_prev[b, A], st.has_prev[b, A], masked_rows, A,
+                        shape, setup, t)
+        sel = unmask_select(A, rec["conf"], masked_rows, lo, hi, setup.tokens_per_step)
+        st.tokens[b, A[sel]] = rec["pred"][sel]
+        st.masked[b, A[sel]] = False
+        st.lp_prev[b, A] = lp
+        st.has_prev[b, A] = True
+        lk = rec["lock"]
+        st.locked[b, A[lk]] = True
+        st.lock_t[b, A[lk]] = t
+        st.act[b] = compact(A, lk)
+        rec.update({"z": z, "lp": lp, "pos": A, "unmasked": A[sel], "block_inputs": blk})
+        out.append(rec)
+    return out
+
+
+def surelock_sampler(shape, w: dict, tokens: np.ndarray, masked: np.ndarray, setup,
+                     dtype=np.float64, keep_records: bool = False):
+    """Full SureLock decode.  Returns (final tokens, final log-probs [B, N, V],
+    active counts per step [T+1, B], per-step records if keep_records)."""
+    st = init_state(shape, tokens, masked, dtype)
+    counts = [[len(a) for a in st.act]]
+    recs = []
+    for t in range(setup.steps):
+        r = step(shape, w, st, setup, t)
+        counts.append([len(a) for a in st.act])
+        if keep_records:
+            recs.append(r)
+    return st.tokens, st.lp_prev, np.array(counts), (recs if keep_records else None), st
+
+
+def plain_sampler(shape, w: dict, tokens: np.ndarray, masked: np.ndarray, setup):
+    """The same sampler without locking: every step runs the full denoiser on all
+    N positions (no active set, no cache).  Returns (final tokens, final
+    log-probs [B, N, V])."""
+    tok = tokens.astype(np.int32).copy()
+    msk = masked.astype(bool).copy()
+    B, N = tok.shape
+    lp = None
+    pos = np.arange(N, dtype=np.int32)
+    lps = [None] * B
+    for t in range(setup.steps):
+        lo, hi = setup.block_bounds(t)
+        for b in range(B):
+            lp = log_softmax(om.forward_full(shape, w, tok[b]))
+            conf, pred = prediction(lp, shape.mask_id)
+            sel = unmask_select(pos, conf, msk[b], lo, hi, setup.tokens_per_step)
+            tok[b, sel] = pred[sel]
+            msk[b, sel] = False
+            lps[b] = lp
+    return tok, np.stack(lps)
+
+
+def flops_per_step(shape, m_rows: int, n_ctx_rows: int) -> float:
+    """Algorithmic FLOPs of one step on m_rows active rows attending to
+    n_ctx_rows keys: 2 M (L (4 d^2 + 3 d f) + V d) + 4 L M N d."""
+    d, f, V, L = shape.d_model, shape.d_ffn, shape.vocab, shape.n_layers
+    return 2.0 * m_rows * (L * (4 * d * d + 3 * d * f) + V * d) + 4.0 * L * m_rows * n_ctx_rows * d
