@@ -1,0 +1,281 @@
+/*
+ * surelock.h -- C ABI of libsurelock.so: the SureLock decoding step on B200 (sm_100a).
+ *
+ * SureLock ("Stopping Computation for Converged Tokens in Masked Diffusion-LM
+ * Decoding", Oba, Bollegala, Kaneko, Okazaki) keeps two disjoint sets of
+ * positions while a masked diffusion LM denoises: the active set A_t, which the
+ * denoiser computes, and the locked set L_t, whose rows skip the query
+ * projection and the FFN but keep their attention keys/values cached so that
+ * active rows still attend to them (Paper-Notes, "Method: overall framework" and
+ * "Key design: permanent locking"; Abstract).  A position locks once its
+ * posterior is stable: D_t = KL(p_t || p_{t-1}) <= eps at an unmasked position
+ * (Paper-Notes, "lock criterion: step-to-step KL"; Abstract), optionally also
+ * requiring u_t = 1 - max_v p_t(v) <= q_m(u_t), a quantile of u over the active
+ * tokens (Paper-Notes, "optional confidence gate"; gist.science/it section 2,
+ * "Filtro di Confidenza").  The active set only shrinks (Paper-Notes, "Key
+ * findings").
+ *
+ * Conventions for every entry point:
+ *  - Pointers named d_* are device pointers (cudaMalloc'd or torch-allocated on
+ *    the current device); h_* are host pointers.  `stream` is a cudaStream_t
+ *    passed as void* (NULL = the legacy default stream).
+ *  - Work is enqueued asynchronously on `stream`.  Argument and state errors are
+ *    detected on the host before anything is enqueued and return SL_ERR_INVALID
+ *    or SL_ERR_STATE; CUDA launch errors return SL_ERR_CUDA.  sl_last_error()
+ *    returns a message for the calling thread's last non-OK status.
+ *  - Layouts are row-major.  Weights are [out_features, in_features].  Token
+ *    positions of sequence b are b * n_ctx + i, i in [0, n_ctx).
+ *  - Ownership: the caller owns weights, tokens, logits and per-row outputs;
+ *    the model only borrows weight pointers (they must outlive it).  Objects
+ *    created here (model, KV cache, active list, sampler) own their device
+ *    memory and free it on destroy.
+ *  - An object is used from one stream at a time.
+ */
+#ifndef SURELOCK_H
+#define SURELOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SL_MAX_BATCH 64
+
+typedef enum sl_status {
+  SL_OK = 0,
+  SL_ERR_INVALID = 1,     /* bad argument: null pointer, size out of range, unsupported shape */
+  SL_ERR_CUDA = 2,        /* a CUDA runtime call or launch failed */
+  SL_ERR_OOM = 3,         /* device or pinned allocation failed */
+  SL_ERR_UNSUPPORTED = 4, /* valid request this build does not implement */
+  SL_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait and flagged it */
+  SL_ERR_STATE = 6        /* call out of order (e.g. stepping a finished sampler) */
+} sl_status;
+
+typedef enum sl_dtype { SL_F32 = 0, SL_BF16 = 1 } sl_dtype;
+
+/* Denoiser shape.  head_dim * n_heads must equal d_model.  dtype selects fp32
+ * weights/activations/cache/logits (SIMT path) or bf16 (tensor-core path;
+ * d_model, d_ffn and vocab must be multiples of 128, head_dim 128). */
+typedef struct sl_config {
+  int n_layers, d_model, n_heads, head_dim, d_ffn, vocab, mask_id;
+  float rms_eps, rope_theta;
+  int dtype; /* sl_dtype */
+} sl_config;
+
+/* One transformer block: RMSNorm gains [d], Wq/Wk/Wv/Wo [d, d], W_gate/W_up [f, d],
+ * W_down [d, f]; all in the model dtype. */
+typedef struct sl_layer_weights {
+  const void *attn_norm, *wq, *wk, *wv, *wo, *ffn_norm, *w_gate, *w_up, *w_down;
+} sl_layer_weights;
+
+/* tok_emb [V, d], final_norm [d], lm_head [V, d]; layers: host array of n_layers. */
+typedef struct sl_weights {
+  const void *tok_emb, *final_norm, *lm_head;
+  const sl_layer_weights *layers;
+} sl_weights;
+
+typedef struct sl_model sl_model;
+typedef struct sl_kv_cache sl_kv_cache;
+typedef struct sl_active sl_active;
+typedef struct sl_sampler sl_sampler;
+
+const char *sl_last_error(void);
+const char *sl_version(void);
+
+/* ---------------------------------------------------------------- model --- */
+
+/* Borrow device weights and build the per-model launch state (TMA descriptors
+ * for the bf16 path).  Fails with SL_ERR_INVALID on an inconsistent config. */
+sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, sl_model **out);
+void sl_model_destroy(sl_model *m);
+
+/* --------------------------------------------------------------- KV cache --- */
+
+/* The cache C of the pages (Paper-Notes, "permanent locking": K^all[L_t] <-
+ * C.k[L_t]; gist.science/it section 2 "Azione di Blocco": K and V of a locked
+ * token are kept for every layer).  Per layer, k and v are [batch][n_ctx][d_model]
+ * in the model dtype (head h occupies columns h*head_dim .. +head_dim; k is stored
+ * after the rotary embedding).  The object also owns the activation workspace
+ * for up to batch * n_ctx active rows.  Contents start at zero. */
+sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx, sl_kv_cache **out);
+sl_status sl_kv_cache_reset(sl_kv_cache *c, void *stream);
+/* Device pointers of layer `layer`'s k and v (for inspection and teacher forcing). */
+sl_status sl_kv_cache_view(const sl_kv_cache *c, int layer, void **d_k, void **d_v);
+void sl_kv_cache_destroy(sl_kv_cache *c);
+
+/* ------------------------------------------------------------ active set --- */
+
+/* A_t for a batch: on the device, a flat ascending list of positions
+ * rows[0..M) (entry b*n_ctx + i) and per-sequence offsets seq_off[0..batch]
+ * (seq_off[batch] = M).  A_0 holds every position.  The host keeps a mirror of
+ * the per-sequence counts, refreshed by sl_active_counts. */
+sl_status sl_active_create(int batch, int n_ctx, sl_active **out);
+/* A_0 = {0..n_ctx-1} for every sequence. */
+sl_status sl_active_reset(sl_active *a, void *stream);
+/* Teacher forcing: h_counts[batch], h_pos = the concatenated ascending local
+ * positions (i in [0, n_ctx)) of every sequence.  SL_ERR_INVALID if a list is
+ * not strictly ascending or out of range. */
+sl_status sl_active_load(sl_active *a, const int32_t *h_counts, const int32_t *h_pos, void *stream);
+/* Per-sequence counts |A_t^b| into h_counts[batch]; waits for the last update
+ * enqueued on the active set to finish. */
+sl_status sl_active_counts(sl_active *a, int32_t *h_counts);
+sl_status sl_active_view(const sl_active *a, int32_t **d_rows, int32_t **d_seq_off);
+void sl_active_destroy(sl_active *a);
+
+/* --------------------------------------------------------- the hot path --- */
+
+/* One denoiser pass on the active rows only (Abstract: locked positions skip
+ * the query projection and FFN; attention cost O(M N d) instead of O(N^2 d),
+ * gist.science/nl section 2 "Complexiteitsvermindering"):
+ *   h = E[x[rows]]; per layer: a = RMSNorm(h); q,k,v = a Wq^T, a Wk^T, a Wv^T;
+ *   RoPE(q, k) at the absolute position; C.k/C.v[layer][rows] <- k, v;
+ *   h += Attn(q, C.k[layer][seq], C.v[layer][seq]) Wo^T  (all n_ctx keys);
+ *   b = RMSNorm(h); h += (silu(b Wg^T) * (b Wu^T)) Wd^T;
+ *   logits[rows] = RMSNorm(h) W_out^T.
+ * d_tokens: [batch][n_ctx] int32 ids x_t.  d_logits: [batch][n_ctx][vocab] in the
+ * model dtype; only the active rows are written.  The cache must have been
+ * created for the same batch and n_ctx as the active set. */
+sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
+                  void *d_logits, void *stream);
+
+typedef struct sl_lock_params {
+  float eps;             /* KL threshold; eps <= 0 disables locking */
+  float gate_q;          /* confidence-gate quantile in [0,1]; < 0 = gate off */
+  int has_prev;          /* 0 at t = 0: no previous posterior, nothing locks */
+  int scripted_target;   /* < 0: the KL test.  >= 0: scripted mode, lock eligible
+                            rows in ascending (D, position) order until each
+                            sequence has this many active rows */
+} sl_lock_params;
+
+/* The sure test on the active rows (Paper-Notes, "lock criterion" and
+ * "optional confidence gate"; Abstract, "unmasked position"):
+ *   lse_j = logsumexp(z_cur[row_j]);  log p = z - lse
+ *   D_j = max(0, sum_v p_cur (log p_cur - log p_prev))
+ *       = max(0, E_pcur[z_cur - z_prev] - lse_cur + lse_prev)
+ *   u_j = 1 - max_v p_cur(v);  conf_j / argmax_j over v != mask_id (lowest id on ties)
+ *   thr_b = sorted(u over A_t^b)[floor(gate_q (M_b - 1))]
+ *   lock_j = eps > 0 && !masked[row_j] && has_prev && D_j <= eps && (gate off || u_j <= thr_b)
+ * d_logits_cur/prev: [batch*n_ctx][vocab] (dtype), read at the active rows;
+ * d_lse_prev / d_lse_cur: [batch*n_ctx] fp32 (lse_cur written at active rows);
+ * d_masked: [batch*n_ctx] u8 mask flags at the start of the step.
+ * Outputs indexed by active-row index j in [0, M): d_kl, d_unc, d_conf (fp32),
+ * d_argmax (int32), d_lock (u8).  Needs vocab % 8 == 0 for bf16. */
+sl_status sl_kl_lock(sl_active *a, int vocab, int mask_id, int logits_dtype,
+                     const void *d_logits_cur, const void *d_logits_prev,
+                     const float *d_lse_prev, float *d_lse_cur, const uint8_t *d_masked,
+                     const sl_lock_params *p, float *d_kl, float *d_unc, float *d_conf,
+                     int32_t *d_argmax, uint8_t *d_lock, void *stream);
+
+/* Sampler step: among the masked active rows with local position in
+ * [block_lo, block_hi), unmask the k with the highest confidence (ties to the
+ * lower position): tokens[row] = argmax, masked[row] = 0.  This is the
+ * unmodified sampler the pages compare against (Abstract: "the same sampler
+ * without locking"). */
+sl_status sl_unmask_topk(sl_active *a, const float *d_conf, const int32_t *d_argmax,
+                         int block_lo, int block_hi, int k, int32_t *d_tokens,
+                         uint8_t *d_masked, void *stream);
+
+/* Stable compaction: A_{t+1} = [row_j in A_t : !lock_j] in ascending order, and
+ * locked[row] = 1, lock_t[row] = step for each locked row (Paper-Notes,
+ * "permanent locking": the active set only shrinks).  d_lock is indexed by
+ * active-row index; d_locked/d_lock_t are [batch*n_ctx]. */
+sl_status sl_compact_active(sl_active *a, const uint8_t *d_lock, uint8_t *d_locked,
+                            int32_t *d_lock_t, int step, void *stream);
+
+/* One transformer block of layer `layer` on the active rows, the body of
+ * sl_step's layer loop: d_h [M][d_model] fp32 holds the block inputs of the
+ * active rows (in active-list order) and is overwritten with the block outputs;
+ * C.k/C.v[layer] rows of the active positions receive the fresh k, v.  Frozen
+ * block inputs of locked rows are never touched (gist.science/it section 2,
+ * "Azione di Blocco"). */
+sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, float *d_h,
+                           void *stream);
+
+/* Attention of the active rows over all n_ctx cached keys of their sequence in
+ * layer `layer`: d_q [M][d_model] (after the rotary embedding), d_o [M][d_model],
+ * both in the model dtype. */
+sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, const void *d_q,
+                       void *d_o, void *stream);
+
+/* The tensor-core GEMM of the bf16 path, C = A[M,K] * B[N,K]^T (bf16 operands,
+ * fp32 accumulation), exposed for kernel-level checks and benchmarks.
+ *   SL_GEMM_STORE : out bf16 [.][ldo], row r written to row d_row_map[r] (or r)
+ *   SL_GEMM_RESID : out fp32 [M][ldo] += C
+ *   SL_GEMM_SWIGLU: d_b = W_gate [F][K], d_b2 = W_up [F][K], N = 2F;
+ *                   out bf16 [M][ldo] = silu(A W_gate^T) * (A W_up^T)
+ *   SL_GEMM_ACCUM : out fp32 [M][ldo] += C (atomic; with d_b2, gate/up halves
+ *                   accumulate into columns [0,F) and [F,2F))
+ * bn (64/128/256) and splits (>= 1, RESID/ACCUM only) pick the tiling; bn = 0
+ * lets the library choose.  K % 64 == 0, N % bn == 0, pointers 16-byte aligned. */
+enum { SL_GEMM_STORE = 0, SL_GEMM_RESID = 1, SL_GEMM_SWIGLU = 2, SL_GEMM_ACCUM = 3 };
+sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b, const void *d_b2,
+                       int N, void *d_out, int ldo, const int32_t *d_row_map, int bn, int splits,
+                       void *stream);
+
+/* ---------------------------------------------------------------- sampler --- */
+
+/* Semi-autoregressive SureLock decode driven by the library: prompt_len given
+ * tokens then gen_len [MASK] tokens; gen region split in blocks of block_len,
+ * steps/(gen_len/block_len) steps per block, tokens_per_step unmasked per step. */
+typedef struct sl_sampler_params {
+  int prompt_len, gen_len, steps, block_len, tokens_per_step;
+  float eps, gate_q;
+  int scripted;          /* 1: scripted lock schedule, M decays linearly to 10% of N */
+} sl_sampler_params;
+
+/* Device buffers owned by a sampler (for inspection / teacher forcing). */
+typedef struct sl_sampler_state {
+  int32_t *tokens;       /* [B][N] */
+  uint8_t *masked;       /* [B][N] */
+  uint8_t *locked;       /* [B][N] */
+  int32_t *lock_t;       /* [B][N], -1 if unlocked */
+  void *logits[2];       /* [B][N][V] ping-pong, step t writes logits[t % 2] */
+  float *lse[2];         /* [B][N] */
+  float *kl, *unc, *conf;/* [B*N] by active-row index */
+  int32_t *argmax;       /* [B*N] */
+  uint8_t *lock;         /* [B*N] */
+  sl_kv_cache *cache;
+  sl_active *active;
+  int t;                 /* next step to run */
+  int batch, n_ctx;
+} sl_sampler_state;
+
+sl_status sl_sampler_create(sl_model *m, int batch, const sl_sampler_params *p, sl_sampler **out);
+/* Reset state for a new decode from device prompts [batch][prompt_len]. */
+sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, void *stream);
+/* One denoising step t: sl_step, sl_kl_lock, sl_unmask_topk, sl_compact_active. */
+sl_status sl_sampler_step(sl_sampler *s, void *stream);
+/* Whole decode from host prompts [batch][prompt_len] to host tokens
+ * [batch][n_ctx]; both copies are inside the call. */
+sl_status sl_sampler_generate(sl_sampler *s, const int32_t *h_prompts, int32_t *h_tokens,
+                              void *stream);
+sl_status sl_sampler_get_state(const sl_sampler *s, sl_sampler_state *out);
+void sl_sampler_destroy(sl_sampler *s);
+
+/* ------------------------------------------------------------ diagnostics --- */
+
+/* Per kernel class device time, measured with CUDA events around every launch
+ * of that class while timing is enabled on the model, and the algorithmic work
+ * of those launches (bytes: operands read + results written once; flops:
+ * 2 per multiply-add). */
+enum { SL_K_GEMM = 0, SL_K_ATTN = 1, SL_K_LOCK = 2, SL_K_OTHER = 3, SL_K_COUNT = 4 };
+typedef struct sl_timing {
+  double ms[SL_K_COUNT];
+  double bytes[SL_K_COUNT];
+  double flops[SL_K_COUNT];
+  long long launches[SL_K_COUNT];
+} sl_timing;
+sl_status sl_timing_enable(sl_model *m, int enable);
+/* Synchronises the recorded events, returns the sums since the last reset. */
+sl_status sl_timing_read(sl_model *m, sl_timing *out, int reset);
+
+/* Device error word set by kernels that gave up a bounded wait: returns
+ * SL_ERR_TIMEOUT (and clears it if `clear`) or SL_OK.  Synchronises the device. */
+sl_status sl_device_check(int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SURELOCK_H */

@@ -1,0 +1,72 @@
+"""Helpers shared by the GPU parity tests: moving seeded inputs to the device,
+reading device state back for the oracle, and ambiguity-aware comparison of
+integer decisions.
+
+Tolerances (from the target stated for this path):
+  * logits: max abs 1e-4 for fp32 models, 5e-2 for bf16 models;
+  * final log-probs: 2e-2;
+  * index, lock-set and compaction outputs: bit-exact, except decisions whose
+    deciding quantity lies inside the rounding band: |D - eps| < 1e-4,
+    |u - thr| < 1e-4, or two unmasking candidates whose confidences differ by
+    less than 1e-5 relative (fp32 exp/log rounding of conf = exp(z - lse) with
+    lse ~ 16 is a few 1e-6 relative).  Those are counted and reported.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import workloads as wl
+from oracle import model as om
+from oracle import surelock as osl
+
+LOGIT_TOL = {"f32": 1e-4, "bf16": 5e-2}
+FINAL_LP_TOL = 2e-2
+BAND_D = 1e-4
+BAND_U = 1e-4
+BAND_CONF_REL = 1e-5
+
+
+def weights_to_device(w_np: dict, dtype: str, device) -> dict:
+    """numpy fp32 weights -> contiguous device tensors (bf16 rounds to nearest)."""
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+
+    def t(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=tdt)
+
+    out = {k: t(v) for k, v in w_np.items() if k != "layers"}
+    out["layers"] = [{k: t(v) for k, v in lw.items()} for lw in w_np["layers"]]
+    return out
+
+
+def weights_for_oracle(w_dev: dict) -> dict:
+    """The device weights exactly as stored (bf16 values upcast), in float64."""
+    def h(t):
+        return t.float().cpu().numpy().astype(np.float64)
+    out = {k: h(v) for k, v in w_dev.items() if k != "layers"}
+    out["layers"] = [{k: h(v) for k, v in lw.items()} for lw in w_dev["layers"]]
+    return out
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def compare_locks(gpu_lock, ora_lock, D, u, eps, thr=None, gate=False):
+    """(mismatches, ambiguous) between lock flags; D, u from the oracle."""
+    gpu_lock = np.asarray(gpu_lock).astype(bool)
+    ora_lock = np.asarray(ora_lock).astype(bool)
+    amb = np.abs(D - eps) < BAND_D
+    if gate and thr is not None and np.isfinite(thr):
+        amb |= np.abs(u - thr) < BAND_U
+    diff = gpu_lock != ora_lock
+    return int(np.sum(diff & ~amb)), int(np.sum(diff & amb))
+
+
+def conf_ambiguous(conf: np.ndarray, chosen: np.ndarray, cands: np.ndarray) -> bool:
+    """True if the k-th and (k+1)-th candidate confidences are within the band."""
+    if len(cands) <= len(chosen):
+        return False
+    c = np.sort(conf[cands])[::-1]
+    k = len(chosen)
+    return abs(c[k - 1] - c[k]) <= BAND_CONF_REL * max(abs(c[k - 1]), 1e-30)

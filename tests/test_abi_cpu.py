@@ -1,0 +1,66 @@
+"""The C ABI library loads without a GPU and exports everything the header
+declares; host-side argument checks reject bad calls before touching CUDA."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "surelock.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = set(re.findall(r"\b(sl_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_locking_b200 import _abi
+    if not os.path.exists(_abi.LIB_PATH):
+        from token_locking_b200 import build
+        build.build()
+    return _abi.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from token_locking_b200 import _abi
+    declared = _declared()
+    assert len(declared) >= 25
+    for name in sorted(declared):
+        assert hasattr(lib, name), f"{name} declared in include/surelock.h but not exported"
+        assert name in _abi.SIGNATURES, f"{name} has no ctypes signature"
+    assert set(_abi.SIGNATURES) == declared
+
+
+def test_version_and_error_strings(lib):
+    assert b"sm_100a" in lib.sl_version()
+    assert isinstance(lib.sl_last_error(), bytes)
+
+
+def test_host_side_argument_checks(lib):
+    from token_locking_b200 import _abi as A
+    out = C.c_void_p()
+    assert lib.sl_model_create(None, None, C.byref(out)) == A.SL_ERR_INVALID
+    cfg = A.Config(2, 64, 4, 15, 256, 512, 511, 1e-5, 1e4, A.SL_F32)   # 4 * 15 != 64
+    w = A.Weights()
+    assert lib.sl_model_create(C.byref(cfg), C.byref(w), C.byref(out)) == A.SL_ERR_INVALID
+    assert b"head_dim" in lib.sl_last_error()
+    cfg = A.Config(2, 64, 4, 16, 256, 512, 512, 1e-5, 1e4, A.SL_F32)   # mask id out of range
+    assert lib.sl_model_create(C.byref(cfg), C.byref(w), C.byref(out)) == A.SL_ERR_INVALID
+    assert lib.sl_active_create(0, 10, C.byref(out)) == A.SL_ERR_INVALID
+    assert lib.sl_active_create(1, 0, C.byref(out)) == A.SL_ERR_INVALID
+    assert lib.sl_active_create(A.SL_MAX_BATCH + 1, 8, C.byref(out)) == A.SL_ERR_INVALID
+    assert lib.sl_kv_cache_create(None, 1, 8, C.byref(out)) == A.SL_ERR_INVALID
+    p = A.LockParams(0.01, -1.0, 1, -1)
+    assert lib.sl_kl_lock(None, 512, 0, 0, None, None, None, None, None, C.byref(p),
+                          None, None, None, None, None, None) == A.SL_ERR_INVALID
+    assert lib.sl_unmask_topk(None, None, None, 0, 1, 1, None, None, None) == A.SL_ERR_INVALID
+    assert lib.sl_compact_active(None, None, None, None, 0, None) == A.SL_ERR_INVALID
+    assert lib.sl_step(None, None, None, None, None, None) == A.SL_ERR_INVALID
+    assert lib.sl_sampler_step(None, None) == A.SL_ERR_INVALID
+    # GEMM: K must be a multiple of 64; a bad epilogue code is rejected
+    assert lib.sl_gemm_bf16(0, 16, 8, 100, 16, None, 128, 16, 128, None, 128, 1, None) == A.SL_ERR_INVALID
+    assert lib.sl_gemm_bf16(9, 16, 8, 128, 16, None, 128, 16, 128, None, 128, 1, None) == A.SL_ERR_INVALID

@@ -1,0 +1,101 @@
+"""tcgen05 GEMM (sl_gemm_bf16) against the plain definition C = A B^T in fp64,
+over every epilogue, tile width and K split, with ragged M tails."""
+import numpy as np
+import pytest
+import torch
+
+from token_locking_b200 import _abi as A
+from token_locking_b200 import runtime as rt
+
+pytestmark = pytest.mark.gpu
+
+
+def _mk(shape, seed, dev):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    return torch.randn(shape, generator=g).to(dev, torch.bfloat16)
+
+
+def _ref(a, b):
+    return a.double().cpu() @ b.double().cpu().T
+
+
+def _close(got, ref, K, bf16_out):
+    got = got.double().cpu()
+    scale = ref.abs().max().item() + 1e-6
+    err = (got - ref).abs().max().item()
+    # fp32 accumulation of K bf16 products; bf16 output rounding 2^-8 relative
+    tol = (4e-3 * scale) if bf16_out else (1e-5 * np.sqrt(K) * scale + 1e-4)
+    assert err <= tol, f"max err {err} > tol {tol} (scale {scale})"
+
+
+@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("M", [1, 37, 128, 301])
+def test_store_rowmap(cuda_dev, bn, M):
+    K, N = 512, 768
+    a, b = _mk((M, K), 1, cuda_dev), _mk((N, K), 2, cuda_dev)
+    perm = torch.randperm(M + 5, generator=torch.Generator().manual_seed(3))[:M].to(torch.int32)
+    out = torch.full((M + 5, N), 7.0, device=cuda_dev, dtype=torch.bfloat16)
+    rt.gemm_bf16(A.GEMM_STORE, a, b, out, row_map=perm.to(cuda_dev), bn=bn, splits=1)
+    torch.cuda.synchronize()
+    ref = _ref(a, b)
+    _close(out[perm.long()], ref, K, True)
+    untouched = torch.ones(M + 5, dtype=torch.bool)
+    untouched[perm.long()] = False
+    assert torch.all(out[untouched.to(cuda_dev)] == 7.0)
+    rt.device_check()
+
+
+@pytest.mark.parametrize("bn,splits", [(64, 1), (128, 3), (256, 2), (128, 8)])
+@pytest.mark.parametrize("M", [5, 130])
+def test_resid_split(cuda_dev, bn, splits, M):
+    K, N = 1024, 512
+    a, b = _mk((M, K), 4, cuda_dev), _mk((N, K), 5, cuda_dev)
+    h0 = torch.randn((M, N), generator=torch.Generator().manual_seed(6)).to(cuda_dev)
+    h = h0.clone()
+    rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=bn, splits=splits)
+    torch.cuda.synchronize()
+    _close(h - h0, _ref(a, b), K, False)
+    rt.device_check()
+
+
+@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("M", [3, 129])
+def test_swiglu(cuda_dev, bn, M):
+    K, F = 256, 384
+    if F % (bn // 2):
+        pytest.skip("F must split into bn/2 halves")
+    a = _mk((M, K), 7, cuda_dev)
+    wg, wu = _mk((F, K), 8, cuda_dev) * 0.1, _mk((F, K), 9, cuda_dev) * 0.1
+    out = torch.zeros((M, F), device=cuda_dev, dtype=torch.bfloat16)
+    rt.gemm_bf16(A.GEMM_SWIGLU, a, wg, out, b2=wu, bn=bn, splits=1)
+    torch.cuda.synchronize()
+    g, u = _ref(a, wg), _ref(a, wu)
+    ref = g / (1 + torch.exp(-g)) * u
+    _close(out, ref, K, True)
+    rt.device_check()
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+def test_accum_split(cuda_dev, swiglu):
+    M, K, F = 77, 768, 256
+    a = _mk((M, K), 10, cuda_dev)
+    b = _mk((F, K), 11, cuda_dev)
+    b2 = _mk((F, K), 12, cuda_dev) if swiglu else None
+    N = 2 * F if swiglu else F
+    ws = torch.zeros((M, N), device=cuda_dev)
+    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=4)
+    torch.cuda.synchronize()
+    ref = torch.cat([_ref(a, b), _ref(a, b2)], dim=1) if swiglu else _ref(a, b)
+    _close(ws, ref, K, False)
+    rt.device_check()
+
+
+def test_large_k_full_shape_tile(cuda_dev):
+    """LLaDA-8B FFN-down shape slice: K = 12288, several M tiles."""
+    M, K, N = 260, 12288, 512
+    a, b = _mk((M, K), 13, cuda_dev) * 0.05, _mk((N, K), 14, cuda_dev) * 0.05
+    h = torch.zeros((M, N), device=cuda_dev)
+    rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=256, splits=1)
+    torch.cuda.synchronize()
+    _close(h, _ref(a, b), K, False)
+    rt.device_check()

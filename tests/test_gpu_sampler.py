@@ -1,0 +1,160 @@
+"""The library-driven SureLock decode (sl_sampler_*) against the oracle,
+teacher-forced step by step: before every GPU step the oracle is handed the
+GPU's state (tokens, mask flags, active list, cache, previous logits) and runs
+the same step; logits, sure-test outputs, lock decisions, unmasking and the
+compacted active list are compared.  Also a free-running tiny decode."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import model as om
+from oracle import surelock as osl
+from token_locking_b200 import runtime as rt
+from parity_util import (BAND_CONF_REL, FINAL_LP_TOL, LOGIT_TOL, compare_locks, conf_ambiguous,
+                         to64, weights_for_oracle, weights_to_device)
+
+pytestmark = pytest.mark.gpu
+
+MINI_BF16 = wl.ModelShape(n_layers=2, d_model=256, n_heads=2, head_dim=128, d_ffn=512,
+                          vocab=1024, mask_id=1023, rope_theta=10000.0)
+
+
+def _sampler(setup, dev, std=0.02, seed_w=0):
+    shape = setup.shape
+    w_np = wl.np_weights(shape, seed=seed_w, std=std)
+    w_dev = weights_to_device(w_np, setup.dtype, dev)
+    model = rt.Model(shape, w_dev, setup.dtype)
+    s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, setup.steps,
+                   setup.block_len, setup.tokens_per_step, setup.eps, setup.gate_q,
+                   setup.scripted)
+    prompts = wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab, shape.mask_id)
+    return model, s, weights_for_oracle(w_dev), prompts
+
+
+def _snapshot(s, setup):
+    st = s.state()
+    B, N = setup.batch, setup.n_ctx
+    L = setup.shape.n_layers
+    ks, vs = [], []
+    for l in range(L):
+        k, v = st["cache"].view(l)
+        ks.append(to64(k).reshape(B, N, -1))
+        vs.append(to64(v).reshape(B, N, -1))
+    t = st["t"]
+    prv = (t - 1) & 1 if t > 0 else 0
+    return {
+        "t": t,
+        "tokens": st["tokens"].cpu().numpy().copy(),
+        "masked": st["masked"].cpu().numpy().astype(bool),
+        "locked": st["locked"].cpu().numpy().astype(bool),
+        "act": st["active"].positions(),
+        "ck": np.stack(ks, 1), "cv": np.stack(vs, 1),
+        "z_prev": to64(st["logits"][prv]).reshape(B, N, -1),
+    }
+
+
+def _teacher_forced(setup, dev, steps, std=0.02):
+    model, s, w64, prompts = _sampler(setup, dev, std)
+    shape = setup.shape
+    B, N = setup.batch, setup.n_ctx
+    s.start(torch.from_numpy(prompts).to(dev))
+    stats = {"mismatch": 0, "ambiguous": 0, "locks": 0, "unmask_amb": 0}
+    for t in range(steps):
+        snap = _snapshot(s, setup)
+        assert snap["t"] == t
+        s.step()
+        torch.cuda.synchronize()
+        rt.device_check()
+        st = s.state()
+        cur = t & 1
+        z_gpu = to64(st["logits"][cur]).reshape(B, N, -1)
+        kl_g = st["kl"].cpu().numpy(); unc_g = st["unc"].cpu().numpy()
+        conf_g = st["conf"].cpu().numpy(); am_g = st["argmax"].cpu().numpy()
+        lock_g = st["lock"].cpu().numpy().astype(bool)
+        new_act = st["active"].positions()
+        tok_after = st["tokens"].cpu().numpy()
+        msk_after = st["masked"].cpu().numpy().astype(bool)
+        j0 = 0
+        for b in range(B):
+            A = snap["act"][b]
+            m = len(A)
+            # forward: oracle on the GPU's state
+            ck = np.ascontiguousarray(snap["ck"][b]); cv = np.ascontiguousarray(snap["cv"][b])
+            z = om.forward_active(shape, w64, snap["tokens"][b], A, ck, cv)
+            err = np.abs(z_gpu[b, A] - z).max() if m else 0.0
+            assert err <= LOGIT_TOL[setup.dtype], f"t={t} b={b}: logits err {err}"
+            # sure test / gate / unmask on the GPU's logits (same inputs, same decisions)
+            lp = osl.log_softmax(z_gpu[b, A])
+            lpp = osl.log_softmax(snap["z_prev"][b, A])
+            hp = np.full(m, t > 0)
+            rec = osl.lock_test(lp, lpp, hp, snap["masked"][b, A], A, shape, setup, t)
+            sl_ = slice(j0, j0 + m)
+            np.testing.assert_array_equal(am_g[sl_], rec["pred"])
+            np.testing.assert_allclose(conf_g[sl_], rec["conf"], rtol=2e-5)
+            np.testing.assert_allclose(unc_g[sl_], rec["u"], atol=2e-6)
+            if t > 0:
+                np.testing.assert_allclose(kl_g[sl_], rec["D"], atol=2e-5, rtol=1e-4)
+            mi, am = compare_locks(lock_g[sl_], rec["lock"], rec["D"], rec["u"], setup.eps,
+                                   rec["thr"], setup.gate_q >= 0)
+            stats["mismatch"] += mi
+            stats["ambiguous"] += am
+            stats["locks"] += int(lock_g[sl_].sum())
+            # unmasking: the k highest-confidence masked rows of the block
+            lo, hi = setup.block_bounds(t)
+            sel = osl.unmask_select(A, conf_g[sl_].astype(np.float64), snap["masked"][b, A],
+                                    lo, hi, setup.tokens_per_step)
+            want_tok = snap["tokens"][b].copy()
+            want_tok[A[sel]] = am_g[sl_][sel]
+            if not np.array_equal(tok_after[b], want_tok):
+                cands = np.nonzero(snap["masked"][b, A] & (A >= lo) & (A < hi))[0]
+                assert conf_ambiguous(conf_g[sl_], sel, cands), f"t={t} b={b}: unmasking differs"
+                stats["unmask_amb"] += 1
+            # masked rows never lock; compaction is the stable removal of GPU locks
+            assert not np.any(lock_g[sl_] & snap["masked"][b, A])
+            np.testing.assert_array_equal(new_act[b], osl.compact(A, lock_g[sl_]))
+            assert np.array_equal(msk_after[b], tok_after[b] == shape.mask_id)
+            j0 += m
+    model_locked = s.state()["locked"].cpu().numpy().astype(bool)
+    assert stats["mismatch"] == 0, stats
+    return stats, model_locked
+
+
+def test_tiny_decode_teacher_forced(cuda_dev):
+    stats, locked = _teacher_forced(wl.CFG_TINY, cuda_dev, wl.CFG_TINY.steps)
+    assert stats["locks"] > 10, stats
+
+
+def test_tiny_decode_gate_and_scripted(cuda_dev):
+    _teacher_forced(dataclasses.replace(wl.CFG_TINY, gate_q=0.5, eps=0.05), cuda_dev, 8)
+    _teacher_forced(dataclasses.replace(wl.CFG_TINY, scripted=True, eps=0.0), cuda_dev, 8)
+
+
+def test_bf16_mini_decode_teacher_forced(cuda_dev):
+    setup = wl.SamplerSetup(MINI_BF16, "bf16", batch=2, prompt_len=40, gen_len=160, steps=40,
+                            block_len=32, tokens_per_step=4, eps=0.01, gate_q=0.5)
+    setup.validate()
+    stats, _ = _teacher_forced(setup, cuda_dev, 12, std=0.05)
+
+
+def test_tiny_free_running_matches_oracle(cuda_dev):
+    """Whole decode without teacher forcing: final tokens identical and final
+    log-probs within 2e-2 of the oracle's (all 16 steps of the tiny setting)."""
+    setup = wl.CFG_TINY
+    model, s, w64, prompts = _sampler(setup, cuda_dev)
+    out = s.generate(prompts)
+    tok0, msk0 = wl.initial_tokens(prompts, setup.gen_len, setup.shape.mask_id)
+    tokT, lpT, counts, _, st = osl.surelock_sampler(setup.shape, w64, tok0, msk0, setup)
+    np.testing.assert_array_equal(out, tokT)
+    # final log-probs: each position's last posterior (frozen at its lock step)
+    sst = s.state()
+    lt = sst["lock_t"].cpu().numpy().reshape(-1)
+    z = [to64(sst["logits"][i]) for i in range(2)]
+    lse = [sst["lse"][i].cpu().numpy().astype(np.float64) for i in range(2)]
+    last = np.where(lt >= 0, lt, setup.steps - 1)
+    lp_gpu = np.stack([z[last[p] & 1][p] - lse[last[p] & 1][p] for p in range(len(last))])
+    err = np.abs(lp_gpu - lpT.reshape(len(last), -1)).max()
+    assert err <= FINAL_LP_TOL, err
+    assert list(s.state()["active"].counts()) == [counts[-1][0]]

@@ -1,0 +1,1149 @@
+// Host runtime behind the C ABI: model / KV cache / active set / sampler
+// objects, workspace ownership, GEMM tile planning and launch sequencing.
+//
+// The step follows the A_t / L_t / C formulation of SureLock ("Stopping
+// Computation for Converged Tokens in Masked Diffusion-LM Decoding"):
+// computation runs on the active rows only, locked rows are served from the
+// cache C, and the active list is compacted after every sure test
+// (Paper-Notes, "Method: overall framework" and "Key design").
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <array>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+// ------------------------------------------------------------------ errors --
+static thread_local std::string g_last_error;
+
+namespace sl {
+
+sl_status fail(sl_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+sl_status cuda_fail(cudaError_t e, const char *what) {
+  if (e == cudaErrorMemoryAllocation)
+    return fail(SL_ERR_OOM, "%s: %s", what, cudaGetErrorString(e));
+  return fail(SL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int *device_error_word() {
+  static int *words[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!words[dev]) {
+    int *p = nullptr;
+    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) return nullptr;
+    if (cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return nullptr;
+    words[dev] = p;
+  }
+  return words[dev];
+}
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+static size_t dsize(int dtype) { return dtype == SL_BF16 ? 2 : 4; }
+
+}  // namespace sl
+
+using namespace sl;
+
+// ---------------------------------------------------------------- objects --
+// Weight descriptors for the tensor-core path: one TMA map per box height
+// (32, 64, 128, 256 rows) so any tile width can be launched.
+struct WMaps {
+  TmaMat m[4];
+  const TmaMat *box(int rows) const {
+    switch (rows) {
+      case 32: return &m[0];
+      case 64: return &m[1];
+      case 128: return &m[2];
+      default: return &m[3];
+    }
+  }
+};
+
+enum { W_Q = 0, W_K, W_V, W_O, W_G, W_U, W_D, W_COUNT };
+
+struct TimingRec {
+  int cls;
+  double bytes, flops;
+  cudaEvent_t e0, e1;
+};
+
+struct sl_model {
+  sl_config cfg;
+  const void *tok_emb, *final_norm, *lm_head;
+  std::vector<sl_layer_weights> layers;
+  std::vector<std::array<WMaps, W_COUNT>> maps;
+  WMaps head_map;
+  int num_sms;
+  int *err;
+  bool timing = false;
+  std::vector<cudaEvent_t> ev_free;
+  std::vector<TimingRec> recs;
+  sl_timing acc{};
+};
+
+struct sl_kv_cache {
+  const sl_model *m;
+  int batch, n_ctx, max_rows;
+  std::vector<void *> k, v;
+  float2 *rope = nullptr;
+  float *h = nullptr;      // [max_rows][d] fp32 residual stream
+  void *a = nullptr;       // [max_rows][d] normed activations
+  void *qkv = nullptr;     // [max_rows][3d]
+  void *q = nullptr;       // [max_rows][d]
+  void *o = nullptr;       // [max_rows][d]
+  void *act = nullptr;     // [max_rows][f]
+  float *ws = nullptr;     // [max_rows][max(3d, 2f)] fp32 split-K workspace, kept zero
+  float *attn_ws = nullptr;
+  int attn_max_splits = 16;
+  TmaMat map_a, map_o, map_act;
+  int map_rows = -1;
+};
+
+struct sl_active {
+  int batch, n_ctx;
+  int32_t *rows = nullptr, *seq_off = nullptr;
+  int32_t *h_off = nullptr;          // pinned mirror of seq_off
+  cudaEvent_t ev = nullptr;
+  bool pending = false;
+  float4 *part = nullptr;            // lock-stats partial records
+  unsigned int *counters = nullptr;  // per row, zero between calls
+  int max_splits = 64;
+  int num_sms;
+};
+
+struct sl_sampler {
+  sl_model *m;
+  sl_sampler_params p;
+  int batch, n_ctx;
+  sl_kv_cache *cache = nullptr;
+  sl_active *act = nullptr;
+  int32_t *tokens = nullptr;
+  uint8_t *masked = nullptr, *locked = nullptr, *lock = nullptr;
+  int32_t *lock_t = nullptr, *argmax = nullptr, *d_prompts = nullptr;
+  void *logits[2] = {nullptr, nullptr};
+  float *lse[2] = {nullptr, nullptr};
+  float *kl = nullptr, *unc = nullptr, *conf = nullptr;
+  int t = 0;
+  bool started = false;
+};
+
+// ----------------------------------------------------------------- timing --
+namespace {
+
+struct Timed {
+  sl_model *m;
+  TimingRec rec;
+  bool on;
+  Timed(sl_model *m_, int cls, double bytes, double flops, cudaStream_t s) : m(m_), on(false) {
+    if (!m || !m->timing) return;
+    rec.cls = cls;
+    rec.bytes = bytes;
+    rec.flops = flops;
+    for (int i = 0; i < 2; ++i) {
+      cudaEvent_t e;
+      if (!m->ev_free.empty()) {
+        e = m->ev_free.back();
+        m->ev_free.pop_back();
+      } else if (cudaEventCreate(&e) != cudaSuccess) {
+        return;
+      }
+      (i == 0 ? rec.e0 : rec.e1) = e;
+    }
+    cudaEventRecord(rec.e0, s);
+    on = true;
+    stream = s;
+  }
+  cudaStream_t stream = nullptr;
+  ~Timed() {
+    if (!on) return;
+    cudaEventRecord(rec.e1, stream);
+    m->recs.push_back(rec);
+  }
+};
+
+}  // namespace
+
+// ------------------------------------------------------------------ version --
+extern "C" const char *sl_last_error(void) { return g_last_error.c_str(); }
+extern "C" const char *sl_version(void) { return "surelock-b200 0.1 (sm_100a)"; }
+
+// ------------------------------------------------------------------- model --
+extern "C" sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, sl_model **out) {
+  if (!cfg || !w || !out) return fail(SL_ERR_INVALID, "sl_model_create: null argument");
+  *out = nullptr;
+  const sl_config &c = *cfg;
+  if (c.n_layers <= 0 || c.d_model <= 0 || c.n_heads <= 0 || c.head_dim <= 0 || c.d_ffn <= 0 ||
+      c.vocab <= 0)
+    return fail(SL_ERR_INVALID, "sl_model_create: non-positive dimension");
+  if (c.n_heads * c.head_dim != c.d_model)
+    return fail(SL_ERR_INVALID, "sl_model_create: n_heads * head_dim != d_model");
+  if (c.mask_id < 0 || c.mask_id >= c.vocab)
+    return fail(SL_ERR_INVALID, "sl_model_create: mask_id out of range");
+  if (c.head_dim % 2 != 0) return fail(SL_ERR_INVALID, "sl_model_create: odd head_dim");
+  if (c.vocab % 8 != 0) return fail(SL_ERR_INVALID, "sl_model_create: vocab must be a multiple of 8");
+  if (c.dtype == SL_BF16) {
+    if (c.head_dim != 128)
+      return fail(SL_ERR_UNSUPPORTED, "sl_model_create: bf16 path needs head_dim 128");
+    if (c.d_model % 256 != 0 || c.d_ffn % 256 != 0 || c.vocab % 128 != 0)
+      return fail(SL_ERR_UNSUPPORTED,
+                  "sl_model_create: bf16 path needs d_model, d_ffn multiples of 256, vocab of 128");
+  } else if (c.dtype == SL_F32) {
+    if (c.head_dim != 8 && c.head_dim != 16 && c.head_dim != 32 && c.head_dim != 64)
+      return fail(SL_ERR_UNSUPPORTED, "sl_model_create: fp32 path needs head_dim in {8,16,32,64}");
+  } else {
+    return fail(SL_ERR_INVALID, "sl_model_create: unknown dtype %d", c.dtype);
+  }
+  if (!w->tok_emb || !w->final_norm || !w->lm_head || !w->layers)
+    return fail(SL_ERR_INVALID, "sl_model_create: null weight pointer");
+  for (int l = 0; l < c.n_layers; ++l) {
+    const sl_layer_weights &lw = w->layers[l];
+    const void *ps[9] = {lw.attn_norm, lw.wq, lw.wk, lw.wv, lw.wo, lw.ffn_norm, lw.w_gate,
+                         lw.w_up, lw.w_down};
+    for (int i = 0; i < 9; ++i)
+      if (!ps[i]) return fail(SL_ERR_INVALID, "sl_model_create: layer %d weight %d is null", l, i);
+  }
+  sl_model *m = new sl_model();
+  m->cfg = c;
+  m->tok_emb = w->tok_emb;
+  m->final_norm = w->final_norm;
+  m->lm_head = w->lm_head;
+  m->layers.assign(w->layers, w->layers + c.n_layers);
+  m->num_sms = sm_count();
+  m->err = device_error_word();
+  if (!m->err) {
+    delete m;
+    return fail(SL_ERR_CUDA, "sl_model_create: cannot allocate the device error word");
+  }
+  if (c.dtype == SL_BF16) {
+    const int boxes[4] = {32, 64, 128, 256};
+    m->maps.resize(c.n_layers);
+    for (int l = 0; l < c.n_layers; ++l) {
+      const sl_layer_weights &lw = m->layers[l];
+      const void *ptr[W_COUNT] = {lw.wq, lw.wk, lw.wv, lw.wo, lw.w_gate, lw.w_up, lw.w_down};
+      const int rows[W_COUNT] = {c.d_model, c.d_model, c.d_model, c.d_model, c.d_ffn, c.d_ffn,
+                                 c.d_model};
+      const int cols[W_COUNT] = {c.d_model, c.d_model, c.d_model, c.d_model, c.d_model,
+                                 c.d_model, c.d_ffn};
+      for (int i = 0; i < W_COUNT; ++i)
+        for (int b = 0; b < 4; ++b)
+          if (!tma_encode(&m->maps[l][i].m[b], ptr[i], rows[i], cols[i], boxes[b])) {
+            delete m;
+            return fail(SL_ERR_INVALID,
+                        "sl_model_create: TMA descriptor for layer %d weight %d failed "
+                        "(pointer must be 16-byte aligned)", l, i);
+          }
+    }
+    for (int b = 0; b < 4; ++b)
+      if (!tma_encode(&m->head_map.m[b], m->lm_head, c.vocab, c.d_model, boxes[b])) {
+        delete m;
+        return fail(SL_ERR_INVALID, "sl_model_create: TMA descriptor for lm_head failed");
+      }
+  }
+  *out = m;
+  return SL_OK;
+}
+
+extern "C" void sl_model_destroy(sl_model *m) {
+  if (!m) return;
+  for (auto &r : m->recs) {
+    cudaEventDestroy(r.e0);
+    cudaEventDestroy(r.e1);
+  }
+  for (auto e : m->ev_free) cudaEventDestroy(e);
+  delete m;
+}
+
+extern "C" sl_status sl_timing_enable(sl_model *m, int enable) {
+  if (!m) return fail(SL_ERR_INVALID, "sl_timing_enable: null model");
+  m->timing = enable != 0;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_timing_read(sl_model *m, sl_timing *out, int reset) {
+  if (!m || !out) return fail(SL_ERR_INVALID, "sl_timing_read: null argument");
+  for (auto &r : m->recs) {
+    if (cudaEventSynchronize(r.e1) != cudaSuccess) return cuda_fail(cudaGetLastError(), "event sync");
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, r.e0, r.e1);
+    m->acc.ms[r.cls] += ms;
+    m->acc.bytes[r.cls] += r.bytes;
+    m->acc.flops[r.cls] += r.flops;
+    m->acc.launches[r.cls] += 1;
+    m->ev_free.push_back(r.e0);
+    m->ev_free.push_back(r.e1);
+  }
+  m->recs.clear();
+  *out = m->acc;
+  if (reset) memset(&m->acc, 0, sizeof(m->acc));
+  return SL_OK;
+}
+
+extern "C" sl_status sl_device_check(int clear) {
+  int *w = device_error_word();
+  if (!w) return fail(SL_ERR_CUDA, "sl_device_check: no device error word");
+  SL_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  SL_CUDA(cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v != 0) {
+    if (clear) SL_CUDA(cudaMemset(w, 0, sizeof(int)));
+    return fail(SL_ERR_TIMEOUT, "a kernel gave up a bounded wait (code %d)", v);
+  }
+  return SL_OK;
+}
+
+// ---------------------------------------------------------------- KV cache --
+extern "C" void sl_kv_cache_destroy(sl_kv_cache *c) {
+  if (!c) return;
+  for (void *p : c->k) cudaFree(p);
+  for (void *p : c->v) cudaFree(p);
+  void *ps[] = {c->rope, c->h, c->a, c->qkv, c->q, c->o, c->act, c->ws, c->attn_ws};
+  for (void *p : ps)
+    if (p) cudaFree(p);
+  delete c;
+}
+
+extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
+                                        sl_kv_cache **out) {
+  if (!m || !out) return fail(SL_ERR_INVALID, "sl_kv_cache_create: null argument");
+  *out = nullptr;
+  if (batch <= 0 || batch > SL_MAX_BATCH || n_ctx <= 0)
+    return fail(SL_ERR_INVALID, "sl_kv_cache_create: batch in [1, %d] and n_ctx > 0 required",
+                SL_MAX_BATCH);
+  const sl_config &cfg = m->cfg;
+  const size_t es = dsize(cfg.dtype);
+  const int d = cfg.d_model, f = cfg.d_ffn;
+  sl_kv_cache *c = new sl_kv_cache();
+  c->m = m;
+  c->batch = batch;
+  c->n_ctx = n_ctx;
+  c->max_rows = batch * n_ctx;
+  const size_t rows = (size_t)c->max_rows;
+  const size_t layer_bytes = rows * d * es;
+  auto alloc = [&](void **p, size_t bytes) -> bool {
+    if (cudaMalloc(p, bytes) != cudaSuccess) return false;
+    return cudaMemset(*p, 0, bytes) == cudaSuccess;
+  };
+  bool ok = true;
+  c->k.assign(cfg.n_layers, nullptr);
+  c->v.assign(cfg.n_layers, nullptr);
+  for (int l = 0; l < cfg.n_layers && ok; ++l)
+    ok = alloc(&c->k[l], layer_bytes) && alloc(&c->v[l], layer_bytes);
+  const size_t wsc = std::max((size_t)3 * d, (size_t)2 * f);
+  ok = ok && alloc((void **)&c->h, rows * d * 4) && alloc(&c->a, rows * d * es) &&
+       alloc(&c->qkv, rows * 3 * d * es) && alloc(&c->q, rows * d * es) &&
+       alloc(&c->o, rows * d * es) && alloc(&c->act, rows * f * es) &&
+       alloc((void **)&c->ws, rows * wsc * 4);
+  if (ok && cfg.dtype == SL_BF16)
+    ok = alloc((void **)&c->attn_ws, attn_bf16_workspace_bytes(c->max_rows, cfg.n_heads,
+                                                               c->attn_max_splits));
+  if (ok) {
+    // rotary table in double precision: angle = pos * theta^(-2i/dh)
+    const int half = cfg.head_dim / 2;
+    std::vector<float2> tab((size_t)n_ctx * half);
+    for (int pos = 0; pos < n_ctx; ++pos)
+      for (int i = 0; i < half; ++i) {
+        double inv = pow((double)cfg.rope_theta, -2.0 * i / cfg.head_dim);
+        double ang = (double)pos * inv;
+        tab[(size_t)pos * half + i] = make_float2((float)cos(ang), (float)sin(ang));
+      }
+    ok = alloc((void **)&c->rope, tab.size() * sizeof(float2)) &&
+         cudaMemcpy(c->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice) ==
+             cudaSuccess;
+  }
+  if (!ok) {
+    sl_kv_cache_destroy(c);
+    return fail(SL_ERR_OOM, "sl_kv_cache_create: device allocation failed");
+  }
+  *out = c;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_kv_cache_reset(sl_kv_cache *c, void *stream) {
+  if (!c) return fail(SL_ERR_INVALID, "sl_kv_cache_reset: null cache");
+  const size_t bytes = (size_t)c->max_rows * c->m->cfg.d_model * dsize(c->m->cfg.dtype);
+  for (size_t l = 0; l < c->k.size(); ++l) {
+    SL_CUDA(cudaMemsetAsync(c->k[l], 0, bytes, (cudaStream_t)stream));
+    SL_CUDA(cudaMemsetAsync(c->v[l], 0, bytes, (cudaStream_t)stream));
+  }
+  return SL_OK;
+}
+
+extern "C" sl_status sl_kv_cache_view(const sl_kv_cache *c, int layer, void **k, void **v) {
+  if (!c || !k || !v) return fail(SL_ERR_INVALID, "sl_kv_cache_view: null argument");
+  if (layer < 0 || layer >= (int)c->k.size())
+    return fail(SL_ERR_INVALID, "sl_kv_cache_view: layer %d out of range", layer);
+  *k = c->k[layer];
+  *v = c->v[layer];
+  return SL_OK;
+}
+
+// -------------------------------------------------------------- active set --
+extern "C" void sl_active_destroy(sl_active *a) {
+  if (!a) return;
+  if (a->rows) cudaFree(a->rows);
+  if (a->seq_off) cudaFree(a->seq_off);
+  if (a->part) cudaFree(a->part);
+  if (a->counters) cudaFree(a->counters);
+  if (a->h_off) cudaFreeHost(a->h_off);
+  if (a->ev) cudaEventDestroy(a->ev);
+  delete a;
+}
+
+extern "C" sl_status sl_active_create(int batch, int n_ctx, sl_active **out) {
+  if (!out) return fail(SL_ERR_INVALID, "sl_active_create: null out");
+  *out = nullptr;
+  if (batch <= 0 || batch > SL_MAX_BATCH || n_ctx <= 0)
+    return fail(SL_ERR_INVALID, "sl_active_create: batch in [1, %d] and n_ctx > 0 required",
+                SL_MAX_BATCH);
+  sl_active *a = new sl_active();
+  a->batch = batch;
+  a->n_ctx = n_ctx;
+  a->num_sms = sm_count();
+  const size_t rows = (size_t)batch * n_ctx;
+  bool ok = cudaMalloc(&a->rows, rows * 4) == cudaSuccess &&
+            cudaMalloc(&a->seq_off, (batch + 1) * 4) == cudaSuccess &&
+            cudaMalloc(&a->part, rows * a->max_splits * 2 * sizeof(float4)) == cudaSuccess &&
+            cudaMalloc(&a->counters, rows * sizeof(unsigned)) == cudaSuccess &&
+            cudaMemset(a->counters, 0, rows * sizeof(unsigned)) == cudaSuccess &&
+            cudaMallocHost(&a->h_off, (batch + 1) * 4) == cudaSuccess &&
+            cudaEventCreateWithFlags(&a->ev, cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    sl_active_destroy(a);
+    return fail(SL_ERR_OOM, "sl_active_create: allocation failed");
+  }
+  for (int b = 0; b <= batch; ++b) a->h_off[b] = b * n_ctx;
+  *out = a;
+  return SL_OK;
+}
+
+static sl_status active_mirror(sl_active *a, cudaStream_t s) {
+  SL_CUDA(cudaMemcpyAsync(a->h_off, a->seq_off, (a->batch + 1) * 4, cudaMemcpyDeviceToHost, s));
+  SL_CUDA(cudaEventRecord(a->ev, s));
+  a->pending = true;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_active_reset(sl_active *a, void *stream) {
+  if (!a) return fail(SL_ERR_INVALID, "sl_active_reset: null");
+  SL_CUDA(launch_active_fill(a->rows, a->seq_off, a->batch, a->n_ctx, (cudaStream_t)stream));
+  return active_mirror(a, (cudaStream_t)stream);
+}
+
+extern "C" sl_status sl_active_load(sl_active *a, const int32_t *h_counts, const int32_t *h_pos,
+                                    void *stream) {
+  if (!a || !h_counts || (!h_pos)) return fail(SL_ERR_INVALID, "sl_active_load: null argument");
+  std::vector<int32_t> rows, off(a->batch + 1, 0);
+  int k = 0;
+  for (int b = 0; b < a->batch; ++b) {
+    if (h_counts[b] < 0 || h_counts[b] > a->n_ctx)
+      return fail(SL_ERR_INVALID, "sl_active_load: count %d of sequence %d out of range",
+                  h_counts[b], b);
+    off[b] = (int)rows.size();
+    int prev = -1;
+    for (int i = 0; i < h_counts[b]; ++i, ++k) {
+      int p = h_pos[k];
+      if (p <= prev || p >= a->n_ctx)
+        return fail(SL_ERR_INVALID, "sl_active_load: positions of sequence %d not strictly "
+                                    "ascending in [0, n_ctx)", b);
+      prev = p;
+      rows.push_back(b * a->n_ctx + p);
+    }
+  }
+  off[a->batch] = (int)rows.size();
+  cudaStream_t s = (cudaStream_t)stream;
+  // synchronous copies from pageable memory: the host vectors die on return
+  SL_CUDA(cudaStreamSynchronize(s));
+  if (!rows.empty()) SL_CUDA(cudaMemcpy(a->rows, rows.data(), rows.size() * 4, cudaMemcpyHostToDevice));
+  SL_CUDA(cudaMemcpy(a->seq_off, off.data(), off.size() * 4, cudaMemcpyHostToDevice));
+  return active_mirror(a, s);
+}
+
+extern "C" sl_status sl_active_counts(sl_active *a, int32_t *h_counts) {
+  if (!a || !h_counts) return fail(SL_ERR_INVALID, "sl_active_counts: null argument");
+  if (a->pending) {
+    SL_CUDA(cudaEventSynchronize(a->ev));
+    a->pending = false;
+  }
+  for (int b = 0; b < a->batch; ++b) h_counts[b] = a->h_off[b + 1] - a->h_off[b];
+  return SL_OK;
+}
+
+extern "C" sl_status sl_active_view(const sl_active *a, int32_t **d_rows, int32_t **d_seq_off) {
+  if (!a || !d_rows || !d_seq_off) return fail(SL_ERR_INVALID, "sl_active_view: null argument");
+  *d_rows = a->rows;
+  *d_seq_off = a->seq_off;
+  return SL_OK;
+}
+
+// --------------------------------------------------------- GEMM planning ---
+namespace {
+
+struct Plan {
+  int bn, splits;
+  double cost;
+};
+
+// Choose the tile width and K split of one GEMM: minimise the modelled
+// makespan  waves * per-unit time, where a unit streams kb_per_split K-blocks
+// of a BN-row weight tile (HBM-bound at small M) or issues their MMAs
+// (tensor-bound at large M), plus a fixed per-unit overhead.
+Plan plan_gemm(int M, int N, int K, bool allow_split, int num_sms, bool swiglu) {
+  const double bw_sm = 6.5e12 / num_sms;         // bytes/s per SM
+  const double fl_sm = 1.6e15 / num_sms;         // flop/s per SM at N=256 tiles
+  const int mt = (M + 127) / 128;
+  const int kblocks = K / 64;
+  Plan best{0, 1, 1e30};
+  const int bns[3] = {256, 128, 64};
+  for (int bi = 0; bi < 3; ++bi) {
+    const int bn = bns[bi];
+    if (N % bn) continue;
+    if (swiglu && (N / 2) % (bn / 2)) continue;
+    const double mma_eff = bn == 256 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
+    const int max_s = allow_split ? std::min(32, std::max(1, kblocks / 4)) : 1;
+    for (int s = 1; s <= max_s; ++s) {
+      const int kbp = (kblocks + s - 1) / s;
+      const int ss = (kblocks + kbp - 1) / kbp;
+      const long units = (long)mt * (N / bn) * ss;
+      const long waves = (units + num_sms - 1) / num_sms;
+      const double t_mem = kbp * (bn * 128.0 + 128 * 128.0 * 0.25) / bw_sm;
+      const double t_mma = kbp * (2.0 * 128 * bn * 64) / (fl_sm * mma_eff);
+      double t = waves * (std::max(t_mem, t_mma) + 1.0e-6);
+      if (ss > 1) t += 3.0e-6;                    // finalize / atomics overhead
+      if (t < best.cost - 1e-9) best = Plan{bn, ss, t};
+    }
+  }
+  return best;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------- step --
+// Algorithmic bytes of a GEMM: weights + activations in + results out, bf16
+// (fp32 for fp32 models), each counted once.
+static double gemm_bytes(double M, double N, double K, double es) {
+  return es * (N * K + M * K + M * N);
+}
+
+static sl_status layer_f32(sl_model *m, sl_kv_cache *c, sl_active *a, int l, float *h, int M,
+                           cudaStream_t s) {
+  const sl_config &cfg = m->cfg;
+  const int d = cfg.d_model, f = cfg.d_ffn;
+  float *an = (float *)c->a, *qkv = (float *)c->qkv, *q = (float *)c->q;
+  float *o = (float *)c->o, *ws = c->ws, *act = (float *)c->act;
+  const sl_layer_weights &lw = m->layers[l];
+  SL_CUDA(launch_rmsnorm(SL_F32, h, lw.attn_norm, d, cfg.rms_eps, M, an, s));
+  {
+    Timed t(m, SL_K_GEMM, gemm_bytes(M, 3.0 * d, d, 4), 6.0 * M * d * d, s);
+    SL_CUDA(launch_gemm_f32(EPI_STORE, an, M, d, (const float *)lw.wq, d, qkv, 3 * d, 0, nullptr, s));
+    SL_CUDA(launch_gemm_f32(EPI_STORE, an, M, d, (const float *)lw.wk, d, qkv, 3 * d, d, nullptr, s));
+    SL_CUDA(launch_gemm_f32(EPI_STORE, an, M, d, (const float *)lw.wv, d, qkv, 3 * d, 2 * d, nullptr, s));
+  }
+  SL_CUDA(launch_rope_scatter(SL_F32, qkv, true, false, M, a->rows, c->n_ctx, cfg.n_heads,
+                              cfg.head_dim, c->rope, q, c->k[l], c->v[l], s));
+  {
+    Timed t(m, SL_K_ATTN, 4.0 * (2.0 * M * d + 2.0 * c->batch * c->n_ctx * d),
+            4.0 * M * c->n_ctx * d, s);
+    SL_CUDA(launch_attn_f32(q, (const float *)c->k[l], (const float *)c->v[l], a->rows, M,
+                            c->n_ctx, cfg.n_heads, cfg.head_dim, o, s));
+  }
+  {
+    Timed t(m, SL_K_GEMM, gemm_bytes(M, d, d, 4), 2.0 * M * d * d, s);
+    SL_CUDA(launch_gemm_f32(EPI_RESID, o, M, d, (const float *)lw.wo, d, h, d, 0, nullptr, s));
+  }
+  SL_CUDA(launch_rmsnorm(SL_F32, h, lw.ffn_norm, d, cfg.rms_eps, M, an, s));
+  {
+    Timed t(m, SL_K_GEMM, gemm_bytes(M, 2.0 * f, d, 4), 4.0 * M * d * f, s);
+    SL_CUDA(launch_gemm_f32(EPI_STORE, an, M, d, (const float *)lw.w_gate, f, ws, 2 * f, 0, nullptr, s));
+    SL_CUDA(launch_gemm_f32(EPI_STORE, an, M, d, (const float *)lw.w_up, f, ws, 2 * f, f, nullptr, s));
+  }
+  SL_CUDA(launch_swiglu(SL_F32, ws, true, false, M, f, act, s));
+  {
+    Timed t(m, SL_K_GEMM, gemm_bytes(M, d, f, 4), 2.0 * M * d * f, s);
+    SL_CUDA(launch_gemm_f32(EPI_RESID, act, M, f, (const float *)lw.w_down, d, h, d, 0, nullptr, s));
+  }
+  return SL_OK;
+}
+
+static sl_status tc_gemm(sl_model *m, const TcGemmArgs &g, cudaStream_t s) {
+  cudaError_t e = launch_gemm_tc(g, m->num_sms, m->err, s);
+  if (e != cudaSuccess) return cuda_fail(e, "tcgen05 GEMM launch");
+  return SL_OK;
+}
+
+struct BfPlans {
+  Plan qkv, o, gu, dn, hd;
+};
+
+static BfPlans plans_for(const sl_config &cfg, int M, int ns) {
+  const int d = cfg.d_model, f = cfg.d_ffn;
+  BfPlans p;
+  p.qkv = plan_gemm(M, 3 * d, d, true, ns, false);
+  p.o = plan_gemm(M, d, d, true, ns, false);
+  p.gu = plan_gemm(M, 2 * f, d, true, ns, true);
+  p.dn = plan_gemm(M, d, f, true, ns, false);
+  p.hd = plan_gemm(M, cfg.vocab, d, false, ns, false);
+  return p;
+}
+
+static sl_status ensure_maps(sl_kv_cache *c, int M) {
+  if (c->map_rows == M) return SL_OK;
+  const sl_config &cfg = c->m->cfg;
+  if (!tma_encode(&c->map_a, c->a, M, cfg.d_model, 128) ||
+      !tma_encode(&c->map_o, c->o, M, cfg.d_model, 128) ||
+      !tma_encode(&c->map_act, c->act, M, cfg.d_ffn, 128))
+    return fail(SL_ERR_CUDA, "activation TMA descriptor encoding failed");
+  c->map_rows = M;
+  return SL_OK;
+}
+
+static void fill_seqs(AttnSeqs &seqs, const sl_active *a, const int32_t *counts) {
+  seqs.batch = a->batch;
+  int off = 0;
+  for (int b = 0; b < a->batch; ++b) {
+    seqs.seq_start[b] = off;
+    seqs.seq_count[b] = counts[b];
+    off += counts[b];
+  }
+}
+
+static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, int l, int M,
+                           const void *q, void *o, cudaStream_t s) {
+  const int d = m->cfg.d_model;
+  Timed t(m, SL_K_ATTN, 2.0 * (2.0 * M * d + 2.0 * seqs.batch * c->n_ctx * d),
+          4.0 * (double)M * c->n_ctx * d, s);
+  SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
+                           c->attn_ws, c->attn_max_splits, m->num_sms, s));
+  return SL_OK;
+}
+
+static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, float *h, int M,
+                            const AttnSeqs &seqs, const BfPlans &pl, cudaStream_t s) {
+  const sl_config &cfg = m->cfg;
+  const int d = cfg.d_model, f = cfg.d_ffn, H = cfg.n_heads;
+  const sl_layer_weights &lw = m->layers[l];
+  const auto &mp = m->maps[l];
+  const double Md = (double)M;
+  sl_status st;
+  SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s));
+  {
+    // fused Q | K | V projection over the three weight matrices
+    TcGemmArgs g{};
+    g.A = &c->map_a;
+    g.B[0] = mp[W_Q].box(pl.qkv.bn);
+    g.B[1] = mp[W_K].box(pl.qkv.bn);
+    g.B[2] = mp[W_V].box(pl.qkv.bn);
+    g.n_seg[0] = d;
+    g.n_seg[1] = d;
+    g.n_seg[2] = d;
+    g.M = M;
+    g.N = 3 * d;
+    g.K = d;
+    g.bn = pl.qkv.bn;
+    g.splits = pl.qkv.splits;
+    const bool split = pl.qkv.splits > 1;
+    g.epi = split ? EPI_ACCUM : EPI_STORE;
+    g.out = split ? (void *)c->ws : c->qkv;
+    g.ldo = 3 * d;
+    {
+      Timed t(m, SL_K_GEMM, gemm_bytes(Md, 3.0 * d, d, 2), 6.0 * Md * d * d, s);
+      if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
+    }
+    SL_CUDA(launch_rope_scatter(SL_BF16, split ? (void *)c->ws : c->qkv, split, split, M,
+                                a->rows, c->n_ctx, H, cfg.head_dim, c->rope, c->q, c->k[l],
+                                c->v[l], s));
+  }
+  if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, s)) != SL_OK) return st;
+  {
+    TcGemmArgs g{};
+    g.A = &c->map_o;
+    g.B[0] = mp[W_O].box(pl.o.bn);
+    g.n_seg[0] = d;
+    g.M = M;
+    g.N = d;
+    g.K = d;
+    g.bn = pl.o.bn;
+    g.splits = pl.o.splits;
+    g.epi = EPI_RESID;
+    g.out = h;
+    g.ldo = d;
+    Timed t(m, SL_K_GEMM, gemm_bytes(Md, d, d, 2), 2.0 * Md * d * d, s);
+    if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
+  }
+  SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.ffn_norm, d, cfg.rms_eps, M, c->a, s));
+  {
+    TcGemmArgs g{};
+    g.A = &c->map_a;
+    g.B[0] = mp[W_G].box(pl.gu.bn / 2);
+    g.B[1] = mp[W_U].box(pl.gu.bn / 2);
+    g.b_swiglu = 1;
+    g.M = M;
+    g.N = 2 * f;
+    g.K = d;
+    g.bn = pl.gu.bn;
+    g.splits = pl.gu.splits;
+    const bool split = pl.gu.splits > 1;
+    g.epi = split ? EPI_ACCUM : EPI_SWIGLU;
+    g.out = split ? (void *)c->ws : c->act;
+    g.ldo = split ? 2 * f : f;
+    {
+      Timed t(m, SL_K_GEMM, gemm_bytes(Md, 2.0 * f, d, 2) - 2.0 * Md * f, 4.0 * Md * d * f, s);
+      if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
+    }
+    if (split) SL_CUDA(launch_swiglu(SL_BF16, c->ws, true, true, M, f, c->act, s));
+  }
+  {
+    TcGemmArgs g{};
+    g.A = &c->map_act;
+    g.B[0] = mp[W_D].box(pl.dn.bn);
+    g.n_seg[0] = d;
+    g.M = M;
+    g.N = d;
+    g.K = f;
+    g.bn = pl.dn.bn;
+    g.splits = pl.dn.splits;
+    g.epi = EPI_RESID;
+    g.out = h;
+    g.ldo = d;
+    Timed t(m, SL_K_GEMM, gemm_bytes(Md, d, f, 2), 2.0 * Md * d * f, s);
+    if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
+  }
+  return SL_OK;
+}
+
+static sl_status check_pair(sl_model *m, sl_kv_cache *c, sl_active *a, const char *who) {
+  if (!m || !c || !a) return fail(SL_ERR_INVALID, "%s: null argument", who);
+  if (c->m != m) return fail(SL_ERR_INVALID, "%s: cache belongs to another model", who);
+  if (c->batch != a->batch || c->n_ctx != a->n_ctx)
+    return fail(SL_ERR_INVALID, "%s: cache (%d x %d) and active set (%d x %d) differ", who,
+                c->batch, c->n_ctx, a->batch, a->n_ctx);
+  return SL_OK;
+}
+
+extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
+                             void *d_logits, void *stream) {
+  sl_status st = check_pair(m, c, a, "sl_step");
+  if (st != SL_OK) return st;
+  if (!d_tokens || !d_logits) return fail(SL_ERR_INVALID, "sl_step: null argument");
+  if (m->cfg.dtype == SL_BF16 && ((uintptr_t)d_logits & 15))
+    return fail(SL_ERR_INVALID, "sl_step: logits must be 16-byte aligned");
+  int32_t counts[SL_MAX_BATCH];
+  if ((st = sl_active_counts(a, counts)) != SL_OK) return st;
+  int M = 0;
+  for (int b = 0; b < a->batch; ++b) M += counts[b];
+  if (M == 0) return SL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const sl_config &cfg = m->cfg;
+  const int d = cfg.d_model, V = cfg.vocab;
+  SL_CUDA(launch_gather_embed(cfg.dtype, d_tokens, a->rows, M, m->tok_emb, d, c->h, s));
+  if (cfg.dtype == SL_F32) {
+    for (int l = 0; l < cfg.n_layers; ++l)
+      if ((st = layer_f32(m, c, a, l, c->h, M, s)) != SL_OK) return st;
+    SL_CUDA(launch_rmsnorm(SL_F32, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
+    Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 4), 2.0 * M * d * V, s);
+    SL_CUDA(launch_gemm_f32(EPI_STORE, (const float *)c->a, M, d, (const float *)m->lm_head, V,
+                            (float *)d_logits, V, 0, a->rows, s));
+    return SL_OK;
+  }
+  if ((st = ensure_maps(c, M)) != SL_OK) return st;
+  AttnSeqs seqs;
+  fill_seqs(seqs, a, counts);
+  const BfPlans pl = plans_for(cfg, M, m->num_sms);
+  for (int l = 0; l < cfg.n_layers; ++l)
+    if ((st = layer_bf16(m, c, a, l, c->h, M, seqs, pl, s)) != SL_OK) return st;
+  SL_CUDA(launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
+  TcGemmArgs g{};
+  g.A = &c->map_a;
+  g.B[0] = m->head_map.box(pl.hd.bn);
+  g.n_seg[0] = V;
+  g.M = M;
+  g.N = V;
+  g.K = d;
+  g.bn = pl.hd.bn;
+  g.splits = 1;
+  g.epi = EPI_STORE;
+  g.out = d_logits;
+  g.ldo = V;
+  g.row_map = a->rows;
+  Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 2), 2.0 * (double)M * d * V, s);
+  return tc_gemm(m, g, s);
+}
+
+extern "C" sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
+                                      float *d_h, void *stream) {
+  sl_status st = check_pair(m, c, a, "sl_layer_forward");
+  if (st != SL_OK) return st;
+  if (!d_h) return fail(SL_ERR_INVALID, "sl_layer_forward: null hidden states");
+  if (layer < 0 || layer >= m->cfg.n_layers)
+    return fail(SL_ERR_INVALID, "sl_layer_forward: layer %d out of range", layer);
+  if ((uintptr_t)d_h & 15) return fail(SL_ERR_INVALID, "sl_layer_forward: d_h must be 16-byte aligned");
+  int32_t counts[SL_MAX_BATCH];
+  if ((st = sl_active_counts(a, counts)) != SL_OK) return st;
+  int M = 0;
+  for (int b = 0; b < a->batch; ++b) M += counts[b];
+  if (M == 0) return SL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (m->cfg.dtype == SL_F32) return layer_f32(m, c, a, layer, d_h, M, s);
+  if ((st = ensure_maps(c, M)) != SL_OK) return st;
+  AttnSeqs seqs;
+  fill_seqs(seqs, a, counts);
+  return layer_bf16(m, c, a, layer, d_h, M, seqs, plans_for(m->cfg, M, m->num_sms), s);
+}
+
+extern "C" sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
+                                  const void *d_q, void *d_o, void *stream) {
+  sl_status st = check_pair(m, c, a, "sl_attention");
+  if (st != SL_OK) return st;
+  if (!d_q || !d_o) return fail(SL_ERR_INVALID, "sl_attention: null argument");
+  if (layer < 0 || layer >= m->cfg.n_layers)
+    return fail(SL_ERR_INVALID, "sl_attention: layer %d out of range", layer);
+  int32_t counts[SL_MAX_BATCH];
+  if ((st = sl_active_counts(a, counts)) != SL_OK) return st;
+  int M = 0;
+  for (int b = 0; b < a->batch; ++b) M += counts[b];
+  if (M == 0) return SL_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (m->cfg.dtype == SL_F32) {
+    Timed t(m, SL_K_ATTN, 4.0 * (2.0 * M * m->cfg.d_model + 2.0 * c->batch * c->n_ctx * m->cfg.d_model),
+            4.0 * M * c->n_ctx * m->cfg.d_model, s);
+    SL_CUDA(launch_attn_f32((const float *)d_q, (const float *)c->k[layer],
+                            (const float *)c->v[layer], a->rows, M, c->n_ctx, m->cfg.n_heads,
+                            m->cfg.head_dim, (float *)d_o, s));
+    return SL_OK;
+  }
+  AttnSeqs seqs;
+  fill_seqs(seqs, a, counts);
+  return attn_bf16(m, c, seqs, layer, M, d_q, d_o, s);
+}
+
+extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b,
+                                  const void *d_b2, int N, void *d_out, int ldo,
+                                  const int32_t *d_row_map, int bn, int splits, void *stream) {
+  if (!d_a || !d_b || !d_out) return fail(SL_ERR_INVALID, "sl_gemm_bf16: null argument");
+  if (epi < SL_GEMM_STORE || epi > SL_GEMM_ACCUM) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bad epi");
+  if (M < 0 || K <= 0 || N <= 0 || K % 64 != 0)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: need M >= 0, K > 0 with K %% 64 == 0, N > 0");
+  const bool swiglu = epi == SL_GEMM_SWIGLU || (epi == SL_GEMM_ACCUM && d_b2);
+  if (epi == SL_GEMM_SWIGLU && !d_b2) return fail(SL_ERR_INVALID, "sl_gemm_bf16: SWIGLU needs d_b2");
+  if (swiglu && N % 2) return fail(SL_ERR_INVALID, "sl_gemm_bf16: gate/up needs even N");
+  if (((uintptr_t)d_a | (uintptr_t)d_b | (uintptr_t)(d_b2 ? d_b2 : d_b) | (uintptr_t)d_out) & 15)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: pointers must be 16-byte aligned");
+  if (M == 0) return SL_OK;
+  const int ns = sm_count();
+  if (bn == 0) {
+    Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID || epi == SL_GEMM_ACCUM, ns, swiglu);
+    bn = p.bn;
+    if (splits <= 0) splits = p.splits;
+  }
+  if (bn != 64 && bn != 128 && bn != 256) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bn must be 64/128/256");
+  if (N % bn || (swiglu && (N / 2) % (bn / 2)))
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: N must be a multiple of bn");
+  if (splits < 1) splits = 1;
+  const int epi_k = epi == SL_GEMM_STORE ? EPI_STORE : epi == SL_GEMM_RESID ? EPI_RESID
+                    : epi == SL_GEMM_SWIGLU ? EPI_SWIGLU : EPI_ACCUM;
+  const int brows = swiglu ? bn / 2 : bn;
+  TmaMat ma, mb, mb2;
+  if (!tma_encode(&ma, d_a, M, K, 128) || !tma_encode(&mb, d_b, swiglu ? N / 2 : N, K, brows) ||
+      (swiglu && !tma_encode(&mb2, d_b2, N / 2, K, brows)))
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: TMA descriptor encoding failed");
+  TcGemmArgs g{};
+  g.epi = epi_k;
+  g.A = &ma;
+  g.B[0] = &mb;
+  g.B[1] = swiglu ? &mb2 : nullptr;
+  g.b_swiglu = swiglu ? 1 : 0;
+  g.n_seg[0] = swiglu ? 0 : N;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.bn = bn;
+  g.splits = splits;
+  g.out = d_out;
+  g.ldo = ldo;
+  g.row_map = d_row_map;
+  int *err = device_error_word();
+  if (!err) return fail(SL_ERR_CUDA, "sl_gemm_bf16: no device error word");
+  cudaError_t e = launch_gemm_tc(g, ns, err, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sl_gemm_bf16 launch");
+  return SL_OK;
+}
+
+// -------------------------------------------------------------- lock test --
+static sl_status kl_lock_impl(sl_model *timing_model, sl_active *a, int vocab, int mask_id,
+                              int dtype, const void *cur, const void *prev, const float *lse_prev,
+                              float *lse_cur, const uint8_t *masked, const sl_lock_params *p,
+                              float *kl, float *unc, float *conf, int32_t *argmax,
+                              uint8_t *lock, cudaStream_t s) {
+  if (!a || !cur || !lse_cur || !masked || !p || !kl || !unc || !conf || !argmax || !lock)
+    return fail(SL_ERR_INVALID, "sl_kl_lock: null argument");
+  if (p->has_prev && (!prev || !lse_prev))
+    return fail(SL_ERR_INVALID, "sl_kl_lock: has_prev needs previous logits and lse");
+  if (vocab <= 0 || vocab % 8 != 0)
+    return fail(SL_ERR_INVALID, "sl_kl_lock: vocab must be a positive multiple of 8");
+  if (mask_id < -1 || mask_id >= vocab) return fail(SL_ERR_INVALID, "sl_kl_lock: bad mask_id");
+  if (dtype != SL_F32 && dtype != SL_BF16) return fail(SL_ERR_INVALID, "sl_kl_lock: bad dtype");
+  if (p->gate_q > 1.f) return fail(SL_ERR_INVALID, "sl_kl_lock: gate_q must be <= 1");
+  if (((uintptr_t)cur & 15) || (prev && ((uintptr_t)prev & 15)))
+    return fail(SL_ERR_INVALID, "sl_kl_lock: logits must be 16-byte aligned");
+  int32_t counts[SL_MAX_BATCH];
+  sl_status st = sl_active_counts(a, counts);
+  if (st != SL_OK) return st;
+  int M = 0;
+  for (int b = 0; b < a->batch; ++b) M += counts[b];
+  if (M == 0) return SL_OK;
+  LockStatsArgs la;
+  la.dtype = dtype;
+  la.cur = cur;
+  la.prev = prev;
+  la.lse_prev = lse_prev;
+  la.lse_cur = lse_cur;
+  la.rows = a->rows;
+  la.M = M;
+  la.V = vocab;
+  la.mask_id = mask_id;
+  la.has_prev = p->has_prev ? 1 : 0;
+  la.kl = kl;
+  la.unc = unc;
+  la.conf = conf;
+  la.argmax = argmax;
+  la.part = a->part;
+  la.counters = a->counters;
+  la.splits = std::min(a->max_splits, lock_stats_splits(M, vocab, a->num_sms));
+  {
+    const double bytes = (double)M * vocab * dsize(dtype) * (p->has_prev ? 2 : 1) + 24.0 * M;
+    Timed t(timing_model, SL_K_LOCK, bytes, 6.0 * M * vocab, s);
+    SL_CUDA(launch_lock_stats(la, s));
+  }
+  SL_CUDA(launch_lock_decide(a->seq_off, a->batch, a->rows, kl, unc, masked, p->eps, p->gate_q,
+                             p->has_prev, p->scripted_target, lock, s));
+  return SL_OK;
+}
+
+extern "C" sl_status sl_kl_lock(sl_active *a, int vocab, int mask_id, int logits_dtype,
+                                const void *d_logits_cur, const void *d_logits_prev,
+                                const float *d_lse_prev, float *d_lse_cur,
+                                const uint8_t *d_masked, const sl_lock_params *p, float *d_kl,
+                                float *d_unc, float *d_conf, int32_t *d_argmax, uint8_t *d_lock,
+                                void *stream) {
+  return kl_lock_impl(nullptr, a, vocab, mask_id, logits_dtype, d_logits_cur, d_logits_prev,
+                      d_lse_prev, d_lse_cur, d_masked, p, d_kl, d_unc, d_conf, d_argmax, d_lock,
+                      (cudaStream_t)stream);
+}
+
+extern "C" sl_status sl_unmask_topk(sl_active *a, const float *d_conf, const int32_t *d_argmax,
+                                    int block_lo, int block_hi, int k, int32_t *d_tokens,
+                                    uint8_t *d_masked, void *stream) {
+  if (!a || !d_conf || !d_argmax || !d_tokens || !d_masked)
+    return fail(SL_ERR_INVALID, "sl_unmask_topk: null argument");
+  if (block_lo < 0 || block_hi > a->n_ctx || block_lo > block_hi || k < 0)
+    return fail(SL_ERR_INVALID, "sl_unmask_topk: bad block [%d, %d) or k %d", block_lo,
+                block_hi, k);
+  if (block_hi - block_lo > 2048)
+    return fail(SL_ERR_UNSUPPORTED, "sl_unmask_topk: blocks longer than 2048");
+  if (k == 0 || block_hi == block_lo) return SL_OK;
+  SL_CUDA(launch_unmask(a->seq_off, a->batch, a->rows, a->n_ctx, d_conf, d_argmax, block_lo,
+                        block_hi, k, d_tokens, d_masked, (cudaStream_t)stream));
+  return SL_OK;
+}
+
+extern "C" sl_status sl_compact_active(sl_active *a, const uint8_t *d_lock, uint8_t *d_locked,
+                                       int32_t *d_lock_t, int step, void *stream) {
+  if (!a || !d_lock || !d_locked || !d_lock_t)
+    return fail(SL_ERR_INVALID, "sl_compact_active: null argument");
+  cudaStream_t s = (cudaStream_t)stream;
+  SL_CUDA(launch_compact(a->rows, a->seq_off, a->batch, d_lock, d_locked, d_lock_t, step, s));
+  return active_mirror(a, s);
+}
+
+// ----------------------------------------------------------------- sampler --
+extern "C" void sl_sampler_destroy(sl_sampler *s) {
+  if (!s) return;
+  sl_kv_cache_destroy(s->cache);
+  sl_active_destroy(s->act);
+  void *ps[] = {s->tokens, s->masked, s->locked, s->lock, s->lock_t, s->argmax, s->d_prompts,
+                s->logits[0], s->logits[1], s->lse[0], s->lse[1], s->kl, s->unc, s->conf};
+  for (void *p : ps)
+    if (p) cudaFree(p);
+  delete s;
+}
+
+extern "C" sl_status sl_sampler_create(sl_model *m, int batch, const sl_sampler_params *p,
+                                       sl_sampler **out) {
+  if (!m || !p || !out) return fail(SL_ERR_INVALID, "sl_sampler_create: null argument");
+  *out = nullptr;
+  const sl_sampler_params &q = *p;
+  if (q.prompt_len < 0 || q.gen_len <= 0 || q.steps <= 0 || q.block_len <= 0 ||
+      q.tokens_per_step <= 0)
+    return fail(SL_ERR_INVALID, "sl_sampler_create: non-positive sizes");
+  if (q.gen_len % q.block_len != 0 || q.steps % (q.gen_len / q.block_len) != 0)
+    return fail(SL_ERR_INVALID,
+                "sl_sampler_create: gen_len must split into blocks and steps into blocks");
+  if (q.block_len > 2048) return fail(SL_ERR_UNSUPPORTED, "sl_sampler_create: block_len > 2048");
+  if (q.gate_q > 1.f) return fail(SL_ERR_INVALID, "sl_sampler_create: gate_q must be <= 1");
+  sl_sampler *s = new sl_sampler();
+  s->m = m;
+  s->p = q;
+  s->batch = batch;
+  s->n_ctx = q.prompt_len + q.gen_len;
+  sl_status st = sl_kv_cache_create(m, batch, s->n_ctx, &s->cache);
+  if (st == SL_OK) st = sl_active_create(batch, s->n_ctx, &s->act);
+  if (st != SL_OK) {
+    sl_sampler_destroy(s);
+    return st;
+  }
+  const size_t rows = (size_t)batch * s->n_ctx;
+  const size_t es = dsize(m->cfg.dtype);
+  bool ok = cudaMalloc(&s->tokens, rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->masked, rows) == cudaSuccess &&
+            cudaMalloc(&s->locked, rows) == cudaSuccess &&
+            cudaMalloc(&s->lock, rows) == cudaSuccess &&
+            cudaMalloc(&s->lock_t, rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->argmax, rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->d_prompts, std::max<size_t>(1, (size_t)batch * q.prompt_len) * 4) ==
+                cudaSuccess &&
+            cudaMalloc(&s->logits[0], rows * m->cfg.vocab * es) == cudaSuccess &&
+            cudaMalloc(&s->logits[1], rows * m->cfg.vocab * es) == cudaSuccess &&
+            cudaMalloc(&s->lse[0], rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->lse[1], rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->kl, rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->unc, rows * 4) == cudaSuccess &&
+            cudaMalloc(&s->conf, rows * 4) == cudaSuccess;
+  if (!ok) {
+    sl_sampler_destroy(s);
+    return fail(SL_ERR_OOM, "sl_sampler_create: device allocation failed");
+  }
+  *out = s;
+  return SL_OK;
+}
+
+namespace {
+__global__ void sampler_init_kernel(const int32_t *prompts, int batch, int prompt_len, int n_ctx,
+                                    int mask_id, int32_t *tokens, uint8_t *masked,
+                                    uint8_t *locked, int32_t *lock_t) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= batch * n_ctx) return;
+  int b = i / n_ctx, pos = i - b * n_ctx;
+  bool prompt = pos < prompt_len;
+  tokens[i] = prompt ? prompts[b * prompt_len + pos] : mask_id;
+  masked[i] = prompt ? 0 : 1;
+  locked[i] = 0;
+  lock_t[i] = -1;
+}
+}  // namespace
+
+extern "C" sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, void *stream) {
+  if (!s || (!d_prompts && s->p.prompt_len > 0))
+    return fail(SL_ERR_INVALID, "sl_sampler_start: null argument");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int rows = s->batch * s->n_ctx;
+  sampler_init_kernel<<<(rows + 255) / 256, 256, 0, st>>>(
+      d_prompts, s->batch, s->p.prompt_len, s->n_ctx, s->m->cfg.mask_id, s->tokens, s->masked,
+      s->locked, s->lock_t);
+  SL_CUDA(cudaGetLastError());
+  sl_status r = sl_kv_cache_reset(s->cache, stream);
+  if (r != SL_OK) return r;
+  r = sl_active_reset(s->act, stream);
+  if (r != SL_OK) return r;
+  s->t = 0;
+  s->started = true;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
+  if (!s) return fail(SL_ERR_INVALID, "sl_sampler_step: null sampler");
+  if (!s->started) return fail(SL_ERR_STATE, "sl_sampler_step: call sl_sampler_start first");
+  if (s->t >= s->p.steps) return fail(SL_ERR_STATE, "sl_sampler_step: decode already finished");
+  const int t = s->t;
+  const int cur = t & 1, prv = cur ^ 1;
+  const sl_config &cfg = s->m->cfg;
+  sl_status st = sl_step(s->m, s->cache, s->act, s->tokens, s->logits[cur], stream);
+  if (st != SL_OK) return st;
+  sl_lock_params lp;
+  lp.eps = s->p.eps;
+  lp.gate_q = s->p.gate_q;
+  lp.has_prev = t > 0 ? 1 : 0;
+  lp.scripted_target = -1;
+  if (s->p.scripted) {
+    // M_{t+1} = round-half-up(N - 0.9 N (t+1)/(T-1))
+    const double n = s->n_ctx;
+    const double x = s->p.steps > 1 ? n - 0.9 * n * (t + 1) / (s->p.steps - 1) : n;
+    lp.scripted_target = (int)floor(x + 0.5);
+    if (lp.scripted_target < 0) lp.scripted_target = 0;
+  }
+  st = kl_lock_impl(s->m, s->act, cfg.vocab, cfg.mask_id, cfg.dtype, s->logits[cur],
+                    s->logits[prv], s->lse[prv], s->lse[cur], s->masked, &lp, s->kl, s->unc,
+                    s->conf, s->argmax, s->lock, (cudaStream_t)stream);
+  if (st != SL_OK) return st;
+  const int spb = s->p.steps / (s->p.gen_len / s->p.block_len);
+  const int lo = s->p.prompt_len + (t / spb) * s->p.block_len;
+  st = sl_unmask_topk(s->act, s->conf, s->argmax, lo, lo + s->p.block_len, s->p.tokens_per_step,
+                      s->tokens, s->masked, stream);
+  if (st != SL_OK) return st;
+  st = sl_compact_active(s->act, s->lock, s->locked, s->lock_t, t, stream);
+  if (st != SL_OK) return st;
+  s->t = t + 1;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_sampler_generate(sl_sampler *s, const int32_t *h_prompts,
+                                         int32_t *h_tokens, void *stream) {
+  if (!s || !h_tokens || (!h_prompts && s->p.prompt_len > 0))
+    return fail(SL_ERR_INVALID, "sl_sampler_generate: null argument");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (s->p.prompt_len > 0)
+    SL_CUDA(cudaMemcpyAsync(s->d_prompts, h_prompts, (size_t)s->batch * s->p.prompt_len * 4,
+                            cudaMemcpyHostToDevice, st));
+  sl_status r = sl_sampler_start(s, s->d_prompts, stream);
+  if (r != SL_OK) return r;
+  while (s->t < s->p.steps) {
+    r = sl_sampler_step(s, stream);
+    if (r != SL_OK) return r;
+  }
+  SL_CUDA(cudaMemcpyAsync(h_tokens, s->tokens, (size_t)s->batch * s->n_ctx * 4,
+                          cudaMemcpyDeviceToHost, st));
+  SL_CUDA(cudaStreamSynchronize(st));
+  return SL_OK;
+}
+
+extern "C" sl_status sl_sampler_get_state(const sl_sampler *s, sl_sampler_state *o) {
+  if (!s || !o) return fail(SL_ERR_INVALID, "sl_sampler_get_state: null argument");
+  o->tokens = s->tokens;
+  o->masked = s->masked;
+  o->locked = s->locked;
+  o->lock_t = s->lock_t;
+  o->logits[0] = s->logits[0];
+  o->logits[1] = s->logits[1];
+  o->lse[0] = s->lse[0];
+  o->lse[1] = s->lse[1];
+  o->kl = s->kl;
+  o->unc = s->unc;
+  o->conf = s->conf;
+  o->argmax = s->argmax;
+  o->lock = s->lock;
+  o->cache = s->cache;
+  o->active = s->act;
+  o->t = s->t;
+  o->batch = s->batch;
+  o->n_ctx = s->n_ctx;
+  return SL_OK;
+}

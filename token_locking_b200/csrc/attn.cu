@@ -1,0 +1,325 @@
+// Attention of the M active queries over all N cached keys of their sequence,
+// bf16 in, fp32 softmax/accumulation (head_dim 128).
+//
+// The pages reduce per-step attention from O(N^2 d) to O(M N d) by issuing
+// queries for the active rows only while keys/values of every position are
+// read from the cache C (Abstract; Paper-Notes, "permanent locking":
+// K^all[L_t] <- C.k[L_t]).  One CTA owns 64 queries of one (sequence, head)
+// and a range of 64-key tiles; K/V tiles stream through shared memory with
+// cp.async double buffering and an online softmax.  When the query tiles alone
+// cannot fill the GPU (few active rows), the key range is split across CTAs
+// and a second kernel merges the partial (max, sum, output) records.
+#include "common.cuh"
+#include "internal.h"
+
+namespace sl {
+
+constexpr int AT_Q = 64;       // queries per CTA
+constexpr int AT_K = 64;       // keys per tile
+constexpr int AT_D = 128;      // head dim
+constexpr int AT_THREADS = 128;
+constexpr int AT_SMEM = (AT_Q + 4 * AT_K) * AT_D * 2;   // Q + 2x(K,V)
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+// 16-byte chunk c of row r in a [rows][128] bf16 tile, XOR-swizzled.
+__device__ __forceinline__ uint32_t tile_off(int r, int c) {
+  return (uint32_t)(r * 256 + ((c ^ (r & 7)) << 4));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  int sz = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(sz));
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N> __device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1,
+                                          uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float *c, const uint32_t *a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+struct AttnParams {
+  const bf16 *q;         // [M][d]
+  const bf16 *ck, *cv;   // [B*n_ctx][d]
+  bf16 *o;               // [M][d]
+  float *ws_o;           // [splits][M][H][128]
+  float *ws_ml;          // [splits][M][H][2]
+  AttnSeqs seqs;
+  int M, n_ctx, n_heads, splits, kblocks;
+};
+
+__global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sQ = smem_u32(smem);
+  const uint32_t sK0 = sQ + AT_Q * AT_D * 2;
+  const uint32_t sV0 = sK0 + 2 * AT_K * AT_D * 2;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.y, split = blockIdx.z;
+  const int d = p.n_heads * AT_D;
+
+  // locate (sequence, query tile)
+  int tile = blockIdx.x, b = 0, q0 = 0, qn = 0;
+  for (; b < p.seqs.batch; ++b) {
+    int nt = (p.seqs.seq_count[b] + AT_Q - 1) / AT_Q;
+    if (tile < nt) break;
+    tile -= nt;
+  }
+  if (b >= p.seqs.batch) return;
+  q0 = p.seqs.seq_start[b] + tile * AT_Q;
+  qn = min(AT_Q, p.seqs.seq_count[b] - tile * AT_Q);
+
+  const int per = (p.kblocks + p.splits - 1) / p.splits;
+  const int kb0 = split * per;
+  const int kb1 = min(p.kblocks, kb0 + per);
+
+  const bf16 *kbase = p.ck + (size_t)b * p.n_ctx * d + h * AT_D;
+  const bf16 *vbase = p.cv + (size_t)b * p.n_ctx * d + h * AT_D;
+
+  // Q tile
+  for (int e = tid; e < AT_Q * 16; e += AT_THREADS) {
+    int r = e >> 4, c = e & 15;
+    bool ok = r < qn;
+    const bf16 *src = p.q + (size_t)(q0 + (ok ? r : 0)) * d + h * AT_D + c * 8;
+    cp_async16(sQ + tile_off(r, c), src, ok);
+  }
+  auto load_kv = [&](int kb, int buf) {
+    const uint32_t sK = sK0 + buf * AT_K * AT_D * 2;
+    const uint32_t sV = sV0 + buf * AT_K * AT_D * 2;
+    for (int e = tid; e < AT_K * 16; e += AT_THREADS) {
+      int r = e >> 4, c = e & 15;
+      int key = kb * AT_K + r;
+      bool ok = key < p.n_ctx;
+      size_t off = (size_t)(ok ? key : 0) * d + c * 8;
+      cp_async16(sK + tile_off(r, c), kbase + off, ok);
+      cp_async16(sV + tile_off(r, c), vbase + off, ok);
+    }
+  };
+  if (kb0 < kb1) load_kv(kb0, 0);
+  cp_commit();
+
+  const float sl2 = 1.4426950408889634f * rsqrtf((float)AT_D);   // log2(e)/sqrt(dh)
+  float o_acc[16][4];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
+  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+  uint32_t qf[8][4];
+  const int g = lane >> 2, c4 = lane & 3;
+
+  for (int kb = kb0; kb < kb1; ++kb) {
+    const int buf = (kb - kb0) & 1;
+    if (kb + 1 < kb1) load_kv(kb + 1, buf ^ 1);
+    cp_commit();
+    cp_wait<1>();
+    __syncthreads();
+    if (kb == kb0) {
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        int r = warp * 16 + (lane & 15);
+        int c = 2 * kk + (lane >> 4);
+        ldsm_x4(sQ + tile_off(r, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+      }
+    }
+    const uint32_t sK = sK0 + buf * AT_K * AT_D * 2;
+    const uint32_t sV = sV0 + buf * AT_K * AT_D * 2;
+    float s[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+      for (int nt = 0; nt < 8; nt += 2) {
+        int r = nt * 8 + (lane & 7) + ((lane >> 4) << 3);
+        int c = 2 * kk + ((lane >> 3) & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(sK + tile_off(r, c), b0, b1, b2, b3);
+        mma16816(s[nt], qf[kk], b0, b1);
+        mma16816(s[nt + 1], qf[kk], b2, b3);
+      }
+    }
+    // online softmax (base 2) on rows g and g+8 of this warp
+    float tmax[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int key = kb * AT_K + nt * 8 + 2 * c4 + (e & 1);
+        float v = (key < p.n_ctx) ? s[nt][e] * sl2 : -INFINITY;
+        s[nt][e] = v;
+        tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
+      }
+    }
+    float corr[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 1));
+      tmax[r] = fmaxf(tmax[r], __shfl_xor_sync(0xffffffffu, tmax[r], 2));
+      float mn = fmaxf(m_r[r], tmax[r]);
+      corr[r] = (m_r[r] == -INFINITY) ? 0.f : exp2f(m_r[r] - mn);
+      m_r[r] = mn;
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float mm = m_r[e >> 1];
+        float pv = (mm == -INFINITY) ? 0.f : exp2f(s[nt][e] - mm);
+        s[nt][e] = pv;
+        rs[e >> 1] += pv;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 1);
+      rs[r] += __shfl_xor_sync(0xffffffffu, rs[r], 2);
+      l_r[r] = l_r[r] * corr[r] + rs[r];
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      o_acc[i][0] *= corr[0]; o_acc[i][1] *= corr[0];
+      o_acc[i][2] *= corr[1]; o_acc[i][3] *= corr[1];
+    }
+    // O += P V
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc) {
+      uint32_t pa[4];
+      pa[0] = pack_bf16(s[2 * kc][0], s[2 * kc][1]);
+      pa[1] = pack_bf16(s[2 * kc][2], s[2 * kc][3]);
+      pa[2] = pack_bf16(s[2 * kc + 1][0], s[2 * kc + 1][1]);
+      pa[3] = pack_bf16(s[2 * kc + 1][2], s[2 * kc + 1][3]);
+#pragma unroll
+      for (int dt = 0; dt < 16; dt += 2) {
+        int r = kc * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        int c = dt + (lane >> 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(sV + tile_off(r, c), b0, b1, b2, b3);
+        mma16816(o_acc[dt], pa, b0, b1);
+        mma16816(o_acc[dt + 1], pa, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  cp_wait<0>();
+
+  // epilogue: rows g and g+8 of this warp's 16
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    int qr = warp * 16 + g + 8 * r;
+    if (qr >= qn) continue;
+    int j = q0 + qr;
+    if (p.splits == 1) {
+      float inv = l_r[r] > 0.f ? 1.f / l_r[r] : 0.f;
+      bf16 *dst = p.o + (size_t)j * d + h * AT_D;
+#pragma unroll
+      for (int dt = 0; dt < 16; ++dt) {
+        *reinterpret_cast<uint32_t *>(dst + dt * 8 + 2 * c4) =
+            pack_bf16(o_acc[dt][2 * r] * inv, o_acc[dt][2 * r + 1] * inv);
+      }
+    } else {
+      size_t rec = ((size_t)split * p.M + j) * p.n_heads + h;
+      float *dst = p.ws_o + rec * AT_D;
+#pragma unroll
+      for (int dt = 0; dt < 16; ++dt)
+        *reinterpret_cast<float2 *>(dst + dt * 8 + 2 * c4) =
+            make_float2(o_acc[dt][2 * r], o_acc[dt][2 * r + 1]);
+      if (c4 == 0) *reinterpret_cast<float2 *>(p.ws_ml + rec * 2) = make_float2(m_r[r], l_r[r]);
+    }
+  }
+}
+
+// Merge split-KV partials: one warp per (row, head), 4 dims per lane.
+__global__ void attn_combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml,
+                                    int M, int n_heads, int splits, bf16 *__restrict__ o) {
+  int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (w >= M * n_heads) return;
+  int j = w / n_heads, h = w % n_heads;
+  float mx = -INFINITY;
+  for (int s = 0; s < splits; ++s) {
+    size_t rec = ((size_t)s * M + j) * n_heads + h;
+    mx = fmaxf(mx, ws_ml[rec * 2]);
+  }
+  float L = 0.f;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int s = 0; s < splits; ++s) {
+    size_t rec = ((size_t)s * M + j) * n_heads + h;
+    float m = ws_ml[rec * 2], l = ws_ml[rec * 2 + 1];
+    float c = (m == -INFINITY) ? 0.f : exp2f(m - mx);
+    L += l * c;
+    float4 v = *reinterpret_cast<const float4 *>(ws_o + rec * AT_D + lane * 4);
+    acc[0] += v.x * c; acc[1] += v.y * c; acc[2] += v.z * c; acc[3] += v.w * c;
+  }
+  float inv = L > 0.f ? 1.f / L : 0.f;
+  bf16 *dst = o + (size_t)j * n_heads * AT_D + h * AT_D + lane * 4;
+  *reinterpret_cast<uint2 *>(dst) =
+      make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+}
+
+size_t attn_bf16_workspace_bytes(int max_rows, int n_heads, int max_splits) {
+  return (size_t)max_splits * max_rows * n_heads * (AT_D + 2) * sizeof(float);
+}
+
+cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
+                             int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
+                             int num_sms, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int tiles = 0;
+  for (int b = 0; b < seqs.batch; ++b) tiles += (seqs.seq_count[b] + AT_Q - 1) / AT_Q;
+  if (tiles == 0) return cudaSuccess;
+  const int kblocks = (n_ctx + AT_K - 1) / AT_K;
+  const int ctas = tiles * n_heads;
+  int splits = (2 * num_sms + ctas - 1) / ctas;
+  int max_by_keys = kblocks / 2 > 0 ? kblocks / 2 : 1;
+  if (splits > max_by_keys) splits = max_by_keys;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  AttnParams p;
+  p.q = (const bf16 *)q;
+  p.ck = (const bf16 *)ck;
+  p.cv = (const bf16 *)cv;
+  p.o = (bf16 *)o;
+  p.ws_o = ws;
+  p.ws_ml = ws + (size_t)splits * M * n_heads * AT_D;
+  p.seqs = seqs;
+  p.M = M;
+  p.n_ctx = n_ctx;
+  p.n_heads = n_heads;
+  p.splits = splits;
+  p.kblocks = kblocks;
+  dim3 grid(tiles, n_heads, splits);
+  attn_bf16_kernel<<<grid, AT_THREADS, AT_SMEM, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  int warps = M * n_heads;
+  attn_combine_kernel<<<(warps * 32 + 255) / 256, 256, 0, s>>>(p.ws_o, p.ws_ml, M, n_heads,
+                                                                splits, (bf16 *)o);
+  return cudaGetLastError();
+}
+
+}  // namespace sl

@@ -1,0 +1,501 @@
+// Projection / FFN / LM-head GEMMs of the active rows on the 5th-generation
+// tensor cores (tcgen05 + TMEM), operands staged by TMA.
+//
+//   C[M, N] = A[M, K] * B[N, K]^T      A = bf16 activations of the M active rows,
+//                                      B = bf16 weights [out, in] (both K-major)
+//
+// Locked rows skip the query projection and the FFN (Abstract; Paper-Notes,
+// "permanent locking"), so every GEMM here runs on the M active rows only:
+// O(M d^2) work per layer (gist.science/nl section 2).
+//
+// Design (sm_100a, one CTA per SM, persistent):
+//   warp 0      TMA producer: A tile 128x64 and B tile BNx64 per stage, 128B swizzle
+//   warp 1      TMEM allocation + single-thread tcgen05.mma issue (M=128, N=BN, K=16)
+//   warps 2..5  epilogue: tcgen05.ld 32x32b of the fp32 accumulator, fused
+//               output transform (bf16 store with optional row scatter, fp32
+//               residual add, SiLU(gate)*up, or fp32 split-K accumulation)
+// Two TMEM accumulators (2 x BN columns) let the epilogue of one tile overlap
+// the main loop of the next.  Every barrier wait is bounded; on timeout the
+// kernel records it in the device error word and winds down.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace sl {
+
+// ------------------------------------------------------------- host: TMA ---
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+bool tma_encode(TmaMat *m, const void *ptr, int rows, int cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || rows <= 0 || cols % 64 != 0 || ((uintptr_t)ptr & 15) != 0) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&m->map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), gdim,
+                  gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  m->ptr = ptr;
+  m->rows = rows;
+  m->cols = cols;
+  m->box_rows = box_rows;
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------- device: PTX glue ---
+__device__ __forceinline__ uint32_t s_addr(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+// Bounded wait: false after WAIT_LIMIT_NS or once another role has aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile int *abort_flag) {
+  if (mbar_try(bar, parity)) return true;
+  unsigned long long t0 = global_ns();
+  uint32_t spins = 0;
+  while (!mbar_try(bar, parity)) {
+    if ((++spins & 255u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 64 bf16 (128 B), 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);   // start address
+  d |= (uint64_t)1 << 16;                    // leading byte offset (unused for SW128 K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                    // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                    // SWIZZLE_128B
+  return d;
+}
+
+template <int BN>
+__device__ __forceinline__ constexpr uint32_t idesc_bf16_f32() {
+  return (1u << 4)            // D: fp32
+         | (1u << 7)          // A: bf16
+         | (1u << 10)         // B: bf16
+         | ((uint32_t)(BN >> 3) << 17)
+         | ((uint32_t)(128 >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- kernel ---
+struct TcParams {
+  CUtensorMap a;
+  CUtensorMap b[3];
+  int seg0, seg1;          // output column boundaries of segments 0 and 1
+  int b_swiglu;            // 1: B tile = gate rows | up rows (halves of BN)
+  int M, N, K;
+  int m_tiles, n_tiles, splits, kb_per_split, kblocks, units;
+  void *out;
+  int ldo;
+  int ffn;                 // SWIGLU/ACCUM-swiglu: F (columns of one half)
+  const int32_t *row_map;
+  int *err;
+};
+
+constexpr int GROUP_M = 16;
+
+__device__ __forceinline__ void decode_unit(const TcParams &p, int u, int &mt, int &nt, int &sp) {
+  const int per_group = GROUP_M * p.n_tiles * p.splits;
+  const int g = u / per_group;
+  const int r = u - g * per_group;
+  const int first_m = g * GROUP_M;
+  const int gm = min(GROUP_M, p.m_tiles - first_m);
+  mt = first_m + r % gm;
+  const int nn = r / gm;
+  nt = nn / p.splits;
+  sp = nn - nt * p.splits;
+}
+
+template <int BN, int STAGES>
+struct TcSmem {
+  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int B_BYTES = BN * 64 * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;   // barriers + alignment slack
+};
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ TcParams p) {
+  using L = TcSmem<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s_addr(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
+  const uint32_t bar0 = s_addr(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::BAR_OFF + 8 * (2 * STAGES + 5));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&p.a);
+    tma_prefetch_desc(&p.b[0]);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     s_addr(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_stage = -1;
+      uint32_t last_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int mt, nt, sp;
+        decode_unit(p, u, mt, nt, sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          const uint32_t sb = sa + L::A_BYTES;
+          mbar_expect_tx(full_bar(stage), L::STAGE_BYTES);
+          tma_load_2d(sa, &p.a, kb * 64, mt * 128, full_bar(stage));
+          if (p.b_swiglu) {
+            const int f0 = nt * (BN / 2);
+            tma_load_2d(sb, &p.b[0], kb * 64, f0, full_bar(stage));
+            tma_load_2d(sb + (BN / 2) * 128, &p.b[1], kb * 64, f0, full_bar(stage));
+          } else {
+            const int c0 = nt * BN;
+            if (c0 < p.seg0) tma_load_2d(sb, &p.b[0], kb * 64, c0, full_bar(stage));
+            else if (c0 < p.seg1) tma_load_2d(sb, &p.b[1], kb * 64, c0 - p.seg0, full_bar(stage));
+            else tma_load_2d(sb, &p.b[2], kb * 64, c0 - p.seg1, full_bar(stage));
+          }
+          last_stage = stage;
+          last_phase = phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        atomicExch(p.err, DEV_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+      }
+      // make sure the last issued copy has landed before the CTA can exit
+      if (last_stage >= 0) {
+        volatile int never = 0;
+        mbar_wait(full_bar(last_stage), last_phase, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32<BN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int mt, nt, sp;
+        decode_unit(p, u, mt, nt, sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          const uint32_t sb = sa + L::A_BYTES;
+          const uint64_t adesc = smem_desc_sw128(sa);
+          const uint64_t bdesc = smem_desc_sw128(sb);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.err, DEV_TIMEOUT_MMA);
+        *abort_flag = 1;
+      }
+      // wait for every issued MMA to finish before TMEM can be released
+      tc_commit(drain_bar);
+      volatile int never = 0;
+      mbar_wait(drain_bar, 0, &never);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q = warp & 3;                 // TMEM lane quarter of this warp
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+      int mt, nt, sp;
+      decode_unit(p, u, mt, nt, sp);
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const int r = mt * 128 + q * 32 + lane;
+      const bool live = r < p.M;
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      float v[32];
+      if (EPI == EPI_SWIGLU) {
+        const int f0 = nt * (BN / 2);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          float g[32];
+          tmem_ld32(taddr + c, g);
+          tmem_ld32(taddr + BN / 2 + c, v);
+          if (live) {
+            bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)r * p.ldo + f0 + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              Pack8 pk;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(silu_f(g[i + e]) * v[i + e]);
+              *reinterpret_cast<uint4 *>(dst + i) = pk.u;
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          tmem_ld32(taddr + c, v);
+          if (!live) continue;
+          if (EPI == EPI_STORE) {
+            const int orow = p.row_map ? p.row_map[r] : r;
+            bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)orow * p.ldo + nt * BN + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              Pack8 pk;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(v[i + e]);
+              *reinterpret_cast<uint4 *>(dst + i) = pk.u;
+            }
+          } else {
+            int col;
+            if (p.b_swiglu) {   // accumulate gate into [0, F), up into [F, 2F)
+              const int half = BN / 2;
+              const int f0 = nt * half;
+              col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
+            } else {
+              col = nt * BN + c;
+            }
+            float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + col;
+            if (EPI == EPI_RESID && p.splits == 1) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                float4 o = *reinterpret_cast<float4 *>(dst + i);
+                o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
+                *reinterpret_cast<float4 *>(dst + i) = o;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                atomicAdd(reinterpret_cast<float4 *>(dst + i),
+                          make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (!ok && lane == 0) {
+      atomicExch(p.err, DEV_TIMEOUT_EPI);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host ---
+template <int BN, int STAGES, int EPI>
+static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
+  using L = TcSmem<BN, STAGES>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  gemm_tc_kernel<BN, STAGES, EPI><<<grid, 192, L::TOTAL, s>>>(p);
+  return cudaGetLastError();
+}
+
+template <int BN, int STAGES>
+static cudaError_t run_epi(int epi, const TcParams &p, int grid, cudaStream_t s) {
+  switch (epi) {
+    case EPI_STORE: return run_tc<BN, STAGES, EPI_STORE>(p, grid, s);
+    case EPI_RESID: return run_tc<BN, STAGES, EPI_RESID>(p, grid, s);
+    case EPI_SWIGLU: return run_tc<BN, STAGES, EPI_SWIGLU>(p, grid, s);
+    case EPI_ACCUM: return run_tc<BN, STAGES, EPI_ACCUM>(p, grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s) {
+  if (a.M <= 0) return cudaSuccess;
+  const int bn = a.bn;
+  if ((bn != 64 && bn != 128 && bn != 256) || a.K % 64 != 0 || a.N % bn != 0)
+    return cudaErrorInvalidValue;
+  const bool swiglu_b = a.b_swiglu != 0;
+  if (a.epi == EPI_SWIGLU && !swiglu_b) return cudaErrorInvalidValue;
+  TcParams p;
+  memset(&p, 0, sizeof(p));
+  p.a = a.A->map;
+  for (int i = 0; i < 3; ++i)
+    if (a.B[i]) p.b[i] = a.B[i]->map;
+  p.b_swiglu = swiglu_b ? 1 : 0;
+  p.seg0 = a.n_seg[0];
+  p.seg1 = a.n_seg[0] + a.n_seg[1];
+  if (!swiglu_b && p.seg0 == 0) p.seg0 = a.N;    // single segment
+  if (p.seg1 < p.seg0) p.seg1 = p.seg0;
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.m_tiles = (a.M + 127) / 128;
+  p.n_tiles = a.N / bn;
+  p.kblocks = a.K / 64;
+  int splits = a.splits < 1 ? 1 : a.splits;
+  if (a.epi != EPI_RESID && a.epi != EPI_ACCUM) splits = 1;
+  if (splits > p.kblocks) splits = p.kblocks;
+  p.kb_per_split = (p.kblocks + splits - 1) / splits;
+  p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;   // no empty split
+  p.units = p.m_tiles * p.n_tiles * p.splits;
+  p.out = a.out;
+  p.ldo = a.ldo;
+  p.ffn = a.N / 2;
+  p.row_map = a.row_map;
+  p.err = err;
+  int grid = p.units < num_sms ? p.units : num_sms;
+  switch (bn) {
+    case 256: return run_epi<256, 4>(a.epi, p, grid, s);
+    case 128: return run_epi<128, 6>(a.epi, p, grid, s);
+    default: return run_epi<64, 8>(a.epi, p, grid, s);
+  }
+}
+
+}  // namespace sl

@@ -1,0 +1,122 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "surelock.h"
+
+namespace sl {
+
+// ------------------------------------------------------------------ errors --
+sl_status fail(sl_status st, const char *fmt, ...);
+sl_status cuda_fail(cudaError_t e, const char *what);
+int *device_error_word();   // per-device int, allocated on first use; nullptr on failure
+
+#define SL_CUDA(call)                                  \
+  do {                                                 \
+    cudaError_t _e = (call);                           \
+    if (_e != cudaSuccess) return ::sl::cuda_fail(_e, #call); \
+  } while (0)
+
+// ----------------------------------------------------- epilogue selection --
+enum GemmEpi : int {
+  EPI_STORE = 0,      // out[row_map ? row_map[r] : r][col_off + c] = acc   (dtype)
+  EPI_RESID = 1,      // resid[r][c] += acc   (fp32; atomic when split over K)
+  EPI_SWIGLU = 2,     // out[r][c] = silu(gate) * up      (dtype; tile = gate|up halves)
+  EPI_ACCUM = 3       // ws[r][col] += acc  (fp32 atomics, split-K workspace)
+};
+
+// ------------------------------------------------------------------ layers.cu
+cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
+                                const void *emb, int d, float *h, cudaStream_t s);
+cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
+                           void *out, cudaStream_t s);
+// qkv_in: [M][3d] (in_f32 ? float : dtype).  q_out [M][d] dtype; ck/cv: the layer's
+// cache [B*n_ctx][d]; rope: [n_ctx][head_dim/2] (cos, sin).  zero_in: clear the
+// fp32 input after reading (split-K workspace).
+cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool zero_in, int M,
+                                const int32_t *rows, int n_ctx, int n_heads, int head_dim,
+                                const float2 *rope, void *q_out, void *ck, void *cv,
+                                cudaStream_t s);
+// act[r][c] = silu(ws[r][c]) * ws[r][F + c]; ws fp32 [M][2F] (zeroed after use) or dtype.
+cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, int M, int F,
+                          void *act, cudaStream_t s);
+// fp32 SIMT GEMM: C = A[M,K] * B[N,K]^T with EPI_STORE (ldc, col_off, row_map) or EPI_RESID.
+cudaError_t launch_gemm_f32(int epi, const float *A, int M, int K, const float *B, int N,
+                            float *C, int ldc, int col_off, const int32_t *row_map,
+                            cudaStream_t s);
+// fp32 attention, head_dim <= 64: o[j] = softmax(q_j K_b^T / sqrt(dh)) V_b.
+cudaError_t launch_attn_f32(const float *q, const float *ck, const float *cv,
+                            const int32_t *rows, int M, int n_ctx, int n_heads, int head_dim,
+                            float *o, cudaStream_t s);
+
+// -------------------------------------------------------------------- attn.cu
+// Query tiles per sequence for the bf16 attention kernel.
+struct AttnSeqs {
+  int batch;
+  int seq_start[SL_MAX_BATCH];   // first active-row index of the sequence
+  int seq_count[SL_MAX_BATCH];   // active rows of the sequence
+};
+size_t attn_bf16_workspace_bytes(int max_rows, int n_heads, int max_splits);
+cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
+                             int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
+                             int num_sms, cudaStream_t s);
+
+// ----------------------------------------------------------------- gemm_tc.cu
+// A bf16 K-major operand in global memory with its TMA descriptor.
+struct TmaMat {
+  CUtensorMap map;
+  const void *ptr;
+  int rows, cols;        // cols = K (contiguous)
+  int box_rows;          // rows per TMA box
+};
+bool tma_encode(TmaMat *m, const void *ptr, int rows, int cols, int box_rows);
+
+struct TcGemmArgs {
+  int epi;               // GemmEpi
+  const TmaMat *A;       // activations [rows >= M][K]
+  const TmaMat *B[3];    // weight segments, each [n_i][K]; SWIGLU: B[0]=gate, B[1]=up
+  int n_seg[3];          // rows of each segment (STORE/ACCUM may use up to 3; others 1)
+  int M, N, K;           // N = total output columns (SWIGLU: 2F)
+  int splits;            // K splits (EPI_RESID / EPI_ACCUM only)
+  int bn;                // 64, 128 or 256
+  int b_swiglu;          // B tile = BN/2 gate rows (B[0]) | BN/2 up rows (B[1])
+  void *out;             // STORE/SWIGLU: dtype out; RESID: fp32 resid; ACCUM: fp32 ws
+  int ldo;               // leading dimension of out (elements)
+  const int32_t *row_map;// STORE: output row index per A row (or null)
+};
+cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s);
+
+// ------------------------------------------------------------------ lock.cu
+struct LockStatsArgs {
+  int dtype;
+  const void *cur, *prev;        // [rows][V]
+  const float *lse_prev;
+  float *lse_cur;
+  const int32_t *rows;           // active rows (flat positions)
+  int M, V, mask_id, has_prev;
+  float *kl, *unc, *conf;
+  int32_t *argmax;
+  float4 *part;                  // [M * splits * 2] partial records
+  unsigned int *counters;        // [M], zero between calls
+  int splits;
+};
+cudaError_t launch_lock_stats(const LockStatsArgs &a, cudaStream_t s);
+int lock_stats_splits(int M, int V, int num_sms);
+
+cudaError_t launch_lock_decide(const int32_t *seq_off, int batch, const int32_t *rows,
+                               const float *kl, const float *unc, const uint8_t *masked,
+                               float eps, float gate_q, int has_prev, int scripted_target,
+                               uint8_t *lock, cudaStream_t s);
+cudaError_t launch_compact(int32_t *rows, int32_t *seq_off, int batch, const uint8_t *lock,
+                           uint8_t *locked, int32_t *lock_t, int step, cudaStream_t s);
+cudaError_t launch_unmask(const int32_t *seq_off, int batch, const int32_t *rows, int n_ctx,
+                          const float *conf, const int32_t *argmax, int lo, int hi, int k,
+                          int32_t *tokens, uint8_t *masked, cudaStream_t s);
+cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n_ctx,
+                               cudaStream_t s);
+
+}  // namespace sl

@@ -1,0 +1,296 @@
+// Row-wise kernels of the denoiser on the active rows, and the fp32 SIMT
+// GEMM/attention used by fp32 models.
+//
+// The gather, norm, rotary, scatter and SwiGLU kernels are memory-bound: one
+// CTA per active row, 16-byte vector accesses on the bf16 path.
+#include "common.cuh"
+#include "internal.h"
+
+namespace sl {
+
+// ---------------------------------------------------------------- gather ---
+// h[j, :] = E[tokens[rows[j]], :]  (fp32 residual stream).  Only the M active
+// rows are embedded: locked rows keep a frozen block input and are not
+// recomputed (gist.science/it section 2, "Azione di Blocco").
+template <typename T>
+__global__ void gather_embed_kernel(const int32_t *__restrict__ tokens,
+                                    const int32_t *__restrict__ rows, int M,
+                                    const T *__restrict__ emb, int d, float *__restrict__ h) {
+  int j = blockIdx.x;
+  if (j >= M) return;
+  const T *e = emb + (size_t)tokens[rows[j]] * d;
+  float *o = h + (size_t)j * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = to_f(e[c]);
+}
+
+cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
+                                const void *emb, int d, float *h, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (dtype == SL_BF16)
+    gather_embed_kernel<bf16><<<M, 256, 0, s>>>(tokens, rows, M, (const bf16 *)emb, d, h);
+  else
+    gather_embed_kernel<float><<<M, 256, 0, s>>>(tokens, rows, M, (const float *)emb, d, h);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------------- rmsnorm ---
+// out = h / sqrt(mean(h^2) + eps) * g, rounded to the model dtype.
+template <typename T>
+__global__ void rmsnorm_kernel(const float *__restrict__ h, const T *__restrict__ g, int d,
+                               float eps, int M, T *__restrict__ out) {
+  int j = blockIdx.x;
+  if (j >= M) return;
+  const float *x = h + (size_t)j * d;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) ss += x[c] * x[c];
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  float r = rsqrtf(red[0] / (float)d + eps);
+  T *o = out + (size_t)j * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = from_f<T>(x[c] * r * to_f(g[c]));
+}
+
+cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
+                           void *out, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  int th = d >= 1024 ? 512 : 128;
+  if (dtype == SL_BF16)
+    rmsnorm_kernel<bf16><<<M, th, 0, s>>>(h, (const bf16 *)g, d, eps, M, (bf16 *)out);
+  else
+    rmsnorm_kernel<float><<<M, th, 0, s>>>(h, (const float *)g, d, eps, M, (float *)out);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------- rotary + scatter ---
+// From the fused projection output [M][3d] (q | k | v): q_out[j] = RoPE(q_j),
+// C.k[rows[j]] = RoPE(k_j), C.v[rows[j]] = v_j.  RoPE is rotate-half on the
+// pair (i, i + dh/2) at the absolute position rows[j] % n_ctx; the (cos, sin)
+// table is precomputed in double precision on the host.  Writing the fresh k,v
+// of active rows into the cache is the "K^all[A_t]" half of the pages'
+// K^all[L_t] <- C.k[L_t] (Paper-Notes, "permanent locking").
+template <typename Tin, typename T>
+__global__ void rope_scatter_kernel(Tin *__restrict__ qkv, bool zero_in, int M,
+                                    const int32_t *__restrict__ rows, int n_ctx, int n_heads,
+                                    int dh, const float2 *__restrict__ rope, T *__restrict__ q_out,
+                                    T *__restrict__ ck, T *__restrict__ cv) {
+  int j = blockIdx.x;
+  if (j >= M) return;
+  int d = n_heads * dh;
+  int half = dh >> 1;
+  int p = rows[j];
+  int pos = p % n_ctx;
+  Tin *in = qkv + (size_t)j * 3 * d;
+  const float2 *tab = rope + (size_t)pos * half;
+  T *qo = q_out + (size_t)j * d;
+  T *ko = ck + (size_t)p * d;
+  T *vo = cv + (size_t)p * d;
+  int npairs = n_heads * half;
+  for (int t = threadIdx.x; t < npairs; t += blockDim.x) {
+    int hh = t / half, i = t - hh * half;
+    int c0 = hh * dh + i, c1 = c0 + half;
+    float2 cs = tab[i];
+    float q0 = to_f(in[c0]), q1 = to_f(in[c1]);
+    float k0 = to_f(in[d + c0]), k1 = to_f(in[d + c1]);
+    qo[c0] = from_f<T>(q0 * cs.x - q1 * cs.y);
+    qo[c1] = from_f<T>(q1 * cs.x + q0 * cs.y);
+    ko[c0] = from_f<T>(k0 * cs.x - k1 * cs.y);
+    ko[c1] = from_f<T>(k1 * cs.x + k0 * cs.y);
+    vo[c0] = from_f<T>(to_f(in[2 * d + c0]));
+    vo[c1] = from_f<T>(to_f(in[2 * d + c1]));
+    if (zero_in) {
+      in[c0] = Tin(0.f); in[c1] = Tin(0.f);
+      in[d + c0] = Tin(0.f); in[d + c1] = Tin(0.f);
+      in[2 * d + c0] = Tin(0.f); in[2 * d + c1] = Tin(0.f);
+    }
+  }
+}
+
+cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool zero_in, int M,
+                                const int32_t *rows, int n_ctx, int n_heads, int head_dim,
+                                const float2 *rope, void *q_out, void *ck, void *cv,
+                                cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  int th = 256;
+  if (dtype == SL_BF16) {
+    if (in_f32)
+      rope_scatter_kernel<float, bf16><<<M, th, 0, s>>>((float *)qkv_in, zero_in, M, rows, n_ctx,
+          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv);
+    else
+      rope_scatter_kernel<bf16, bf16><<<M, th, 0, s>>>((bf16 *)qkv_in, false, M, rows, n_ctx,
+          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv);
+  } else {
+    rope_scatter_kernel<float, float><<<M, th, 0, s>>>((float *)qkv_in, zero_in, M, rows, n_ctx,
+        n_heads, head_dim, rope, (float *)q_out, (float *)ck, (float *)cv);
+  }
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------- swiglu ---
+template <typename Tin, typename T>
+__global__ void swiglu_kernel(Tin *__restrict__ ws, bool zero_in, int M, int F,
+                              T *__restrict__ act) {
+  int j = blockIdx.x;
+  if (j >= M) return;
+  Tin *g = ws + (size_t)j * 2 * F;
+  T *o = act + (size_t)j * F;
+  for (int c = threadIdx.x; c < F; c += blockDim.x) {
+    float gv = to_f(g[c]), uv = to_f(g[F + c]);
+    o[c] = from_f<T>(silu_f(gv) * uv);
+    if (zero_in) { g[c] = Tin(0.f); g[F + c] = Tin(0.f); }
+  }
+}
+
+cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, int M, int F,
+                          void *act, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (dtype == SL_BF16) {
+    if (in_f32)
+      swiglu_kernel<float, bf16><<<M, 512, 0, s>>>((float *)ws, zero_in, M, F, (bf16 *)act);
+    else
+      swiglu_kernel<bf16, bf16><<<M, 512, 0, s>>>((bf16 *)ws, false, M, F, (bf16 *)act);
+  } else {
+    swiglu_kernel<float, float><<<M, 256, 0, s>>>((float *)ws, zero_in, M, F, (float *)act);
+  }
+  return cudaGetLastError();
+}
+
+// -------------------------------------------------------- fp32 SIMT GEMM ---
+// C[M,N] = A[M,K] B[N,K]^T, 64x64 tiles, 16x16 threads with 4x4 outputs each.
+// Used only for fp32 models (tiny shapes); bf16 models run on tcgen05.
+constexpr int FT = 64, FK = 16;
+
+__global__ void __launch_bounds__(256) gemm_f32_kernel(int epi, const float *__restrict__ A, int M,
+                                                       int K, const float *__restrict__ B, int N,
+                                                       float *__restrict__ C, int ldc, int col_off,
+                                                       const int32_t *__restrict__ row_map) {
+  __shared__ float As[FK][FT + 1];
+  __shared__ float Bs[FK][FT + 1];
+  int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  int m0 = blockIdx.y * FT, n0 = blockIdx.x * FT;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += FK) {
+    for (int e = threadIdx.x; e < FT * FK; e += 256) {
+      int r = e / FK, kk = e % FK;
+      int gm = m0 + r, gn = n0 + r, gk = k0 + kk;
+      As[kk][r] = (gm < M && gk < K) ? A[(size_t)gm * K + gk] : 0.f;
+      Bs[kk][r] = (gn < N && gk < K) ? B[(size_t)gn * K + gk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < FK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) b[i] = Bs[kk][tx * 4 + i];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(a[i], b[jj], acc[i][jj]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int gm = m0 + ty * 4 + i;
+    if (gm >= M) continue;
+    int orow = row_map ? row_map[gm] : gm;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      int gn = n0 + tx * 4 + jj;
+      if (gn >= N) continue;
+      float *dst = C + (size_t)orow * ldc + col_off + gn;
+      if (epi == EPI_RESID) *dst += acc[i][jj];
+      else *dst = acc[i][jj];
+    }
+  }
+}
+
+cudaError_t launch_gemm_f32(int epi, const float *A, int M, int K, const float *B, int N,
+                            float *C, int ldc, int col_off, const int32_t *row_map,
+                            cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  dim3 grid((N + FT - 1) / FT, (M + FT - 1) / FT);
+  gemm_f32_kernel<<<grid, 256, 0, s>>>(epi, A, M, K, B, N, C, ldc, col_off, row_map);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------- fp32 attention ---
+// One warp per (active row, head).  Keys of the row's sequence are processed in
+// chunks of 32 (one key per lane) with an online softmax; each lane keeps a
+// partial output over its keys, reduced across the warp at the end.
+template <int DH>
+__global__ void attn_f32_kernel(const float *__restrict__ q, const float *__restrict__ ck,
+                                const float *__restrict__ cv, const int32_t *__restrict__ rows,
+                                int M, int n_ctx, int n_heads, float *__restrict__ o) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= M * n_heads) return;
+  int j = warp / n_heads, hh = warp % n_heads;
+  int d = n_heads * DH;
+  int b = rows[j] / n_ctx;
+  const float *qv = q + (size_t)j * d + hh * DH;
+  float qr[DH];
+#pragma unroll
+  for (int i = 0; i < DH; ++i) qr[i] = qv[i];
+  const float scale = rsqrtf((float)DH);
+  float m = -INFINITY, l = 0.f;
+  float acc[DH];
+#pragma unroll
+  for (int i = 0; i < DH; ++i) acc[i] = 0.f;
+  for (int n0 = 0; n0 < n_ctx; n0 += 32) {
+    int n = n0 + lane;
+    float sc = -INFINITY;
+    const size_t kr = ((size_t)b * n_ctx + n) * d + hh * DH;
+    if (n < n_ctx) {
+      float dot = 0.f;
+#pragma unroll
+      for (int i = 0; i < DH; ++i) dot = fmaf(qr[i], ck[kr + i], dot);
+      sc = dot * scale;
+    }
+    float cm = warp_max(sc);
+    float mn = fmaxf(m, cm);
+    float corr = __expf(m - mn);
+    float pe = (n < n_ctx) ? __expf(sc - mn) : 0.f;
+    l = l * corr + warp_sum(pe);
+#pragma unroll
+    for (int i = 0; i < DH; ++i) acc[i] *= corr;
+    if (n < n_ctx) {
+#pragma unroll
+      for (int i = 0; i < DH; ++i) acc[i] = fmaf(pe, cv[kr + i], acc[i]);
+    }
+    m = mn;
+  }
+  float *ov = o + (size_t)j * d + hh * DH;
+#pragma unroll
+  for (int i = 0; i < DH; ++i) {
+    float v = warp_sum(acc[i]);
+    if (lane == 0) ov[i] = v / l;
+  }
+}
+
+cudaError_t launch_attn_f32(const float *q, const float *ck, const float *cv,
+                            const int32_t *rows, int M, int n_ctx, int n_heads, int head_dim,
+                            float *o, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  int warps = M * n_heads;
+  int blocks = (warps * 32 + 255) / 256;
+  switch (head_dim) {
+    case 8: attn_f32_kernel<8><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 16: attn_f32_kernel<16><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 32: attn_f32_kernel<32><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 64: attn_f32_kernel<64><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sl
