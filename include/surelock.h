@@ -266,6 +266,7 @@ typedef struct sl_timing {
   double bytes[SL_K_COUNT];
   double flops[SL_K_COUNT];
   long long launches[SL_K_COUNT];
+  long long kernels;     /* kernels this library launched (all classes, all objects) */
 } sl_timing;
 sl_status sl_timing_enable(sl_model *m, int enable);
 /* Synchronises the recorded events, returns the sums since the last reset. */

@@ -58,7 +58,8 @@ class SamplerState(C.Structure):
 
 class Timing(C.Structure):
     _fields_ = [("ms", C.c_double * K_COUNT), ("bytes", C.c_double * K_COUNT),
-                ("flops", C.c_double * K_COUNT), ("launches", C.c_longlong * K_COUNT)]
+                ("flops", C.c_double * K_COUNT), ("launches", C.c_longlong * K_COUNT),
+                ("kernels", C.c_longlong)]
 
 
 _P = C.c_void_p

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <array>
 #include <string>
 #include <vector>
@@ -52,6 +53,10 @@ int *device_error_word() {
   }
   return words[dev];
 }
+
+static std::atomic<long long> g_launches{0};
+void note_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+long long launches_total() { return g_launches.load(std::memory_order_relaxed); }
 
 static int sm_count() {
   int dev = 0, n = 148;
@@ -100,6 +105,7 @@ struct sl_model {
   std::vector<cudaEvent_t> ev_free;
   std::vector<TimingRec> recs;
   sl_timing acc{};
+  long long launch_base = 0;
 };
 
 struct sl_kv_cache {
@@ -280,10 +286,17 @@ extern "C" sl_status sl_timing_enable(sl_model *m, int enable) {
   return SL_OK;
 }
 
-extern "C" sl_status sl_timing_read(sl_model *m, sl_timing *out, int reset) {
-  if (!m || !out) return fail(SL_ERR_INVALID, "sl_timing_read: null argument");
-  for (auto &r : m->recs) {
-    if (cudaEventSynchronize(r.e1) != cudaSuccess) return cuda_fail(cudaGetLastError(), "event sync");
+// Fold completed timing records into the totals and recycle their events.
+// With `wait`, block until every record has completed.
+static sl_status timing_harvest(sl_model *m, bool wait) {
+  size_t i = 0;
+  for (; i < m->recs.size(); ++i) {
+    TimingRec &r = m->recs[i];
+    if (wait) {
+      if (cudaEventSynchronize(r.e1) != cudaSuccess) return cuda_fail(cudaGetLastError(), "event sync");
+    } else if (cudaEventQuery(r.e1) != cudaSuccess) {
+      break;
+    }
     float ms = 0.f;
     cudaEventElapsedTime(&ms, r.e0, r.e1);
     m->acc.ms[r.cls] += ms;
@@ -293,9 +306,21 @@ extern "C" sl_status sl_timing_read(sl_model *m, sl_timing *out, int reset) {
     m->ev_free.push_back(r.e0);
     m->ev_free.push_back(r.e1);
   }
-  m->recs.clear();
+  m->recs.erase(m->recs.begin(), m->recs.begin() + i);
+  cudaGetLastError();   // clear cudaErrorNotReady left by the query
+  return SL_OK;
+}
+
+extern "C" sl_status sl_timing_read(sl_model *m, sl_timing *out, int reset) {
+  if (!m || !out) return fail(SL_ERR_INVALID, "sl_timing_read: null argument");
+  sl_status st = timing_harvest(m, true);
+  if (st != SL_OK) return st;
+  m->acc.kernels = launches_total() - m->launch_base;
   *out = m->acc;
-  if (reset) memset(&m->acc, 0, sizeof(m->acc));
+  if (reset) {
+    memset(&m->acc, 0, sizeof(m->acc));
+    m->launch_base = launches_total();
+  }
   return SL_OK;
 }
 
@@ -507,9 +532,13 @@ struct Plan {
 // Choose the tile width and K split of one GEMM: minimise the modelled
 // makespan  waves * per-unit time, where a unit streams kb_per_split K-blocks
 // of a BN-row weight tile (HBM-bound at small M) or issues their MMAs
-// (tensor-bound at large M), plus a fixed per-unit overhead.
-Plan plan_gemm(int M, int N, int K, bool allow_split, int num_sms, bool swiglu) {
-  const double bw_sm = 6.5e12 / num_sms;         // bytes/s per SM
+// (tensor-bound at large M), plus a fixed per-unit overhead and, for split-K,
+// the fp32 partial-sum traffic (atomics, and for SPLIT_ACCUM the finalize pass).
+enum SplitKind { SPLIT_NONE = 0, SPLIT_RESID = 1, SPLIT_ACCUM = 2 };
+
+Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu) {
+  const double bw = 6.5e12;
+  const double bw_sm = bw / num_sms;             // bytes/s per SM
   const double fl_sm = 1.6e15 / num_sms;         // flop/s per SM at N=256 tiles
   const int mt = (M + 127) / 128;
   const int kblocks = K / 64;
@@ -520,7 +549,7 @@ Plan plan_gemm(int M, int N, int K, bool allow_split, int num_sms, bool swiglu) 
     if (N % bn) continue;
     if (swiglu && (N / 2) % (bn / 2)) continue;
     const double mma_eff = bn == 256 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
-    const int max_s = allow_split ? std::min(32, std::max(1, kblocks / 4)) : 1;
+    const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
     for (int s = 1; s <= max_s; ++s) {
       const int kbp = (kblocks + s - 1) / s;
       const int ss = (kblocks + kbp - 1) / kbp;
@@ -529,7 +558,10 @@ Plan plan_gemm(int M, int N, int K, bool allow_split, int num_sms, bool swiglu) 
       const double t_mem = kbp * (bn * 128.0 + 128 * 128.0 * 0.25) / bw_sm;
       const double t_mma = kbp * (2.0 * 128 * bn * 64) / (fl_sm * mma_eff);
       double t = waves * (std::max(t_mem, t_mma) + 1.0e-6);
-      if (ss > 1) t += 3.0e-6;                    // finalize / atomics overhead
+      if (ss > 1) {
+        t += (double)M * N * 4.0 * ss / bw;                          // fp32 atomics
+        if (split_kind == SPLIT_ACCUM) t += (double)M * N * 4.0 * 2 / bw + 3.0e-6;   // finalize
+      }
       if (t < best.cost - 1e-9) best = Plan{bn, ss, t};
     }
   }
@@ -598,11 +630,11 @@ struct BfPlans {
 static BfPlans plans_for(const sl_config &cfg, int M, int ns) {
   const int d = cfg.d_model, f = cfg.d_ffn;
   BfPlans p;
-  p.qkv = plan_gemm(M, 3 * d, d, true, ns, false);
-  p.o = plan_gemm(M, d, d, true, ns, false);
-  p.gu = plan_gemm(M, 2 * f, d, true, ns, true);
-  p.dn = plan_gemm(M, d, f, true, ns, false);
-  p.hd = plan_gemm(M, cfg.vocab, d, false, ns, false);
+  p.qkv = plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false);
+  p.o = plan_gemm(M, d, d, SPLIT_RESID, ns, false);
+  p.gu = plan_gemm(M, 2 * f, d, SPLIT_ACCUM, ns, true);
+  p.dn = plan_gemm(M, d, f, SPLIT_RESID, ns, false);
+  p.hd = plan_gemm(M, cfg.vocab, d, SPLIT_NONE, ns, false);
   return p;
 }
 
@@ -785,8 +817,13 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   g.out = d_logits;
   g.ldo = V;
   g.row_map = a->rows;
-  Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 2), 2.0 * (double)M * d * V, s);
-  return tc_gemm(m, g, s);
+  {
+    Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 2), 2.0 * (double)M * d * V, s);
+    if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
+  }
+  // the previous step's timing events completed before this step was planned
+  if (m->timing) timing_harvest(m, false);
+  return SL_OK;
 }
 
 extern "C" sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
@@ -851,7 +888,8 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   if (M == 0) return SL_OK;
   const int ns = sm_count();
   if (bn == 0) {
-    Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID || epi == SL_GEMM_ACCUM, ns, swiglu);
+    Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID ? SPLIT_RESID
+                                : epi == SL_GEMM_ACCUM ? SPLIT_ACCUM : SPLIT_NONE, ns, swiglu);
     bn = p.bn;
     if (splits <= 0) splits = p.splits;
   }
@@ -1060,6 +1098,7 @@ extern "C" sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, v
       d_prompts, s->batch, s->p.prompt_len, s->n_ctx, s->m->cfg.mask_id, s->tokens, s->masked,
       s->locked, s->lock_t);
   SL_CUDA(cudaGetLastError());
+  note_launch();
   sl_status r = sl_kv_cache_reset(s->cache, stream);
   if (r != SL_OK) return r;
   r = sl_active_reset(s->act, stream);

@@ -313,12 +313,12 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
   p.splits = splits;
   p.kblocks = kblocks;
   dim3 grid(tiles, n_heads, splits);
-  attn_bf16_kernel<<<grid, AT_THREADS, AT_SMEM, s>>>(p);
+  attn_bf16_kernel<<<grid, AT_THREADS, AT_SMEM, s>>>(p); note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
   int warps = M * n_heads;
   attn_combine_kernel<<<(warps * 32 + 255) / 256, 256, 0, s>>>(p.ws_o, p.ws_ml, M, n_heads,
-                                                                splits, (bf16 *)o);
+                                                                splits, (bf16 *)o); note_launch();
   return cudaGetLastError();
 }
 

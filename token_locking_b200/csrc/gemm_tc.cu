@@ -441,7 +441,7 @@ static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  gemm_tc_kernel<BN, STAGES, EPI><<<grid, 192, L::TOTAL, s>>>(p);
+  gemm_tc_kernel<BN, STAGES, EPI><<<grid, 192, L::TOTAL, s>>>(p); note_launch();
   return cudaGetLastError();
 }
 

@@ -14,6 +14,8 @@ namespace sl {
 sl_status fail(sl_status st, const char *fmt, ...);
 sl_status cuda_fail(cudaError_t e, const char *what);
 int *device_error_word();   // per-device int, allocated on first use; nullptr on failure
+void note_launch(int n = 1); // count kernels launched by this library
+long long launches_total();
 
 #define SL_CUDA(call)                                  \
   do {                                                 \

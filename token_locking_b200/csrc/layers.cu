@@ -26,10 +26,11 @@ __global__ void gather_embed_kernel(const int32_t *__restrict__ tokens,
 cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
                                 const void *emb, int d, float *h, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  if (dtype == SL_BF16)
-    gather_embed_kernel<bf16><<<M, 256, 0, s>>>(tokens, rows, M, (const bf16 *)emb, d, h);
-  else
-    gather_embed_kernel<float><<<M, 256, 0, s>>>(tokens, rows, M, (const float *)emb, d, h);
+  if (dtype == SL_BF16) {
+    gather_embed_kernel<bf16><<<M, 256, 0, s>>>(tokens, rows, M, (const bf16 *)emb, d, h); note_launch();
+  } else {
+    gather_embed_kernel<float><<<M, 256, 0, s>>>(tokens, rows, M, (const float *)emb, d, h); note_launch();
+  }
   return cudaGetLastError();
 }
 
@@ -62,10 +63,11 @@ cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, floa
                            void *out, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   int th = d >= 1024 ? 512 : 128;
-  if (dtype == SL_BF16)
-    rmsnorm_kernel<bf16><<<M, th, 0, s>>>(h, (const bf16 *)g, d, eps, M, (bf16 *)out);
-  else
-    rmsnorm_kernel<float><<<M, th, 0, s>>>(h, (const float *)g, d, eps, M, (float *)out);
+  if (dtype == SL_BF16) {
+    rmsnorm_kernel<bf16><<<M, th, 0, s>>>(h, (const bf16 *)g, d, eps, M, (bf16 *)out); note_launch();
+  } else {
+    rmsnorm_kernel<float><<<M, th, 0, s>>>(h, (const float *)g, d, eps, M, (float *)out); note_launch();
+  }
   return cudaGetLastError();
 }
 
@@ -120,15 +122,16 @@ cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool
   if (M <= 0) return cudaSuccess;
   int th = 256;
   if (dtype == SL_BF16) {
-    if (in_f32)
+    if (in_f32) {
       rope_scatter_kernel<float, bf16><<<M, th, 0, s>>>((float *)qkv_in, zero_in, M, rows, n_ctx,
-          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv);
-    else
+          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv); note_launch();
+    } else {
       rope_scatter_kernel<bf16, bf16><<<M, th, 0, s>>>((bf16 *)qkv_in, false, M, rows, n_ctx,
-          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv);
+          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv); note_launch();
+    }
   } else {
     rope_scatter_kernel<float, float><<<M, th, 0, s>>>((float *)qkv_in, zero_in, M, rows, n_ctx,
-        n_heads, head_dim, rope, (float *)q_out, (float *)ck, (float *)cv);
+        n_heads, head_dim, rope, (float *)q_out, (float *)ck, (float *)cv); note_launch();
   }
   return cudaGetLastError();
 }
@@ -152,12 +155,13 @@ cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, 
                           void *act, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   if (dtype == SL_BF16) {
-    if (in_f32)
-      swiglu_kernel<float, bf16><<<M, 512, 0, s>>>((float *)ws, zero_in, M, F, (bf16 *)act);
-    else
-      swiglu_kernel<bf16, bf16><<<M, 512, 0, s>>>((bf16 *)ws, false, M, F, (bf16 *)act);
+    if (in_f32) {
+      swiglu_kernel<float, bf16><<<M, 512, 0, s>>>((float *)ws, zero_in, M, F, (bf16 *)act); note_launch();
+    } else {
+      swiglu_kernel<bf16, bf16><<<M, 512, 0, s>>>((bf16 *)ws, false, M, F, (bf16 *)act); note_launch();
+    }
   } else {
-    swiglu_kernel<float, float><<<M, 256, 0, s>>>((float *)ws, zero_in, M, F, (float *)act);
+    swiglu_kernel<float, float><<<M, 256, 0, s>>>((float *)ws, zero_in, M, F, (float *)act); note_launch();
   }
   return cudaGetLastError();
 }
@@ -219,7 +223,7 @@ cudaError_t launch_gemm_f32(int epi, const float *A, int M, int K, const float *
                             cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   dim3 grid((N + FT - 1) / FT, (M + FT - 1) / FT);
-  gemm_f32_kernel<<<grid, 256, 0, s>>>(epi, A, M, K, B, N, C, ldc, col_off, row_map);
+  gemm_f32_kernel<<<grid, 256, 0, s>>>(epi, A, M, K, B, N, C, ldc, col_off, row_map); note_launch();
   return cudaGetLastError();
 }
 
@@ -284,10 +288,10 @@ cudaError_t launch_attn_f32(const float *q, const float *ck, const float *cv,
   int warps = M * n_heads;
   int blocks = (warps * 32 + 255) / 256;
   switch (head_dim) {
-    case 8: attn_f32_kernel<8><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
-    case 16: attn_f32_kernel<16><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
-    case 32: attn_f32_kernel<32><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
-    case 64: attn_f32_kernel<64><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 8: attn_f32_kernel<8><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
+    case 16: attn_f32_kernel<16><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
+    case 32: attn_f32_kernel<32><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
+    case 64: attn_f32_kernel<64><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -214,8 +214,7 @@ cudaError_t launch_lock_stats(const LockStatsArgs &a, cudaStream_t s) {
   const long blocks = (long)a.splits * a.M;
   if (blocks > 0x7fffffffL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)blocks);
-  if (a.dtype == SL_BF16) lock_stats_kernel<bf16><<<grid, LOCK_THREADS, 0, s>>>(a);
-  else lock_stats_kernel<float><<<grid, LOCK_THREADS, 0, s>>>(a);
+  if (a.dtype == SL_BF16) { lock_stats_kernel<bf16><<<grid, LOCK_THREADS, 0, s>>>(a); note_launch(); } else { lock_stats_kernel<float><<<grid, LOCK_THREADS, 0, s>>>(a); note_launch(); }
   return cudaGetLastError();
 }
 
@@ -346,7 +345,7 @@ cudaError_t launch_lock_decide(const int32_t *seq_off, int batch, const int32_t 
                                float eps, float gate_q, int has_prev, int scripted_target,
                                uint8_t *lock, cudaStream_t s) {
   lock_decide_kernel<<<batch, DEC_THREADS, 0, s>>>(seq_off, rows, kl, unc, masked, eps, gate_q,
-                                                    has_prev, scripted_target, lock);
+                                                    has_prev, scripted_target, lock); note_launch();
   return cudaGetLastError();
 }
 
@@ -407,7 +406,7 @@ __global__ void __launch_bounds__(DEC_THREADS) compact_kernel(
 
 cudaError_t launch_compact(int32_t *rows, int32_t *seq_off, int batch, const uint8_t *lock,
                            uint8_t *locked, int32_t *lock_t, int step, cudaStream_t s) {
-  compact_kernel<<<1, DEC_THREADS, 0, s>>>(rows, seq_off, batch, lock, locked, lock_t, step);
+  compact_kernel<<<1, DEC_THREADS, 0, s>>>(rows, seq_off, batch, lock, locked, lock_t, step); note_launch();
   return cudaGetLastError();
 }
 
@@ -456,7 +455,7 @@ cudaError_t launch_unmask(const int32_t *seq_off, int batch, const int32_t *rows
                           int32_t *tokens, uint8_t *masked, cudaStream_t s) {
   if (hi - lo > UNMASK_MAX_CAND) return cudaErrorInvalidValue;
   unmask_kernel<<<batch, 256, 0, s>>>(seq_off, rows, n_ctx, conf, argmax, lo, hi, k, tokens,
-                                      masked);
+                                      masked); note_launch();
   return cudaGetLastError();
 }
 
@@ -472,7 +471,7 @@ cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n
                                cudaStream_t s) {
   int total = batch * n_ctx;
   int n = total > batch + 1 ? total : batch + 1;
-  active_fill_kernel<<<(n + 255) / 256, 256, 0, s>>>(rows, seq_off, batch, n_ctx);
+  active_fill_kernel<<<(n + 255) / 256, 256, 0, s>>>(rows, seq_off, batch, n_ctx); note_launch();
   return cudaGetLastError();
 }
 

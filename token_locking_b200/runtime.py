@@ -103,8 +103,10 @@ class Model:
         t = A.Timing()
         A.check(A.lib().sl_timing_read(self.handle, C.byref(t), 1 if reset else 0), "sl_timing_read")
         names = ["gemm", "attn", "lock", "other"]
-        return {n: {"ms": t.ms[i], "bytes": t.bytes[i], "flops": t.flops[i],
-                    "launches": int(t.launches[i])} for i, n in enumerate(names)}
+        out = {n: {"ms": t.ms[i], "bytes": t.bytes[i], "flops": t.flops[i],
+                   "launches": int(t.launches[i])} for i, n in enumerate(names)}
+        out["kernels"] = int(t.kernels)
+        return out
 
 
 class KVCache:
