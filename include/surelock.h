@@ -214,6 +214,30 @@ sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b, 
                        int N, void *d_out, int ldo, const int32_t *d_row_map, int bn, int splits,
                        void *stream);
 
+/* The per-row statistics of sl_kl_lock (lse, D, u, conf, argmax; no gate and
+ * no lock flags) for callers that cannot allocate device memory: hosts whose
+ * device memory is owned by another runtime's pool (a serving engine that
+ * reserves nearly all of HBM at start-up, so cudaMalloc would fail), and code
+ * that must not trigger cudaMalloc's implicit device synchronisation.  It
+ * allocates nothing: the split-reduction scratch is a static device array
+ * built into this library (about 560 KB per GPU that loads it, kept until the
+ * process exits).  The pages have no counterpart; this is a library-level
+ * entry point.
+ *   d_rows [M]: flat positions of the rows to test, as in sl_active.
+ *   Outputs as sl_kl_lock: d_kl, d_unc, d_conf, d_argmax by row index j,
+ *   d_lse_cur at position d_rows[j].  has_prev = 0 writes D = +inf.
+ * Limits: 0 <= M <= 8192 (SL_ERR_INVALID otherwise); vocab % 8 == 0.
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, once per device); make that first call before any
+ * stream capture.  All calls share the one scratch array, so calls whose
+ * kernels overlap on the GPU (other streams, other threads) race and corrupt
+ * each other's results: serialise them. */
+sl_status sl_kl_stats_noalloc(const int32_t *d_rows, int M, int vocab, int mask_id,
+                              int logits_dtype, const void *d_logits_cur,
+                              const void *d_logits_prev, const float *d_lse_prev,
+                              float *d_lse_cur, int has_prev, float *d_kl, float *d_unc,
+                              float *d_conf, int32_t *d_argmax, void *stream);
+
 /* ---------------------------------------------------------------- sampler --- */
 
 /* Semi-autoregressive SureLock decode driven by the library: prompt_len given

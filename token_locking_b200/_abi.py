@@ -83,6 +83,7 @@ SIGNATURES = {
     "sl_step": (_I, [_P, _P, _P, _P, _P, _P]),
     "sl_kl_lock": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, C.POINTER(LockParams),
                         _P, _P, _P, _P, _P, _P]),
+    "sl_kl_stats_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
     "sl_unmask_topk": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "sl_compact_active": (_I, [_P, _P, _P, _P, _I, _P]),
     "sl_sampler_create": (_I, [_P, _I, C.POINTER(SamplerParams), C.POINTER(_P)]),

@@ -11,6 +11,8 @@
 //   schedule (radix select on (D, position)); writes the lock flags.
 // compact: stable block-wide ballot/prefix-sum compaction of the active list.
 // unmask: top-k confidence among the masked rows of the current block.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -476,3 +478,100 @@ cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n
 }
 
 }  // namespace sl
+
+// ---------------------------------------------------- no-allocation variant --
+// The per-row sure-test statistics for callers that cannot allocate device
+// memory.  The chunk records and tickets that the split reduction needs live
+// in this file-scope array instead of a workspace: NOALLOC_MAX_RECORDS
+// (row, vocab-chunk) records of two float4 each, followed by one ticket
+// counter per row for up to NOALLOC_MAX_ROWS rows (about 560 KB per GPU that
+// loads the library, held until the process exits).
+namespace sl {
+namespace {
+constexpr int NOALLOC_MAX_ROWS = 8192;
+constexpr int NOALLOC_MAX_RECORDS = 16384;
+constexpr int NOALLOC_FLOAT4S = NOALLOC_MAX_RECORDS * 2 + NOALLOC_MAX_ROWS / 4;
+static __device__ __align__(256) float4 g_noalloc_scratch[NOALLOC_FLOAT4S];
+
+// Host-side device address of g_noalloc_scratch, resolved once per device.
+// In host code the symbol itself is only a stand-in, never a device pointer.
+struct NoallocSlot {
+  bool ready;
+  float4 *ptr;
+};
+NoallocSlot g_noalloc_slots[64];
+std::mutex g_noalloc_mu;
+}  // namespace
+}  // namespace sl
+
+extern "C" sl_status sl_kl_stats_noalloc(const int32_t *d_rows, int M, int vocab, int mask_id,
+                                         int logits_dtype, const void *d_logits_cur,
+                                         const void *d_logits_prev, const float *d_lse_prev,
+                                         float *d_lse_cur, int has_prev, float *d_kl,
+                                         float *d_unc, float *d_conf, int32_t *d_argmax,
+                                         void *stream) {
+  using namespace sl;
+  if (M < 0 || M > NOALLOC_MAX_ROWS)
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: M = %d outside [0, %d], the size of its "
+                "built-in scratch", M, NOALLOC_MAX_ROWS);
+  if (M == 0) return SL_OK;
+  if (!d_rows || !d_logits_cur || !d_lse_cur || !d_kl || !d_unc || !d_conf || !d_argmax)
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: null argument");
+  if (has_prev && (!d_logits_prev || !d_lse_prev))
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: has_prev needs previous logits and lse");
+  if (vocab <= 0 || vocab % 8 != 0)
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: vocab must be a positive multiple of 8");
+  if (mask_id < -1 || mask_id >= vocab)
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: bad mask_id");
+  if (logits_dtype != SL_F32 && logits_dtype != SL_BF16)
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: bad dtype");
+  if (((uintptr_t)d_logits_cur & 15) || (d_logits_prev && ((uintptr_t)d_logits_prev & 15)))
+    return fail(SL_ERR_INVALID, "sl_kl_stats_noalloc: logits must be 16-byte aligned");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "sl_kl_stats_noalloc: cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(SL_ERR_UNSUPPORTED, "sl_kl_stats_noalloc: device %d", dev);
+  float4 *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> g(g_noalloc_mu);
+    NoallocSlot &slot = g_noalloc_slots[dev];
+    if (!slot.ready) {
+      e = cudaGetSymbolAddress((void **)&slot.ptr, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "sl_kl_stats_noalloc: cudaGetSymbolAddress");
+      slot.ready = true;
+    }
+    scratch = slot.ptr;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int splits = lock_stats_splits(M, vocab, sms);
+  if (splits > NOALLOC_MAX_RECORDS / M) splits = NOALLOC_MAX_RECORDS / M;
+  if (splits < 1) splits = 1;
+  unsigned int *tickets = reinterpret_cast<unsigned int *>(scratch + NOALLOC_MAX_RECORDS * 2);
+  cudaStream_t s = (cudaStream_t)stream;
+  // tickets must start at zero; the array keeps whatever the last call left
+  e = cudaMemsetAsync(tickets, 0, (size_t)M * sizeof(unsigned int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "sl_kl_stats_noalloc: clearing tickets");
+  LockStatsArgs a;
+  a.dtype = logits_dtype;
+  a.cur = d_logits_cur;
+  a.prev = d_logits_prev;
+  a.lse_prev = d_lse_prev;
+  a.lse_cur = d_lse_cur;
+  a.rows = d_rows;
+  a.M = M;
+  a.V = vocab;
+  a.mask_id = mask_id;
+  a.has_prev = has_prev ? 1 : 0;
+  a.kl = d_kl;
+  a.unc = d_unc;
+  a.conf = d_conf;
+  a.argmax = d_argmax;
+  a.part = scratch;
+  a.counters = tickets;
+  a.splits = splits;
+  e = launch_lock_stats(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sl_kl_stats_noalloc: launch");
+  return SL_OK;
+}
+

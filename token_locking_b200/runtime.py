@@ -255,6 +255,22 @@ def kl_lock(active: Active, vocab: int, mask_id: int, logits_cur: torch.Tensor,
                                _ptr(argmax), _ptr(lock), _stream(stream)), "sl_kl_lock")
 
 
+def kl_stats_noalloc(rows: torch.Tensor, vocab: int, mask_id: int, logits_cur: torch.Tensor,
+                     logits_prev: Optional[torch.Tensor], lse_prev: Optional[torch.Tensor],
+                     lse_cur: torch.Tensor, kl: torch.Tensor, unc: torch.Tensor,
+                     conf: torch.Tensor, argmax: torch.Tensor, has_prev: bool = True,
+                     stream=None):
+    """Sure-test statistics without any device allocation by the library
+    (sl_kl_stats_noalloc): for hosts that own all device memory themselves."""
+    if rows.dtype != torch.int32:
+        raise ValueError("rows must be int32")
+    A.check(A.lib().sl_kl_stats_noalloc(_ptr(rows), rows.numel(), vocab, mask_id,
+                                        _dtype_code(logits_cur.dtype), _ptr(logits_cur),
+                                        _ptr(logits_prev), _ptr(lse_prev), _ptr(lse_cur),
+                                        1 if has_prev else 0, _ptr(kl), _ptr(unc), _ptr(conf),
+                                        _ptr(argmax), _stream(stream)), "sl_kl_stats_noalloc")
+
+
 def unmask_topk(active: Active, conf: torch.Tensor, argmax: torch.Tensor, block_lo: int,
                 block_hi: int, k: int, tokens: torch.Tensor, masked: torch.Tensor, stream=None):
     A.check(A.lib().sl_unmask_topk(active.handle, _ptr(conf), _ptr(argmax), block_lo, block_hi, k,
