@@ -261,11 +261,9 @@ def run_ours(args, rank: int, world: int):
     for _ in range(args.warmup):
         decode()
     torch.cuda.synchronize()
-    model.timing_read(reset=True)
-    model.timing_enable(True)
-    model.timing_read(reset=True)
     clocks = ClockSampler(gpu_id_for(dev), os.path.join(args.out_dir, f"clocks_rank{rank}.csv")) \
         if rank == 0 else None
+    model.timing_read(reset=True)           # zero the library's kernel-launch counter
     barrier()
     torch.cuda.synchronize()
     if clocks:
@@ -279,10 +277,29 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     ms_local = ev0.elapsed_time(ev1)
     clk = clocks.stop() if clocks else None
+    kernels_timed = model.timing_read(reset=True)["kernels"]
     barrier()
+    ms = max_over_ranks(ms_local)
+
+    # Per-kernel CUDA events around every GEMM / attention / lock launch.  An
+    # event between two kernels also removes the programmatic-launch overlap at
+    # that boundary, so this instrumented pass over the same K decodes is timed
+    # separately from the headline number above.
+    model.timing_read(reset=True)
+    model.timing_enable(True)
+    model.timing_read(reset=True)
+    barrier()
+    torch.cuda.synchronize()
+    ei0, ei1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ei0.record()
+    for _ in range(args.steps):
+        decode()
+    ei1.record()
+    torch.cuda.synchronize()
+    ms_instr = max_over_ranks(ei0.elapsed_time(ei1))
     model.timing_enable(False)
     tim = model.timing_read(reset=True)
-    ms = max_over_ranks(ms_local)
+    barrier()
 
     # trajectory of the last decode and per-step times of one more (untimed) decode
     st = s.state()
@@ -382,7 +399,9 @@ def run_ours(args, rank: int, world: int):
                          "frac": round(ach / peak, 4), "traffic": None,
                          "kernel": "gemm_tc_kernel (tcgen05)",
                          "launches": g["launches"], "kernel_ms": round(g["ms"], 3),
-                         "peak_source": peaks["source"]},
+                         "peak_source": peaks["source"],
+                         "measured_in": f"instrumented pass of the same {args.steps} decodes "
+                                        f"({ms_instr / args.steps:.1f} ms/decode with events)"},
             "step_roofline": {"frac": round(step_frac, 4), "roofline_ms_per_decode":
                               round(sum(roof) * 1e3, 3), "measured_ms_per_decode":
                               round(decode_ms, 3), "peaks": "burst (bf16_tflops, hbm_gbs)"},
@@ -391,7 +410,7 @@ def run_ours(args, rank: int, world: int):
             "curve": curve,
             "cpu_baseline": cpu,
             "clocks": clk,
-            "gpu_launches": int(tim["kernels"]),
+            "gpu_launches": int(kernels_timed),
         }
     s.close()
     model.close()

@@ -207,8 +207,10 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
  *                   out bf16 [M][ldo] = silu(A W_gate^T) * (A W_up^T)
  *   SL_GEMM_ACCUM : out fp32 [M][ldo] += C (atomic; with d_b2, gate/up halves
  *                   accumulate into columns [0,F) and [F,2F))
- * bn (64/128/256) and splits (>= 1, RESID/ACCUM only) pick the tiling; bn = 0
- * lets the library choose.  K % 64 == 0, N % bn == 0, pointers 16-byte aligned. */
+ * bn (64/128/256) and splits (>= 1, RESID/ACCUM only) pick the tiling, with
+ * 128 rows of A per tile; -64/-128/-256 select 256-row tiles (two tensor-core
+ * accumulators share each weight tile); bn = 0 lets the library choose.
+ * K % 64 == 0, N % |bn| == 0, pointers 16-byte aligned. */
 enum { SL_GEMM_STORE = 0, SL_GEMM_RESID = 1, SL_GEMM_SWIGLU = 2, SL_GEMM_ACCUM = 3 };
 sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b, const void *d_b2,
                        int N, void *d_out, int ldo, const int32_t *d_row_map, int bn, int splits,

@@ -28,7 +28,7 @@ def _close(got, ref, K, bf16_out):
     assert err <= tol, f"max err {err} > tol {tol} (scale {scale})"
 
 
-@pytest.mark.parametrize("bn", [64, 128, 256])
+@pytest.mark.parametrize("bn", [64, 128, 256, -64, -128, -256])
 @pytest.mark.parametrize("M", [1, 37, 128, 301])
 def test_store_rowmap(cuda_dev, bn, M):
     K, N = 512, 768
@@ -45,8 +45,9 @@ def test_store_rowmap(cuda_dev, bn, M):
     rt.device_check()
 
 
-@pytest.mark.parametrize("bn,splits", [(64, 1), (128, 3), (256, 2), (128, 8)])
-@pytest.mark.parametrize("M", [5, 130])
+@pytest.mark.parametrize("bn,splits", [(64, 1), (128, 3), (256, 2), (128, 8), (-256, 3),
+                                       (-128, 1), (-64, 2)])
+@pytest.mark.parametrize("M", [5, 130, 600])
 def test_resid_split(cuda_dev, bn, splits, M):
     K, N = 1024, 512
     a, b = _mk((M, K), 4, cuda_dev), _mk((N, K), 5, cuda_dev)
@@ -58,11 +59,11 @@ def test_resid_split(cuda_dev, bn, splits, M):
     rt.device_check()
 
 
-@pytest.mark.parametrize("bn", [64, 128, 256])
-@pytest.mark.parametrize("M", [3, 129])
+@pytest.mark.parametrize("bn", [64, 128, 256, -128, -256])
+@pytest.mark.parametrize("M", [3, 129, 300])
 def test_swiglu(cuda_dev, bn, M):
     K, F = 256, 384
-    if F % (bn // 2):
+    if F % (abs(bn) // 2):
         pytest.skip("F must split into bn/2 halves")
     a = _mk((M, K), 7, cuda_dev)
     wg, wu = _mk((F, K), 8, cuda_dev) * 0.1, _mk((F, K), 9, cuda_dev) * 0.1

@@ -379,9 +379,10 @@ extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
        alloc(&c->qkv, rows * 3 * d * es) && alloc(&c->q, rows * d * es) &&
        alloc(&c->o, rows * d * es) && alloc(&c->act, rows * f * es) &&
        alloc((void **)&c->ws, rows * wsc * 4);
-  if (ok && cfg.dtype == SL_BF16)
+  if (ok && cfg.dtype == SL_BF16) {
     ok = alloc((void **)&c->attn_ws, attn_bf16_workspace_bytes(c->max_rows, cfg.n_heads,
                                                                c->attn_max_splits));
+  }
   if (ok) {
     // rotary table in double precision: angle = pos * theta^(-2i/dh)
     const int half = cfg.head_dim / 2;
@@ -525,44 +526,53 @@ extern "C" sl_status sl_active_view(const sl_active *a, int32_t **d_rows, int32_
 namespace {
 
 struct Plan {
-  int bn, splits;
+  int bn, splits, msub;
   double cost;
 };
 
-// Choose the tile width and K split of one GEMM: minimise the modelled
-// makespan  waves * per-unit time, where a unit streams kb_per_split K-blocks
-// of a BN-row weight tile (HBM-bound at small M) or issues their MMAs
-// (tensor-bound at large M), plus a fixed per-unit overhead and, for split-K,
-// the fp32 partial-sum traffic (atomics, and for SPLIT_ACCUM the finalize pass).
+// Choose the tile shape (BN, 128 or 256 rows per unit) and K split of one
+// GEMM by a small cost model: the kernel time is the largest of the weight
+// stream from HBM (read once), the operand traffic from L2 into the SMs (every
+// unit re-reads its A and B tiles), and the tensor-core time of the padded
+// tiles, stretched by wave quantisation over the SMs, plus a fixed cost per
+// wave and, for split-K, the fp32 partial-sum traffic (atomics, and for
+// SPLIT_ACCUM the finalize pass).
 enum SplitKind { SPLIT_NONE = 0, SPLIT_RESID = 1, SPLIT_ACCUM = 2 };
 
-Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu) {
-  const double bw = 6.5e12;
-  const double bw_sm = bw / num_sms;             // bytes/s per SM
-  const double fl_sm = 1.6e15 / num_sms;         // flop/s per SM at N=256 tiles
-  const int mt = (M + 127) / 128;
+Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, int min_bn = 64) {
+  const double bw_hbm = 6.5e12, bw_l2 = 9.0e12, peak = 1.6e15;
   const int kblocks = K / 64;
-  Plan best{0, 1, 1e30};
-  const int bns[3] = {256, 128, 64};
-  for (int bi = 0; bi < 3; ++bi) {
-    const int bn = bns[bi];
-    if (N % bn) continue;
-    if (swiglu && (N / 2) % (bn / 2)) continue;
-    const double mma_eff = bn == 256 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
-    const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
-    for (int s = 1; s <= max_s; ++s) {
-      const int kbp = (kblocks + s - 1) / s;
-      const int ss = (kblocks + kbp - 1) / kbp;
-      const long units = (long)mt * (N / bn) * ss;
-      const long waves = (units + num_sms - 1) / num_sms;
-      const double t_mem = kbp * (bn * 128.0 + 128 * 128.0 * 0.25) / bw_sm;
-      const double t_mma = kbp * (2.0 * 128 * bn * 64) / (fl_sm * mma_eff);
-      double t = waves * (std::max(t_mem, t_mma) + 1.0e-6);
-      if (ss > 1) {
-        t += (double)M * N * 4.0 * ss / bw;                          // fp32 atomics
-        if (split_kind == SPLIT_ACCUM) t += (double)M * N * 4.0 * 2 / bw + 3.0e-6;   // finalize
+  Plan best{0, 1, 1, 1e30};
+  for (int msub = 1; msub <= 2; ++msub) {
+    if (msub == 2 && M <= 128) continue;
+    const int rows_unit = 128 * msub;
+    const int mt = (M + rows_unit - 1) / rows_unit;
+    const double rows_live = std::min(M, rows_unit);
+    const int bns[3] = {256, 128, 64};
+    for (int bi = 0; bi < 3; ++bi) {
+      const int bn = bns[bi];
+      if (N % bn || bn < min_bn) continue;
+      if (swiglu && (N / 2) % (bn / 2)) continue;
+      const bool single_acc = 2 * msub * bn > 512;
+      const double mma_eff = bn == 256 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
+      const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
+      for (int sp = 1; sp <= max_s; ++sp) {
+        const int kbp = (kblocks + sp - 1) / sp;
+        const int ss = (kblocks + kbp - 1) / kbp;
+        const long units = (long)mt * (N / bn) * ss;
+        const long waves = (units + num_sms - 1) / num_sms;
+        const double quant = (double)(waves * num_sms) / units;
+        const double t_hbm = 2.0 * ((double)N * K + (double)M * K) / bw_hbm;
+        const double t_l2 = (double)units * kbp * (bn * 128.0 + rows_live * 128.0) / bw_l2;
+        const double t_mma = (double)units * kbp * 2.0 * rows_unit * bn * 64 / (peak * mma_eff);
+        double t = std::max(t_hbm, std::max(t_l2, t_mma)) * std::min(quant, 2.0) + waves * 1.0e-6;
+        if (single_acc && waves > 1) t += waves * 2.0e-6;     // epilogue not overlapped
+        if (ss > 1) {
+          t += (double)M * N * 4.0 * ss / bw_l2;                               // fp32 atomics
+          if (split_kind == SPLIT_ACCUM) t += (double)M * N * 8.0 / bw_hbm + 3.0e-6;   // finalize
+        }
+        if (t < best.cost - 1e-9) best = Plan{bn, ss, msub, t};
       }
-      if (t < best.cost - 1e-9) best = Plan{bn, ss, t};
     }
   }
   return best;
@@ -630,7 +640,7 @@ struct BfPlans {
 static BfPlans plans_for(const sl_config &cfg, int M, int ns) {
   const int d = cfg.d_model, f = cfg.d_ffn;
   BfPlans p;
-  p.qkv = plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false);
+  p.qkv = plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128);
   p.o = plan_gemm(M, d, d, SPLIT_RESID, ns, false);
   p.gu = plan_gemm(M, 2 * f, d, SPLIT_ACCUM, ns, true);
   p.dn = plan_gemm(M, d, f, SPLIT_RESID, ns, false);
@@ -693,17 +703,30 @@ static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, fl
     g.K = d;
     g.bn = pl.qkv.bn;
     g.splits = pl.qkv.splits;
+    g.msub = pl.qkv.msub;
     const bool split = pl.qkv.splits > 1;
-    g.epi = split ? EPI_ACCUM : EPI_STORE;
-    g.out = split ? (void *)c->ws : c->qkv;
-    g.ldo = 3 * d;
+    if (split) {
+      // K split across CTAs: fp32 partial sums, then RoPE + scatter from them
+      g.epi = EPI_ACCUM;
+      g.out = c->ws;
+      g.ldo = 3 * d;
+    } else {
+      // epilogue: RoPE(q) -> q, RoPE(k) and v -> C.k/C.v at the rows' positions
+      g.epi = EPI_QKV;
+      g.row_map = a->rows;
+      g.rope = c->rope;
+      g.n_ctx = c->n_ctx;
+      g.q_out = c->q;
+      g.ck = c->k[l];
+      g.cv = c->v[l];
+    }
     {
       Timed t(m, SL_K_GEMM, gemm_bytes(Md, 3.0 * d, d, 2), 6.0 * Md * d * d, s);
       if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
     }
-    SL_CUDA(launch_rope_scatter(SL_BF16, split ? (void *)c->ws : c->qkv, split, split, M,
-                                a->rows, c->n_ctx, H, cfg.head_dim, c->rope, c->q, c->k[l],
-                                c->v[l], s));
+    if (split)
+      SL_CUDA(launch_rope_scatter(SL_BF16, c->ws, true, true, M, a->rows, c->n_ctx, H,
+                                  cfg.head_dim, c->rope, c->q, c->k[l], c->v[l], s));
   }
   if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, s)) != SL_OK) return st;
   {
@@ -716,6 +739,7 @@ static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, fl
     g.K = d;
     g.bn = pl.o.bn;
     g.splits = pl.o.splits;
+    g.msub = pl.o.msub;
     g.epi = EPI_RESID;
     g.out = h;
     g.ldo = d;
@@ -734,6 +758,7 @@ static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, fl
     g.K = d;
     g.bn = pl.gu.bn;
     g.splits = pl.gu.splits;
+    g.msub = pl.gu.msub;
     const bool split = pl.gu.splits > 1;
     g.epi = split ? EPI_ACCUM : EPI_SWIGLU;
     g.out = split ? (void *)c->ws : c->act;
@@ -754,6 +779,7 @@ static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, fl
     g.K = f;
     g.bn = pl.dn.bn;
     g.splits = pl.dn.splits;
+    g.msub = pl.dn.msub;
     g.epi = EPI_RESID;
     g.out = h;
     g.ldo = d;
@@ -813,6 +839,7 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   g.K = d;
   g.bn = pl.hd.bn;
   g.splits = 1;
+  g.msub = pl.hd.msub;
   g.epi = EPI_STORE;
   g.out = d_logits;
   g.ldo = V;
@@ -887,10 +914,16 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: pointers must be 16-byte aligned");
   if (M == 0) return SL_OK;
   const int ns = sm_count();
+  int msub = 1;
+  if (bn < 0) {
+    msub = 2;
+    bn = -bn;
+  }
   if (bn == 0) {
     Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID ? SPLIT_RESID
                                 : epi == SL_GEMM_ACCUM ? SPLIT_ACCUM : SPLIT_NONE, ns, swiglu);
     bn = p.bn;
+    msub = p.msub;
     if (splits <= 0) splits = p.splits;
   }
   if (bn != 64 && bn != 128 && bn != 256) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bn must be 64/128/256");
@@ -919,6 +952,7 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   g.out = d_out;
   g.ldo = ldo;
   g.row_map = d_row_map;
+  g.msub = msub;
   int *err = device_error_word();
   if (!err) return fail(SL_ERR_CUDA, "sl_gemm_bf16: no device error word");
   cudaError_t e = launch_gemm_tc(g, ns, err, (cudaStream_t)stream);
@@ -1078,6 +1112,7 @@ namespace {
 __global__ void sampler_init_kernel(const int32_t *prompts, int batch, int prompt_len, int n_ctx,
                                     int mask_id, int32_t *tokens, uint8_t *masked,
                                     uint8_t *locked, int32_t *lock_t) {
+  pdl_wait();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= batch * n_ctx) return;
   int b = i / n_ctx, pos = i - b * n_ctx;
@@ -1094,11 +1129,9 @@ extern "C" sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, v
     return fail(SL_ERR_INVALID, "sl_sampler_start: null argument");
   cudaStream_t st = (cudaStream_t)stream;
   const int rows = s->batch * s->n_ctx;
-  sampler_init_kernel<<<(rows + 255) / 256, 256, 0, st>>>(
-      d_prompts, s->batch, s->p.prompt_len, s->n_ctx, s->m->cfg.mask_id, s->tokens, s->masked,
-      s->locked, s->lock_t);
-  SL_CUDA(cudaGetLastError());
-  note_launch();
+  SL_CUDA(launch_k(sampler_init_kernel, (rows + 255) / 256, 256, 0, st, d_prompts, s->batch,
+                   s->p.prompt_len, s->n_ctx, s->m->cfg.mask_id, s->tokens, s->masked, s->locked,
+                   s->lock_t));
   sl_status r = sl_kv_cache_reset(s->cache, stream);
   if (r != SL_OK) return r;
   r = sl_active_reset(s->act, stream);

@@ -8,7 +8,8 @@
 // and a range of 64-key tiles; K/V tiles stream through shared memory with
 // cp.async double buffering and an online softmax.  When the query tiles alone
 // cannot fill the GPU (few active rows), the key range is split across CTAs
-// and a second kernel merges the partial (max, sum, output) records.
+// and a second kernel merges the partial (max, sum, output) records, one warp
+// per (row, head) so the merge spreads over every SM.
 #include "common.cuh"
 #include "internal.h"
 
@@ -18,6 +19,7 @@ constexpr int AT_Q = 64;       // queries per CTA
 constexpr int AT_K = 64;       // keys per tile
 constexpr int AT_D = 128;      // head dim
 constexpr int AT_THREADS = 128;
+constexpr int ATTN_MAX_SPLITS = 16;    // split-KV partials merged in-kernel
 constexpr int AT_SMEM = (AT_Q + 4 * AT_K) * AT_D * 2;   // Q + 2x(K,V)
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -93,6 +95,7 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
 
   const bf16 *kbase = p.ck + (size_t)b * p.n_ctx * d + h * AT_D;
   const bf16 *vbase = p.cv + (size_t)b * p.n_ctx * d + h * AT_D;
+  pdl_wait();
 
   // Q tile
   for (int e = tid; e < AT_Q * 16; e += AT_THREADS) {
@@ -219,6 +222,7 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
     __syncthreads();
   }
   cp_wait<0>();
+  pdl_trigger();
 
   // epilogue: rows g and g+8 of this warp's 16
 #pragma unroll
@@ -249,38 +253,52 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
 // Merge split-KV partials: one warp per (row, head), 4 dims per lane.
 __global__ void attn_combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_ml,
                                     int M, int n_heads, int splits, bf16 *__restrict__ o) {
-  int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  int lane = threadIdx.x & 31;
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
   if (w >= M * n_heads) return;
-  int j = w / n_heads, h = w % n_heads;
+  pdl_wait();
+  const int j = w / n_heads, h = w % n_heads;
+  float m[ATTN_MAX_SPLITS], l[ATTN_MAX_SPLITS];
   float mx = -INFINITY;
-  for (int s = 0; s < splits; ++s) {
-    size_t rec = ((size_t)s * M + j) * n_heads + h;
-    mx = fmaxf(mx, ws_ml[rec * 2]);
+#pragma unroll
+  for (int sp = 0; sp < ATTN_MAX_SPLITS; ++sp) {
+    m[sp] = -INFINITY;
+    l[sp] = 0.f;
+    if (sp < splits) {
+      const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + (((size_t)sp * M + j) * n_heads + h) * 2);
+      m[sp] = ml.x;
+      l[sp] = ml.y;
+      mx = fmaxf(mx, ml.x);
+    }
   }
   float L = 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int s = 0; s < splits; ++s) {
-    size_t rec = ((size_t)s * M + j) * n_heads + h;
-    float m = ws_ml[rec * 2], l = ws_ml[rec * 2 + 1];
-    float c = (m == -INFINITY) ? 0.f : exp2f(m - mx);
-    L += l * c;
-    float4 v = *reinterpret_cast<const float4 *>(ws_o + rec * AT_D + lane * 4);
-    acc[0] += v.x * c; acc[1] += v.y * c; acc[2] += v.z * c; acc[3] += v.w * c;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int sp = 0; sp < ATTN_MAX_SPLITS; ++sp) {
+    if (sp < splits) {
+      const float c = (m[sp] == -INFINITY) ? 0.f : exp2f(m[sp] - mx);
+      L += l[sp] * c;
+      const float4 v = *reinterpret_cast<const float4 *>(
+          ws_o + (((size_t)sp * M + j) * n_heads + h) * AT_D + lane * 4);
+      acc.x += v.x * c; acc.y += v.y * c; acc.z += v.z * c; acc.w += v.w * c;
+    }
   }
-  float inv = L > 0.f ? 1.f / L : 0.f;
+  pdl_trigger();
+  const float inv = L > 0.f ? 1.f / L : 0.f;
   bf16 *dst = o + (size_t)j * n_heads * AT_D + h * AT_D + lane * 4;
   *reinterpret_cast<uint2 *>(dst) =
-      make_uint2(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv));
+      make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
 }
 
 size_t attn_bf16_workspace_bytes(int max_rows, int n_heads, int max_splits) {
   return (size_t)max_splits * max_rows * n_heads * (AT_D + 2) * sizeof(float);
 }
 
+
 cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
                              int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
                              int num_sms, cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   static bool attr_set = false;
   if (!attr_set) {
@@ -313,13 +331,11 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
   p.splits = splits;
   p.kblocks = kblocks;
   dim3 grid(tiles, n_heads, splits);
-  attn_bf16_kernel<<<grid, AT_THREADS, AT_SMEM, s>>>(p); note_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || splits == 1) return e;
-  int warps = M * n_heads;
-  attn_combine_kernel<<<(warps * 32 + 255) / 256, 256, 0, s>>>(p.ws_o, p.ws_ml, M, n_heads,
-                                                                splits, (bf16 *)o); note_launch();
-  return cudaGetLastError();
+  err = launch_k(attn_bf16_kernel, grid, AT_THREADS, AT_SMEM, s, p);
+  if (err != cudaSuccess || splits == 1) return err;
+  const int warps = M * n_heads;
+  return launch_k(attn_combine_kernel, (warps * 32 + 255) / 256, 256, 0, s, (const float *)p.ws_o,
+                  (const float *)p.ws_ml, M, n_heads, splits, (bf16 *)o);
 }
 
 }  // namespace sl

@@ -47,6 +47,16 @@ __device__ __forceinline__ unsigned long long global_ns() {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 
+// Programmatic dependent launch: every kernel of the step is launched with
+// programmatic stream serialisation, waits for its predecessor's results with
+// pdl_wait() before touching memory the predecessor writes (or reads), and
+// calls pdl_trigger() once its own main work is issued so the next kernel's
+// launch and prologue overlap this kernel's tail.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // 8 x bf16 <-> 16-byte vector
 union Pack8 {
   uint4 u;

@@ -170,8 +170,12 @@ struct TcParams {
   void *out;
   int ldo;
   int ffn;                 // SWIGLU/ACCUM-swiglu: F (columns of one half)
-  const int32_t *row_map;
+  const int32_t *row_map;  // STORE: output row per A row; QKV: flat position per row
   int *err;
+  // QKV epilogue: rotary table [n_ctx][64] (cos, sin), q out [M][d], cache k/v
+  const float2 *rope;
+  int n_ctx, dmodel;
+  bf16 *q_out, *ck, *cv;
 };
 
 constexpr int GROUP_M = 16;
@@ -188,18 +192,41 @@ __device__ __forceinline__ void decode_unit(const TcParams &p, int u, int &mt, i
   sp = nn - nt * p.splits;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MSUB>
 struct TcSmem {
-  static constexpr int A_BYTES = 128 * 64 * 2;
+  static constexpr int A_BYTES = MSUB * 128 * 64 * 2;   // MSUB 128-row A tiles per stage
   static constexpr int B_BYTES = BN * 64 * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;   // barriers + alignment slack
 };
 
-template <int BN, int STAGES, int EPI>
+// B tile of K-block kb for output tile nt: BN rows of one weight segment, or
+// BN/2 gate rows followed by the matching BN/2 up rows.
+template <int BN>
+__device__ __forceinline__ void load_b(const TcParams &p, uint32_t sb, int nt, int kb,
+                                       uint32_t bar) {
+  if (p.b_swiglu) {
+    const int f0 = nt * (BN / 2);
+    tma_load_2d(sb, &p.b[0], kb * 64, f0, bar);
+    tma_load_2d(sb + (BN / 2) * 128, &p.b[1], kb * 64, f0, bar);
+  } else {
+    const int c0 = nt * BN;
+    if (c0 < p.seg0) tma_load_2d(sb, &p.b[0], kb * 64, c0, bar);
+    else if (c0 < p.seg1) tma_load_2d(sb, &p.b[1], kb * 64, c0 - p.seg0, bar);
+    else tma_load_2d(sb, &p.b[2], kb * 64, c0 - p.seg1, bar);
+  }
+}
+
+// MSUB = 1: one 128-row tile of A per unit; MSUB = 2: two (256 rows) sharing
+// each B tile, accumulated in two TMEM accumulators (halves the weight-tile
+// re-reads when 128 < M <= 256).  Accumulators are double-buffered when
+// 2 * MSUB * BN TMEM columns fit in 512.
+template <int BN, int STAGES, int EPI, int MSUB>
 __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__ TcParams p) {
-  using L = TcSmem<BN, STAGES>;
+  using L = TcSmem<BN, STAGES, MSUB>;
+  constexpr int ACC_BUFS = (2 * MSUB * BN <= 512) ? 2 : 1;
+  constexpr int ACC_COLS = MSUB * BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s_addr(smem);
@@ -215,7 +242,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t TMEM_COLS = ACC_BUFS * ACC_COLS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -247,40 +274,55 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
+      // Weight tiles do not depend on the previous kernel: issue the B loads of
+      // the first stages of this CTA's first unit before waiting on it, so the
+      // weight stream starts while the previous kernel drains.
+      int npre = 0;
+      if ((int)blockIdx.x < p.units) {
+        int mt, nt, sp;
+        decode_unit(p, blockIdx.x, mt, nt, sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        npre = min(STAGES, kb1 - kb0);
+        for (int i = 0; i < npre; ++i) {
+          const uint32_t sb = sbase + i * L::STAGE_BYTES + L::A_BYTES;
+          mbar_expect_tx(full_bar(i), L::STAGE_BYTES);
+          load_b<BN>(p, sb, nt, kb0 + i, full_bar(i));
+        }
+      }
+      pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
       int last_stage = -1;
       uint32_t last_phase = 0;
       bool ok = true;
+      bool first = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         int mt, nt, sp;
         decode_unit(p, u, mt, nt, sp);
         const int kb0 = sp * p.kb_per_split;
         const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
-            ok = false;
-            break;
+          const bool pre = first && (kb - kb0) < npre;
+          if (!pre) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(full_bar(stage), L::STAGE_BYTES);
           }
           const uint32_t sa = sbase + stage * L::STAGE_BYTES;
-          const uint32_t sb = sa + L::A_BYTES;
-          mbar_expect_tx(full_bar(stage), L::STAGE_BYTES);
-          tma_load_2d(sa, &p.a, kb * 64, mt * 128, full_bar(stage));
-          if (p.b_swiglu) {
-            const int f0 = nt * (BN / 2);
-            tma_load_2d(sb, &p.b[0], kb * 64, f0, full_bar(stage));
-            tma_load_2d(sb + (BN / 2) * 128, &p.b[1], kb * 64, f0, full_bar(stage));
-          } else {
-            const int c0 = nt * BN;
-            if (c0 < p.seg0) tma_load_2d(sb, &p.b[0], kb * 64, c0, full_bar(stage));
-            else if (c0 < p.seg1) tma_load_2d(sb, &p.b[1], kb * 64, c0 - p.seg0, full_bar(stage));
-            else tma_load_2d(sb, &p.b[2], kb * 64, c0 - p.seg1, full_bar(stage));
-          }
+#pragma unroll
+          for (int sub = 0; sub < MSUB; ++sub)
+            tma_load_2d(sa + sub * 16384, &p.a, kb * 64, (mt * MSUB + sub) * 128, full_bar(stage));
+          if (!pre) load_b<BN>(p, sa + L::A_BYTES, nt, kb, full_bar(stage));
           last_stage = stage;
           last_phase = phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        first = false;
       }
+      pdl_trigger();
       if (!ok) {
         atomicExch(p.err, DEV_TIMEOUT_PRODUCER);
         *abort_flag = 1;
@@ -307,23 +349,27 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = sbase + stage * L::STAGE_BYTES;
           const uint32_t sb = sa + L::A_BYTES;
-          const uint64_t adesc = smem_desc_sw128(sa);
           const uint64_t bdesc = smem_desc_sw128(sb);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            tc_mma(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          for (int sub = 0; sub < MSUB; ++sub) {
+            const uint64_t adesc = smem_desc_sw128(sa + sub * 16384);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              tc_mma(d_tmem + sub * BN, adesc + 2 * k, bdesc + 2 * k, idesc,
+                     (kb > kb0 || k > 0) ? 1u : 0u);
+          }
           tc_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc_commit(tfull_bar(acc));
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
       }
       if (!ok) {
         atomicExch(p.err, DEV_TIMEOUT_MMA);
@@ -336,6 +382,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     }
   } else {
     // ---------------------------------------------------------- epilogue
+    pdl_wait();                             // outputs may be in use by the previous kernel
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -345,11 +392,34 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       decode_unit(p, u, mt, nt, sp);
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      const int r = mt * 128 + q * 32 + lane;
+#pragma unroll 1
+      for (int sub = 0; sub < MSUB; ++sub) {
+      const int r = (mt * MSUB + sub) * 128 + q * 32 + lane;
       const bool live = r < p.M;
-      const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * ACC_COLS + sub * BN) +
+                             ((uint32_t)(q * 32) << 16);
       float v[32];
-      if (EPI == EPI_SWIGLU) {
+      if (EPI == EPI_ACCUM) {
+        // split-K partial sum of this tile: fp32 atomics into the workspace
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          tmem_ld32(taddr + c, v);
+          if (!live) continue;
+          int col;
+          if (p.b_swiglu) {   // gate into [0, F), up into [F, 2F)
+            const int half = BN / 2;
+            const int f0 = nt * half;
+            col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
+          } else {
+            col = nt * BN + c;
+          }
+          float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + col;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            atomicAdd(reinterpret_cast<float4 *>(dst + i),
+                      make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        }
+      } else if (EPI == EPI_SWIGLU) {
         const int f0 = nt * (BN / 2);
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
@@ -364,6 +434,51 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 #pragma unroll
               for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(silu_f(g[i + e]) * v[i + e]);
               *reinterpret_cast<uint4 *>(dst + i) = pk.u;
+            }
+          }
+        }
+      } else if (EPI == EPI_QKV) {
+        // whole heads per tile: pair (i, i + 64) of a head is rotated together
+        const int col0 = nt * BN;
+        const int seg = col0 / p.dmodel;              // 0 q, 1 k, 2 v
+        const int pos_flat = live ? p.row_map[r] : 0;
+        const int pos = pos_flat % p.n_ctx;
+#pragma unroll 1
+        for (int hd = 0; hd < BN / 128; ++hd) {
+          const int cbase = col0 - seg * p.dmodel + hd * 128;   // column of the head in its segment
+#pragma unroll 1
+          for (int j = 0; j < 2; ++j) {
+            float x2[32];
+            tmem_ld32(taddr + hd * 128 + 32 * j, v);
+            tmem_ld32(taddr + hd * 128 + 64 + 32 * j, x2);
+            if (!live) continue;
+            bf16 *dst;
+            if (seg == 0) dst = p.q_out + (size_t)r * p.dmodel + cbase;
+            else if (seg == 1) dst = p.ck + (size_t)pos_flat * p.dmodel + cbase;
+            else dst = p.cv + (size_t)pos_flat * p.dmodel + cbase;
+            if (seg < 2) {
+              const float4 *tab =
+                  reinterpret_cast<const float4 *>(p.rope + (size_t)pos * 64 + 32 * j);
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float4 cs = __ldg(tab + (e >> 1));   // (cos, sin) of e and e+1
+                const float a0 = v[e], b0 = x2[e], a1 = v[e + 1], b1 = x2[e + 1];
+                v[e] = a0 * cs.x - b0 * cs.y;
+                x2[e] = b0 * cs.x + a0 * cs.y;
+                v[e + 1] = a1 * cs.z - b1 * cs.w;
+                x2[e + 1] = b1 * cs.z + a1 * cs.w;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+              Pack8 lo, hi;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                lo.h[e] = __float2bfloat16_rn(v[i + e]);
+                hi.h[e] = __float2bfloat16_rn(x2[i + e]);
+              }
+              *reinterpret_cast<uint4 *>(dst + 32 * j + i) = lo.u;
+              *reinterpret_cast<uint4 *>(dst + 64 + 32 * j + i) = hi.u;
             }
           }
         }
@@ -382,17 +497,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
               for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(v[i + e]);
               *reinterpret_cast<uint4 *>(dst + i) = pk.u;
             }
-          } else {
-            int col;
-            if (p.b_swiglu) {   // accumulate gate into [0, F), up into [F, 2F)
-              const int half = BN / 2;
-              const int f0 = nt * half;
-              col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
-            } else {
-              col = nt * BN + c;
-            }
-            float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + col;
-            if (EPI == EPI_RESID && p.splits == 1) {
+          } else {   // EPI_RESID: h += partial (atomic when K is split)
+            float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + nt * BN + c;
+            if (p.splits == 1) {
 #pragma unroll
               for (int i = 0; i < 32; i += 4) {
                 float4 o = *reinterpret_cast<float4 *>(dst + i);
@@ -408,10 +515,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           }
         }
       }
+      }   // sub
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty_bar(acc));
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
+
     }
     if (!ok && lane == 0) {
       atomicExch(p.err, DEV_TIMEOUT_EPI);
@@ -431,27 +540,29 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 }
 
 // ------------------------------------------------------------------ host ---
-template <int BN, int STAGES, int EPI>
+template <int BN, int STAGES, int EPI, int MSUB>
 static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
-  using L = TcSmem<BN, STAGES>;
+  cudaError_t err = cudaSuccess;
+  using L = TcSmem<BN, STAGES, MSUB>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, EPI>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, EPI, MSUB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  gemm_tc_kernel<BN, STAGES, EPI><<<grid, 192, L::TOTAL, s>>>(p); note_launch();
-  return cudaGetLastError();
+  err = launch_k(gemm_tc_kernel<BN, STAGES, EPI, MSUB>, grid, 192, L::TOTAL, s, p);
+  return err;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int MSUB>
 static cudaError_t run_epi(int epi, const TcParams &p, int grid, cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE: return run_tc<BN, STAGES, EPI_STORE>(p, grid, s);
-    case EPI_RESID: return run_tc<BN, STAGES, EPI_RESID>(p, grid, s);
-    case EPI_SWIGLU: return run_tc<BN, STAGES, EPI_SWIGLU>(p, grid, s);
-    case EPI_ACCUM: return run_tc<BN, STAGES, EPI_ACCUM>(p, grid, s);
+    case EPI_STORE: return run_tc<BN, STAGES, EPI_STORE, MSUB>(p, grid, s);
+    case EPI_RESID: return run_tc<BN, STAGES, EPI_RESID, MSUB>(p, grid, s);
+    case EPI_SWIGLU: return run_tc<BN, STAGES, EPI_SWIGLU, MSUB>(p, grid, s);
+    case EPI_ACCUM: return run_tc<BN, STAGES, EPI_ACCUM, MSUB>(p, grid, s);
+    case EPI_QKV: return run_tc<BN, STAGES, EPI_QKV, MSUB>(p, grid, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -476,11 +587,15 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
-  p.m_tiles = (a.M + 127) / 128;
+  const int msub = a.msub == 2 ? 2 : 1;
+  p.m_tiles = (a.M + 128 * msub - 1) / (128 * msub);
   p.n_tiles = a.N / bn;
   p.kblocks = a.K / 64;
   int splits = a.splits < 1 ? 1 : a.splits;
-  if (a.epi != EPI_RESID && a.epi != EPI_ACCUM) splits = 1;
+  if (a.epi == EPI_STORE || a.epi == EPI_QKV || a.epi == EPI_SWIGLU) splits = 1;
+  if (a.epi == EPI_QKV && (bn < 128 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||
+                           (a.N % 3) != 0 || ((a.N / 3) % 128) != 0))
+    return cudaErrorInvalidValue;
   if (splits > p.kblocks) splits = p.kblocks;
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;   // no empty split
@@ -490,11 +605,24 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.ffn = a.N / 2;
   p.row_map = a.row_map;
   p.err = err;
+  p.rope = a.rope;
+  p.n_ctx = a.n_ctx;
+  p.dmodel = a.epi == EPI_QKV ? a.N / 3 : 0;
+  p.q_out = (bf16 *)a.q_out;
+  p.ck = (bf16 *)a.ck;
+  p.cv = (bf16 *)a.cv;
   int grid = p.units < num_sms ? p.units : num_sms;
+  if (msub == 2) {
+    switch (bn) {
+      case 256: return run_epi<256, 3, 2>(a.epi, p, grid, s);
+      case 128: return run_epi<128, 4, 2>(a.epi, p, grid, s);
+      default: return run_epi<64, 5, 2>(a.epi, p, grid, s);
+    }
+  }
   switch (bn) {
-    case 256: return run_epi<256, 4>(a.epi, p, grid, s);
-    case 128: return run_epi<128, 6>(a.epi, p, grid, s);
-    default: return run_epi<64, 8>(a.epi, p, grid, s);
+    case 256: return run_epi<256, 4, 1>(a.epi, p, grid, s);
+    case 128: return run_epi<128, 6, 1>(a.epi, p, grid, s);
+    default: return run_epi<64, 8, 1>(a.epi, p, grid, s);
   }
 }
 

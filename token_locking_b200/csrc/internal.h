@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
 #include <vector>
 
 #include "surelock.h"
@@ -23,12 +24,31 @@ long long launches_total();
     if (_e != cudaSuccess) return ::sl::cuda_fail(_e, #call); \
   } while (0)
 
+// Launch with programmatic stream serialisation (see pdl_wait/pdl_trigger).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ----------------------------------------------------- epilogue selection --
 enum GemmEpi : int {
   EPI_STORE = 0,      // out[row_map ? row_map[r] : r][col_off + c] = acc   (dtype)
   EPI_RESID = 1,      // resid[r][c] += acc   (fp32; atomic when split over K)
   EPI_SWIGLU = 2,     // out[r][c] = silu(gate) * up      (dtype; tile = gate|up halves)
-  EPI_ACCUM = 3       // ws[r][col] += acc  (fp32 atomics, split-K workspace)
+  EPI_ACCUM = 3,      // ws[r][col] += acc  (fp32 atomics, split-K workspace)
+  EPI_QKV = 4         // fused Q|K|V: RoPE(q) -> q_out[r], RoPE(k), v -> cache rows row_map[r]
 };
 
 // ------------------------------------------------------------------ layers.cu
@@ -86,9 +106,14 @@ struct TcGemmArgs {
   int splits;            // K splits (EPI_RESID / EPI_ACCUM only)
   int bn;                // 64, 128 or 256
   int b_swiglu;          // B tile = BN/2 gate rows (B[0]) | BN/2 up rows (B[1])
+  int msub;              // 1: 128-row units; 2: 256-row units (two accumulators per B tile)
   void *out;             // STORE/SWIGLU: dtype out; RESID: fp32 resid; ACCUM: fp32 ws
   int ldo;               // leading dimension of out (elements)
-  const int32_t *row_map;// STORE: output row index per A row (or null)
+  const int32_t *row_map;// STORE: output row index per A row (or null); QKV: flat positions
+  // QKV: rotary table [n_ctx][64], q out [M][d], this layer's cache k/v [B*n_ctx][d]
+  const float2 *rope;
+  int n_ctx;
+  void *q_out, *ck, *cv;
 };
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s);
 

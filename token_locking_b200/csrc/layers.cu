@@ -18,20 +18,23 @@ __global__ void gather_embed_kernel(const int32_t *__restrict__ tokens,
                                     const T *__restrict__ emb, int d, float *__restrict__ h) {
   int j = blockIdx.x;
   if (j >= M) return;
+  pdl_wait();
   const T *e = emb + (size_t)tokens[rows[j]] * d;
   float *o = h + (size_t)j * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = to_f(e[c]);
+  pdl_trigger();
 }
 
 cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
                                 const void *emb, int d, float *h, cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   if (dtype == SL_BF16) {
-    gather_embed_kernel<bf16><<<M, 256, 0, s>>>(tokens, rows, M, (const bf16 *)emb, d, h); note_launch();
+    err = launch_k(gather_embed_kernel<bf16>, M, 256, 0, s, tokens, rows, M, (const bf16 *)emb, d, h);
   } else {
-    gather_embed_kernel<float><<<M, 256, 0, s>>>(tokens, rows, M, (const float *)emb, d, h); note_launch();
+    err = launch_k(gather_embed_kernel<float>, M, 256, 0, s, tokens, rows, M, (const float *)emb, d, h);
   }
-  return cudaGetLastError();
+  return err;
 }
 
 // --------------------------------------------------------------- rmsnorm ---
@@ -41,6 +44,7 @@ __global__ void rmsnorm_kernel(const float *__restrict__ h, const T *__restrict_
                                float eps, int M, T *__restrict__ out) {
   int j = blockIdx.x;
   if (j >= M) return;
+  pdl_wait();
   const float *x = h + (size_t)j * d;
   float ss = 0.f;
   for (int c = threadIdx.x; c < d; c += blockDim.x) ss += x[c] * x[c];
@@ -57,62 +61,123 @@ __global__ void rmsnorm_kernel(const float *__restrict__ h, const T *__restrict_
   float r = rsqrtf(red[0] / (float)d + eps);
   T *o = out + (size_t)j * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = from_f<T>(x[c] * r * to_f(g[c]));
+  pdl_trigger();
+}
+
+// bf16 output: one CTA of 256 threads per row, the row held in registers as
+// VPT float4 per thread, so the row is read once and the sum of squares needs a
+// single block reduction.
+template <int VPT>
+__global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float *__restrict__ h,
+                                                           const bf16 *__restrict__ g, int d,
+                                                           float eps, int M,
+                                                           bf16 *__restrict__ out) {
+  const int j = blockIdx.x;
+  if (j >= M) return;
+  pdl_wait();
+  const float4 *x = reinterpret_cast<const float4 *>(h + (size_t)j * d);
+  const int n4 = d >> 2;
+  float4 v[VPT];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * 256;
+    v[k] = i < n4 ? x[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[k].x * v[k].x + v[k].y * v[k].y + v[k].z * v[k].z + v[k].w * v[k].w;
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) tot += red[w];
+  const float r = rsqrtf(tot / (float)d + eps);
+  const uint2 *g2 = reinterpret_cast<const uint2 *>(g);
+  uint2 *o2 = reinterpret_cast<uint2 *>(out + (size_t)j * d);
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < n4) {
+      union { uint2 u; __nv_bfloat162 b[2]; } gg, oo;
+      gg.u = g2[i];
+      const float2 g0 = __bfloat1622float2(gg.b[0]), g1 = __bfloat1622float2(gg.b[1]);
+      oo.b[0] = __floats2bfloat162_rn(v[k].x * r * g0.x, v[k].y * r * g0.y);
+      oo.b[1] = __floats2bfloat162_rn(v[k].z * r * g1.x, v[k].w * r * g1.y);
+      o2[i] = oo.u;
+    }
+  }
+  pdl_trigger();
 }
 
 cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
                            void *out, cudaStream_t s) {
+  if (dtype == SL_BF16 && d % 4 == 0 && d <= 8 * 1024) {
+    if (M <= 0) return cudaSuccess;
+    const int vpt = (d / 4 + 255) / 256;
+    const bf16 *gb = (const bf16 *)g;
+    bf16 *ob = (bf16 *)out;
+    if (vpt <= 1) return launch_k(rmsnorm_bf16_kernel<1>, M, 256, 0, s, h, gb, d, eps, M, ob);
+    if (vpt <= 2) return launch_k(rmsnorm_bf16_kernel<2>, M, 256, 0, s, h, gb, d, eps, M, ob);
+    if (vpt <= 4) return launch_k(rmsnorm_bf16_kernel<4>, M, 256, 0, s, h, gb, d, eps, M, ob);
+    return launch_k(rmsnorm_bf16_kernel<8>, M, 256, 0, s, h, gb, d, eps, M, ob);
+  }
+  cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   int th = d >= 1024 ? 512 : 128;
   if (dtype == SL_BF16) {
-    rmsnorm_kernel<bf16><<<M, th, 0, s>>>(h, (const bf16 *)g, d, eps, M, (bf16 *)out); note_launch();
+    err = launch_k(rmsnorm_kernel<bf16>, M, th, 0, s, h, (const bf16 *)g, d, eps, M, (bf16 *)out);
   } else {
-    rmsnorm_kernel<float><<<M, th, 0, s>>>(h, (const float *)g, d, eps, M, (float *)out); note_launch();
+    err = launch_k(rmsnorm_kernel<float>, M, th, 0, s, h, (const float *)g, d, eps, M, (float *)out);
   }
-  return cudaGetLastError();
+  return err;
 }
 
 // ------------------------------------------------------- rotary + scatter ---
-// From the fused projection output [M][3d] (q | k | v): q_out[j] = RoPE(q_j),
+// From the projection output [M][3d] (q | k | v): q_out[j] = RoPE(q_j),
 // C.k[rows[j]] = RoPE(k_j), C.v[rows[j]] = v_j.  RoPE is rotate-half on the
 // pair (i, i + dh/2) at the absolute position rows[j] % n_ctx; the (cos, sin)
 // table is precomputed in double precision on the host.  Writing the fresh k,v
 // of active rows into the cache is the "K^all[A_t]" half of the pages'
-// K^all[L_t] <- C.k[L_t] (Paper-Notes, "permanent locking").
+// K^all[L_t] <- C.k[L_t] (Paper-Notes, "permanent locking").  One thread per
+// (row, pair) so that a few rows still spread over every SM; used after a
+// split-K projection (input = the fp32 partial-sum workspace, cleared here for
+// the next split-K GEMM) and on the fp32 path.
 template <typename Tin, typename T>
-__global__ void rope_scatter_kernel(Tin *__restrict__ qkv, bool zero_in, int M,
-                                    const int32_t *__restrict__ rows, int n_ctx, int n_heads,
-                                    int dh, const float2 *__restrict__ rope, T *__restrict__ q_out,
-                                    T *__restrict__ ck, T *__restrict__ cv) {
-  int j = blockIdx.x;
-  if (j >= M) return;
-  int d = n_heads * dh;
-  int half = dh >> 1;
-  int p = rows[j];
-  int pos = p % n_ctx;
-  Tin *in = qkv + (size_t)j * 3 * d;
-  const float2 *tab = rope + (size_t)pos * half;
-  T *qo = q_out + (size_t)j * d;
-  T *ko = ck + (size_t)p * d;
-  T *vo = cv + (size_t)p * d;
-  int npairs = n_heads * half;
-  for (int t = threadIdx.x; t < npairs; t += blockDim.x) {
-    int hh = t / half, i = t - hh * half;
-    int c0 = hh * dh + i, c1 = c0 + half;
-    float2 cs = tab[i];
-    float q0 = to_f(in[c0]), q1 = to_f(in[c1]);
-    float k0 = to_f(in[d + c0]), k1 = to_f(in[d + c1]);
-    qo[c0] = from_f<T>(q0 * cs.x - q1 * cs.y);
-    qo[c1] = from_f<T>(q1 * cs.x + q0 * cs.y);
-    ko[c0] = from_f<T>(k0 * cs.x - k1 * cs.y);
-    ko[c1] = from_f<T>(k1 * cs.x + k0 * cs.y);
-    vo[c0] = from_f<T>(to_f(in[2 * d + c0]));
-    vo[c1] = from_f<T>(to_f(in[2 * d + c1]));
+__global__ void __launch_bounds__(256) rope_scatter_kernel(
+    Tin *__restrict__ qkv, bool zero_in, int M, const int32_t *__restrict__ rows, int n_ctx,
+    int n_heads, int dh, const float2 *__restrict__ rope, T *__restrict__ q_out,
+    T *__restrict__ ck, T *__restrict__ cv) {
+  // grid: x = chunks of 256 pairs within a row (3 * d / 2 pairs), y = row
+  const int j = blockIdx.y;
+  const int d = n_heads * dh;
+  const int half = dh >> 1;
+  const int per_seg = d >> 1;
+  const int pr_all = blockIdx.x * 256 + threadIdx.x;
+  pdl_wait();
+  if (pr_all < 3 * per_seg) {
+    const int seg = pr_all / per_seg;
+    const int pr = pr_all - seg * per_seg;
+    const int hh = pr / half, i = pr - hh * half;
+    const int c0 = hh * dh + i, c1 = c0 + half;
+    Tin *in = qkv + (size_t)j * 3 * d + seg * d;
+    const float x0 = to_f(in[c0]), x1 = to_f(in[c1]);
     if (zero_in) {
-      in[c0] = Tin(0.f); in[c1] = Tin(0.f);
-      in[d + c0] = Tin(0.f); in[d + c1] = Tin(0.f);
-      in[2 * d + c0] = Tin(0.f); in[2 * d + c1] = Tin(0.f);
+      in[c0] = Tin(0.f);
+      in[c1] = Tin(0.f);
+    }
+    const int p = rows[j];
+    T *dst = seg == 0 ? q_out + (size_t)j * d : (seg == 1 ? ck : cv) + (size_t)p * d;
+    if (seg < 2) {
+      const float2 cs = rope[(size_t)(p % n_ctx) * half + i];
+      dst[c0] = from_f<T>(x0 * cs.x - x1 * cs.y);
+      dst[c1] = from_f<T>(x1 * cs.x + x0 * cs.y);
+    } else {
+      dst[c0] = from_f<T>(x0);
+      dst[c1] = from_f<T>(x1);
     }
   }
+  pdl_trigger();
 }
 
 cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool zero_in, int M,
@@ -120,50 +185,60 @@ cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool
                                 const float2 *rope, void *q_out, void *ck, void *cv,
                                 cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
-  int th = 256;
+  if (M > 65535) return cudaErrorInvalidValue;
+  const dim3 grid((3 * n_heads * head_dim / 2 + 255) / 256, M);
   if (dtype == SL_BF16) {
-    if (in_f32) {
-      rope_scatter_kernel<float, bf16><<<M, th, 0, s>>>((float *)qkv_in, zero_in, M, rows, n_ctx,
-          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv); note_launch();
-    } else {
-      rope_scatter_kernel<bf16, bf16><<<M, th, 0, s>>>((bf16 *)qkv_in, false, M, rows, n_ctx,
-          n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv); note_launch();
-    }
-  } else {
-    rope_scatter_kernel<float, float><<<M, th, 0, s>>>((float *)qkv_in, zero_in, M, rows, n_ctx,
-        n_heads, head_dim, rope, (float *)q_out, (float *)ck, (float *)cv); note_launch();
+    if (in_f32)
+      return launch_k(rope_scatter_kernel<float, bf16>, grid, 256, 0, s, (float *)qkv_in, zero_in,
+                      M, rows, n_ctx, n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck,
+                      (bf16 *)cv);
+    return launch_k(rope_scatter_kernel<bf16, bf16>, grid, 256, 0, s, (bf16 *)qkv_in, false, M,
+                    rows, n_ctx, n_heads, head_dim, rope, (bf16 *)q_out, (bf16 *)ck, (bf16 *)cv);
   }
-  return cudaGetLastError();
+  return launch_k(rope_scatter_kernel<float, float>, grid, 256, 0, s, (float *)qkv_in, zero_in, M,
+                  rows, n_ctx, n_heads, head_dim, rope, (float *)q_out, (float *)ck, (float *)cv);
 }
 
 // ----------------------------------------------------------------- swiglu ---
+// act[j][c] = silu(g[j][c]) * u[j][c] from a [M][2F] buffer (gate | up); grid
+// x = chunks of 1024 columns (4 per thread), y = row; the fp32 workspace is
+// cleared for the next split-K GEMM.
 template <typename Tin, typename T>
-__global__ void swiglu_kernel(Tin *__restrict__ ws, bool zero_in, int M, int F,
-                              T *__restrict__ act) {
-  int j = blockIdx.x;
-  if (j >= M) return;
+__global__ void __launch_bounds__(256) swiglu_kernel(Tin *__restrict__ ws, bool zero_in, int M,
+                                                     int F, T *__restrict__ act) {
+  const int j = blockIdx.y;
+  pdl_wait();
   Tin *g = ws + (size_t)j * 2 * F;
   T *o = act + (size_t)j * F;
-  for (int c = threadIdx.x; c < F; c += blockDim.x) {
-    float gv = to_f(g[c]), uv = to_f(g[F + c]);
-    o[c] = from_f<T>(silu_f(gv) * uv);
-    if (zero_in) { g[c] = Tin(0.f); g[F + c] = Tin(0.f); }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = blockIdx.x * 1024 + k * 256 + threadIdx.x;
+    if (c < F) {
+      const float gv = to_f(g[c]), uv = to_f(g[F + c]);
+      if (zero_in) {
+        g[c] = Tin(0.f);
+        g[F + c] = Tin(0.f);
+      }
+      o[c] = from_f<T>(silu_f(gv) * uv);
+    }
   }
+  pdl_trigger();
 }
 
 cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, int M, int F,
                           void *act, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
+  if (M > 65535) return cudaErrorInvalidValue;
+  const dim3 grid((F + 1023) / 1024, M);
   if (dtype == SL_BF16) {
-    if (in_f32) {
-      swiglu_kernel<float, bf16><<<M, 512, 0, s>>>((float *)ws, zero_in, M, F, (bf16 *)act); note_launch();
-    } else {
-      swiglu_kernel<bf16, bf16><<<M, 512, 0, s>>>((bf16 *)ws, false, M, F, (bf16 *)act); note_launch();
-    }
-  } else {
-    swiglu_kernel<float, float><<<M, 256, 0, s>>>((float *)ws, zero_in, M, F, (float *)act); note_launch();
+    if (in_f32)
+      return launch_k(swiglu_kernel<float, bf16>, grid, 256, 0, s, (float *)ws, zero_in, M, F,
+                      (bf16 *)act);
+    return launch_k(swiglu_kernel<bf16, bf16>, grid, 256, 0, s, (bf16 *)ws, false, M, F,
+                    (bf16 *)act);
   }
-  return cudaGetLastError();
+  return launch_k(swiglu_kernel<float, float>, grid, 256, 0, s, (float *)ws, zero_in, M, F,
+                  (float *)act);
 }
 
 // -------------------------------------------------------- fp32 SIMT GEMM ---
@@ -177,6 +252,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(int epi, const float *__r
                                                        const int32_t *__restrict__ row_map) {
   __shared__ float As[FK][FT + 1];
   __shared__ float Bs[FK][FT + 1];
+  pdl_wait();
   int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   int m0 = blockIdx.y * FT, n0 = blockIdx.x * FT;
   float acc[4][4] = {};
@@ -216,15 +292,17 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(int epi, const float *__r
       else *dst = acc[i][jj];
     }
   }
+  pdl_trigger();
 }
 
 cudaError_t launch_gemm_f32(int epi, const float *A, int M, int K, const float *B, int N,
                             float *C, int ldc, int col_off, const int32_t *row_map,
                             cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   dim3 grid((N + FT - 1) / FT, (M + FT - 1) / FT);
-  gemm_f32_kernel<<<grid, 256, 0, s>>>(epi, A, M, K, B, N, C, ldc, col_off, row_map); note_launch();
-  return cudaGetLastError();
+  err = launch_k(gemm_f32_kernel, grid, 256, 0, s, epi, A, M, K, B, N, C, ldc, col_off, row_map);
+  return err;
 }
 
 // --------------------------------------------------------- fp32 attention ---
@@ -238,6 +316,7 @@ __global__ void attn_f32_kernel(const float *__restrict__ q, const float *__rest
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   if (warp >= M * n_heads) return;
+  pdl_wait();
   int j = warp / n_heads, hh = warp % n_heads;
   int d = n_heads * DH;
   int b = rows[j] / n_ctx;
@@ -279,22 +358,24 @@ __global__ void attn_f32_kernel(const float *__restrict__ q, const float *__rest
     float v = warp_sum(acc[i]);
     if (lane == 0) ov[i] = v / l;
   }
+  pdl_trigger();
 }
 
 cudaError_t launch_attn_f32(const float *q, const float *ck, const float *cv,
                             const int32_t *rows, int M, int n_ctx, int n_heads, int head_dim,
                             float *o, cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   int warps = M * n_heads;
   int blocks = (warps * 32 + 255) / 256;
   switch (head_dim) {
-    case 8: attn_f32_kernel<8><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
-    case 16: attn_f32_kernel<16><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
-    case 32: attn_f32_kernel<32><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
-    case 64: attn_f32_kernel<64><<<blocks, 256, 0, s>>>(q, ck, cv, rows, M, n_ctx, n_heads, o); note_launch(); break;
+    case 8: err = launch_k(attn_f32_kernel<8>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 16: err = launch_k(attn_f32_kernel<16>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 32: err = launch_k(attn_f32_kernel<32>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 64: err = launch_k(attn_f32_kernel<64>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace sl

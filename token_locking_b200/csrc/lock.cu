@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(LOCK_THREADS) lock_stats_kernel(LockStatsArgs 
   const int j = blockIdx.x / a.splits;
   const int sidx = blockIdx.x - j * a.splits;
   if (j >= a.M) return;
+  pdl_wait();
   const int V = a.V;
   const int p = a.rows[j];
   const T *cur = reinterpret_cast<const T *>(a.cur) + (size_t)p * V;
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(LOCK_THREADS) lock_stats_kernel(LockStatsArgs 
     }
   }
 
+  pdl_trigger();
   // block reduction
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -212,12 +214,13 @@ int lock_stats_splits(int M, int V, int num_sms) {
 }
 
 cudaError_t launch_lock_stats(const LockStatsArgs &a, cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   if (a.M <= 0) return cudaSuccess;
   const long blocks = (long)a.splits * a.M;
   if (blocks > 0x7fffffffL) return cudaErrorInvalidValue;
   dim3 grid((unsigned)blocks);
-  if (a.dtype == SL_BF16) { lock_stats_kernel<bf16><<<grid, LOCK_THREADS, 0, s>>>(a); note_launch(); } else { lock_stats_kernel<float><<<grid, LOCK_THREADS, 0, s>>>(a); note_launch(); }
-  return cudaGetLastError();
+  if (a.dtype == SL_BF16) { err = launch_k(lock_stats_kernel<bf16>, grid, LOCK_THREADS, 0, s, a); } else { err = launch_k(lock_stats_kernel<float>, grid, LOCK_THREADS, 0, s, a); }
+  return err;
 }
 
 // ---------------------------------------------------------- radix select ---
@@ -285,6 +288,8 @@ __global__ void __launch_bounds__(DEC_THREADS) lock_decide_kernel(
   __shared__ unsigned int sh_p32;
   __shared__ int sh_rank;
   __shared__ int sh_cnt;
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const int s0 = seq_off[b], s1 = seq_off[b + 1];
   const int Mb = s1 - s0;
@@ -346,9 +351,10 @@ cudaError_t launch_lock_decide(const int32_t *seq_off, int batch, const int32_t 
                                const float *kl, const float *unc, const uint8_t *masked,
                                float eps, float gate_q, int has_prev, int scripted_target,
                                uint8_t *lock, cudaStream_t s) {
-  lock_decide_kernel<<<batch, DEC_THREADS, 0, s>>>(seq_off, rows, kl, unc, masked, eps, gate_q,
-                                                    has_prev, scripted_target, lock); note_launch();
-  return cudaGetLastError();
+  cudaError_t err = cudaSuccess;
+  err = launch_k(lock_decide_kernel, batch, DEC_THREADS, 0, s, seq_off, rows, kl, unc, masked, eps, gate_q,
+                                                    has_prev, scripted_target, lock);
+  return err;
 }
 
 // ------------------------------------------------------------- compaction ---
@@ -361,6 +367,8 @@ __global__ void __launch_bounds__(DEC_THREADS) compact_kernel(
   __shared__ int old_off[SL_MAX_BATCH + 1];
   __shared__ int wsum[DEC_THREADS / 32];
   __shared__ int total;
+  pdl_wait();
+  pdl_trigger();
   for (int i = threadIdx.x; i <= batch; i += blockDim.x) old_off[i] = seq_off[i];
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -408,8 +416,9 @@ __global__ void __launch_bounds__(DEC_THREADS) compact_kernel(
 
 cudaError_t launch_compact(int32_t *rows, int32_t *seq_off, int batch, const uint8_t *lock,
                            uint8_t *locked, int32_t *lock_t, int step, cudaStream_t s) {
-  compact_kernel<<<1, DEC_THREADS, 0, s>>>(rows, seq_off, batch, lock, locked, lock_t, step); note_launch();
-  return cudaGetLastError();
+  cudaError_t err = cudaSuccess;
+  err = launch_k(compact_kernel, 1, DEC_THREADS, 0, s, rows, seq_off, batch, lock, locked, lock_t, step);
+  return err;
 }
 
 // --------------------------------------------------------------- unmask ----
@@ -421,6 +430,8 @@ __global__ void __launch_bounds__(256) unmask_kernel(
     int32_t *__restrict__ tokens, uint8_t *__restrict__ masked) {
   __shared__ int cj[UNMASK_MAX_CAND];
   __shared__ int ncand;
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const int s0 = seq_off[b], s1 = seq_off[b + 1];
   if (threadIdx.x == 0) ncand = 0;
@@ -455,14 +466,17 @@ __global__ void __launch_bounds__(256) unmask_kernel(
 cudaError_t launch_unmask(const int32_t *seq_off, int batch, const int32_t *rows, int n_ctx,
                           const float *conf, const int32_t *argmax, int lo, int hi, int k,
                           int32_t *tokens, uint8_t *masked, cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   if (hi - lo > UNMASK_MAX_CAND) return cudaErrorInvalidValue;
-  unmask_kernel<<<batch, 256, 0, s>>>(seq_off, rows, n_ctx, conf, argmax, lo, hi, k, tokens,
-                                      masked); note_launch();
-  return cudaGetLastError();
+  err = launch_k(unmask_kernel, batch, 256, 0, s, seq_off, rows, n_ctx, conf, argmax, lo, hi, k, tokens,
+                                      masked);
+  return err;
 }
 
 // ------------------------------------------------------------ active fill ---
 __global__ void active_fill_kernel(int32_t *rows, int32_t *seq_off, int batch, int n_ctx) {
+  pdl_wait();
+  pdl_trigger();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   int total = batch * n_ctx;
   if (i < total) rows[i] = i;
@@ -471,10 +485,11 @@ __global__ void active_fill_kernel(int32_t *rows, int32_t *seq_off, int batch, i
 
 cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n_ctx,
                                cudaStream_t s) {
+  cudaError_t err = cudaSuccess;
   int total = batch * n_ctx;
   int n = total > batch + 1 ? total : batch + 1;
-  active_fill_kernel<<<(n + 255) / 256, 256, 0, s>>>(rows, seq_off, batch, n_ctx); note_launch();
-  return cudaGetLastError();
+  err = launch_k(active_fill_kernel, (n + 255) / 256, 256, 0, s, rows, seq_off, batch, n_ctx);
+  return err;
 }
 
 }  // namespace sl

@@ -1,0 +1,271 @@
+"""Kernel-level benchmarks of the SureLock step on B200 (also the target of ncu
+captures).
+
+  python -m token_locking_b200.microbench layer [--m 2048,1024,...] [--iters K]
+      One LLaDA-8B-shaped transformer block (d=4096, 32 heads x 128, SwiGLU
+      12288) on M active rows of a sequence of N=2048 positions: random active
+      subset (seed 2), cache filled N(0,1), hidden states N(0,1).  Runs the
+      block through sl_layer_forward (gather of the active rows' inputs is the
+      caller's; norms, fused QKV + RoPE + cache scatter, attention over all
+      2048 keys, output projection + residual, SwiGLU FFN + residual).
+  python -m token_locking_b200.microbench lock [--m 64,512,2048] [--iters K]
+      The sure test on M rows of vocab 126464 bf16 logits, N(0,3) with a spike
+      (row max + 8) on a random half of the rows, previous logits perturbed by
+      N(0,0.05); KL test eps in {0.01, 0.05} with the 0.5-quantile confidence
+      gate, then compaction.
+  python -m token_locking_b200.microbench decode [--steps S]
+      The first S denoising steps of the LLaDA-8B-shaped decode (N=384).
+  python -m token_locking_b200.microbench gemm [--m 8,64,...]
+      Sweep of the tensor-core GEMM tilings (tile width, 128/256-row tiles,
+      K splits) on the LLaDA-8B projection shapes; one JSON line per tiling.
+
+Each case prints one JSON line: mean time per call (CUDA events, after
+warm-up, L2 flushed between calls by a 256 MB write), the roofline time of the
+case's algorithmic work and their ratio.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+from token_locking_b200 import runtime as rt  # noqa: E402
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]) * 1e9, float(d["bf16_tflops"]) * 1e12, "measured"
+    except Exception:
+        return 6650e9, 1590e12, "fallback"
+
+
+class _Flush:
+    def __init__(self, dev):
+        self.buf = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def _time(fn, iters, warmup, flush):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(iters):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        tot += e0.elapsed_time(e1)
+    return tot / iters
+
+
+def layer_work(shape, M, N):
+    d, f = shape.d_model, shape.d_ffn
+    flops = 2.0 * M * (4 * d * d + 3 * d * f) + 4.0 * M * N * d
+    byts = 2.0 * (4 * d * d + 3 * d * f) + 2.0 * 2 * N * d + 2.0 * 2 * M * d + 4.0 * 2 * M * d
+    return flops, byts
+
+
+def bench_layer(args, dev):
+    shape = wl.ModelShape(n_layers=1, d_model=4096, n_heads=32, head_dim=128, d_ffn=12288,
+                          vocab=126464, mask_id=126336, rope_theta=500000.0)
+    N = wl.LAYER_MICRO_N
+    w = wl.torch_weights(shape, dev)
+    model = rt.Model(shape, w, "bf16")
+    cache = rt.KVCache(model, 1, N)
+    g = torch.Generator(device=dev).manual_seed(wl.SEED_MICRO)
+    k, v = cache.view(0)
+    k.normal_(generator=g)
+    v.normal_(generator=g)
+    pb, pf, src = _peaks()
+    flush = _Flush(dev)
+    out = []
+    for M in args.m:
+        act = rt.Active(1, N)
+        act.load([wl.np_active_subset(N, M)])
+        h0 = torch.randn((M, shape.d_model), device=dev, generator=g)
+        h = h0.clone()
+
+        def fn():
+            h.copy_(h0)
+            rt.layer_forward(model, cache, act, 0, h)
+
+        ms = _time(fn, args.iters, 3, flush)
+        model.timing_enable(True)
+        model.timing_read(reset=True)
+        fn()
+        torch.cuda.synchronize()
+        tim = model.timing_read(reset=True)
+        model.timing_enable(False)
+        fl, by = layer_work(shape, M, N)
+        roof = max(fl / pf, by / pb) * 1e3
+        rec = {"case": "layer", "M": M, "N": N, "ms": round(ms, 4), "roofline_ms": round(roof, 4),
+               "frac": round(roof / ms, 4), "bound": "tensor" if fl / pf > by / pb else "hbm",
+               "gemm_ms": round(tim["gemm"]["ms"], 4), "attn_ms": round(tim["attn"]["ms"], 4),
+               "gemm_GBps": round(tim["gemm"]["bytes"] / tim["gemm"]["ms"] / 1e6, 1),
+               "gemm_TFLOPs": round(tim["gemm"]["flops"] / tim["gemm"]["ms"] / 1e9, 1),
+               "attn_TFLOPs": round(tim["attn"]["flops"] / max(tim["attn"]["ms"], 1e-9) / 1e9, 1),
+               "peaks": src}
+        print(json.dumps(rec), flush=True)
+        out.append(rec)
+        act.close()
+    model.close()
+    return out
+
+
+def bench_lock(args, dev):
+    V = wl.LLADA8B.vocab
+    pb, pf, src = _peaks()
+    flush = _Flush(dev)
+    for M in args.m:
+        z, zp, _ = wl.torch_lock_logits(M, V, dev)
+        lse_prev = torch.logsumexp(zp.float(), 1).contiguous()
+        act = rt.Active(1, M)
+        R = M
+        outs = dict(lse=torch.zeros(R, device=dev), kl=torch.zeros(R, device=dev),
+                    unc=torch.zeros(R, device=dev), conf=torch.zeros(R, device=dev),
+                    am=torch.zeros(R, device=dev, dtype=torch.int32),
+                    lock=torch.zeros(R, device=dev, dtype=torch.uint8))
+        masked = torch.zeros(R, device=dev, dtype=torch.uint8)
+        locked = torch.zeros(R, device=dev, dtype=torch.uint8)
+        lock_t = torch.zeros(R, device=dev, dtype=torch.int32)
+        for eps in wl.LOCK_MICRO_EPS:
+            def fn():
+                rt.kl_lock(act, V, wl.LLADA8B.mask_id, z, zp, lse_prev, outs["lse"], masked,
+                           outs["kl"], outs["unc"], outs["conf"], outs["am"], outs["lock"],
+                           eps=eps, gate_q=wl.LOCK_MICRO_GATE_Q)
+
+            act.reset()
+            ms = _time(fn, args.iters, 3, flush)
+            n_lock = int(outs["lock"].sum())
+            rt.compact_active(act, outs["lock"], locked, lock_t, 1)
+            m_after = int(act.counts()[0])
+            by = 4.0 * M * V + 16.0 * M
+            roof = by / pb * 1e3
+            print(json.dumps({"case": "lock", "M": M, "V": V, "eps": eps, "gate_q": 0.5,
+                              "ms": round(ms, 4), "roofline_ms": round(roof, 4),
+                              "frac": round(roof / ms, 4),
+                              "GBps": round(by / ms / 1e6, 1), "locked": n_lock,
+                              "M_after": m_after, "peaks": src}), flush=True)
+        act.close()
+
+
+def bench_decode(args, dev):
+    setup = wl.cfg_full8b(eps=0.05)
+    shape = setup.shape
+    w = wl.torch_weights(shape, dev)
+    model = rt.Model(shape, w, "bf16")
+    s = rt.Sampler(model, 1, setup.prompt_len, setup.gen_len, setup.steps, setup.block_len,
+                   setup.tokens_per_step, setup.eps)
+    prompts = torch.from_numpy(wl.np_prompts(1, setup.prompt_len, shape.vocab, shape.mask_id)).to(dev)
+    s.start(prompts)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    evs[0].record()
+    for t in range(args.steps):
+        s.step()
+        evs[t + 1].record()
+    torch.cuda.synchronize()
+    ms = [evs[t].elapsed_time(evs[t + 1]) for t in range(args.steps)]
+    print(json.dumps({"case": "decode", "steps": args.steps, "ms": [round(x, 3) for x in ms]}))
+
+
+def bench_gemm(args, dev):
+    from token_locking_b200 import _abi as A
+    d, f, V = 4096, 12288, 126464
+    pb, pf, src = _peaks()
+    g = torch.Generator(device=dev).manual_seed(3)
+
+    def w(*s):
+        return (torch.randn(s, device=dev, generator=g) * 0.02).to(torch.bfloat16)
+
+    shapes = {"qkv": (3 * d, d), "o": (d, d), "gu": (2 * f, d), "down": (d, f)}
+    if args.head:
+        shapes["head"] = (V, d)
+    weights = {k: w(n, kk) for k, (n, kk) in shapes.items() if k != "gu"}
+    wg, wu = w(f, d), w(f, d)
+    flush = _Flush(dev)
+    for M in args.m:
+        for name, (N, K) in shapes.items():
+            a = w(M, K)
+            outb = torch.zeros((M, N), device=dev, dtype=torch.bfloat16)
+            outf = torch.zeros((M, N), device=dev, dtype=torch.float32)
+            outa = torch.zeros((M, f), device=dev, dtype=torch.bfloat16)
+            for bn in (256, 128, 64, -256, -128, -64):
+                if abs(bn) < 128 and name == "qkv":
+                    continue
+                if (bn < 0 and M <= 128) or N % abs(bn):
+                    continue
+                for sp in (1, 2, 3, 4, 6, 8, 9, 12, 16):
+                    if sp > 1 and name == "head":
+                        continue
+                    if name == "gu":
+                        epi, b, b2, out = ((A.GEMM_SWIGLU, wg, wu, outa) if sp == 1 else
+                                           (A.GEMM_ACCUM, wg, wu, outf))
+                    elif name in ("o", "down"):
+                        epi, b, b2, out = A.GEMM_RESID, weights[name], None, outf
+                    else:
+                        epi, b, b2, out = ((A.GEMM_STORE, weights[name], None, outb) if sp == 1
+                                           else (A.GEMM_ACCUM, weights[name], None, outf))
+
+                    def fn():
+                        rt.gemm_bf16(epi, a, b, out, b2=b2, bn=bn, splits=sp)
+
+                    ms = _time(fn, args.iters, 2, flush)
+                    by = 2.0 * (N * K + M * K + M * N)
+                    fl = 2.0 * M * N * K
+                    print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": abs(bn),
+                                      "msub": 2 if bn < 0 else 1, "splits": sp,
+                                      "us": round(ms * 1e3, 2),
+                                      "GBps": round(by / ms / 1e6, 1),
+                                      "TFLOPs": round(fl / ms / 1e9, 1)}), flush=True)
+            # the library's own choice
+            if name == "gu":
+                epi, b, b2, out = A.GEMM_SWIGLU, wg, wu, outa
+            elif name in ("o", "down"):
+                epi, b, b2, out = A.GEMM_RESID, weights[name], None, outf
+            else:
+                epi, b, b2, out = A.GEMM_STORE, weights[name], None, outb
+
+            def fn():
+                rt.gemm_bf16(epi, a, b, out, b2=b2, bn=0, splits=0)
+
+            ms = _time(fn, args.iters, 2, flush)
+            print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": 0, "msub": 0,
+                              "splits": 0, "us": round(ms * 1e3, 2),
+                              "GBps": round(2.0 * (N * K + M * K + M * N) / ms / 1e6, 1)}),
+                  flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["layer", "lock", "decode", "gemm"])
+    ap.add_argument("--head", action="store_true")
+    ap.add_argument("--m", default=None)
+    ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=8)
+    args = ap.parse_args()
+    default = {"layer": wl.LAYER_MICRO_M, "lock": wl.LOCK_MICRO_M, "decode": (),
+               "gemm": (8, 64, 128, 200, 256, 384, 1024)}[args.case]
+    args.m = [int(x) for x in args.m.split(",")] if args.m else list(default)
+    dev = torch.device("cuda:0")
+    {"layer": bench_layer, "lock": bench_lock, "decode": bench_decode,
+     "gemm": bench_gemm}[args.case](args, dev)
+
+
+if __name__ == "__main__":
+    main()
