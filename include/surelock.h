@@ -240,6 +240,19 @@ sl_status sl_kl_stats_noalloc(const int32_t *d_rows, int M, int vocab, int mask_
                               float *d_lse_cur, int has_prev, float *d_kl, float *d_unc,
                               float *d_conf, int32_t *d_argmax, void *stream);
 
+/* Autotune the tensor-core GEMM tilings of this model on this device: every
+ * valid (tile width, 128/256-row tiles, K split) of the five projection GEMMs
+ * (fused QKV, output projection, fused gate/up, down projection, LM head) is
+ * timed at each row-count bucket up to max_rows, and later sl_step /
+ * sl_layer_forward calls use the fastest (untuned sizes use an analytic cost
+ * model).  Runs synchronously on `stream` (seconds at most); overwrites the
+ * cache's KV and workspace contents, so call it before a decode starts.
+ * A no-op for fp32 models. */
+sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows, void *stream);
+/* The tiling sl_step would use for GEMM `kind` (0 QKV, 1 output projection,
+ * 2 gate/up, 3 down, 4 LM head) at M rows. */
+sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits, int *msub);
+
 /* ---------------------------------------------------------------- sampler --- */
 
 /* Semi-autoregressive SureLock decode driven by the library: prompt_len given

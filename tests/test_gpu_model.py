@@ -127,3 +127,36 @@ def test_layer_forward_bf16_matches_oracle(cuda_dev):
     err = np.abs(h.double().cpu().numpy() - ref).max()
     assert err <= 5e-2 * max(1.0, np.abs(ref).max()), err
     model.close()
+
+
+def test_autotuned_step_matches_oracle(cuda_dev):
+    """After autotuning, the tilings chosen per row count are valid and the step
+    still agrees with the oracle (the tuning only changes the schedule)."""
+    shape = MINI_BF16
+    B, n_ctx = 2, 200
+    w_np = wl.np_weights(shape, seed=0, std=0.05, gain_jitter=0.1)
+    w_dev = weights_to_device(w_np, "bf16", cuda_dev)
+    w64 = weights_for_oracle(w_dev)
+    model = rt.Model(shape, w_dev, "bf16")
+    cache = rt.KVCache(model, B, n_ctx)
+    model.autotune(cache, B * n_ctx)
+    for kind in range(5):
+        for M in (1, 100, 257, 400):
+            bn, sp, ms = model.tuning(kind, M)
+            assert bn in (64, 128, 256) and sp >= 1 and ms in (1, 2)
+    act = rt.Active(B, n_ctx)
+    tokens, positions, ck, cv = _state(shape, B, n_ctx, [160, 130], seed=11, dev=cuda_dev,
+                                       dtype="bf16")
+    act.load(positions)
+    _load_cache(cache, ck, cv, torch.bfloat16)
+    tok = torch.from_numpy(tokens).to(cuda_dev)
+    logits = torch.zeros((B * n_ctx, shape.vocab), device=cuda_dev, dtype=torch.bfloat16)
+    rt.step(model, cache, act, tok, logits)
+    torch.cuda.synchronize()
+    rt.device_check()
+    zs, _, _ = _oracle_step(shape, w64, tokens, positions, ck, cv, n_ctx)
+    lg = to64(logits)
+    for b in range(B):
+        err = np.abs(lg[positions[b] + b * n_ctx] - zs[b]).max()
+        assert err <= LOGIT_TOL["bf16"], err
+    model.close()

@@ -106,6 +106,8 @@ struct sl_model {
   std::vector<TimingRec> recs;
   sl_timing acc{};
   long long launch_base = 0;
+  // autotuned GEMM tilings: [kind][row-count bucket] = {bn, splits, msub} (bn 0 = untuned)
+  std::vector<std::array<int, 3>> tuned[5];
 };
 
 struct sl_kv_cache {
@@ -637,14 +639,44 @@ struct BfPlans {
   Plan qkv, o, gu, dn, hd;
 };
 
-static BfPlans plans_for(const sl_config &cfg, int M, int ns) {
+enum GemmKind { G_QKV = 0, G_O = 1, G_GU = 2, G_DN = 3, G_HD = 4, G_KINDS = 5 };
+
+// Row-count buckets of the GEMM autotuner: a step with M active rows uses the
+// tiling tuned at the smallest bound >= M.
+static const int kTuneBounds[] = {16,   32,   64,   96,   128,  160,  192,  224,  256,
+                                  320,  384,  512,  768,  1024, 1536, 2048, 3072, 4096,
+                                  6144, 8192, 12288, 16384, 24576, 32768, 65536, 131072};
+static const int kTuneCount = sizeof(kTuneBounds) / sizeof(kTuneBounds[0]);
+static int tune_bucket(int M) {
+  for (int i = 0; i < kTuneCount; ++i)
+    if (M <= kTuneBounds[i]) return i;
+  return -1;
+}
+
+static Plan plan_kind(const sl_model *m, int kind, int M, int ns) {
+  const int bkt = tune_bucket(M);
+  if (bkt >= 0 && bkt < (int)m->tuned[kind].size() && m->tuned[kind][bkt][0] > 0) {
+    const auto &t = m->tuned[kind][bkt];
+    return Plan{t[0], t[1], t[2], 0.0};
+  }
+  const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn;
+  switch (kind) {
+    case G_QKV: return plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128);
+    case G_O: return plan_gemm(M, d, d, SPLIT_RESID, ns, false);
+    case G_GU: return plan_gemm(M, 2 * f, d, SPLIT_ACCUM, ns, true);
+    case G_DN: return plan_gemm(M, d, f, SPLIT_RESID, ns, false);
+    default: return plan_gemm(M, cfg.vocab, d, SPLIT_NONE, ns, false);
+  }
+}
+
+static BfPlans plans_for(const sl_model *m, int M, int ns) {
   BfPlans p;
-  p.qkv = plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128);
-  p.o = plan_gemm(M, d, d, SPLIT_RESID, ns, false);
-  p.gu = plan_gemm(M, 2 * f, d, SPLIT_ACCUM, ns, true);
-  p.dn = plan_gemm(M, d, f, SPLIT_RESID, ns, false);
-  p.hd = plan_gemm(M, cfg.vocab, d, SPLIT_NONE, ns, false);
+  p.qkv = plan_kind(m, G_QKV, M, ns);
+  p.o = plan_kind(m, G_O, M, ns);
+  p.gu = plan_kind(m, G_GU, M, ns);
+  p.dn = plan_kind(m, G_DN, M, ns);
+  p.hd = plan_kind(m, G_HD, M, ns);
   return p;
 }
 
@@ -679,114 +711,125 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
   return SL_OK;
 }
 
+// One of the step's projection GEMMs on the current activation descriptors,
+// with the split-K finalize pass when the plan splits K:
+//   G_QKV  a (normed h) x [Wq|Wk|Wv]^T -> RoPE(q) -> q, RoPE(k), v -> C.k/C.v[rows]
+//   G_O    o x Wo^T, added to the residual h
+//   G_GU   b x [Wg|Wu]^T -> silu(gate) * up -> act
+//   G_DN   act x Wd^T, added to the residual h
+//   G_HD   RMSNorm(h) x W_out^T -> logits[rows]
+static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int l, int kind,
+                          const Plan &pl, int M, float *h, void *logits, cudaStream_t s) {
+  const sl_config &cfg = m->cfg;
+  const int d = cfg.d_model, f = cfg.d_ffn, V = cfg.vocab, H = cfg.n_heads;
+  const double Md = (double)M;
+  const bool split = pl.splits > 1;
+  TcGemmArgs g{};
+  g.M = M;
+  g.bn = pl.bn;
+  g.splits = pl.splits;
+  g.msub = pl.msub;
+  double bytes = 0, flops = 0;
+  switch (kind) {
+    case G_QKV: {
+      const auto &mp = m->maps[l];
+      g.A = &c->map_a;
+      g.B[0] = mp[W_Q].box(pl.bn);
+      g.B[1] = mp[W_K].box(pl.bn);
+      g.B[2] = mp[W_V].box(pl.bn);
+      g.n_seg[0] = g.n_seg[1] = g.n_seg[2] = d;
+      g.N = 3 * d;
+      g.K = d;
+      if (split) {
+        // K split across CTAs: fp32 partial sums, then RoPE + scatter from them
+        g.epi = EPI_ACCUM;
+        g.out = c->ws;
+        g.ldo = 3 * d;
+      } else {
+        g.epi = EPI_QKV;
+        g.row_map = rows;
+        g.rope = c->rope;
+        g.n_ctx = c->n_ctx;
+        g.q_out = c->q;
+        g.ck = c->k[l];
+        g.cv = c->v[l];
+      }
+      bytes = gemm_bytes(Md, 3.0 * d, d, 2);
+      flops = 6.0 * Md * d * d;
+      break;
+    }
+    case G_O:
+    case G_DN: {
+      const auto &mp = m->maps[l];
+      const int K = kind == G_O ? d : f;
+      g.A = kind == G_O ? &c->map_o : &c->map_act;
+      g.B[0] = mp[kind == G_O ? W_O : W_D].box(pl.bn);
+      g.n_seg[0] = d;
+      g.N = d;
+      g.K = K;
+      g.epi = EPI_RESID;
+      g.out = h;
+      g.ldo = d;
+      bytes = gemm_bytes(Md, d, K, 2);
+      flops = 2.0 * Md * d * K;
+      break;
+    }
+    case G_GU: {
+      const auto &mp = m->maps[l];
+      g.A = &c->map_a;
+      g.B[0] = mp[W_G].box(pl.bn / 2);
+      g.B[1] = mp[W_U].box(pl.bn / 2);
+      g.b_swiglu = 1;
+      g.N = 2 * f;
+      g.K = d;
+      g.epi = split ? EPI_ACCUM : EPI_SWIGLU;
+      g.out = split ? (void *)c->ws : c->act;
+      g.ldo = split ? 2 * f : f;
+      bytes = gemm_bytes(Md, 2.0 * f, d, 2) - 2.0 * Md * f;
+      flops = 4.0 * Md * d * f;
+      break;
+    }
+    default: {   // G_HD
+      g.A = &c->map_a;
+      g.B[0] = m->head_map.box(pl.bn);
+      g.n_seg[0] = V;
+      g.N = V;
+      g.K = d;
+      g.splits = 1;
+      g.epi = EPI_STORE;
+      g.out = logits;
+      g.ldo = V;
+      g.row_map = rows;
+      bytes = gemm_bytes(Md, V, d, 2);
+      flops = 2.0 * Md * d * V;
+      break;
+    }
+  }
+  {
+    Timed t(m, SL_K_GEMM, bytes, flops, s);
+    sl_status st = tc_gemm(m, g, s);
+    if (st != SL_OK) return st;
+  }
+  if (split && kind == G_QKV)
+    SL_CUDA(launch_rope_scatter(SL_BF16, c->ws, true, true, M, rows, c->n_ctx, H, cfg.head_dim,
+                                c->rope, c->q, c->k[l], c->v[l], s));
+  if (split && kind == G_GU) SL_CUDA(launch_swiglu(SL_BF16, c->ws, true, true, M, f, c->act, s));
+  return SL_OK;
+}
+
 static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, float *h, int M,
                             const AttnSeqs &seqs, const BfPlans &pl, cudaStream_t s) {
   const sl_config &cfg = m->cfg;
-  const int d = cfg.d_model, f = cfg.d_ffn, H = cfg.n_heads;
+  const int d = cfg.d_model;
   const sl_layer_weights &lw = m->layers[l];
-  const auto &mp = m->maps[l];
-  const double Md = (double)M;
   sl_status st;
   SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s));
-  {
-    // fused Q | K | V projection over the three weight matrices
-    TcGemmArgs g{};
-    g.A = &c->map_a;
-    g.B[0] = mp[W_Q].box(pl.qkv.bn);
-    g.B[1] = mp[W_K].box(pl.qkv.bn);
-    g.B[2] = mp[W_V].box(pl.qkv.bn);
-    g.n_seg[0] = d;
-    g.n_seg[1] = d;
-    g.n_seg[2] = d;
-    g.M = M;
-    g.N = 3 * d;
-    g.K = d;
-    g.bn = pl.qkv.bn;
-    g.splits = pl.qkv.splits;
-    g.msub = pl.qkv.msub;
-    const bool split = pl.qkv.splits > 1;
-    if (split) {
-      // K split across CTAs: fp32 partial sums, then RoPE + scatter from them
-      g.epi = EPI_ACCUM;
-      g.out = c->ws;
-      g.ldo = 3 * d;
-    } else {
-      // epilogue: RoPE(q) -> q, RoPE(k) and v -> C.k/C.v at the rows' positions
-      g.epi = EPI_QKV;
-      g.row_map = a->rows;
-      g.rope = c->rope;
-      g.n_ctx = c->n_ctx;
-      g.q_out = c->q;
-      g.ck = c->k[l];
-      g.cv = c->v[l];
-    }
-    {
-      Timed t(m, SL_K_GEMM, gemm_bytes(Md, 3.0 * d, d, 2), 6.0 * Md * d * d, s);
-      if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
-    }
-    if (split)
-      SL_CUDA(launch_rope_scatter(SL_BF16, c->ws, true, true, M, a->rows, c->n_ctx, H,
-                                  cfg.head_dim, c->rope, c->q, c->k[l], c->v[l], s));
-  }
+  if ((st = run_gemm(m, c, a->rows, l, G_QKV, pl.qkv, M, h, nullptr, s)) != SL_OK) return st;
   if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, s)) != SL_OK) return st;
-  {
-    TcGemmArgs g{};
-    g.A = &c->map_o;
-    g.B[0] = mp[W_O].box(pl.o.bn);
-    g.n_seg[0] = d;
-    g.M = M;
-    g.N = d;
-    g.K = d;
-    g.bn = pl.o.bn;
-    g.splits = pl.o.splits;
-    g.msub = pl.o.msub;
-    g.epi = EPI_RESID;
-    g.out = h;
-    g.ldo = d;
-    Timed t(m, SL_K_GEMM, gemm_bytes(Md, d, d, 2), 2.0 * Md * d * d, s);
-    if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
-  }
+  if ((st = run_gemm(m, c, a->rows, l, G_O, pl.o, M, h, nullptr, s)) != SL_OK) return st;
   SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.ffn_norm, d, cfg.rms_eps, M, c->a, s));
-  {
-    TcGemmArgs g{};
-    g.A = &c->map_a;
-    g.B[0] = mp[W_G].box(pl.gu.bn / 2);
-    g.B[1] = mp[W_U].box(pl.gu.bn / 2);
-    g.b_swiglu = 1;
-    g.M = M;
-    g.N = 2 * f;
-    g.K = d;
-    g.bn = pl.gu.bn;
-    g.splits = pl.gu.splits;
-    g.msub = pl.gu.msub;
-    const bool split = pl.gu.splits > 1;
-    g.epi = split ? EPI_ACCUM : EPI_SWIGLU;
-    g.out = split ? (void *)c->ws : c->act;
-    g.ldo = split ? 2 * f : f;
-    {
-      Timed t(m, SL_K_GEMM, gemm_bytes(Md, 2.0 * f, d, 2) - 2.0 * Md * f, 4.0 * Md * d * f, s);
-      if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
-    }
-    if (split) SL_CUDA(launch_swiglu(SL_BF16, c->ws, true, true, M, f, c->act, s));
-  }
-  {
-    TcGemmArgs g{};
-    g.A = &c->map_act;
-    g.B[0] = mp[W_D].box(pl.dn.bn);
-    g.n_seg[0] = d;
-    g.M = M;
-    g.N = d;
-    g.K = f;
-    g.bn = pl.dn.bn;
-    g.splits = pl.dn.splits;
-    g.msub = pl.dn.msub;
-    g.epi = EPI_RESID;
-    g.out = h;
-    g.ldo = d;
-    Timed t(m, SL_K_GEMM, gemm_bytes(Md, d, f, 2), 2.0 * Md * d * f, s);
-    if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
-  }
-  return SL_OK;
+  if ((st = run_gemm(m, c, a->rows, l, G_GU, pl.gu, M, h, nullptr, s)) != SL_OK) return st;
+  return run_gemm(m, c, a->rows, l, G_DN, pl.dn, M, h, nullptr, s);
 }
 
 static sl_status check_pair(sl_model *m, sl_kv_cache *c, sl_active *a, const char *who) {
@@ -826,28 +869,11 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   if ((st = ensure_maps(c, M)) != SL_OK) return st;
   AttnSeqs seqs;
   fill_seqs(seqs, a, counts);
-  const BfPlans pl = plans_for(cfg, M, m->num_sms);
+  const BfPlans pl = plans_for(m, M, m->num_sms);
   for (int l = 0; l < cfg.n_layers; ++l)
     if ((st = layer_bf16(m, c, a, l, c->h, M, seqs, pl, s)) != SL_OK) return st;
   SL_CUDA(launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
-  TcGemmArgs g{};
-  g.A = &c->map_a;
-  g.B[0] = m->head_map.box(pl.hd.bn);
-  g.n_seg[0] = V;
-  g.M = M;
-  g.N = V;
-  g.K = d;
-  g.bn = pl.hd.bn;
-  g.splits = 1;
-  g.msub = pl.hd.msub;
-  g.epi = EPI_STORE;
-  g.out = d_logits;
-  g.ldo = V;
-  g.row_map = a->rows;
-  {
-    Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 2), 2.0 * (double)M * d * V, s);
-    if ((st = tc_gemm(m, g, s)) != SL_OK) return st;
-  }
+  if ((st = run_gemm(m, c, a->rows, 0, G_HD, pl.hd, M, c->h, d_logits, s)) != SL_OK) return st;
   // the previous step's timing events completed before this step was planned
   if (m->timing) timing_harvest(m, false);
   return SL_OK;
@@ -871,7 +897,7 @@ extern "C" sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a,
   if ((st = ensure_maps(c, M)) != SL_OK) return st;
   AttnSeqs seqs;
   fill_seqs(seqs, a, counts);
-  return layer_bf16(m, c, a, layer, d_h, M, seqs, plans_for(m->cfg, M, m->num_sms), s);
+  return layer_bf16(m, c, a, layer, d_h, M, seqs, plans_for(m, M, m->num_sms), s);
 }
 
 extern "C" sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
@@ -957,6 +983,121 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   if (!err) return fail(SL_ERR_CUDA, "sl_gemm_bf16: no device error word");
   cudaError_t e = launch_gemm_tc(g, ns, err, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "sl_gemm_bf16 launch");
+  return SL_OK;
+}
+
+// --------------------------------------------------------------- autotune --
+// Time every valid tiling of the five projection GEMMs at each row-count bucket
+// up to max_rows on this device, keep the fastest.  Uses layer 0's weights
+// and the cache's workspaces (their contents are overwritten).
+extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows, void *stream) {
+  if (!m || !c) return fail(SL_ERR_INVALID, "sl_model_autotune: null argument");
+  if (c->m != m) return fail(SL_ERR_INVALID, "sl_model_autotune: cache belongs to another model");
+  if (m->cfg.dtype != SL_BF16) return SL_OK;            // the fp32 path has one tiling
+  if (max_rows <= 0) return fail(SL_ERR_INVALID, "sl_model_autotune: max_rows must be positive");
+  max_rows = std::min(max_rows, c->max_rows);
+  cudaStream_t s = (cudaStream_t)stream;
+  const sl_config &cfg = m->cfg;
+  const int d = cfg.d_model, f = cfg.d_ffn, V = cfg.vocab;
+  const int head_rows = std::min(max_rows, 8192);
+  int32_t *rows = nullptr;
+  void *logits = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  std::vector<int32_t> h_rows(max_rows);
+  for (int i = 0; i < max_rows; ++i) h_rows[i] = i;
+  sl_status st = SL_OK;
+  const bool was_timing = m->timing;
+  m->timing = false;
+  auto cleanup = [&]() {
+    if (rows) cudaFree(rows);
+    if (logits) cudaFree(logits);
+    if (e0) cudaEventDestroy(e0);
+    if (e1) cudaEventDestroy(e1);
+    m->timing = was_timing;
+    c->map_rows = -1;
+  };
+  if (cudaMalloc(&rows, max_rows * sizeof(int32_t)) != cudaSuccess ||
+      cudaMalloc(&logits, (size_t)head_rows * V * 2) != cudaSuccess ||
+      cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) {
+    cleanup();
+    return fail(SL_ERR_OOM, "sl_model_autotune: scratch allocation failed");
+  }
+  if (cudaMemcpy(rows, h_rows.data(), max_rows * sizeof(int32_t), cudaMemcpyHostToDevice) !=
+      cudaSuccess) {
+    cleanup();
+    return fail(SL_ERR_CUDA, "sl_model_autotune: copy failed");
+  }
+  for (int k = 0; k < G_KINDS; ++k) m->tuned[k].assign(kTuneCount, {0, 1, 1});
+  const int Ns[G_KINDS] = {3 * d, d, 2 * f, d, V};
+  const int Ks[G_KINDS] = {d, d, d, f, d};
+  const int split_opts[] = {1, 2, 3, 4, 6, 8, 9, 12, 16};
+  for (int b = 0; b < kTuneCount && st == SL_OK; ++b) {
+    if (b > 0 && kTuneBounds[b - 1] >= max_rows) break;
+    const int Mb = std::min(kTuneBounds[b], max_rows);
+    if ((st = ensure_maps(c, Mb)) != SL_OK) break;
+    for (int kind = 0; kind < G_KINDS && st == SL_OK; ++kind) {
+      if (kind == G_HD && Mb > head_rows) continue;
+      const int N = Ns[kind], K = Ks[kind], kblocks = K / 64;
+      double best_ms = 1e30;
+      std::array<int, 3> best = {0, 1, 1};
+      for (int msub = 1; msub <= 2; ++msub) {
+        if (msub == 2 && Mb <= 128) continue;
+        for (int bn : {256, 128, 64}) {
+          if (N % bn || (kind == G_QKV && bn < 128)) continue;
+          if (kind == G_GU && (N / 2) % (bn / 2)) continue;
+          int last_ss = 0;
+          for (int sp : split_opts) {
+            if (kind == G_HD && sp > 1) break;
+            if (sp > std::max(1, kblocks / 2)) break;
+            const int kbp = (kblocks + sp - 1) / sp;
+            const int ss = (kblocks + kbp - 1) / kbp;
+            if (ss == last_ss) continue;
+            last_ss = ss;
+            const long units = (long)((Mb + 128 * msub - 1) / (128 * msub)) * (N / bn) * ss;
+            if (units > 24L * m->num_sms) continue;
+            const Plan pl{bn, ss, msub, 0.0};
+            auto launch = [&]() {
+              return run_gemm(m, c, rows, 0, kind, pl, Mb, c->h, logits, s);
+            };
+            if ((st = launch()) != SL_OK) break;
+            cudaEventRecord(e0, s);
+            for (int it = 0; it < 3 && st == SL_OK; ++it) st = launch();
+            cudaEventRecord(e1, s);
+            if (st != SL_OK) break;
+            if (cudaEventSynchronize(e1) != cudaSuccess) {
+              st = cuda_fail(cudaGetLastError(), "sl_model_autotune: timing");
+              break;
+            }
+            float ms = 0.f;
+            cudaEventElapsedTime(&ms, e0, e1);
+            if (ms < best_ms) {
+              best_ms = ms;
+              best = {bn, ss, msub};
+            }
+          }
+          if (st != SL_OK) break;
+        }
+        if (st != SL_OK) break;
+      }
+      m->tuned[kind][b] = best;
+    }
+  }
+  cleanup();
+  if (st != SL_OK) {
+    for (int k = 0; k < G_KINDS; ++k) m->tuned[k].clear();
+    return st;
+  }
+  return SL_OK;
+}
+
+extern "C" sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits,
+                                     int *msub) {
+  if (!m || !bn || !splits || !msub || kind < 0 || kind >= G_KINDS || M <= 0)
+    return fail(SL_ERR_INVALID, "sl_model_tuning: bad argument");
+  const Plan p = plan_kind(m, kind, M, m->num_sms);
+  *bn = p.bn;
+  *splits = p.splits;
+  *msub = p.msub;
   return SL_OK;
 }
 

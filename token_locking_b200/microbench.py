@@ -89,6 +89,8 @@ def bench_layer(args, dev):
     model = rt.Model(shape, w, "bf16")
     cache = rt.KVCache(model, 1, N)
     g = torch.Generator(device=dev).manual_seed(wl.SEED_MICRO)
+    if not args.no_tune:
+        model.autotune(cache, N)
     k, v = cache.view(0)
     k.normal_(generator=g)
     v.normal_(generator=g)
@@ -172,6 +174,8 @@ def bench_decode(args, dev):
     model = rt.Model(shape, w, "bf16")
     s = rt.Sampler(model, 1, setup.prompt_len, setup.gen_len, setup.steps, setup.block_len,
                    setup.tokens_per_step, setup.eps)
+    if not args.no_tune:
+        s.autotune()
     prompts = torch.from_numpy(wl.np_prompts(1, setup.prompt_len, shape.vocab, shape.mask_id)).to(dev)
     s.start(prompts)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
@@ -255,6 +259,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["layer", "lock", "decode", "gemm"])
     ap.add_argument("--head", action="store_true")
+    ap.add_argument("--no-tune", action="store_true")
     ap.add_argument("--m", default=None)
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--steps", type=int, default=8)

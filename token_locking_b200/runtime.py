@@ -96,6 +96,17 @@ class Model:
         except Exception:
             pass
 
+    def autotune(self, cache: "KVCache", max_rows: int, stream=None):
+        """Time the GEMM tilings on this device and keep the fastest per row count."""
+        A.check(A.lib().sl_model_autotune(self.handle, cache.handle, max_rows, _stream(stream)),
+                "sl_model_autotune")
+
+    def tuning(self, kind: int, M: int):
+        bn, sp, ms = C.c_int(), C.c_int(), C.c_int()
+        A.check(A.lib().sl_model_tuning(self.handle, kind, M, C.byref(bn), C.byref(sp),
+                                        C.byref(ms)), "sl_model_tuning")
+        return bn.value, sp.value, ms.value
+
     def timing_enable(self, on: bool = True):
         A.check(A.lib().sl_timing_enable(self.handle, 1 if on else 0), "sl_timing_enable")
 
@@ -320,6 +331,13 @@ class Sampler:
     def generate_ptr(self, h_prompts_ptr: int, h_out_ptr: int, stream=None):
         A.check(A.lib().sl_sampler_generate(self.handle, h_prompts_ptr, h_out_ptr,
                                             _stream(stream)), "sl_sampler_generate")
+
+    def autotune(self, stream=None):
+        """Autotune the model's GEMM tilings for this sampler's batch and length."""
+        st = A.SamplerState()
+        A.check(A.lib().sl_sampler_get_state(self.handle, C.byref(st)), "sl_sampler_get_state")
+        cache = KVCache.wrap(st.cache, self.model, st.batch, st.n_ctx)
+        self.model.autotune(cache, st.batch * st.n_ctx, stream)
 
     def state(self) -> dict:
         st = A.SamplerState()
