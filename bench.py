@@ -71,6 +71,21 @@ def make_setup(name: str, eps, scripted: bool) -> wl.SamplerSetup:
     return s
 
 
+def gemm_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu capture, or None when
+    the kernel source changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")) as f:
+            rec = json.load(f)
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+                return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def step_work(shape: wl.ModelShape, m_rows: int, batch: int, n_ctx: int):
     """Algorithmic FLOPs and HBM bytes of one denoising step on m_rows active
     rows (all sequences of the batch), attending to n_ctx keys per sequence."""
@@ -352,6 +367,7 @@ def run_ours(args, rank: int, world: int):
         g = tim["gemm"]
         t_f = g["flops"] / pf
         t_b = g["bytes"] / pb
+        traffic = gemm_traffic()
         if t_b >= t_f:
             bound, ach, peak, unit = "hbm", g["bytes"] / (g["ms"] / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
         else:
@@ -399,7 +415,8 @@ def run_ours(args, rank: int, world: int):
                     "h2d_bytes_per_step": int(prompts.nbytes),
                     "d2h_bytes_per_step": int(setup.batch * setup.n_ctx * 4)},
             "roofline": {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
-                         "frac": round(ach / peak, 4), "traffic": None,
+                         "frac": round(ach / peak, 4), "traffic": traffic,
+                         "algorithmic_bytes_per_launch": round(g["bytes"] / max(1, g["launches"])),
                          "kernel": "gemm_tc_kernel (tcgen05)",
                          "launches": g["launches"], "kernel_ms": round(g["ms"], 3),
                          "peak_source": peaks["source"],

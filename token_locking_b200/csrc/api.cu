@@ -1056,8 +1056,15 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
             const long units = (long)((Mb + 128 * msub - 1) / (128 * msub)) * (N / bn) * ss;
             if (units > 24L * m->num_sms) continue;
             const Plan pl{bn, ss, msub, 0.0};
+            // each repetition is followed by a small kernel (an RMSNorm, as in
+            // the layer) so that successive GEMMs cannot overlap each other
+            // through programmatic launch and flatter tilings with few CTAs
             auto launch = [&]() {
-              return run_gemm(m, c, rows, 0, kind, pl, Mb, c->h, logits, s);
+              sl_status r = run_gemm(m, c, rows, 0, kind, pl, Mb, c->h, logits, s);
+              if (r != SL_OK) return r;
+              cudaError_t e = launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, Mb,
+                                             c->a, s);
+              return e == cudaSuccess ? SL_OK : cuda_fail(e, "sl_model_autotune: spacer");
             };
             if ((st = launch()) != SL_OK) break;
             cudaEventRecord(e0, s);

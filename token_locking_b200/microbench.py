@@ -97,6 +97,8 @@ def bench_layer(args, dev):
     pb, pf, src = _peaks()
     flush = _Flush(dev)
     out = []
+    torch.cuda.synchronize()
+    torch.cuda.profiler.start()          # ncu --profile-from-start off captures from here
     for M in args.m:
         act = rt.Active(1, N)
         act.load([wl.np_active_subset(N, M)])
@@ -126,6 +128,7 @@ def bench_layer(args, dev):
         print(json.dumps(rec), flush=True)
         out.append(rec)
         act.close()
+    torch.cuda.profiler.stop()
     model.close()
     return out
 
@@ -134,6 +137,8 @@ def bench_lock(args, dev):
     V = wl.LLADA8B.vocab
     pb, pf, src = _peaks()
     flush = _Flush(dev)
+    torch.cuda.synchronize()
+    torch.cuda.profiler.start()
     for M in args.m:
         z, zp, _ = wl.torch_lock_logits(M, V, dev)
         lse_prev = torch.logsumexp(zp.float(), 1).contiguous()
@@ -165,6 +170,7 @@ def bench_lock(args, dev):
                               "GBps": round(by / ms / 1e6, 1), "locked": n_lock,
                               "M_after": m_after, "peaks": src}), flush=True)
         act.close()
+    torch.cuda.profiler.stop()
 
 
 def bench_decode(args, dev):
@@ -178,12 +184,15 @@ def bench_decode(args, dev):
         s.autotune()
     prompts = torch.from_numpy(wl.np_prompts(1, setup.prompt_len, shape.vocab, shape.mask_id)).to(dev)
     s.start(prompts)
+    torch.cuda.synchronize()
+    torch.cuda.profiler.start()          # ncu --profile-from-start off captures from here
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     evs[0].record()
     for t in range(args.steps):
         s.step()
         evs[t + 1].record()
     torch.cuda.synchronize()
+    torch.cuda.profiler.stop()
     ms = [evs[t].elapsed_time(evs[t + 1]) for t in range(args.steps)]
     print(json.dumps({"case": "decode", "steps": args.steps, "ms": [round(x, 3) for x in ms]}))
 
