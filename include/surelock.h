@@ -207,14 +207,16 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
  *                   out bf16 [M][ldo] = silu(A W_gate^T) * (A W_up^T)
  *   SL_GEMM_ACCUM : out fp32 [M][ldo] += C (atomic; with d_b2, gate/up halves
  *                   accumulate into columns [0,F) and [F,2F))
- * bn (64/128/256) and splits (>= 1, RESID/ACCUM only) pick the tiling, with
- * 128 rows of A per tile; -64/-128/-256 select 256-row tiles (two tensor-core
- * accumulators share each weight tile); bn = 0 lets the library choose.
- * K % 64 == 0, N % |bn| == 0, pointers 16-byte aligned. */
+ * bn (64/128/256) and splits (>= 1, RESID/ACCUM only) pick the tiling; variant
+ * picks the kernel: 0 = one CTA per 128 x bn tile, 1 = one CTA per 256 x bn
+ * tile (two accumulators share each weight tile), 2 = a CTA pair per 256 x bn
+ * tile with 2-SM tensor-core instructions (bn 128 or 256).  bn = 0 lets the
+ * library choose everything.  K % 64 == 0, N % bn == 0, pointers 16-byte
+ * aligned. */
 enum { SL_GEMM_STORE = 0, SL_GEMM_RESID = 1, SL_GEMM_SWIGLU = 2, SL_GEMM_ACCUM = 3 };
 sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b, const void *d_b2,
                        int N, void *d_out, int ldo, const int32_t *d_row_map, int bn, int splits,
-                       void *stream);
+                       int variant, void *stream);
 
 /* The per-row statistics of sl_kl_lock (lse, D, u, conf, argmax; no gate and
  * no lock flags) for callers that cannot allocate device memory: hosts whose
@@ -250,8 +252,8 @@ sl_status sl_kl_stats_noalloc(const int32_t *d_rows, int M, int vocab, int mask_
  * A no-op for fp32 models. */
 sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows, void *stream);
 /* The tiling sl_step would use for GEMM `kind` (0 QKV, 1 output projection,
- * 2 gate/up, 3 down, 4 LM head) at M rows. */
-sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits, int *msub);
+ * 2 gate/up, 3 down, 4 LM head) at M rows; *variant as for sl_gemm_bf16. */
+sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits, int *variant);
 
 /* ---------------------------------------------------------------- sampler --- */
 

@@ -62,5 +62,6 @@ def test_host_side_argument_checks(lib):
     assert lib.sl_step(None, None, None, None, None, None) == A.SL_ERR_INVALID
     assert lib.sl_sampler_step(None, None) == A.SL_ERR_INVALID
     # GEMM: K must be a multiple of 64; a bad epilogue code is rejected
-    assert lib.sl_gemm_bf16(0, 16, 8, 100, 16, None, 128, 16, 128, None, 128, 1, None) == A.SL_ERR_INVALID
-    assert lib.sl_gemm_bf16(9, 16, 8, 128, 16, None, 128, 16, 128, None, 128, 1, None) == A.SL_ERR_INVALID
+    assert lib.sl_gemm_bf16(0, 16, 8, 100, 16, None, 128, 16, 128, None, 128, 1, 0, None) == A.SL_ERR_INVALID
+    assert lib.sl_gemm_bf16(9, 16, 8, 128, 16, None, 128, 16, 128, None, 128, 1, 0, None) == A.SL_ERR_INVALID
+    assert lib.sl_gemm_bf16(0, 16, 8, 128, 16, None, 128, 16, 128, None, 128, 1, 3, None) == A.SL_ERR_INVALID

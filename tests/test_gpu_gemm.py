@@ -28,14 +28,18 @@ def _close(got, ref, K, bf16_out):
     assert err <= tol, f"max err {err} > tol {tol} (scale {scale})"
 
 
-@pytest.mark.parametrize("bn", [64, 128, 256, -64, -128, -256])
+VARIANTS = [(64, 0), (128, 0), (256, 0), (64, 1), (128, 1), (256, 1), (128, 2), (256, 2)]
+
+
+@pytest.mark.parametrize("bn,variant", VARIANTS)
 @pytest.mark.parametrize("M", [1, 37, 128, 301])
-def test_store_rowmap(cuda_dev, bn, M):
+def test_store_rowmap(cuda_dev, bn, variant, M):
     K, N = 512, 768
     a, b = _mk((M, K), 1, cuda_dev), _mk((N, K), 2, cuda_dev)
     perm = torch.randperm(M + 5, generator=torch.Generator().manual_seed(3))[:M].to(torch.int32)
     out = torch.full((M + 5, N), 7.0, device=cuda_dev, dtype=torch.bfloat16)
-    rt.gemm_bf16(A.GEMM_STORE, a, b, out, row_map=perm.to(cuda_dev), bn=bn, splits=1)
+    rt.gemm_bf16(A.GEMM_STORE, a, b, out, row_map=perm.to(cuda_dev), bn=bn, splits=1,
+                 variant=variant)
     torch.cuda.synchronize()
     ref = _ref(a, b)
     _close(out[perm.long()], ref, K, True)
@@ -45,30 +49,32 @@ def test_store_rowmap(cuda_dev, bn, M):
     rt.device_check()
 
 
-@pytest.mark.parametrize("bn,splits", [(64, 1), (128, 3), (256, 2), (128, 8), (-256, 3),
-                                       (-128, 1), (-64, 2)])
+@pytest.mark.parametrize("bn,splits,variant", [(64, 1, 0), (128, 3, 0), (256, 2, 0), (128, 8, 0),
+                                               (256, 3, 1), (128, 1, 1), (64, 2, 1), (256, 1, 2),
+                                               (256, 3, 2), (128, 2, 2)])
 @pytest.mark.parametrize("M", [5, 130, 600])
-def test_resid_split(cuda_dev, bn, splits, M):
+def test_resid_split(cuda_dev, bn, splits, variant, M):
     K, N = 1024, 512
     a, b = _mk((M, K), 4, cuda_dev), _mk((N, K), 5, cuda_dev)
     h0 = torch.randn((M, N), generator=torch.Generator().manual_seed(6)).to(cuda_dev)
     h = h0.clone()
-    rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=bn, splits=splits)
+    rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=bn, splits=splits, variant=variant)
     torch.cuda.synchronize()
     _close(h - h0, _ref(a, b), K, False)
     rt.device_check()
 
 
-@pytest.mark.parametrize("bn", [64, 128, 256, -128, -256])
+@pytest.mark.parametrize("bn,variant", [(64, 0), (128, 0), (256, 0), (128, 1), (256, 1),
+                                        (128, 2), (256, 2)])
 @pytest.mark.parametrize("M", [3, 129, 300])
-def test_swiglu(cuda_dev, bn, M):
+def test_swiglu(cuda_dev, bn, variant, M):
     K, F = 256, 384
-    if F % (abs(bn) // 2):
+    if F % (bn // 2):
         pytest.skip("F must split into bn/2 halves")
     a = _mk((M, K), 7, cuda_dev)
     wg, wu = _mk((F, K), 8, cuda_dev) * 0.1, _mk((F, K), 9, cuda_dev) * 0.1
     out = torch.zeros((M, F), device=cuda_dev, dtype=torch.bfloat16)
-    rt.gemm_bf16(A.GEMM_SWIGLU, a, wg, out, b2=wu, bn=bn, splits=1)
+    rt.gemm_bf16(A.GEMM_SWIGLU, a, wg, out, b2=wu, bn=bn, splits=1, variant=variant)
     torch.cuda.synchronize()
     g, u = _ref(a, wg), _ref(a, wu)
     ref = g / (1 + torch.exp(-g)) * u
@@ -86,6 +92,10 @@ def test_accum_split(cuda_dev, swiglu):
     ws = torch.zeros((M, N), device=cuda_dev)
     rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=4)
     torch.cuda.synchronize()
+    _close(ws, torch.cat([_ref(a, b), _ref(a, b2)], dim=1) if swiglu else _ref(a, b), K, False)
+    ws.zero_()
+    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=4, variant=2)
+    torch.cuda.synchronize()
     ref = torch.cat([_ref(a, b), _ref(a, b2)], dim=1) if swiglu else _ref(a, b)
     _close(ws, ref, K, False)
     rt.device_check()
@@ -97,6 +107,10 @@ def test_large_k_full_shape_tile(cuda_dev):
     a, b = _mk((M, K), 13, cuda_dev) * 0.05, _mk((N, K), 14, cuda_dev) * 0.05
     h = torch.zeros((M, N), device=cuda_dev)
     rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=256, splits=1)
+    torch.cuda.synchronize()
+    _close(h, _ref(a, b), K, False)
+    h.zero_()
+    rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=256, splits=1, variant=2)
     torch.cuda.synchronize()
     _close(h, _ref(a, b), K, False)
     rt.device_check()

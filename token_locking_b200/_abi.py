@@ -94,7 +94,7 @@ SIGNATURES = {
     "sl_sampler_destroy": (None, [_P]),
     "sl_layer_forward": (_I, [_P, _P, _P, _I, _P, _P]),
     "sl_attention": (_I, [_P, _P, _P, _I, _P, _P, _P]),
-    "sl_gemm_bf16": (_I, [_I, _P, _I, _I, _P, _P, _I, _P, _I, _P, _I, _I, _P]),
+    "sl_gemm_bf16": (_I, [_I, _P, _I, _I, _P, _P, _I, _P, _I, _P, _I, _I, _I, _P]),
     "sl_model_autotune": (_I, [_P, _P, _I, _P]),
     "sl_model_tuning": (_I, [_P, _I, _I, C.POINTER(_I), C.POINTER(_I), C.POINTER(_I)]),
     "sl_timing_enable": (_I, [_P, _I]),

@@ -106,7 +106,7 @@ struct sl_model {
   std::vector<TimingRec> recs;
   sl_timing acc{};
   long long launch_base = 0;
-  // autotuned GEMM tilings: [kind][row-count bucket] = {bn, splits, msub} (bn 0 = untuned)
+  // autotuned GEMM tilings: [kind][row-count bucket] = {bn, splits, variant} (bn 0 = untuned)
   std::vector<std::array<int, 3>> tuned[5];
 };
 
@@ -530,6 +530,7 @@ namespace {
 struct Plan {
   int bn, splits, msub;
   double cost;
+  int pair = 0;     // 1: CTA-pair kernel (2-SM MMA)
 };
 
 // Choose the tile shape (BN, 128 or 256 rows per unit) and K split of one
@@ -574,6 +575,37 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
           if (split_kind == SPLIT_ACCUM) t += (double)M * N * 8.0 / bw_hbm + 3.0e-6;   // finalize
         }
         if (t < best.cost - 1e-9) best = Plan{bn, ss, msub, t};
+      }
+    }
+  }
+  // CTA pairs: 256 x BN tiles on two SMs, each SM staging 128 rows of A and
+  // BN/2 rows of B per K-block
+  if (M > 128) {
+    const int pairs = num_sms / 2;
+    const int mt = (M + 255) / 256;
+    const double rows_live = std::min(M, 256);
+    for (int bn : {256, 128}) {
+      if (N % bn || bn < min_bn) continue;
+      if (swiglu && (N / 2) % (bn / 2)) continue;
+      const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
+      for (int sp = 1; sp <= max_s; ++sp) {
+        const int kbp = (kblocks + sp - 1) / sp;
+        const int ss = (kblocks + kbp - 1) / kbp;
+        const long units = (long)mt * (N / bn) * ss;
+        const long waves = (units + pairs - 1) / pairs;
+        const double quant = (double)(waves * pairs) / units;
+        const double t_hbm = 2.0 * ((double)N * K + (double)M * K) / bw_hbm;
+        const double t_l2 = (double)units * kbp * (bn * 128.0 + rows_live * 128.0) / bw_l2;
+        const double t_mma = (double)units * kbp * 2.0 * 256 * bn * 64 / peak;
+        double t = std::max(t_hbm, std::max(t_l2, t_mma)) * std::min(quant, 2.0) + waves * 1.0e-6;
+        if (ss > 1) {
+          t += (double)M * N * 4.0 * ss / bw_l2;
+          if (split_kind == SPLIT_ACCUM) t += (double)M * N * 8.0 / bw_hbm + 3.0e-6;
+        }
+        if (t < best.cost - 1e-9) {
+          best = Plan{bn, ss, 2, t};
+          best.pair = 1;
+        }
       }
     }
   }
@@ -657,7 +689,9 @@ static Plan plan_kind(const sl_model *m, int kind, int M, int ns) {
   const int bkt = tune_bucket(M);
   if (bkt >= 0 && bkt < (int)m->tuned[kind].size() && m->tuned[kind][bkt][0] > 0) {
     const auto &t = m->tuned[kind][bkt];
-    return Plan{t[0], t[1], t[2], 0.0};
+    Plan pl{t[0], t[1], t[2] == 1 ? 2 : 1, 0.0};
+    pl.pair = t[2] == 2 ? 1 : 0;
+    return pl;
   }
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn;
@@ -729,14 +763,16 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
   g.bn = pl.bn;
   g.splits = pl.splits;
   g.msub = pl.msub;
+  g.pair = pl.pair;
+  const int bbox = pl.pair ? pl.bn / 2 : pl.bn;    // weight rows per TMA box
   double bytes = 0, flops = 0;
   switch (kind) {
     case G_QKV: {
       const auto &mp = m->maps[l];
       g.A = &c->map_a;
-      g.B[0] = mp[W_Q].box(pl.bn);
-      g.B[1] = mp[W_K].box(pl.bn);
-      g.B[2] = mp[W_V].box(pl.bn);
+      g.B[0] = mp[W_Q].box(bbox);
+      g.B[1] = mp[W_K].box(bbox);
+      g.B[2] = mp[W_V].box(bbox);
       g.n_seg[0] = g.n_seg[1] = g.n_seg[2] = d;
       g.N = 3 * d;
       g.K = d;
@@ -763,7 +799,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       const auto &mp = m->maps[l];
       const int K = kind == G_O ? d : f;
       g.A = kind == G_O ? &c->map_o : &c->map_act;
-      g.B[0] = mp[kind == G_O ? W_O : W_D].box(pl.bn);
+      g.B[0] = mp[kind == G_O ? W_O : W_D].box(bbox);
       g.n_seg[0] = d;
       g.N = d;
       g.K = K;
@@ -791,7 +827,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
     }
     default: {   // G_HD
       g.A = &c->map_a;
-      g.B[0] = m->head_map.box(pl.bn);
+      g.B[0] = m->head_map.box(bbox);
       g.n_seg[0] = V;
       g.N = V;
       g.K = d;
@@ -928,7 +964,8 @@ extern "C" sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int
 
 extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b,
                                   const void *d_b2, int N, void *d_out, int ldo,
-                                  const int32_t *d_row_map, int bn, int splits, void *stream) {
+                                  const int32_t *d_row_map, int bn, int splits, int variant,
+                                  void *stream) {
   if (!d_a || !d_b || !d_out) return fail(SL_ERR_INVALID, "sl_gemm_bf16: null argument");
   if (epi < SL_GEMM_STORE || epi > SL_GEMM_ACCUM) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bad epi");
   if (M < 0 || K <= 0 || N <= 0 || K % 64 != 0)
@@ -940,25 +977,26 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: pointers must be 16-byte aligned");
   if (M == 0) return SL_OK;
   const int ns = sm_count();
-  int msub = 1;
-  if (bn < 0) {
-    msub = 2;
-    bn = -bn;
-  }
+  if (variant < 0 || variant > 2) return fail(SL_ERR_INVALID, "sl_gemm_bf16: variant must be 0, 1 or 2");
+  int msub = variant == 0 ? 1 : 2;
+  int pair = variant == 2 ? 1 : 0;
   if (bn == 0) {
     Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID ? SPLIT_RESID
                                 : epi == SL_GEMM_ACCUM ? SPLIT_ACCUM : SPLIT_NONE, ns, swiglu);
     bn = p.bn;
     msub = p.msub;
+    pair = p.pair;
     if (splits <= 0) splits = p.splits;
   }
+  if (pair && bn != 128 && bn != 256)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: the CTA-pair kernel needs bn 128 or 256");
   if (bn != 64 && bn != 128 && bn != 256) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bn must be 64/128/256");
   if (N % bn || (swiglu && (N / 2) % (bn / 2)))
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: N must be a multiple of bn");
   if (splits < 1) splits = 1;
   const int epi_k = epi == SL_GEMM_STORE ? EPI_STORE : epi == SL_GEMM_RESID ? EPI_RESID
                     : epi == SL_GEMM_SWIGLU ? EPI_SWIGLU : EPI_ACCUM;
-  const int brows = swiglu ? bn / 2 : bn;
+  const int brows = (swiglu || pair) ? bn / 2 : bn;
   TmaMat ma, mb, mb2;
   if (!tma_encode(&ma, d_a, M, K, 128) || !tma_encode(&mb, d_b, swiglu ? N / 2 : N, K, brows) ||
       (swiglu && !tma_encode(&mb2, d_b2, N / 2, K, brows)))
@@ -979,6 +1017,7 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   g.ldo = ldo;
   g.row_map = d_row_map;
   g.msub = msub;
+  g.pair = pair;
   int *err = device_error_word();
   if (!err) return fail(SL_ERR_CUDA, "sl_gemm_bf16: no device error word");
   cudaError_t e = launch_gemm_tc(g, ns, err, (cudaStream_t)stream);
@@ -1040,10 +1079,12 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
       const int N = Ns[kind], K = Ks[kind], kblocks = K / 64;
       double best_ms = 1e30;
       std::array<int, 3> best = {0, 1, 1};
-      for (int msub = 1; msub <= 2; ++msub) {
-        if (msub == 2 && Mb <= 128) continue;
+      for (int variant = 0; variant <= 2; ++variant) {
+        const int msub = variant == 0 ? 1 : 2;
+        if (variant > 0 && Mb <= 128) continue;
         for (int bn : {256, 128, 64}) {
           if (N % bn || (kind == G_QKV && bn < 128)) continue;
+          if (variant == 2 && bn < 128) continue;
           if (kind == G_GU && (N / 2) % (bn / 2)) continue;
           int last_ss = 0;
           for (int sp : split_opts) {
@@ -1055,7 +1096,8 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
             last_ss = ss;
             const long units = (long)((Mb + 128 * msub - 1) / (128 * msub)) * (N / bn) * ss;
             if (units > 24L * m->num_sms) continue;
-            const Plan pl{bn, ss, msub, 0.0};
+            Plan pl{bn, ss, msub, 0.0};
+            pl.pair = variant == 2 ? 1 : 0;
             // each repetition is followed by a small kernel (an RMSNorm, as in
             // the layer) so that successive GEMMs cannot overlap each other
             // through programmatic launch and flatter tilings with few CTAs
@@ -1079,7 +1121,7 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
             cudaEventElapsedTime(&ms, e0, e1);
             if (ms < best_ms) {
               best_ms = ms;
-              best = {bn, ss, msub};
+              best = {bn, ss, variant};
             }
           }
           if (st != SL_OK) break;
@@ -1098,13 +1140,13 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
 }
 
 extern "C" sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits,
-                                     int *msub) {
-  if (!m || !bn || !splits || !msub || kind < 0 || kind >= G_KINDS || M <= 0)
+                                     int *variant) {
+  if (!m || !bn || !splits || !variant || kind < 0 || kind >= G_KINDS || M <= 0)
     return fail(SL_ERR_INVALID, "sl_model_tuning: bad argument");
   const Plan p = plan_kind(m, kind, M, m->num_sms);
   *bn = p.bn;
   *splits = p.splits;
-  *msub = p.msub;
+  *variant = p.pair ? 2 : (p.msub == 2 ? 1 : 0);
   return SL_OK;
 }
 

@@ -257,6 +257,7 @@ __global__ void attn_combine_kernel(const float *__restrict__ ws_o, const float 
   const int lane = threadIdx.x & 31;
   if (w >= M * n_heads) return;
   pdl_wait();
+  pdl_trigger();
   const int j = w / n_heads, h = w % n_heads;
   float m[ATTN_MAX_SPLITS], l[ATTN_MAX_SPLITS];
   float mx = -INFINITY;
@@ -283,7 +284,6 @@ __global__ void attn_combine_kernel(const float *__restrict__ ws_o, const float 
       acc.x += v.x * c; acc.y += v.y * c; acc.z += v.z * c; acc.w += v.w * c;
     }
   }
-  pdl_trigger();
   const float inv = L > 0.f ? 1.f / L : 0.f;
   bf16 *dst = o + (size_t)j * n_heads * AT_D + h * AT_D + lane * 4;
   *reinterpret_cast<uint2 *>(dst) =

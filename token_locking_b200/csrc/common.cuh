@@ -48,10 +48,12 @@ __device__ __forceinline__ unsigned long long global_ns() {
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
 
 // Programmatic dependent launch: every kernel of the step is launched with
-// programmatic stream serialisation, waits for its predecessor's results with
-// pdl_wait() before touching memory the predecessor writes (or reads), and
-// calls pdl_trigger() once its own main work is issued so the next kernel's
-// launch and prologue overlap this kernel's tail.
+// programmatic stream serialisation and waits for its predecessor's results
+// with pdl_wait() before touching memory the predecessor writes (or reads).
+// Light kernels (norms, finalize passes, merges) call pdl_trigger() right
+// after that wait, so the next GEMM's CTAs become resident beside them and
+// stream their weight tiles meanwhile; heavy kernels trigger once their main
+// work is issued.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

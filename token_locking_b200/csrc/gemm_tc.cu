@@ -138,6 +138,59 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// --- CTA-pair (cluster of 2) helpers for the 2-SM MMA variant
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(saddr), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on the
+// pair leader's barrier (cluster address); no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                                 uint32_t leader_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(leader_bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this offset in both CTAs of the pair once the
+// issued MMAs complete
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar), "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 64 bf16 (128 B), 8-row groups 1024 B apart.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
@@ -150,13 +203,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   return d;
 }
 
-template <int BN>
+template <int BN, int MMA_M = 128>
 __device__ __forceinline__ constexpr uint32_t idesc_bf16_f32() {
   return (1u << 4)            // D: fp32
          | (1u << 7)          // A: bf16
          | (1u << 10)         // B: bf16
          | ((uint32_t)(BN >> 3) << 17)
-         | ((uint32_t)(128 >> 4) << 24);
+         | ((uint32_t)(MMA_M >> 4) << 24);
 }
 
 // ---------------------------------------------------------------- kernel ---
@@ -215,6 +268,130 @@ __device__ __forceinline__ void load_b(const TcParams &p, uint32_t sb, int nt, i
     if (c0 < p.seg0) tma_load_2d(sb, &p.b[0], kb * 64, c0, bar);
     else if (c0 < p.seg1) tma_load_2d(sb, &p.b[1], kb * 64, c0 - p.seg0, bar);
     else tma_load_2d(sb, &p.b[2], kb * 64, c0 - p.seg1, bar);
+  }
+}
+
+// Epilogue of one 128-row accumulator tile: TMEM lane quarter of the calling
+// warp (taddr carries the lane offset) for A row r, output tile nt.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile(const TcParams &p, uint32_t taddr, int r, int nt) {
+  const bool live = r < p.M;
+  float v[32];
+  if (EPI == EPI_ACCUM) {
+    // split-K partial sum of this tile: fp32 atomics into the workspace
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      tmem_ld32(taddr + c, v);
+      if (!live) continue;
+      int col;
+      if (p.b_swiglu) {   // gate into [0, F), up into [F, 2F)
+        const int half = BN / 2;
+        const int f0 = nt * half;
+        col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
+      } else {
+        col = nt * BN + c;
+      }
+      float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + col;
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        atomicAdd(reinterpret_cast<float4 *>(dst + i),
+                  make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+    }
+  } else if (EPI == EPI_SWIGLU) {
+    const int f0 = nt * (BN / 2);
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 32) {
+      float g[32];
+      tmem_ld32(taddr + c, g);
+      tmem_ld32(taddr + BN / 2 + c, v);
+      if (live) {
+        bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)r * p.ldo + f0 + c;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          Pack8 pk;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(silu_f(g[i + e]) * v[i + e]);
+          *reinterpret_cast<uint4 *>(dst + i) = pk.u;
+        }
+      }
+    }
+  } else if (EPI == EPI_QKV) {
+    // whole heads per tile: pair (i, i + 64) of a head is rotated together
+    const int col0 = nt * BN;
+    const int seg = col0 / p.dmodel;              // 0 q, 1 k, 2 v
+    const int pos_flat = live ? p.row_map[r] : 0;
+    const int pos = pos_flat % p.n_ctx;
+#pragma unroll 1
+    for (int hd = 0; hd < BN / 128; ++hd) {
+      const int cbase = col0 - seg * p.dmodel + hd * 128;   // column of the head in its segment
+#pragma unroll 1
+      for (int j = 0; j < 2; ++j) {
+        float x2[32];
+        tmem_ld32(taddr + hd * 128 + 32 * j, v);
+        tmem_ld32(taddr + hd * 128 + 64 + 32 * j, x2);
+        if (!live) continue;
+        bf16 *dst;
+        if (seg == 0) dst = p.q_out + (size_t)r * p.dmodel + cbase;
+        else if (seg == 1) dst = p.ck + (size_t)pos_flat * p.dmodel + cbase;
+        else dst = p.cv + (size_t)pos_flat * p.dmodel + cbase;
+        if (seg < 2) {
+          const float4 *tab =
+              reinterpret_cast<const float4 *>(p.rope + (size_t)pos * 64 + 32 * j);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float4 cs = __ldg(tab + (e >> 1));   // (cos, sin) of e and e+1
+            const float a0 = v[e], b0 = x2[e], a1 = v[e + 1], b1 = x2[e + 1];
+            v[e] = a0 * cs.x - b0 * cs.y;
+            x2[e] = b0 * cs.x + a0 * cs.y;
+            v[e + 1] = a1 * cs.z - b1 * cs.w;
+            x2[e + 1] = b1 * cs.z + a1 * cs.w;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          Pack8 lo, hi;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            lo.h[e] = __float2bfloat16_rn(v[i + e]);
+            hi.h[e] = __float2bfloat16_rn(x2[i + e]);
+          }
+          *reinterpret_cast<uint4 *>(dst + 32 * j + i) = lo.u;
+          *reinterpret_cast<uint4 *>(dst + 64 + 32 * j + i) = hi.u;
+        }
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      tmem_ld32(taddr + c, v);
+      if (!live) continue;
+      if (EPI == EPI_STORE) {
+        const int orow = p.row_map ? p.row_map[r] : r;
+        bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)orow * p.ldo + nt * BN + c;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          Pack8 pk;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(v[i + e]);
+          *reinterpret_cast<uint4 *>(dst + i) = pk.u;
+        }
+      } else {   // EPI_RESID: h += partial (atomic when K is split)
+        float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + nt * BN + c;
+        if (p.splits == 1) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float4 o = *reinterpret_cast<float4 *>(dst + i);
+            o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
+            *reinterpret_cast<float4 *>(dst + i) = o;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            atomicAdd(reinterpret_cast<float4 *>(dst + i),
+                      make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+        }
+      }
+    }
   }
 }
 
@@ -395,126 +572,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
 #pragma unroll 1
       for (int sub = 0; sub < MSUB; ++sub) {
       const int r = (mt * MSUB + sub) * 128 + q * 32 + lane;
-      const bool live = r < p.M;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * ACC_COLS + sub * BN) +
                              ((uint32_t)(q * 32) << 16);
-      float v[32];
-      if (EPI == EPI_ACCUM) {
-        // split-K partial sum of this tile: fp32 atomics into the workspace
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          tmem_ld32(taddr + c, v);
-          if (!live) continue;
-          int col;
-          if (p.b_swiglu) {   // gate into [0, F), up into [F, 2F)
-            const int half = BN / 2;
-            const int f0 = nt * half;
-            col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
-          } else {
-            col = nt * BN + c;
-          }
-          float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + col;
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            atomicAdd(reinterpret_cast<float4 *>(dst + i),
-                      make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
-        }
-      } else if (EPI == EPI_SWIGLU) {
-        const int f0 = nt * (BN / 2);
-#pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
-          float g[32];
-          tmem_ld32(taddr + c, g);
-          tmem_ld32(taddr + BN / 2 + c, v);
-          if (live) {
-            bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)r * p.ldo + f0 + c;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              Pack8 pk;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(silu_f(g[i + e]) * v[i + e]);
-              *reinterpret_cast<uint4 *>(dst + i) = pk.u;
-            }
-          }
-        }
-      } else if (EPI == EPI_QKV) {
-        // whole heads per tile: pair (i, i + 64) of a head is rotated together
-        const int col0 = nt * BN;
-        const int seg = col0 / p.dmodel;              // 0 q, 1 k, 2 v
-        const int pos_flat = live ? p.row_map[r] : 0;
-        const int pos = pos_flat % p.n_ctx;
-#pragma unroll 1
-        for (int hd = 0; hd < BN / 128; ++hd) {
-          const int cbase = col0 - seg * p.dmodel + hd * 128;   // column of the head in its segment
-#pragma unroll 1
-          for (int j = 0; j < 2; ++j) {
-            float x2[32];
-            tmem_ld32(taddr + hd * 128 + 32 * j, v);
-            tmem_ld32(taddr + hd * 128 + 64 + 32 * j, x2);
-            if (!live) continue;
-            bf16 *dst;
-            if (seg == 0) dst = p.q_out + (size_t)r * p.dmodel + cbase;
-            else if (seg == 1) dst = p.ck + (size_t)pos_flat * p.dmodel + cbase;
-            else dst = p.cv + (size_t)pos_flat * p.dmodel + cbase;
-            if (seg < 2) {
-              const float4 *tab =
-                  reinterpret_cast<const float4 *>(p.rope + (size_t)pos * 64 + 32 * j);
-#pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                const float4 cs = __ldg(tab + (e >> 1));   // (cos, sin) of e and e+1
-                const float a0 = v[e], b0 = x2[e], a1 = v[e + 1], b1 = x2[e + 1];
-                v[e] = a0 * cs.x - b0 * cs.y;
-                x2[e] = b0 * cs.x + a0 * cs.y;
-                v[e + 1] = a1 * cs.z - b1 * cs.w;
-                x2[e + 1] = b1 * cs.z + a1 * cs.w;
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              Pack8 lo, hi;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                lo.h[e] = __float2bfloat16_rn(v[i + e]);
-                hi.h[e] = __float2bfloat16_rn(x2[i + e]);
-              }
-              *reinterpret_cast<uint4 *>(dst + 32 * j + i) = lo.u;
-              *reinterpret_cast<uint4 *>(dst + 64 + 32 * j + i) = hi.u;
-            }
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          tmem_ld32(taddr + c, v);
-          if (!live) continue;
-          if (EPI == EPI_STORE) {
-            const int orow = p.row_map ? p.row_map[r] : r;
-            bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)orow * p.ldo + nt * BN + c;
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              Pack8 pk;
-#pragma unroll
-              for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(v[i + e]);
-              *reinterpret_cast<uint4 *>(dst + i) = pk.u;
-            }
-          } else {   // EPI_RESID: h += partial (atomic when K is split)
-            float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + nt * BN + c;
-            if (p.splits == 1) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                float4 o = *reinterpret_cast<float4 *>(dst + i);
-                o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
-                *reinterpret_cast<float4 *>(dst + i) = o;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                atomicAdd(reinterpret_cast<float4 *>(dst + i),
-                          make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
-            }
-          }
-        }
-      }
+      epilogue_tile<BN, EPI>(p, taddr, r, nt);
       }   // sub
       tc_fence_before();
       __syncwarp();
@@ -539,6 +599,201 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   }
 }
 
+// ------------------------------------------------------ CTA-pair kernel ---
+// The same GEMM with 2-SM tensor-core instructions: a cluster of two CTAs
+// computes a 256 x BN tile; each CTA stages its own 128 rows of A and its half
+// (BN/2 rows) of the weight tile, the pair leader issues tcgen05.mma.cta_group::2
+// (M = 256) over both CTAs' shared memory, and each CTA's TMEM holds the
+// accumulator of its 128 rows.  Per SM this halves the weight-tile traffic
+// from L2 and the shared-memory operand reads of the 1-SM kernel.
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant__ TcParams p) {
+  constexpr int A_BYTES = 128 * 64 * 2;
+  constexpr int B_BYTES = (BN / 2) * 64 * 2;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s_addr(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + BAR_OFF);
+  const uint32_t bar0 = s_addr(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + BAR_OFF + 8 * (2 * STAGES + 5));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 8);     // 4 epilogue warps in each CTA
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&p.a);
+    tma_prefetch_desc(&p.b[0]);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     s_addr(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      auto load_b_half = [&](uint32_t sb, int nt, int kb, uint32_t bar) {
+        if (p.b_swiglu) {
+          tma_load_2d_pair(sb, &p.b[rank], kb * 64, nt * (BN / 2), bar);
+        } else {
+          const int c0 = nt * BN + (int)rank * (BN / 2);
+          if (c0 < p.seg0) tma_load_2d_pair(sb, &p.b[0], kb * 64, c0, bar);
+          else if (c0 < p.seg1) tma_load_2d_pair(sb, &p.b[1], kb * 64, c0 - p.seg0, bar);
+          else tma_load_2d_pair(sb, &p.b[2], kb * 64, c0 - p.seg1, bar);
+        }
+      };
+      int npre = 0;
+      if (pair < p.units) {
+        int mt, nt, sp;
+        decode_unit(p, pair, mt, nt, sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        npre = min(STAGES, kb1 - kb0);
+        for (int i = 0; i < npre; ++i) {
+          if (leader) mbar_expect_tx(full_bar(i), 2 * STAGE_BYTES);
+          load_b_half(sbase + i * STAGE_BYTES + A_BYTES, nt, kb0 + i, map_to_rank(full_bar(i), 0));
+        }
+      }
+      pdl_wait();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, first = true;
+      for (int u = pair; u < p.units && ok; u += n_pairs) {
+        int mt, nt, sp;
+        decode_unit(p, u, mt, nt, sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const bool pre = first && (kb - kb0) < npre;
+          if (!pre) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+            if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+          }
+          const uint32_t sa = sbase + stage * STAGE_BYTES;
+          const uint32_t lbar = map_to_rank(full_bar(stage), 0);
+          tma_load_2d_pair(sa, &p.a, kb * 64, mt * 256 + (int)rank * 128, lbar);
+          if (!pre) load_b_half(sa + A_BYTES, nt, kb, lbar);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        first = false;
+      }
+      pdl_trigger();
+      if (!ok) {
+        atomicExch(p.err, DEV_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA (pair leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32<BN, 256>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int u = pair; u < p.units && ok; u += n_pairs) {
+        int mt, nt, sp;
+        decode_unit(p, u, mt, nt, sp);
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * STAGE_BYTES;
+          const uint64_t adesc = smem_desc_sw128(sa);
+          const uint64_t bdesc = smem_desc_sw128(sa + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          tc_commit_pair_both(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(tfull_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.err, DEV_TIMEOUT_MMA);
+        *abort_flag = 1;
+      }
+      tc_commit_pair(drain_bar);
+      volatile int never = 0;
+      mbar_wait(drain_bar, 0, &never);
+    }
+  } else {
+    // ------------------------------------------------- epilogue (both CTAs)
+    pdl_wait();
+    const int q = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int u = pair; u < p.units; u += n_pairs) {
+      int mt, nt, sp;
+      decode_unit(p, u, mt, nt, sp);
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const int r = mt * 256 + (int)rank * 128 + q * 32 + lane;
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      epilogue_tile<BN, EPI>(p, taddr, r, nt);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (!ok && lane == 0) {
+      atomicExch(p.err, DEV_TIMEOUT_EPI);
+      *abort_flag = 1;
+    }
+  }
+
+  // neither CTA leaves while the pair's MMAs may still read its shared memory
+  // or its epilogue may still signal the leader
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ host ---
 template <int BN, int STAGES, int EPI, int MSUB>
 static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
@@ -553,6 +808,49 @@ static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
   }
   err = launch_k(gemm_tc_kernel<BN, STAGES, EPI, MSUB>, grid, 192, L::TOTAL, s, p);
   return err;
+}
+
+// `pairs` CTA pairs, capped at the number of pairs the GPU holds at once
+// (a GPC with an odd number of usable SMs leaves one SM out of the pairing).
+template <int BN, int STAGES, int EPI>
+static cudaError_t run_tc2(const TcParams &p, int pairs, cudaStream_t s) {
+  constexpr int SMEM = STAGES * (16384 + (BN / 2) * 128) + 256 + 1024;
+  static int max_pairs = 0;
+  if (max_pairs == 0) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = SMEM;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = 2;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, STAGES, EPI>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n <= 0) return cudaErrorInvalidConfiguration;
+    max_pairs = n;
+  }
+  if (pairs > max_pairs) pairs = max_pairs;
+  return launch_k_cluster2(gemm_tc2_kernel<BN, STAGES, EPI>, 2 * pairs, 192, SMEM, s, p);
+}
+
+template <int BN, int STAGES>
+static cudaError_t run_epi2(int epi, const TcParams &p, int pairs, cudaStream_t s) {
+  switch (epi) {
+    case EPI_STORE: return run_tc2<BN, STAGES, EPI_STORE>(p, pairs, s);
+    case EPI_RESID: return run_tc2<BN, STAGES, EPI_RESID>(p, pairs, s);
+    case EPI_SWIGLU: return run_tc2<BN, STAGES, EPI_SWIGLU>(p, pairs, s);
+    case EPI_ACCUM: return run_tc2<BN, STAGES, EPI_ACCUM>(p, pairs, s);
+    case EPI_QKV: return run_tc2<BN, STAGES, EPI_QKV>(p, pairs, s);
+  }
+  return cudaErrorInvalidValue;
 }
 
 template <int BN, int STAGES, int MSUB>
@@ -587,7 +885,9 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
-  const int msub = a.msub == 2 ? 2 : 1;
+  const bool pair_mma = a.pair != 0;
+  if (pair_mma && bn != 128 && bn != 256) return cudaErrorInvalidValue;
+  const int msub = (a.msub == 2 || pair_mma) ? 2 : 1;   // a pair owns 256 rows
   p.m_tiles = (a.M + 128 * msub - 1) / (128 * msub);
   p.n_tiles = a.N / bn;
   p.kblocks = a.K / 64;
@@ -611,6 +911,11 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.q_out = (bf16 *)a.q_out;
   p.ck = (bf16 *)a.ck;
   p.cv = (bf16 *)a.cv;
+  if (pair_mma) {
+    const int pairs = p.units < num_sms / 2 ? p.units : num_sms / 2;
+    if (bn == 256) return run_epi2<256, 6>(a.epi, p, pairs, s);
+    return run_epi2<128, 6>(a.epi, p, pairs, s);
+  }
   int grid = p.units < num_sms ? p.units : num_sms;
   if (msub == 2) {
     switch (bn) {

@@ -42,6 +42,28 @@ inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The same with a cluster of 2 CTAs along x (CTA pairs for 2-SM MMAs).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k_cluster2(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                     cudaStream_t s, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ----------------------------------------------------- epilogue selection --
 enum GemmEpi : int {
   EPI_STORE = 0,      // out[row_map ? row_map[r] : r][col_off + c] = acc   (dtype)
@@ -107,6 +129,7 @@ struct TcGemmArgs {
   int bn;                // 64, 128 or 256
   int b_swiglu;          // B tile = BN/2 gate rows (B[0]) | BN/2 up rows (B[1])
   int msub;              // 1: 128-row units; 2: 256-row units (two accumulators per B tile)
+  int pair;              // 1: CTA-pair kernel (2-SM MMA, 256-row units, B maps with BN/2 boxes)
   void *out;             // STORE/SWIGLU: dtype out; RESID: fp32 resid; ACCUM: fp32 ws
   int ldo;               // leading dimension of out (elements)
   const int32_t *row_map;// STORE: output row index per A row (or null); QKV: flat positions

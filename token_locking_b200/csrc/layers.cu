@@ -19,10 +19,10 @@ __global__ void gather_embed_kernel(const int32_t *__restrict__ tokens,
   int j = blockIdx.x;
   if (j >= M) return;
   pdl_wait();
+  pdl_trigger();
   const T *e = emb + (size_t)tokens[rows[j]] * d;
   float *o = h + (size_t)j * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = to_f(e[c]);
-  pdl_trigger();
 }
 
 cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
@@ -45,6 +45,7 @@ __global__ void rmsnorm_kernel(const float *__restrict__ h, const T *__restrict_
   int j = blockIdx.x;
   if (j >= M) return;
   pdl_wait();
+  pdl_trigger();
   const float *x = h + (size_t)j * d;
   float ss = 0.f;
   for (int c = threadIdx.x; c < d; c += blockDim.x) ss += x[c] * x[c];
@@ -61,7 +62,6 @@ __global__ void rmsnorm_kernel(const float *__restrict__ h, const T *__restrict_
   float r = rsqrtf(red[0] / (float)d + eps);
   T *o = out + (size_t)j * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = from_f<T>(x[c] * r * to_f(g[c]));
-  pdl_trigger();
 }
 
 // bf16 output: one CTA of 256 threads per row, the row held in registers as
@@ -75,6 +75,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float *__restri
   const int j = blockIdx.x;
   if (j >= M) return;
   pdl_wait();
+  pdl_trigger();
   const float4 *x = reinterpret_cast<const float4 *>(h + (size_t)j * d);
   const int n4 = d >> 2;
   float4 v[VPT];
@@ -107,7 +108,6 @@ __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float *__restri
       o2[i] = oo.u;
     }
   }
-  pdl_trigger();
 }
 
 cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
@@ -155,6 +155,7 @@ __global__ void __launch_bounds__(256) rope_scatter_kernel(
   const int per_seg = d >> 1;
   const int pr_all = blockIdx.x * 256 + threadIdx.x;
   pdl_wait();
+  pdl_trigger();
   if (pr_all < 3 * per_seg) {
     const int seg = pr_all / per_seg;
     const int pr = pr_all - seg * per_seg;
@@ -177,7 +178,6 @@ __global__ void __launch_bounds__(256) rope_scatter_kernel(
       dst[c1] = from_f<T>(x1);
     }
   }
-  pdl_trigger();
 }
 
 cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool zero_in, int M,
@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(256) swiglu_kernel(Tin *__restrict__ ws, bool 
                                                      int F, T *__restrict__ act) {
   const int j = blockIdx.y;
   pdl_wait();
+  pdl_trigger();
   Tin *g = ws + (size_t)j * 2 * F;
   T *o = act + (size_t)j * F;
 #pragma unroll
@@ -222,7 +223,6 @@ __global__ void __launch_bounds__(256) swiglu_kernel(Tin *__restrict__ ws, bool 
       o[c] = from_f<T>(silu_f(gv) * uv);
     }
   }
-  pdl_trigger();
 }
 
 cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, int M, int F,

@@ -218,10 +218,11 @@ def bench_gemm(args, dev):
             outb = torch.zeros((M, N), device=dev, dtype=torch.bfloat16)
             outf = torch.zeros((M, N), device=dev, dtype=torch.float32)
             outa = torch.zeros((M, f), device=dev, dtype=torch.bfloat16)
-            for bn in (256, 128, 64, -256, -128, -64):
-                if abs(bn) < 128 and name == "qkv":
+            for bn, variant in ((256, 0), (128, 0), (64, 0), (256, 1), (128, 1), (64, 1), (256, 2),
+                                (128, 2)):
+                if bn < 128 and name == "qkv":
                     continue
-                if (bn < 0 and M <= 128) or N % abs(bn):
+                if (variant > 0 and M <= 128) or N % bn:
                     continue
                 for sp in (1, 2, 3, 4, 6, 8, 9, 12, 16):
                     if sp > 1 and name == "head":
@@ -236,13 +237,13 @@ def bench_gemm(args, dev):
                                            else (A.GEMM_ACCUM, weights[name], None, outf))
 
                     def fn():
-                        rt.gemm_bf16(epi, a, b, out, b2=b2, bn=bn, splits=sp)
+                        rt.gemm_bf16(epi, a, b, out, b2=b2, bn=bn, splits=sp, variant=variant)
 
                     ms = _time(fn, args.iters, 2, flush)
                     by = 2.0 * (N * K + M * K + M * N)
                     fl = 2.0 * M * N * K
-                    print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": abs(bn),
-                                      "msub": 2 if bn < 0 else 1, "splits": sp,
+                    print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": bn,
+                                      "variant": variant, "splits": sp,
                                       "us": round(ms * 1e3, 2),
                                       "GBps": round(by / ms / 1e6, 1),
                                       "TFLOPs": round(fl / ms / 1e9, 1)}), flush=True)
@@ -258,7 +259,7 @@ def bench_gemm(args, dev):
                 rt.gemm_bf16(epi, a, b, out, b2=b2, bn=0, splits=0)
 
             ms = _time(fn, args.iters, 2, flush)
-            print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": 0, "msub": 0,
+            print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": 0, "variant": -1,
                               "splits": 0, "us": round(ms * 1e3, 2),
                               "GBps": round(2.0 * (N * K + M * K + M * N) / ms / 1e6, 1)}),
                   flush=True)

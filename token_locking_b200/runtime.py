@@ -102,10 +102,11 @@ class Model:
                 "sl_model_autotune")
 
     def tuning(self, kind: int, M: int):
-        bn, sp, ms = C.c_int(), C.c_int(), C.c_int()
+        """(bn, splits, variant) of GEMM `kind` at M rows."""
+        bn, sp, var = C.c_int(), C.c_int(), C.c_int()
         A.check(A.lib().sl_model_tuning(self.handle, kind, M, C.byref(bn), C.byref(sp),
-                                        C.byref(ms)), "sl_model_tuning")
-        return bn.value, sp.value, ms.value
+                                        C.byref(var)), "sl_model_tuning")
+        return bn.value, sp.value, var.value
 
     def timing_enable(self, on: bool = True):
         A.check(A.lib().sl_timing_enable(self.handle, 1 if on else 0), "sl_timing_enable")
@@ -241,13 +242,14 @@ def attention(model: Model, cache: KVCache, active: Active, layer: int, q: torch
 
 
 def gemm_bf16(epi: int, a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, b2=None, ldo=None,
-              row_map=None, bn: int = 0, splits: int = 0, stream=None):
+              row_map=None, bn: int = 0, splits: int = 0, variant: int = 0, stream=None):
     """out (op)= a @ b.T on the tensor cores (see sl_gemm_bf16)."""
     M, K = a.shape
     N = b.shape[0] * (2 if b2 is not None else 1)
     ldo = out.shape[-1] if ldo is None else ldo
     A.check(A.lib().sl_gemm_bf16(epi, _ptr(a), M, K, _ptr(b), _ptr(b2), N, _ptr(out), ldo,
-                                 _ptr(row_map), bn, splits, _stream(stream)), "sl_gemm_bf16")
+                                 _ptr(row_map), bn, splits, variant, _stream(stream)),
+            "sl_gemm_bf16")
 
 
 def device_check(clear: bool = True):
