@@ -207,7 +207,9 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
  *                   out bf16 [M][ldo] = silu(A W_gate^T) * (A W_up^T)
  *   SL_GEMM_ACCUM : out fp32 [M][ldo] += C (atomic; with d_b2, gate/up halves
  *                   accumulate into columns [0,F) and [F,2F))
- * bn (64/128/256) and splits (>= 1, RESID/ACCUM only) pick the tiling; variant
+ * bn (64/128/256) and splits (>= 1, RESID/ACCUM only; -1 = stream-K: every SM
+ * or CTA pair takes an equal share of the tiles x 64-wide K-blocks and adds
+ * its partial tiles atomically) pick the tiling; variant
  * picks the kernel: 0 = one CTA per 128 x bn tile, 1 = one CTA per 256 x bn
  * tile (two accumulators share each weight tile), 2 = a CTA pair per 256 x bn
  * tile with 2-SM tensor-core instructions (bn 128 or 256).  bn = 0 lets the
@@ -252,8 +254,14 @@ sl_status sl_kl_stats_noalloc(const int32_t *d_rows, int M, int vocab, int mask_
  * A no-op for fp32 models. */
 sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows, void *stream);
 /* The tiling sl_step would use for GEMM `kind` (0 QKV, 1 output projection,
- * 2 gate/up, 3 down, 4 LM head) at M rows; *variant as for sl_gemm_bf16. */
+ * 2 gate/up, 3 down, 4 LM head) at M rows; *splits and *variant as for
+ * sl_gemm_bf16. */
 sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits, int *variant);
+/* Pin the tiling of GEMM `kind` for the row-count bucket that holds M (the
+ * buckets of sl_model_autotune); arguments as for sl_gemm_bf16.  Returns
+ * SL_ERR_INVALID for a tiling the GEMM cannot use (the LM head takes no K
+ * split).  bf16 models only. */
+sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits, int variant);
 
 /* ---------------------------------------------------------------- sampler --- */
 

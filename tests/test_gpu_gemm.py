@@ -51,7 +51,8 @@ def test_store_rowmap(cuda_dev, bn, variant, M):
 
 @pytest.mark.parametrize("bn,splits,variant", [(64, 1, 0), (128, 3, 0), (256, 2, 0), (128, 8, 0),
                                                (256, 3, 1), (128, 1, 1), (64, 2, 1), (256, 1, 2),
-                                               (256, 3, 2), (128, 2, 2)])
+                                               (256, 3, 2), (128, 2, 2), (256, -1, 0), (64, -1, 0),
+                                               (128, -1, 1), (256, -1, 2), (128, -1, 2)])
 @pytest.mark.parametrize("M", [5, 130, 600])
 def test_resid_split(cuda_dev, bn, splits, variant, M):
     K, N = 1024, 512
@@ -83,18 +84,15 @@ def test_swiglu(cuda_dev, bn, variant, M):
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
-def test_accum_split(cuda_dev, swiglu):
+@pytest.mark.parametrize("splits,variant", [(4, 0), (4, 2), (-1, 0), (-1, 1), (-1, 2)])
+def test_accum_split(cuda_dev, swiglu, splits, variant):
     M, K, F = 77, 768, 256
     a = _mk((M, K), 10, cuda_dev)
     b = _mk((F, K), 11, cuda_dev)
     b2 = _mk((F, K), 12, cuda_dev) if swiglu else None
     N = 2 * F if swiglu else F
     ws = torch.zeros((M, N), device=cuda_dev)
-    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=4)
-    torch.cuda.synchronize()
-    _close(ws, torch.cat([_ref(a, b), _ref(a, b2)], dim=1) if swiglu else _ref(a, b), K, False)
-    ws.zero_()
-    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=4, variant=2)
+    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=splits, variant=variant)
     torch.cuda.synchronize()
     ref = torch.cat([_ref(a, b), _ref(a, b2)], dim=1) if swiglu else _ref(a, b)
     _close(ws, ref, K, False)
@@ -114,3 +112,23 @@ def test_large_k_full_shape_tile(cuda_dev):
     torch.cuda.synchronize()
     _close(h, _ref(a, b), K, False)
     rt.device_check()
+
+
+@pytest.mark.parametrize("variant", [0, 2])
+def test_stream_k_many_tiles(cuda_dev, variant):
+    """Stream-K where worker shares cross several tile boundaries (more tiles
+    than SMs) and where a share is a few K-blocks of one tile."""
+    for M, K, N in ((700, 256, 2048), (200, 4096, 768)):
+        a, b = _mk((M, K), 15, cuda_dev) * 0.1, _mk((N, K), 16, cuda_dev) * 0.1
+        h = torch.zeros((M, N), device=cuda_dev)
+        rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=128, splits=-1, variant=variant)
+        torch.cuda.synchronize()
+        _close(h, _ref(a, b), K, False)
+    rt.device_check()
+
+
+def test_stream_k_rejected_for_store(cuda_dev):
+    a, b = _mk((8, 64), 1, cuda_dev), _mk((128, 64), 2, cuda_dev)
+    out = torch.zeros((8, 128), device=cuda_dev, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError):
+        rt.gemm_bf16(A.GEMM_STORE, a, b, out, bn=128, splits=-1)

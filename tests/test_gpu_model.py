@@ -143,7 +143,7 @@ def test_autotuned_step_matches_oracle(cuda_dev):
     for kind in range(5):
         for M in (1, 100, 257, 400):
             bn, sp, var = model.tuning(kind, M)
-            assert bn in (64, 128, 256) and sp >= 1 and var in (0, 1, 2)
+            assert bn in (64, 128, 256) and (sp >= 1 or sp == -1) and var in (0, 1, 2)
     act = rt.Active(B, n_ctx)
     tokens, positions, ck, cv = _state(shape, B, n_ctx, [160, 130], seed=11, dev=cuda_dev,
                                        dtype="bf16")
@@ -155,6 +155,43 @@ def test_autotuned_step_matches_oracle(cuda_dev):
     torch.cuda.synchronize()
     rt.device_check()
     zs, _, _ = _oracle_step(shape, w64, tokens, positions, ck, cv, n_ctx)
+    lg = to64(logits)
+    for b in range(B):
+        err = np.abs(lg[positions[b] + b * n_ctx] - zs[b]).max()
+        assert err <= LOGIT_TOL["bf16"], err
+    model.close()
+
+
+@pytest.mark.parametrize("tiling", [(256, -1, 2), (128, -1, 0), (256, -1, 1), (128, 3, 2)])
+def test_pinned_tilings_step_matches_oracle(cuda_dev, tiling):
+    """Every projection GEMM pinned to one tiling (stream-K or split K, CTA
+    pairs or single CTAs; the LM head keeps its own), through the workspace
+    and finalize kernels of the split paths."""
+    shape = MINI_BF16
+    B, n_ctx = 2, 200
+    w_np = wl.np_weights(shape, seed=1, std=0.05, gain_jitter=0.1)
+    w_dev = weights_to_device(w_np, "bf16", cuda_dev)
+    w64 = weights_for_oracle(w_dev)
+    model = rt.Model(shape, w_dev, "bf16")
+    cache = rt.KVCache(model, B, n_ctx)
+    counts = [170, 123]
+    M = sum(counts)
+    bn, sp, var = tiling
+    for kind in range(4):
+        model.set_tuning(kind, M, bn, sp, var)
+        assert model.tuning(kind, M) == (bn, sp, var)
+    with pytest.raises(RuntimeError):
+        model.set_tuning(4, M, 128, -1, 0)            # the LM head takes no K split
+    act = rt.Active(B, n_ctx)
+    tokens, positions, ck, cv = _state(shape, B, n_ctx, counts, seed=12, dev=cuda_dev, dtype="bf16")
+    act.load(positions)
+    _load_cache(cache, ck, cv, torch.bfloat16)
+    tok = torch.from_numpy(tokens).to(cuda_dev)
+    logits = torch.zeros((B * n_ctx, shape.vocab), device=cuda_dev, dtype=torch.bfloat16)
+    rt.step(model, cache, act, tok, logits)
+    torch.cuda.synchronize()
+    rt.device_check()
+    zs, ck2, cv2 = _oracle_step(shape, w64, tokens, positions, ck, cv, n_ctx)
     lg = to64(logits)
     for b in range(B):
         err = np.abs(lg[positions[b] + b * n_ctx] - zs[b]).max()

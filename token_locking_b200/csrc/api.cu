@@ -609,6 +609,37 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
       }
     }
   }
+  // stream-K (splits = -1): every worker (SM, or CTA pair) runs an equal share
+  // of the tiles x K-blocks; each flushes about (tiles + workers) / workers
+  // partial tiles with fp32 atomics
+  if (split_kind != SPLIT_NONE) {
+    for (int variant = 0; variant <= 2; ++variant) {
+      if (variant > 0 && M <= 128) continue;
+      const int rows_unit = variant == 0 ? 128 : 256;
+      const int workers = variant == 2 ? num_sms / 2 : num_sms;
+      const double rate = variant == 2 ? 2.0 * peak / num_sms : peak / num_sms;
+      const int mt = (M + rows_unit - 1) / rows_unit;
+      const double rows_live = std::min(M, rows_unit);
+      for (int bn : {256, 128}) {
+        if (N % bn || bn < min_bn) continue;
+        if (swiglu && (N / 2) % (bn / 2)) continue;
+        if (variant == 1 && 4 * bn > 512) continue;      // keep double-buffered accumulators
+        const long tiles = (long)mt * (N / bn);
+        const long iters = tiles * kblocks;
+        const double per_worker = std::ceil((double)iters / workers);
+        const double t_hbm = 2.0 * ((double)N * K + (double)M * K) / bw_hbm;
+        const double t_l2 = (double)iters * (bn * 128.0 + rows_live * 128.0) / bw_l2;
+        const double t_mma = per_worker * 2.0 * rows_unit * bn * 64 / rate;
+        double t = std::max(t_hbm, std::max(t_l2, t_mma)) + 1.0e-6;
+        t += (double)M * N * 4.0 * (1.0 + (double)workers / tiles) / bw_l2;
+        if (split_kind == SPLIT_ACCUM) t += (double)M * N * 8.0 / bw_hbm + 3.0e-6;
+        if (t < best.cost - 1e-9) {
+          best = Plan{bn, -1, variant == 0 ? 1 : 2, t};
+          best.pair = variant == 2 ? 1 : 0;
+        }
+      }
+    }
+  }
   return best;
 }
 
@@ -757,7 +788,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn, V = cfg.vocab, H = cfg.n_heads;
   const double Md = (double)M;
-  const bool split = pl.splits > 1;
+  const bool split = pl.splits != 1;      // split K or stream-K: partial sums
   TcGemmArgs g{};
   g.M = M;
   g.bn = pl.bn;
@@ -986,14 +1017,16 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
     bn = p.bn;
     msub = p.msub;
     pair = p.pair;
-    if (splits <= 0) splits = p.splits;
+    if (splits == 0) splits = p.splits;
   }
   if (pair && bn != 128 && bn != 256)
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: the CTA-pair kernel needs bn 128 or 256");
   if (bn != 64 && bn != 128 && bn != 256) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bn must be 64/128/256");
   if (N % bn || (swiglu && (N / 2) % (bn / 2)))
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: N must be a multiple of bn");
-  if (splits < 1) splits = 1;
+  if (splits < 1 && splits != -1) splits = 1;
+  if (splits == -1 && epi != SL_GEMM_RESID && epi != SL_GEMM_ACCUM)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: stream-K (splits -1) needs RESID or ACCUM");
   const int epi_k = epi == SL_GEMM_STORE ? EPI_STORE : epi == SL_GEMM_RESID ? EPI_RESID
                     : epi == SL_GEMM_SWIGLU ? EPI_SWIGLU : EPI_ACCUM;
   const int brows = (swiglu || pair) ? bn / 2 : bn;
@@ -1069,7 +1102,7 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
   for (int k = 0; k < G_KINDS; ++k) m->tuned[k].assign(kTuneCount, {0, 1, 1});
   const int Ns[G_KINDS] = {3 * d, d, 2 * f, d, V};
   const int Ks[G_KINDS] = {d, d, d, f, d};
-  const int split_opts[] = {1, 2, 3, 4, 6, 8, 9, 12, 16};
+  const int split_opts[] = {1, 2, 3, 4, 6, 8, 9, 12, 16, -1};   // -1: stream-K
   for (int b = 0; b < kTuneCount && st == SL_OK; ++b) {
     if (b > 0 && kTuneBounds[b - 1] >= max_rows) break;
     const int Mb = std::min(kTuneBounds[b], max_rows);
@@ -1088,14 +1121,17 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
           if (kind == G_GU && (N / 2) % (bn / 2)) continue;
           int last_ss = 0;
           for (int sp : split_opts) {
-            if (kind == G_HD && sp > 1) break;
-            if (sp > std::max(1, kblocks / 2)) break;
-            const int kbp = (kblocks + sp - 1) / sp;
-            const int ss = (kblocks + kbp - 1) / kbp;
-            if (ss == last_ss) continue;
-            last_ss = ss;
-            const long units = (long)((Mb + 128 * msub - 1) / (128 * msub)) * (N / bn) * ss;
-            if (units > 24L * m->num_sms) continue;
+            if (kind == G_HD && sp != 1) break;
+            int ss = -1;
+            if (sp > 0) {
+              if (sp > std::max(1, kblocks / 2)) continue;
+              const int kbp = (kblocks + sp - 1) / sp;
+              ss = (kblocks + kbp - 1) / kbp;
+              if (ss == last_ss) continue;
+              last_ss = ss;
+              const long units = (long)((Mb + 128 * msub - 1) / (128 * msub)) * (N / bn) * ss;
+              if (units > 24L * m->num_sms) continue;
+            }
             Plan pl{bn, ss, msub, 0.0};
             pl.pair = variant == 2 ? 1 : 0;
             // each repetition is followed by a small kernel (an RMSNorm, as in
@@ -1147,6 +1183,24 @@ extern "C" sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn
   *bn = p.bn;
   *splits = p.splits;
   *variant = p.pair ? 2 : (p.msub == 2 ? 1 : 0);
+  return SL_OK;
+}
+
+extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits,
+                                         int variant) {
+  if (!m || kind < 0 || kind >= G_KINDS || M <= 0)
+    return fail(SL_ERR_INVALID, "sl_model_set_tuning: bad argument");
+  if (m->cfg.dtype != SL_BF16) return fail(SL_ERR_INVALID, "sl_model_set_tuning: bf16 models only");
+  const int d = m->cfg.d_model, f = m->cfg.d_ffn, V = m->cfg.vocab;
+  const int Ns[G_KINDS] = {3 * d, d, 2 * f, d, V};
+  const int N = Ns[kind];
+  if ((bn != 64 && bn != 128 && bn != 256) || N % bn || (kind == G_GU && f % (bn / 2)) ||
+      (kind == G_QKV && bn < 128) || variant < 0 || variant > 2 || (variant == 2 && bn < 128) ||
+      (splits < 1 && splits != -1) || (kind == G_HD && splits != 1))
+    return fail(SL_ERR_INVALID, "sl_model_set_tuning: tiling not valid for this GEMM");
+  if (m->tuned[kind].empty())
+    for (int k = 0; k < G_KINDS; ++k) m->tuned[k].assign(kTuneCount, {0, 1, 1});
+  m->tuned[kind][tune_bucket(M)] = {bn, splits, variant};
   return SL_OK;
 }
 

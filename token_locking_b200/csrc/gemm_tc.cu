@@ -220,6 +220,8 @@ struct TcParams {
   int b_swiglu;            // 1: B tile = gate rows | up rows (halves of BN)
   int M, N, K;
   int m_tiles, n_tiles, splits, kb_per_split, kblocks, units;
+  int stream_k;            // 1: balanced split of the tile x K-block space (see WorkIter)
+  int atomic_out;          // 1: partial sums (split K or stream-K) are added atomically
   void *out;
   int ldo;
   int ffn;                 // SWIGLU/ACCUM-swiglu: F (columns of one half)
@@ -233,17 +235,63 @@ struct TcParams {
 
 constexpr int GROUP_M = 16;
 
-__device__ __forceinline__ void decode_unit(const TcParams &p, int u, int &mt, int &nt, int &sp) {
-  const int per_group = GROUP_M * p.n_tiles * p.splits;
+// Unit u of m_tiles x n_tiles x splits: groups of GROUP_M row tiles walk the
+// column tiles together, row tile fastest, so a weight tile is read from HBM
+// once and re-read by the group's row tiles from L2.
+__device__ __forceinline__ void decode_unit(const TcParams &p, int u, int splits, int &mt, int &nt,
+                                            int &sp) {
+  const int per_group = GROUP_M * p.n_tiles * splits;
   const int g = u / per_group;
   const int r = u - g * per_group;
   const int first_m = g * GROUP_M;
   const int gm = min(GROUP_M, p.m_tiles - first_m);
   mt = first_m + r % gm;
   const int nn = r / gm;
-  nt = nn / p.splits;
-  sp = nn - nt * p.splits;
+  nt = nn / splits;
+  sp = nn - nt * splits;
 }
+
+// The work of one worker (a CTA, or a CTA pair) as a sequence of (output tile,
+// K-block range) items; the producer, MMA and epilogue roles each walk the
+// same sequence.  Grid-stride mode: units w, w + nw, ... of the m_tiles x
+// n_tiles x splits units.  Stream-K mode: the worker's equal share
+// [w I / nw, (w + 1) I / nw) of the I = tiles x kblocks iteration space, cut
+// where it passes from one tile to the next, so that every worker runs the
+// same number of K-blocks whatever the tile count (partial tiles are summed
+// atomically by the epilogue).
+struct WorkIter {
+  long long pos, end;
+  int step;
+  __device__ __forceinline__ WorkIter(const TcParams &p, int w, int nw) {
+    if (p.stream_k) {
+      const long long I = (long long)p.m_tiles * p.n_tiles * p.kblocks;
+      pos = I * w / nw;
+      end = I * (w + 1) / nw;
+      step = 0;
+    } else {
+      pos = w;
+      end = p.units;
+      step = nw;
+    }
+  }
+  __device__ __forceinline__ bool next(const TcParams &p, int &mt, int &nt, int &kb0, int &kb1) {
+    if (pos >= end) return false;
+    int sp;
+    if (p.stream_k) {
+      const int t = (int)(pos / p.kblocks);
+      kb0 = (int)(pos - (long long)t * p.kblocks);
+      kb1 = (int)min((long long)p.kblocks, (long long)kb0 + (end - pos));
+      pos = (long long)t * p.kblocks + kb1;
+      decode_unit(p, t, 1, mt, nt, sp);
+    } else {
+      decode_unit(p, (int)pos, p.splits, mt, nt, sp);
+      kb0 = sp * p.kb_per_split;
+      kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      pos += step;
+    }
+    return true;
+  }
+};
 
 template <int BN, int STAGES, int MSUB>
 struct TcSmem {
@@ -377,7 +425,7 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, uint32_t taddr,
         }
       } else {   // EPI_RESID: h += partial (atomic when K is split)
         float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + nt * BN + c;
-        if (p.splits == 1) {
+        if (!p.atomic_out) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
             float4 o = *reinterpret_cast<float4 *>(dst + i);
@@ -455,11 +503,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       // the first stages of this CTA's first unit before waiting on it, so the
       // weight stream starts while the previous kernel drains.
       int npre = 0;
-      if ((int)blockIdx.x < p.units) {
-        int mt, nt, sp;
-        decode_unit(p, blockIdx.x, mt, nt, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      WorkIter first_it(p, blockIdx.x, gridDim.x);
+      int mt, nt, kb0, kb1;
+      if (first_it.next(p, mt, nt, kb0, kb1)) {
         npre = min(STAGES, kb1 - kb0);
         for (int i = 0; i < npre; ++i) {
           const uint32_t sb = sbase + i * L::STAGE_BYTES + L::A_BYTES;
@@ -474,11 +520,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       uint32_t last_phase = 0;
       bool ok = true;
       bool first = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        int mt, nt, sp;
-        decode_unit(p, u, mt, nt, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      WorkIter it(p, blockIdx.x, gridDim.x);
+      while (ok && it.next(p, mt, nt, kb0, kb1)) {
         for (int kb = kb0; kb < kb1; ++kb) {
           const bool pre = first && (kb - kb0) < npre;
           if (!pre) {
@@ -519,11 +562,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        int mt, nt, sp;
-        decode_unit(p, u, mt, nt, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      WorkIter it(p, blockIdx.x, gridDim.x);
+      int mt, nt, kb0, kb1;
+      while (ok && it.next(p, mt, nt, kb0, kb1)) {
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
@@ -564,9 +605,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-      int mt, nt, sp;
-      decode_unit(p, u, mt, nt, sp);
+    WorkIter it(p, blockIdx.x, gridDim.x);
+    int mt, nt, kb0, kb1;
+    while (it.next(p, mt, nt, kb0, kb1)) {
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
@@ -673,11 +714,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
         }
       };
       int npre = 0;
-      if (pair < p.units) {
-        int mt, nt, sp;
-        decode_unit(p, pair, mt, nt, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      WorkIter first_it(p, pair, n_pairs);
+      int mt, nt, kb0, kb1;
+      if (first_it.next(p, mt, nt, kb0, kb1)) {
         npre = min(STAGES, kb1 - kb0);
         for (int i = 0; i < npre; ++i) {
           if (leader) mbar_expect_tx(full_bar(i), 2 * STAGE_BYTES);
@@ -688,11 +727,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true, first = true;
-      for (int u = pair; u < p.units && ok; u += n_pairs) {
-        int mt, nt, sp;
-        decode_unit(p, u, mt, nt, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      WorkIter it(p, pair, n_pairs);
+      while (ok && it.next(p, mt, nt, kb0, kb1)) {
         for (int kb = kb0; kb < kb1; ++kb) {
           const bool pre = first && (kb - kb0) < npre;
           if (!pre) {
@@ -722,11 +758,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int u = pair; u < p.units && ok; u += n_pairs) {
-        int mt, nt, sp;
-        decode_unit(p, u, mt, nt, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+      WorkIter it(p, pair, n_pairs);
+      int mt, nt, kb0, kb1;
+      while (ok && it.next(p, mt, nt, kb0, kb1)) {
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -761,9 +795,9 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int u = pair; u < p.units; u += n_pairs) {
-      int mt, nt, sp;
-      decode_unit(p, u, mt, nt, sp);
+    WorkIter it(p, pair, n_pairs);
+    int mt, nt, kb0, kb1;
+    while (it.next(p, mt, nt, kb0, kb1)) {
       if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
       const int r = mt * 256 + (int)rank * 128 + q * 32 + lane;
@@ -891,6 +925,8 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.m_tiles = (a.M + 128 * msub - 1) / (128 * msub);
   p.n_tiles = a.N / bn;
   p.kblocks = a.K / 64;
+  // splits < 0: stream-K (partial sums must be summable: RESID and ACCUM only)
+  const bool stream_k = a.splits < 0 && (a.epi == EPI_RESID || a.epi == EPI_ACCUM);
   int splits = a.splits < 1 ? 1 : a.splits;
   if (a.epi == EPI_STORE || a.epi == EPI_QKV || a.epi == EPI_SWIGLU) splits = 1;
   if (a.epi == EPI_QKV && (bn < 128 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||
@@ -900,6 +936,10 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;   // no empty split
   p.units = p.m_tiles * p.n_tiles * p.splits;
+  p.stream_k = stream_k ? 1 : 0;
+  p.atomic_out = (p.splits > 1 || stream_k) ? 1 : 0;
+  // stream-K: one worker per SM (CTA pair), never more than there are K-blocks
+  const long long sk_iters = (long long)p.m_tiles * p.n_tiles * p.kblocks;
   p.out = a.out;
   p.ldo = a.ldo;
   p.ffn = a.N / 2;
@@ -912,11 +952,13 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.ck = (bf16 *)a.ck;
   p.cv = (bf16 *)a.cv;
   if (pair_mma) {
-    const int pairs = p.units < num_sms / 2 ? p.units : num_sms / 2;
+    const long long work = stream_k ? sk_iters : p.units;
+    const int pairs = work < num_sms / 2 ? (int)work : num_sms / 2;
     if (bn == 256) return run_epi2<256, 6>(a.epi, p, pairs, s);
     return run_epi2<128, 6>(a.epi, p, pairs, s);
   }
-  int grid = p.units < num_sms ? p.units : num_sms;
+  const long long work = stream_k ? sk_iters : p.units;
+  int grid = work < num_sms ? (int)work : num_sms;
   if (msub == 2) {
     switch (bn) {
       case 256: return run_epi<256, 3, 2>(a.epi, p, grid, s);

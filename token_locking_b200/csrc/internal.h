@@ -125,7 +125,7 @@ struct TcGemmArgs {
   const TmaMat *B[3];    // weight segments, each [n_i][K]; SWIGLU: B[0]=gate, B[1]=up
   int n_seg[3];          // rows of each segment (STORE/ACCUM may use up to 3; others 1)
   int M, N, K;           // N = total output columns (SWIGLU: 2F)
-  int splits;            // K splits (EPI_RESID / EPI_ACCUM only)
+  int splits;            // K splits (EPI_RESID / EPI_ACCUM only); -1: stream-K
   int bn;                // 64, 128 or 256
   int b_swiglu;          // B tile = BN/2 gate rows (B[0]) | BN/2 up rows (B[1])
   int msub;              // 1: 128-row units; 2: 256-row units (two accumulators per B tile)

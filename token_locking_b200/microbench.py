@@ -209,6 +209,10 @@ def bench_gemm(args, dev):
     shapes = {"qkv": (3 * d, d), "o": (d, d), "gu": (2 * f, d), "down": (d, f)}
     if args.head:
         shapes["head"] = (V, d)
+    if args.gemms:
+        shapes = {k: shapes[k] if k != "head" else (V, d) for k in args.gemms.split(",")}
+    # fixed tilings "bn:variant:splits,..." instead of the sweep
+    fixed = [tuple(int(x) for x in t.split(":")) for t in args.tiles.split(",")] if args.tiles else None
     weights = {k: w(n, kk) for k, (n, kk) in shapes.items() if k != "gu"}
     wg, wu = w(f, d), w(f, d)
     flush = _Flush(dev)
@@ -218,15 +222,19 @@ def bench_gemm(args, dev):
             outb = torch.zeros((M, N), device=dev, dtype=torch.bfloat16)
             outf = torch.zeros((M, N), device=dev, dtype=torch.float32)
             outa = torch.zeros((M, f), device=dev, dtype=torch.bfloat16)
-            for bn, variant in ((256, 0), (128, 0), (64, 0), (256, 1), (128, 1), (64, 1), (256, 2),
-                                (128, 2)):
+            sweep = fixed or [(bn, variant, sp)
+                              for bn, variant in ((256, 0), (128, 0), (64, 0), (256, 1), (128, 1),
+                                                  (64, 1), (256, 2), (128, 2))
+                              for sp in (1, 2, 3, 4, 6, 8, 9, 12, 16, -1)]
+            torch.cuda.profiler.start()          # ncu --profile-from-start off captures from here
+            for bn, variant, sp in sweep:
                 if bn < 128 and name == "qkv":
                     continue
-                if (variant > 0 and M <= 128) or N % bn:
+                if (variant > 0 and M <= 128 and not fixed) or N % bn:
                     continue
-                for sp in (1, 2, 3, 4, 6, 8, 9, 12, 16):
-                    if sp > 1 and name == "head":
-                        continue
+                if sp != 1 and name == "head":
+                    continue
+                if True:
                     if name == "gu":
                         epi, b, b2, out = ((A.GEMM_SWIGLU, wg, wu, outa) if sp == 1 else
                                            (A.GEMM_ACCUM, wg, wu, outf))
@@ -247,6 +255,9 @@ def bench_gemm(args, dev):
                                       "us": round(ms * 1e3, 2),
                                       "GBps": round(by / ms / 1e6, 1),
                                       "TFLOPs": round(fl / ms / 1e9, 1)}), flush=True)
+            torch.cuda.profiler.stop()
+            if fixed:
+                continue
             # the library's own choice
             if name == "gu":
                 epi, b, b2, out = A.GEMM_SWIGLU, wg, wu, outa
@@ -269,6 +280,8 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["layer", "lock", "decode", "gemm"])
     ap.add_argument("--head", action="store_true")
+    ap.add_argument("--gemms", default=None, help="gemm case: comma list of qkv,o,gu,down,head")
+    ap.add_argument("--tiles", default=None, help="gemm case: fixed bn:variant:splits list")
     ap.add_argument("--no-tune", action="store_true")
     ap.add_argument("--m", default=None)
     ap.add_argument("--iters", type=int, default=10)

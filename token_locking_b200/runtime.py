@@ -108,6 +108,11 @@ class Model:
                                         C.byref(var)), "sl_model_tuning")
         return bn.value, sp.value, var.value
 
+    def set_tuning(self, kind: int, M: int, bn: int, splits: int, variant: int):
+        """Pin GEMM `kind`'s tiling for the row-count bucket of M (splits -1: stream-K)."""
+        A.check(A.lib().sl_model_set_tuning(self.handle, kind, M, bn, splits, variant),
+                "sl_model_set_tuning")
+
     def timing_enable(self, on: bool = True):
         A.check(A.lib().sl_timing_enable(self.handle, 1 if on else 0), "sl_timing_enable")
 
