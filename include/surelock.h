@@ -202,7 +202,7 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
 /* The tensor-core GEMM of the bf16 path, C = A[M,K] * B[N,K]^T (bf16 operands,
  * fp32 accumulation), exposed for kernel-level checks and benchmarks.
  *   SL_GEMM_STORE : out bf16 [.][ldo], row r written to row d_row_map[r] (or r)
- *   SL_GEMM_RESID : out fp32 [M][ldo] += C
+ *   SL_GEMM_RESID : out fp32 [M][ldo] += C (added in L2 by TMA reduce-add)
  *   SL_GEMM_SWIGLU: d_b = W_gate [F][K], d_b2 = W_up [F][K], N = 2F;
  *                   out bf16 [M][ldo] = silu(A W_gate^T) * (A W_up^T)
  *   SL_GEMM_ACCUM : out fp32 [M][ldo] += C (atomic; with d_b2, gate/up halves
@@ -214,7 +214,8 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
  * tile (two accumulators share each weight tile), 2 = a CTA pair per 256 x bn
  * tile with 2-SM tensor-core instructions (bn 128 or 256).  bn = 0 lets the
  * library choose everything.  K % 64 == 0, N % bn == 0, pointers 16-byte
- * aligned. */
+ * aligned, ldo >= the output columns (N, or F for SWIGLU) with 16-byte rows
+ * (ldo % 4 == 0 for fp32 outputs, % 8 for bf16); SL_ERR_INVALID otherwise. */
 enum { SL_GEMM_STORE = 0, SL_GEMM_RESID = 1, SL_GEMM_SWIGLU = 2, SL_GEMM_ACCUM = 3 };
 sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b, const void *d_b2,
                        int N, void *d_out, int ldo, const int32_t *d_row_map, int bn, int splits,

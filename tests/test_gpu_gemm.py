@@ -132,3 +132,16 @@ def test_stream_k_rejected_for_store(cuda_dev):
     out = torch.zeros((8, 128), device=cuda_dev, dtype=torch.bfloat16)
     with pytest.raises(RuntimeError):
         rt.gemm_bf16(A.GEMM_STORE, a, b, out, bn=128, splits=-1)
+
+
+@pytest.mark.parametrize("variant,splits", [(0, 1), (2, -1)])
+def test_resid_strided_output(cuda_dev, variant, splits):
+    """fp32 output rows with a pitch wider than N (columns past N untouched)."""
+    M, K, N, ldo = 150, 512, 256, 288
+    a, b = _mk((M, K), 17, cuda_dev), _mk((N, K), 18, cuda_dev)
+    buf = torch.full((M, ldo), 3.0, device=cuda_dev)
+    rt.gemm_bf16(A.GEMM_RESID, a, b, buf, ldo=ldo, bn=128, splits=splits, variant=variant)
+    torch.cuda.synchronize()
+    _close(buf[:, :N] - 3.0, _ref(a, b), K, False)
+    assert torch.all(buf[:, N:] == 3.0)
+    rt.device_check()

@@ -125,6 +125,10 @@ struct sl_kv_cache {
   float *attn_ws = nullptr;
   int attn_max_splits = 16;
   TmaMat map_a, map_o, map_act;
+  // epilogue destinations at the current M: residual h (fp32), split-K
+  // workspace as [M][3d] and [M][2f] (fp32), gate/up product act (bf16)
+  TmaMat out_h, out_ws3, out_ws2, out_act;
+  TmaMat out_hx{};            // a caller's hidden states (sl_layer_forward), by pointer
   int map_rows = -1;
 };
 
@@ -748,9 +752,13 @@ static BfPlans plans_for(const sl_model *m, int M, int ns) {
 static sl_status ensure_maps(sl_kv_cache *c, int M) {
   if (c->map_rows == M) return SL_OK;
   const sl_config &cfg = c->m->cfg;
-  if (!tma_encode(&c->map_a, c->a, M, cfg.d_model, 128) ||
-      !tma_encode(&c->map_o, c->o, M, cfg.d_model, 128) ||
-      !tma_encode(&c->map_act, c->act, M, cfg.d_ffn, 128))
+  const int d = cfg.d_model, f = cfg.d_ffn;
+  if (!tma_encode(&c->map_a, c->a, M, d, 128) || !tma_encode(&c->map_o, c->o, M, d, 128) ||
+      !tma_encode(&c->map_act, c->act, M, f, 128) ||
+      !tma_encode_out(&c->out_h, c->h, M, d, d, true) ||
+      !tma_encode_out(&c->out_ws3, c->ws, M, 3 * d, 3 * d, true) ||
+      !tma_encode_out(&c->out_ws2, c->ws, M, 2 * f, 2 * f, true) ||
+      !tma_encode_out(&c->out_act, c->act, M, f, f, false))
     return fail(SL_ERR_CUDA, "activation TMA descriptor encoding failed");
   c->map_rows = M;
   return SL_OK;
@@ -812,6 +820,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
         g.epi = EPI_ACCUM;
         g.out = c->ws;
         g.ldo = 3 * d;
+        g.OUT = &c->out_ws3;
       } else {
         g.epi = EPI_QKV;
         g.row_map = rows;
@@ -837,6 +846,15 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       g.epi = EPI_RESID;
       g.out = h;
       g.ldo = d;
+      if (h == c->h) {
+        g.OUT = &c->out_h;
+      } else {   // a caller's hidden states (sl_layer_forward)
+        if (c->out_hx.ptr != h || c->out_hx.rows != M) {
+          if (!tma_encode_out(&c->out_hx, h, M, d, d, true))
+            return fail(SL_ERR_INVALID, "hidden-state TMA descriptor encoding failed");
+        }
+        g.OUT = &c->out_hx;
+      }
       bytes = gemm_bytes(Md, d, K, 2);
       flops = 2.0 * Md * d * K;
       break;
@@ -852,6 +870,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       g.epi = split ? EPI_ACCUM : EPI_SWIGLU;
       g.out = split ? (void *)c->ws : c->act;
       g.ldo = split ? 2 * f : f;
+      g.OUT = split ? &c->out_ws2 : &c->out_act;
       bytes = gemm_bytes(Md, 2.0 * f, d, 2) - 2.0 * Md * f;
       flops = 4.0 * Md * d * f;
       break;
@@ -1006,6 +1025,14 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   if (swiglu && N % 2) return fail(SL_ERR_INVALID, "sl_gemm_bf16: gate/up needs even N");
   if (((uintptr_t)d_a | (uintptr_t)d_b | (uintptr_t)(d_b2 ? d_b2 : d_b) | (uintptr_t)d_out) & 15)
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: pointers must be 16-byte aligned");
+  {
+    // output rows: fp32 (RESID/ACCUM) or bf16 (STORE/SWIGLU), 16-byte row pitch
+    const bool f32_out = epi == SL_GEMM_RESID || epi == SL_GEMM_ACCUM;
+    const int out_cols = epi == SL_GEMM_SWIGLU ? N / 2 : N;
+    if (ldo < out_cols || ldo % (f32_out ? 4 : 8) != 0)
+      return fail(SL_ERR_INVALID, "sl_gemm_bf16: ldo must cover the output columns and give "
+                                  "16-byte aligned rows");
+  }
   if (M == 0) return SL_OK;
   const int ns = sm_count();
   if (variant < 0 || variant > 2) return fail(SL_ERR_INVALID, "sl_gemm_bf16: variant must be 0, 1 or 2");
@@ -1051,6 +1078,15 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   g.row_map = d_row_map;
   g.msub = msub;
   g.pair = pair;
+  // TMA epilogue when the output rows qualify (16-byte row pitch)
+  TmaMat mo;
+  if (epi == SL_GEMM_RESID || epi == SL_GEMM_ACCUM) {
+    if (!tma_encode_out(&mo, d_out, M, N, ldo, true))
+      return fail(SL_ERR_INVALID, "sl_gemm_bf16: output TMA descriptor encoding failed");
+    g.OUT = &mo;
+  } else if (epi == SL_GEMM_SWIGLU && bn >= 128) {
+    if (tma_encode_out(&mo, d_out, M, N / 2, ldo, false)) g.OUT = &mo;
+  }
   int *err = device_error_word();
   if (!err) return fail(SL_ERR_CUDA, "sl_gemm_bf16: no device error word");
   cudaError_t e = launch_gemm_tc(g, ns, err, (cudaStream_t)stream);

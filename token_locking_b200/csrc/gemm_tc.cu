@@ -55,6 +55,30 @@ bool tma_encode(TmaMat *m, const void *ptr, int rows, int cols, int box_rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Output descriptor for the TMA epilogue: [rows][cols] with leading dimension
+// ld (elements), 32-row boxes of 128 bytes (32 fp32 or 64 bf16 columns), 128-byte
+// swizzle.  Rows past `rows` are clipped by the copy engine.
+bool tma_encode_out(TmaMat *m, const void *ptr, int rows, int cols, int ld, bool f32) {
+  auto fn = encode_fn();
+  const int esz = f32 ? 4 : 2, box_cols = f32 ? 32 : 64;
+  if (!fn || rows <= 0 || cols % box_cols != 0 || ld < cols || ((size_t)ld * esz) % 16 != 0 ||
+      ((uintptr_t)ptr & 15) != 0)
+    return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)ld * esz};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(&m->map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  2, const_cast<void *>(ptr), gdim, gstride, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  m->ptr = ptr;
+  m->rows = rows;
+  m->cols = cols;
+  m->box_rows = 32;
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------- device: PTX glue ---
 __device__ __forceinline__ uint32_t s_addr(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -98,6 +122,39 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+// Epilogue stores from shared memory (bulk async-group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x, int y,
+                                                  uint32_t src) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -216,12 +273,13 @@ __device__ __forceinline__ constexpr uint32_t idesc_bf16_f32() {
 struct TcParams {
   CUtensorMap a;
   CUtensorMap b[3];
+  CUtensorMap out_map;     // TMA epilogue destination (tma_out)
   int seg0, seg1;          // output column boundaries of segments 0 and 1
   int b_swiglu;            // 1: B tile = gate rows | up rows (halves of BN)
   int M, N, K;
   int m_tiles, n_tiles, splits, kb_per_split, kblocks, units;
   int stream_k;            // 1: balanced split of the tile x K-block space (see WorkIter)
-  int atomic_out;          // 1: partial sums (split K or stream-K) are added atomically
+  int tma_out;             // 1: RESID/ACCUM/SWIGLU tiles leave through out_map (see epilogue)
   void *out;
   int ldo;
   int ffn;                 // SWIGLU/ACCUM-swiglu: F (columns of one half)
@@ -234,6 +292,9 @@ struct TcParams {
 };
 
 constexpr int GROUP_M = 16;
+// Epilogue staging: each of the 4 epilogue warps owns one 32-row x 128-byte box
+// (128-byte swizzled, as the output descriptors expect).
+constexpr int EPI_STAGING_BYTES = 4 * 4096;
 
 // Unit u of m_tiles x n_tiles x splits: groups of GROUP_M row tiles walk the
 // column tiles together, row tile fastest, so a weight tile is read from HBM
@@ -298,7 +359,8 @@ struct TcSmem {
   static constexpr int A_BYTES = MSUB * 128 * 64 * 2;   // MSUB 128-row A tiles per stage
   static constexpr int B_BYTES = BN * 64 * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;          // epilogue staging, 4 warps x 4 KB
+  static constexpr int BAR_OFF = EPI_OFF + EPI_STAGING_BYTES;
   static constexpr int TOTAL = BAR_OFF + 256 + 1024;   // barriers + alignment slack
 };
 
@@ -319,33 +381,92 @@ __device__ __forceinline__ void load_b(const TcParams &p, uint32_t sb, int nt, i
   }
 }
 
-// Epilogue of one 128-row accumulator tile: TMEM lane quarter of the calling
-// warp (taddr carries the lane offset) for A row r, output tile nt.
+// Put 128 bytes of row `lane` into the warp's staging box (16-byte chunk j at
+// j ^ (row % 8): the 128-byte swizzle, and conflict-free per 8 lanes) once the
+// previous bulk copy out of the box has read it.
+__device__ __forceinline__ void stage_wait(int lane) {
+  if (lane == 0) bulk_wait_read0();
+  __syncwarp();
+}
+__device__ __forceinline__ void stage_chunk(uint32_t stg, int lane, int j, uint32_t a, uint32_t b,
+                                            uint32_t c, uint32_t d) {
+  st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), a, b, c, d);
+}
+__device__ __forceinline__ void stage_done() {
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+  return l | (h << 16);
+}
+
+// TMA epilogue of RESID / ACCUM (fp32 reduce-add) and SWIGLU (bf16 store): the
+// warp's 32 rows x 32 (64) columns go through its staging box and leave as one
+// bulk tensor copy, whole 128-byte lines; boxes past the live rows are skipped.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_tile_tma(const TcParams &p, uint32_t taddr, int row0,
+                                                  int nt, uint32_t stg, int lane) {
+  if (row0 >= p.M) return;
+  float v[32];
+  if (EPI == EPI_SWIGLU) {
+    const int f0 = nt * (BN / 2);
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 64) {
+      stage_wait(lane);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float g[32];
+        tmem_ld32(taddr + c + 32 * h, g);
+        tmem_ld32(taddr + BN / 2 + c + 32 * h, v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16(silu_f(g[8 * j + 2 * e]) * v[8 * j + 2 * e],
+                             silu_f(g[8 * j + 2 * e + 1]) * v[8 * j + 2 * e + 1]);
+          stage_chunk(stg, lane, 4 * h + j, w[0], w[1], w[2], w[3]);
+        }
+      }
+      stage_done();
+      if (lane == 0) {
+        tma_store_2d(&p.out_map, f0 + c, row0, stg);
+        bulk_commit();
+      }
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      tmem_ld32(taddr + c, v);
+      int col = nt * BN + c;
+      if (EPI == EPI_ACCUM && p.b_swiglu) {   // gate into [0, F), up into [F, 2F)
+        const int half = BN / 2, f0 = nt * half;
+        col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
+      }
+      stage_wait(lane);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        stage_chunk(stg, lane, j, __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                    __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+      stage_done();
+      if (lane == 0) {
+        tma_reduce_add_2d(&p.out_map, col, row0, stg);
+        bulk_commit();
+      }
+    }
+  }
+}
+
+// Per-thread epilogue of one 128-row accumulator tile (STORE, QKV, and SWIGLU
+// without an output descriptor): TMEM lane quarter of the calling warp (taddr
+// carries the lane offset), A row r, output tile nt; each thread writes its row.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile(const TcParams &p, uint32_t taddr, int r, int nt) {
   const bool live = r < p.M;
   float v[32];
-  if (EPI == EPI_ACCUM) {
-    // split-K partial sum of this tile: fp32 atomics into the workspace
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      tmem_ld32(taddr + c, v);
-      if (!live) continue;
-      int col;
-      if (p.b_swiglu) {   // gate into [0, F), up into [F, 2F)
-        const int half = BN / 2;
-        const int f0 = nt * half;
-        col = (c < half) ? (f0 + c) : (p.ffn + f0 + (c - half));
-      } else {
-        col = nt * BN + c;
-      }
-      float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + col;
-#pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        atomicAdd(reinterpret_cast<float4 *>(dst + i),
-                  make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
-    }
-  } else if (EPI == EPI_SWIGLU) {
+  if (EPI == EPI_SWIGLU) {
     const int f0 = nt * (BN / 2);
 #pragma unroll 1
     for (int c = 0; c < BN / 2; c += 32) {
@@ -413,31 +534,15 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, uint32_t taddr,
     for (int c = 0; c < BN; c += 32) {
       tmem_ld32(taddr + c, v);
       if (!live) continue;
-      if (EPI == EPI_STORE) {
-        const int orow = p.row_map ? p.row_map[r] : r;
-        bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)orow * p.ldo + nt * BN + c;
+      // EPI_STORE
+      const int orow = p.row_map ? p.row_map[r] : r;
+      bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)orow * p.ldo + nt * BN + c;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          Pack8 pk;
+      for (int i = 0; i < 32; i += 8) {
+        Pack8 pk;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(v[i + e]);
-          *reinterpret_cast<uint4 *>(dst + i) = pk.u;
-        }
-      } else {   // EPI_RESID: h += partial (atomic when K is split)
-        float *dst = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo + nt * BN + c;
-        if (!p.atomic_out) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4 o = *reinterpret_cast<float4 *>(dst + i);
-            o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
-            *reinterpret_cast<float4 *>(dst + i) = o;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            atomicAdd(reinterpret_cast<float4 *>(dst + i),
-                      make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
-        }
+        for (int e = 0; e < 8; ++e) pk.h[e] = __float2bfloat16_rn(v[i + e]);
+        *reinterpret_cast<uint4 *>(dst + i) = pk.u;
       }
     }
   }
@@ -615,7 +720,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const int r = (mt * MSUB + sub) * 128 + q * 32 + lane;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * ACC_COLS + sub * BN) +
                              ((uint32_t)(q * 32) << 16);
-      epilogue_tile<BN, EPI>(p, taddr, r, nt);
+      if constexpr (EPI == EPI_RESID || EPI == EPI_ACCUM)
+        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane);
+      else if (EPI == EPI_SWIGLU && BN >= 128 && p.tma_out)
+        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane);
+      else
+        epilogue_tile<BN, EPI>(p, taddr, r, nt);
       }   // sub
       tc_fence_before();
       __syncwarp();
@@ -623,6 +733,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       if (++acc == ACC_BUFS) { acc = 0; acc_phase ^= 1u; }
 
     }
+    if (lane == 0) bulk_wait0();          // staged tiles written before the CTA exits
     if (!ok && lane == 0) {
       atomicExch(p.err, DEV_TIMEOUT_EPI);
       *abort_flag = 1;
@@ -652,7 +763,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
   constexpr int A_BYTES = 128 * 64 * 2;
   constexpr int B_BYTES = (BN / 2) * 64 * 2;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+  constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  constexpr int BAR_OFF = EPI_OFF + EPI_STAGING_BYTES;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -802,12 +914,18 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       tc_fence_after();
       const int r = mt * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
-      epilogue_tile<BN, EPI>(p, taddr, r, nt);
+      if constexpr (EPI == EPI_RESID || EPI == EPI_ACCUM)
+        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane);
+      else if (EPI == EPI_SWIGLU && p.tma_out)
+        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane);
+      else
+        epilogue_tile<BN, EPI>(p, taddr, r, nt);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait0();          // staged tiles written before the CTA exits
     if (!ok && lane == 0) {
       atomicExch(p.err, DEV_TIMEOUT_EPI);
       *abort_flag = 1;
@@ -848,7 +966,7 @@ static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
 // (a GPC with an odd number of usable SMs leaves one SM out of the pairing).
 template <int BN, int STAGES, int EPI>
 static cudaError_t run_tc2(const TcParams &p, int pairs, cudaStream_t s) {
-  constexpr int SMEM = STAGES * (16384 + (BN / 2) * 128) + 256 + 1024;
+  constexpr int SMEM = STAGES * (16384 + (BN / 2) * 128) + EPI_STAGING_BYTES + 256 + 1024;
   static int max_pairs = 0;
   if (max_pairs == 0) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc2_kernel<BN, STAGES, EPI>,
@@ -937,7 +1055,11 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;   // no empty split
   p.units = p.m_tiles * p.n_tiles * p.splits;
   p.stream_k = stream_k ? 1 : 0;
-  p.atomic_out = (p.splits > 1 || stream_k) ? 1 : 0;
+  if ((a.epi == EPI_RESID || a.epi == EPI_ACCUM) && !a.OUT) return cudaErrorInvalidValue;
+  if (a.OUT && (a.epi == EPI_RESID || a.epi == EPI_ACCUM || (a.epi == EPI_SWIGLU && bn >= 128))) {
+    p.out_map = a.OUT->map;
+    p.tma_out = 1;
+  }
   // stream-K: one worker per SM (CTA pair), never more than there are K-blocks
   const long long sk_iters = (long long)p.m_tiles * p.n_tiles * p.kblocks;
   p.out = a.out;

@@ -118,6 +118,7 @@ struct TmaMat {
   int box_rows;          // rows per TMA box
 };
 bool tma_encode(TmaMat *m, const void *ptr, int rows, int cols, int box_rows);
+bool tma_encode_out(TmaMat *m, const void *ptr, int rows, int cols, int ld, bool f32);
 
 struct TcGemmArgs {
   int epi;               // GemmEpi
@@ -130,6 +131,8 @@ struct TcGemmArgs {
   int b_swiglu;          // B tile = BN/2 gate rows (B[0]) | BN/2 up rows (B[1])
   int msub;              // 1: 128-row units; 2: 256-row units (two accumulators per B tile)
   int pair;              // 1: CTA-pair kernel (2-SM MMA, 256-row units, B maps with BN/2 boxes)
+  const TmaMat *OUT;     // RESID/ACCUM (fp32) or SWIGLU (bf16) output descriptor from
+                         // tma_encode_out: tiles leave by TMA reduce-add / store (optional)
   void *out;             // STORE/SWIGLU: dtype out; RESID: fp32 resid; ACCUM: fp32 ws
   int ldo;               // leading dimension of out (elements)
   const int32_t *row_map;// STORE: output row index per A row (or null); QKV: flat positions
