@@ -207,12 +207,12 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
  *                   out bf16 [M][ldo] = silu(A W_gate^T) * (A W_up^T)
  *   SL_GEMM_ACCUM : out fp32 [M][ldo] += C (atomic; with d_b2, gate/up halves
  *                   accumulate into columns [0,F) and [F,2F))
- * bn (64/128/256) and splits (>= 1, RESID/ACCUM only; -1 = stream-K: every SM
+ * bn (64/128/192/256) and splits (>= 1, RESID/ACCUM only; -1 = stream-K: every SM
  * or CTA pair takes an equal share of the tiles x 64-wide K-blocks and adds
  * its partial tiles atomically) pick the tiling; variant
  * picks the kernel: 0 = one CTA per 128 x bn tile, 1 = one CTA per 256 x bn
  * tile (two accumulators share each weight tile), 2 = a CTA pair per 256 x bn
- * tile with 2-SM tensor-core instructions (bn 128 or 256).  bn = 0 lets the
+ * tile with 2-SM tensor-core instructions (bn 128, 192 or 256).  bn = 0 lets the
  * library choose everything.  K % 64 == 0, N % bn == 0, pointers 16-byte
  * aligned, ldo >= the output columns (N, or F for SWIGLU) with 16-byte rows
  * (ldo % 4 == 0 for fp32 outputs, % 8 for bf16); SL_ERR_INVALID otherwise. */
@@ -258,6 +258,12 @@ sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows, void *str
  * 2 gate/up, 3 down, 4 LM head) at M rows; *splits and *variant as for
  * sl_gemm_bf16. */
 sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits, int *variant);
+/* Pin the attention layout of sl_step / sl_attention on this model:
+ * queries_per_cta 16, 32 or 64 (the four warps of a CTA then split every
+ * 64-key tile 4, 2 or 1 ways) and the split of the key range across CTAs
+ * (1..16, capped so every split keeps >= 4 tiles); 0 leaves either to the
+ * library's cost model.  SL_ERR_INVALID for other values. */
+sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits);
 /* Pin the tiling of GEMM `kind` for the row-count bucket that holds M (the
  * buckets of sl_model_autotune); arguments as for sl_gemm_bf16.  Returns
  * SL_ERR_INVALID for a tiling the GEMM cannot use (the LM head takes no K

@@ -1,0 +1,75 @@
+"""Attention of the active queries over every cached key (sl_attention, bf16
+path) against the oracle's attention in fp64: each warp layout of the kernel
+(16, 32 or 64 queries per CTA, the key tile shared by 4, 2 or 1 warps), with and
+without the key range split across CTAs, ragged query counts, empty sequences
+and key counts off the 64-key tile grid; every layout is pinned in turn
+(sl_model_set_attention) as well as left to the library's cost model."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from oracle import model as om
+from token_locking_b200 import runtime as rt
+from parity_util import to64, weights_to_device
+
+pytestmark = pytest.mark.gpu
+
+SHAPE = wl.ModelShape(n_layers=1, d_model=512, n_heads=4, head_dim=128, d_ffn=512, vocab=1024,
+                      mask_id=1023, rope_theta=10000.0)
+
+CASES = [
+    ([5], 384),             # a handful of queries over the bench's key count
+    ([1], 64),              # one query, one key tile
+    ([16, 3], 130),         # ragged key tail
+    ([30, 17], 700),
+    ([100, 64, 1], 384),    # query tiles of several sizes in one launch
+    ([7], 4000),            # long key range (splits of many tiles)
+    ([200], 2500),
+    ([0, 40, 0], 260),      # empty sequences
+]
+
+
+# (queries per CTA, cross-CTA key split); 0 = the library's cost model
+LAYOUTS = [(0, 0), (16, 1), (32, 1), (64, 1), (16, 4), (32, 2), (64, 3)]
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("counts,n_ctx", CASES)
+def test_attention_matches_oracle(cuda_dev, counts, n_ctx, layout):
+    B = len(counts)
+    H, dh, d = SHAPE.n_heads, SHAPE.head_dim, SHAPE.d_model
+    w_dev = weights_to_device(wl.np_weights(SHAPE, seed=0, std=0.05), "bf16", cuda_dev)
+    model = rt.Model(SHAPE, w_dev, "bf16")
+    model.set_attention(*layout)
+    cache = rt.KVCache(model, B, n_ctx)
+    act = rt.Active(B, n_ctx)
+    rng = np.random.default_rng(sum(counts) + n_ctx)
+    positions = [np.sort(rng.choice(n_ctx, c, replace=False)).astype(np.int32) for c in counts]
+    act.load(positions)
+    k_np = wl.round_bf16(rng.standard_normal((B * n_ctx, d)).astype(np.float32))
+    v_np = wl.round_bf16(rng.standard_normal((B * n_ctx, d)).astype(np.float32))
+    k, v = cache.view(0)
+    k.copy_(torch.from_numpy(k_np).to(cuda_dev, torch.bfloat16))
+    v.copy_(torch.from_numpy(v_np).to(cuda_dev, torch.bfloat16))
+    M = sum(counts)
+    q_np = wl.round_bf16(rng.standard_normal((max(M, 1), d)).astype(np.float32))[:M]
+    q = torch.from_numpy(q_np).to(cuda_dev, torch.bfloat16)
+    o = torch.full((max(M, 1), d), 9.0, device=cuda_dev, dtype=torch.bfloat16)
+    rt.attention(model, cache, act, 0, q, o)
+    torch.cuda.synchronize()
+    rt.device_check()
+    got = to64(o)
+    off = 0
+    for b, c in enumerate(counts):
+        if c == 0:
+            continue
+        qb = q_np[off:off + c].astype(np.float64).reshape(c, H, dh)
+        kb = k_np[b * n_ctx:(b + 1) * n_ctx].astype(np.float64).reshape(n_ctx, H, dh)
+        vb = v_np[b * n_ctx:(b + 1) * n_ctx].astype(np.float64).reshape(n_ctx, H, dh)
+        ref = om.attention(qb, kb, vb).reshape(c, d)
+        # P is rounded to bf16 before P V, the output to bf16
+        err = np.abs(got[off:off + c] - ref).max()
+        assert err <= 2e-2 * max(1.0, np.abs(ref).max()), f"seq {b}: max err {err}"
+        off += c
+    model.close()

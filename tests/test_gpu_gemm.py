@@ -28,7 +28,8 @@ def _close(got, ref, K, bf16_out):
     assert err <= tol, f"max err {err} > tol {tol} (scale {scale})"
 
 
-VARIANTS = [(64, 0), (128, 0), (256, 0), (64, 1), (128, 1), (256, 1), (128, 2), (256, 2)]
+VARIANTS = [(64, 0), (128, 0), (192, 0), (256, 0), (64, 1), (128, 1), (192, 1), (256, 1), (128, 2),
+            (192, 2), (256, 2)]
 
 
 @pytest.mark.parametrize("bn,variant", VARIANTS)
@@ -52,10 +53,11 @@ def test_store_rowmap(cuda_dev, bn, variant, M):
 @pytest.mark.parametrize("bn,splits,variant", [(64, 1, 0), (128, 3, 0), (256, 2, 0), (128, 8, 0),
                                                (256, 3, 1), (128, 1, 1), (64, 2, 1), (256, 1, 2),
                                                (256, 3, 2), (128, 2, 2), (256, -1, 0), (64, -1, 0),
-                                               (128, -1, 1), (256, -1, 2), (128, -1, 2)])
+                                               (128, -1, 1), (256, -1, 2), (128, -1, 2), (192, 1, 0),
+                                               (192, 3, 1), (192, -1, 0), (192, 2, 2), (192, -1, 2)])
 @pytest.mark.parametrize("M", [5, 130, 600])
 def test_resid_split(cuda_dev, bn, splits, variant, M):
-    K, N = 1024, 512
+    K, N = 1024, 768
     a, b = _mk((M, K), 4, cuda_dev), _mk((N, K), 5, cuda_dev)
     h0 = torch.randn((M, N), generator=torch.Generator().manual_seed(6)).to(cuda_dev)
     h = h0.clone()
@@ -65,8 +67,8 @@ def test_resid_split(cuda_dev, bn, splits, variant, M):
     rt.device_check()
 
 
-@pytest.mark.parametrize("bn,variant", [(64, 0), (128, 0), (256, 0), (128, 1), (256, 1),
-                                        (128, 2), (256, 2)])
+@pytest.mark.parametrize("bn,variant", [(64, 0), (128, 0), (192, 0), (256, 0), (128, 1), (192, 1),
+                                        (256, 1), (128, 2), (192, 2), (256, 2)])
 @pytest.mark.parametrize("M", [3, 129, 300])
 def test_swiglu(cuda_dev, bn, variant, M):
     K, F = 256, 384
@@ -84,15 +86,16 @@ def test_swiglu(cuda_dev, bn, variant, M):
 
 
 @pytest.mark.parametrize("swiglu", [False, True])
-@pytest.mark.parametrize("splits,variant", [(4, 0), (4, 2), (-1, 0), (-1, 1), (-1, 2)])
-def test_accum_split(cuda_dev, swiglu, splits, variant):
-    M, K, F = 77, 768, 256
+@pytest.mark.parametrize("splits,variant,bn", [(4, 0, 128), (4, 2, 128), (-1, 0, 128), (-1, 1, 128),
+                                               (-1, 2, 128), (3, 0, 192), (-1, 2, 192)])
+def test_accum_split(cuda_dev, swiglu, splits, variant, bn):
+    M, K, F = 77, 768, 384
     a = _mk((M, K), 10, cuda_dev)
     b = _mk((F, K), 11, cuda_dev)
     b2 = _mk((F, K), 12, cuda_dev) if swiglu else None
     N = 2 * F if swiglu else F
     ws = torch.zeros((M, N), device=cuda_dev)
-    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=128, splits=splits, variant=variant)
+    rt.gemm_bf16(A.GEMM_ACCUM, a, b, ws, b2=b2, bn=bn, splits=splits, variant=variant)
     torch.cuda.synchronize()
     ref = torch.cat([_ref(a, b), _ref(a, b2)], dim=1) if swiglu else _ref(a, b)
     _close(ws, ref, K, False)

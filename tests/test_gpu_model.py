@@ -197,3 +197,49 @@ def test_pinned_tilings_step_matches_oracle(cuda_dev, tiling):
         err = np.abs(lg[positions[b] + b * n_ctx] - zs[b]).max()
         assert err <= LOGIT_TOL["bf16"], err
     model.close()
+
+
+MINI_768 = wl.ModelShape(n_layers=2, d_model=768, n_heads=6, head_dim=128, d_ffn=768,
+                         vocab=1024, mask_id=1023, rope_theta=10000.0)
+
+
+@pytest.mark.parametrize("splits,variant", [(1, 0), (-1, 2), (2, 1)])
+def test_bn192_tilings_step_matches_oracle(cuda_dev, splits, variant):
+    """192-column tiles for every projection (QKV, whose unsplit epilogue
+    rotates whole heads, through its split path): the step agrees with the
+    oracle and with the same step on the library's default tilings."""
+    shape = MINI_768
+    B, n_ctx = 1, 300
+    # weight scale of the d_model = 256 models (logits of the same magnitude)
+    w_np = wl.np_weights(shape, seed=2, std=0.05 * (256 / 768) ** 0.5, gain_jitter=0.1)
+    w_dev = weights_to_device(w_np, "bf16", cuda_dev)
+    w64 = weights_for_oracle(w_dev)
+    counts = [260]
+    M = sum(counts)
+    tokens, positions, ck, cv = _state(shape, B, n_ctx, counts, seed=13, dev=cuda_dev, dtype="bf16")
+    tok = torch.from_numpy(tokens).to(cuda_dev)
+
+    def run(pin):
+        model = rt.Model(shape, w_dev, "bf16")
+        if pin:
+            for kind in range(4):
+                sp = 2 if (kind == 0 and splits == 1) else splits
+                model.set_tuning(kind, M, 192, sp, variant)
+            with pytest.raises(RuntimeError):
+                model.set_tuning(0, M, 192, 1, 0)          # unsplit QKV needs whole heads
+        cache = rt.KVCache(model, B, n_ctx)
+        act = rt.Active(B, n_ctx)
+        act.load(positions)
+        _load_cache(cache, ck, cv, torch.bfloat16)
+        logits = torch.zeros((B * n_ctx, shape.vocab), device=cuda_dev, dtype=torch.bfloat16)
+        rt.step(model, cache, act, tok, logits)
+        torch.cuda.synchronize()
+        rt.device_check()
+        model.close()
+        return to64(logits)[positions[0]]
+
+    pinned, default = run(True), run(False)
+    zs, _, _ = _oracle_step(shape, w64, tokens, positions, ck, cv, n_ctx)
+    assert np.abs(pinned - zs[0]).max() <= LOGIT_TOL["bf16"]
+    assert np.abs(default - zs[0]).max() <= LOGIT_TOL["bf16"]
+    assert np.abs(pinned - default).max() <= LOGIT_TOL["bf16"]

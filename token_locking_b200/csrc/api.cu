@@ -72,16 +72,15 @@ using namespace sl;
 
 // ---------------------------------------------------------------- objects --
 // Weight descriptors for the tensor-core path: one TMA map per box height
-// (32, 64, 128, 256 rows) so any tile width can be launched.
+// (32, 64, 96, 128, 192, 256 rows: whole, half and pair-half tiles of every
+// tile width) so any tiling can be launched.
+constexpr int kBoxRows[6] = {32, 64, 96, 128, 192, 256};
 struct WMaps {
-  TmaMat m[4];
+  TmaMat m[6];
   const TmaMat *box(int rows) const {
-    switch (rows) {
-      case 32: return &m[0];
-      case 64: return &m[1];
-      case 128: return &m[2];
-      default: return &m[3];
-    }
+    for (int i = 0; i < 5; ++i)
+      if (kBoxRows[i] == rows) return &m[i];
+    return &m[5];
   }
 };
 
@@ -98,6 +97,7 @@ struct sl_model {
   const void *tok_emb, *final_norm, *lm_head;
   std::vector<sl_layer_weights> layers;
   std::vector<std::array<WMaps, W_COUNT>> maps;
+  int attn_q = 0, attn_splits = 0;   // pinned attention layout (0 = cost model)
   WMaps head_map;
   int num_sms;
   int *err;
@@ -248,7 +248,7 @@ extern "C" sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, 
     return fail(SL_ERR_CUDA, "sl_model_create: cannot allocate the device error word");
   }
   if (c.dtype == SL_BF16) {
-    const int boxes[4] = {32, 64, 128, 256};
+    const int *boxes = kBoxRows;
     m->maps.resize(c.n_layers);
     for (int l = 0; l < c.n_layers; ++l) {
       const sl_layer_weights &lw = m->layers[l];
@@ -258,7 +258,7 @@ extern "C" sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, 
       const int cols[W_COUNT] = {c.d_model, c.d_model, c.d_model, c.d_model, c.d_model,
                                  c.d_model, c.d_ffn};
       for (int i = 0; i < W_COUNT; ++i)
-        for (int b = 0; b < 4; ++b)
+        for (int b = 0; b < 6; ++b)
           if (!tma_encode(&m->maps[l][i].m[b], ptr[i], rows[i], cols[i], boxes[b])) {
             delete m;
             return fail(SL_ERR_INVALID,
@@ -266,7 +266,7 @@ extern "C" sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, 
                         "(pointer must be 16-byte aligned)", l, i);
           }
     }
-    for (int b = 0; b < 4; ++b)
+    for (int b = 0; b < 6; ++b)
       if (!tma_encode(&m->head_map.m[b], m->lm_head, c.vocab, c.d_model, boxes[b])) {
         delete m;
         return fail(SL_ERR_INVALID, "sl_model_create: TMA descriptor for lm_head failed");
@@ -546,7 +546,10 @@ struct Plan {
 // SPLIT_ACCUM the finalize pass).
 enum SplitKind { SPLIT_NONE = 0, SPLIT_RESID = 1, SPLIT_ACCUM = 2 };
 
-Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, int min_bn = 64) {
+// heads: the unsplit QKV epilogue rotates whole 128-column heads, so unsplit
+// plans keep bn a multiple of 128.
+Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, int min_bn = 64,
+               bool heads = false) {
   const double bw_hbm = 6.5e12, bw_l2 = 9.0e12, peak = 1.6e15;
   const int kblocks = K / 64;
   Plan best{0, 1, 1, 1e30};
@@ -555,13 +558,13 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
     const int rows_unit = 128 * msub;
     const int mt = (M + rows_unit - 1) / rows_unit;
     const double rows_live = std::min(M, rows_unit);
-    const int bns[3] = {256, 128, 64};
-    for (int bi = 0; bi < 3; ++bi) {
+    const int bns[4] = {256, 192, 128, 64};
+    for (int bi = 0; bi < 4; ++bi) {
       const int bn = bns[bi];
       if (N % bn || bn < min_bn) continue;
       if (swiglu && (N / 2) % (bn / 2)) continue;
       const bool single_acc = 2 * msub * bn > 512;
-      const double mma_eff = bn == 256 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
+      const double mma_eff = bn >= 192 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
       const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
       for (int sp = 1; sp <= max_s; ++sp) {
         const int kbp = (kblocks + sp - 1) / sp;
@@ -574,6 +577,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
         const double t_mma = (double)units * kbp * 2.0 * rows_unit * bn * 64 / (peak * mma_eff);
         double t = std::max(t_hbm, std::max(t_l2, t_mma)) * std::min(quant, 2.0) + waves * 1.0e-6;
         if (single_acc && waves > 1) t += waves * 2.0e-6;     // epilogue not overlapped
+        if (heads && bn % 128 != 0 && ss == 1) continue;
         if (ss > 1) {
           t += (double)M * N * 4.0 * ss / bw_l2;                               // fp32 atomics
           if (split_kind == SPLIT_ACCUM) t += (double)M * N * 8.0 / bw_hbm + 3.0e-6;   // finalize
@@ -588,7 +592,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
     const int pairs = num_sms / 2;
     const int mt = (M + 255) / 256;
     const double rows_live = std::min(M, 256);
-    for (int bn : {256, 128}) {
+    for (int bn : {256, 192, 128}) {
       if (N % bn || bn < min_bn) continue;
       if (swiglu && (N / 2) % (bn / 2)) continue;
       const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
@@ -602,6 +606,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
         const double t_l2 = (double)units * kbp * (bn * 128.0 + rows_live * 128.0) / bw_l2;
         const double t_mma = (double)units * kbp * 2.0 * 256 * bn * 64 / peak;
         double t = std::max(t_hbm, std::max(t_l2, t_mma)) * std::min(quant, 2.0) + waves * 1.0e-6;
+        if (heads && bn % 128 != 0 && ss == 1) continue;
         if (ss > 1) {
           t += (double)M * N * 4.0 * ss / bw_l2;
           if (split_kind == SPLIT_ACCUM) t += (double)M * N * 8.0 / bw_hbm + 3.0e-6;
@@ -624,7 +629,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
       const double rate = variant == 2 ? 2.0 * peak / num_sms : peak / num_sms;
       const int mt = (M + rows_unit - 1) / rows_unit;
       const double rows_live = std::min(M, rows_unit);
-      for (int bn : {256, 128}) {
+      for (int bn : {256, 192, 128}) {
         if (N % bn || bn < min_bn) continue;
         if (swiglu && (N / 2) % (bn / 2)) continue;
         if (variant == 1 && 4 * bn > 512) continue;      // keep double-buffered accumulators
@@ -731,7 +736,7 @@ static Plan plan_kind(const sl_model *m, int kind, int M, int ns) {
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn;
   switch (kind) {
-    case G_QKV: return plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128);
+    case G_QKV: return plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128, true);
     case G_O: return plan_gemm(M, d, d, SPLIT_RESID, ns, false);
     case G_GU: return plan_gemm(M, 2 * f, d, SPLIT_ACCUM, ns, true);
     case G_DN: return plan_gemm(M, d, f, SPLIT_RESID, ns, false);
@@ -780,7 +785,8 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
   Timed t(m, SL_K_ATTN, 2.0 * (2.0 * M * d + 2.0 * seqs.batch * c->n_ctx * d),
           4.0 * (double)M * c->n_ctx * d, s);
   SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
-                           c->attn_ws, c->attn_max_splits, m->num_sms, s));
+                           c->attn_ws, c->attn_max_splits, m->num_sms, s, m->attn_q,
+                           m->attn_splits));
   return SL_OK;
 }
 
@@ -1046,9 +1052,10 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
     pair = p.pair;
     if (splits == 0) splits = p.splits;
   }
-  if (pair && bn != 128 && bn != 256)
-    return fail(SL_ERR_INVALID, "sl_gemm_bf16: the CTA-pair kernel needs bn 128 or 256");
-  if (bn != 64 && bn != 128 && bn != 256) return fail(SL_ERR_INVALID, "sl_gemm_bf16: bn must be 64/128/256");
+  if (pair && bn < 128)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: the CTA-pair kernel needs bn 128, 192 or 256");
+  if (bn != 64 && bn != 128 && bn != 192 && bn != 256)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: bn must be 64/128/192/256");
   if (N % bn || (swiglu && (N / 2) % (bn / 2)))
     return fail(SL_ERR_INVALID, "sl_gemm_bf16: N must be a multiple of bn");
   if (splits < 1 && splits != -1) splits = 1;
@@ -1084,7 +1091,7 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
     if (!tma_encode_out(&mo, d_out, M, N, ldo, true))
       return fail(SL_ERR_INVALID, "sl_gemm_bf16: output TMA descriptor encoding failed");
     g.OUT = &mo;
-  } else if (epi == SL_GEMM_SWIGLU && bn >= 128) {
+  } else if (epi == SL_GEMM_SWIGLU && (bn / 2) % 64 == 0) {
     if (tma_encode_out(&mo, d_out, M, N / 2, ldo, false)) g.OUT = &mo;
   }
   int *err = device_error_word();
@@ -1151,13 +1158,14 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
       for (int variant = 0; variant <= 2; ++variant) {
         const int msub = variant == 0 ? 1 : 2;
         if (variant > 0 && Mb <= 128) continue;
-        for (int bn : {256, 128, 64}) {
+        for (int bn : {256, 192, 128, 64}) {
           if (N % bn || (kind == G_QKV && bn < 128)) continue;
           if (variant == 2 && bn < 128) continue;
           if (kind == G_GU && (N / 2) % (bn / 2)) continue;
           int last_ss = 0;
           for (int sp : split_opts) {
             if (kind == G_HD && sp != 1) break;
+            if (kind == G_QKV && sp == 1 && bn % 128 != 0) continue;   // whole heads unsplit
             int ss = -1;
             if (sp > 0) {
               if (sp > std::max(1, kblocks / 2)) continue;
@@ -1222,6 +1230,16 @@ extern "C" sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn
   return SL_OK;
 }
 
+extern "C" sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits) {
+  if (!m || (queries_per_cta != 0 && queries_per_cta != 16 && queries_per_cta != 32 &&
+             queries_per_cta != 64) ||
+      splits < 0 || splits > 16)
+    return fail(SL_ERR_INVALID, "sl_model_set_attention: queries_per_cta 0/16/32/64, splits 0..16");
+  m->attn_q = queries_per_cta;
+  m->attn_splits = splits;
+  return SL_OK;
+}
+
 extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits,
                                          int variant) {
   if (!m || kind < 0 || kind >= G_KINDS || M <= 0)
@@ -1230,8 +1248,9 @@ extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, i
   const int d = m->cfg.d_model, f = m->cfg.d_ffn, V = m->cfg.vocab;
   const int Ns[G_KINDS] = {3 * d, d, 2 * f, d, V};
   const int N = Ns[kind];
-  if ((bn != 64 && bn != 128 && bn != 256) || N % bn || (kind == G_GU && f % (bn / 2)) ||
-      (kind == G_QKV && bn < 128) || variant < 0 || variant > 2 || (variant == 2 && bn < 128) ||
+  if ((bn != 64 && bn != 128 && bn != 192 && bn != 256) || N % bn || (kind == G_GU && f % (bn / 2)) ||
+      (kind == G_QKV && (bn < 128 || (bn % 128 != 0 && splits == 1))) || variant < 0 ||
+      variant > 2 || (variant == 2 && bn < 128) ||
       (splits < 1 && splits != -1) || (kind == G_HD && splits != 1))
     return fail(SL_ERR_INVALID, "sl_model_set_tuning: tiling not valid for this GEMM");
   if (m->tuned[kind].empty())

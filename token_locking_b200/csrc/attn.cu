@@ -4,23 +4,41 @@
 // The pages reduce per-step attention from O(N^2 d) to O(M N d) by issuing
 // queries for the active rows only while keys/values of every position are
 // read from the cache C (Abstract; Paper-Notes, "permanent locking":
-// K^all[L_t] <- C.k[L_t]).  One CTA owns 64 queries of one (sequence, head)
-// and a range of 64-key tiles; K/V tiles stream through shared memory with
-// cp.async double buffering and an online softmax.  When the query tiles alone
-// cannot fill the GPU (few active rows), the key range is split across CTAs
-// and a second kernel merges the partial (max, sum, output) records, one warp
-// per (row, head) so the merge spreads over every SM.
+// K^all[L_t] <- C.k[L_t]).  One CTA owns 16 * QW queries of one (sequence,
+// head) and a range of 64-key tiles, which stream through a 3-deep
+// shared-memory ring (cp.async) with an online softmax.  Its four warps are
+// QW query warps x 4/QW key warps: with few active rows per sequence (the
+// late denoising steps) the warps split every key tile between them instead
+// of idling on empty query rows, and merge their (max, sum, output) states
+// through shared memory at the end.  Only when the CTAs cannot fill the GPU
+// and the key range is long is it also split across CTAs, with a second
+// kernel merging those partial records, one warp per (row, head).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace sl {
 
-constexpr int AT_Q = 64;       // queries per CTA
 constexpr int AT_K = 64;       // keys per tile
 constexpr int AT_D = 128;      // head dim
 constexpr int AT_THREADS = 128;
-constexpr int ATTN_MAX_SPLITS = 16;    // split-KV partials merged in-kernel
-constexpr int AT_SMEM = (AT_Q + 4 * AT_K) * AT_D * 2;   // Q + 2x(K,V)
+constexpr int AT_STAGES = 3;   // K/V tiles in flight
+constexpr int ATTN_MAX_SPLITS = 16;    // cross-CTA split-KV partials merged by attn_combine
+
+template <int QW>
+struct AtCfg {
+  static constexpr int KW = 4 / QW;          // warps sharing each key tile
+  static constexpr int TQ = 16 * QW;         // queries per CTA
+  static constexpr int KS = AT_K / KW;       // keys of a tile per warp: 64, 32 or 16
+  static constexpr int Q_BYTES = TQ * AT_D * 2;
+  static constexpr int KV_BYTES = AT_K * AT_D * 2;   // one K (or V) tile
+  static constexpr int SMEM = Q_BYTES + AT_STAGES * 2 * KV_BYTES;
+  // merge scratch (reuses the K/V ring): per partial warp 32 lanes x (64 + 4) floats
+  static constexpr int PART_FLOATS = 68;
+  static_assert(QW * (KW - 1) * 32 * (PART_FLOATS + 4) * 4 <= AT_STAGES * 2 * KV_BYTES,
+                "merge scratch must fit in the K/V ring");
+};
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -69,44 +87,46 @@ struct AttnParams {
   int M, n_ctx, n_heads, splits, kblocks;
 };
 
+template <int QW>
 __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_constant__ AttnParams p) {
+  using C = AtCfg<QW>;
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sQ = smem_u32(smem);
-  const uint32_t sK0 = sQ + AT_Q * AT_D * 2;
-  const uint32_t sV0 = sK0 + 2 * AT_K * AT_D * 2;
+  const uint32_t sKV = sQ + C::Q_BYTES;      // stage s: K tile, then V tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qw = warp / C::KW, kw = warp % C::KW;
   const int h = blockIdx.y, split = blockIdx.z;
   const int d = p.n_heads * AT_D;
 
   // locate (sequence, query tile)
   int tile = blockIdx.x, b = 0, q0 = 0, qn = 0;
   for (; b < p.seqs.batch; ++b) {
-    int nt = (p.seqs.seq_count[b] + AT_Q - 1) / AT_Q;
+    int nt = (p.seqs.seq_count[b] + C::TQ - 1) / C::TQ;
     if (tile < nt) break;
     tile -= nt;
   }
   if (b >= p.seqs.batch) return;
-  q0 = p.seqs.seq_start[b] + tile * AT_Q;
-  qn = min(AT_Q, p.seqs.seq_count[b] - tile * AT_Q);
+  q0 = p.seqs.seq_start[b] + tile * C::TQ;
+  qn = min(C::TQ, p.seqs.seq_count[b] - tile * C::TQ);
 
   const int per = (p.kblocks + p.splits - 1) / p.splits;
   const int kb0 = split * per;
   const int kb1 = min(p.kblocks, kb0 + per);
+  const int ntiles = max(0, kb1 - kb0);
 
   const bf16 *kbase = p.ck + (size_t)b * p.n_ctx * d + h * AT_D;
   const bf16 *vbase = p.cv + (size_t)b * p.n_ctx * d + h * AT_D;
   pdl_wait();
 
-  // Q tile
-  for (int e = tid; e < AT_Q * 16; e += AT_THREADS) {
+  for (int e = tid; e < C::TQ * 16; e += AT_THREADS) {
     int r = e >> 4, c = e & 15;
     bool ok = r < qn;
     const bf16 *src = p.q + (size_t)(q0 + (ok ? r : 0)) * d + h * AT_D + c * 8;
     cp_async16(sQ + tile_off(r, c), src, ok);
   }
-  auto load_kv = [&](int kb, int buf) {
-    const uint32_t sK = sK0 + buf * AT_K * AT_D * 2;
-    const uint32_t sV = sV0 + buf * AT_K * AT_D * 2;
+  auto load_kv = [&](int kb, int stage) {
+    const uint32_t sK = sKV + stage * 2 * C::KV_BYTES;
+    const uint32_t sV = sK + C::KV_BYTES;
     for (int e = tid; e < AT_K * 16; e += AT_THREADS) {
       int r = e >> 4, c = e & 15;
       int key = kb * AT_K + r;
@@ -116,8 +136,12 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
       cp_async16(sV + tile_off(r, c), vbase + off, ok);
     }
   };
-  if (kb0 < kb1) load_kv(kb0, 0);
-  cp_commit();
+  // groups: {Q, tile 0}, {tile 1}, then one per iteration (possibly empty)
+#pragma unroll
+  for (int i = 0; i < AT_STAGES - 1; ++i) {
+    if (i < ntiles) load_kv(kb0 + i, i);
+    cp_commit();
+  }
 
   const float sl2 = 1.4426950408889634f * rsqrtf((float)AT_D);   // log2(e)/sqrt(dh)
   float o_acc[16][4];
@@ -126,31 +150,32 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
   float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
   uint32_t qf[8][4];
   const int g = lane >> 2, c4 = lane & 3;
+  constexpr int NT = C::KS / 8;     // 8-key score tiles per warp
 
-  for (int kb = kb0; kb < kb1; ++kb) {
-    const int buf = (kb - kb0) & 1;
-    if (kb + 1 < kb1) load_kv(kb + 1, buf ^ 1);
+  for (int i = 0; i < ntiles; ++i) {
+    const int kb = kb0 + i, stage = i % AT_STAGES;
+    if (i + AT_STAGES - 1 < ntiles) load_kv(kb + AT_STAGES - 1, (i + AT_STAGES - 1) % AT_STAGES);
     cp_commit();
-    cp_wait<1>();
+    cp_wait<AT_STAGES - 1>();
     __syncthreads();
-    if (kb == kb0) {
+    if (i == 0) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        int r = warp * 16 + (lane & 15);
+        int r = qw * 16 + (lane & 15);
         int c = 2 * kk + (lane >> 4);
         ldsm_x4(sQ + tile_off(r, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
       }
     }
-    const uint32_t sK = sK0 + buf * AT_K * AT_D * 2;
-    const uint32_t sV = sV0 + buf * AT_K * AT_D * 2;
-    float s[8][4];
+    const uint32_t sK = sKV + stage * 2 * C::KV_BYTES;
+    const uint32_t sV = sK + C::KV_BYTES;
+    float s[NT][4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+    for (int t = 0; t < NT; ++t) s[t][0] = s[t][1] = s[t][2] = s[t][3] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-      for (int nt = 0; nt < 8; nt += 2) {
-        int r = nt * 8 + (lane & 7) + ((lane >> 4) << 3);
+      for (int nt = 0; nt < NT; nt += 2) {
+        int r = kw * C::KS + nt * 8 + (lane & 7) + ((lane >> 4) << 3);
         int c = 2 * kk + ((lane >> 3) & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(sK + tile_off(r, c), b0, b1, b2, b3);
@@ -158,13 +183,13 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
         mma16816(s[nt + 1], qf[kk], b2, b3);
       }
     }
-    // online softmax (base 2) on rows g and g+8 of this warp
+    // online softmax (base 2) on rows g and g+8 of this warp's 16 queries
     float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        int key = kb * AT_K + nt * 8 + 2 * c4 + (e & 1);
+        int key = kb * AT_K + kw * C::KS + nt * 8 + 2 * c4 + (e & 1);
         float v = (key < p.n_ctx) ? s[nt][e] * sl2 : -INFINITY;
         s[nt][e] = v;
         tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
@@ -181,7 +206,7 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
     }
     float rs[2] = {0.f, 0.f};
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float mm = m_r[e >> 1];
@@ -197,13 +222,13 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
       l_r[r] = l_r[r] * corr[r] + rs[r];
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o_acc[i][0] *= corr[0]; o_acc[i][1] *= corr[0];
-      o_acc[i][2] *= corr[1]; o_acc[i][3] *= corr[1];
+    for (int t = 0; t < 16; ++t) {
+      o_acc[t][0] *= corr[0]; o_acc[t][1] *= corr[0];
+      o_acc[t][2] *= corr[1]; o_acc[t][3] *= corr[1];
     }
-    // O += P V
+    // O += P V over this warp's keys of the tile
 #pragma unroll
-    for (int kc = 0; kc < 4; ++kc) {
+    for (int kc = 0; kc < NT / 2; ++kc) {
       uint32_t pa[4];
       pa[0] = pack_bf16(s[2 * kc][0], s[2 * kc][1]);
       pa[1] = pack_bf16(s[2 * kc][2], s[2 * kc][3]);
@@ -211,7 +236,7 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
       pa[3] = pack_bf16(s[2 * kc + 1][2], s[2 * kc + 1][3]);
 #pragma unroll
       for (int dt = 0; dt < 16; dt += 2) {
-        int r = kc * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+        int r = kw * C::KS + kc * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
         int c = dt + (lane >> 4);
         uint32_t b0, b1, b2, b3;
         ldsm_x4_t(sV + tile_off(r, c), b0, b1, b2, b3);
@@ -219,15 +244,56 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
         mma16816(o_acc[dt + 1], pa, b2, b3);
       }
     }
-    __syncthreads();
+    __syncthreads();      // the stage is refilled by the next iteration's load
   }
   cp_wait<0>();
   pdl_trigger();
 
-  // epilogue: rows g and g+8 of this warp's 16
+  if constexpr (C::KW > 1) {
+    // key warps 1.. hand their (max, sum, output) states to key warp 0 of the
+    // same query warp through the (now idle) K/V ring
+    __syncthreads();
+    float *part = reinterpret_cast<float *>(smem + C::Q_BYTES);
+    float4 *ml = reinterpret_cast<float4 *>(part + QW * (C::KW - 1) * 32 * C::PART_FLOATS);
+    if (kw > 0) {
+      const int slot = (qw * (C::KW - 1) + kw - 1) * 32 + lane;
+      float4 *dst = reinterpret_cast<float4 *>(part + slot * C::PART_FLOATS);
+#pragma unroll
+      for (int t = 0; t < 16; ++t) dst[t] = make_float4(o_acc[t][0], o_acc[t][1], o_acc[t][2], o_acc[t][3]);
+      ml[slot] = make_float4(m_r[0], m_r[1], l_r[0], l_r[1]);
+    }
+    __syncthreads();
+    if (kw > 0) return;
+#pragma unroll 1
+    for (int j = 1; j < C::KW; ++j) {
+      const int slot = (qw * (C::KW - 1) + j - 1) * 32 + lane;
+      const float4 pm = ml[slot];
+      const float om[2] = {pm.x, pm.y}, ol[2] = {pm.z, pm.w};
+      float c1[2], c2[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const float mx = fmaxf(m_r[r], om[r]);
+        c1[r] = (m_r[r] == -INFINITY) ? 0.f : exp2f(m_r[r] - mx);
+        c2[r] = (om[r] == -INFINITY) ? 0.f : exp2f(om[r] - mx);
+        l_r[r] = l_r[r] * c1[r] + ol[r] * c2[r];
+        m_r[r] = mx;
+      }
+      const float4 *src = reinterpret_cast<const float4 *>(part + slot * C::PART_FLOATS);
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const float4 v = src[t];
+        o_acc[t][0] = o_acc[t][0] * c1[0] + v.x * c2[0];
+        o_acc[t][1] = o_acc[t][1] * c1[0] + v.y * c2[0];
+        o_acc[t][2] = o_acc[t][2] * c1[1] + v.z * c2[1];
+        o_acc[t][3] = o_acc[t][3] * c1[1] + v.w * c2[1];
+      }
+    }
+  }
+
+  // epilogue: rows g and g+8 of this query warp's 16
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    int qr = warp * 16 + g + 8 * r;
+    int qr = qw * 16 + g + 8 * r;
     if (qr >= qn) continue;
     int j = q0 + qr;
     if (p.splits == 1) {
@@ -295,28 +361,52 @@ size_t attn_bf16_workspace_bytes(int max_rows, int n_heads, int max_splits) {
 }
 
 
-cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
-                             int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
-                             int num_sms, cudaStream_t s) {
-  cudaError_t err = cudaSuccess;
-  if (M <= 0) return cudaSuccess;
+template <int QW>
+static cudaError_t run_attn(const AttnParams &p, int tiles, cudaStream_t s) {
+  using C = AtCfg<QW>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, AT_SMEM);
+    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<QW>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  int tiles = 0;
-  for (int b = 0; b < seqs.batch; ++b) tiles += (seqs.seq_count[b] + AT_Q - 1) / AT_Q;
-  if (tiles == 0) return cudaSuccess;
+  return launch_k(attn_bf16_kernel<QW>, dim3(tiles, p.n_heads, p.splits), AT_THREADS, C::SMEM, s, p);
+}
+
+cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
+                             int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
+                             int num_sms, cudaStream_t s, int force_q, int force_splits) {
+  cudaError_t err = cudaSuccess;
+  if (M <= 0) return cudaSuccess;
+  // Queries per CTA (16 * qw) and cross-CTA key split from a small cost model:
+  // mma.sync instructions per warp (16 queries x its share of the keys), about
+  // 15 ns each once two CTAs share every SM; the K/V re-reads from L2, one per
+  // query tile; and a fixed cost for the merge kernel of a split.
   const int kblocks = (n_ctx + AT_K - 1) / AT_K;
-  const int ctas = tiles * n_heads;
-  int splits = (2 * num_sms + ctas - 1) / ctas;
-  int max_by_keys = kblocks / 2 > 0 ? kblocks / 2 : 1;
-  if (splits > max_by_keys) splits = max_by_keys;
-  if (splits > max_splits) splits = max_splits;
-  if (splits < 1) splits = 1;
+  int qw = 4, splits = 1, tiles = 0;
+  double best = 1e30;
+  const int max_sp = std::min(std::max(kblocks / 4, 1), std::min(max_splits, ATTN_MAX_SPLITS));
+  for (int cq : {4, 2, 1}) {
+    int nt = 0;
+    for (int b = 0; b < seqs.batch; ++b) nt += (seqs.seq_count[b] + 16 * cq - 1) / (16 * cq);
+    if (nt == 0) return cudaSuccess;
+    for (int sp = 1; sp <= max_sp; ++sp) {
+      const double warps = 4.0 * nt * n_heads * sp;
+      const double per_warp = 2.0 * ((double)kblocks * AT_K / sp) / (4 / cq);
+      const double t_mma = per_warp * std::max(1.0, warps / (8.0 * num_sms)) * 15e-9;
+      const double t_l2 = (double)nt * n_heads * n_ctx * AT_D * 4.0 / 8e12;
+      const double t = std::max(t_mma, t_l2) + (sp > 1 ? 3e-6 : 0.0);
+      if (force_q && 16 * cq != force_q) continue;
+      if (force_splits && sp != std::min(force_splits, max_sp)) continue;
+      if (t < best - 1e-12) {
+        best = t;
+        qw = cq;
+        splits = sp;
+        tiles = nt;
+      }
+    }
+  }
   AttnParams p;
   p.q = (const bf16 *)q;
   p.ck = (const bf16 *)ck;
@@ -330,8 +420,8 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
   p.n_heads = n_heads;
   p.splits = splits;
   p.kblocks = kblocks;
-  dim3 grid(tiles, n_heads, splits);
-  err = launch_k(attn_bf16_kernel, grid, AT_THREADS, AT_SMEM, s, p);
+  err = qw == 4 ? run_attn<4>(p, tiles, s) : qw == 2 ? run_attn<2>(p, tiles, s)
+                                                     : run_attn<1>(p, tiles, s);
   if (err != cudaSuccess || splits == 1) return err;
   const int warps = M * n_heads;
   return launch_k(attn_combine_kernel, (warps * 32 + 255) / 256, 256, 0, s, (const float *)p.ws_o,

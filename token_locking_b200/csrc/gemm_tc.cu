@@ -292,6 +292,11 @@ struct TcParams {
 };
 
 constexpr int GROUP_M = 16;
+__host__ __device__ constexpr uint32_t tmem_cols_pow2(uint32_t n) {
+  uint32_t c = 32;
+  while (c < n) c <<= 1;
+  return c;
+}
 // Epilogue staging: each of the 4 epilogue warps owns one 32-row x 128-byte box
 // (128-byte swizzled, as the output descriptors expect).
 constexpr int EPI_STAGING_BYTES = 4 * 4096;
@@ -572,7 +577,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr uint32_t TMEM_COLS = ACC_BUFS * ACC_COLS;
+  // tcgen05.alloc takes a power of two >= 32 columns
+  constexpr uint32_t TMEM_COLS = tmem_cols_pow2(ACC_BUFS * ACC_COLS);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -722,7 +728,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
                              ((uint32_t)(q * 32) << 16);
       if constexpr (EPI == EPI_RESID || EPI == EPI_ACCUM)
         epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane);
-      else if (EPI == EPI_SWIGLU && BN >= 128 && p.tma_out)
+      else if (EPI == EPI_SWIGLU && (BN / 2) % 64 == 0 && p.tma_out)
         epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane);
       else
         epilogue_tile<BN, EPI>(p, taddr, r, nt);
@@ -765,7 +771,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr int EPI_OFF = STAGES * STAGE_BYTES;
   constexpr int BAR_OFF = EPI_OFF + EPI_STAGING_BYTES;
-  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t TMEM_COLS = tmem_cols_pow2(2 * BN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s_addr(smem);
@@ -916,7 +922,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       if constexpr (EPI == EPI_RESID || EPI == EPI_ACCUM)
         epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane);
-      else if (EPI == EPI_SWIGLU && p.tma_out)
+      else if (EPI == EPI_SWIGLU && (BN / 2) % 64 == 0 && p.tma_out)
         epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane);
       else
         epilogue_tile<BN, EPI>(p, taddr, r, nt);
@@ -1020,7 +1026,7 @@ static cudaError_t run_epi(int epi, const TcParams &p, int grid, cudaStream_t s)
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
   const int bn = a.bn;
-  if ((bn != 64 && bn != 128 && bn != 256) || a.K % 64 != 0 || a.N % bn != 0)
+  if ((bn != 64 && bn != 128 && bn != 192 && bn != 256) || a.K % 64 != 0 || a.N % bn != 0)
     return cudaErrorInvalidValue;
   const bool swiglu_b = a.b_swiglu != 0;
   if (a.epi == EPI_SWIGLU && !swiglu_b) return cudaErrorInvalidValue;
@@ -1038,7 +1044,7 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.N = a.N;
   p.K = a.K;
   const bool pair_mma = a.pair != 0;
-  if (pair_mma && bn != 128 && bn != 256) return cudaErrorInvalidValue;
+  if (pair_mma && bn < 128) return cudaErrorInvalidValue;
   const int msub = (a.msub == 2 || pair_mma) ? 2 : 1;   // a pair owns 256 rows
   p.m_tiles = (a.M + 128 * msub - 1) / (128 * msub);
   p.n_tiles = a.N / bn;
@@ -1047,7 +1053,7 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   const bool stream_k = a.splits < 0 && (a.epi == EPI_RESID || a.epi == EPI_ACCUM);
   int splits = a.splits < 1 ? 1 : a.splits;
   if (a.epi == EPI_STORE || a.epi == EPI_QKV || a.epi == EPI_SWIGLU) splits = 1;
-  if (a.epi == EPI_QKV && (bn < 128 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||
+  if (a.epi == EPI_QKV && (bn % 128 != 0 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||
                            (a.N % 3) != 0 || ((a.N / 3) % 128) != 0))
     return cudaErrorInvalidValue;
   if (splits > p.kblocks) splits = p.kblocks;
@@ -1056,7 +1062,8 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.units = p.m_tiles * p.n_tiles * p.splits;
   p.stream_k = stream_k ? 1 : 0;
   if ((a.epi == EPI_RESID || a.epi == EPI_ACCUM) && !a.OUT) return cudaErrorInvalidValue;
-  if (a.OUT && (a.epi == EPI_RESID || a.epi == EPI_ACCUM || (a.epi == EPI_SWIGLU && bn >= 128))) {
+  if (a.OUT && (a.epi == EPI_RESID || a.epi == EPI_ACCUM ||
+                (a.epi == EPI_SWIGLU && (bn / 2) % 64 == 0))) {
     p.out_map = a.OUT->map;
     p.tma_out = 1;
   }
@@ -1077,6 +1084,7 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
     const long long work = stream_k ? sk_iters : p.units;
     const int pairs = work < num_sms / 2 ? (int)work : num_sms / 2;
     if (bn == 256) return run_epi2<256, 6>(a.epi, p, pairs, s);
+    if (bn == 192) return run_epi2<192, 7>(a.epi, p, pairs, s);
     return run_epi2<128, 6>(a.epi, p, pairs, s);
   }
   const long long work = stream_k ? sk_iters : p.units;
@@ -1084,12 +1092,14 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   if (msub == 2) {
     switch (bn) {
       case 256: return run_epi<256, 3, 2>(a.epi, p, grid, s);
+      case 192: return run_epi<192, 3, 2>(a.epi, p, grid, s);
       case 128: return run_epi<128, 4, 2>(a.epi, p, grid, s);
       default: return run_epi<64, 5, 2>(a.epi, p, grid, s);
     }
   }
   switch (bn) {
     case 256: return run_epi<256, 4, 1>(a.epi, p, grid, s);
+    case 192: return run_epi<192, 5, 1>(a.epi, p, grid, s);
     case 128: return run_epi<128, 6, 1>(a.epi, p, grid, s);
     default: return run_epi<64, 8, 1>(a.epi, p, grid, s);
   }

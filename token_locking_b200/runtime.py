@@ -108,6 +108,11 @@ class Model:
                                         C.byref(var)), "sl_model_tuning")
         return bn.value, sp.value, var.value
 
+    def set_attention(self, queries_per_cta: int = 0, splits: int = 0):
+        """Pin the attention layout (0 = the library's cost model)."""
+        A.check(A.lib().sl_model_set_attention(self.handle, queries_per_cta, splits),
+                "sl_model_set_attention")
+
     def set_tuning(self, kind: int, M: int, bn: int, splits: int, variant: int):
         """Pin GEMM `kind`'s tiling for the row-count bucket of M (splits -1: stream-K)."""
         A.check(A.lib().sl_model_set_tuning(self.handle, kind, M, bn, splits, variant),
