@@ -784,9 +784,10 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
   const int d = m->cfg.d_model;
   Timed t(m, SL_K_ATTN, 2.0 * (2.0 * M * d + 2.0 * seqs.batch * c->n_ctx * d),
           4.0 * (double)M * c->n_ctx * d, s);
+  // the output projection's weights follow; the attention leaves HBM idle
   SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
                            c->attn_ws, c->attn_max_splits, m->num_sms, s, m->attn_q,
-                           m->attn_splits));
+                           m->attn_splits, m->layers[l].wo, (size_t)d * d * 2));
   return SL_OK;
 }
 

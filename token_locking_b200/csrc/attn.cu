@@ -85,6 +85,8 @@ struct AttnParams {
   float *ws_ml;          // [splits][M][H][2]
   AttnSeqs seqs;
   int M, n_ctx, n_heads, splits, kblocks;
+  const void *pf;        // the next GEMM's weights, prefetched into L2 (optional)
+  size_t pf_bytes;
 };
 
 template <int QW>
@@ -116,6 +118,10 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
 
   const bf16 *kbase = p.ck + (size_t)b * p.n_ctx * d + h * AT_D;
   const bf16 *vbase = p.cv + (size_t)b * p.n_ctx * d + h * AT_D;
+  if (tid == 0) {
+    const int cta = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+    l2_prefetch_share(p.pf, p.pf_bytes, cta, gridDim.x * gridDim.y * gridDim.z);
+  }
   pdl_wait();
 
   for (int e = tid; e < C::TQ * 16; e += AT_THREADS) {
@@ -376,7 +382,8 @@ static cudaError_t run_attn(const AttnParams &p, int tiles, cudaStream_t s) {
 
 cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
                              int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
-                             int num_sms, cudaStream_t s, int force_q, int force_splits) {
+                             int num_sms, cudaStream_t s, int force_q, int force_splits,
+                             const void *pf, size_t pf_bytes) {
   cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   // Queries per CTA (16 * qw) and cross-CTA key split from a small cost model:
@@ -420,6 +427,8 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
   p.n_heads = n_heads;
   p.splits = splits;
   p.kblocks = kblocks;
+  p.pf = pf;
+  p.pf_bytes = pf_bytes;
   err = qw == 4 ? run_attn<4>(p, tiles, s) : qw == 2 ? run_attn<2>(p, tiles, s)
                                                      : run_attn<1>(p, tiles, s);
   if (err != cudaSuccess || splits == 1) return err;

@@ -60,6 +60,24 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 
 // 8 x bf16 <-> 16-byte vector
+// Fire-and-forget L2 prefetch of this CTA's share of [ptr, ptr + bytes): the
+// next kernel's weights, brought in while the running kernel leaves HBM idle.
+// ptr 16-byte aligned; pieces of at most 64 KB.
+__device__ __forceinline__ void l2_prefetch_share(const void *ptr, size_t bytes, int cta,
+                                                  int ctas) {
+  if (!ptr || bytes < 16) return;
+  const size_t units = bytes >> 4;                        // 16-byte units
+  const size_t per = (units + ctas - 1) / ctas;
+  size_t u0 = per * (size_t)cta, u1 = u0 + per;
+  if (u1 > units) u1 = units;
+  const char *base = reinterpret_cast<const char *>(ptr);
+  for (size_t u = u0; u < u1; u += 4096) {
+    const uint32_t n = (uint32_t)((u1 - u < 4096 ? u1 - u : 4096) << 4);
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + (u << 4)), "r"(n)
+                 : "memory");
+  }
+}
+
 union Pack8 {
   uint4 u;
   bf16 h[8];

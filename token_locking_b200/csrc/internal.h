@@ -106,10 +106,12 @@ struct AttnSeqs {
 };
 size_t attn_bf16_workspace_bytes(int max_rows, int n_heads, int max_splits);
 // force_q (16/32/64) and force_splits (>= 1) pin the layout; 0 = cost model.
+// [pf, pf + pf_bytes) is prefetched into L2 while the attention runs.
 cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
                              int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
                              int num_sms, cudaStream_t s, int force_q = 0,
-                             int force_splits = 0);
+                             int force_splits = 0, const void *pf = nullptr,
+                             size_t pf_bytes = 0);
 
 // ----------------------------------------------------------------- gemm_tc.cu
 // A bf16 K-major operand in global memory with its TMA descriptor.

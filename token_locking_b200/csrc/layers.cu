@@ -180,12 +180,71 @@ __global__ void __launch_bounds__(256) rope_scatter_kernel(
   }
 }
 
+// The same from the fp32 split-K workspace into bf16, eight pairs per thread:
+// 16-byte loads of both halves, the (cos, sin) table and the clearing stores,
+// 16-byte bf16 stores (head_dim % 16 == 0).
+__global__ void __launch_bounds__(256) rope_scatter_ws_kernel(
+    float *__restrict__ ws, int M, const int32_t *__restrict__ rows, int n_ctx, int n_heads,
+    int dh, const float2 *__restrict__ rope, bf16 *__restrict__ q_out, bf16 *__restrict__ ck,
+    bf16 *__restrict__ cv) {
+  const int j = blockIdx.y;
+  const int d = n_heads * dh;
+  const int half = dh >> 1;
+  const int groups = half >> 3;                      // 8-pair groups per head
+  const int t = blockIdx.x * 256 + threadIdx.x;      // (segment, head, group)
+  pdl_wait();
+  pdl_trigger();
+  if (t >= 3 * n_heads * groups) return;
+  const int seg = t / (n_heads * groups);
+  const int rem = t - seg * n_heads * groups;
+  const int hh = rem / groups, i0 = (rem - hh * groups) * 8;
+  const int c0 = hh * dh + i0, c1 = c0 + half;
+  float4 *in0 = reinterpret_cast<float4 *>(ws + (size_t)j * 3 * d + seg * d + c0);
+  float4 *in1 = reinterpret_cast<float4 *>(ws + (size_t)j * 3 * d + seg * d + c1);
+  const float4 a0 = in0[0], a1 = in0[1], b0 = in1[0], b1 = in1[1];
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  in0[0] = z;
+  in0[1] = z;
+  in1[0] = z;
+  in1[1] = z;
+  const float x0[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  const float x1[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+  const int p = rows[j];
+  bf16 *dst = seg == 0 ? q_out + (size_t)j * d : (seg == 1 ? ck : cv) + (size_t)p * d;
+  Pack8 lo, hi;
+  if (seg < 2) {
+    const float4 *tab = reinterpret_cast<const float4 *>(rope + (size_t)(p % n_ctx) * half + i0);
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float4 cs = tab[e >> 1];                 // (cos, sin) of pairs e and e + 1
+      lo.h[e] = __float2bfloat16_rn(x0[e] * cs.x - x1[e] * cs.y);
+      hi.h[e] = __float2bfloat16_rn(x1[e] * cs.x + x0[e] * cs.y);
+      lo.h[e + 1] = __float2bfloat16_rn(x0[e + 1] * cs.z - x1[e + 1] * cs.w);
+      hi.h[e + 1] = __float2bfloat16_rn(x1[e + 1] * cs.z + x0[e + 1] * cs.w);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      lo.h[e] = __float2bfloat16_rn(x0[e]);
+      hi.h[e] = __float2bfloat16_rn(x1[e]);
+    }
+  }
+  *reinterpret_cast<uint4 *>(dst + c0) = lo.u;
+  *reinterpret_cast<uint4 *>(dst + c1) = hi.u;
+}
+
 cudaError_t launch_rope_scatter(int dtype, const void *qkv_in, bool in_f32, bool zero_in, int M,
                                 const int32_t *rows, int n_ctx, int n_heads, int head_dim,
                                 const float2 *rope, void *q_out, void *ck, void *cv,
                                 cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   if (M > 65535) return cudaErrorInvalidValue;
+  if (dtype == SL_BF16 && in_f32 && zero_in && head_dim % 16 == 0) {
+    const int threads = 3 * n_heads * (head_dim / 16);
+    return launch_k(rope_scatter_ws_kernel, dim3((threads + 255) / 256, M), 256, 0, s,
+                    (float *)qkv_in, M, rows, n_ctx, n_heads, head_dim, rope, (bf16 *)q_out,
+                    (bf16 *)ck, (bf16 *)cv);
+  }
   const dim3 grid((3 * n_heads * head_dim / 2 + 255) / 256, M);
   if (dtype == SL_BF16) {
     if (in_f32)
@@ -225,10 +284,38 @@ __global__ void __launch_bounds__(256) swiglu_kernel(Tin *__restrict__ ws, bool 
   }
 }
 
+// The same from the fp32 split-K workspace into bf16, eight columns per thread
+// (F % 8 == 0): 16-byte loads and clearing stores, one 16-byte bf16 store.
+__global__ void __launch_bounds__(256) swiglu_ws_kernel(float *__restrict__ ws, int M, int F,
+                                                        bf16 *__restrict__ act) {
+  const int j = blockIdx.y;
+  const int c = (blockIdx.x * 256 + threadIdx.x) * 8;
+  pdl_wait();
+  pdl_trigger();
+  if (c >= F) return;
+  float4 *g = reinterpret_cast<float4 *>(ws + (size_t)j * 2 * F + c);
+  float4 *u = reinterpret_cast<float4 *>(ws + (size_t)j * 2 * F + F + c);
+  const float4 g0 = g[0], g1 = g[1], u0 = u[0], u1 = u[1];
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  g[0] = z;
+  g[1] = z;
+  u[0] = z;
+  u[1] = z;
+  const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+  const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+  Pack8 o;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) o.h[e] = __float2bfloat16_rn(silu_f(gv[e]) * uv[e]);
+  *reinterpret_cast<uint4 *>(act + (size_t)j * F + c) = o.u;
+}
+
 cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, int M, int F,
                           void *act, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   if (M > 65535) return cudaErrorInvalidValue;
+  if (dtype == SL_BF16 && in_f32 && zero_in && F % 8 == 0)
+    return launch_k(swiglu_ws_kernel, dim3((F / 8 + 255) / 256, M), 256, 0, s, (float *)ws, M, F,
+                    (bf16 *)act);
   const dim3 grid((F + 1023) / 1024, M);
   if (dtype == SL_BF16) {
     if (in_f32)

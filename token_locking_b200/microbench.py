@@ -180,10 +180,44 @@ def bench_decode(args, dev):
     model = rt.Model(shape, w, "bf16")
     s = rt.Sampler(model, 1, setup.prompt_len, setup.gen_len, setup.steps, setup.block_len,
                    setup.tokens_per_step, setup.eps)
-    if not args.no_tune:
+    max_rows = setup.prompt_len + setup.gen_len
+    if args.tuning_in:
+        for kind, M, bn, sp, var in json.load(open(args.tuning_in)):
+            model.set_tuning(kind, M, bn, sp, var)
+    elif not args.no_tune:
         s.autotune()
+    if args.tuning_out:
+        json.dump([[kind, M, *model.tuning(kind, M)] for kind in range(5)
+                   for M in range(1, max_rows + 1)], open(args.tuning_out, "w"))
     prompts = torch.from_numpy(wl.np_prompts(1, setup.prompt_len, shape.vocab, shape.mask_id)).to(dev)
     s.start(prompts)
+    if args.windows:
+        # profiled windows of --steps steps starting at the given step indices;
+        # the library's own count of algorithmic GEMM bytes over the same launches
+        t, tot_b, tot_n = 0, 0.0, 0
+        for w0 in (int(x) for x in args.windows.split(",")):
+            while t < w0:
+                s.step()
+                t += 1
+            torch.cuda.synchronize()
+            model.timing_read(reset=True)
+            model.timing_enable(True)
+            torch.cuda.profiler.start()
+            for _ in range(args.steps):
+                s.step()
+                t += 1
+            torch.cuda.synchronize()
+            torch.cuda.profiler.stop()
+            tim = model.timing_read(reset=True)
+            model.timing_enable(False)
+            tot_b += tim["gemm"]["bytes"]
+            tot_n += tim["gemm"]["launches"]
+        print(json.dumps({"case": "decode_windows", "windows": args.windows, "steps": args.steps,
+                          "gemm_launches": tot_n,
+                          "gemm_algorithmic_bytes_per_launch": round(tot_b / max(1, tot_n))}))
+        return
+    for _ in range(args.skip):           # advance to later (smaller M) steps untimed
+        s.step()
     torch.cuda.synchronize()
     torch.cuda.profiler.start()          # ncu --profile-from-start off captures from here
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
@@ -195,6 +229,51 @@ def bench_decode(args, dev):
     torch.cuda.profiler.stop()
     ms = [evs[t].elapsed_time(evs[t + 1]) for t in range(args.steps)]
     print(json.dumps({"case": "decode", "steps": args.steps, "ms": [round(x, 3) for x in ms]}))
+
+
+def bench_attn(args, dev):
+    """sl_attention alone at the LLaDA-8B head layout (32 x 128), warm, for each
+    layout (queries per CTA, key split) and the library's own choice."""
+    shape = wl.LLADA8B
+    d = shape.d_model
+    tiny = wl.ModelShape(n_layers=1, d_model=d, n_heads=shape.n_heads, head_dim=128, d_ffn=256,
+                         vocab=256, mask_id=255, rope_theta=shape.rope_theta)
+    model = rt.Model(tiny, wl.torch_weights(tiny, dev), "bf16")
+    g = torch.Generator(device=dev).manual_seed(5)
+    for n_ctx in args.n_ctx:
+        cache = rt.KVCache(model, 1, n_ctx)
+        k, v = cache.view(0)
+        k.copy_(torch.randn(k.shape, device=dev, generator=g).to(torch.bfloat16))
+        v.copy_(torch.randn(v.shape, device=dev, generator=g).to(torch.bfloat16))
+        for M in args.m:
+            if M > n_ctx:
+                continue
+            act = rt.Active(1, n_ctx)
+            act.load([np.sort(np.random.default_rng(M).choice(n_ctx, M, replace=False))])
+            q = torch.randn((M, d), device=dev, generator=g).to(torch.bfloat16)
+            o = torch.empty((M, d), device=dev, dtype=torch.bfloat16)
+            for qpc, sp in ((0, 0), (16, 1), (32, 1), (64, 1), (16, 2), (16, 4), (64, 4)):
+                model.set_attention(qpc, sp)
+
+                def fn():
+                    rt.attention(model, cache, act, 0, q, o)
+
+                for _ in range(5):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(args.iters):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+                us = e0.elapsed_time(e1) * 1e3 / args.iters
+                fl = 4.0 * M * n_ctx * d
+                print(json.dumps({"case": "attn", "M": M, "n_ctx": n_ctx, "q_per_cta": qpc,
+                                  "splits": sp, "us": round(us, 2),
+                                  "TFLOPs": round(fl / us / 1e6, 1)}), flush=True)
+        cache.close()
+    model.set_attention(0, 0)
 
 
 def bench_gemm(args, dev):
@@ -278,7 +357,7 @@ def bench_gemm(args, dev):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["layer", "lock", "decode", "gemm"])
+    ap.add_argument("case", choices=["layer", "lock", "decode", "gemm", "attn"])
     ap.add_argument("--head", action="store_true")
     ap.add_argument("--gemms", default=None, help="gemm case: comma list of qkv,o,gu,down,head")
     ap.add_argument("--tiles", default=None, help="gemm case: fixed bn:variant:splits list")
@@ -286,13 +365,21 @@ def main():
     ap.add_argument("--m", default=None)
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--steps", type=int, default=8)
+    ap.add_argument("--skip", type=int, default=0, help="decode: denoising steps run before timing")
+    ap.add_argument("--windows", default=None,
+                    help="decode: profile --steps steps at each of these step indices")
+    ap.add_argument("--n-ctx", default="384,2048", help="attn: key counts")
+    ap.add_argument("--tuning-out", default=None, help="decode: save the autotuned GEMM tilings")
+    ap.add_argument("--tuning-in", default=None,
+                    help="decode: load GEMM tilings instead of autotuning (e.g. under a profiler)")
     args = ap.parse_args()
     default = {"layer": wl.LAYER_MICRO_M, "lock": wl.LOCK_MICRO_M, "decode": (),
-               "gemm": (8, 64, 128, 200, 256, 384, 1024)}[args.case]
+               "gemm": (8, 64, 128, 200, 256, 384, 1024), "attn": (8, 58, 198, 384)}[args.case]
+    args.n_ctx = [int(x) for x in args.n_ctx.split(",")]
     args.m = [int(x) for x in args.m.split(",")] if args.m else list(default)
     dev = torch.device("cuda:0")
     {"layer": bench_layer, "lock": bench_lock, "decode": bench_decode,
-     "gemm": bench_gemm}[args.case](args, dev)
+     "gemm": bench_gemm, "attn": bench_attn}[args.case](args, dev)
 
 
 if __name__ == "__main__":
