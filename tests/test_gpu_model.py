@@ -143,7 +143,7 @@ def test_autotuned_step_matches_oracle(cuda_dev):
     for kind in range(5):
         for M in (1, 100, 257, 400):
             bn, sp, var = model.tuning(kind, M)
-            assert bn in (64, 128, 256) and (sp >= 1 or sp == -1) and var in (0, 1, 2)
+            assert bn in (64, 128, 192, 256) and (sp >= 1 or sp == -1) and var in (0, 1, 2)
     act = rt.Active(B, n_ctx)
     tokens, positions, ck, cv = _state(shape, B, n_ctx, [160, 130], seed=11, dev=cuda_dev,
                                        dtype="bf16")

@@ -338,7 +338,8 @@ extern "C" sl_status sl_device_check(int clear) {
   SL_CUDA(cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost));
   if (v != 0) {
     if (clear) SL_CUDA(cudaMemset(w, 0, sizeof(int)));
-    return fail(SL_ERR_TIMEOUT, "a kernel gave up a bounded wait (code %d)", v);
+    if (v >= 1 && v <= 3) return fail(SL_ERR_TIMEOUT, "a kernel gave up a bounded wait (code %d)", v);
+    return fail(SL_ERR_CUDA, "a kernel reported device error %d (4: index out of range)", v);
   }
   return SL_OK;
 }
@@ -537,6 +538,14 @@ struct Plan {
   int pair = 0;     // 1: CTA-pair kernel (2-SM MMA)
 };
 
+// Kernel variant codes (sl_gemm_bf16, tuning tables): 0 = 1-SM 128-row units,
+// 1 = 1-SM 256-row units, 2 = CTA pair.
+static int plan_variant(const Plan &p) { return p.pair ? 2 : (p.msub == 2 ? 1 : 0); }
+static void plan_set_variant(Plan &p, int v) {
+  p.msub = v >= 1 ? 2 : 1;
+  p.pair = v == 2 ? 1 : 0;
+}
+
 // Choose the tile shape (BN, 128 or 256 rows per unit) and K split of one
 // GEMM by a small cost model: the kernel time is the largest of the weight
 // stream from HBM (read once), the operand traffic from L2 into the SMs (every
@@ -729,8 +738,8 @@ static Plan plan_kind(const sl_model *m, int kind, int M, int ns) {
   const int bkt = tune_bucket(M);
   if (bkt >= 0 && bkt < (int)m->tuned[kind].size() && m->tuned[kind][bkt][0] > 0) {
     const auto &t = m->tuned[kind][bkt];
-    Plan pl{t[0], t[1], t[2] == 1 ? 2 : 1, 0.0};
-    pl.pair = t[2] == 2 ? 1 : 0;
+    Plan pl{t[0], t[1], 1, 0.0};
+    plan_set_variant(pl, t[2]);
     return pl;
   }
   const sl_config &cfg = m->cfg;
@@ -1042,8 +1051,9 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   }
   if (M == 0) return SL_OK;
   const int ns = sm_count();
-  if (variant < 0 || variant > 2) return fail(SL_ERR_INVALID, "sl_gemm_bf16: variant must be 0, 1 or 2");
-  int msub = variant == 0 ? 1 : 2;
+  if (variant < 0 || variant > 2)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: variant must be 0, 1 or 2");
+  int msub = variant >= 1 ? 2 : 1;
   int pair = variant == 2 ? 1 : 0;
   if (bn == 0) {
     Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID ? SPLIT_RESID
@@ -1157,8 +1167,8 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
       double best_ms = 1e30;
       std::array<int, 3> best = {0, 1, 1};
       for (int variant = 0; variant <= 2; ++variant) {
-        const int msub = variant == 0 ? 1 : 2;
-        if (variant > 0 && Mb <= 128) continue;
+        const int msub = variant >= 1 ? 2 : 1;
+        if (variant >= 1 && Mb <= 128) continue;
         for (int bn : {256, 192, 128, 64}) {
           if (N % bn || (kind == G_QKV && bn < 128)) continue;
           if (variant == 2 && bn < 128) continue;
@@ -1178,7 +1188,7 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
               if (units > 24L * m->num_sms) continue;
             }
             Plan pl{bn, ss, msub, 0.0};
-            pl.pair = variant == 2 ? 1 : 0;
+            plan_set_variant(pl, variant);
             // each repetition is followed by a small kernel (an RMSNorm, as in
             // the layer) so that successive GEMMs cannot overlap each other
             // through programmatic launch and flatter tilings with few CTAs
@@ -1227,7 +1237,7 @@ extern "C" sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn
   const Plan p = plan_kind(m, kind, M, m->num_sms);
   *bn = p.bn;
   *splits = p.splits;
-  *variant = p.pair ? 2 : (p.msub == 2 ? 1 : 0);
+  *variant = plan_variant(p);
   return SL_OK;
 }
 
