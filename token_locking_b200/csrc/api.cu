@@ -129,11 +129,6 @@ struct sl_kv_cache {
   // workspace as [M][3d] and [M][2f] (fp32), gate/up product act (bf16)
   TmaMat out_h, out_ws3, out_ws2, out_act;
   TmaMat out_hx{};            // a caller's hidden states (sl_layer_forward), by pointer
-  // step chain: arrival counter in device memory and the value it reaches once
-  // every kernel launched so far has arrived (reset at the start of each step)
-  unsigned long long *chain = nullptr;
-  unsigned long long chain_val = 0;
-  bool chain_tail = false;    // the last kernel launched arrives on the chain
   int map_rows = -1;
 };
 
@@ -354,7 +349,7 @@ extern "C" void sl_kv_cache_destroy(sl_kv_cache *c) {
   if (!c) return;
   for (void *p : c->k) cudaFree(p);
   for (void *p : c->v) cudaFree(p);
-  void *ps[] = {c->rope, c->h, c->a, c->qkv, c->q, c->o, c->act, c->ws, c->attn_ws, c->chain};
+  void *ps[] = {c->rope, c->h, c->a, c->qkv, c->q, c->o, c->act, c->ws, c->attn_ws};
   for (void *p : ps)
     if (p) cudaFree(p);
   delete c;
@@ -393,9 +388,7 @@ extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
        alloc((void **)&c->ws, rows * wsc * 4);
   if (ok && cfg.dtype == SL_BF16) {
     ok = alloc((void **)&c->attn_ws, attn_bf16_workspace_bytes(c->max_rows, cfg.n_heads,
-                                                               c->attn_max_splits)) &&
-         alloc((void **)&c->chain, sizeof(unsigned long long)) &&
-         cudaMemset(c->chain, 0, sizeof(unsigned long long)) == cudaSuccess;
+                                                               c->attn_max_splits));
   }
   if (ok) {
     // rotary table in double precision: angle = pos * theta^(-2i/dh)
@@ -815,8 +808,7 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
 //   G_DN   act x Wd^T, added to the residual h
 //   G_HD   RMSNorm(h) x W_out^T -> logits[rows]
 static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int l, int kind,
-                          const Plan &pl, int M, float *h, void *logits, cudaStream_t s,
-                          const ChainArgs *chain = nullptr, int *ctas = nullptr) {
+                          const Plan &pl, int M, float *h, void *logits, cudaStream_t s) {
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn, V = cfg.vocab, H = cfg.n_heads;
   const double Md = (double)M;
@@ -827,8 +819,6 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
   g.splits = pl.splits;
   g.msub = pl.msub;
   g.pair = pl.pair;
-  if (chain) g.chain = *chain;
-  g.ctas = ctas;
   const int bbox = pl.pair ? pl.bn / 2 : pl.bn;    // weight rows per TMA box
   double bytes = 0, flops = 0;
   switch (kind) {
@@ -935,39 +925,13 @@ static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, fl
   const int d = cfg.d_model;
   const sl_layer_weights &lw = m->layers[l];
   sl_status st;
-  int ctas = 0;
-  // (previous layer's down projection ->) RMSNorm -> fused QKV
-  if (c->chain_tail) {
-    const ChainArgs ch_n{c->chain, c->chain_val, 1};
-    SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s, &ch_n, m->err));
-    c->chain_val += M;
-    const ChainArgs ch_q{c->chain, c->chain_val, 0};
-    if ((st = run_gemm(m, c, a->rows, l, G_QKV, pl.qkv, M, h, nullptr, s, &ch_q)) != SL_OK)
-      return st;
-  } else {
-    SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s));
-    if ((st = run_gemm(m, c, a->rows, l, G_QKV, pl.qkv, M, h, nullptr, s)) != SL_OK) return st;
-  }
-  c->chain_tail = false;
+  SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s));
+  if ((st = run_gemm(m, c, a->rows, l, G_QKV, pl.qkv, M, h, nullptr, s)) != SL_OK) return st;
   if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, s)) != SL_OK) return st;
-  // output projection -> RMSNorm -> gate/up hand over through the step chain
-  const ChainArgs ch_o{c->chain, 0, 1};
-  if ((st = run_gemm(m, c, a->rows, l, G_O, pl.o, M, h, nullptr, s, &ch_o, &ctas)) != SL_OK)
-    return st;
-  c->chain_val += ctas;
-  const ChainArgs ch_n{c->chain, c->chain_val, 1};
-  SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.ffn_norm, d, cfg.rms_eps, M, c->a, s, &ch_n, m->err));
-  c->chain_val += M;
-  const ChainArgs ch_g{c->chain, c->chain_val, 0};
-  if ((st = run_gemm(m, c, a->rows, l, G_GU, pl.gu, M, h, nullptr, s, &ch_g)) != SL_OK) return st;
-  // down projection arrives for the next RMSNorm (next layer, or the final one)
-  const ChainArgs ch_d{c->chain, 0, 1};
-  ctas = 0;
-  if ((st = run_gemm(m, c, a->rows, l, G_DN, pl.dn, M, h, nullptr, s, &ch_d, &ctas)) != SL_OK)
-    return st;
-  c->chain_val += ctas;
-  c->chain_tail = true;
-  return SL_OK;
+  if ((st = run_gemm(m, c, a->rows, l, G_O, pl.o, M, h, nullptr, s)) != SL_OK) return st;
+  SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.ffn_norm, d, cfg.rms_eps, M, c->a, s));
+  if ((st = run_gemm(m, c, a->rows, l, G_GU, pl.gu, M, h, nullptr, s)) != SL_OK) return st;
+  return run_gemm(m, c, a->rows, l, G_DN, pl.dn, M, h, nullptr, s);
 }
 
 static sl_status check_pair(sl_model *m, sl_kv_cache *c, sl_active *a, const char *who) {
@@ -994,11 +958,6 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   cudaStream_t s = (cudaStream_t)stream;
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, V = cfg.vocab;
-  if (c->chain) {
-    SL_CUDA(cudaMemsetAsync(c->chain, 0, sizeof(unsigned long long), s));
-    c->chain_val = 0;
-    c->chain_tail = false;
-  }
   SL_CUDA(launch_gather_embed(cfg.dtype, d_tokens, a->rows, M, m->tok_emb, d, c->h, s));
   if (cfg.dtype == SL_F32) {
     for (int l = 0; l < cfg.n_layers; ++l)
@@ -1015,14 +974,8 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   const BfPlans pl = plans_for(m, M, m->num_sms);
   for (int l = 0; l < cfg.n_layers; ++l)
     if ((st = layer_bf16(m, c, a, l, c->h, M, seqs, pl, s)) != SL_OK) return st;
-  // last down projection -> final RMSNorm -> LM head over the step chain
-  const ChainArgs ch_n{c->chain, c->chain_tail ? c->chain_val : 0, 1};
-  SL_CUDA(launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s, &ch_n, m->err));
-  c->chain_val += M;
-  const ChainArgs ch_h{c->chain, c->chain_val, 0};
-  c->chain_tail = false;
-  if ((st = run_gemm(m, c, a->rows, 0, G_HD, pl.hd, M, c->h, d_logits, s, &ch_h)) != SL_OK)
-    return st;
+  SL_CUDA(launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
+  if ((st = run_gemm(m, c, a->rows, 0, G_HD, pl.hd, M, c->h, d_logits, s)) != SL_OK) return st;
   // the previous step's timing events completed before this step was planned
   if (m->timing) timing_harvest(m, false);
   return SL_OK;
@@ -1046,9 +999,6 @@ extern "C" sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a,
   if ((st = ensure_maps(c, M)) != SL_OK) return st;
   AttnSeqs seqs;
   fill_seqs(seqs, a, counts);
-  SL_CUDA(cudaMemsetAsync(c->chain, 0, sizeof(unsigned long long), s));
-  c->chain_val = 0;
-  c->chain_tail = false;
   return layer_bf16(m, c, a, layer, d_h, M, seqs, plans_for(m, M, m->num_sms), s);
 }
 

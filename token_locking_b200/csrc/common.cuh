@@ -10,7 +10,7 @@ typedef __nv_bfloat16 bf16;
 
 // Error codes a kernel writes into the device error word.
 enum : int { DEV_OK = 0, DEV_TIMEOUT_PRODUCER = 1, DEV_TIMEOUT_MMA = 2, DEV_TIMEOUT_EPI = 3,
-             DEV_BAD_INDEX = 4, DEV_TIMEOUT_CHAIN = 5 };
+             DEV_BAD_INDEX = 4 };
 
 // Spin-wait limit for every wait on a barrier a kernel of this library can
 // issue: after this many nanoseconds of globaltimer the wait gives up, the
@@ -57,48 +57,6 @@ __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// ------------------------------------------------------------ step chain ---
-// griddepcontrol.wait returns a few microseconds after the predecessor's last
-// CTA has ended (grid completion and its memory flush).  Inside a step the
-// kernels can hand over sooner through an arrival counter in device memory:
-// every CTA of a kernel adds 1 once its writes are done (release), and the next
-// kernel, already resident through programmatic launch, spins (acquire) until
-// the count reaches the target the host computed from the grids it launched.
-// Programmatic launch starts a kernel only after every CTA of its predecessor
-// has triggered, so the predecessor is entirely resident while it is awaited.
-struct ChainArgs {
-  unsigned long long *ctr;    // arrival counter (null: no chain)
-  unsigned long long wait;    // 0: griddepcontrol.wait; else spin until *ctr >= wait
-  int arrive;                 // 1: every CTA adds 1 at its end
-};
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-// Bounded: false once WAIT_LIMIT_NS passed without the target.  A counter
-// wait is followed by a proxy fence so that TMA reads see the data.
-__device__ __forceinline__ bool chain_wait(const ChainArgs &c) {
-  if (c.wait == 0 || !c.ctr) {
-    pdl_wait();
-    return true;
-  }
-  if (ld_acquire_u64(c.ctr) < c.wait) {
-    const unsigned long long t0 = global_ns();
-    while (ld_acquire_u64(c.ctr) < c.wait)
-      if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
-  }
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  return true;
-}
-// Thread 0 of a CTA, after a barrier that follows all of the CTA's writes.
-__device__ __forceinline__ void chain_arrive(const ChainArgs &c) {
-  if (!c.ctr || !c.arrive) return;
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  __threadfence();
-  asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(c.ctr) : "memory");
 }
 
 // 8 x bf16 <-> 16-byte vector

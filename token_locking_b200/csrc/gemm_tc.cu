@@ -283,7 +283,6 @@ struct TcParams {
   int m_tiles, n_tiles, splits, kb_per_split, kblocks, units;
   int stream_k;            // 1: balanced split of the tile x K-block space (see WorkIter)
   int tma_out;             // 1: RESID/ACCUM/SWIGLU tiles leave through out_map (see epilogue)
-  ChainArgs chain;         // dependency on the previous kernel of the step
   void *out;
   int ldo;
   int ffn;                 // SWIGLU/ACCUM-swiglu: F (columns of one half)
@@ -635,12 +634,12 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           load_b<BN>(p, sb, nt, kb0 + i, full_bar(i));
         }
       }
-      bool ok = chain_wait(p.chain);
-      if (!ok) atomicExch(p.err, DEV_TIMEOUT_CHAIN);
+      pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
       int last_stage = -1;
       uint32_t last_phase = 0;
+      bool ok = true;
       bool first = true;
       WorkIter it(p, blockIdx.x, gridDim.x);
       while (ok && it.next(p, mt, nt, kb0, kb1)) {
@@ -722,13 +721,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // outputs may be in use by the previous kernel
-    if (p.chain.wait == 0) {
-      pdl_wait();
-    } else {
-      if (lane == 0 && !chain_wait(p.chain)) atomicExch(p.err, DEV_TIMEOUT_CHAIN);
-      __syncwarp();
-    }
+    pdl_wait();                             // outputs may be in use by the previous kernel
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -766,7 +759,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (threadIdx.x == 0) chain_arrive(p.chain);
   if (warp == 1) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -859,11 +851,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
           load_b_half(sbase + i * STAGE_BYTES + A_BYTES, nt, kb0 + i, map_to_rank(full_bar(i), 0));
         }
       }
-      bool ok = chain_wait(p.chain);
-      if (!ok) atomicExch(p.err, DEV_TIMEOUT_CHAIN);
+      pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
-      bool first = true;
+      bool ok = true, first = true;
       WorkIter it(p, pair, n_pairs);
       while (ok && it.next(p, mt, nt, kb0, kb1)) {
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -927,12 +918,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
     }
   } else {
     // ------------------------------------------------- epilogue (both CTAs)
-    if (p.chain.wait == 0) {
-      pdl_wait();
-    } else {
-      if (lane == 0 && !chain_wait(p.chain)) atomicExch(p.err, DEV_TIMEOUT_CHAIN);
-      __syncwarp();
-    }
+    pdl_wait();
     const int q = warp & 3;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -968,7 +954,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
   __syncthreads();
   cluster_sync_all();
   tc_fence_after();
-  if (threadIdx.x == 0) chain_arrive(p.chain);
   if (warp == 1) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -996,7 +981,7 @@ static cudaError_t run_tc(const TcParams &p, int grid, cudaStream_t s) {
 // `pairs` CTA pairs, capped at the number of pairs the GPU holds at once
 // (a GPC with an odd number of usable SMs leaves one SM out of the pairing).
 template <int BN, int STAGES, int EPI>
-static cudaError_t run_tc2(const TcParams &p, int pairs, cudaStream_t s, int *ctas) {
+static cudaError_t run_tc2(const TcParams &p, int pairs, cudaStream_t s) {
   constexpr int SMEM = STAGES * (16384 + (BN / 2) * 128) + EPI_STAGING_BYTES + 256 + 1024;
   static int max_pairs = 0;
   if (max_pairs == 0) {
@@ -1021,18 +1006,17 @@ static cudaError_t run_tc2(const TcParams &p, int pairs, cudaStream_t s, int *ct
     max_pairs = n;
   }
   if (pairs > max_pairs) pairs = max_pairs;
-  if (ctas) *ctas = 2 * pairs;
   return launch_k_cluster2(gemm_tc2_kernel<BN, STAGES, EPI>, 2 * pairs, 192, SMEM, s, p);
 }
 
 template <int BN, int STAGES>
-static cudaError_t run_epi2(int epi, const TcParams &p, int pairs, cudaStream_t s, int *ctas) {
+static cudaError_t run_epi2(int epi, const TcParams &p, int pairs, cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE: return run_tc2<BN, STAGES, EPI_STORE>(p, pairs, s, ctas);
-    case EPI_RESID: return run_tc2<BN, STAGES, EPI_RESID>(p, pairs, s, ctas);
-    case EPI_SWIGLU: return run_tc2<BN, STAGES, EPI_SWIGLU>(p, pairs, s, ctas);
-    case EPI_ACCUM: return run_tc2<BN, STAGES, EPI_ACCUM>(p, pairs, s, ctas);
-    case EPI_QKV: return run_tc2<BN, STAGES, EPI_QKV>(p, pairs, s, ctas);
+    case EPI_STORE: return run_tc2<BN, STAGES, EPI_STORE>(p, pairs, s);
+    case EPI_RESID: return run_tc2<BN, STAGES, EPI_RESID>(p, pairs, s);
+    case EPI_SWIGLU: return run_tc2<BN, STAGES, EPI_SWIGLU>(p, pairs, s);
+    case EPI_ACCUM: return run_tc2<BN, STAGES, EPI_ACCUM>(p, pairs, s);
+    case EPI_QKV: return run_tc2<BN, STAGES, EPI_QKV>(p, pairs, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -1087,7 +1071,6 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;   // no empty split
   p.units = p.m_tiles * p.n_tiles * p.splits;
   p.stream_k = stream_k ? 1 : 0;
-  p.chain = a.chain;
   if ((a.epi == EPI_RESID || a.epi == EPI_ACCUM) && !a.OUT) return cudaErrorInvalidValue;
   if (a.OUT && (a.epi == EPI_RESID || a.epi == EPI_ACCUM ||
                 (a.epi == EPI_SWIGLU && (bn / 2) % 64 == 0))) {
@@ -1110,13 +1093,12 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   if (pair_mma) {
     const long long work = stream_k ? sk_iters : p.units;
     const int pairs = work < num_sms / 2 ? (int)work : num_sms / 2;
-    if (bn == 256) return run_epi2<256, 6>(a.epi, p, pairs, s, a.ctas);
-    if (bn == 192) return run_epi2<192, 7>(a.epi, p, pairs, s, a.ctas);
-    return run_epi2<128, 6>(a.epi, p, pairs, s, a.ctas);
+    if (bn == 256) return run_epi2<256, 6>(a.epi, p, pairs, s);
+    if (bn == 192) return run_epi2<192, 7>(a.epi, p, pairs, s);
+    return run_epi2<128, 6>(a.epi, p, pairs, s);
   }
   const long long work = stream_k ? sk_iters : p.units;
   int grid = work < num_sms ? (int)work : num_sms;
-  if (a.ctas) *a.ctas = grid;
   if (msub == 2) {
     switch (bn) {
       case 256: return run_epi<256, 3, 2>(a.epi, p, grid, s);

@@ -77,8 +77,7 @@ enum GemmEpi : int {
 cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
                                 const void *emb, int d, float *h, cudaStream_t s);
 cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
-                           void *out, cudaStream_t s,
-                           const ChainArgs *chain = nullptr, int *err = nullptr);
+                           void *out, cudaStream_t s);
 // qkv_in: [M][3d] (in_f32 ? float : dtype).  q_out [M][d] dtype; ck/cv: the layer's
 // cache [B*n_ctx][d]; rope: [n_ctx][head_dim/2] (cos, sin).  zero_in: clear the
 // fp32 input after reading (split-K workspace).
@@ -136,8 +135,6 @@ struct TcGemmArgs {
   int b_swiglu;          // B tile = BN/2 gate rows (B[0]) | BN/2 up rows (B[1])
   int msub;              // 1: 128-row units; 2: 256-row units (two accumulators per B tile)
   int pair;              // 1: CTA-pair kernel (2-SM MMA, 256-row units, B maps with BN/2 boxes)
-  ChainArgs chain;       // dependency on the previous kernel of the step (default: none)
-  int *ctas;             // out: CTAs launched (the chain's arrivals), or null
   const TmaMat *OUT;     // RESID/ACCUM (fp32) or SWIGLU (bf16) output descriptor from
                          // tma_encode_out: tiles leave by TMA reduce-add / store (optional)
   void *out;             // STORE/SWIGLU: dtype out; RESID: fp32 resid; ACCUM: fp32 ws

@@ -71,18 +71,11 @@ template <int VPT>
 __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float *__restrict__ h,
                                                            const bf16 *__restrict__ g, int d,
                                                            float eps, int M,
-                                                           bf16 *__restrict__ out,
-                                                           ChainArgs chain, int *err) {
+                                                           bf16 *__restrict__ out) {
   const int j = blockIdx.x;
   if (j >= M) return;
-  if (chain.wait == 0) {
-    pdl_wait();
-    pdl_trigger();
-  } else {
-    pdl_trigger();
-    if (threadIdx.x == 0 && !chain_wait(chain) && err) atomicExch(err, DEV_TIMEOUT_CHAIN);
-    __syncthreads();
-  }
+  pdl_wait();
+  pdl_trigger();
   const float4 *x = reinterpret_cast<const float4 *>(h + (size_t)j * d);
   const int n4 = d >> 2;
   float4 v[VPT];
@@ -115,29 +108,20 @@ __global__ void __launch_bounds__(256) rmsnorm_bf16_kernel(const float *__restri
       o2[i] = oo.u;
     }
   }
-  if (chain.arrive) {
-    __syncthreads();
-    if (threadIdx.x == 0) chain_arrive(chain);
-  }
 }
 
 cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
-                           void *out, cudaStream_t s, const ChainArgs *chain, int *dev_err) {
+                           void *out, cudaStream_t s) {
   if (dtype == SL_BF16 && d % 4 == 0 && d <= 8 * 1024) {
     if (M <= 0) return cudaSuccess;
     const int vpt = (d / 4 + 255) / 256;
     const bf16 *gb = (const bf16 *)g;
     bf16 *ob = (bf16 *)out;
-    const ChainArgs ch = chain ? *chain : ChainArgs{nullptr, 0, 0};
-    if (vpt <= 1)
-      return launch_k(rmsnorm_bf16_kernel<1>, M, 256, 0, s, h, gb, d, eps, M, ob, ch, dev_err);
-    if (vpt <= 2)
-      return launch_k(rmsnorm_bf16_kernel<2>, M, 256, 0, s, h, gb, d, eps, M, ob, ch, dev_err);
-    if (vpt <= 4)
-      return launch_k(rmsnorm_bf16_kernel<4>, M, 256, 0, s, h, gb, d, eps, M, ob, ch, dev_err);
-    return launch_k(rmsnorm_bf16_kernel<8>, M, 256, 0, s, h, gb, d, eps, M, ob, ch, dev_err);
+    if (vpt <= 1) return launch_k(rmsnorm_bf16_kernel<1>, M, 256, 0, s, h, gb, d, eps, M, ob);
+    if (vpt <= 2) return launch_k(rmsnorm_bf16_kernel<2>, M, 256, 0, s, h, gb, d, eps, M, ob);
+    if (vpt <= 4) return launch_k(rmsnorm_bf16_kernel<4>, M, 256, 0, s, h, gb, d, eps, M, ob);
+    return launch_k(rmsnorm_bf16_kernel<8>, M, 256, 0, s, h, gb, d, eps, M, ob);
   }
-  if (chain && chain->wait) return cudaErrorInvalidValue;   // the chain is bf16-only
   cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   int th = d >= 1024 ? 512 : 128;
