@@ -30,6 +30,7 @@ import argparse
 import json
 import math
 import os
+import tempfile
 import subprocess
 import sys
 import time
@@ -69,6 +70,24 @@ def make_setup(name: str, eps, scripted: bool) -> wl.SamplerSetup:
         raise SystemExit(f"unknown workload {name}")
     s.validate()
     return s
+
+
+DATA_DESC = "synthetic (random-init N(0,0.02) weights, uniform random prompt ids)"
+
+
+def workload_config(args, setup: wl.SamplerSetup, world: int) -> dict:
+    """The `config` object of the JSON line (the same for both arms)."""
+    T = setup.steps
+    return {"workload": f"{args.workload}: LLaDA-8B shape, batch {setup.batch}, "
+                        f"{setup.prompt_len} prompt + {setup.gen_len} masked "
+                        f"(N={setup.n_ctx}), {T} steps, blocks of {setup.block_len}, "
+                        f"{setup.tokens_per_step} token(s)/step, eps={setup.eps}"
+                        + (f", gate q={setup.gate_q}" if setup.gate_q >= 0 else "")
+                        + (", scripted lock schedule" if setup.scripted else ""),
+            "bench_step": f"one full decode ({T} denoising steps)",
+            "global_batch": world * setup.batch, "seq_len": setup.n_ctx,
+            "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (15 GB of weights streamed per step)"}
 
 
 def gemm_traffic():
@@ -398,17 +417,8 @@ def run_ours(args, rank: int, world: int):
             "scaling": "weak",
             "vs_baseline": None,
             "dtype": "bf16",
-            "data": "synthetic (random-init N(0,0.02) bf16 weights, uniform random prompt ids)",
-            "config": {"workload": f"{args.workload}: LLaDA-8B shape, batch {setup.batch}, "
-                                   f"{setup.prompt_len} prompt + {setup.gen_len} masked "
-                                   f"(N={setup.n_ctx}), {T} steps, blocks of {setup.block_len}, "
-                                   f"{setup.tokens_per_step} token(s)/step, eps={setup.eps}"
-                                   + (f", gate q={setup.gate_q}" if setup.gate_q >= 0 else "")
-                                   + (", scripted lock schedule" if setup.scripted else ""),
-                       "bench_step": f"one full decode ({T} denoising steps)",
-                       "global_batch": world * setup.batch, "seq_len": setup.n_ctx,
-                       "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (15 GB of weights streamed per step)"},
+            "data": DATA_DESC,
+            "config": workload_config(args, setup, world),
             "gen_tok_s": round(gen_tokens / (ms / 1e3), 3),
             "e2e": {"value": round(e2e_value, 3), "unit": "denoise steps/s",
                     "gen_tok_s": round(gen_tokens / (e2e_ms / 1e3), 3),
@@ -467,7 +477,7 @@ def run_reference(args, rank: int, world: int):
             "value": round(value, 6), "unit": "denoise steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": args.workload, "parallelism": "cpu"},
+            "data": DATA_DESC, "config": workload_config(args, setup, world),
             "cpu_baseline": {"value": round(value, 6), "unit": "denoise steps/s", "cores": thr,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 6), "unit": "denoise steps/s",
@@ -484,7 +494,8 @@ def main():
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--scripted", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--out-dir", default=os.path.join(ROOT, "gpurun_out"))
+    ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "surelock_bench"),
+                    help="where the per-rank clock samples (CSV) are written")
     args = ap.parse_args()
     os.makedirs(args.out_dir, exist_ok=True)
     rank = int(os.environ.get("RANK", "0"))

@@ -13,7 +13,7 @@ What the pages fix:
     (gist.science/nl section 2 "Complexiteitsvermindering"; gist.science/it
     section 2 "Complessita Computazionale").
 
-Readings where the pages are silent (all listed in the design doc):
+Readings where the pages are silent (the plainest reading consistent with them):
   * RMSNorm with eps = rms_eps (1e-5) and per-channel gains; no biases anywhere;
     untied LM head; SwiGLU FFN  W_down( silu(W_gate b) * (W_up b) ).
   * Rotary embedding in rotate-half form on pairs (i, i + head_dim/2) with

@@ -18,7 +18,7 @@ Diffusion-LM Decoding"):
     (Paper-Notes, "permanent locking", core idea).
   * The comparison sampler is "the same sampler without locking" (Abstract).
 
-Readings where the pages are silent (listed in the design doc):
+Readings where the pages are silent (the plainest reading consistent with them):
   R4  "unmasked" means not [MASK] in the step's input x_t; prompt positions count.
   R5  no previous posterior at t = 0, so nothing locks at t = 0.
   R6  eps <= 0 disables locking (the pages' test D <= eps would fire at D = 0).
