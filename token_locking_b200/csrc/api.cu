@@ -1199,17 +1199,24 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
                                              c->a, s);
               return e == cudaSuccess ? SL_OK : cuda_fail(e, "sl_model_autotune: spacer");
             };
+            // three blocks of three back-to-back repetitions; the candidate's
+            // time is the median block (a stray slow block does not decide)
             if ((st = launch()) != SL_OK) break;
-            cudaEventRecord(e0, s);
-            for (int it = 0; it < 3 && st == SL_OK; ++it) st = launch();
-            cudaEventRecord(e1, s);
-            if (st != SL_OK) break;
-            if (cudaEventSynchronize(e1) != cudaSuccess) {
-              st = cuda_fail(cudaGetLastError(), "sl_model_autotune: timing");
-              break;
+            float blocks[3] = {0.f, 0.f, 0.f};
+            for (int blk = 0; blk < 3 && st == SL_OK; ++blk) {
+              cudaEventRecord(e0, s);
+              for (int it = 0; it < 3 && st == SL_OK; ++it) st = launch();
+              cudaEventRecord(e1, s);
+              if (st != SL_OK) break;
+              if (cudaEventSynchronize(e1) != cudaSuccess) {
+                st = cuda_fail(cudaGetLastError(), "sl_model_autotune: timing");
+                break;
+              }
+              cudaEventElapsedTime(&blocks[blk], e0, e1);
             }
-            float ms = 0.f;
-            cudaEventElapsedTime(&ms, e0, e1);
+            if (st != SL_OK) break;
+            std::sort(blocks, blocks + 3);
+            const float ms = blocks[1];
             if (ms < best_ms) {
               best_ms = ms;
               best = {bn, ss, variant};
