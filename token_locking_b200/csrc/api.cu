@@ -556,9 +556,11 @@ static void plan_set_variant(Plan &p, int v) {
 enum SplitKind { SPLIT_NONE = 0, SPLIT_RESID = 1, SPLIT_ACCUM = 2 };
 
 // heads: the unsplit QKV epilogue rotates whole 128-column heads, so unsplit
-// plans keep bn a multiple of 128.
+// plans keep bn a multiple of 128.  seg: the weight is several matrices of
+// `seg` rows stacked (Q|K|V); a tile takes its rows from one of them, so bn
+// must divide seg.
 Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, int min_bn = 64,
-               bool heads = false) {
+               bool heads = false, int seg = 0) {
   const double bw_hbm = 6.5e12, bw_l2 = 9.0e12, peak = 1.6e15;
   const int kblocks = K / 64;
   Plan best{0, 1, 1, 1e30};
@@ -570,7 +572,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
     const int bns[4] = {256, 192, 128, 64};
     for (int bi = 0; bi < 4; ++bi) {
       const int bn = bns[bi];
-      if (N % bn || bn < min_bn) continue;
+      if (N % bn || bn < min_bn || (seg && seg % bn)) continue;
       if (swiglu && (N / 2) % (bn / 2)) continue;
       const bool single_acc = 2 * msub * bn > 512;
       const double mma_eff = bn >= 192 ? 1.0 : (bn == 128 ? 0.8 : 0.5);
@@ -602,7 +604,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
     const int mt = (M + 255) / 256;
     const double rows_live = std::min(M, 256);
     for (int bn : {256, 192, 128}) {
-      if (N % bn || bn < min_bn) continue;
+      if (N % bn || bn < min_bn || (seg && seg % bn)) continue;
       if (swiglu && (N / 2) % (bn / 2)) continue;
       const int max_s = split_kind != SPLIT_NONE ? std::min(32, std::max(1, kblocks / 4)) : 1;
       for (int sp = 1; sp <= max_s; ++sp) {
@@ -639,7 +641,7 @@ Plan plan_gemm(int M, int N, int K, int split_kind, int num_sms, bool swiglu, in
       const int mt = (M + rows_unit - 1) / rows_unit;
       const double rows_live = std::min(M, rows_unit);
       for (int bn : {256, 192, 128}) {
-        if (N % bn || bn < min_bn) continue;
+        if (N % bn || bn < min_bn || (seg && seg % bn)) continue;
         if (swiglu && (N / 2) % (bn / 2)) continue;
         if (variant == 1 && 4 * bn > 512) continue;      // keep double-buffered accumulators
         const long tiles = (long)mt * (N / bn);
@@ -745,7 +747,7 @@ static Plan plan_kind(const sl_model *m, int kind, int M, int ns) {
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn;
   switch (kind) {
-    case G_QKV: return plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128, true);
+    case G_QKV: return plan_gemm(M, 3 * d, d, SPLIT_ACCUM, ns, false, 128, true, d);
     case G_O: return plan_gemm(M, d, d, SPLIT_RESID, ns, false);
     case G_GU: return plan_gemm(M, 2 * f, d, SPLIT_ACCUM, ns, true);
     case G_DN: return plan_gemm(M, d, f, SPLIT_RESID, ns, false);
@@ -823,6 +825,8 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
   double bytes = 0, flops = 0;
   switch (kind) {
     case G_QKV: {
+      // a tile's weight rows come from one of Wq, Wk, Wv
+      if (d % pl.bn) return fail(SL_ERR_INVALID, "QKV tile width %d does not divide d_model", pl.bn);
       const auto &mp = m->maps[l];
       g.A = &c->map_a;
       g.B[0] = mp[W_Q].box(bbox);
@@ -1170,7 +1174,7 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
         const int msub = variant >= 1 ? 2 : 1;
         if (variant >= 1 && Mb <= 128) continue;
         for (int bn : {256, 192, 128, 64}) {
-          if (N % bn || (kind == G_QKV && bn < 128)) continue;
+          if (N % bn || (kind == G_QKV && (bn < 128 || d % bn))) continue;
           if (variant == 2 && bn < 128) continue;
           if (kind == G_GU && (N / 2) % (bn / 2)) continue;
           int last_ss = 0;
@@ -1267,7 +1271,7 @@ extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, i
   const int Ns[G_KINDS] = {3 * d, d, 2 * f, d, V};
   const int N = Ns[kind];
   if ((bn != 64 && bn != 128 && bn != 192 && bn != 256) || N % bn || (kind == G_GU && f % (bn / 2)) ||
-      (kind == G_QKV && (bn < 128 || (bn % 128 != 0 && splits == 1))) || variant < 0 ||
+      (kind == G_QKV && (bn < 128 || d % bn || (bn % 128 != 0 && splits == 1))) || variant < 0 ||
       variant > 2 || (variant == 2 && bn < 128) ||
       (splits < 1 && splits != -1) || (kind == G_HD && splits != 1))
     return fail(SL_ERR_INVALID, "sl_model_set_tuning: tiling not valid for this GEMM");
