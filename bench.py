@@ -250,6 +250,52 @@ def _blas_threads() -> int:
 
 
 # ------------------------------------------------------------ GPU arm ---
+class Ranks:
+    """The replicas' process group (one rank per GPU under torchrun): a barrier
+    around the timed region and the max over ranks of a time.  No data-path
+    collective exists; nccl on the GPUs, gloo where there are none."""
+
+    def __init__(self, world: int, backend: str = "nccl", device=None, timeout_s: int = 600):
+        import torch
+        self.world, self.dist = world, None
+        self.device = device if device is not None else torch.device("cpu")
+        if world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.dist is None:
+            return x
+        import torch
+        t = torch.tensor([x], device=self.device, dtype=torch.float64)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def replica_prompt_seed(rank: int) -> int:
+    """Each replica decodes its own prompts."""
+    return wl.SEED_PROMPTS + rank
+
+
+def aggregate_rate(world: int, steps_per_rank: int, ms_max: float) -> float:
+    """Denoising steps per second of the whole job: every rank's steps over the
+    slowest rank's time."""
+    return world * steps_per_rank / (ms_max / 1e3)
+
+
 def run_ours(args, rank: int, world: int):
     import torch
     from token_locking_b200 import runtime as rt
@@ -260,23 +306,8 @@ def run_ours(args, rank: int, world: int):
     setup = make_setup(args.workload, args.eps, args.scripted)
     shape = setup.shape
     T = setup.steps
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks(world, "nccl", dev)
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     weights = wl.torch_weights(shape, dev)
     torch.cuda.synchronize()
@@ -284,7 +315,7 @@ def run_ours(args, rank: int, world: int):
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, T, setup.block_len,
                    setup.tokens_per_step, setup.eps, setup.gate_q, setup.scripted)
     prompts = wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab, shape.mask_id,
-                            seed=wl.SEED_PROMPTS + rank)
+                            seed=replica_prompt_seed(rank))
     d_prompts = torch.from_numpy(prompts).to(dev)
     t_tune = time.perf_counter()
     s.autotune()                 # GEMM tilings timed on this device (setup, untimed)
@@ -369,9 +400,8 @@ def run_ours(args, rank: int, world: int):
     result = None
     if rank == 0:
         peaks = load_peaks()
-        denoise_steps = world * args.steps * T
-        value = denoise_steps / (ms / 1e3)
-        e2e_value = denoise_steps / (e2e_ms / 1e3)
+        value = aggregate_rate(world, args.steps * T, ms)
+        e2e_value = aggregate_rate(world, args.steps * T, e2e_ms)
         gen_tokens = world * args.steps * setup.batch * setup.gen_len
         # per-step roofline over the trajectory, burst peaks
         pf = peaks["bf16_tflops"] * 1e12
@@ -445,9 +475,7 @@ def run_ours(args, rank: int, world: int):
         }
     s.close()
     model.close()
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
     return result
 
 

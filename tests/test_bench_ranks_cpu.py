@@ -1,0 +1,50 @@
+"""The replica plumbing of bench.py on two CPU ranks (gloo): the barrier, the
+max over ranks of a time, per-replica prompts, the whole-job rate, and that the
+reference arm does its work on rank 0 only."""
+import json
+import os
+import socket
+import sys
+
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, out_dir: str):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    ranks = bench.Ranks(world, "gloo", timeout_s=60)
+    ranks.barrier()
+    slowest = ranks.max(10.0 + 5.0 * rank)           # this rank's "time"
+    prompts = wl.np_prompts(1, 16, 512, 511, seed=bench.replica_prompt_seed(rank))
+    ref = bench.run_reference(None, rank, world) if rank != 0 else "skipped"
+    ranks.close()
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"max": slowest, "prompts": prompts.tolist(), "ref": ref}, f)
+
+
+def test_two_gloo_ranks(tmp_path):
+    mp.spawn(_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True)
+    r0 = json.load(open(tmp_path / "rank0.json"))
+    r1 = json.load(open(tmp_path / "rank1.json"))
+    assert r0["max"] == r1["max"] == 15.0              # both ranks see the slowest time
+    assert r0["prompts"] != r1["prompts"]              # independent replicas
+    assert r1["ref"] is None                           # the reference arm: rank 0 only
+
+
+def test_aggregate_rate():
+    sys.path.insert(0, ROOT)
+    import bench
+    # 2 ranks x 3 decodes x 256 steps over the slowest rank's 1.5 s
+    assert bench.aggregate_rate(2, 3 * 256, 1500.0) == 1024.0
+    assert bench.aggregate_rate(1, 256, 1000.0) == 256.0
