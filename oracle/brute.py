@@ -53,11 +53,13 @@ def silu(x):
     return x / (1.0 + math.exp(-x))
 
 
-def forward_active(shape, w, tokens, pos, ck, cv):
+def forward_active(shape, w, tokens, pos, ck, cv, no_kv_cache=False):
     """Loop restatement of the denoiser on active rows `pos` of one sequence.
-    ck, cv: lists [L][N][d] updated in place at rows `pos`.  Returns logits."""
+    ck, cv: lists [L][N][d] updated in place at rows `pos`.  With no_kv_cache a
+    query sees the keys of the rows `pos` only.  Returns logits."""
     H, dh, d = shape.n_heads, shape.head_dim, shape.d_model
     N = len(ck[0])
+    seen = list(pos) if no_kv_cache else list(range(N))
     h = [list(map(float, w["tok_emb"][tokens[p]])) for p in pos]
     for l, lw in enumerate(w["layers"]):
         a = rmsnorm(h, lw["attn_norm"], shape.rms_eps)
@@ -76,8 +78,8 @@ def forward_active(shape, w, tokens, pos, ck, cv):
             row = []
             for hh in range(H):
                 sl = slice(hh * dh, (hh + 1) * dh)
-                row += attention_head(q[m][sl], [ck[l][n][sl] for n in range(N)],
-                                      [cv[l][n][sl] for n in range(N)])
+                row += attention_head(q[m][sl], [ck[l][n][sl] for n in seen],
+                                      [cv[l][n][sl] for n in seen])
             o.append(row)
         ow = matvec_rows(o, lw["wo"])
         h = [[h[m][i] + ow[m][i] for i in range(d)] for m in range(len(pos))]

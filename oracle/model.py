@@ -23,6 +23,12 @@ Readings where the pages are silent (the plainest reading consistent with them):
   * K/V projections are skipped for locked rows too: with a frozen block input
     they would reproduce the cached values exactly.
   * Weights are row-major [out, in]; y = x @ W.T.
+
+Ablation (Paper-Notes, ablation table, row "no KV cache": locked tokens can no
+longer be attended, so their information is lost):
+  * `no_kv_cache=True` restricts every query's keys to the active rows of its
+    sequence (their fresh k, v); the cached rows of locked positions are not
+    read at all.  Positions, and so the rotary angles, stay absolute.
 """
 from __future__ import annotations
 
@@ -81,14 +87,14 @@ def attention(q: np.ndarray, k_all: np.ndarray, v_all: np.ndarray) -> np.ndarray
 
 
 def layer_forward(shape, lw: dict, h: np.ndarray, pos: np.ndarray,
-                  ck: np.ndarray, cv: np.ndarray) -> np.ndarray:
+                  ck: np.ndarray, cv: np.ndarray, no_kv_cache: bool = False) -> np.ndarray:
     """One transformer block on the active rows of one sequence.
 
     h: [M, d] block input of the active rows at positions `pos` (ascending).
     ck, cv: [N, d] this layer's cache for the sequence; rows `pos` are
     overwritten with the fresh k, v (the scatter into C), all other rows are
-    read as they are (frozen K/V of locked positions).  Returns the block
-    output [M, d]."""
+    read as they are (frozen K/V of locked positions).  With no_kv_cache the
+    queries attend to the rows `pos` only.  Returns the block output [M, d]."""
     H, dh = shape.n_heads, shape.head_dim
     M = h.shape[0]
     a = rmsnorm(h, lw["attn_norm"], shape.rms_eps)
@@ -99,8 +105,9 @@ def layer_forward(shape, lw: dict, h: np.ndarray, pos: np.ndarray,
     k = rope(k, pos, shape.rope_theta)
     ck[pos] = k.reshape(M, H * dh)
     cv[pos] = v.reshape(M, H * dh)
-    N = ck.shape[0]
-    o = attention(q, ck.reshape(N, H, dh), cv.reshape(N, H, dh)).reshape(M, H * dh)
+    keys = pos if no_kv_cache else np.arange(ck.shape[0])
+    n = keys.shape[0]
+    o = attention(q, ck[keys].reshape(n, H, dh), cv[keys].reshape(n, H, dh)).reshape(M, H * dh)
     h = h + o @ lw["wo"].T
     b = rmsnorm(h, lw["ffn_norm"], shape.rms_eps)
     h = h + (silu(b @ lw["w_gate"].T) * (b @ lw["w_up"].T)) @ lw["w_down"].T
@@ -108,18 +115,20 @@ def layer_forward(shape, lw: dict, h: np.ndarray, pos: np.ndarray,
 
 
 def forward_active(shape, w: dict, tokens: np.ndarray, pos: np.ndarray,
-                   ck: np.ndarray, cv: np.ndarray, block_inputs: list = None) -> np.ndarray:
+                   ck: np.ndarray, cv: np.ndarray, block_inputs: list = None,
+                   no_kv_cache: bool = False) -> np.ndarray:
     """Logits z [M, V] of the active rows `pos` of one sequence.
 
     tokens: [N] current ids x_t; ck, cv: [L, N, d] the sequence's cache,
     updated in place at rows `pos`.  If block_inputs is a list, the input h of
     every block is appended to it (used to check that K/V of locked rows are
-    reproducible from their frozen block inputs)."""
+    reproducible from their frozen block inputs).  no_kv_cache: the ablation
+    in which the active rows attend to one another only."""
     h = w["tok_emb"][tokens[pos]]
     for l, lw in enumerate(w["layers"]):
         if block_inputs is not None:
             block_inputs.append(h.copy())
-        h = layer_forward(shape, lw, h, pos, ck[l], cv[l])
+        h = layer_forward(shape, lw, h, pos, ck[l], cv[l], no_kv_cache)
     hf = rmsnorm(h, w["final_norm"], shape.rms_eps)
     return hf @ w["lm_head"].T
 

@@ -33,6 +33,15 @@ Readings where the pages are silent (the plainest reading consistent with them):
   Scripted mode: instead of the KL test, lock the eligible (unmasked, with a
   previous posterior) active rows in ascending (D, position) order until the
   active count reaches a target.
+
+Ablations (Paper-Notes, ablation table):
+  * gate only ("confidence gate only"): the gate is the sole lock criterion,
+    lock_j = not masked_j and has_prev_j and u_j <= thr.  Only the KL
+    inequality is dropped; eligibility stays as in the full test, so nothing
+    locks at t = 0 and a row is first tested the step after it is unmasked.
+    eps plays no part; the gate must be on (gate_q >= 0).
+  * no KV cache ("locked tokens cannot be attended"): the denoiser's queries
+    see the keys of the active rows only (model.forward_active, no_kv_cache).
 """
 from __future__ import annotations
 
@@ -80,9 +89,15 @@ def gate_threshold(u_active: np.ndarray, q: float) -> float:
     return np.sort(u_active, kind="stable")[r]
 
 
-def lock_decision(D, u, masked, has_prev, eps: float, gate_q: float, thr):
+def lock_decision(D, u, masked, has_prev, eps: float, gate_q: float, thr,
+                  gate_only: bool = False):
     """lock_j = eps>0 and not masked_j and has_prev_j and D_j<=eps and
-    (gate off or u_j <= thr)."""
+    (gate off or u_j <= thr).  gate_only: lock_j = not masked_j and has_prev_j
+    and u_j <= thr, whatever eps and D."""
+    if gate_only:
+        if gate_q < 0:
+            raise ValueError("the gate-only criterion needs the confidence gate (gate_q >= 0)")
+        return (~masked.astype(bool)) & has_prev.astype(bool) & (u <= thr)
     if eps <= 0:
         return np.zeros(D.shape, dtype=bool)
     ok = (~masked.astype(bool)) & has_prev.astype(bool) & (D <= eps)
@@ -162,7 +177,8 @@ def lock_test(lp: np.ndarray, lp_prev: np.ndarray, has_prev: np.ndarray,
         target = setup.scripted_target(t) if n_active_target is None else n_active_target
         lock = scripted_locks(D, masked, hp, pos, lp.shape[0] - target)
     else:
-        lock = lock_decision(D, u, masked, hp, setup.eps, setup.gate_q, thr)
+        lock = lock_decision(D, u, masked, hp, setup.eps, setup.gate_q, thr,
+                             setup.gate_only)
     return {"D": D, "u": u, "conf": conf, "pred": pred, "thr": thr, "lock": lock}
 
 
@@ -178,7 +194,8 @@ def step(shape, w: dict, st: State, setup, t: int, record_block_inputs: bool = F
     for b in range(st.tokens.shape[0]):
         A = st.act[b]
         blk = [] if record_block_inputs else None
-        z = om.forward_active(shape, w, st.tokens[b], A, st.ck[b], st.cv[b], blk)
+        z = om.forward_active(shape, w, st.tokens[b], A, st.ck[b], st.cv[b], blk,
+                              setup.no_kv_cache)
         lp = log_softmax(z)
         masked_rows = st.masked[b, A].copy()
         rec = lock_test(lp, st.lp_prev[b, A], st.has_prev[b, A], masked_rows, A,

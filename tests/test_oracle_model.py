@@ -138,3 +138,69 @@ def test_kv_of_block_input_reproduces_cache():
         k, v = om.kv_of_block_input(MICRO, w["layers"][l], blk[l], pos)
         np.testing.assert_array_equal(k, ck[l])
         np.testing.assert_array_equal(v, cv[l])
+
+
+# ------------------------------------------- ablation: no KV cache ---
+
+def _micro_case(seed, N):
+    rng = np.random.default_rng(seed)
+    tokens = rng.integers(0, MICRO.vocab, N).astype(np.int32)
+    ck = rng.standard_normal((MICRO.n_layers, N, MICRO.d_model))
+    cv = rng.standard_normal((MICRO.n_layers, N, MICRO.d_model))
+    return tokens, ck, cv
+
+
+def test_no_kv_cache_matches_loops():
+    """Queries attend to the active rows only: vectorised vs scalar loops."""
+    w = _micro_weights()
+    tokens, ck, cv = _micro_case(10, 6)
+    pos = np.array([0, 2, 3, 5], dtype=np.int32)
+    bk, bv = ck.tolist(), cv.tolist()
+    z = om.forward_active(MICRO, w, tokens, pos, ck, cv, no_kv_cache=True)
+    wl_ = {k: (v.tolist() if hasattr(v, "tolist") else v) for k, v in w.items() if k != "layers"}
+    wl_["layers"] = [{k: v.tolist() for k, v in lw.items()} for lw in w["layers"]]
+    zb = brute.forward_active(MICRO, wl_, tokens.tolist(), pos.tolist(), bk, bv, no_kv_cache=True)
+    np.testing.assert_allclose(z, zb, rtol=1e-11, atol=1e-12)
+    # and it is a different computation from the method's (locked keys matter there)
+    z_full = om.forward_active(MICRO, w, tokens, pos, *_micro_case(10, 6)[1:])
+    assert np.abs(z - z_full).max() > 1e-3
+
+
+def test_no_kv_cache_contiguous_run_is_the_full_denoiser_on_it():
+    """A contiguous active run [p0, p0 + M) attending only to itself is the
+    unmodified denoiser on that sub-sequence: rotary scores depend on relative
+    positions only, so the absolute offset p0 drops out (up to rounding)."""
+    w = _micro_weights(3)
+    N, p0, M = 11, 4, 5
+    tokens, ck, cv = _micro_case(11, N)
+    pos = np.arange(p0, p0 + M, dtype=np.int32)
+    z = om.forward_active(MICRO, w, tokens, pos, ck, cv, no_kv_cache=True)
+    np.testing.assert_allclose(z, om.forward_full(MICRO, w, tokens[p0:p0 + M]), rtol=1e-10, atol=1e-10)
+
+
+def test_no_kv_cache_ignores_locked_rows_cache():
+    w = _micro_weights(4)
+    N = 8
+    tokens, ck, cv = _micro_case(12, N)
+    pos = np.array([1, 2, 6], dtype=np.int32)
+    locked = np.setdiff1d(np.arange(N), pos)
+    ck2, cv2 = ck.copy(), cv.copy()
+    ck2[:, locked] += 5.0
+    cv2[:, locked] -= 3.0
+    za = om.forward_active(MICRO, w, tokens, pos, ck.copy(), cv.copy(), no_kv_cache=True)
+    zb = om.forward_active(MICRO, w, tokens, pos, ck2.copy(), cv2.copy(), no_kv_cache=True)
+    np.testing.assert_array_equal(za, zb)
+    # the method reads those rows, so the same change moves its logits
+    zc = om.forward_active(MICRO, w, tokens, pos, ck.copy(), cv.copy())
+    zd = om.forward_active(MICRO, w, tokens, pos, ck2.copy(), cv2.copy())
+    assert np.abs(zc - zd).max() > 1e-3
+
+
+def test_no_kv_cache_with_every_row_active_is_the_method_bitwise():
+    w = _micro_weights(5)
+    N = 7
+    tokens, ck, cv = _micro_case(13, N)
+    pos = np.arange(N, dtype=np.int32)
+    np.testing.assert_array_equal(
+        om.forward_active(MICRO, w, tokens, pos, ck.copy(), cv.copy(), no_kv_cache=True),
+        om.forward_active(MICRO, w, tokens, pos, ck.copy(), cv.copy()))

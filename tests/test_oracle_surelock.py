@@ -103,6 +103,37 @@ def test_lock_decision_truth_table():
                             0.01, 0.5, 0.3).tolist() == [True]
 
 
+def test_gate_only_truth_table():
+    """Gate-only ablation: the gate alone decides among unmasked rows with a
+    previous posterior; D and eps play no part."""
+    D = np.array([0.001, 5.0, 0.001, 0.02, 0.001, 7.0])
+    u = np.array([0.1, 0.1, 0.1, 0.1, 0.9, 0.5])
+    masked = np.array([0, 0, 1, 0, 0, 0], dtype=bool)
+    hp = np.array([1, 1, 1, 0, 1, 1], dtype=bool)
+    for eps in (0.0, 0.01, -1.0):
+        assert sl.lock_decision(D, u, masked, hp, eps, 0.5, 0.5, gate_only=True).tolist() == \
+            [True, True, False, False, False, True]
+    with pytest.raises(ValueError):
+        sl.lock_decision(D, u, masked, hp, 0.01, -1, np.inf, gate_only=True)
+
+
+def test_gate_only_is_the_full_test_with_an_unbounded_eps():
+    """gate_only == the KL test with eps = +inf (D <= inf always holds), the
+    identity by which the library runs the ablation."""
+    rng = np.random.default_rng(21)
+    for trial in range(30):
+        n = int(rng.integers(1, 40))
+        D = rng.exponential(0.05, n) * (rng.random(n) < 0.9) + (rng.random(n) < 0.1) * 1e30
+        u = np.round(rng.random(n), 2)
+        masked = rng.random(n) < 0.3
+        hp = rng.random(n) < 0.8
+        q = float(rng.random())
+        thr = sl.gate_threshold(u, q)
+        np.testing.assert_array_equal(
+            sl.lock_decision(D, u, masked, hp, 0.0, q, thr, gate_only=True),
+            sl.lock_decision(D, u, masked, hp, np.inf, q, thr))
+
+
 def test_scripted_locks_brute():
     rng = np.random.default_rng(3)
     n = 12
@@ -258,3 +289,51 @@ def test_flops_model():
     # per-row linear FLOPs 2 (L (4 d^2 + 3 d f) + V d) = 2 * 7.497e9
     assert sl.flops_per_step(s, 1, 0) == pytest.approx(2 * 7.497e9, rel=1e-3)
     assert sl.flops_per_step(s, 10, 100) - sl.flops_per_step(s, 10, 0) == 4 * 32 * 10 * 100 * 4096
+
+
+# ---------------------------------------------------------------- ablations --
+
+def test_gate_only_sampler_equals_unbounded_eps_with_gate():
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    a = sl.surelock_sampler(cfg.shape, w, tok, msk, dataclasses.replace(cfg, gate_q=0.3, gate_only=True))
+    b = sl.surelock_sampler(cfg.shape, w, tok, msk, dataclasses.replace(cfg, gate_q=0.3, eps=1e30))
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    np.testing.assert_array_equal(a[2], b[2])
+    assert a[2][-1, 0] < cfg.n_ctx            # the gate alone does lock rows
+
+
+def test_no_kv_cache_sampler_without_locks_is_the_plain_sampler():
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    c0 = dataclasses.replace(cfg, eps=0.0, no_kv_cache=True)
+    t1, lp1, counts, _, _ = sl.surelock_sampler(cfg.shape, w, tok, msk, c0)
+    t2, lp2 = sl.plain_sampler(cfg.shape, w, tok, msk, c0)
+    assert np.all(counts == cfg.n_ctx)
+    np.testing.assert_array_equal(t1, t2)
+    np.testing.assert_array_equal(lp1, lp2)
+
+
+def test_no_kv_cache_sampler_departs_only_after_the_first_lock():
+    """The ablation changes nothing until some row is locked; from the step
+    after the first lock the active rows' posteriors differ."""
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    st_a = sl.init_state(cfg.shape, tok, msk)
+    st_b = sl.init_state(cfg.shape, tok, msk)
+    cfg_b = dataclasses.replace(cfg, no_kv_cache=True)
+    first_lock = None
+    for t in range(cfg.steps):
+        ra = sl.step(cfg.shape, w, st_a, cfg, t)[0]
+        rb = sl.step(cfg.shape, w, st_b, cfg_b, t)[0]
+        if first_lock is None:
+            np.testing.assert_array_equal(ra["lp"], rb["lp"])
+            np.testing.assert_array_equal(ra["lock"], rb["lock"])
+            if ra["lock"].any():
+                first_lock = t
+        elif t == first_lock + 1:
+            assert np.abs(ra["lp"] - rb["lp"]).max() > 1e-6
+            break
+        assert np.all(np.diff(st_b.act[0]) > 0)
+    assert first_lock is not None

@@ -72,6 +72,10 @@ class SamplerSetup:
     eps: float
     gate_q: float = -1.0  # < 0: confidence gate off
     scripted: bool = False
+    # ablations: the confidence gate as the only lock criterion; queries that
+    # see the active rows' keys only (locked rows' cached K/V unused)
+    gate_only: bool = False
+    no_kv_cache: bool = False
 
     @property
     def n_ctx(self) -> int:
