@@ -136,7 +136,8 @@ void sl_active_destroy(sl_active *a);
  *   logits[rows] = RMSNorm(h) W_out^T.
  * d_tokens: [batch][n_ctx] int32 ids x_t.  d_logits: [batch][n_ctx][vocab] in the
  * model dtype; only the active rows are written.  The cache must have been
- * created for the same batch and n_ctx as the active set. */
+ * created for the same batch and n_ctx as the active set.  Under the
+ * SL_ABLATE_NO_KV_CACHE ablation the attention sees the active rows' keys only. */
 sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
                   void *d_logits, void *stream);
 
@@ -147,6 +148,10 @@ typedef struct sl_lock_params {
   int scripted_target;   /* < 0: the KL test.  >= 0: scripted mode, lock eligible
                             rows in ascending (D, position) order until each
                             sequence has this many active rows */
+  int gate_only;         /* ablation (Paper-Notes, ablation table, "confidence gate
+                            only"): lock_j = !masked[row_j] && has_prev &&
+                            u_j <= thr_b, eps and D play no part; needs gate_q >= 0
+                            (SL_ERR_INVALID otherwise).  Ignored in scripted mode. */
 } sl_lock_params;
 
 /* The sure test on the active rows (Paper-Notes, "lock criterion" and
@@ -194,8 +199,9 @@ sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
                            void *stream);
 
 /* Attention of the active rows over all n_ctx cached keys of their sequence in
- * layer `layer`: d_q [M][d_model] (after the rotary embedding), d_o [M][d_model],
- * both in the model dtype. */
+ * layer `layer` (over the active rows' keys only under SL_ABLATE_NO_KV_CACHE):
+ * d_q [M][d_model] (after the rotary embedding), d_o [M][d_model], both in the
+ * model dtype. */
 sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, const void *d_q,
                        void *d_o, void *stream);
 
@@ -269,6 +275,20 @@ sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits);
  * SL_ERR_INVALID for a tiling the GEMM cannot use (the LM head takes no K
  * split).  bf16 models only. */
 sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits, int variant);
+
+/* Ablations of the method (Paper-Notes, ablation table), a bit set; 0 (the
+ * default) is the method itself.
+ *   SL_ABLATE_NO_KV_CACHE  "no KV cache": the queries of sl_step, sl_layer_forward
+ *       and sl_attention attend to the keys of their sequence's active rows only;
+ *       the cached K/V of locked rows are not read.  Same FLOPs, locked tokens'
+ *       information is lost to the active ones.
+ *   SL_ABLATE_GATE_ONLY    "confidence gate only": the model's samplers lock with
+ *       the gate alone (sl_lock_params.gate_only); the sampler then needs
+ *       gate_q >= 0, else sl_sampler_step returns SL_ERR_INVALID.
+ * Unknown bits: SL_ERR_INVALID.  Takes effect from the next call on the model. */
+#define SL_ABLATE_NO_KV_CACHE 1
+#define SL_ABLATE_GATE_ONLY 2
+sl_status sl_model_set_ablation(sl_model *m, int flags);
 
 /* ---------------------------------------------------------------- sampler --- */
 

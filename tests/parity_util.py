@@ -56,7 +56,8 @@ def compare_locks(gpu_lock, ora_lock, D, u, eps, thr=None, gate=False):
     """(mismatches, ambiguous) between lock flags; D, u from the oracle."""
     gpu_lock = np.asarray(gpu_lock).astype(bool)
     ora_lock = np.asarray(ora_lock).astype(bool)
-    amb = np.abs(D - eps) < BAND_D
+    with np.errstate(invalid="ignore"):     # D = inf (no previous posterior) vs eps = inf
+        amb = np.abs(D - eps) < BAND_D
     if gate and thr is not None and np.isfinite(thr):
         amb |= np.abs(u - thr) < BAND_U
     diff = gpu_lock != ora_lock

@@ -66,6 +66,7 @@ def test_host_side_argument_checks(lib):
     assert lib.sl_gemm_bf16(9, 16, 8, 128, 16, None, 128, 16, 128, None, 128, 1, 0, None) == A.SL_ERR_INVALID
     assert lib.sl_gemm_bf16(0, 16, 8, 128, 16, None, 128, 16, 128, None, 128, 1, 3, None) == A.SL_ERR_INVALID
     assert lib.sl_model_set_attention(None, 16, 1) == A.SL_ERR_INVALID
+    assert lib.sl_model_set_ablation(None, A.ABLATE_NO_KV_CACHE) == A.SL_ERR_INVALID
     # output pitch: fp32 rows need ldo % 4 == 0, bf16 rows ldo % 8 == 0, ldo >= N
     assert lib.sl_gemm_bf16(1, 16, 8, 128, 16, None, 128, 16, 130, None, 128, 1, 0, None) == A.SL_ERR_INVALID
     assert lib.sl_gemm_bf16(0, 16, 8, 128, 16, None, 128, 16, 132, None, 128, 1, 0, None) == A.SL_ERR_INVALID

@@ -73,3 +73,109 @@ def test_attention_matches_oracle(cuda_dev, counts, n_ctx, layout):
         assert err <= 2e-2 * max(1.0, np.abs(ref).max()), f"seq {b}: max err {err}"
         off += c
     model.close()
+
+
+# ---------------------------------------------- ablation: no KV cache ---
+# Queries see the keys of their own sequence's active rows only (key stamps).
+
+NOKV_CASES = [
+    ([5], 384, None),
+    ([16, 3], 130, None),
+    ([100, 64, 1], 384, None),
+    ([200], 2500, None),
+    ([0, 40, 0], 260, None),
+    # every active row in the first key tile of a long range: whole key splits
+    # and tiles see no visible key at all
+    ([12], 4000, "head"),
+    # active rows only at the end of the range
+    ([9, 20], 3000, "tail"),
+]
+NOKV_LAYOUTS = [(0, 0), (16, 1), (32, 2), (64, 3), (16, 4)]
+
+
+def _positions(rng, counts, n_ctx, where):
+    out = []
+    for c in counts:
+        if where == "head":
+            out.append(np.sort(rng.choice(64, c, replace=False)).astype(np.int32))
+        elif where == "tail":
+            out.append(np.sort(n_ctx - 1 - rng.choice(100, c, replace=False)).astype(np.int32))
+        else:
+            out.append(np.sort(rng.choice(n_ctx, c, replace=False)).astype(np.int32))
+    return out
+
+
+def _attention_case(cuda_dev, model, cache, act, positions, n_ctx, shape, dtype, rng):
+    B = len(positions)
+    H, dh, d = shape.n_heads, shape.head_dim, shape.d_model
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    rnd = wl.round_bf16 if dtype == "bf16" else (lambda x: x)
+    act.load(positions)
+    k_np = rnd(rng.standard_normal((B * n_ctx, d)).astype(np.float32))
+    v_np = rnd(rng.standard_normal((B * n_ctx, d)).astype(np.float32))
+    k, v = cache.view(0)
+    k.copy_(torch.from_numpy(k_np).to(cuda_dev, tdt))
+    v.copy_(torch.from_numpy(v_np).to(cuda_dev, tdt))
+    M = sum(len(p) for p in positions)
+    q_np = rnd(rng.standard_normal((max(M, 1), d)).astype(np.float32))[:M]
+    q = torch.from_numpy(q_np).to(cuda_dev, tdt)
+    o = torch.full((max(M, 1), d), 9.0, device=cuda_dev, dtype=tdt)
+    rt.attention(model, cache, act, 0, q, o)
+    torch.cuda.synchronize()
+    rt.device_check()
+    got = to64(o)
+    off = 0
+    worst = 0.0
+    for b, pos in enumerate(positions):
+        c = len(pos)
+        if c == 0:
+            continue
+        qb = q_np[off:off + c].astype(np.float64).reshape(c, H, dh)
+        kb = k_np[b * n_ctx:(b + 1) * n_ctx].astype(np.float64).reshape(n_ctx, H, dh)[pos]
+        vb = v_np[b * n_ctx:(b + 1) * n_ctx].astype(np.float64).reshape(n_ctx, H, dh)[pos]
+        ref = om.attention(qb, kb, vb).reshape(c, d)
+        worst = max(worst, np.abs(got[off:off + c] - ref).max() / max(1.0, np.abs(ref).max()))
+        off += c
+    return worst
+
+
+@pytest.mark.parametrize("layout", NOKV_LAYOUTS)
+@pytest.mark.parametrize("counts,n_ctx,where", NOKV_CASES)
+def test_attention_no_kv_cache_matches_oracle(cuda_dev, counts, n_ctx, where, layout):
+    B = len(counts)
+    w_dev = weights_to_device(wl.np_weights(SHAPE, seed=0, std=0.05), "bf16", cuda_dev)
+    model = rt.Model(SHAPE, w_dev, "bf16")
+    model.set_attention(*layout)
+    model.set_ablation(no_kv_cache=True)
+    cache = rt.KVCache(model, B, n_ctx)
+    act = rt.Active(B, n_ctx)
+    rng = np.random.default_rng(7 * sum(counts) + n_ctx)
+    # two calls on one cache with different active sets: the second must not
+    # see the first call's keys
+    for _ in range(2):
+        positions = _positions(rng, counts, n_ctx, where)
+        err = _attention_case(cuda_dev, model, cache, act, positions, n_ctx, SHAPE, "bf16", rng)
+        assert err <= 2e-2, f"max rel err {err}"
+    model.close()
+
+
+SHAPE_F32 = wl.ModelShape(n_layers=1, d_model=64, n_heads=4, head_dim=16, d_ffn=64, vocab=64,
+                          mask_id=63, rope_theta=10000.0)
+
+
+@pytest.mark.parametrize("counts,n_ctx,where", [([7, 0, 30], 100, None), ([5], 300, "tail"),
+                                                ([3, 4], 200, "head")])
+def test_attention_f32_no_kv_cache_matches_oracle(cuda_dev, counts, n_ctx, where):
+    """fp32 path: 32-key chunks with no visible key, before and after the first."""
+    B = len(counts)
+    w_dev = weights_to_device(wl.np_weights(SHAPE_F32, seed=0, std=0.05), "f32", cuda_dev)
+    model = rt.Model(SHAPE_F32, w_dev, "f32")
+    model.set_ablation(no_kv_cache=True)
+    cache = rt.KVCache(model, B, n_ctx)
+    act = rt.Active(B, n_ctx)
+    rng = np.random.default_rng(n_ctx)
+    for _ in range(2):
+        positions = _positions(rng, counts, n_ctx, where)
+        err = _attention_case(cuda_dev, model, cache, act, positions, n_ctx, SHAPE_F32, "f32", rng)
+        assert err <= 1e-5, f"max rel err {err}"
+    model.close()

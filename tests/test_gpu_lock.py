@@ -21,7 +21,7 @@ def _setup_logits(rows_total, V, dtype, seed, sigma_prev=0.05, spike=True):
 
 
 def _run(dev, B, n_ctx, positions, V, dtype, eps, gate_q, has_prev, scripted_target, seed,
-         masked_frac=0.3, sigma_prev=0.05):
+         masked_frac=0.3, sigma_prev=0.05, gate_only=False):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     R = B * n_ctx
     z, zp = _setup_logits(R, V, dtype, seed, sigma_prev)
@@ -45,7 +45,8 @@ def _run(dev, B, n_ctx, positions, V, dtype, eps, gate_q, has_prev, scripted_tar
     amax = torch.zeros(R, device=dev, dtype=torch.int32)
     lock = torch.zeros(R, device=dev, dtype=torch.uint8)
     rt.kl_lock(act, V, mask_id, cur, prv, lse_p, lse_c, msk, kl, unc, conf, amax, lock,
-               eps=eps, gate_q=gate_q, has_prev=has_prev, scripted_target=scripted_target)
+               eps=eps, gate_q=gate_q, has_prev=has_prev, scripted_target=scripted_target,
+               gate_only=gate_only)
     torch.cuda.synchronize()
     rt.device_check()
     out = dict(kl=kl.cpu().numpy(), unc=unc.cpu().numpy(), conf=conf.cpu().numpy(),
@@ -54,7 +55,7 @@ def _run(dev, B, n_ctx, positions, V, dtype, eps, gate_q, has_prev, scripted_tar
                           mask_id=mask_id, lock_t=None), (msk, lock)
 
 
-def _oracle_seq(pos_flat, ref, eps, gate_q, has_prev, scripted_target):
+def _oracle_seq(pos_flat, ref, eps, gate_q, has_prev, scripted_target, gate_only=False):
     lp = ref["lp_cur"][pos_flat]
     lpp = ref["lp_prev"][pos_flat]
     D = osl.kl_rows(lp, lpp) if has_prev else np.full(len(pos_flat), np.inf)
@@ -66,7 +67,7 @@ def _oracle_seq(pos_flat, ref, eps, gate_q, has_prev, scripted_target):
     if scripted_target >= 0:
         lock = osl.scripted_locks(D, masked, hp, pos_flat, len(pos_flat) - scripted_target)
     else:
-        lock = osl.lock_decision(D, u, masked, hp, eps, gate_q, thr)
+        lock = osl.lock_decision(D, u, masked, hp, eps, gate_q, thr, gate_only)
     lse = (ref["z"][pos_flat].astype(np.float64) - lp)[:, 0]
     return dict(D=D, u=u, conf=conf, pred=pred, thr=thr, lock=lock, lse=lse)
 
@@ -202,3 +203,33 @@ def test_unmask_topk_matches_oracle(cuda_dev, k):
         j0 += m
     np.testing.assert_array_equal(t_tok.cpu().numpy(), want_tok)
     np.testing.assert_array_equal(t_msk.cpu().numpy(), want_msk)
+
+
+@pytest.mark.parametrize("eps,gate_q,has_prev", [(0.01, 0.5, True), (0.0, 0.25, True),
+                                                 (-1.0, 0.9, True), (0.01, 0.5, False)])
+def test_gate_only_matches_oracle(cuda_dev, eps, gate_q, has_prev):
+    """The gate-only ablation: the gate alone decides, eps is ignored."""
+    B, n_ctx, V = 3, 100, 1024
+    rng = np.random.default_rng(77)
+    positions = [np.sort(rng.choice(n_ctx, c, replace=False)).astype(np.int32) for c in (100, 9, 57)]
+    act, out, ref, _ = _run(cuda_dev, B, n_ctx, positions, V, "bf16", eps, gate_q, has_prev, -1,
+                            seed=31, sigma_prev=0.2, gate_only=True)
+    j0 = n_mis = 0
+    n_lock = 0
+    for b in range(B):
+        pf = positions[b] + b * n_ctx
+        m = len(pf)
+        o = _oracle_seq(pf, ref, eps, gate_q, has_prev, -1, gate_only=True)
+        sl = slice(j0, j0 + m)
+        mi, _ = compare_locks(out["lock"][sl], o["lock"], o["D"], o["u"], np.inf, o["thr"], True)
+        n_mis += mi
+        n_lock += int(out["lock"][sl].sum())
+        j0 += m
+    assert n_mis == 0
+    assert (n_lock > 0) == has_prev
+
+
+def test_gate_only_needs_the_gate(cuda_dev):
+    positions = [np.arange(10, dtype=np.int32)]
+    with pytest.raises(RuntimeError):
+        _run(cuda_dev, 1, 10, positions, 512, "f32", 0.01, -1.0, True, -1, seed=3, gate_only=True)

@@ -27,6 +27,7 @@ def _sampler(setup, dev, std=0.02, seed_w=0):
     w_np = wl.np_weights(shape, seed=seed_w, std=std)
     w_dev = weights_to_device(w_np, setup.dtype, dev)
     model = rt.Model(shape, w_dev, setup.dtype)
+    model.set_ablation(no_kv_cache=setup.no_kv_cache, gate_only=setup.gate_only)
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, setup.steps,
                    setup.block_len, setup.tokens_per_step, setup.eps, setup.gate_q,
                    setup.scripted)
@@ -83,7 +84,8 @@ def _teacher_forced(setup, dev, steps, std=0.02):
             m = len(A)
             # forward: oracle on the GPU's state
             ck = np.ascontiguousarray(snap["ck"][b]); cv = np.ascontiguousarray(snap["cv"][b])
-            z = om.forward_active(shape, w64, snap["tokens"][b], A, ck, cv)
+            z = om.forward_active(shape, w64, snap["tokens"][b], A, ck, cv,
+                                  no_kv_cache=setup.no_kv_cache)
             err = np.abs(z_gpu[b, A] - z).max() if m else 0.0
             assert err <= LOGIT_TOL[setup.dtype], f"t={t} b={b}: logits err {err}"
             # sure test / gate / unmask on the GPU's logits (same inputs, same decisions)
@@ -110,7 +112,9 @@ def _teacher_forced(setup, dev, steps, std=0.02):
                     am = 0
                 mi = int(diff.sum()) - am
             else:
-                mi, am = compare_locks(lock_g[sl_], rec["lock"], rec["D"], rec["u"], setup.eps,
+                # gate only: D plays no part, so no D band either
+                eps_band = np.inf if setup.gate_only else setup.eps
+                mi, am = compare_locks(lock_g[sl_], rec["lock"], rec["D"], rec["u"], eps_band,
                                        rec["thr"], setup.gate_q >= 0)
             stats["mismatch"] += mi
             stats["ambiguous"] += am
@@ -171,3 +175,49 @@ def test_tiny_free_running_matches_oracle(cuda_dev):
     err = np.abs(lp_gpu - lpT.reshape(len(last), -1)).max()
     assert err <= FINAL_LP_TOL, err
     assert list(s.state()["active"].counts()) == [counts[-1][0]]
+
+
+# ------------------------------------------------------------------ ablations --
+
+def test_tiny_decode_no_kv_cache_teacher_forced(cuda_dev):
+    """Queries see the active rows' keys only (fp32 attention with key stamps)."""
+    stats, _ = _teacher_forced(dataclasses.replace(wl.CFG_TINY, no_kv_cache=True), cuda_dev,
+                               wl.CFG_TINY.steps)
+    assert stats["locks"] > 10, stats
+
+
+def test_tiny_decode_gate_only_teacher_forced(cuda_dev):
+    stats, _ = _teacher_forced(dataclasses.replace(wl.CFG_TINY, gate_q=0.5, gate_only=True),
+                               cuda_dev, 8)
+    assert stats["locks"] > 0, stats
+
+
+def test_bf16_mini_decode_no_kv_cache_teacher_forced(cuda_dev):
+    """The bf16 step with the masked attention kernel, two sequences."""
+    setup = wl.SamplerSetup(MINI_BF16, "bf16", batch=2, prompt_len=40, gen_len=160, steps=40,
+                            block_len=32, tokens_per_step=4, eps=0.01, gate_q=0.5,
+                            no_kv_cache=True)
+    setup.validate()
+    stats, _ = _teacher_forced(setup, cuda_dev, 12, std=0.05)
+    assert stats["locks"] > 0, stats
+
+
+def test_tiny_free_running_ablations_match_oracle(cuda_dev):
+    for setup in (dataclasses.replace(wl.CFG_TINY, no_kv_cache=True),
+                  dataclasses.replace(wl.CFG_TINY, gate_q=0.3, gate_only=True)):
+        model, s, w64, prompts = _sampler(setup, cuda_dev)
+        out = s.generate(prompts)
+        tok0, msk0 = wl.initial_tokens(prompts, setup.gen_len, setup.shape.mask_id)
+        tokT, _, counts, _, _ = osl.surelock_sampler(setup.shape, w64, tok0, msk0, setup)
+        np.testing.assert_array_equal(out, tokT)
+        assert list(s.state()["active"].counts()) == [counts[-1][0]]
+        assert counts[-1][0] < setup.n_ctx
+
+
+def test_gate_only_sampler_needs_the_gate(cuda_dev):
+    setup = dataclasses.replace(wl.CFG_TINY, gate_only=True)     # gate_q < 0
+    model, s, w64, prompts = _sampler(setup, cuda_dev)
+    s.start(torch.from_numpy(prompts).to(cuda_dev))
+    with pytest.raises(RuntimeError):
+        s.step()
+    assert s.state()["t"] == 0                                    # nothing ran

@@ -16,6 +16,7 @@ SL_F32, SL_BF16 = 0, 1
 SL_MAX_BATCH = 64
 K_GEMM, K_ATTN, K_LOCK, K_OTHER, K_COUNT = range(5)
 GEMM_STORE, GEMM_RESID, GEMM_SWIGLU, GEMM_ACCUM = range(4)
+ABLATE_NO_KV_CACHE, ABLATE_GATE_ONLY = 1, 2
 STATUS_NAMES = ["SL_OK", "SL_ERR_INVALID", "SL_ERR_CUDA", "SL_ERR_OOM", "SL_ERR_UNSUPPORTED",
                 "SL_ERR_TIMEOUT", "SL_ERR_STATE"]
 
@@ -39,7 +40,7 @@ class Weights(C.Structure):
 
 class LockParams(C.Structure):
     _fields_ = [("eps", C.c_float), ("gate_q", C.c_float), ("has_prev", C.c_int),
-                ("scripted_target", C.c_int)]
+                ("scripted_target", C.c_int), ("gate_only", C.c_int)]
 
 
 class SamplerParams(C.Structure):
@@ -86,6 +87,7 @@ SIGNATURES = {
     "sl_kl_stats_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
     "sl_unmask_topk": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "sl_compact_active": (_I, [_P, _P, _P, _P, _I, _P]),
+    "sl_model_set_ablation": (_I, [_P, _I]),
     "sl_sampler_create": (_I, [_P, _I, C.POINTER(SamplerParams), C.POINTER(_P)]),
     "sl_sampler_start": (_I, [_P, _P, _P]),
     "sl_sampler_step": (_I, [_P, _P]),

@@ -6,6 +6,7 @@
 // computation runs on the active rows only, locked rows are served from the
 // cache C, and the active list is compacted after every sure test
 // (Paper-Notes, "Method: overall framework" and "Key design").
+#include <limits.h>
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -98,6 +99,7 @@ struct sl_model {
   std::vector<sl_layer_weights> layers;
   std::vector<std::array<WMaps, W_COUNT>> maps;
   int attn_q = 0, attn_splits = 0;   // pinned attention layout (0 = cost model)
+  int ablation = 0;                  // SL_ABLATE_* bits (0: the method itself)
   WMaps head_map;
   int num_sms;
   int *err;
@@ -124,6 +126,8 @@ struct sl_kv_cache {
   float *ws = nullptr;     // [max_rows][max(3d, 2f)] fp32 split-K workspace, kept zero
   float *attn_ws = nullptr;
   int attn_max_splits = 16;
+  int32_t *key_stamp = nullptr;   // [max_rows] visible-key stamps (no-KV-cache ablation)
+  int key_gen = 0;                // the current stamp generation
   TmaMat map_a, map_o, map_act;
   // epilogue destinations at the current M: residual h (fp32), split-K
   // workspace as [M][3d] and [M][2f] (fp32), gate/up product act (bf16)
@@ -349,7 +353,7 @@ extern "C" void sl_kv_cache_destroy(sl_kv_cache *c) {
   if (!c) return;
   for (void *p : c->k) cudaFree(p);
   for (void *p : c->v) cudaFree(p);
-  void *ps[] = {c->rope, c->h, c->a, c->qkv, c->q, c->o, c->act, c->ws, c->attn_ws};
+  void *ps[] = {c->rope, c->h, c->a, c->qkv, c->q, c->o, c->act, c->ws, c->attn_ws, c->key_stamp};
   for (void *p : ps)
     if (p) cudaFree(p);
   delete c;
@@ -385,7 +389,7 @@ extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
   ok = ok && alloc((void **)&c->h, rows * d * 4) && alloc(&c->a, rows * d * es) &&
        alloc(&c->qkv, rows * 3 * d * es) && alloc(&c->q, rows * d * es) &&
        alloc(&c->o, rows * d * es) && alloc(&c->act, rows * f * es) &&
-       alloc((void **)&c->ws, rows * wsc * 4);
+       alloc((void **)&c->ws, rows * wsc * 4) && alloc((void **)&c->key_stamp, rows * 4);
   if (ok && cfg.dtype == SL_BF16) {
     ok = alloc((void **)&c->attn_ws, attn_bf16_workspace_bytes(c->max_rows, cfg.n_heads,
                                                                c->attn_max_splits));
@@ -672,8 +676,32 @@ static double gemm_bytes(double M, double N, double K, double es) {
   return es * (N * K + M * K + M * N);
 }
 
+// The keys this step's queries may attend to.  The method: every cached key
+// (stamp null).  The no-KV-cache ablation: the active rows' own keys, marked
+// with a fresh stamp generation once per call (the stamps start at zero, so
+// generation 1 onwards never matches a row that was not stamped).
+struct KeySet {
+  const int32_t *stamp = nullptr;
+  int gen = 0;
+};
+
+static sl_status visible_keys(const sl_model *m, sl_kv_cache *c, const sl_active *a, int M,
+                              cudaStream_t s, KeySet *ks) {
+  *ks = KeySet{};
+  if (!(m->ablation & SL_ABLATE_NO_KV_CACHE)) return SL_OK;
+  if (c->key_gen == INT_MAX) {
+    SL_CUDA(cudaMemsetAsync(c->key_stamp, 0, (size_t)c->max_rows * 4, s));
+    c->key_gen = 0;
+  }
+  ++c->key_gen;
+  SL_CUDA(launch_key_stamp(a->rows, M, c->key_gen, c->key_stamp, s));
+  ks->stamp = c->key_stamp;
+  ks->gen = c->key_gen;
+  return SL_OK;
+}
+
 static sl_status layer_f32(sl_model *m, sl_kv_cache *c, sl_active *a, int l, float *h, int M,
-                           cudaStream_t s) {
+                           const KeySet &ks, cudaStream_t s) {
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn;
   float *an = (float *)c->a, *qkv = (float *)c->qkv, *q = (float *)c->q;
@@ -692,7 +720,7 @@ static sl_status layer_f32(sl_model *m, sl_kv_cache *c, sl_active *a, int l, flo
     Timed t(m, SL_K_ATTN, 4.0 * (2.0 * M * d + 2.0 * c->batch * c->n_ctx * d),
             4.0 * M * c->n_ctx * d, s);
     SL_CUDA(launch_attn_f32(q, (const float *)c->k[l], (const float *)c->v[l], a->rows, M,
-                            c->n_ctx, cfg.n_heads, cfg.head_dim, o, s));
+                            c->n_ctx, cfg.n_heads, cfg.head_dim, o, s, ks.stamp, ks.gen));
   }
   {
     Timed t(m, SL_K_GEMM, gemm_bytes(M, d, d, 4), 2.0 * M * d * d, s);
@@ -791,14 +819,15 @@ static void fill_seqs(AttnSeqs &seqs, const sl_active *a, const int32_t *counts)
 }
 
 static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, int l, int M,
-                           const void *q, void *o, cudaStream_t s) {
+                           const void *q, void *o, const KeySet &ks, cudaStream_t s) {
   const int d = m->cfg.d_model;
   Timed t(m, SL_K_ATTN, 2.0 * (2.0 * M * d + 2.0 * seqs.batch * c->n_ctx * d),
           4.0 * (double)M * c->n_ctx * d, s);
   // the output projection's weights follow; the attention leaves HBM idle
   SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
                            c->attn_ws, c->attn_max_splits, m->num_sms, s, m->attn_q,
-                           m->attn_splits, m->layers[l].wo, (size_t)d * d * 2));
+                           m->attn_splits, m->layers[l].wo, (size_t)d * d * 2, ks.stamp,
+                           ks.gen));
   return SL_OK;
 }
 
@@ -924,14 +953,15 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
 }
 
 static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, float *h, int M,
-                            const AttnSeqs &seqs, const BfPlans &pl, cudaStream_t s) {
+                            const AttnSeqs &seqs, const BfPlans &pl, const KeySet &ks,
+                            cudaStream_t s) {
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model;
   const sl_layer_weights &lw = m->layers[l];
   sl_status st;
   SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s));
   if ((st = run_gemm(m, c, a->rows, l, G_QKV, pl.qkv, M, h, nullptr, s)) != SL_OK) return st;
-  if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, s)) != SL_OK) return st;
+  if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, ks, s)) != SL_OK) return st;
   if ((st = run_gemm(m, c, a->rows, l, G_O, pl.o, M, h, nullptr, s)) != SL_OK) return st;
   SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.ffn_norm, d, cfg.rms_eps, M, c->a, s));
   if ((st = run_gemm(m, c, a->rows, l, G_GU, pl.gu, M, h, nullptr, s)) != SL_OK) return st;
@@ -962,10 +992,12 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   cudaStream_t s = (cudaStream_t)stream;
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, V = cfg.vocab;
+  KeySet ks;
+  if ((st = visible_keys(m, c, a, M, s, &ks)) != SL_OK) return st;
   SL_CUDA(launch_gather_embed(cfg.dtype, d_tokens, a->rows, M, m->tok_emb, d, c->h, s));
   if (cfg.dtype == SL_F32) {
     for (int l = 0; l < cfg.n_layers; ++l)
-      if ((st = layer_f32(m, c, a, l, c->h, M, s)) != SL_OK) return st;
+      if ((st = layer_f32(m, c, a, l, c->h, M, ks, s)) != SL_OK) return st;
     SL_CUDA(launch_rmsnorm(SL_F32, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
     Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 4), 2.0 * M * d * V, s);
     SL_CUDA(launch_gemm_f32(EPI_STORE, (const float *)c->a, M, d, (const float *)m->lm_head, V,
@@ -977,7 +1009,7 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   fill_seqs(seqs, a, counts);
   const BfPlans pl = plans_for(m, M, m->num_sms);
   for (int l = 0; l < cfg.n_layers; ++l)
-    if ((st = layer_bf16(m, c, a, l, c->h, M, seqs, pl, s)) != SL_OK) return st;
+    if ((st = layer_bf16(m, c, a, l, c->h, M, seqs, pl, ks, s)) != SL_OK) return st;
   SL_CUDA(launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
   if ((st = run_gemm(m, c, a->rows, 0, G_HD, pl.hd, M, c->h, d_logits, s)) != SL_OK) return st;
   // the previous step's timing events completed before this step was planned
@@ -999,11 +1031,13 @@ extern "C" sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a,
   for (int b = 0; b < a->batch; ++b) M += counts[b];
   if (M == 0) return SL_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  if (m->cfg.dtype == SL_F32) return layer_f32(m, c, a, layer, d_h, M, s);
+  KeySet ks;
+  if ((st = visible_keys(m, c, a, M, s, &ks)) != SL_OK) return st;
+  if (m->cfg.dtype == SL_F32) return layer_f32(m, c, a, layer, d_h, M, ks, s);
   if ((st = ensure_maps(c, M)) != SL_OK) return st;
   AttnSeqs seqs;
   fill_seqs(seqs, a, counts);
-  return layer_bf16(m, c, a, layer, d_h, M, seqs, plans_for(m, M, m->num_sms), s);
+  return layer_bf16(m, c, a, layer, d_h, M, seqs, plans_for(m, M, m->num_sms), ks, s);
 }
 
 extern "C" sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
@@ -1019,17 +1053,19 @@ extern "C" sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int
   for (int b = 0; b < a->batch; ++b) M += counts[b];
   if (M == 0) return SL_OK;
   cudaStream_t s = (cudaStream_t)stream;
+  KeySet ks;
+  if ((st = visible_keys(m, c, a, M, s, &ks)) != SL_OK) return st;
   if (m->cfg.dtype == SL_F32) {
     Timed t(m, SL_K_ATTN, 4.0 * (2.0 * M * m->cfg.d_model + 2.0 * c->batch * c->n_ctx * m->cfg.d_model),
             4.0 * M * c->n_ctx * m->cfg.d_model, s);
     SL_CUDA(launch_attn_f32((const float *)d_q, (const float *)c->k[layer],
                             (const float *)c->v[layer], a->rows, M, c->n_ctx, m->cfg.n_heads,
-                            m->cfg.head_dim, (float *)d_o, s));
+                            m->cfg.head_dim, (float *)d_o, s, ks.stamp, ks.gen));
     return SL_OK;
   }
   AttnSeqs seqs;
   fill_seqs(seqs, a, counts);
-  return attn_bf16(m, c, seqs, layer, M, d_q, d_o, s);
+  return attn_bf16(m, c, seqs, layer, M, d_q, d_o, ks, s);
 }
 
 extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b,
@@ -1252,6 +1288,14 @@ extern "C" sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn
   return SL_OK;
 }
 
+extern "C" sl_status sl_model_set_ablation(sl_model *m, int flags) {
+  if (!m) return fail(SL_ERR_INVALID, "sl_model_set_ablation: null model");
+  if (flags & ~(SL_ABLATE_NO_KV_CACHE | SL_ABLATE_GATE_ONLY))
+    return fail(SL_ERR_INVALID, "sl_model_set_ablation: unknown flags 0x%x", flags);
+  m->ablation = flags;
+  return SL_OK;
+}
+
 extern "C" sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits) {
   if (!m || (queries_per_cta != 0 && queries_per_cta != 16 && queries_per_cta != 32 &&
              queries_per_cta != 64) ||
@@ -1296,6 +1340,9 @@ static sl_status kl_lock_impl(sl_model *timing_model, sl_active *a, int vocab, i
   if (mask_id < -1 || mask_id >= vocab) return fail(SL_ERR_INVALID, "sl_kl_lock: bad mask_id");
   if (dtype != SL_F32 && dtype != SL_BF16) return fail(SL_ERR_INVALID, "sl_kl_lock: bad dtype");
   if (p->gate_q > 1.f) return fail(SL_ERR_INVALID, "sl_kl_lock: gate_q must be <= 1");
+  const bool gate_only = p->gate_only && p->scripted_target < 0;
+  if (gate_only && !(p->gate_q >= 0.f))
+    return fail(SL_ERR_INVALID, "sl_kl_lock: the gate-only criterion needs gate_q >= 0");
   if (((uintptr_t)cur & 15) || (prev && ((uintptr_t)prev & 15)))
     return fail(SL_ERR_INVALID, "sl_kl_lock: logits must be 16-byte aligned");
   int32_t counts[SL_MAX_BATCH];
@@ -1327,7 +1374,10 @@ static sl_status kl_lock_impl(sl_model *timing_model, sl_active *a, int vocab, i
     Timed t(timing_model, SL_K_LOCK, bytes, 6.0 * M * vocab, s);
     SL_CUDA(launch_lock_stats(la, s));
   }
-  SL_CUDA(launch_lock_decide(a->seq_off, a->batch, a->rows, kl, unc, masked, p->eps, p->gate_q,
+  // gate only: the same decision with the KL bound at +inf, where D <= eps
+  // always holds, so the gate alone decides among the eligible rows
+  const float eps = gate_only ? INFINITY : p->eps;
+  SL_CUDA(launch_lock_decide(a->seq_off, a->batch, a->rows, kl, unc, masked, eps, p->gate_q,
                              p->has_prev, p->scripted_target, lock, s));
   return SL_OK;
 }
@@ -1466,6 +1516,8 @@ extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
   if (!s) return fail(SL_ERR_INVALID, "sl_sampler_step: null sampler");
   if (!s->started) return fail(SL_ERR_STATE, "sl_sampler_step: call sl_sampler_start first");
   if (s->t >= s->p.steps) return fail(SL_ERR_STATE, "sl_sampler_step: decode already finished");
+  if ((s->m->ablation & SL_ABLATE_GATE_ONLY) && !s->p.scripted && !(s->p.gate_q >= 0.f))
+    return fail(SL_ERR_INVALID, "sl_sampler_step: the gate-only ablation needs gate_q >= 0");
   const int t = s->t;
   const int cur = t & 1, prv = cur ^ 1;
   const sl_config &cfg = s->m->cfg;
@@ -1476,6 +1528,7 @@ extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
   lp.gate_q = s->p.gate_q;
   lp.has_prev = t > 0 ? 1 : 0;
   lp.scripted_target = -1;
+  lp.gate_only = (s->m->ablation & SL_ABLATE_GATE_ONLY) ? 1 : 0;
   if (s->p.scripted) {
     // M_{t+1} = round-half-up(N - 0.9 N (t+1)/(T-1))
     const double n = s->n_ctx;

@@ -13,6 +13,10 @@
 // through shared memory at the end.  Only when the CTAs cannot fill the GPU
 // and the key range is long is it also split across CTAs, with a second
 // kernel merging those partial records, one warp per (row, head).
+//
+// The MASK instantiation serves the no-KV-cache ablation: a key takes part
+// only if its stamp equals the step's generation (the active rows' keys); the
+// others score -inf exactly like the ragged tail beyond n_ctx.
 #include <algorithm>
 
 #include "common.cuh"
@@ -87,9 +91,11 @@ struct AttnParams {
   int M, n_ctx, n_heads, splits, kblocks;
   const void *pf;        // the next GEMM's weights, prefetched into L2 (optional)
   size_t pf_bytes;
+  const int32_t *stamp;  // [B*n_ctx] key stamps (MASK instantiation only)
+  int gen;               // stamp value of a visible key
 };
 
-template <int QW>
+template <int QW, bool MASK>
 __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_constant__ AttnParams p) {
   using C = AtCfg<QW>;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -196,7 +202,9 @@ __global__ void __launch_bounds__(AT_THREADS) attn_bf16_kernel(const __grid_cons
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         int key = kb * AT_K + kw * C::KS + nt * 8 + 2 * c4 + (e & 1);
-        float v = (key < p.n_ctx) ? s[nt][e] * sl2 : -INFINITY;
+        bool live = key < p.n_ctx;
+        if constexpr (MASK) live = live && p.stamp[(size_t)b * p.n_ctx + key] == p.gen;
+        float v = live ? s[nt][e] * sl2 : -INFINITY;
         s[nt][e] = v;
         tmax[e >> 1] = fmaxf(tmax[e >> 1], v);
       }
@@ -367,23 +375,30 @@ size_t attn_bf16_workspace_bytes(int max_rows, int n_heads, int max_splits) {
 }
 
 
-template <int QW>
+template <int QW, bool MASK>
 static cudaError_t run_attn(const AttnParams &p, int tiles, cudaStream_t s) {
   using C = AtCfg<QW>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<QW>,
+    cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<QW, MASK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_k(attn_bf16_kernel<QW>, dim3(tiles, p.n_heads, p.splits), AT_THREADS, C::SMEM, s, p);
+  return launch_k(attn_bf16_kernel<QW, MASK>, dim3(tiles, p.n_heads, p.splits), AT_THREADS,
+                  C::SMEM, s, p);
+}
+
+template <bool MASK>
+static cudaError_t run_attn_qw(int qw, const AttnParams &p, int tiles, cudaStream_t s) {
+  return qw == 4 ? run_attn<4, MASK>(p, tiles, s)
+                 : qw == 2 ? run_attn<2, MASK>(p, tiles, s) : run_attn<1, MASK>(p, tiles, s);
 }
 
 cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, const AttnSeqs &seqs,
                              int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
                              int num_sms, cudaStream_t s, int force_q, int force_splits,
-                             const void *pf, size_t pf_bytes) {
+                             const void *pf, size_t pf_bytes, const int32_t *stamp, int gen) {
   cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   // Queries per CTA (16 * qw) and cross-CTA key split from a small cost model:
@@ -429,8 +444,9 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
   p.kblocks = kblocks;
   p.pf = pf;
   p.pf_bytes = pf_bytes;
-  err = qw == 4 ? run_attn<4>(p, tiles, s) : qw == 2 ? run_attn<2>(p, tiles, s)
-                                                     : run_attn<1>(p, tiles, s);
+  p.stamp = stamp;
+  p.gen = gen;
+  err = stamp ? run_attn_qw<true>(qw, p, tiles, s) : run_attn_qw<false>(qw, p, tiles, s);
   if (err != cudaSuccess || splits == 1) return err;
   const int warps = M * n_heads;
   return launch_k(attn_combine_kernel, (warps * 32 + 255) / 256, 256, 0, s, (const float *)p.ws_o,

@@ -92,10 +92,15 @@ cudaError_t launch_swiglu(int dtype, const void *ws, bool in_f32, bool zero_in, 
 cudaError_t launch_gemm_f32(int epi, const float *A, int M, int K, const float *B, int N,
                             float *C, int ldc, int col_off, const int32_t *row_map,
                             cudaStream_t s);
-// fp32 attention, head_dim <= 64: o[j] = softmax(q_j K_b^T / sqrt(dh)) V_b.
+// fp32 attention, head_dim <= 64: o[j] = softmax(q_j K_b^T / sqrt(dh)) V_b;
+// with stamp non-null, over the keys n with stamp[b * n_ctx + n] == gen only.
 cudaError_t launch_attn_f32(const float *q, const float *ck, const float *cv,
                             const int32_t *rows, int M, int n_ctx, int n_heads, int head_dim,
-                            float *o, cudaStream_t s);
+                            float *o, cudaStream_t s, const int32_t *stamp = nullptr,
+                            int gen = 0);
+// stamp[rows[j]] = gen for j < M: marks the active rows' keys visible.
+cudaError_t launch_key_stamp(const int32_t *rows, int M, int gen, int32_t *stamp,
+                             cudaStream_t s);
 
 // -------------------------------------------------------------------- attn.cu
 // Query tiles per sequence for the bf16 attention kernel.
@@ -111,7 +116,8 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
                              int M, int n_ctx, int n_heads, void *o, float *ws, int max_splits,
                              int num_sms, cudaStream_t s, int force_q = 0,
                              int force_splits = 0, const void *pf = nullptr,
-                             size_t pf_bytes = 0);
+                             size_t pf_bytes = 0, const int32_t *stamp = nullptr,
+                             int gen = 0);
 
 // ----------------------------------------------------------------- gemm_tc.cu
 // A bf16 K-major operand in global memory with its TMA descriptor.

@@ -392,14 +392,36 @@ cudaError_t launch_gemm_f32(int epi, const float *A, int M, int K, const float *
   return err;
 }
 
+// ------------------------------------------------------------ key stamps ---
+// The no-KV-cache ablation (the pages' ablation table: locked tokens cannot be
+// attended): the keys a query may see are its sequence's active rows.  Each
+// call stamps stamp[row] = gen at the active rows with a new generation, and the
+// attention kernels take a key as visible iff its stamp equals gen, so rows
+// that left the active set drop out without a clearing pass.
+__global__ void key_stamp_kernel(const int32_t *__restrict__ rows, int M, int gen,
+                                 int32_t *__restrict__ stamp) {
+  pdl_wait();
+  pdl_trigger();
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < M) stamp[rows[j]] = gen;
+}
+
+cudaError_t launch_key_stamp(const int32_t *rows, int M, int gen, int32_t *stamp,
+                             cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  return launch_k(key_stamp_kernel, (M + 255) / 256, 256, 0, s, rows, M, gen, stamp);
+}
+
 // --------------------------------------------------------- fp32 attention ---
 // One warp per (active row, head).  Keys of the row's sequence are processed in
 // chunks of 32 (one key per lane) with an online softmax; each lane keeps a
-// partial output over its keys, reduced across the warp at the end.
+// partial output over its keys, reduced across the warp at the end.  With
+// `stamp` non-null only keys whose stamp equals `gen` take part.
 template <int DH>
 __global__ void attn_f32_kernel(const float *__restrict__ q, const float *__restrict__ ck,
                                 const float *__restrict__ cv, const int32_t *__restrict__ rows,
-                                int M, int n_ctx, int n_heads, float *__restrict__ o) {
+                                int M, int n_ctx, int n_heads, const int32_t *__restrict__ stamp,
+                                int gen, float *__restrict__ o) {
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   if (warp >= M * n_heads) return;
@@ -418,9 +440,10 @@ __global__ void attn_f32_kernel(const float *__restrict__ q, const float *__rest
   for (int i = 0; i < DH; ++i) acc[i] = 0.f;
   for (int n0 = 0; n0 < n_ctx; n0 += 32) {
     int n = n0 + lane;
+    const bool live = n < n_ctx && (stamp == nullptr || stamp[(size_t)b * n_ctx + n] == gen);
     float sc = -INFINITY;
     const size_t kr = ((size_t)b * n_ctx + n) * d + hh * DH;
-    if (n < n_ctx) {
+    if (live) {
       float dot = 0.f;
 #pragma unroll
       for (int i = 0; i < DH; ++i) dot = fmaf(qr[i], ck[kr + i], dot);
@@ -428,12 +451,13 @@ __global__ void attn_f32_kernel(const float *__restrict__ q, const float *__rest
     }
     float cm = warp_max(sc);
     float mn = fmaxf(m, cm);
-    float corr = __expf(m - mn);
-    float pe = (n < n_ctx) ? __expf(sc - mn) : 0.f;
+    // a chunk with no visible key while nothing has been seen leaves m = -inf
+    float corr = (m == -INFINITY) ? 0.f : __expf(m - mn);
+    float pe = live ? __expf(sc - mn) : 0.f;
     l = l * corr + warp_sum(pe);
 #pragma unroll
     for (int i = 0; i < DH; ++i) acc[i] *= corr;
-    if (n < n_ctx) {
+    if (live) {
 #pragma unroll
       for (int i = 0; i < DH; ++i) acc[i] = fmaf(pe, cv[kr + i], acc[i]);
     }
@@ -450,16 +474,16 @@ __global__ void attn_f32_kernel(const float *__restrict__ q, const float *__rest
 
 cudaError_t launch_attn_f32(const float *q, const float *ck, const float *cv,
                             const int32_t *rows, int M, int n_ctx, int n_heads, int head_dim,
-                            float *o, cudaStream_t s) {
+                            float *o, cudaStream_t s, const int32_t *stamp, int gen) {
   cudaError_t err = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   int warps = M * n_heads;
   int blocks = (warps * 32 + 255) / 256;
   switch (head_dim) {
-    case 8: err = launch_k(attn_f32_kernel<8>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
-    case 16: err = launch_k(attn_f32_kernel<16>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
-    case 32: err = launch_k(attn_f32_kernel<32>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
-    case 64: err = launch_k(attn_f32_kernel<64>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, o); break;
+    case 8: err = launch_k(attn_f32_kernel<8>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, stamp, gen, o); break;
+    case 16: err = launch_k(attn_f32_kernel<16>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, stamp, gen, o); break;
+    case 32: err = launch_k(attn_f32_kernel<32>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, stamp, gen, o); break;
+    case 64: err = launch_k(attn_f32_kernel<64>, blocks, 256, 0, s, q, ck, cv, rows, M, n_ctx, n_heads, stamp, gen, o); break;
     default: return cudaErrorInvalidValue;
   }
   return err;

@@ -113,6 +113,12 @@ class Model:
         A.check(A.lib().sl_model_set_attention(self.handle, queries_per_cta, splits),
                 "sl_model_set_attention")
 
+    def set_ablation(self, no_kv_cache: bool = False, gate_only: bool = False):
+        """Ablations of the method: attention without the locked rows' cached
+        K/V; the confidence gate as the only lock criterion of the samplers."""
+        flags = (A.ABLATE_NO_KV_CACHE if no_kv_cache else 0) | (A.ABLATE_GATE_ONLY if gate_only else 0)
+        A.check(A.lib().sl_model_set_ablation(self.handle, flags), "sl_model_set_ablation")
+
     def set_tuning(self, kind: int, M: int, bn: int, splits: int, variant: int):
         """Pin GEMM `kind`'s tiling for the row-count bucket of M (splits -1: stream-K)."""
         A.check(A.lib().sl_model_set_tuning(self.handle, kind, M, bn, splits, variant),
@@ -270,8 +276,9 @@ def kl_lock(active: Active, vocab: int, mask_id: int, logits_cur: torch.Tensor,
             logits_prev: Optional[torch.Tensor], lse_prev: Optional[torch.Tensor],
             lse_cur: torch.Tensor, masked: torch.Tensor, kl: torch.Tensor, unc: torch.Tensor,
             conf: torch.Tensor, argmax: torch.Tensor, lock: torch.Tensor, eps: float,
-            gate_q: float = -1.0, has_prev: bool = True, scripted_target: int = -1, stream=None):
-    p = A.LockParams(eps, gate_q, 1 if has_prev else 0, scripted_target)
+            gate_q: float = -1.0, has_prev: bool = True, scripted_target: int = -1,
+            gate_only: bool = False, stream=None):
+    p = A.LockParams(eps, gate_q, 1 if has_prev else 0, scripted_target, 1 if gate_only else 0)
     A.check(A.lib().sl_kl_lock(active.handle, vocab, mask_id, _dtype_code(logits_cur.dtype),
                                _ptr(logits_cur), _ptr(logits_prev), _ptr(lse_prev), _ptr(lse_cur),
                                _ptr(masked), C.byref(p), _ptr(kl), _ptr(unc), _ptr(conf),
