@@ -58,7 +58,8 @@ def load_peaks():
 
 
 # ------------------------------------------------------------- workload ---
-def make_setup(name: str, eps, scripted: bool) -> wl.SamplerSetup:
+def make_setup(name: str, eps, scripted: bool, batch=None) -> wl.SamplerSetup:
+    """The workload's decode; `batch` (1..64 sequences per GPU) overrides its batch."""
     if name == "full8b":
         s = wl.cfg_full8b(eps=0.05 if eps is None else eps, scripted=scripted)
     elif name == "long8b":
@@ -68,6 +69,11 @@ def make_setup(name: str, eps, scripted: bool) -> wl.SamplerSetup:
             s = dataclasses.replace(s, eps=eps)
     else:
         raise SystemExit(f"unknown workload {name}")
+    if batch is not None:
+        if not 1 <= batch <= 64:
+            raise SystemExit(f"--batch must be in [1, 64], got {batch}")
+        import dataclasses
+        s = dataclasses.replace(s, batch=batch)
     s.validate()
     return s
 
@@ -303,7 +309,7 @@ def run_ours(args, rank: int, world: int):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    setup = make_setup(args.workload, args.eps, args.scripted)
+    setup = make_setup(args.workload, args.eps, args.scripted, args.batch)
     shape = setup.shape
     T = setup.steps
     ranks = Ranks(world, "nccl", dev)
@@ -485,7 +491,7 @@ def run_reference(args, rank: int, world: int):
     bench step is one bounded sample (see oracle_sample)."""
     if rank != 0:
         return None
-    setup = make_setup(args.workload, args.eps, args.scripted)
+    setup = make_setup(args.workload, args.eps, args.scripted, args.batch)
     T = setup.steps
     # the dense trajectory shape of the scripted/KL schedule is not known on the
     # CPU side; use the linear decay from N to the masked-only floor
@@ -521,6 +527,8 @@ def main():
     ap.add_argument("--workload", default="full8b")
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--scripted", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="sequences per GPU (default: the workload's own batch)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "surelock_bench"),
                     help="where the per-rank clock samples (CSV) are written")

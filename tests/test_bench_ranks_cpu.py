@@ -48,3 +48,19 @@ def test_aggregate_rate():
     # 2 ranks x 3 decodes x 256 steps over the slowest rank's 1.5 s
     assert bench.aggregate_rate(2, 3 * 256, 1500.0) == 1024.0
     assert bench.aggregate_rate(1, 256, 1000.0) == 256.0
+
+
+def test_batch_override():
+    import types
+    import pytest
+    sys.path.insert(0, ROOT)
+    import bench
+    s = bench.make_setup("full8b", None, False, 8)
+    assert (s.batch, s.n_ctx, s.steps) == (8, 384, 256)
+    args = types.SimpleNamespace(workload="full8b")
+    cfg = bench.workload_config(args, s, 2)
+    assert cfg["global_batch"] == 16 and "batch 8" in cfg["workload"]
+    assert bench.make_setup("long8b", None, False).batch == 4
+    for bad in (0, 65):
+        with pytest.raises(SystemExit):
+            bench.make_setup("full8b", None, False, bad)
