@@ -81,7 +81,10 @@ typedef struct sl_kv_cache sl_kv_cache;
 typedef struct sl_active sl_active;
 typedef struct sl_sampler sl_sampler;
 
+/* Message for the calling thread's last non-OK status (thread-local, owned by
+ * the library; valid until the thread's next failing call; "" if none). */
 const char *sl_last_error(void);
+/* Library version string (static, owned by the library). */
 const char *sl_version(void);
 
 /* ---------------------------------------------------------------- model --- */
@@ -89,6 +92,8 @@ const char *sl_version(void);
 /* Borrow device weights and build the per-model launch state (TMA descriptors
  * for the bf16 path).  Fails with SL_ERR_INVALID on an inconsistent config. */
 sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, sl_model **out);
+/* Frees the model's launch state (not the borrowed weights).  Caches and
+ * samplers created from it must be destroyed first.  NULL is a no-op. */
 void sl_model_destroy(sl_model *m);
 
 /* --------------------------------------------------------------- KV cache --- */
@@ -294,10 +299,13 @@ sl_status sl_model_set_ablation(sl_model *m, int flags);
 
 /* Semi-autoregressive SureLock decode driven by the library: prompt_len given
  * tokens then gen_len [MASK] tokens; gen region split in blocks of block_len,
- * steps/(gen_len/block_len) steps per block, tokens_per_step unmasked per step. */
+ * steps/(gen_len/block_len) steps per block, tokens_per_step unmasked per step
+ * (the unmodified sampler the pages compare against, Abstract: "the same
+ * sampler without locking", with the sure test of sl_kl_lock between steps). */
 typedef struct sl_sampler_params {
   int prompt_len, gen_len, steps, block_len, tokens_per_step;
-  float eps, gate_q;
+  float eps;             /* KL threshold; eps <= 0 disables locking */
+  float gate_q;          /* confidence-gate quantile in [0,1]; < 0 = gate off */
   int scripted;          /* 1: scripted lock schedule, M decays linearly to 10% of N */
 } sl_sampler_params;
 
@@ -318,6 +326,12 @@ typedef struct sl_sampler_state {
   int batch, n_ctx;
 } sl_sampler_state;
 
+/* Creates a sampler for `batch` sequences (1..SL_MAX_BATCH) of n_ctx =
+ * prompt_len + gen_len positions, with its own KV cache, active set, token,
+ * flag and logit buffers (two [batch][n_ctx][vocab] logit buffers in the model
+ * dtype).  SL_ERR_INVALID if gen_len does not split into blocks or steps into
+ * blocks, or gate_q > 1; SL_ERR_UNSUPPORTED for block_len > 2048; SL_ERR_OOM if
+ * the buffers do not fit.  The model must outlive the sampler. */
 sl_status sl_sampler_create(sl_model *m, int batch, const sl_sampler_params *p, sl_sampler **out);
 /* Reset state for a new decode from device prompts [batch][prompt_len]. */
 sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, void *stream);
@@ -327,6 +341,8 @@ sl_status sl_sampler_step(sl_sampler *s, void *stream);
  * [batch][n_ctx]; both copies are inside the call. */
 sl_status sl_sampler_generate(sl_sampler *s, const int32_t *h_prompts, int32_t *h_tokens,
                               void *stream);
+/* The sampler's buffers and step counter; the pointers stay owned by the
+ * sampler and valid until it is destroyed. */
 sl_status sl_sampler_get_state(const sl_sampler *s, sl_sampler_state *out);
 void sl_sampler_destroy(sl_sampler *s);
 
