@@ -22,7 +22,8 @@ Multi-GPU (torchrun): independent replicas, one decode per rank; the timed
 region is bracketed by barriers and the max over ranks is taken.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload full8b|long8b] [--eps E] [--scripted]
+                  [--workload full8b|long8b] [--eps E] [--scripted] [--batch B]
+                  [--gate-q Q] [--ablation none|no_kv_cache|gate_only]
 """
 from __future__ import annotations
 
@@ -58,8 +59,11 @@ def load_peaks():
 
 
 # ------------------------------------------------------------- workload ---
-def make_setup(name: str, eps, scripted: bool, batch=None) -> wl.SamplerSetup:
-    """The workload's decode; `batch` (1..64 sequences per GPU) overrides its batch."""
+def make_setup(name: str, eps, scripted: bool, batch=None, gate_q=None,
+               ablation: str = "none") -> wl.SamplerSetup:
+    """The workload's decode; `batch` (1..64 sequences per GPU) overrides its batch,
+    `gate_q` its confidence gate, and `ablation` selects one of the pages'
+    ablations (no_kv_cache, gate_only) instead of the method itself."""
     if name == "full8b":
         s = wl.cfg_full8b(eps=0.05 if eps is None else eps, scripted=scripted)
     elif name == "long8b":
@@ -69,13 +73,28 @@ def make_setup(name: str, eps, scripted: bool, batch=None) -> wl.SamplerSetup:
             s = dataclasses.replace(s, eps=eps)
     else:
         raise SystemExit(f"unknown workload {name}")
+    import dataclasses
     if batch is not None:
         if not 1 <= batch <= 64:
             raise SystemExit(f"--batch must be in [1, 64], got {batch}")
-        import dataclasses
         s = dataclasses.replace(s, batch=batch)
+    if gate_q is not None:
+        if gate_q > 1.0:
+            raise SystemExit(f"--gate-q must be <= 1 (< 0: gate off), got {gate_q}")
+        s = dataclasses.replace(s, gate_q=gate_q)
+    if ablation not in ("none", "no_kv_cache", "gate_only"):
+        raise SystemExit(f"unknown ablation {ablation}")
+    if ablation == "gate_only" and s.gate_q < 0:
+        raise SystemExit("--ablation gate_only needs the confidence gate (--gate-q in [0, 1])")
+    s = dataclasses.replace(s, no_kv_cache=ablation == "no_kv_cache",
+                            gate_only=ablation == "gate_only")
     s.validate()
     return s
+
+
+def setup_from_args(args) -> wl.SamplerSetup:
+    return make_setup(args.workload, args.eps, args.scripted, args.batch, args.gate_q,
+                      args.ablation)
 
 
 DATA_DESC = "synthetic (random-init N(0,0.02) weights, uniform random prompt ids)"
@@ -89,7 +108,10 @@ def workload_config(args, setup: wl.SamplerSetup, world: int) -> dict:
                         f"(N={setup.n_ctx}), {T} steps, blocks of {setup.block_len}, "
                         f"{setup.tokens_per_step} token(s)/step, eps={setup.eps}"
                         + (f", gate q={setup.gate_q}" if setup.gate_q >= 0 else "")
-                        + (", scripted lock schedule" if setup.scripted else ""),
+                        + (", scripted lock schedule" if setup.scripted else "")
+                        + (", ablation: no KV cache (active rows' keys only)"
+                           if setup.no_kv_cache else "")
+                        + (", ablation: confidence gate only" if setup.gate_only else ""),
             "bench_step": f"one full decode ({T} denoising steps)",
             "global_batch": world * setup.batch, "seq_len": setup.n_ctx,
             "parallelism": f"replicas{world}",
@@ -309,7 +331,7 @@ def run_ours(args, rank: int, world: int):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    setup = make_setup(args.workload, args.eps, args.scripted, args.batch)
+    setup = setup_from_args(args)
     shape = setup.shape
     T = setup.steps
     ranks = Ranks(world, "nccl", dev)
@@ -318,6 +340,7 @@ def run_ours(args, rank: int, world: int):
     weights = wl.torch_weights(shape, dev)
     torch.cuda.synchronize()
     model = rt.Model(shape, weights, "bf16")
+    model.set_ablation(no_kv_cache=setup.no_kv_cache, gate_only=setup.gate_only)
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, T, setup.block_len,
                    setup.tokens_per_step, setup.eps, setup.gate_q, setup.scripted)
     prompts = wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab, shape.mask_id,
@@ -491,7 +514,7 @@ def run_reference(args, rank: int, world: int):
     bench step is one bounded sample (see oracle_sample)."""
     if rank != 0:
         return None
-    setup = make_setup(args.workload, args.eps, args.scripted, args.batch)
+    setup = setup_from_args(args)
     T = setup.steps
     # the dense trajectory shape of the scripted/KL schedule is not known on the
     # CPU side; use the linear decay from N to the masked-only floor
@@ -529,6 +552,10 @@ def main():
     ap.add_argument("--scripted", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per GPU (default: the workload's own batch)")
+    ap.add_argument("--gate-q", type=float, default=None,
+                    help="confidence-gate quantile (default: the workload's; < 0 = off)")
+    ap.add_argument("--ablation", default="none", choices=["none", "no_kv_cache", "gate_only"],
+                    help="run one of the pages' ablations instead of the method")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "surelock_bench"),
                     help="where the per-rank clock samples (CSV) are written")

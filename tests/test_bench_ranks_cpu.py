@@ -64,3 +64,32 @@ def test_batch_override():
     for bad in (0, 65):
         with pytest.raises(SystemExit):
             bench.make_setup("full8b", None, False, bad)
+
+
+def test_ablation_and_gate_flags():
+    import types
+    import pytest
+    sys.path.insert(0, ROOT)
+    import bench
+    s = bench.make_setup("full8b", None, False, None, None, "none")
+    assert not s.no_kv_cache and not s.gate_only and s.gate_q < 0
+    s = bench.make_setup("full8b", None, False, None, None, "no_kv_cache")
+    assert s.no_kv_cache and not s.gate_only
+    args = types.SimpleNamespace(workload="full8b")
+    assert "no KV cache" in bench.workload_config(args, s, 1)["workload"]
+    with pytest.raises(SystemExit):                  # gate-only needs the gate
+        bench.make_setup("full8b", None, False, None, None, "gate_only")
+    s = bench.make_setup("full8b", None, False, None, 0.5, "gate_only")
+    assert s.gate_only and s.gate_q == 0.5
+    cfg = bench.workload_config(args, s, 1)["workload"]
+    assert "gate q=0.5" in cfg and "confidence gate only" in cfg
+    for bad in (dict(gate_q=1.5), dict(ablation="nope")):
+        kw = dict(gate_q=None, ablation="none")
+        kw.update(bad)
+        with pytest.raises(SystemExit):
+            bench.make_setup("full8b", None, False, None, kw["gate_q"], kw["ablation"])
+    # the command line reaches the same setup
+    a = types.SimpleNamespace(workload="long8b", eps=None, scripted=False, batch=2, gate_q=None,
+                              ablation="no_kv_cache")
+    s = bench.setup_from_args(a)
+    assert (s.batch, s.n_ctx, s.no_kv_cache, s.gate_q) == (2, 2048, True, 0.5)
