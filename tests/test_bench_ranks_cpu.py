@@ -93,3 +93,38 @@ def test_ablation_and_gate_flags():
                               ablation="no_kv_cache")
     s = bench.setup_from_args(a)
     assert (s.batch, s.n_ctx, s.no_kv_cache, s.gate_q) == (2, 2048, True, 0.5)
+
+
+def test_clock_sampler_summary(tmp_path):
+    """The clocks object of the JSON line from nvidia-smi's CSV rows: median SM
+    clock over the rows under load (power > 200 W), the max clock, and the
+    throttle reasons seen active under load."""
+    sys.path.insert(0, ROOT)
+    import bench
+    rows = [
+        "0, 1980, 1965, 120.5, 0x0, Not Active, Not Active, Not Active, Not Active",   # idle
+        "0, 1830, 1965, 980.1, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1820, 1965, 990.7, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1845, 1965, 960.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+    ]
+    path = tmp_path / "clocks.csv"
+    path.write_text("\n".join(rows) + "\n")
+
+    class Done:                       # stands in for the finished nvidia-smi process
+        def terminate(self): pass
+        def wait(self, timeout=None): return 0
+        def kill(self): pass
+
+    cs = bench.ClockSampler("GPU-x", str(path))
+    cs.proc, cs.f = Done(), open(path)
+    out = cs.stop()
+    assert out["sm_mhz"] == 1830.0 and out["sm_max_mhz"] == 1965.0
+    assert out["samples"] == 4 and out["samples_under_load"] == 3
+    assert out["reasons"] == ["sw_power_cap"] and out["power_w_max"] == 990.7
+    # a hardware slowdown under load is reported by name
+    path.write_text("0, 1500, 1965, 700.0, 0x8, Active, Not Active, Not Active, Not Active\n")
+    cs.f = open(path)
+    assert bench.ClockSampler.stop(cs)["reasons"] == ["hw_slowdown"]
+    # no nvidia-smi: no clocks object
+    assert bench.ClockSampler("GPU-x", str(path)).stop() is None
