@@ -1,11 +1,13 @@
-"""The replica plumbing of bench.py on two CPU ranks (gloo): the barrier, the
-max over ranks of a time, per-replica prompts, the whole-job rate, and that the
-reference arm does its work on rank 0 only."""
+"""bench.py's host logic on the CPU: the replica plumbing on two gloo ranks (the
+barrier, the max over ranks of a time, per-replica prompts, the whole-job rate,
+the reference arm on rank 0 only), the workload flags, the clock summary, and
+the per-step work behind the roofline fraction."""
 import json
 import os
 import socket
 import sys
 
+import numpy as np
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -128,3 +130,33 @@ def test_clock_sampler_summary(tmp_path):
     assert bench.ClockSampler.stop(cs)["reasons"] == ["hw_slowdown"]
     # no nvidia-smi: no clocks object
     assert bench.ClockSampler("GPU-x", str(path)).stop() is None
+
+
+def test_step_work_against_the_oracle_flop_model():
+    """The bench's per-step roofline work: FLOPs equal the oracle's FLOP model
+    (written separately), and the bytes at the LLaDA-8B shape match the stated
+    figures (15.0 GB of weights; K/V, posterior and gather terms)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    from oracle import surelock as osl
+    shape = wl.LLADA8B
+    for m, n in ((1, 384), (58, 384), (384, 384), (2048, 2048)):
+        fl, _ = bench.step_work(shape, m, 1, n)
+        assert fl == osl.flops_per_step(shape, m, n)
+    _, b0 = bench.step_work(shape, 0, 1, 384)
+    d, L, V = shape.d_model, shape.n_layers, shape.vocab
+    weights = b0 - 1 * L * 2 * 384 * d * 2
+    assert abs(weights / 1e9 - 15.0) < 0.05          # 2 (L (4d^2 + 3df) + Vd) bytes
+    _, b1 = bench.step_work(shape, 1, 1, 384)
+    assert b1 - b0 == L * 2 * d * 2 + 4 * V + 2 * d  # per active row: K/V write, posterior, gather
+    _, b4 = bench.step_work(shape, 0, 4, 384)
+    assert b4 - b0 == 3 * L * 2 * 384 * d * 2        # every sequence's cache is read
+
+
+def test_trajectory_from_lock_steps():
+    sys.path.insert(0, ROOT)
+    import bench
+    lock_t = np.array([-1, 0, 0, 2, -1, 1, 2, 2], dtype=np.int32)
+    # all 8 rows active at step 0; 2 locked at step 0, 1 at step 1, 3 at step 2
+    assert bench.trajectory_from_lock_t(lock_t, 4).tolist() == [8, 6, 5, 2]
