@@ -1,8 +1,11 @@
 """The C ABI library loads without a GPU and exports everything the header
-declares; host-side argument checks reject bad calls before touching CUDA."""
+declares; the header is plain C and every entry point links from a C program;
+host-side argument checks reject bad calls before touching CUDA."""
 import ctypes as C
 import os
 import re
+import shutil
+import subprocess
 
 import pytest
 
@@ -71,3 +74,37 @@ def test_host_side_argument_checks(lib):
     assert lib.sl_gemm_bf16(1, 16, 8, 128, 16, None, 128, 16, 130, None, 128, 1, 0, None) == A.SL_ERR_INVALID
     assert lib.sl_gemm_bf16(0, 16, 8, 128, 16, None, 128, 16, 132, None, 128, 1, 0, None) == A.SL_ERR_INVALID
     assert lib.sl_gemm_bf16(0, 16, 8, 128, 16, None, 128, 16, 64, None, 128, 1, 0, None) == A.SL_ERR_INVALID
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not on PATH")
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/surelock.h compiles as strict C99 (no C++ in the boundary), and a
+    C program that takes the address of every declared entry point links
+    against libsurelock.so and runs a host-side check through it."""
+    from token_locking_b200 import _abi
+    from token_locking_b200 import build
+    build.build()
+    names = sorted(_declared())
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        '#include "surelock.h"\n#include <string.h>\n'
+        "typedef void (*fnp)(void);\n"
+        "static const fnp entry_points[] = {\n"
+        + "".join(f"  (fnp){n},\n" for n in names)
+        + "};\n"
+        "int main(void) {\n"
+        "  sl_lock_params lp = {0.05f, -1.0f, 1, -1, 0};\n"
+        "  (void)lp;\n"
+        "  if (sizeof(entry_points) / sizeof(entry_points[0]) != %d) return 2;\n" % len(names)
+        + "  if (!strstr(sl_version(), \"sm_100a\")) return 3;\n"
+        "  return sl_model_set_ablation(NULL, SL_ABLATE_NO_KV_CACHE) == SL_ERR_INVALID ? 0 : 4;\n"
+        "}\n")
+    exe = str(tmp_path / "use_abi")
+    libdir = os.path.dirname(_abi.LIB_PATH)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+           "-I" + os.path.join(ROOT, "include"), str(src), "-L" + libdir, "-lsurelock",
+           "-Wl,-rpath," + libdir, "-o", exe]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-4000:]
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
