@@ -19,9 +19,10 @@ captures).
       Sweep of the tensor-core GEMM tilings (tile width, 128/256-row tiles,
       K splits) on the LLaDA-8B projection shapes; one JSON line per tiling.
 
-Each case prints one JSON line: mean time per call (CUDA events, after
-warm-up, L2 flushed between calls by a 256 MB write), the roofline time of the
-case's algorithmic work and their ratio.
+Each case prints one JSON line: the median time per call over --iters calls
+(default 20; CUDA events, after 5 warm-up calls, L2 flushed before every call
+by a 256 MB write), the roofline time of the case's algorithmic work and their
+ratio.  The attn case times a warm back-to-back burst instead (mean per call).
 """
 from __future__ import annotations
 
@@ -58,11 +59,16 @@ class _Flush:
         self.buf.fill_(1)
 
 
-def _time(fn, iters, warmup, flush):
+WARMUP = 5
+
+
+def _time(fn, iters, flush, warmup=WARMUP):
+    """Median CUDA-event time (ms) of one call over `iters` calls, each after an
+    L2 flush, following `warmup` untimed calls."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    tot = 0.0
+    times = []
     for _ in range(iters):
         flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -70,8 +76,8 @@ def _time(fn, iters, warmup, flush):
         fn()
         e1.record()
         torch.cuda.synchronize()
-        tot += e0.elapsed_time(e1)
-    return tot / iters
+        times.append(e0.elapsed_time(e1))
+    return float(np.median(times))
 
 
 def layer_work(shape, M, N):
@@ -109,7 +115,7 @@ def bench_layer(args, dev):
             h.copy_(h0)
             rt.layer_forward(model, cache, act, 0, h)
 
-        ms = _time(fn, args.iters, 3, flush)
+        ms = _time(fn, args.iters, flush)
         model.timing_enable(True)
         model.timing_read(reset=True)
         fn()
@@ -158,7 +164,7 @@ def bench_lock(args, dev):
                            eps=eps, gate_q=wl.LOCK_MICRO_GATE_Q)
 
             act.reset()
-            ms = _time(fn, args.iters, 3, flush)
+            ms = _time(fn, args.iters, flush)
             n_lock = int(outs["lock"].sum())
             rt.compact_active(act, outs["lock"], locked, lock_t, 1)
             m_after = int(act.counts()[0])
@@ -326,7 +332,7 @@ def bench_gemm(args, dev):
                     def fn():
                         rt.gemm_bf16(epi, a, b, out, b2=b2, bn=bn, splits=sp, variant=variant)
 
-                    ms = _time(fn, args.iters, 2, flush)
+                    ms = _time(fn, args.iters, flush)
                     by = 2.0 * (N * K + M * K + M * N)
                     fl = 2.0 * M * N * K
                     print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": bn,
@@ -348,7 +354,7 @@ def bench_gemm(args, dev):
             def fn():
                 rt.gemm_bf16(epi, a, b, out, b2=b2, bn=0, splits=0)
 
-            ms = _time(fn, args.iters, 2, flush)
+            ms = _time(fn, args.iters, flush)
             print(json.dumps({"case": "gemm", "M": M, "gemm": name, "bn": 0, "variant": -1,
                               "splits": 0, "us": round(ms * 1e3, 2),
                               "GBps": round(2.0 * (N * K + M * K + M * N) / ms / 1e6, 1)}),
@@ -363,7 +369,7 @@ def main():
     ap.add_argument("--tiles", default=None, help="gemm case: fixed bn:variant:splits list")
     ap.add_argument("--no-tune", action="store_true")
     ap.add_argument("--m", default=None)
-    ap.add_argument("--iters", type=int, default=10)
+    ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--steps", type=int, default=8)
     ap.add_argument("--skip", type=int, default=0, help="decode: denoising steps run before timing")
     ap.add_argument("--windows", default=None,
