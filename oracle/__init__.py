@@ -27,6 +27,6 @@ Pins: every function here is checked by `tests/test_oracle_*.py` against closed
 forms, invariants the pages state, special cases that reduce to a library
 routine, or brute force on tiny inputs.  Two parts carry no such pin
 ("parity unpinned"): the error bound of Theorem 1, whose constants the pages do
-not define (only a diagnostic ratio is reported), and full-model values at the
-LLaDA-8B shape, which no page prints.
+not define (nothing here computes it), and full-model values at the LLaDA-8B
+shape, which no page prints.
 """
