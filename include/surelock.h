@@ -160,7 +160,8 @@ typedef struct sl_lock_params {
 } sl_lock_params;
 
 /* The sure test on the active rows (Paper-Notes, "lock criterion" and
- * "optional confidence gate"; Abstract, "unmasked position"):
+ * "optional confidence gate"; Abstract: the test applies to positions that are
+ * no longer masked):
  *   lse_j = logsumexp(z_cur[row_j]);  log p = z - lse
  *   D_j = max(0, sum_v p_cur (log p_cur - log p_prev))
  *       = max(0, E_pcur[z_cur - z_prev] - lse_cur + lse_prev)
@@ -181,8 +182,8 @@ sl_status sl_kl_lock(sl_active *a, int vocab, int mask_id, int logits_dtype,
 /* Sampler step: among the masked active rows with local position in
  * [block_lo, block_hi), unmask the k with the highest confidence (ties to the
  * lower position): tokens[row] = argmax, masked[row] = 0.  This is the
- * unmodified sampler the pages compare against (Abstract: "the same sampler
- * without locking"). */
+ * unmodified sampler the pages compare against (Abstract: the baseline is this
+ * sampler with locking switched off). */
 sl_status sl_unmask_topk(sl_active *a, const float *d_conf, const int32_t *d_argmax,
                          int block_lo, int block_hi, int k, int32_t *d_tokens,
                          uint8_t *d_masked, void *stream);
@@ -300,8 +301,9 @@ sl_status sl_model_set_ablation(sl_model *m, int flags);
 /* Semi-autoregressive SureLock decode driven by the library: prompt_len given
  * tokens then gen_len [MASK] tokens; gen region split in blocks of block_len,
  * steps/(gen_len/block_len) steps per block, tokens_per_step unmasked per step
- * (the unmodified sampler the pages compare against, Abstract: "the same
- * sampler without locking", with the sure test of sl_kl_lock between steps). */
+ * (the unmodified sampler the pages compare against, Abstract: their baseline
+ * is this sampler with locking switched off; here the sure test of sl_kl_lock
+ * runs between steps). */
 typedef struct sl_sampler_params {
   int prompt_len, gen_len, steps, block_len, tokens_per_step;
   float eps;             /* KL threshold; eps <= 0 disables locking */

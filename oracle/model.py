@@ -36,18 +36,22 @@ import numpy as np
 
 
 def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
-    """y = x / sqrt(mean(x^2) + eps) * g over the last axis."""
+    """y = x / sqrt(mean(x^2) + eps) * g over the last axis.
+    Reading (the pages are silent on the model): RMSNorm with per-channel gains."""
     ms = np.mean(x * x, axis=-1, keepdims=True)
     return x / np.sqrt(ms + eps) * g
 
 
 def silu(x: np.ndarray) -> np.ndarray:
-    """x * sigmoid(x)."""
+    """x * sigmoid(x), the gate of the SwiGLU FFN (reading: the pages are silent
+    on the FFN; LLaDA-style SwiGLU)."""
     return x / (1.0 + np.exp(-x))
 
 
 def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
     """Rotate-half rotary embedding.  x: [M, H, dh], pos: [M] absolute positions.
+    Reading (the pages are silent on positions): rotate-half RoPE at the
+    absolute position, so active and cached keys keep their places.
 
     For i < dh/2, the pair (x_i, x_{i+dh/2}) is rotated by angle pos * theta^(-2i/dh):
       out_i        = x_i cos - x_{i+dh/2} sin
@@ -66,6 +70,7 @@ def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
 
 
 def softmax(s: np.ndarray, axis: int = -1) -> np.ndarray:
+    """exp(s - max) / sum exp(s - max) along `axis` (the attention weights)."""
     m = np.max(s, axis=axis, keepdims=True)
     e = np.exp(s - m)
     return e / np.sum(e, axis=axis, keepdims=True)
@@ -75,7 +80,10 @@ def attention(q: np.ndarray, k_all: np.ndarray, v_all: np.ndarray) -> np.ndarray
     """Bidirectional attention of M queries over all N keys of one sequence.
 
     q: [M, H, dh]; k_all, v_all: [N, H, dh] (cached rows for locked positions,
-    fresh rows for active ones).  Returns [M, H, dh]."""
+    fresh rows for active ones).  Returns [M, H, dh].
+    Abstract: the keys and values of a locked position stay cached and the
+    active positions keep attending to them; Paper-Notes, "permanent locking":
+    K^all[L_t] <- C.k[L_t]."""
     dh = q.shape[-1]
     qh = np.transpose(q, (1, 0, 2))               # [H, M, dh]
     kh = np.transpose(k_all, (1, 2, 0))           # [H, dh, N]
@@ -94,7 +102,10 @@ def layer_forward(shape, lw: dict, h: np.ndarray, pos: np.ndarray,
     ck, cv: [N, d] this layer's cache for the sequence; rows `pos` are
     overwritten with the fresh k, v (the scatter into C), all other rows are
     read as they are (frozen K/V of locked positions).  With no_kv_cache the
-    queries attend to the rows `pos` only.  Returns the block output [M, d]."""
+    queries attend to the rows `pos` only.  Returns the block output [M, d].
+    Abstract: locked positions skip the query projection and feed-forward
+    sublayers; gist.science/it section 2, "Azione di Blocco": their block input
+    is frozen and their K/V are cached for every layer."""
     H, dh = shape.n_heads, shape.head_dim
     M = h.shape[0]
     a = rmsnorm(h, lw["attn_norm"], shape.rms_eps)
@@ -123,7 +134,9 @@ def forward_active(shape, w: dict, tokens: np.ndarray, pos: np.ndarray,
     updated in place at rows `pos`.  If block_inputs is a list, the input h of
     every block is appended to it (used to check that K/V of locked rows are
     reproducible from their frozen block inputs).  no_kv_cache: the ablation
-    in which the active rows attend to one another only."""
+    in which the active rows attend to one another only.
+    gist.science/nl section 2, "Complexiteitsvermindering": the step costs
+    O(M N d) for attention and O(M d^2) for the projections and FFN."""
     h = w["tok_emb"][tokens[pos]]
     for l, lw in enumerate(w["layers"]):
         if block_inputs is not None:
@@ -134,7 +147,9 @@ def forward_active(shape, w: dict, tokens: np.ndarray, pos: np.ndarray,
 
 
 def kv_of_block_input(shape, lw: dict, h: np.ndarray, pos: np.ndarray):
-    """k (after RoPE) and v [M, d] that a block would produce from input h."""
+    """k (after RoPE) and v [M, d] that a block would produce from input h
+    (gist.science/it section 2, "Azione di Blocco": a locked row's cached K/V
+    are those of its frozen block input)."""
     H, dh = shape.n_heads, shape.head_dim
     M = h.shape[0]
     a = rmsnorm(h, lw["attn_norm"], shape.rms_eps)
@@ -145,8 +160,9 @@ def kv_of_block_input(shape, lw: dict, h: np.ndarray, pos: np.ndarray):
 
 def forward_full(shape, w: dict, tokens: np.ndarray) -> np.ndarray:
     """Logits [N, V] of the unmodified denoiser on every position of one
-    sequence (the sampler without locking).  Written without any gather,
-    cache or scatter, so it is an independent restatement of the same block."""
+    sequence: the comparison run of the Abstract, the sampler with locking
+    switched off.  Written without any gather, cache or scatter, so it is an
+    independent restatement of the same block."""
     H, dh = shape.n_heads, shape.head_dim
     N = tokens.shape[0]
     pos = np.arange(N)

@@ -16,7 +16,7 @@ Diffusion-LM Decoding"):
     active tokens (gist.science/it section 2, "Filtro di Confidenza").
   * After the lock step t*, the posterior stays frozen: p_hat_t = p_{t*}
     (Paper-Notes, "permanent locking", core idea).
-  * The comparison sampler is "the same sampler without locking" (Abstract).
+  * The comparison run is the same sampler with locking switched off (Abstract).
 
 Readings where the pages are silent (the plainest reading consistent with them):
   R4  "unmasked" means not [MASK] in the step's input x_t; prompt positions count.
@@ -40,7 +40,7 @@ Ablations (Paper-Notes, ablation table):
     inequality is dropped; eligibility stays as in the full test, so nothing
     locks at t = 0 and a row is first tested the step after it is unmasked.
     eps plays no part; the gate must be on (gate_q >= 0).
-  * no KV cache ("locked tokens cannot be attended"): the denoiser's queries
+  * no KV cache (the table's note: locked tokens drop out of attention): the denoiser's queries
     see the keys of the active rows only (model.forward_active, no_kv_cache).
 """
 from __future__ import annotations
@@ -230,7 +230,7 @@ def surelock_sampler(shape, w: dict, tokens: np.ndarray, masked: np.ndarray, set
 
 
 def plain_sampler(shape, w: dict, tokens: np.ndarray, masked: np.ndarray, setup):
-    """The same sampler without locking: every step runs the full denoiser on all
+    """The sampler with locking switched off: every step runs the full denoiser on all
     N positions (no active set, no cache).  Returns (final tokens, final
     log-probs [B, N, V])."""
     tok = tokens.astype(np.int32).copy()
