@@ -54,25 +54,30 @@ from . import model as om
 
 
 def log_softmax(z: np.ndarray) -> np.ndarray:
-    """log p = z - logsumexp(z) over the last axis."""
+    """log p = z - logsumexp(z) over the last axis: the per-position posterior
+    p_t that the lock criterion compares (Paper-Notes, "lock criterion")."""
     m = np.max(z, axis=-1, keepdims=True)
     return z - (m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True)))
 
 
 def kl_rows(lp_cur: np.ndarray, lp_prev: np.ndarray) -> np.ndarray:
-    """D = max(0, sum_v p_cur(v) (log p_cur(v) - log p_prev(v))) per row."""
+    """D = max(0, sum_v p_cur(v) (log p_cur(v) - log p_prev(v))) per row: the
+    step-to-step KL of the lock criterion (Paper-Notes, "lock criterion";
+    gist.science/it section 2, "Criterio di Blocco"), clamped at 0 (reading R7)."""
     p = np.exp(lp_cur)
     return np.maximum(0.0, np.sum(p * (lp_cur - lp_prev), axis=-1))
 
 
 def uncertainty(lp_cur: np.ndarray) -> np.ndarray:
-    """u = 1 - max_v p(v) per row (all vocab entries, [MASK] included)."""
+    """u = 1 - max_v p(v) per row (all vocab entries, [MASK] included): the
+    gate's uncertainty (Paper-Notes, "optional confidence gate")."""
     return 1.0 - np.exp(np.max(lp_cur, axis=-1))
 
 
 def prediction(lp_cur: np.ndarray, mask_id: int):
     """(conf, pred): the largest probability over v != mask_id and its lowest
-    index; this is what the sampler unmasks with."""
+    index; this is what the sampler unmasks with (readings R9, R11: the pages
+    name the sampler but not its details)."""
     lp = np.array(lp_cur, copy=True)
     lp[..., mask_id] = -np.inf
     pred = np.argmax(lp, axis=-1)           # first occurrence = lowest id
@@ -81,7 +86,9 @@ def prediction(lp_cur: np.ndarray, mask_id: int):
 
 
 def gate_threshold(u_active: np.ndarray, q: float) -> float:
-    """q-quantile of u over the active rows, lower order statistic."""
+    """q-quantile of u over the active rows, lower order statistic: q_m(u_t) of
+    the gate (Paper-Notes, "optional confidence gate"; gist.science/it section
+    2, "Filtro di Confidenza"; reading R8 for the order statistic)."""
     m = u_active.shape[0]
     if m == 0:
         return np.inf
@@ -93,7 +100,10 @@ def lock_decision(D, u, masked, has_prev, eps: float, gate_q: float, thr,
                   gate_only: bool = False):
     """lock_j = eps>0 and not masked_j and has_prev_j and D_j<=eps and
     (gate off or u_j <= thr).  gate_only: lock_j = not masked_j and has_prev_j
-    and u_j <= thr, whatever eps and D."""
+    and u_j <= thr, whatever eps and D.
+    Paper-Notes, "lock criterion" and "optional confidence gate"; Abstract:
+    only unmasked positions are tested; readings R4-R6; gate only: the
+    Paper-Notes ablation table."""
     if gate_only:
         if gate_q < 0:
             raise ValueError("the gate-only criterion needs the confidence gate (gate_q >= 0)")
@@ -107,7 +117,8 @@ def lock_decision(D, u, masked, has_prev, eps: float, gate_q: float, thr,
 
 
 def scripted_locks(D, masked, has_prev, pos, n_lock: int):
-    """Lock the n_lock eligible rows with the smallest (D, position)."""
+    """Lock the n_lock eligible rows with the smallest (D, position): the
+    scripted schedule of the benchmark (a fixed M_t decay, not from the pages)."""
     elig = (~masked.astype(bool)) & has_prev.astype(bool)
     idx = np.nonzero(elig)[0]
     order = idx[np.lexsort((pos[idx], D[idx]))]
@@ -117,14 +128,16 @@ def scripted_locks(D, masked, has_prev, pos, n_lock: int):
 
 
 def compact(act: np.ndarray, lock: np.ndarray) -> np.ndarray:
-    """Stable removal of the locked rows from the active list."""
+    """Stable removal of the locked rows from the active list: the active set
+    only shrinks (Paper-Notes, "permanent locking"; reading R9 for the order)."""
     return act[~lock]
 
 
 def unmask_select(pos: np.ndarray, conf: np.ndarray, masked_rows: np.ndarray,
                   lo: int, hi: int, k: int) -> np.ndarray:
     """Indices (into the active rows) of the k masked rows in [lo, hi) with the
-    highest confidence, ties to the lower position."""
+    highest confidence, ties to the lower position (reading R11: the
+    semi-autoregressive sampler the pages compare against)."""
     cand = np.nonzero(masked_rows.astype(bool) & (pos >= lo) & (pos < hi))[0]
     order = cand[np.lexsort((pos[cand], -conf[cand]))]
     return order[:k]
@@ -150,6 +163,8 @@ class State:
 
 
 def init_state(shape, tokens: np.ndarray, masked: np.ndarray, dtype=np.float64) -> State:
+    """A_0 = every position, nothing locked, no previous posterior (reading R5),
+    an all-zero cache."""
     B, N = tokens.shape
     L, d, V = shape.n_layers, shape.d_model, shape.vocab
     return State(tokens=tokens.astype(np.int32).copy(), masked=masked.astype(bool).copy(),
@@ -165,7 +180,8 @@ def lock_test(lp: np.ndarray, lp_prev: np.ndarray, has_prev: np.ndarray,
               masked: np.ndarray, pos: np.ndarray, shape, setup, t: int,
               n_active_target: Optional[int] = None):
     """The sure test of one sequence's active rows.  Returns a dict with D, u,
-    conf, pred, thr and the lock flags."""
+    conf, pred, thr and the lock flags (the pieces above, in the order of
+    Paper-Notes, "lock criterion" and "optional confidence gate")."""
     D = np.full(lp.shape[0], np.inf, dtype=lp.dtype)
     hp = has_prev.astype(bool)
     if np.any(hp):
@@ -188,7 +204,9 @@ def step(shape, w: dict, st: State, setup, t: int, record_block_inputs: bool = F
     Order: forward on A_t (fresh K/V scattered into C) -> log-softmax -> sure
     test on the mask flags at the start of the step -> unmask the top-k of the
     current block -> record p_t for the active rows (frozen for those that lock)
-    -> remove the locked rows from A_t.  Returns one record per sequence."""
+    -> remove the locked rows from A_t.  Returns one record per sequence.
+    Paper-Notes, "Method: overall framework" (compute A_t, serve L_t from the
+    cache) and "permanent locking" (a locked row's posterior is frozen)."""
     out = []
     lo, hi = setup.block_bounds(t)
     for b in range(st.tokens.shape[0]):
@@ -217,7 +235,8 @@ def step(shape, w: dict, st: State, setup, t: int, record_block_inputs: bool = F
 def surelock_sampler(shape, w: dict, tokens: np.ndarray, masked: np.ndarray, setup,
                      dtype=np.float64, keep_records: bool = False):
     """Full SureLock decode.  Returns (final tokens, final log-probs [B, N, V],
-    active counts per step [T+1, B], per-step records if keep_records)."""
+    active counts per step [T+1, B], per-step records if keep_records).
+    Paper-Notes, "Method: overall framework"; "key findings": M_t only falls."""
     st = init_state(shape, tokens, masked, dtype)
     counts = [[len(a) for a in st.act]]
     recs = []
@@ -253,6 +272,8 @@ def plain_sampler(shape, w: dict, tokens: np.ndarray, masked: np.ndarray, setup)
 
 def flops_per_step(shape, m_rows: int, n_ctx_rows: int) -> float:
     """Algorithmic FLOPs of one step on m_rows active rows attending to
-    n_ctx_rows keys: 2 M (L (4 d^2 + 3 d f) + V d) + 4 L M N d."""
+    n_ctx_rows keys: 2 M (L (4 d^2 + 3 d f) + V d) + 4 L M N d (gist.science/nl
+    section 2, "Complexiteitsvermindering": O(M d^2) for the projections and FFN,
+    O(M N d) for attention)."""
     d, f, V, L = shape.d_model, shape.d_ffn, shape.vocab, shape.n_layers
     return 2.0 * m_rows * (L * (4 * d * d + 3 * d * f) + V * d) + 4.0 * L * m_rows * n_ctx_rows * d
