@@ -50,6 +50,7 @@ def attention_head(q, keys, vals):
 
 
 def silu(x):
+    """x * sigmoid(x) on one scalar."""
     return x / (1.0 + math.exp(-x))
 
 
@@ -94,6 +95,7 @@ def forward_active(shape, w, tokens, pos, ck, cv, no_kv_cache=False):
 
 
 def log_softmax_row(z):
+    """z - log(sum exp z) for one row, shifted by its max."""
     mx = max(z)
     lse = mx + math.log(sum(math.exp(v - mx) for v in z))
     return [v - lse for v in z]
