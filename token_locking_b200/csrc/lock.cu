@@ -1,5 +1,10 @@
 // The sure test, the confidence gate, compaction of the active set and the
-// sampler's unmasking step.
+// sampler's unmasking step: the step-to-step KL test D_t = KL(p_t || p_{t-1})
+// <= eps at unmasked positions (Paper-Notes, "lock criterion"; Abstract), the
+// optional gate u_t = 1 - max p_t <= q_m(u_t) over the active tokens
+// (Paper-Notes, "optional confidence gate"; gist.science/it section 2,
+// "Filtro di Confidenza"), and the active set that only shrinks (Paper-Notes,
+// "permanent locking").
 //
 // lock_stats: one streaming read of the current and previous logits of every
 //   active row.  Each CTA reduces a contiguous vocab chunk of one row with an
