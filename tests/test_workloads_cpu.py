@@ -104,3 +104,28 @@ def test_weights_reproducible_and_scaled():
     np.testing.assert_array_equal(j["lm_head"], a["lm_head"])
     g = np.concatenate([lw["ffn_norm"] for lw in j["layers"]])
     assert abs(g.mean() - 1.0) < 0.05 and 0.05 < g.std() < 0.15
+
+
+def test_torch_weights_recipe():
+    """The device-side generator of the benchmark's weights, run on the CPU:
+    bf16 [out, in] matrices N(0, std), unit gains, reproducible from the seed,
+    and `layers` truncating the same draw sequence."""
+    shape = wl.ModelShape(n_layers=3, d_model=128, n_heads=1, head_dim=128, d_ffn=256, vocab=512,
+                          mask_id=511, rope_theta=1e4)
+    cpu = torch.device("cpu")
+    a = wl.torch_weights(shape, cpu)
+    b = wl.torch_weights(shape, cpu)
+    assert a["tok_emb"].dtype == torch.bfloat16 and tuple(a["tok_emb"].shape) == (512, 128)
+    assert tuple(a["layers"][0]["w_gate"].shape) == (256, 128)
+    assert tuple(a["layers"][0]["w_down"].shape) == (128, 256)
+    assert tuple(a["lm_head"].shape) == (512, 128) and len(a["layers"]) == 3
+    assert torch.equal(a["layers"][2]["wv"], b["layers"][2]["wv"])
+    assert torch.all(a["final_norm"] == 1) and torch.all(a["layers"][1]["ffn_norm"] == 1)
+    allw = torch.cat([a["tok_emb"].float().ravel()] +
+                     [v.float().ravel() for lw in a["layers"] for k, v in lw.items()
+                      if not k.endswith("norm")])
+    assert abs(allw.std().item() - 0.02) < 0.001 and abs(allw.mean().item()) < 0.001
+    # fewer layers: the same first draws
+    c = wl.torch_weights(shape, cpu, layers=1)
+    assert len(c["layers"]) == 1 and torch.equal(c["layers"][0]["wq"], a["layers"][0]["wq"])
+    assert not torch.equal(wl.torch_weights(shape, cpu, seed=7)["lm_head"], a["lm_head"])
