@@ -63,9 +63,13 @@ def log_softmax(z: np.ndarray) -> np.ndarray:
 def kl_rows(lp_cur: np.ndarray, lp_prev: np.ndarray) -> np.ndarray:
     """D = max(0, sum_v p_cur(v) (log p_cur(v) - log p_prev(v))) per row: the
     step-to-step KL of the lock criterion (Paper-Notes, "lock criterion";
-    gist.science/it section 2, "Criterio di Blocco"), clamped at 0 (reading R7)."""
+    gist.science/it section 2, "Criterio di Blocco"), clamped at 0 (reading R7).
+    A term with p_cur(v) = 0 (a -inf logit) is 0, the usual 0 log 0 = 0 of the
+    KL's definition; p_cur(v) > 0 with p_prev(v) = 0 makes D infinite."""
     p = np.exp(lp_cur)
-    return np.maximum(0.0, np.sum(p * (lp_cur - lp_prev), axis=-1))
+    with np.errstate(invalid="ignore"):
+        terms = np.where(p > 0, p * (lp_cur - lp_prev), 0.0)
+    return np.maximum(0.0, np.sum(terms, axis=-1))
 
 
 def uncertainty(lp_cur: np.ndarray) -> np.ndarray:

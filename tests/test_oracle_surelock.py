@@ -35,6 +35,30 @@ def test_kl_bernoulli_closed_form():
     assert abs(d_rev[0] - c["kl"]) > 1e-3
 
 
+def test_kl_with_zero_probability_entries():
+    """Entries with a -inf logit have probability 0 and add no term to the KL
+    (0 log 0 = 0 in its definition), so a two-outcome pair padded with -inf
+    logits keeps the Bernoulli closed form; an outcome the previous posterior
+    gave probability 0 while the current one does not makes D infinite."""
+    c = GOLD["bernoulli_kl"]
+    ninf = -np.inf
+    lp = np.array([[np.log(c["p"][0]), ninf, np.log(c["p"][1]), ninf]])
+    lq = np.array([[np.log(c["q"][0]), ninf, np.log(c["q"][1]), ninf]])
+    d = sl.kl_rows(lp, lq)
+    assert d[0] == pytest.approx(c["kl"], rel=1e-14)
+    # current posterior puts 0 where the previous one did not: still finite
+    lq2 = np.array([[np.log(0.3), np.log(0.1), np.log(0.6), ninf]])
+    want = c["p"][0] * math.log(c["p"][0] / 0.3) + c["p"][1] * math.log(c["p"][1] / 0.6)
+    assert sl.kl_rows(lp, lq2)[0] == pytest.approx(want, rel=1e-13)
+    # current puts mass where the previous had none: infinite divergence
+    assert sl.kl_rows(lq2, lp)[0] == np.inf
+    # log_softmax of logits with -inf entries: those stay -inf, the rest normalise
+    z = np.array([[1.0, ninf, 2.0, ninf]])
+    lpz = sl.log_softmax(z)
+    assert np.isneginf(lpz[0, 1]) and np.isneginf(lpz[0, 3])
+    assert np.exp(lpz[0, [0, 2]]).sum() == pytest.approx(1.0, rel=1e-15)
+
+
 def test_kl_zero_nonneg_shift_and_brute():
     rng = np.random.default_rng(1)
     z = rng.standard_normal((6, 40)) * 2
