@@ -147,6 +147,23 @@ def step_work(shape: wl.ModelShape, m_rows: int, batch: int, n_ctx: int):
     return flops, byts
 
 
+def stored_trajectory(workload: str):
+    """The M_t trajectory a GPU run of this exact workload recorded
+    (profiles/trajectory_*.json, copied from the bench line's "trajectory"), or
+    None.  It only weights the CPU oracle's timed sample by the work of each
+    step; it is never an input or an expected value of a parity check."""
+    import glob
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "trajectory_*.json"))):
+        try:
+            with open(path) as f:
+                rec = json.load(f)
+        except Exception:
+            continue
+        if rec.get("workload") == workload and rec.get("M_t"):
+            return np.asarray(rec["M_t"], dtype=np.int64), os.path.basename(path)
+    return None
+
+
 def trajectory_from_lock_t(lock_t: np.ndarray, steps: int) -> np.ndarray:
     """Active rows at the start of every step: all rows minus those locked earlier."""
     lt = lock_t.reshape(-1)
@@ -232,26 +249,28 @@ def oracle_sample(setup: wl.SamplerSetup, traj: np.ndarray, layers: int = 2,
     d, f, V = shape.d_model, shape.d_ffn, shape.vocab
     B, N = setup.batch, setup.n_ctx
     rng = np.random.default_rng(seed)
+    f32 = np.float32
 
     def w(*s):
-        return rng.standard_normal(s) * 0.02
+        return rng.standard_normal(s, dtype=f32) * f32(0.02)
 
     Vs = V // vocab_frac
-    h = rng.standard_normal((N, d))
+    h = rng.standard_normal((N, d), dtype=f32)
     pos = np.arange(N)
+    one = np.ones(d, dtype=f32)
     lws = [{"wq": w(d, d), "wk": w(d, d), "wv": w(d, d), "wo": w(d, d), "w_gate": w(f, d),
-            "w_up": w(f, d), "w_down": w(d, f), "attn_norm": np.ones(d), "ffn_norm": np.ones(d)}
+            "w_up": w(f, d), "w_down": w(d, f), "attn_norm": one, "ffn_norm": one}
            for _ in range(layers)]
     head = w(Vs, d)
-    ck = np.zeros((N, d)); cv = np.zeros((N, d))
+    ck = np.zeros((N, d), dtype=f32); cv = np.zeros((N, d), dtype=f32)
     t0 = time.perf_counter()
     for lw in lws:
         for _ in range(B):
             h = om.layer_forward(shape, lw, h, pos, ck, cv)
     t1 = time.perf_counter()
-    z = om.rmsnorm(h, np.ones(d), shape.rms_eps) @ head.T
+    z = om.rmsnorm(h, one, shape.rms_eps) @ head.T
     lp = osl.log_softmax(z)
-    osl.kl_rows(lp, osl.log_softmax(z + 0.05))
+    osl.kl_rows(lp, osl.log_softmax(z + f32(0.05)))
     osl.uncertainty(lp)
     osl.prediction(lp, 0)
     t2 = time.perf_counter()
@@ -259,7 +278,7 @@ def oracle_sample(setup: wl.SamplerSetup, traj: np.ndarray, layers: int = 2,
     f_dense = step_work(shape, B * N, B, N)[0]
     t_traj = sum(t_dense * step_work(shape, int(m), B, N)[0] / f_dense for m in traj)
     threads = _blas_threads()
-    desc = (f"oracle (NumPy float64) on {layers} of {shape.n_layers} layers x {B} sequence(s) "
+    desc = (f"oracle (NumPy float32) on {layers} of {shape.n_layers} layers x {B} sequence(s) "
             f"at M={B * N} rows + LM head/sure test on {Vs} of {V} vocab rows, extrapolated "
             f"to the full step ({t_dense:.2f} s) and to the {len(traj)}-step trajectory in "
             f"proportion to per-step FLOPs; measured {t2 - t0:.1f} s")
@@ -497,6 +516,7 @@ def run_ours(args, rank: int, world: int):
             "algorithmic_flops_reduction": round(1.0 - flops_traj / flops_dense, 4),
             "kernel_time_ms": {k: round(tim[k]["ms"], 3) for k in ("gemm", "attn", "lock")},
             "curve": curve,
+            "trajectory": [int(m) for m in traj],
             "cpu_baseline": cpu,
             "clocks": clk,
             "gpu_launches": int(kernels_timed),
@@ -516,10 +536,16 @@ def run_reference(args, rank: int, world: int):
         return None
     setup = setup_from_args(args)
     T = setup.steps
-    # the dense trajectory shape of the scripted/KL schedule is not known on the
-    # CPU side; use the linear decay from N to the masked-only floor
-    traj = np.array([setup.n_ctx - int(round(t * (setup.n_ctx - 1) / max(1, T)))
-                     for t in range(T)])
+    cfg = workload_config(args, setup, world)
+    # the trajectory the GPU arm recorded for this workload (the same M_t the
+    # GPU arm's cpu_baseline uses), else a linear decay from N as a stand-in
+    got = stored_trajectory(cfg["workload"])
+    if got is not None and len(got[0]) == T:
+        traj, traj_note = got[0], f"M_t trajectory from {got[1]}"
+    else:
+        traj = np.array([setup.batch * (setup.n_ctx - int(round(t * (setup.n_ctx - 1) / max(1, T))))
+                         for t in range(T)])
+        traj_note = "M_t trajectory: linear stand-in (no stored GPU trajectory)"
     for _ in range(args.warmup):
         oracle_sample(setup, traj, layers=1, vocab_frac=16)
     vals = []
@@ -529,12 +555,13 @@ def run_reference(args, rank: int, world: int):
         vals.append(v)
     wall = time.perf_counter() - t0
     value = float(np.mean(vals))
+    desc = f"{desc}; {traj_note}"
     return {"impl": "reference", "metric":
             "LLaDA-8B-shape denoise steps/s & gen tok/s; % of per-step roofline vs M_t",
             "value": round(value, 6), "unit": "denoise steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(wall / args.steps * 1e3, 1),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": DATA_DESC, "config": workload_config(args, setup, world),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": DATA_DESC, "config": cfg,
             "cpu_baseline": {"value": round(value, 6), "unit": "denoise steps/s", "cores": thr,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(value, 6), "unit": "denoise steps/s",

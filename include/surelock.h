@@ -179,6 +179,36 @@ sl_status sl_kl_lock(sl_active *a, int vocab, int mask_id, int logits_dtype,
                      const sl_lock_params *p, float *d_kl, float *d_unc, float *d_conf,
                      int32_t *d_argmax, uint8_t *d_lock, void *stream);
 
+/* sl_step and the statistics half of sl_kl_lock in one pass: the LM-head GEMM
+ * rounds each logit to the model dtype, stores it at its row as sl_step does,
+ * and in the same epilogue takes, per (row, vocab tile), the running max, the
+ * sum of exp(z - max), the sum of exp(z - max) (z - z_prev) against
+ * d_logits_prev and the best value over v != mask_id; a per-row merge then
+ * writes lse_cur, D, u, conf and argmax exactly as sl_kl_lock defines them, on
+ * the stored logits, without reading them back.  This fuses the LM head with
+ * the sure test, which the pages name as future work (gist.science/nl section
+ * 5: fused kernels; gist.science/it section 4: kernel fusion to turn the FLOP
+ * savings into wall-clock).  Arguments as sl_step and sl_kl_lock: d_logits_prev
+ * and d_lse_prev [batch*n_ctx][vocab] / [batch*n_ctx] are read at the active
+ * rows when has_prev (otherwise they may be NULL and D = +inf); outputs d_kl,
+ * d_unc, d_conf, d_argmax by active-row index, d_lse_cur at the rows'
+ * positions.  fp32 models run sl_step followed by a separate statistics pass
+ * (same results).  Follow with sl_lock_decide for the lock flags. */
+sl_status sl_step_stats(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
+                        void *d_logits, const void *d_logits_prev, const float *d_lse_prev,
+                        int has_prev, float *d_lse_cur, float *d_kl, float *d_unc,
+                        float *d_conf, int32_t *d_argmax, void *stream);
+
+/* The decision half of sl_kl_lock, from statistics already computed (by
+ * sl_step_stats or sl_kl_lock): per sequence the gate threshold
+ * thr_b = sorted(u over A_t^b)[floor(gate_q (M_b - 1))], then
+ * lock_j = eps > 0 && !masked[row_j] && has_prev && D_j <= eps && (gate off ||
+ * u_j <= thr_b), or the scripted / gate-only variants of sl_lock_params
+ * (Paper-Notes, "lock criterion" and "optional confidence gate").  d_kl, d_unc
+ * and d_lock are indexed by active-row index. */
+sl_status sl_lock_decide(sl_active *a, const uint8_t *d_masked, const sl_lock_params *p,
+                         const float *d_kl, const float *d_unc, uint8_t *d_lock, void *stream);
+
 /* Sampler step: among the masked active rows with local position in
  * [block_lo, block_hi), unmask the k with the highest confidence (ties to the
  * lower position): tokens[row] = argmax, masked[row] = 0.  This is the
@@ -296,6 +326,12 @@ sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits, 
 #define SL_ABLATE_GATE_ONLY 2
 sl_status sl_model_set_ablation(sl_model *m, int flags);
 
+/* Whether this model's samplers take the sure test's statistics from the LM
+ * head's epilogue (sl_step_stats; enable = 1, the default) or from a separate
+ * pass over the stored logits (sl_step then sl_kl_lock; enable = 0).  Same
+ * results either way; a switch for comparing the two. */
+sl_status sl_model_set_head_fusion(sl_model *m, int enable);
+
 /* ---------------------------------------------------------------- sampler --- */
 
 /* Semi-autoregressive SureLock decode driven by the library: prompt_len given
@@ -337,7 +373,8 @@ typedef struct sl_sampler_state {
 sl_status sl_sampler_create(sl_model *m, int batch, const sl_sampler_params *p, sl_sampler **out);
 /* Reset state for a new decode from device prompts [batch][prompt_len]. */
 sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, void *stream);
-/* One denoising step t: sl_step, sl_kl_lock, sl_unmask_topk, sl_compact_active. */
+/* One denoising step t: sl_step_stats and sl_lock_decide (or sl_step and
+ * sl_kl_lock, see sl_model_set_head_fusion), sl_unmask_topk, sl_compact_active. */
 sl_status sl_sampler_step(sl_sampler *s, void *stream);
 /* Whole decode from host prompts [batch][prompt_len] to host tokens
  * [batch][n_ctx]; both copies are inside the call. */
@@ -366,9 +403,26 @@ sl_status sl_timing_enable(sl_model *m, int enable);
 /* Synchronises the recorded events, returns the sums since the last reset. */
 sl_status sl_timing_read(sl_model *m, sl_timing *out, int reset);
 
-/* Device error word set by kernels that gave up a bounded wait: returns
- * SL_ERR_TIMEOUT (and clears it if `clear`) or SL_OK.  Synchronises the device. */
+/* Device error word, set by a kernel that gave up a bounded wait or met a
+ * token id outside [0, vocab) (that row is embedded as zeros, never read from
+ * out of range): returns SL_ERR_TIMEOUT or SL_ERR_STATE respectively (and
+ * clears the word if `clear`), SL_OK if nothing was recorded.  Synchronises
+ * the device. */
 sl_status sl_device_check(int clear);
+
+/* Test hooks for the failure path of the bounded waits.  Neither raises a GPU
+ * fault: they only make a wait run out, after which the kernel records
+ * SL_ERR_TIMEOUT in the device error word, drains its copies, frees its TMEM
+ * and returns, and the context stays usable.
+ *   sl_debug_set_wait_limit: every later tensor-core GEMM launch (sl_step,
+ *     sl_layer_forward, sl_gemm_bf16, autotuning) gives up a barrier wait after
+ *     `ns` nanoseconds instead of the default 2 s; 0 restores the default.
+ *     SL_ERR_INVALID outside [1 ms, 2 s].  Process-wide.
+ *   sl_debug_inject_lost_load: the next tensor-core GEMM launch on the 1-SM
+ *     kernels has its first CTA leave out the operand copies of its first
+ *     pipeline stage, so the MMA warp's wait for them runs out (one-shot). */
+sl_status sl_debug_set_wait_limit(unsigned long long ns);
+sl_status sl_debug_inject_lost_load(void);
 
 #ifdef __cplusplus
 }

@@ -1,9 +1,13 @@
 """Attention of the active queries over every cached key (sl_attention, bf16
-path) against the oracle's attention in fp64: each warp layout of the kernel
-(16, 32 or 64 queries per CTA, the key tile shared by 4, 2 or 1 warps), with and
-without the key range split across CTAs, ragged query counts, empty sequences
-and key counts off the 64-key tile grid; every layout is pinned in turn
-(sl_model_set_attention) as well as left to the library's cost model."""
+path) against the oracle's attention in fp64, for both kernels: the tensor-core
+kernel (128 queries per CTA, tcgen05 + TMEM, TMA-fed K/V; the library's
+default) with its key range whole or split across CTAs (merged by per-row
+tickets), and the mma.sync kernel in each warp layout (16, 32 or 64 queries per
+CTA, the key tile shared by 4, 2 or 1 warps); ragged query counts (several
+128-query tiles, partial last tiles), empty sequences and key counts off the
+tile grids.  Every layout is pinned in turn (sl_model_set_attention) as well as
+left to the library's cost model, and every call runs twice on the same
+workspace so that a ticket left non-zero would show."""
 import numpy as np
 import pytest
 import torch
@@ -27,11 +31,16 @@ CASES = [
     ([7], 4000),            # long key range (splits of many tiles)
     ([200], 2500),
     ([0, 40, 0], 260),      # empty sequences
+    ([300], 700),           # three 128-query tiles, the last one partial
+    ([129, 128, 1], 384),   # tile boundaries one row either side
 ]
 
 
-# (queries per CTA, cross-CTA key split); 0 = the library's cost model
-LAYOUTS = [(0, 0), (16, 1), (32, 1), (64, 1), (16, 4), (32, 2), (64, 3)]
+# (queries per CTA, cross-CTA key split); 0 = the library's cost model.
+# 128 queries per CTA = the tensor-core kernel (the default), 16/32/64 the
+# mma.sync kernel.
+LAYOUTS = [(0, 0), (128, 1), (128, 2), (128, 3), (128, 16), (16, 1), (32, 1), (64, 1), (16, 4),
+           (32, 2), (64, 3)]
 
 
 @pytest.mark.parametrize("layout", LAYOUTS)
@@ -60,6 +69,11 @@ def test_attention_matches_oracle(cuda_dev, counts, n_ctx, layout):
     torch.cuda.synchronize()
     rt.device_check()
     got = to64(o)
+    o2 = torch.full_like(o, -5.0)
+    rt.attention(model, cache, act, 0, q, o2)
+    torch.cuda.synchronize()
+    rt.device_check()
+    assert torch.equal(o[:M], o2[:M]), "a second call on the same workspace differs"
     off = 0
     for b, c in enumerate(counts):
         if c == 0:
@@ -90,7 +104,7 @@ NOKV_CASES = [
     # active rows only at the end of the range
     ([9, 20], 3000, "tail"),
 ]
-NOKV_LAYOUTS = [(0, 0), (16, 1), (32, 2), (64, 3), (16, 4)]
+NOKV_LAYOUTS = [(0, 0), (128, 1), (128, 4), (16, 1), (32, 2), (64, 3), (16, 4)]
 
 
 def _positions(rng, counts, n_ctx, where):

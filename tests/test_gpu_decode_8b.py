@@ -1,0 +1,154 @@
+"""Whole LLaDA-8B-shape decodes (32 layers, d_model 4096, 32 heads of 128,
+d_ffn 12288, vocabulary 126464; random-init bf16 weights, seed 0, the bench's
+prompts), teacher-forced against the oracle at the listed steps, in the launch
+configuration the bench times (autotuned GEMM tilings, the default attention):
+
+* batch 1, 128 prompt + 256 masked positions, 256 steps in blocks of 32, one
+  token per step, for eps in {0, 0.01, 0.05} and the scripted schedule that
+  takes M_t linearly down to 10% of N; checked at steps 0, 1, 2, 31, 32, 128,
+  254 and 255 on every active row;
+* batch 4, 1024 prompt + 1024 masked positions (N = 2048), 512 steps in blocks
+  of 64, two tokens per step, eps 0.05 with the confidence gate at q = 0.5;
+  checked on every active row at steps 255, 510 and 511, and at step 1 (every
+  row active) on 32 sampled rows per sequence with per-block teacher forcing
+  (each block attends over the GPU's cache after the step, which holds every
+  active row's fresh K/V, so the oracle's work scales with the sample).
+
+At each checked step: logits within the bf16 tolerance (max abs 5e-2), the
+fresh K/V the step wrote within 3e-2 relative, the log-probs of the step within
+2e-2, and the sure test, gate, unmasking and compaction decided by the oracle on
+the GPU's own logits equal to the GPU's outside the rounding bands.  The
+observed errors are appended to the JSON-lines file named by SL_PARITY_LOG
+when that variable is set.
+"""
+import json
+import os
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import parity_8b as p8
+import workloads as wl
+from parity_util import FINAL_LP_TOL, LOGIT_TOL
+from token_locking_b200 import runtime as rt
+
+pytestmark = pytest.mark.gpu
+
+CHECK4 = (0, 1, 2, 31, 32, 128, 254, 255)
+CHECK5_FULL = (255, 510, 511)
+CHECK5_SAMPLED = (1,)
+SAMPLE5 = 32
+KV_TOL = 3e-2
+
+
+@pytest.fixture(scope="module")
+def llada8b(cuda_dev):
+    w = wl.torch_weights(wl.LLADA8B, cuda_dev)
+    model = rt.Model(wl.LLADA8B, w, "bf16")
+    w_or = p8.oracle_weights(w)
+    yield model, w, w_or
+    model.close()
+
+
+def _log(rec):
+    path = os.environ.get("SL_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+
+
+def _rel(a, b):
+    return float(np.abs(a - b).max() / max(1.0, float(np.abs(b).max())))
+
+
+def _lp_err(z_gpu, z_or):
+    """max |log p_gpu - log p_oracle| over the row's vocabulary (float64)."""
+    def lsm(z):
+        z = z.astype(np.float64)
+        m = z.max(axis=-1, keepdims=True)
+        return z - (m + np.log(np.exp(z - m).sum(axis=-1, keepdims=True)))
+    return float(np.abs(lsm(z_gpu) - lsm(z_or)).max())
+
+
+def _decode(llada8b, dev, setup, full_steps, sampled_steps, name):
+    model, _, w_or = llada8b
+    shape = setup.shape
+    B = setup.batch
+    s = rt.Sampler(model, B, setup.prompt_len, setup.gen_len, setup.steps, setup.block_len,
+                   setup.tokens_per_step, setup.eps, setup.gate_q, setup.scripted)
+    s.autotune()
+    prompts = wl.np_prompts(B, setup.prompt_len, shape.vocab, shape.mask_id,
+                            seed=wl.SEED_PROMPTS)
+    s.start(torch.from_numpy(prompts).to(dev))
+    stats = {"mismatch": 0, "ambiguous": 0, "locks": 0, "unmask_amb": 0}
+    worst = {"logits": 0.0, "kv": 0.0, "lp": 0.0}
+    for t in range(setup.steps):
+        if t not in full_steps and t not in sampled_steps:
+            s.step()
+            continue
+        full = t in full_steps
+        snap = p8.snapshot(s, setup, want_cache=full)
+        s.step()
+        torch.cuda.synchronize()
+        rt.device_check()
+        g = p8.gpu_after(s, setup, t)
+        t0 = time.time()
+        j0 = 0
+        for b in range(B):
+            A = snap["act"][b]
+            m = len(A)
+            if m == 0:
+                continue
+            if full:
+                z, ck, cv = p8.oracle_logits_full(shape, w_or, snap, b, A)
+                zg = g["z"][b, A]
+                kg, vg = p8.cache_rows(s, setup, b, A)
+                kv = max(_rel(kg, ck[:, A]), _rel(vg, cv[:, A]))
+                n_rows = m
+            else:
+                rng = np.random.default_rng(100 * t + b)
+                idx = np.sort(rng.choice(m, min(SAMPLE5, m), replace=False))
+                k_all, v_all = p8.cache_rows(s, setup, b, np.arange(setup.n_ctx))
+                z, ks, vs = p8.oracle_logits_sampled(shape, w_or, snap["tokens"][b], A, idx,
+                                                     k_all, v_all)
+                zg = g["z"][b, A[idx]]
+                kv = max(_rel(k_all[:, A[idx]], ks), _rel(v_all[:, A[idx]], vs))
+                n_rows = len(idx)
+            zerr = float(np.abs(zg - z).max())
+            lperr = _lp_err(zg, z)
+            worst["logits"] = max(worst["logits"], zerr)
+            worst["kv"] = max(worst["kv"], kv)
+            worst["lp"] = max(worst["lp"], lperr)
+            _log({"test": name, "t": t, "b": b, "M": m, "rows_checked": n_rows,
+                  "logits_max_abs_err": zerr, "logp_max_abs_err": lperr, "kv_max_rel_err": kv,
+                  "z_max_abs": float(np.abs(z).max()), "oracle_s": round(time.time() - t0, 1)})
+            assert zerr <= LOGIT_TOL["bf16"], f"{name} t={t} b={b}: logits err {zerr}"
+            assert kv <= KV_TOL, f"{name} t={t} b={b}: fresh K/V rel err {kv}"
+            assert lperr <= FINAL_LP_TOL, f"{name} t={t} b={b}: log-prob err {lperr}"
+            p8.check_decisions(setup, t, b, A, snap, g, j0, stats)
+            j0 += m            # per-row outputs run over all sequences in order
+    final = s.state()
+    assert int(final["masked"].sum().item()) == 0, "positions left masked at the end"
+    _log({"test": name, "summary": stats, "worst": worst})
+    s.close()
+    assert stats["mismatch"] == 0, stats
+    return stats, worst
+
+
+@pytest.mark.parametrize("arm", ["eps0", "eps0.01", "eps0.05", "scripted"])
+def test_llada8b_b1_n384_teacher_forced(llada8b, cuda_dev, arm):
+    setup = (wl.cfg_full8b(eps=0.05, scripted=True) if arm == "scripted"
+             else wl.cfg_full8b(eps=float(arm[3:])))
+    stats, _ = _decode(llada8b, cuda_dev, setup, CHECK4, (), f"cfg4-{arm}")
+    if arm == "eps0":
+        assert stats["locks"] == 0
+    else:
+        assert stats["locks"] > 0
+
+
+def test_llada8b_b4_n2048_teacher_forced(llada8b, cuda_dev):
+    setup = wl.cfg_long8b()
+    stats, _ = _decode(llada8b, cuda_dev, setup, CHECK5_FULL, CHECK5_SAMPLED, "cfg5")
+    assert stats["locks"] > 0

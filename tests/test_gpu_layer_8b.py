@@ -84,7 +84,7 @@ def _run(block8, cuda_dev, M):
         assert e <= 3e-2 * max(1.0, np.abs(ref_c[R]).max()), f"M={M}: fresh K/V max err {e}"
 
 
-@pytest.mark.parametrize("M", [64, 512, 2048])
+@pytest.mark.parametrize("M", [8, 64, 256, 512, 1024, 2048])
 def test_block_8b_analytic_tilings(block8, cuda_dev, M):
     _run(block8, cuda_dev, M)
 
@@ -100,7 +100,7 @@ def test_qkv_tile_must_divide_segments(block8):
 _TUNED = {}
 
 
-@pytest.mark.parametrize("M", [200, 2048])
+@pytest.mark.parametrize("M", [8, 200, 1024, 2048])
 def test_block_8b_autotuned_tilings(block8, cuda_dev, M):
     model, cache = block8[0], block8[1]
     if not _TUNED:

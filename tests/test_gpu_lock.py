@@ -20,18 +20,48 @@ def _setup_logits(rows_total, V, dtype, seed, sigma_prev=0.05, spike=True):
     return z.astype(np.float32), zp.astype(np.float32)
 
 
+def _lse_of(z, lp):
+    """logsumexp per row as z - log p at the row's largest (finite) logit."""
+    i = np.argmax(z, axis=1)[:, None]
+    return (np.take_along_axis(z, i, 1) - np.take_along_axis(lp, i, 1))[:, 0]
+
+
+def _neg_inf_vocab_mask(z, zp, seed):
+    """Logits with runs of -inf, as a vocabulary mask applied before the sure
+    test leaves them: every row loses a contiguous range of ids plus scattered
+    ids (same in both steps); the first rows lose the start of the vocabulary,
+    so whole 8-wide groups at the front of a chunk are -inf; two rows gain a
+    -inf in the previous step only (D must come out infinite there)."""
+    rng = np.random.default_rng(seed)
+    R, V = z.shape
+    for r in range(R):
+        a = 0 if r < 4 else int(rng.integers(0, V - 64))
+        n = int(rng.integers(8, max(9, V // 4)))
+        z[r, a:a + n] = -np.inf
+        zp[r, a:a + n] = -np.inf
+        cols = rng.choice(V, size=max(1, V // 50), replace=False)
+        z[r, cols] = -np.inf
+        zp[r, cols] = -np.inf
+    for r in (R // 2, R - 1):
+        col = int(np.argmax(np.where(np.isfinite(z[r]), z[r], -np.inf)))
+        zp[r, col] = -np.inf
+    return z, zp
+
+
 def _run(dev, B, n_ctx, positions, V, dtype, eps, gate_q, has_prev, scripted_target, seed,
-         masked_frac=0.3, sigma_prev=0.05, gate_only=False):
+         masked_frac=0.3, sigma_prev=0.05, gate_only=False, neg_inf=False):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     R = B * n_ctx
     z, zp = _setup_logits(R, V, dtype, seed, sigma_prev)
+    if neg_inf:
+        z, zp = _neg_inf_vocab_mask(z, zp, seed + 7)
     rng = np.random.default_rng(seed + 100)
     masked = (rng.random(R) < masked_frac).astype(np.uint8)
     mask_id = V - 3
     # oracle inputs: log-probs of the exact stored values, lse_prev in fp64 -> fp32
     lp_cur_all = osl.log_softmax(z.astype(np.float64))
     lp_prev_all = osl.log_softmax(zp.astype(np.float64))
-    lse_prev = (zp.astype(np.float64) - lp_prev_all)[:, 0].astype(np.float32)
+    lse_prev = _lse_of(zp.astype(np.float64), lp_prev_all).astype(np.float32)
 
     act = rt.Active(B, n_ctx)
     act.load(positions)
@@ -68,7 +98,7 @@ def _oracle_seq(pos_flat, ref, eps, gate_q, has_prev, scripted_target, gate_only
         lock = osl.scripted_locks(D, masked, hp, pos_flat, len(pos_flat) - scripted_target)
     else:
         lock = osl.lock_decision(D, u, masked, hp, eps, gate_q, thr, gate_only)
-    lse = (ref["z"][pos_flat].astype(np.float64) - lp)[:, 0]
+    lse = _lse_of(ref["z"][pos_flat].astype(np.float64), lp)
     return dict(D=D, u=u, conf=conf, pred=pred, thr=thr, lock=lock, lse=lse)
 
 
@@ -83,16 +113,44 @@ CASES = [
     (2, 80, [77, 41], 2048, "bf16", 0.0, -1.0, True, 30, 0.2),
     (1, 64, [64], 126464, "bf16", 0.01, 0.5, True, -1, 0.05),
     (1, 64, [64], 126464, "bf16", 0.05, 0.5, True, -1, 0.2),
+    # the lock-test microbenchmark's larger row counts at the full vocabulary
+    (1, 512, [512], 126464, "bf16", 0.01, 0.5, True, -1, 0.05),
+    (1, 512, [512], 126464, "bf16", 0.05, 0.5, True, -1, 0.2),
+    (1, 2048, [2048], 126464, "bf16", 0.01, 0.5, True, -1, 0.05),
+    (1, 2048, [2048], 126464, "bf16", 0.05, 0.5, True, -1, 0.2),
+]
+
+
+NEG_INF_CASES = [
+    (1, 64, [64], 1024, "f32", 0.05, 0.5, True, -1, 0.2),
+    (2, 100, [100, 37], 4096, "bf16", 0.05, 0.5, True, -1, 0.2),
+    (1, 64, [64], 126464, "bf16", 0.05, -1.0, True, -1, 0.2),
+    (1, 64, [60], 2048, "bf16", 0.05, -1.0, False, -1, 0.2),
 ]
 
 
 @pytest.mark.parametrize("case", CASES)
 def test_kl_lock_matches_oracle(cuda_dev, case):
+    _check_case(cuda_dev, case, neg_inf=False)
+
+
+@pytest.mark.parametrize("case", NEG_INF_CASES)
+def test_kl_lock_with_neg_inf_logits(cuda_dev, case):
+    """Rows holding runs of -inf logits: no NaN anywhere, and the same D, u,
+    conf, argmax, lse and lock flags as the oracle (0 log 0 = 0)."""
+    _check_case(cuda_dev, case, neg_inf=True)
+
+
+def _check_case(cuda_dev, case, neg_inf):
     B, n_ctx, counts, V, dtype, eps, gate_q, has_prev, scripted, sig = case
     rng = np.random.default_rng(sum(counts) + V)
     positions = [np.sort(rng.choice(n_ctx, c, replace=False)).astype(np.int32) for c in counts]
     act, out, ref, _ = _run(cuda_dev, B, n_ctx, positions, V, dtype, eps, gate_q, has_prev,
-                            scripted, seed=V + B, sigma_prev=sig)
+                            scripted, seed=V + B, sigma_prev=sig, neg_inf=neg_inf)
+    M = sum(counts)
+    for k in ("kl", "unc", "conf", "lse"):
+        vals = out[k][:M] if k != "lse" else out[k]
+        assert not np.any(np.isnan(vals)), f"NaN in {k}"
     j0 = 0
     n_mis = n_amb = 0
     for b in range(B):

@@ -22,12 +22,13 @@ MINI_BF16 = wl.ModelShape(n_layers=2, d_model=256, n_heads=2, head_dim=128, d_ff
                           vocab=1024, mask_id=1023, rope_theta=10000.0)
 
 
-def _sampler(setup, dev, std=0.02, seed_w=0):
+def _sampler(setup, dev, std=0.02, seed_w=0, head_fusion=True):
     shape = setup.shape
     w_np = wl.np_weights(shape, seed=seed_w, std=std)
     w_dev = weights_to_device(w_np, setup.dtype, dev)
     model = rt.Model(shape, w_dev, setup.dtype)
     model.set_ablation(no_kv_cache=setup.no_kv_cache, gate_only=setup.gate_only)
+    model.set_head_fusion(head_fusion)
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, setup.steps,
                    setup.block_len, setup.tokens_per_step, setup.eps, setup.gate_q,
                    setup.scripted)
@@ -57,8 +58,8 @@ def _snapshot(s, setup):
     }
 
 
-def _teacher_forced(setup, dev, steps, std=0.02):
-    model, s, w64, prompts = _sampler(setup, dev, std)
+def _teacher_forced(setup, dev, steps, std=0.02, head_fusion=True):
+    model, s, w64, prompts = _sampler(setup, dev, std, head_fusion=head_fusion)
     shape = setup.shape
     B, N = setup.batch, setup.n_ctx
     s.start(torch.from_numpy(prompts).to(dev))
@@ -149,11 +150,14 @@ def test_tiny_decode_gate_and_scripted(cuda_dev):
     _teacher_forced(dataclasses.replace(wl.CFG_TINY, scripted=True, eps=0.0), cuda_dev, 8)
 
 
-def test_bf16_mini_decode_teacher_forced(cuda_dev):
+@pytest.mark.parametrize("head_fusion", [True, False])
+def test_bf16_mini_decode_teacher_forced(cuda_dev, head_fusion):
+    """The sure test's statistics from the LM head's epilogue (the default) or
+    from a separate pass over the stored logits."""
     setup = wl.SamplerSetup(MINI_BF16, "bf16", batch=2, prompt_len=40, gen_len=160, steps=40,
                             block_len=32, tokens_per_step=4, eps=0.01, gate_q=0.5)
     setup.validate()
-    stats, _ = _teacher_forced(setup, cuda_dev, 12, std=0.05)
+    stats, _ = _teacher_forced(setup, cuda_dev, 12, std=0.05, head_fusion=head_fusion)
 
 
 def test_tiny_free_running_matches_oracle(cuda_dev):

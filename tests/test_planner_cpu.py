@@ -14,7 +14,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def test_gemm_planner_choices(tmp_path):
     from token_locking_b200 import build as b
     b.build()
-    objs = [os.path.join(b.BUILD, f) for f in ("layers.o", "lock.o", "attn.o", "gemm_tc.o")]
+    objs = [os.path.join(b.BUILD, f) for f in ("layers.o", "lock.o", "attn.o", "attn_tc.o", "gemm_tc.o")]
     exe = str(tmp_path / "planner_check")
     cmd = ["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O1", "-std=c++17",
            "-I" + os.path.join(ROOT, "include"), "-I" + b.CSRC,

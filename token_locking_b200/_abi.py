@@ -84,6 +84,9 @@ SIGNATURES = {
     "sl_step": (_I, [_P, _P, _P, _P, _P, _P]),
     "sl_kl_lock": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, C.POINTER(LockParams),
                         _P, _P, _P, _P, _P, _P]),
+    "sl_step_stats": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P]),
+    "sl_lock_decide": (_I, [_P, _P, C.POINTER(LockParams), _P, _P, _P, _P]),
+    "sl_model_set_head_fusion": (_I, [_P, _I]),
     "sl_kl_stats_noalloc": (_I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]),
     "sl_unmask_topk": (_I, [_P, _P, _P, _I, _I, _I, _P, _P, _P]),
     "sl_compact_active": (_I, [_P, _P, _P, _P, _I, _P]),
@@ -104,6 +107,8 @@ SIGNATURES = {
     "sl_timing_enable": (_I, [_P, _I]),
     "sl_timing_read": (_I, [_P, C.POINTER(Timing), _I]),
     "sl_device_check": (_I, [_I]),
+    "sl_debug_set_wait_limit": (_I, [C.c_ulonglong]),
+    "sl_debug_inject_lost_load": (_I, []),
 }
 
 _lib = None

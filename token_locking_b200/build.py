@@ -19,8 +19,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsurelock.so")
-SOURCES = ["api.cu", "layers.cu", "lock.cu", "attn.cu", "gemm_tc.cu"]
+SOURCES = ["api.cu", "layers.cu", "lock.cu", "attn.cu", "attn_tc.cu", "gemm_tc.cu"]
 HEADERS = [os.path.join(CSRC, "common.cuh"), os.path.join(CSRC, "internal.h"),
+           os.path.join(CSRC, "tc_ptx.cuh"),
            os.path.join(INCLUDE, "surelock.h")]
 NVCC = os.environ.get("NVCC", "nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -99,6 +99,8 @@ struct sl_model {
   std::vector<sl_layer_weights> layers;
   std::vector<std::array<WMaps, W_COUNT>> maps;
   int attn_q = 0, attn_splits = 0;   // pinned attention layout (0 = cost model)
+  bool head_fusion = true;           // samplers take the sure-test statistics from the
+                                     // LM head's epilogue (bf16 models)
   int ablation = 0;                  // SL_ABLATE_* bits (0: the method itself)
   WMaps head_map;
   int num_sms;
@@ -126,6 +128,12 @@ struct sl_kv_cache {
   float *ws = nullptr;     // [max_rows][max(3d, 2f)] fp32 split-K workspace, kept zero
   float *attn_ws = nullptr;
   int attn_max_splits = 16;
+  unsigned int *attn_tickets = nullptr;   // [max_rows][H] per-row split tickets, kept zero
+  std::vector<TmaMat> k_maps, v_maps;     // per layer, 128-row boxes (tensor-core attention)
+  TmaMat map_q;                           // q workspace [M][d], 128-row boxes
+  TmaMat map_qx{};                        // a caller's q (sl_attention), by pointer and M
+  float4 *head_stat = nullptr;            // [max_rows][V / 64] LM-head tile records (bf16)
+  int *head_stat_idx = nullptr;
   int32_t *key_stamp = nullptr;   // [max_rows] visible-key stamps (no-KV-cache ablation)
   int key_gen = 0;                // the current stamp generation
   TmaMat map_a, map_o, map_act;
@@ -343,7 +351,9 @@ extern "C" sl_status sl_device_check(int clear) {
   if (v != 0) {
     if (clear) SL_CUDA(cudaMemset(w, 0, sizeof(int)));
     if (v >= 1 && v <= 3) return fail(SL_ERR_TIMEOUT, "a kernel gave up a bounded wait (code %d)", v);
-    return fail(SL_ERR_CUDA, "a kernel reported device error %d (4: index out of range)", v);
+    if (v == DEV_BAD_INDEX)
+      return fail(SL_ERR_STATE, "a kernel met a token id outside [0, vocab) and skipped it");
+    return fail(SL_ERR_CUDA, "a kernel reported device error %d", v);
   }
   return SL_OK;
 }
@@ -353,7 +363,10 @@ extern "C" void sl_kv_cache_destroy(sl_kv_cache *c) {
   if (!c) return;
   for (void *p : c->k) cudaFree(p);
   for (void *p : c->v) cudaFree(p);
-  void *ps[] = {c->rope, c->h, c->a, c->qkv, c->q, c->o, c->act, c->ws, c->attn_ws, c->key_stamp};
+  void *ps[] = {c->rope,         c->h,         c->a,          c->qkv,
+                c->q,            c->o,         c->act,        c->ws,
+                c->attn_ws,      c->key_stamp, c->attn_tickets, c->head_stat,
+                c->head_stat_idx};
   for (void *p : ps)
     if (p) cudaFree(p);
   delete c;
@@ -392,7 +405,15 @@ extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
        alloc((void **)&c->ws, rows * wsc * 4) && alloc((void **)&c->key_stamp, rows * 4);
   if (ok && cfg.dtype == SL_BF16) {
     ok = alloc((void **)&c->attn_ws, attn_bf16_workspace_bytes(c->max_rows, cfg.n_heads,
-                                                               c->attn_max_splits));
+                                                               c->attn_max_splits)) &&
+         alloc((void **)&c->attn_tickets, attn_tc_tickets_bytes(c->max_rows, cfg.n_heads)) &&
+         alloc((void **)&c->head_stat, rows * (cfg.vocab / 64) * sizeof(float4)) &&
+         alloc((void **)&c->head_stat_idx, rows * (cfg.vocab / 64) * sizeof(int));
+    c->k_maps.resize(cfg.n_layers);
+    c->v_maps.resize(cfg.n_layers);
+    for (int l = 0; l < cfg.n_layers && ok; ++l)
+      ok = tma_encode(&c->k_maps[l], c->k[l], c->max_rows, d, 128) &&
+           tma_encode(&c->v_maps[l], c->v[l], c->max_rows, d, 128);
   }
   if (ok) {
     // rotary table in double precision: angle = pos * theta^(-2i/dh)
@@ -740,9 +761,33 @@ static sl_status layer_f32(sl_model *m, sl_kv_cache *c, sl_active *a, int l, flo
   return SL_OK;
 }
 
+// Failure-detection test hooks (sl_debug_*): the wait limit of later GEMM
+// launches, and a one-shot lost operand copy in the next one.
+static std::atomic<unsigned long long> g_wait_limit_ns{0};
+static std::atomic<int> g_lost_load{0};
+
+static cudaError_t launch_gemm_hooked(TcGemmArgs g, int num_sms, int *err, cudaStream_t s) {
+  g.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+  g.lost_load = g_lost_load.exchange(0, std::memory_order_relaxed);
+  return launch_gemm_tc(g, num_sms, err, s);
+}
+
 static sl_status tc_gemm(sl_model *m, const TcGemmArgs &g, cudaStream_t s) {
-  cudaError_t e = launch_gemm_tc(g, m->num_sms, m->err, s);
+  cudaError_t e = launch_gemm_hooked(g, m->num_sms, m->err, s);
   if (e != cudaSuccess) return cuda_fail(e, "tcgen05 GEMM launch");
+  return SL_OK;
+}
+
+extern "C" sl_status sl_debug_set_wait_limit(unsigned long long ns) {
+  if (ns != 0 && (ns < 1000000ull || ns > WAIT_LIMIT_NS))
+    return fail(SL_ERR_INVALID, "sl_debug_set_wait_limit: %llu ns outside [1 ms, %llu ns]", ns,
+                WAIT_LIMIT_NS);
+  g_wait_limit_ns.store(ns, std::memory_order_relaxed);
+  return SL_OK;
+}
+
+extern "C" sl_status sl_debug_inject_lost_load(void) {
+  g_lost_load.store(1, std::memory_order_relaxed);
   return SL_OK;
 }
 
@@ -798,6 +843,7 @@ static sl_status ensure_maps(sl_kv_cache *c, int M) {
   const sl_config &cfg = c->m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn;
   if (!tma_encode(&c->map_a, c->a, M, d, 128) || !tma_encode(&c->map_o, c->o, M, d, 128) ||
+      !tma_encode(&c->map_q, c->q, M, d, 128) ||
       !tma_encode(&c->map_act, c->act, M, f, 128) ||
       !tma_encode_out(&c->out_h, c->h, M, d, d, true) ||
       !tma_encode_out(&c->out_ws3, c->ws, M, 3 * d, 3 * d, true) ||
@@ -818,18 +864,39 @@ static void fill_seqs(AttnSeqs &seqs, const sl_active *a, const int32_t *counts)
   }
 }
 
+// q_map: a TMA map over q with 128-row boxes (the tensor-core kernel reads q by
+// TMA).  queries_per_cta 128 (or 0, the default) selects the tensor-core
+// kernel; 16, 32 or 64 the mma.sync kernel with that layout.
 static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, int l, int M,
-                           const void *q, void *o, const KeySet &ks, cudaStream_t s) {
+                           const void *q, const TmaMat &q_map, void *o, const KeySet &ks,
+                           cudaStream_t s) {
   const int d = m->cfg.d_model;
   Timed t(m, SL_K_ATTN, 2.0 * (2.0 * M * d + 2.0 * seqs.batch * c->n_ctx * d),
           4.0 * (double)M * c->n_ctx * d, s);
   // the output projection's weights follow; the attention leaves HBM idle
+  if (m->attn_q == 0 || m->attn_q == 128) {
+    SL_CUDA(launch_attn_tc(q_map, c->k_maps[l], c->v_maps[l], seqs, M, c->n_ctx, m->cfg.n_heads,
+                           o, c->attn_ws, c->attn_tickets, c->attn_max_splits, m->num_sms, m->err,
+                           g_wait_limit_ns.load(std::memory_order_relaxed), s, m->attn_splits,
+                           m->layers[l].wo, (size_t)d * d * 2, ks.stamp, ks.gen));
+    return SL_OK;
+  }
   SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
                            c->attn_ws, c->attn_max_splits, m->num_sms, s, m->attn_q,
                            m->attn_splits, m->layers[l].wo, (size_t)d * d * 2, ks.stamp,
                            ks.gen));
   return SL_OK;
 }
+
+// The sure test's statistics requested from the LM head's epilogue
+// (sl_step_stats): previous logits and lse (null when there is no previous
+// posterior) and the per-row outputs.
+struct HeadStats {
+  const void *prev = nullptr;
+  const float *lse_prev = nullptr;
+  float *lse_cur = nullptr, *kl = nullptr, *unc = nullptr, *conf = nullptr;
+  int32_t *argmax = nullptr;
+};
 
 // One of the step's projection GEMMs on the current activation descriptors,
 // with the split-K finalize pass when the plan splits K:
@@ -839,7 +906,8 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
 //   G_DN   act x Wd^T, added to the residual h
 //   G_HD   RMSNorm(h) x W_out^T -> logits[rows]
 static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int l, int kind,
-                          const Plan &pl, int M, float *h, void *logits, cudaStream_t s) {
+                          const Plan &pl, int M, float *h, void *logits, cudaStream_t s,
+                          const HeadStats *hs = nullptr) {
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn, V = cfg.vocab, H = cfg.n_heads;
   const double Md = (double)M;
@@ -937,6 +1005,14 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       g.row_map = rows;
       bytes = gemm_bytes(Md, V, d, 2);
       flops = 2.0 * Md * d * V;
+      if (hs) {
+        g.epi = EPI_HEAD;
+        g.prev = hs->prev;
+        g.stat = c->head_stat;
+        g.stat_idx = c->head_stat_idx;
+        g.mask_id = cfg.mask_id;
+        if (hs->prev) bytes += 2.0 * Md * V;       // the previous logits, read once
+      }
       break;
     }
   }
@@ -961,7 +1037,7 @@ static sl_status layer_bf16(sl_model *m, sl_kv_cache *c, sl_active *a, int l, fl
   sl_status st;
   SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.attn_norm, d, cfg.rms_eps, M, c->a, s));
   if ((st = run_gemm(m, c, a->rows, l, G_QKV, pl.qkv, M, h, nullptr, s)) != SL_OK) return st;
-  if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->o, ks, s)) != SL_OK) return st;
+  if ((st = attn_bf16(m, c, seqs, l, M, c->q, c->map_q, c->o, ks, s)) != SL_OK) return st;
   if ((st = run_gemm(m, c, a->rows, l, G_O, pl.o, M, h, nullptr, s)) != SL_OK) return st;
   SL_CUDA(launch_rmsnorm(SL_BF16, h, lw.ffn_norm, d, cfg.rms_eps, M, c->a, s));
   if ((st = run_gemm(m, c, a->rows, l, G_GU, pl.gu, M, h, nullptr, s)) != SL_OK) return st;
@@ -977,13 +1053,22 @@ static sl_status check_pair(sl_model *m, sl_kv_cache *c, sl_active *a, const cha
   return SL_OK;
 }
 
-extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
-                             void *d_logits, void *stream) {
+static sl_status kl_stats_unfused(sl_model *timing_model, sl_active *a, int M, int vocab,
+                                  int mask_id, int dtype, const void *cur, const HeadStats &hs,
+                                  cudaStream_t s);
+
+static sl_status step_impl(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
+                           void *d_logits, const HeadStats *hs, void *stream) {
   sl_status st = check_pair(m, c, a, "sl_step");
   if (st != SL_OK) return st;
   if (!d_tokens || !d_logits) return fail(SL_ERR_INVALID, "sl_step: null argument");
   if (m->cfg.dtype == SL_BF16 && ((uintptr_t)d_logits & 15))
     return fail(SL_ERR_INVALID, "sl_step: logits must be 16-byte aligned");
+  if (hs && (!hs->lse_cur || !hs->kl || !hs->unc || !hs->conf || !hs->argmax ||
+             (hs->prev && !hs->lse_prev)))
+    return fail(SL_ERR_INVALID, "sl_step_stats: null statistics argument");
+  if (hs && m->cfg.dtype == SL_BF16 && hs->prev && ((uintptr_t)hs->prev & 15))
+    return fail(SL_ERR_INVALID, "sl_step_stats: previous logits must be 16-byte aligned");
   int32_t counts[SL_MAX_BATCH];
   if ((st = sl_active_counts(a, counts)) != SL_OK) return st;
   int M = 0;
@@ -994,14 +1079,19 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   const int d = cfg.d_model, V = cfg.vocab;
   KeySet ks;
   if ((st = visible_keys(m, c, a, M, s, &ks)) != SL_OK) return st;
-  SL_CUDA(launch_gather_embed(cfg.dtype, d_tokens, a->rows, M, m->tok_emb, d, c->h, s));
+  SL_CUDA(launch_gather_embed(cfg.dtype, d_tokens, a->rows, M, m->tok_emb, d, V, c->h, m->err,
+                              s));
   if (cfg.dtype == SL_F32) {
     for (int l = 0; l < cfg.n_layers; ++l)
       if ((st = layer_f32(m, c, a, l, c->h, M, ks, s)) != SL_OK) return st;
     SL_CUDA(launch_rmsnorm(SL_F32, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
-    Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 4), 2.0 * M * d * V, s);
-    SL_CUDA(launch_gemm_f32(EPI_STORE, (const float *)c->a, M, d, (const float *)m->lm_head, V,
-                            (float *)d_logits, V, 0, a->rows, s));
+    {
+      Timed t(m, SL_K_GEMM, gemm_bytes(M, V, d, 4), 2.0 * M * d * V, s);
+      SL_CUDA(launch_gemm_f32(EPI_STORE, (const float *)c->a, M, d, (const float *)m->lm_head,
+                              V, (float *)d_logits, V, 0, a->rows, s));
+    }
+    // the fp32 path has no tensor-core epilogue: a separate pass over the logits
+    if (hs) return kl_stats_unfused(m, a, M, V, cfg.mask_id, SL_F32, d_logits, *hs, s);
     return SL_OK;
   }
   if ((st = ensure_maps(c, M)) != SL_OK) return st;
@@ -1011,10 +1101,40 @@ extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const in
   for (int l = 0; l < cfg.n_layers; ++l)
     if ((st = layer_bf16(m, c, a, l, c->h, M, seqs, pl, ks, s)) != SL_OK) return st;
   SL_CUDA(launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s));
-  if ((st = run_gemm(m, c, a->rows, 0, G_HD, pl.hd, M, c->h, d_logits, s)) != SL_OK) return st;
+  if ((st = run_gemm(m, c, a->rows, 0, G_HD, pl.hd, M, c->h, d_logits, s, hs)) != SL_OK)
+    return st;
+  if (hs) {
+    Timed t(m, SL_K_LOCK, (double)M * (V / pl.hd.bn) * 20.0 + 24.0 * M, 0.0, s);
+    SL_CUDA(launch_head_stats_merge(c->head_stat, c->head_stat_idx, V / pl.hd.bn, a->rows, M,
+                                    hs->prev ? 1 : 0, hs->lse_prev, hs->lse_cur, hs->kl, hs->unc,
+                                    hs->conf, hs->argmax, s));
+  }
   // the previous step's timing events completed before this step was planned
   if (m->timing) timing_harvest(m, false);
   return SL_OK;
+}
+
+extern "C" sl_status sl_step(sl_model *m, sl_kv_cache *c, sl_active *a, const int32_t *d_tokens,
+                             void *d_logits, void *stream) {
+  return step_impl(m, c, a, d_tokens, d_logits, nullptr, stream);
+}
+
+extern "C" sl_status sl_step_stats(sl_model *m, sl_kv_cache *c, sl_active *a,
+                                   const int32_t *d_tokens, void *d_logits,
+                                   const void *d_logits_prev, const float *d_lse_prev,
+                                   int has_prev, float *d_lse_cur, float *d_kl, float *d_unc,
+                                   float *d_conf, int32_t *d_argmax, void *stream) {
+  HeadStats hs;
+  hs.prev = has_prev ? d_logits_prev : nullptr;
+  hs.lse_prev = has_prev ? d_lse_prev : nullptr;
+  if (has_prev && (!d_logits_prev || !d_lse_prev))
+    return fail(SL_ERR_INVALID, "sl_step_stats: has_prev needs previous logits and lse");
+  hs.lse_cur = d_lse_cur;
+  hs.kl = d_kl;
+  hs.unc = d_unc;
+  hs.conf = d_conf;
+  hs.argmax = d_argmax;
+  return step_impl(m, c, a, d_tokens, d_logits, &hs, stream);
 }
 
 extern "C" sl_status sl_layer_forward(sl_model *m, sl_kv_cache *c, sl_active *a, int layer,
@@ -1063,9 +1183,15 @@ extern "C" sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int
                             m->cfg.head_dim, (float *)d_o, s, ks.stamp, ks.gen));
     return SL_OK;
   }
+  if (((uintptr_t)d_q & 15) || ((uintptr_t)d_o & 15))
+    return fail(SL_ERR_INVALID, "sl_attention: q and o must be 16-byte aligned");
+  if (c->map_qx.ptr != d_q || c->map_qx.rows != M) {
+    if (!tma_encode(&c->map_qx, d_q, M, m->cfg.d_model, 128))
+      return fail(SL_ERR_INVALID, "sl_attention: q TMA descriptor encoding failed");
+  }
   AttnSeqs seqs;
   fill_seqs(seqs, a, counts);
-  return attn_bf16(m, c, seqs, layer, M, d_q, d_o, ks, s);
+  return attn_bf16(m, c, seqs, layer, M, d_q, c->map_qx, d_o, ks, s);
 }
 
 extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const void *d_b,
@@ -1147,7 +1273,7 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   }
   int *err = device_error_word();
   if (!err) return fail(SL_ERR_CUDA, "sl_gemm_bf16: no device error word");
-  cudaError_t e = launch_gemm_tc(g, ns, err, (cudaStream_t)stream);
+  cudaError_t e = launch_gemm_hooked(g, ns, err, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "sl_gemm_bf16 launch");
   return SL_OK;
 }
@@ -1298,9 +1424,10 @@ extern "C" sl_status sl_model_set_ablation(sl_model *m, int flags) {
 
 extern "C" sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits) {
   if (!m || (queries_per_cta != 0 && queries_per_cta != 16 && queries_per_cta != 32 &&
-             queries_per_cta != 64) ||
+             queries_per_cta != 64 && queries_per_cta != 128) ||
       splits < 0 || splits > 16)
-    return fail(SL_ERR_INVALID, "sl_model_set_attention: queries_per_cta 0/16/32/64, splits 0..16");
+    return fail(SL_ERR_INVALID,
+                "sl_model_set_attention: queries_per_cta 0/16/32/64/128, splits 0..16");
   m->attn_q = queries_per_cta;
   m->attn_splits = splits;
   return SL_OK;
@@ -1326,6 +1453,57 @@ extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, i
 }
 
 // -------------------------------------------------------------- lock test --
+// The statistics half of the sure test as its own pass over the stored logits
+// (lock_stats): the path of sl_kl_lock, and of sl_step_stats on fp32 models.
+static sl_status kl_stats_unfused(sl_model *timing_model, sl_active *a, int M, int vocab,
+                                  int mask_id, int dtype, const void *cur, const HeadStats &hs,
+                                  cudaStream_t s) {
+  if (M == 0) return SL_OK;
+  LockStatsArgs la;
+  la.dtype = dtype;
+  la.cur = cur;
+  la.prev = hs.prev;
+  la.lse_prev = hs.lse_prev;
+  la.lse_cur = hs.lse_cur;
+  la.rows = a->rows;
+  la.M = M;
+  la.V = vocab;
+  la.mask_id = mask_id;
+  la.has_prev = hs.prev ? 1 : 0;
+  la.kl = hs.kl;
+  la.unc = hs.unc;
+  la.conf = hs.conf;
+  la.argmax = hs.argmax;
+  la.part = a->part;
+  la.counters = a->counters;
+  la.splits = std::min(a->max_splits, lock_stats_splits(M, vocab, a->num_sms));
+  const double bytes = (double)M * vocab * dsize(dtype) * (hs.prev ? 2 : 1) + 24.0 * M;
+  Timed t(timing_model, SL_K_LOCK, bytes, 6.0 * M * vocab, s);
+  SL_CUDA(launch_lock_stats(la, s));
+  return SL_OK;
+}
+
+// The decision half: gate threshold per sequence and the lock flags.
+static sl_status lock_decide_impl(sl_active *a, const uint8_t *masked, const sl_lock_params *p,
+                                  const float *kl, const float *unc, uint8_t *lock,
+                                  cudaStream_t s) {
+  const bool gate_only = p->gate_only && p->scripted_target < 0;
+  // gate only: the same decision with the KL bound at +inf, where D <= eps
+  // always holds, so the gate alone decides among the eligible rows
+  const float eps = gate_only ? INFINITY : p->eps;
+  SL_CUDA(launch_lock_decide(a->seq_off, a->batch, a->rows, kl, unc, masked, eps, p->gate_q,
+                             p->has_prev, p->scripted_target, lock, s));
+  return SL_OK;
+}
+
+static sl_status check_lock_params(const sl_lock_params *p, const char *who) {
+  if (p->gate_q > 1.f) return fail(SL_ERR_INVALID, "%s: gate_q must be <= 1", who);
+  const bool gate_only = p->gate_only && p->scripted_target < 0;
+  if (gate_only && !(p->gate_q >= 0.f))
+    return fail(SL_ERR_INVALID, "%s: the gate-only criterion needs gate_q >= 0", who);
+  return SL_OK;
+}
+
 static sl_status kl_lock_impl(sl_model *timing_model, sl_active *a, int vocab, int mask_id,
                               int dtype, const void *cur, const void *prev, const float *lse_prev,
                               float *lse_cur, const uint8_t *masked, const sl_lock_params *p,
@@ -1339,46 +1517,42 @@ static sl_status kl_lock_impl(sl_model *timing_model, sl_active *a, int vocab, i
     return fail(SL_ERR_INVALID, "sl_kl_lock: vocab must be a positive multiple of 8");
   if (mask_id < -1 || mask_id >= vocab) return fail(SL_ERR_INVALID, "sl_kl_lock: bad mask_id");
   if (dtype != SL_F32 && dtype != SL_BF16) return fail(SL_ERR_INVALID, "sl_kl_lock: bad dtype");
-  if (p->gate_q > 1.f) return fail(SL_ERR_INVALID, "sl_kl_lock: gate_q must be <= 1");
-  const bool gate_only = p->gate_only && p->scripted_target < 0;
-  if (gate_only && !(p->gate_q >= 0.f))
-    return fail(SL_ERR_INVALID, "sl_kl_lock: the gate-only criterion needs gate_q >= 0");
+  sl_status st = check_lock_params(p, "sl_kl_lock");
+  if (st != SL_OK) return st;
   if (((uintptr_t)cur & 15) || (prev && ((uintptr_t)prev & 15)))
     return fail(SL_ERR_INVALID, "sl_kl_lock: logits must be 16-byte aligned");
   int32_t counts[SL_MAX_BATCH];
-  sl_status st = sl_active_counts(a, counts);
+  st = sl_active_counts(a, counts);
   if (st != SL_OK) return st;
   int M = 0;
   for (int b = 0; b < a->batch; ++b) M += counts[b];
   if (M == 0) return SL_OK;
-  LockStatsArgs la;
-  la.dtype = dtype;
-  la.cur = cur;
-  la.prev = prev;
-  la.lse_prev = lse_prev;
-  la.lse_cur = lse_cur;
-  la.rows = a->rows;
-  la.M = M;
-  la.V = vocab;
-  la.mask_id = mask_id;
-  la.has_prev = p->has_prev ? 1 : 0;
-  la.kl = kl;
-  la.unc = unc;
-  la.conf = conf;
-  la.argmax = argmax;
-  la.part = a->part;
-  la.counters = a->counters;
-  la.splits = std::min(a->max_splits, lock_stats_splits(M, vocab, a->num_sms));
-  {
-    const double bytes = (double)M * vocab * dsize(dtype) * (p->has_prev ? 2 : 1) + 24.0 * M;
-    Timed t(timing_model, SL_K_LOCK, bytes, 6.0 * M * vocab, s);
-    SL_CUDA(launch_lock_stats(la, s));
-  }
-  // gate only: the same decision with the KL bound at +inf, where D <= eps
-  // always holds, so the gate alone decides among the eligible rows
-  const float eps = gate_only ? INFINITY : p->eps;
-  SL_CUDA(launch_lock_decide(a->seq_off, a->batch, a->rows, kl, unc, masked, eps, p->gate_q,
-                             p->has_prev, p->scripted_target, lock, s));
+  HeadStats hs;
+  hs.prev = p->has_prev ? prev : nullptr;
+  hs.lse_prev = p->has_prev ? lse_prev : nullptr;
+  hs.lse_cur = lse_cur;
+  hs.kl = kl;
+  hs.unc = unc;
+  hs.conf = conf;
+  hs.argmax = argmax;
+  if ((st = kl_stats_unfused(timing_model, a, M, vocab, mask_id, dtype, cur, hs, s)) != SL_OK)
+    return st;
+  return lock_decide_impl(a, masked, p, kl, unc, lock, s);
+}
+
+extern "C" sl_status sl_lock_decide(sl_active *a, const uint8_t *d_masked,
+                                    const sl_lock_params *p, const float *d_kl,
+                                    const float *d_unc, uint8_t *d_lock, void *stream) {
+  if (!a || !d_masked || !p || !d_kl || !d_unc || !d_lock)
+    return fail(SL_ERR_INVALID, "sl_lock_decide: null argument");
+  sl_status st = check_lock_params(p, "sl_lock_decide");
+  if (st != SL_OK) return st;
+  return lock_decide_impl(a, d_masked, p, d_kl, d_unc, d_lock, (cudaStream_t)stream);
+}
+
+extern "C" sl_status sl_model_set_head_fusion(sl_model *m, int enable) {
+  if (!m) return fail(SL_ERR_INVALID, "sl_model_set_head_fusion: null model");
+  m->head_fusion = enable != 0;
   return SL_OK;
 }
 
@@ -1521,8 +1695,7 @@ extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
   const int t = s->t;
   const int cur = t & 1, prv = cur ^ 1;
   const sl_config &cfg = s->m->cfg;
-  sl_status st = sl_step(s->m, s->cache, s->act, s->tokens, s->logits[cur], stream);
-  if (st != SL_OK) return st;
+  sl_status st = SL_OK;
   sl_lock_params lp;
   lp.eps = s->p.eps;
   lp.gate_q = s->p.gate_q;
@@ -1536,9 +1709,20 @@ extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
     lp.scripted_target = (int)floor(x + 0.5);
     if (lp.scripted_target < 0) lp.scripted_target = 0;
   }
-  st = kl_lock_impl(s->m, s->act, cfg.vocab, cfg.mask_id, cfg.dtype, s->logits[cur],
-                    s->logits[prv], s->lse[prv], s->lse[cur], s->masked, &lp, s->kl, s->unc,
-                    s->conf, s->argmax, s->lock, (cudaStream_t)stream);
+  if (s->m->head_fusion && cfg.dtype == SL_BF16) {
+    // the sure test's statistics come out of the LM head's epilogue
+    st = sl_step_stats(s->m, s->cache, s->act, s->tokens, s->logits[cur], s->logits[prv],
+                       s->lse[prv], lp.has_prev, s->lse[cur], s->kl, s->unc, s->conf, s->argmax,
+                       stream);
+    if (st != SL_OK) return st;
+    st = lock_decide_impl(s->act, s->masked, &lp, s->kl, s->unc, s->lock, (cudaStream_t)stream);
+  } else {
+    st = sl_step(s->m, s->cache, s->act, s->tokens, s->logits[cur], stream);
+    if (st != SL_OK) return st;
+    st = kl_lock_impl(s->m, s->act, cfg.vocab, cfg.mask_id, cfg.dtype, s->logits[cur],
+                      s->logits[prv], s->lse[prv], s->lse[cur], s->masked, &lp, s->kl, s->unc,
+                      s->conf, s->argmax, s->lock, (cudaStream_t)stream);
+  }
   if (st != SL_OK) return st;
   const int spb = s->p.steps / (s->p.gen_len / s->p.block_len);
   const int lo = s->p.prompt_len + (t / spb) * s->p.block_len;
@@ -1555,6 +1739,11 @@ extern "C" sl_status sl_sampler_generate(sl_sampler *s, const int32_t *h_prompts
                                          int32_t *h_tokens, void *stream) {
   if (!s || !h_tokens || (!h_prompts && s->p.prompt_len > 0))
     return fail(SL_ERR_INVALID, "sl_sampler_generate: null argument");
+  const size_t n_prompt = (size_t)s->batch * s->p.prompt_len;
+  for (size_t i = 0; i < n_prompt; ++i)
+    if (h_prompts[i] < 0 || h_prompts[i] >= s->m->cfg.vocab)
+      return fail(SL_ERR_INVALID, "sl_sampler_generate: prompt id %d at %zu outside [0, %d)",
+                  (int)h_prompts[i], i, s->m->cfg.vocab);
   cudaStream_t st = (cudaStream_t)stream;
   if (s->p.prompt_len > 0)
     SL_CUDA(cudaMemcpyAsync(s->d_prompts, h_prompts, (size_t)s->batch * s->p.prompt_len * 4,

@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_ptx.cuh"
 
 namespace sl {
 
@@ -79,125 +80,6 @@ bool tma_encode_out(TmaMat *m, const void *ptr, int rows, int cols, int ld, bool
   return r == CUDA_SUCCESS;
 }
 
-// ------------------------------------------------------- device: PTX glue ---
-__device__ __forceinline__ uint32_t s_addr(const void *p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-  return ok != 0;
-}
-// Bounded wait: false after WAIT_LIMIT_NS or once another role has aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int *abort_flag) {
-  if (mbar_try(bar, parity)) return true;
-  unsigned long long t0 = global_ns();
-  uint32_t spins = 0;
-  while (!mbar_try(bar, parity)) {
-    if ((++spins & 255u) == 0) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
-    }
-  }
-  return true;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// Epilogue stores from shared memory (bulk async-group of the issuing thread).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, uint32_t src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y), "r"(src)
-               : "memory");
-}
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap *map, int x, int y,
-                                                  uint32_t src) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(x), "r"(y), "r"(src)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait0() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 // --- CTA-pair (cluster of 2) helpers for the 2-SM MMA variant
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -251,27 +133,6 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
                : "memory");
 }
 
-// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
-// 64 bf16 (128 B), 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr & 0x3FFFFu) >> 4);   // start address
-  d |= (uint64_t)1 << 16;                    // leading byte offset (unused for SW128 K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: 8 rows x 128 B
-  d |= (uint64_t)1 << 46;                    // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;                    // SWIZZLE_128B
-  return d;
-}
-
-template <int BN, int MMA_M = 128>
-__device__ __forceinline__ constexpr uint32_t idesc_bf16_f32() {
-  return (1u << 4)            // D: fp32
-         | (1u << 7)          // A: bf16
-         | (1u << 10)         // B: bf16
-         | ((uint32_t)(BN >> 3) << 17)
-         | ((uint32_t)(MMA_M >> 4) << 24);
-}
-
 // ---------------------------------------------------------------- kernel ---
 struct TcParams {
   CUtensorMap a;
@@ -288,6 +149,13 @@ struct TcParams {
   int ffn;                 // SWIGLU/ACCUM-swiglu: F (columns of one half)
   const int32_t *row_map;  // STORE: output row per A row; QKV: flat position per row
   int *err;
+  // HEAD epilogue: previous logits (or null), per (row, vocab tile) records
+  const bf16 *prev;
+  float4 *stat;
+  int *stat_idx;
+  int mask_id;
+  unsigned long long wait_ns;  // limit of every barrier wait (WAIT_LIMIT_NS by default)
+  int lost_load;           // test hook: CTA 0 leaves out its first stage's copies
   // QKV epilogue: rotary table [n_ctx][64] (cos, sin), q out [M][d], cache k/v
   const float2 *rope;
   int n_ctx, dmodel;
@@ -537,6 +405,63 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, uint32_t taddr,
         }
       }
     }
+  } else if (EPI == EPI_HEAD) {
+    // Logits of the row's BN vocab entries, rounded to bf16 and stored; the
+    // sure test's statistics are taken on the stored values, so they equal
+    // what a separate pass over the stored logits would find: running max m,
+    // sum of e = exp(z - m), sum of e (z - z_prev), and the best value over
+    // v != mask_id with its lowest index.
+    const int orow = live ? p.row_map[r] : 0;
+    bf16 *dst = reinterpret_cast<bf16 *>(p.out) + (size_t)orow * p.ldo + nt * BN;
+    const bf16 *zpr = p.prev ? p.prev + (size_t)orow * p.ldo + nt * BN : nullptr;
+    float m = -INFINITY, se = 0.f, st = 0.f, bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      tmem_ld32(taddr + c, v);
+      if (!live) continue;
+      float cm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        Pack8 pk;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          pk.h[e] = __float2bfloat16_rn(v[i + e]);
+          v[i + e] = __bfloat162float(pk.h[e]);
+          cm = fmaxf(cm, v[i + e]);
+        }
+        *reinterpret_cast<uint4 *>(dst + c + i) = pk.u;
+      }
+      if (cm > m) {
+        const float sc = (m == -INFINITY) ? 0.f : __expf(m - cm);
+        se *= sc;
+        st = sc == 0.f ? 0.f : st * sc;
+        m = cm;
+      }
+      float zp[32];
+      if (zpr) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          Pack8 pk;
+          pk.u = __ldcs(reinterpret_cast<const uint4 *>(zpr + c + i));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) zp[i + e] = __bfloat162float(pk.h[e]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float e = (m == -INFINITY) ? 0.f : __expf(v[i] - m);
+        se += e;
+        if (zpr && e > 0.f) st = fmaf(e, v[i] - zp[i], st);
+        const int vi = nt * BN + c + i;
+        if (vi != p.mask_id && v[i] > bv) { bv = v[i]; bi = vi; }
+      }
+    }
+    if (live) {
+      const size_t rec = (size_t)r * p.n_tiles + nt;
+      p.stat[rec] = make_float4(m, se, st, bv);
+      p.stat_idx[rec] = bi;
+    }
   } else {
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
@@ -623,12 +548,17 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       // Weight tiles do not depend on the previous kernel: issue the B loads of
       // the first stages of this CTA's first unit before waiting on it, so the
       // weight stream starts while the previous kernel drains.
+      // Test hook (lost_load): CTA 0 never issues the copies of its first
+      // stage, so the MMA warp's wait for them runs out and the kernel winds
+      // down through its error path; nothing is read or written out of place.
+      const bool lost = p.lost_load && blockIdx.x == 0;
       int npre = 0;
       WorkIter first_it(p, blockIdx.x, gridDim.x);
       int mt, nt, kb0, kb1;
       if (first_it.next(p, mt, nt, kb0, kb1)) {
         npre = min(STAGES, kb1 - kb0);
         for (int i = 0; i < npre; ++i) {
+          if (lost && i == 0) continue;
           const uint32_t sb = sbase + i * L::STAGE_BYTES + L::A_BYTES;
           mbar_expect_tx(full_bar(i), L::STAGE_BYTES);
           load_b<BN>(p, sb, nt, kb0 + i, full_bar(i));
@@ -646,19 +576,22 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
         for (int kb = kb0; kb < kb1; ++kb) {
           const bool pre = first && (kb - kb0) < npre;
           if (!pre) {
-            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.wait_ns)) {
               ok = false;
               break;
             }
             mbar_expect_tx(full_bar(stage), L::STAGE_BYTES);
           }
           const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          if (!(lost && first && kb == kb0)) {
 #pragma unroll
-          for (int sub = 0; sub < MSUB; ++sub)
-            tma_load_2d(sa + sub * 16384, &p.a, kb * 64, (mt * MSUB + sub) * 128, full_bar(stage));
-          if (!pre) load_b<BN>(p, sa + L::A_BYTES, nt, kb, full_bar(stage));
-          last_stage = stage;
-          last_phase = phase;
+            for (int sub = 0; sub < MSUB; ++sub)
+              tma_load_2d(sa + sub * 16384, &p.a, kb * 64, (mt * MSUB + sub) * 128,
+                          full_bar(stage));
+            if (!pre) load_b<BN>(p, sa + L::A_BYTES, nt, kb, full_bar(stage));
+            last_stage = stage;
+            last_phase = phase;
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         first = false;
@@ -671,7 +604,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       // make sure the last issued copy has landed before the CTA can exit
       if (last_stage >= 0) {
         volatile int never = 0;
-        mbar_wait(full_bar(last_stage), last_phase, &never);
+        mbar_wait(full_bar(last_stage), last_phase, &never, p.wait_ns);
       }
     }
   } else if (warp == 1) {
@@ -686,11 +619,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       WorkIter it(p, blockIdx.x, gridDim.x);
       int mt, nt, kb0, kb1;
       while (ok && it.next(p, mt, nt, kb0, kb1)) {
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = sbase + stage * L::STAGE_BYTES;
           const uint32_t sb = sa + L::A_BYTES;
@@ -717,7 +650,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       // wait for every issued MMA to finish before TMEM can be released
       tc_commit(drain_bar);
       volatile int never = 0;
-      mbar_wait(drain_bar, 0, &never);
+      mbar_wait(drain_bar, 0, &never, p.wait_ns);
     }
   } else {
     // ---------------------------------------------------------- epilogue
@@ -729,7 +662,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
     WorkIter it(p, blockIdx.x, gridDim.x);
     int mt, nt, kb0, kb1;
     while (it.next(p, mt, nt, kb0, kb1)) {
-      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int sub = 0; sub < MSUB; ++sub) {
@@ -860,7 +793,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
         for (int kb = kb0; kb < kb1; ++kb) {
           const bool pre = first && (kb - kb0) < npre;
           if (!pre) {
-            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
             if (leader) mbar_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
           }
           const uint32_t sa = sbase + stage * STAGE_BYTES;
@@ -889,11 +822,11 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       WorkIter it(p, pair, n_pairs);
       int mt, nt, kb0, kb1;
       while (ok && it.next(p, mt, nt, kb0, kb1)) {
-        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = sbase + stage * STAGE_BYTES;
           const uint64_t adesc = smem_desc_sw128(sa);
@@ -914,7 +847,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       }
       tc_commit_pair(drain_bar);
       volatile int never = 0;
-      mbar_wait(drain_bar, 0, &never);
+      mbar_wait(drain_bar, 0, &never, p.wait_ns);
     }
   } else {
     // ------------------------------------------------- epilogue (both CTAs)
@@ -926,7 +859,7 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
     WorkIter it(p, pair, n_pairs);
     int mt, nt, kb0, kb1;
     while (it.next(p, mt, nt, kb0, kb1)) {
-      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       const int r = mt * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
@@ -1017,6 +950,7 @@ static cudaError_t run_epi2(int epi, const TcParams &p, int pairs, cudaStream_t 
     case EPI_SWIGLU: return run_tc2<BN, STAGES, EPI_SWIGLU>(p, pairs, s);
     case EPI_ACCUM: return run_tc2<BN, STAGES, EPI_ACCUM>(p, pairs, s);
     case EPI_QKV: return run_tc2<BN, STAGES, EPI_QKV>(p, pairs, s);
+    case EPI_HEAD: return run_tc2<BN, STAGES, EPI_HEAD>(p, pairs, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -1029,6 +963,7 @@ static cudaError_t run_epi(int epi, const TcParams &p, int grid, cudaStream_t s)
     case EPI_SWIGLU: return run_tc<BN, STAGES, EPI_SWIGLU, MSUB>(p, grid, s);
     case EPI_ACCUM: return run_tc<BN, STAGES, EPI_ACCUM, MSUB>(p, grid, s);
     case EPI_QKV: return run_tc<BN, STAGES, EPI_QKV, MSUB>(p, grid, s);
+    case EPI_HEAD: return run_tc<BN, STAGES, EPI_HEAD, MSUB>(p, grid, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -1062,7 +997,9 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   // splits < 0: stream-K (partial sums must be summable: RESID and ACCUM only)
   const bool stream_k = a.splits < 0 && (a.epi == EPI_RESID || a.epi == EPI_ACCUM);
   int splits = a.splits < 1 ? 1 : a.splits;
-  if (a.epi == EPI_STORE || a.epi == EPI_QKV || a.epi == EPI_SWIGLU) splits = 1;
+  if (a.epi == EPI_STORE || a.epi == EPI_QKV || a.epi == EPI_SWIGLU || a.epi == EPI_HEAD)
+    splits = 1;
+  if (a.epi == EPI_HEAD && (!a.row_map || !a.stat || !a.stat_idx)) return cudaErrorInvalidValue;
   if (a.epi == EPI_QKV && (bn % 128 != 0 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||
                            (a.N % 3) != 0 || ((a.N / 3) % 128) != 0))
     return cudaErrorInvalidValue;
@@ -1084,9 +1021,15 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.ffn = a.N / 2;
   p.row_map = a.row_map;
   p.err = err;
+  p.wait_ns = a.wait_ns ? a.wait_ns : WAIT_LIMIT_NS;
+  p.lost_load = a.lost_load && !pair_mma ? 1 : 0;
   p.rope = a.rope;
   p.n_ctx = a.n_ctx;
   p.dmodel = a.epi == EPI_QKV ? a.N / 3 : 0;
+  p.prev = (const bf16 *)a.prev;
+  p.stat = a.stat;
+  p.stat_idx = a.stat_idx;
+  p.mask_id = a.mask_id;
   p.q_out = (bf16 *)a.q_out;
   p.ck = (bf16 *)a.ck;
   p.cv = (bf16 *)a.cv;

@@ -70,12 +70,16 @@ enum GemmEpi : int {
   EPI_RESID = 1,      // resid[r][c] += acc   (fp32; atomic when split over K)
   EPI_SWIGLU = 2,     // out[r][c] = silu(gate) * up      (dtype; tile = gate|up halves)
   EPI_ACCUM = 3,      // ws[r][col] += acc  (fp32 atomics, split-K workspace)
-  EPI_QKV = 4         // fused Q|K|V: RoPE(q) -> q_out[r], RoPE(k), v -> cache rows row_map[r]
+  EPI_QKV = 4,        // fused Q|K|V: RoPE(q) -> q_out[r], RoPE(k), v -> cache rows row_map[r]
+  EPI_HEAD = 5        // LM head: as EPI_STORE (bf16 logits at rows row_map[r]) plus the sure
+                      // test's statistics of each (row, vocab tile) on the stored values
 };
 
 // ------------------------------------------------------------------ layers.cu
+// Out-of-range token ids embed as zeros and set DEV_BAD_INDEX in *err.
 cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
-                                const void *emb, int d, float *h, cudaStream_t s);
+                                const void *emb, int d, int vocab, float *h, int *err,
+                                cudaStream_t s);
 cudaError_t launch_rmsnorm(int dtype, const float *h, const void *g, int d, float eps, int M,
                            void *out, cudaStream_t s);
 // qkv_in: [M][3d] (in_f32 ? float : dtype).  q_out [M][d] dtype; ck/cv: the layer's
@@ -119,6 +123,21 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
                              size_t pf_bytes = 0, const int32_t *stamp = nullptr,
                              int gen = 0);
 
+// ----------------------------------------------------------------- attn_tc.cu
+// Tensor-core attention (head_dim 128, bf16): q_map over q [M][d] and k_map /
+// v_map over the layer's cache [B*n_ctx][d], all with 128-row boxes
+// (tma_encode(.., 128)); ws as for launch_attn_bf16; tickets [M][n_heads]
+// zero between calls.  force_splits >= 1 pins the key split (0 = cost model).
+struct TmaMat;
+size_t attn_tc_tickets_bytes(int max_rows, int n_heads);
+int attn_tc_splits(int q_tiles, int n_heads, int n_ctx, int num_sms, int max_splits);
+cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map, const TmaMat &v_map,
+                           const AttnSeqs &seqs, int M, int n_ctx, int n_heads, void *o,
+                           float *ws, unsigned int *tickets, int max_splits, int num_sms,
+                           int *err, unsigned long long wait_ns, cudaStream_t s,
+                           int force_splits = 0, const void *pf = nullptr, size_t pf_bytes = 0,
+                           const int32_t *stamp = nullptr, int gen = 0);
+
 // ----------------------------------------------------------------- gemm_tc.cu
 // A bf16 K-major operand in global memory with its TMA descriptor.
 struct TmaMat {
@@ -150,6 +169,17 @@ struct TcGemmArgs {
   const float2 *rope;
   int n_ctx;
   void *q_out, *ck, *cv;
+  // HEAD: previous step's logits (same row positions; null = no previous
+  // posterior), per (row, vocab tile) records (max, sum e, sum e (z - z_prev),
+  // best value) and best index over v != mask_id; records [M][N / bn]
+  const void *prev;
+  float4 *stat;
+  int *stat_idx;
+  int mask_id;
+  // failure-detection test hooks: barrier wait limit in ns (0 = WAIT_LIMIT_NS),
+  // and CTA 0 leaving out its first stage's operand copies (1-SM kernel only)
+  unsigned long long wait_ns;
+  int lost_load;
 };
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s);
 
@@ -179,6 +209,12 @@ cudaError_t launch_compact(int32_t *rows, int32_t *seq_off, int batch, const uin
 cudaError_t launch_unmask(const int32_t *seq_off, int batch, const int32_t *rows, int n_ctx,
                           const float *conf, const int32_t *argmax, int lo, int hi, int k,
                           int32_t *tokens, uint8_t *masked, cudaStream_t s);
+// Merge of the LM-head epilogue's per-tile records into the sure test's row
+// statistics (the outputs of lock_stats): one warp per row.
+cudaError_t launch_head_stats_merge(const float4 *stat, const int *stat_idx, int n_tiles,
+                                    const int32_t *rows, int M, int has_prev,
+                                    const float *lse_prev, float *lse_cur, float *kl, float *unc,
+                                    float *conf, int32_t *argmax, cudaStream_t s);
 cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n_ctx,
                                cudaStream_t s);
 

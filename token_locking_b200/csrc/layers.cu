@@ -12,29 +12,42 @@ namespace sl {
 // h[j, :] = E[tokens[rows[j]], :]  (fp32 residual stream).  Only the M active
 // rows are embedded: locked rows keep a frozen block input and are not
 // recomputed (gist.science/it section 2, "Azione di Blocco").
+// A token id outside [0, vocab) is never used as an address: the row is
+// embedded as zeros and DEV_BAD_INDEX goes into the device error word (the
+// first error wins), which sl_device_check reports.
 template <typename T>
 __global__ void gather_embed_kernel(const int32_t *__restrict__ tokens,
                                     const int32_t *__restrict__ rows, int M,
-                                    const T *__restrict__ emb, int d, float *__restrict__ h) {
+                                    const T *__restrict__ emb, int d, int vocab,
+                                    float *__restrict__ h, int *__restrict__ err) {
   int j = blockIdx.x;
   if (j >= M) return;
   pdl_wait();
   pdl_trigger();
-  const T *e = emb + (size_t)tokens[rows[j]] * d;
+  const int tok = tokens[rows[j]];
   float *o = h + (size_t)j * d;
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0 && err) atomicCAS(err, DEV_OK, DEV_BAD_INDEX);
+    for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = 0.f;
+    return;
+  }
+  const T *e = emb + (size_t)tok * d;
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = to_f(e[c]);
 }
 
 cudaError_t launch_gather_embed(int dtype, const int32_t *tokens, const int32_t *rows, int M,
-                                const void *emb, int d, float *h, cudaStream_t s) {
-  cudaError_t err = cudaSuccess;
+                                const void *emb, int d, int vocab, float *h, int *err,
+                                cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
   if (M <= 0) return cudaSuccess;
   if (dtype == SL_BF16) {
-    err = launch_k(gather_embed_kernel<bf16>, M, 256, 0, s, tokens, rows, M, (const bf16 *)emb, d, h);
+    e = launch_k(gather_embed_kernel<bf16>, M, 256, 0, s, tokens, rows, M, (const bf16 *)emb, d,
+                 vocab, h, err);
   } else {
-    err = launch_k(gather_embed_kernel<float>, M, 256, 0, s, tokens, rows, M, (const float *)emb, d, h);
+    e = launch_k(gather_embed_kernel<float>, M, 256, 0, s, tokens, rows, M, (const float *)emb, d,
+                 vocab, h, err);
   }
-  return err;
+  return e;
 }
 
 // --------------------------------------------------------------- rmsnorm ---

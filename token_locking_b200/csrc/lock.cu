@@ -32,12 +32,16 @@ struct Stat {
   int bi;     // its lowest index
 };
 
+// x * c, where a factor c that underflowed to 0 also drops an infinite x (a
+// term whose weight is 0 contributes nothing, as 0 log 0 = 0 in the KL).
+__device__ __forceinline__ float scaled(float x, float c) { return c == 0.f ? 0.f : x * c; }
+
 __device__ __forceinline__ void stat_merge(Stat &a, const Stat &b) {
   float m = fmaxf(a.m, b.m);
   float ca = (a.m == -INFINITY) ? 0.f : __expf(a.m - m);
   float cb = (b.m == -INFINITY) ? 0.f : __expf(b.m - m);
   a.s = a.s * ca + b.s * cb;
-  a.t = a.t * ca + b.t * cb;
+  a.t = scaled(a.t, ca) + scaled(b.t, cb);
   a.m = m;
   if (b.bv > a.bv || (b.bv == a.bv && b.bi < a.bi)) { a.bv = b.bv; a.bi = b.bi; }
 }
@@ -82,14 +86,18 @@ __device__ __forceinline__ void stat_add8(Stat &st, const float *z, const float 
   if (cm > st.m) {
     float c = (st.m == -INFINITY) ? 0.f : __expf(st.m - cm);
     st.s *= c;
-    st.t *= c;
+    st.t = scaled(st.t, c);
     st.m = cm;
   }
+  // A -inf logit has probability 0 and adds nothing to s or t (0 log 0 = 0 in
+  // the KL); while every logit seen so far is -inf, st.m is -inf too and the
+  // exponent would be -inf - -inf, so that case is skipped outright.
+  const bool live = st.m != -INFINITY;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    float e = __expf(z[i] - st.m);
+    const float e = live ? __expf(z[i] - st.m) : 0.f;
     st.s += e;
-    if (has_prev) st.t = fmaf(e, z[i] - zp[i], st.t);
+    if (has_prev && e > 0.f) st.t = fmaf(e, z[i] - zp[i], st.t);
     int v = v0 + i;
     if (v != mask_id && z[i] > st.bv) { st.bv = z[i]; st.bi = v; }
   }
@@ -137,6 +145,7 @@ __global__ void __launch_bounds__(LOCK_THREADS) lock_stats_kernel(LockStatsArgs 
   if (sidx == a.splits - 1) {
     for (int e = nvec * 8 + threadIdx.x; e < V; e += LOCK_THREADS) {
       float z = to_f(cur[e]);
+      if (z == -INFINITY) continue;       // probability 0: no term in s, t or the argmax
       float zp = hp ? to_f(prv[e]) : 0.f;
       Stat one{z, 1.f, hp ? (z - zp) : 0.f, (e != a.mask_id) ? z : -INFINITY,
                (e != a.mask_id) ? e : 0x7fffffff};
@@ -204,6 +213,55 @@ __global__ void __launch_bounds__(LOCK_THREADS) lock_stats_kernel(LockStatsArgs 
     a.conf[j] = __expf(st.bv - lse);
     a.argmax[j] = st.bi;
   }
+}
+
+// ------------------------------------------------------ head_stats_merge ----
+// The LM-head GEMM's epilogue leaves one record per (row, vocab tile) of the
+// stored logits: (max, sum e, sum e (z - z_prev), best value) and the best
+// index over v != mask_id.  One warp per active row merges them into the same
+// outputs as lock_stats.
+__global__ void __launch_bounds__(256) head_stats_merge_kernel(
+    const float4 *__restrict__ stat, const int *__restrict__ stat_idx, int n_tiles,
+    const int32_t *__restrict__ rows, int M, int has_prev, const float *__restrict__ lse_prev,
+    float *__restrict__ lse_cur, float *__restrict__ kl, float *__restrict__ unc,
+    float *__restrict__ conf, int32_t *__restrict__ argmax) {
+  const int j = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
+  if (j >= M) return;
+  Stat st{-INFINITY, 0.f, 0.f, -INFINITY, 0x7fffffff};
+  const float4 *rec = stat + (size_t)j * n_tiles;
+  const int *rid = stat_idx + (size_t)j * n_tiles;
+  for (int q = lane; q < n_tiles; q += 32) {
+    const float4 r = __ldcs(rec + q);
+    Stat y{r.x, r.y, r.z, r.w, __ldcs(rid + q)};
+    stat_merge(st, y);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Stat y = stat_shfl(st, o);
+    stat_merge(st, y);
+  }
+  if (lane == 0) {
+    const int p = rows[j];
+    const float lse = st.m + logf(st.s);
+    lse_cur[p] = lse;
+    kl[j] = has_prev ? fmaxf(0.f, st.t / st.s - lse + lse_prev[p]) : INFINITY;
+    unc[j] = fmaxf(0.f, 1.f - 1.f / st.s);
+    conf[j] = __expf(st.bv - lse);
+    argmax[j] = st.bi;
+  }
+}
+
+cudaError_t launch_head_stats_merge(const float4 *stat, const int *stat_idx, int n_tiles,
+                                    const int32_t *rows, int M, int has_prev,
+                                    const float *lse_prev, float *lse_cur, float *kl, float *unc,
+                                    float *conf, int32_t *argmax, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  const int blocks = (M * 32 + 255) / 256;
+  return launch_k(head_stats_merge_kernel, blocks, 256, 0, s, stat, stat_idx, n_tiles, rows, M,
+                  has_prev, lse_prev, lse_cur, kl, unc, conf, argmax);
 }
 
 int lock_stats_splits(int M, int V, int num_sms) {

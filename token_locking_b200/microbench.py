@@ -239,26 +239,30 @@ def bench_decode(args, dev):
 
 def bench_attn(args, dev):
     """sl_attention alone at the LLaDA-8B head layout (32 x 128), warm, for each
-    layout (queries per CTA, key split) and the library's own choice."""
+    layout (queries per CTA, key split) and the library's own choice: 128
+    queries per CTA is the tensor-core kernel, 16/32/64 the mma.sync one.
+    --batch B runs B sequences of M active rows each."""
     shape = wl.LLADA8B
     d = shape.d_model
     tiny = wl.ModelShape(n_layers=1, d_model=d, n_heads=shape.n_heads, head_dim=128, d_ffn=256,
                          vocab=256, mask_id=255, rope_theta=shape.rope_theta)
     model = rt.Model(tiny, wl.torch_weights(tiny, dev), "bf16")
     g = torch.Generator(device=dev).manual_seed(5)
+    B = args.batch
     for n_ctx in args.n_ctx:
-        cache = rt.KVCache(model, 1, n_ctx)
+        cache = rt.KVCache(model, B, n_ctx)
         k, v = cache.view(0)
         k.copy_(torch.randn(k.shape, device=dev, generator=g).to(torch.bfloat16))
         v.copy_(torch.randn(v.shape, device=dev, generator=g).to(torch.bfloat16))
         for M in args.m:
             if M > n_ctx:
                 continue
-            act = rt.Active(1, n_ctx)
-            act.load([np.sort(np.random.default_rng(M).choice(n_ctx, M, replace=False))])
-            q = torch.randn((M, d), device=dev, generator=g).to(torch.bfloat16)
-            o = torch.empty((M, d), device=dev, dtype=torch.bfloat16)
-            for qpc, sp in ((0, 0), (16, 1), (32, 1), (64, 1), (16, 2), (16, 4), (64, 4)):
+            act = rt.Active(B, n_ctx)
+            act.load([np.sort(np.random.default_rng(M + b).choice(n_ctx, M, replace=False))
+                      for b in range(B)])
+            q = torch.randn((B * M, d), device=dev, generator=g).to(torch.bfloat16)
+            o = torch.empty((B * M, d), device=dev, dtype=torch.bfloat16)
+            for qpc, sp in args.attn_layouts:
                 model.set_attention(qpc, sp)
 
                 def fn():
@@ -274,8 +278,9 @@ def bench_attn(args, dev):
                 e1.record()
                 torch.cuda.synchronize()
                 us = e0.elapsed_time(e1) * 1e3 / args.iters
-                fl = 4.0 * M * n_ctx * d
-                print(json.dumps({"case": "attn", "M": M, "n_ctx": n_ctx, "q_per_cta": qpc,
+                fl = 4.0 * B * M * n_ctx * d
+                print(json.dumps({"case": "attn", "batch": B, "M": M, "n_ctx": n_ctx,
+                                  "q_per_cta": qpc,
                                   "splits": sp, "us": round(us, 2),
                                   "TFLOPs": round(fl / us / 1e6, 1)}), flush=True)
         cache.close()
@@ -375,6 +380,9 @@ def main():
     ap.add_argument("--windows", default=None,
                     help="decode: profile --steps steps at each of these step indices")
     ap.add_argument("--n-ctx", default="384,2048", help="attn: key counts")
+    ap.add_argument("--batch", type=int, default=1, help="attn: sequences")
+    ap.add_argument("--layouts", default="0:0,128:1,128:2,128:4,16:1,32:1,64:1,16:2,16:4,64:4",
+                    help="attn: queries-per-CTA:splits list (0:0 = the library's choice)")
     ap.add_argument("--tuning-out", default=None, help="decode: save the autotuned GEMM tilings")
     ap.add_argument("--tuning-in", default=None,
                     help="decode: load GEMM tilings instead of autotuning (e.g. under a profiler)")
@@ -382,6 +390,7 @@ def main():
     default = {"layer": wl.LAYER_MICRO_M, "lock": wl.LOCK_MICRO_M, "decode": (),
                "gemm": (8, 64, 128, 200, 256, 384, 1024), "attn": (8, 58, 198, 384)}[args.case]
     args.n_ctx = [int(x) for x in args.n_ctx.split(",")]
+    args.attn_layouts = [tuple(int(v) for v in x.split(":")) for x in args.layouts.split(",")]
     args.m = [int(x) for x in args.m.split(",")] if args.m else list(default)
     dev = torch.device("cuda:0")
     {"layer": bench_layer, "lock": bench_lock, "decode": bench_decode,

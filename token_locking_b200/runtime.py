@@ -119,6 +119,12 @@ class Model:
         flags = (A.ABLATE_NO_KV_CACHE if no_kv_cache else 0) | (A.ABLATE_GATE_ONLY if gate_only else 0)
         A.check(A.lib().sl_model_set_ablation(self.handle, flags), "sl_model_set_ablation")
 
+    def set_head_fusion(self, enable: bool = True):
+        """Samplers take the sure test's statistics from the LM head's epilogue
+        (True, the default) or from a separate pass over the logits."""
+        A.check(A.lib().sl_model_set_head_fusion(self.handle, 1 if enable else 0),
+                "sl_model_set_head_fusion")
+
     def set_tuning(self, kind: int, M: int, bn: int, splits: int, variant: int):
         """Pin GEMM `kind`'s tiling for the row-count bucket of M (splits -1: stream-K)."""
         A.check(A.lib().sl_model_set_tuning(self.handle, kind, M, bn, splits, variant),
@@ -272,6 +278,16 @@ def device_check(clear: bool = True):
     A.check(A.lib().sl_device_check(1 if clear else 0), "sl_device_check")
 
 
+def debug_set_wait_limit(ns: int):
+    """Barrier-wait limit of later GEMM launches in ns (0 = the default 2 s)."""
+    A.check(A.lib().sl_debug_set_wait_limit(int(ns)), "sl_debug_set_wait_limit")
+
+
+def debug_inject_lost_load():
+    """The next 1-SM GEMM launch leaves out its first stage's copies (test hook)."""
+    A.check(A.lib().sl_debug_inject_lost_load(), "sl_debug_inject_lost_load")
+
+
 def kl_lock(active: Active, vocab: int, mask_id: int, logits_cur: torch.Tensor,
             logits_prev: Optional[torch.Tensor], lse_prev: Optional[torch.Tensor],
             lse_cur: torch.Tensor, masked: torch.Tensor, kl: torch.Tensor, unc: torch.Tensor,
@@ -283,6 +299,27 @@ def kl_lock(active: Active, vocab: int, mask_id: int, logits_cur: torch.Tensor,
                                _ptr(logits_cur), _ptr(logits_prev), _ptr(lse_prev), _ptr(lse_cur),
                                _ptr(masked), C.byref(p), _ptr(kl), _ptr(unc), _ptr(conf),
                                _ptr(argmax), _ptr(lock), _stream(stream)), "sl_kl_lock")
+
+
+def step_stats(model: Model, cache: KVCache, active: Active, tokens: torch.Tensor,
+               logits: torch.Tensor, logits_prev: Optional[torch.Tensor],
+               lse_prev: Optional[torch.Tensor], lse_cur: torch.Tensor, kl: torch.Tensor,
+               unc: torch.Tensor, conf: torch.Tensor, argmax: torch.Tensor,
+               has_prev: bool = True, stream=None):
+    """sl_step with the sure test's statistics taken in the LM head's epilogue."""
+    A.check(A.lib().sl_step_stats(model.handle, cache.handle, active.handle, _ptr(tokens),
+                                  _ptr(logits), _ptr(logits_prev), _ptr(lse_prev),
+                                  1 if has_prev else 0, _ptr(lse_cur), _ptr(kl), _ptr(unc),
+                                  _ptr(conf), _ptr(argmax), _stream(stream)), "sl_step_stats")
+
+
+def lock_decide(active: Active, masked: torch.Tensor, kl: torch.Tensor, unc: torch.Tensor,
+                lock: torch.Tensor, eps: float, gate_q: float = -1.0, has_prev: bool = True,
+                scripted_target: int = -1, gate_only: bool = False, stream=None):
+    """The lock flags from precomputed statistics (sl_lock_decide)."""
+    p = A.LockParams(eps, gate_q, 1 if has_prev else 0, scripted_target, 1 if gate_only else 0)
+    A.check(A.lib().sl_lock_decide(active.handle, _ptr(masked), C.byref(p), _ptr(kl), _ptr(unc),
+                                   _ptr(lock), _stream(stream)), "sl_lock_decide")
 
 
 def kl_stats_noalloc(rows: torch.Tensor, vocab: int, mask_id: int, logits_cur: torch.Tensor,
