@@ -332,6 +332,12 @@ class Ranks:
             self.dist = None
 
 
+def aux_decodes(k: int, decode_ms: float, budget_ms: float = 20000.0) -> int:
+    """Decodes of each instrumented / end-to-end pass: about `budget_ms` of
+    decoding, at least one, at most the timed count."""
+    return max(1, min(k, int(budget_ms // max(decode_ms, 1e-3))))
+
+
 def replica_prompt_seed(rank: int) -> int:
     """Each replica decodes its own prompts."""
     return wl.SEED_PROMPTS + rank
@@ -396,6 +402,9 @@ def run_ours(args, rank: int, world: int):
     kernels_timed = model.timing_read(reset=True)["kernels"]
     barrier()
     ms = max_over_ranks(ms_local)
+    # the instrumented and end-to-end passes run `aux` decodes (about 20 s of
+    # decoding each, at most K): the timed region above is never shortened
+    aux = aux_decodes(args.steps, ms / args.steps)
 
     # Per-kernel CUDA events around every GEMM / attention / lock launch.  An
     # event between two kernels also removes the programmatic-launch overlap at
@@ -408,7 +417,7 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     ei0, ei1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ei0.record()
-    for _ in range(args.steps):
+    for _ in range(aux):
         decode()
     ei1.record()
     torch.cuda.synchronize()
@@ -438,7 +447,7 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
+    for _ in range(aux):
         s.generate_ptr(h_prompts.data_ptr(), h_out.data_ptr())
     e1.record()
     torch.cuda.synchronize()
@@ -449,7 +458,7 @@ def run_ours(args, rank: int, world: int):
     if rank == 0:
         peaks = load_peaks()
         value = aggregate_rate(world, args.steps * T, ms)
-        e2e_value = aggregate_rate(world, args.steps * T, e2e_ms)
+        e2e_value = aggregate_rate(world, aux * T, e2e_ms)
         gen_tokens = world * args.steps * setup.batch * setup.gen_len
         # per-step roofline over the trajectory, burst peaks
         pf = peaks["bf16_tflops"] * 1e12
@@ -499,7 +508,8 @@ def run_ours(args, rank: int, world: int):
             "config": workload_config(args, setup, world),
             "gen_tok_s": round(gen_tokens / (ms / 1e3), 3),
             "e2e": {"value": round(e2e_value, 3), "unit": "denoise steps/s",
-                    "gen_tok_s": round(gen_tokens / (e2e_ms / 1e3), 3),
+                    "gen_tok_s": round(gen_tokens * aux / args.steps / (e2e_ms / 1e3), 3),
+                    "decodes": aux,
                     "h2d_bytes_per_step": int(prompts.nbytes),
                     "d2h_bytes_per_step": int(setup.batch * setup.n_ctx * 4)},
             "roofline": {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
@@ -508,8 +518,8 @@ def run_ours(args, rank: int, world: int):
                          "kernel": "gemm_tc_kernel (tcgen05)",
                          "launches": g["launches"], "kernel_ms": round(g["ms"], 3),
                          "peak_source": peaks["source"],
-                         "measured_in": f"instrumented pass of the same {args.steps} decodes "
-                                        f"({ms_instr / args.steps:.1f} ms/decode with events)"},
+                         "measured_in": f"instrumented pass of {aux} more decode(s) "
+                                        f"({ms_instr / aux:.1f} ms/decode with events)"},
             "step_roofline": {"frac": round(step_frac, 4), "roofline_ms_per_decode":
                               round(sum(roof) * 1e3, 3), "measured_ms_per_decode":
                               round(decode_ms, 3), "peaks": "burst (bf16_tflops, hbm_gbs)"},

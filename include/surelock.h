@@ -89,8 +89,16 @@ const char *sl_version(void);
 
 /* ---------------------------------------------------------------- model --- */
 
-/* Borrow device weights and build the per-model launch state (TMA descriptors
- * for the bf16 path).  Fails with SL_ERR_INVALID on an inconsistent config. */
+/* The denoiser whose steps the method runs on the active rows only: a
+ * bidirectional masked-diffusion transformer (the pages evaluate LLaDA-8B;
+ * Paper-Notes, "Method: overall framework": the model is applied to the
+ * active set A_t while the locked set L_t is served from the cache).  The
+ * pages give no model details beyond that; the layer layout here (RMSNorm,
+ * rotary attention, SwiGLU FFN, untied LM head) is the LLaDA-style reading.
+ * Borrows the caller's device weights (they must outlive the model; nothing
+ * is copied) and builds the per-model launch state (TMA descriptors for the
+ * bf16 path).  Fails with SL_ERR_INVALID on an inconsistent config (no work
+ * is enqueued), SL_ERR_OOM if its small device state cannot be allocated. */
 sl_status sl_model_create(const sl_config *cfg, const sl_weights *w, sl_model **out);
 /* Frees the model's launch state (not the borrowed weights).  Caches and
  * samplers created from it must be destroyed first.  NULL is a no-op. */
@@ -112,20 +120,28 @@ void sl_kv_cache_destroy(sl_kv_cache *c);
 
 /* ------------------------------------------------------------ active set --- */
 
-/* A_t for a batch: on the device, a flat ascending list of positions
- * rows[0..M) (entry b*n_ctx + i) and per-sequence offsets seq_off[0..batch]
- * (seq_off[batch] = M).  A_0 holds every position.  The host keeps a mirror of
- * the per-sequence counts, refreshed by sl_active_counts. */
+/* The active set A_t of the pages (Paper-Notes, "Method: overall framework":
+ * each step splits the positions into the active set A_t, which is computed,
+ * and the locked set L_t, which is not; "permanent locking": a position never
+ * leaves L_t, so A_t only shrinks).  For a batch: on the device, a flat
+ * ascending list of positions rows[0..M) (entry b*n_ctx + i) and per-sequence
+ * offsets seq_off[0..batch] (seq_off[batch] = M).  The host keeps a mirror of
+ * the per-sequence counts, refreshed by sl_active_counts.  batch in
+ * [1, SL_MAX_BATCH], n_ctx > 0, else SL_ERR_INVALID; SL_ERR_OOM if the device
+ * or pinned buffers cannot be allocated.  Owns its memory (sl_active_destroy). */
 sl_status sl_active_create(int batch, int n_ctx, sl_active **out);
-/* A_0 = {0..n_ctx-1} for every sequence. */
+/* A_0 = {0..n_ctx-1} for every sequence: at the first step nothing is locked
+ * (Paper-Notes, "Method: overall framework"). */
 sl_status sl_active_reset(sl_active *a, void *stream);
 /* Teacher forcing: h_counts[batch], h_pos = the concatenated ascending local
  * positions (i in [0, n_ctx)) of every sequence.  SL_ERR_INVALID if a list is
  * not strictly ascending or out of range. */
 sl_status sl_active_load(sl_active *a, const int32_t *h_counts, const int32_t *h_pos, void *stream);
-/* Per-sequence counts |A_t^b| into h_counts[batch]; waits for the last update
- * enqueued on the active set to finish. */
+/* Per-sequence counts |A_t^b| = M_t of the pages (Paper-Notes, "Key
+ * findings": M_t falls monotonically over the decode) into h_counts[batch];
+ * waits for the last update enqueued on the active set to finish. */
 sl_status sl_active_counts(sl_active *a, int32_t *h_counts);
+/* Device pointers of rows[] and seq_off[] (owned by the active set). */
 sl_status sl_active_view(const sl_active *a, int32_t **d_rows, int32_t **d_seq_off);
 void sl_active_destroy(sl_active *a);
 

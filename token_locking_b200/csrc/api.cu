@@ -10,6 +10,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -132,6 +133,7 @@ struct sl_kv_cache {
   std::vector<TmaMat> k_maps, v_maps;     // per layer, 128-row boxes (tensor-core attention)
   TmaMat map_q;                           // q workspace [M][d], 128-row boxes
   TmaMat map_qx{};                        // a caller's q (sl_attention), by pointer and M
+  unsigned int *fix_ctr = nullptr;        // split-K fix-up tickets [max_rows/32 + 8][384]
   float4 *head_stat = nullptr;            // [max_rows][V / 64] LM-head tile records (bf16)
   int *head_stat_idx = nullptr;
   int32_t *key_stamp = nullptr;   // [max_rows] visible-key stamps (no-KV-cache ablation)
@@ -366,10 +368,17 @@ extern "C" void sl_kv_cache_destroy(sl_kv_cache *c) {
   void *ps[] = {c->rope,         c->h,         c->a,          c->qkv,
                 c->q,            c->o,         c->act,        c->ws,
                 c->attn_ws,      c->key_stamp, c->attn_tickets, c->head_stat,
-                c->head_stat_idx};
+                c->head_stat_idx, c->fix_ctr};
   for (void *p : ps)
     if (p) cudaFree(p);
   delete c;
+}
+
+// Split-K fix-up tickets: one per (32-row group, column tile) of the widest
+// split projection at the narrowest tile (64 columns).
+static size_t fix_ctr_bytes(int max_rows, const sl_config &cfg) {
+  const size_t cols = std::max((size_t)3 * cfg.d_model, (size_t)2 * cfg.d_ffn);
+  return ((size_t)max_rows / 32 + 8) * (cols / 64) * sizeof(unsigned int);
 }
 
 extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
@@ -408,7 +417,8 @@ extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
                                                                c->attn_max_splits)) &&
          alloc((void **)&c->attn_tickets, attn_tc_tickets_bytes(c->max_rows, cfg.n_heads)) &&
          alloc((void **)&c->head_stat, rows * (cfg.vocab / 64) * sizeof(float4)) &&
-         alloc((void **)&c->head_stat_idx, rows * (cfg.vocab / 64) * sizeof(int));
+         alloc((void **)&c->head_stat_idx, rows * (cfg.vocab / 64) * sizeof(int)) &&
+         alloc((void **)&c->fix_ctr, fix_ctr_bytes(c->max_rows, cfg));
     c->k_maps.resize(cfg.n_layers);
     c->v_maps.resize(cfg.n_layers);
     for (int l = 0; l < cfg.n_layers && ok; ++l)
@@ -766,9 +776,32 @@ static sl_status layer_f32(sl_model *m, sl_kv_cache *c, sl_active *a, int l, flo
 static std::atomic<unsigned long long> g_wait_limit_ns{0};
 static std::atomic<int> g_lost_load{0};
 
+// K-blocks of weight tiles a GEMM prefetches into L2 while it waits for its
+// predecessor (SL_GEMM_L2_PREFETCH overrides the default; read once).
+static int gemm_l2_prefetch_kblocks() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("SL_GEMM_L2_PREFETCH");
+    v = e ? std::max(0, std::min(256, atoi(e))) : 0;
+  }
+  return v;
+}
+
+// Split-K tile fix-up in the GEMM epilogue instead of a finalize kernel
+// (SL_GEMM_FIXUP=0 turns it off; read once).
+static bool gemm_fixup_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char *e = getenv("SL_GEMM_FIXUP");
+    v = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+
 static cudaError_t launch_gemm_hooked(TcGemmArgs g, int num_sms, int *err, cudaStream_t s) {
   g.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   g.lost_load = g_lost_load.exchange(0, std::memory_order_relaxed);
+  g.l2_pf = gemm_l2_prefetch_kblocks();
   return launch_gemm_tc(g, num_sms, err, s);
 }
 
@@ -933,11 +966,21 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       g.N = 3 * d;
       g.K = d;
       if (split) {
-        // K split across CTAs: fp32 partial sums, then RoPE + scatter from them
+        // K split across CTAs: fp32 partial sums, then RoPE + scatter from them,
+        // by the tile fix-up in the GEMM's epilogue when tiles hold whole heads
         g.epi = EPI_ACCUM;
         g.out = c->ws;
         g.ldo = 3 * d;
         g.OUT = &c->out_ws3;
+        if (gemm_fixup_enabled() && pl.bn % 128 == 0) {
+          g.fix_ctr = c->fix_ctr;
+          g.row_map = rows;
+          g.rope = c->rope;
+          g.n_ctx = c->n_ctx;
+          g.q_out = c->q;
+          g.ck = c->k[l];
+          g.cv = c->v[l];
+        }
       } else {
         g.epi = EPI_QKV;
         g.row_map = rows;
@@ -988,6 +1031,10 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       g.out = split ? (void *)c->ws : c->act;
       g.ldo = split ? 2 * f : f;
       g.OUT = split ? &c->out_ws2 : &c->out_act;
+      if (split && gemm_fixup_enabled()) {
+        g.fix_ctr = c->fix_ctr;
+        g.fix_act = c->act;
+      }
       bytes = gemm_bytes(Md, 2.0 * f, d, 2) - 2.0 * Md * f;
       flops = 4.0 * Md * d * f;
       break;
@@ -1021,10 +1068,11 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
     sl_status st = tc_gemm(m, g, s);
     if (st != SL_OK) return st;
   }
-  if (split && kind == G_QKV)
+  if (split && kind == G_QKV && !g.fix_ctr)
     SL_CUDA(launch_rope_scatter(SL_BF16, c->ws, true, true, M, rows, c->n_ctx, H, cfg.head_dim,
                                 c->rope, c->q, c->k[l], c->v[l], s));
-  if (split && kind == G_GU) SL_CUDA(launch_swiglu(SL_BF16, c->ws, true, true, M, f, c->act, s));
+  if (split && kind == G_GU && !g.fix_ctr)
+    SL_CUDA(launch_swiglu(SL_BF16, c->ws, true, true, M, f, c->act, s));
   return SL_OK;
 }
 

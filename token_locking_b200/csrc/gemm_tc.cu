@@ -156,6 +156,11 @@ struct TcParams {
   int mask_id;
   unsigned long long wait_ns;  // limit of every barrier wait (WAIT_LIMIT_NS by default)
   int lost_load;           // test hook: CTA 0 leaves out its first stage's copies
+  int fixup;               // ACCUM: the split-K tile fix-up (see accum_fixup)
+  unsigned int *fix_ctr;   // [ceil(M / 32)][n_tiles] arrival tickets, zero between uses
+  bf16 *fix_act;           // gate/up fix-up output [M][ffn]
+  int l2_pf;               // K-blocks of the first unit's weights prefetched into L2
+                           // beyond the ring while waiting on the previous kernel
   // QKV epilogue: rotary table [n_ctx][64] (cos, sin), q out [M][d], cache k/v
   const float2 *rope;
   int n_ctx, dmodel;
@@ -197,19 +202,26 @@ __device__ __forceinline__ void decode_unit(const TcParams &p, int u, int splits
 // same number of K-blocks whatever the tile count (partial tiles are summed
 // atomically by the epilogue).
 struct WorkIter {
-  long long pos, end;
-  int step;
-  __device__ __forceinline__ WorkIter(const TcParams &p, int w, int nw) {
+  long long pos, end, total;
+  int step, nw;
+  int ncontrib;            // partial tiles summed into the current item's tile
+  __device__ __forceinline__ WorkIter(const TcParams &p, int w, int nw_) : nw(nw_) {
     if (p.stream_k) {
-      const long long I = (long long)p.m_tiles * p.n_tiles * p.kblocks;
-      pos = I * w / nw;
-      end = I * (w + 1) / nw;
+      total = (long long)p.m_tiles * p.n_tiles * p.kblocks;
+      pos = total * w / nw;
+      end = total * (w + 1) / nw;
       step = 0;
     } else {
+      total = p.units;
       pos = w;
       end = p.units;
       step = nw;
     }
+  }
+  // Stream-K: the worker whose share holds iteration x (every share is
+  // non-empty: the grid never exceeds the iteration count).
+  __device__ __forceinline__ long long owner(long long x) const {
+    return ((x + 1) * nw - 1) / total;
   }
   __device__ __forceinline__ bool next(const TcParams &p, int &mt, int &nt, int &kb0, int &kb1) {
     if (pos >= end) return false;
@@ -220,11 +232,14 @@ struct WorkIter {
       kb1 = (int)min((long long)p.kblocks, (long long)kb0 + (end - pos));
       pos = (long long)t * p.kblocks + kb1;
       decode_unit(p, t, 1, mt, nt, sp);
+      const long long first = (long long)t * p.kblocks;
+      ncontrib = (int)(owner(first + p.kblocks - 1) - owner(first) + 1);
     } else {
       decode_unit(p, (int)pos, p.splits, mt, nt, sp);
       kb0 = sp * p.kb_per_split;
       kb1 = min(p.kblocks, kb0 + p.kb_per_split);
       pos += step;
+      ncontrib = p.splits;
     }
     return true;
   }
@@ -257,6 +272,21 @@ __device__ __forceinline__ void load_b(const TcParams &p, uint32_t sb, int nt, i
   }
 }
 
+// L2 prefetch of the same B tile (no shared memory involved).
+template <int BN>
+__device__ __forceinline__ void prefetch_b(const TcParams &p, int nt, int kb) {
+  if (p.b_swiglu) {
+    const int f0 = nt * (BN / 2);
+    tma_prefetch_l2_2d(&p.b[0], kb * 64, f0);
+    tma_prefetch_l2_2d(&p.b[1], kb * 64, f0);
+  } else {
+    const int c0 = nt * BN;
+    if (c0 < p.seg0) tma_prefetch_l2_2d(&p.b[0], kb * 64, c0);
+    else if (c0 < p.seg1) tma_prefetch_l2_2d(&p.b[1], kb * 64, c0 - p.seg0);
+    else tma_prefetch_l2_2d(&p.b[2], kb * 64, c0 - p.seg1);
+  }
+}
+
 // Put 128 bytes of row `lane` into the warp's staging box (16-byte chunk j at
 // j ^ (row % 8): the 128-byte swizzle, and conflict-free per 8 lanes) once the
 // previous bulk copy out of the box has read it.
@@ -278,12 +308,99 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return l | (h << 16);
 }
 
+// Split-K tile fix-up: once every partial tile of this warp's 32 rows has been
+// added into the fp32 workspace (per row group and column tile, an arrival
+// ticket counts the contributors), the warp that adds the last one applies
+// the projection's finishing step to those rows itself and clears the
+// workspace for the next split GEMM: RoPE of q and k and the cache scatter of
+// k, v (fused Q|K|V), or SiLU(gate) * up (fused gate/up).  This replaces a
+// separate finalize kernel and its launch boundary.
+template <int BN>
+__device__ __forceinline__ void accum_fixup(const TcParams &p, int row0, int nt, int ncontrib,
+                                            int lane) {
+  int last = 0;
+  if (lane == 0) {
+    bulk_wait0();                                  // this warp's reduce-adds are done
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __threadfence();
+    unsigned int *ctr = p.fix_ctr + (size_t)(row0 >> 5) * p.n_tiles + nt;
+    last = atomicAdd(ctr, 1u) == (unsigned)(ncontrib - 1);
+    if (last) *ctr = 0u;                           // ready for the next launch
+  }
+  last = __shfl_sync(0xffffffffu, last, 0);
+  if (!last) return;
+  __threadfence();
+  const int r = row0 + lane;
+  if (r >= p.M) return;
+  float *wrow = reinterpret_cast<float *>(p.out) + (size_t)r * p.ldo;
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.b_swiglu) {
+    const int f0 = nt * (BN / 2);
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 8) {
+      float4 *g = reinterpret_cast<float4 *>(wrow + f0 + c);
+      float4 *u = reinterpret_cast<float4 *>(wrow + p.ffn + f0 + c);
+      const float4 g0 = __ldcg(g), g1 = __ldcg(g + 1), u0 = __ldcg(u), u1 = __ldcg(u + 1);
+      g[0] = z4; g[1] = z4; u[0] = z4; u[1] = z4;
+      const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+      const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+      Pack8 o;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o.h[e] = __float2bfloat16_rn(silu_f(gv[e]) * uv[e]);
+      *reinterpret_cast<uint4 *>(p.fix_act + (size_t)r * p.ffn + f0 + c) = o.u;
+    }
+    return;
+  }
+  // fused Q|K|V: the tile holds whole heads of one segment
+  const int col0 = nt * BN;
+  const int seg = col0 / p.dmodel;                 // 0 q, 1 k, 2 v
+  const int pos_flat = p.row_map[r];
+  const int pos = pos_flat % p.n_ctx;
+  bf16 *dst_row = seg == 0 ? p.q_out + (size_t)r * p.dmodel
+                           : (seg == 1 ? p.ck : p.cv) + (size_t)pos_flat * p.dmodel;
+#pragma unroll 1
+  for (int hd = 0; hd < BN / 128; ++hd) {
+    const int cw = col0 + hd * 128;                // workspace column of the head
+    const int cs = cw - seg * p.dmodel;            // its column in the segment
+#pragma unroll 1
+    for (int i0 = 0; i0 < 64; i0 += 8) {
+      float4 *a = reinterpret_cast<float4 *>(wrow + cw + i0);
+      float4 *b = reinterpret_cast<float4 *>(wrow + cw + 64 + i0);
+      const float4 a0 = __ldcg(a), a1 = __ldcg(a + 1), b0 = __ldcg(b), b1 = __ldcg(b + 1);
+      a[0] = z4; a[1] = z4; b[0] = z4; b[1] = z4;
+      const float x0[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float x1[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      Pack8 lo, hi;
+      if (seg < 2) {
+        const float4 *tab = reinterpret_cast<const float4 *>(p.rope + (size_t)pos * 64 + i0);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const float4 cs4 = __ldg(tab + (e >> 1));    // (cos, sin) of pairs e and e + 1
+          lo.h[e] = __float2bfloat16_rn(x0[e] * cs4.x - x1[e] * cs4.y);
+          hi.h[e] = __float2bfloat16_rn(x1[e] * cs4.x + x0[e] * cs4.y);
+          lo.h[e + 1] = __float2bfloat16_rn(x0[e + 1] * cs4.z - x1[e + 1] * cs4.w);
+          hi.h[e + 1] = __float2bfloat16_rn(x1[e + 1] * cs4.z + x0[e + 1] * cs4.w);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          lo.h[e] = __float2bfloat16_rn(x0[e]);
+          hi.h[e] = __float2bfloat16_rn(x1[e]);
+        }
+      }
+      *reinterpret_cast<uint4 *>(dst_row + cs + i0) = lo.u;
+      *reinterpret_cast<uint4 *>(dst_row + cs + 64 + i0) = hi.u;
+    }
+  }
+}
+
 // TMA epilogue of RESID / ACCUM (fp32 reduce-add) and SWIGLU (bf16 store): the
 // warp's 32 rows x 32 (64) columns go through its staging box and leave as one
 // bulk tensor copy, whole 128-byte lines; boxes past the live rows are skipped.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_tile_tma(const TcParams &p, uint32_t taddr, int row0,
-                                                  int nt, uint32_t stg, int lane) {
+                                                  int nt, uint32_t stg, int lane,
+                                                  int ncontrib = 0) {
   if (row0 >= p.M) return;
   float v[32];
   if (EPI == EPI_SWIGLU) {
@@ -332,6 +449,7 @@ __device__ __forceinline__ void epilogue_tile_tma(const TcParams &p, uint32_t ta
         bulk_commit();
       }
     }
+    if (EPI == EPI_ACCUM && p.fixup) accum_fixup<BN>(p, row0, nt, ncontrib, lane);
   }
 }
 
@@ -448,13 +566,21 @@ __device__ __forceinline__ void epilogue_tile(const TcParams &p, uint32_t taddr,
           for (int e = 0; e < 8; ++e) zp[i + e] = __bfloat162float(pk.h[e]);
         }
       }
+      // the chunk's terms are summed in groups of 8, then added to the running
+      // sums, so that small terms do not each round against a sum near 1
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float e = (m == -INFINITY) ? 0.f : __expf(v[i] - m);
-        se += e;
-        if (zpr && e > 0.f) st = fmaf(e, v[i] - zp[i], st);
-        const int vi = nt * BN + c + i;
-        if (vi != p.mask_id && v[i] > bv) { bv = v[i]; bi = vi; }
+      for (int i = 0; i < 32; i += 8) {
+        float gs = 0.f, gt = 0.f;
+#pragma unroll
+        for (int e8 = 0; e8 < 8; ++e8) {
+          const float e = (m == -INFINITY) ? 0.f : __expf(v[i + e8] - m);
+          gs += e;
+          if (zpr && e > 0.f) gt = fmaf(e, v[i + e8] - zp[i + e8], gt);
+          const int vi = nt * BN + c + i + e8;
+          if (vi != p.mask_id && v[i + e8] > bv) { bv = v[i + e8]; bi = vi; }
+        }
+        se += gs;
+        st += gt;
       }
     }
     if (live) {
@@ -563,6 +689,10 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           mbar_expect_tx(full_bar(i), L::STAGE_BYTES);
           load_b<BN>(p, sb, nt, kb0 + i, full_bar(i));
         }
+        // while the previous kernel drains, keep HBM busy with the weight
+        // tiles that follow the ring: they wait in L2 for the main loop
+        const int npf = min(p.l2_pf, kb1 - kb0 - npre);
+        for (int i = 0; i < npf; ++i) prefetch_b<BN>(p, nt, kb0 + npre + i);
       }
       pdl_wait();
       int stage = 0;
@@ -670,7 +800,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
       const uint32_t taddr = tmem_base + (uint32_t)(acc * ACC_COLS + sub * BN) +
                              ((uint32_t)(q * 32) << 16);
       if constexpr (EPI == EPI_RESID || EPI == EPI_ACCUM)
-        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane);
+        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane,
+                                   it.ncontrib);
       else if (EPI == EPI_SWIGLU && (BN / 2) % 64 == 0 && p.tma_out)
         epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + L::EPI_OFF + q * 4096, lane);
       else
@@ -783,6 +914,18 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
           if (leader) mbar_expect_tx(full_bar(i), 2 * STAGE_BYTES);
           load_b_half(sbase + i * STAGE_BYTES + A_BYTES, nt, kb0 + i, map_to_rank(full_bar(i), 0));
         }
+        const int npf = min(p.l2_pf, kb1 - kb0 - npre);
+        for (int i = 0; i < npf; ++i) {
+          const int kb = kb0 + npre + i;
+          if (p.b_swiglu) {
+            tma_prefetch_l2_2d(&p.b[rank], kb * 64, nt * (BN / 2));
+          } else {
+            const int c0 = nt * BN + (int)rank * (BN / 2);
+            if (c0 < p.seg0) tma_prefetch_l2_2d(&p.b[0], kb * 64, c0);
+            else if (c0 < p.seg1) tma_prefetch_l2_2d(&p.b[1], kb * 64, c0 - p.seg0);
+            else tma_prefetch_l2_2d(&p.b[2], kb * 64, c0 - p.seg1);
+          }
+        }
       }
       pdl_wait();
       int stage = 0;
@@ -864,7 +1007,8 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
       const int r = mt * 256 + (int)rank * 128 + q * 32 + lane;
       const uint32_t taddr = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
       if constexpr (EPI == EPI_RESID || EPI == EPI_ACCUM)
-        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane);
+        epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane,
+                                   it.ncontrib);
       else if (EPI == EPI_SWIGLU && (BN / 2) % 64 == 0 && p.tma_out)
         epilogue_tile_tma<BN, EPI>(p, taddr, r - lane, nt, sbase + EPI_OFF + q * 4096, lane);
       else
@@ -1023,9 +1167,20 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.err = err;
   p.wait_ns = a.wait_ns ? a.wait_ns : WAIT_LIMIT_NS;
   p.lost_load = a.lost_load && !pair_mma ? 1 : 0;
+  p.l2_pf = a.l2_pf > 0 ? a.l2_pf : 0;
+  if (a.epi == EPI_ACCUM && a.fix_ctr) {
+    // the fix-up needs whole heads per Q|K|V tile and the gate/up output
+    if (!swiglu_b && (bn % 128 != 0 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||
+                      a.N % 3 != 0))
+      return cudaErrorInvalidValue;
+    if (swiglu_b && !a.fix_act) return cudaErrorInvalidValue;
+    p.fixup = 1;
+    p.fix_ctr = a.fix_ctr;
+    p.fix_act = (bf16 *)a.fix_act;
+  }
   p.rope = a.rope;
   p.n_ctx = a.n_ctx;
-  p.dmodel = a.epi == EPI_QKV ? a.N / 3 : 0;
+  p.dmodel = (a.epi == EPI_QKV || (p.fixup && !swiglu_b)) ? a.N / 3 : 0;
   p.prev = (const bf16 *)a.prev;
   p.stat = a.stat;
   p.stat_idx = a.stat_idx;

@@ -180,6 +180,14 @@ struct TcGemmArgs {
   // and CTA 0 leaving out its first stage's operand copies (1-SM kernel only)
   unsigned long long wait_ns;
   int lost_load;
+  // ACCUM split-K tile fix-up (see accum_fixup in gemm_tc.cu): tickets
+  // [ceil(M / 32)][N / bn] zero between uses; QKV uses row_map, rope, n_ctx,
+  // q_out, ck, cv; gate/up writes SiLU(gate) * up to fix_act [M][N / 2]
+  unsigned int *fix_ctr;
+  void *fix_act;
+  // K-blocks of the first unit's weight tiles that follow the shared-memory
+  // ring, prefetched into L2 before waiting on the previous kernel (0 = none)
+  int l2_pf;
 };
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s);
 

@@ -92,15 +92,20 @@ __device__ __forceinline__ void stat_add8(Stat &st, const float *z, const float 
   // A -inf logit has probability 0 and adds nothing to s or t (0 log 0 = 0 in
   // the KL); while every logit seen so far is -inf, st.m is -inf too and the
   // exponent would be -inf - -inf, so that case is skipped outright.
+  // The group's terms are summed first and added to the running sums once, so
+  // a row's many small terms do not each round against a sum near 1.
   const bool live = st.m != -INFINITY;
+  float gs = 0.f, gt = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const float e = live ? __expf(z[i] - st.m) : 0.f;
-    st.s += e;
-    if (has_prev && e > 0.f) st.t = fmaf(e, z[i] - zp[i], st.t);
+    gs += e;
+    if (has_prev && e > 0.f) gt = fmaf(e, z[i] - zp[i], gt);
     int v = v0 + i;
     if (v != mask_id && z[i] > st.bv) { st.bv = z[i]; st.bi = v; }
   }
+  st.s += gs;
+  st.t += gt;
 }
 
 constexpr int LOCK_THREADS = 256;
