@@ -1,12 +1,18 @@
 #!/usr/bin/env python
 """Throughput of the SureLock decoding step on B200.
 
-Default workload: the LLaDA-8B shape (32 layers, d=4096, 32 heads x 128,
-SwiGLU 12288, vocab 126464), random-init bf16 weights, batch 1, 128 random
-prompt ids + 256 masked positions (N = 384), 256 denoising steps in
-semi-autoregressive blocks of 32, one token unmasked per step, KL threshold
-eps = 0.05.  One bench step = one complete decode (256 denoising steps: the
-denoiser on the active rows, the sure test, unmasking and compaction).
+Default workload (--workload long8b): the LLaDA-8B shape (32 layers, d=4096,
+32 heads x 128, SwiGLU 12288, vocab 126464), random-init bf16 weights, batch
+4, 1024 random prompt ids + 1024 masked positions per sequence (N = 2048), 512
+denoising steps in semi-autoregressive blocks of 64 positions, two tokens
+unmasked per step, KL threshold eps = 0.05 with the confidence gate at the
+0.5 quantile.  One bench step = one block of that decode (32 denoising steps:
+the denoiser on the active rows with the sure test's statistics in the LM
+head's epilogue, the lock decisions, unmasking and compaction); decodes run
+back to back and the timed region starts at the first step of a decode, so
+16 bench steps are exactly one decode.
+--workload full8b: batch 1, 128 prompt + 256 masked (N = 384), 256 steps in
+blocks of 32, one token per step, eps = 0.05; one bench step = one decode.
 
 Reported (one JSON line from rank 0):
   value      denoising steps/s over all ranks, inputs resident in HBM
@@ -112,7 +118,11 @@ def workload_config(args, setup: wl.SamplerSetup, world: int) -> dict:
                         + (", ablation: no KV cache (active rows' keys only)"
                            if setup.no_kv_cache else "")
                         + (", ablation: confidence gate only" if setup.gate_only else ""),
-            "bench_step": f"one full decode ({T} denoising steps)",
+            "bench_step": (f"one full decode ({T} denoising steps)"
+                           if bench_unit_steps(args, setup) == T else
+                           f"one semi-autoregressive block ({setup.steps_per_block} denoising "
+                           f"steps, 1/{setup.n_blocks} of a {T}-step decode); decodes run back "
+                           f"to back and the timed region starts at a decode's first step"),
             "global_batch": world * setup.batch, "seq_len": setup.n_ctx,
             "parallelism": f"replicas{world}",
             "l2": "inputs larger than L2 (15 GB of weights streamed per step)"}
@@ -332,6 +342,15 @@ class Ranks:
             self.dist = None
 
 
+def bench_unit_steps(args, setup: wl.SamplerSetup) -> int:
+    """Denoising steps per bench step: one semi-autoregressive block for the
+    long decode (512 steps, ~20 s), a whole decode otherwise."""
+    mode = getattr(args, "bench_step", "auto")
+    if mode == "auto":
+        mode = "block" if args.workload == "long8b" else "decode"
+    return setup.steps_per_block if mode == "block" else setup.steps
+
+
 def aux_decodes(k: int, decode_ms: float, budget_ms: float = 20000.0) -> int:
     """Decodes of each instrumented / end-to-end pass: about `budget_ms` of
     decoding, at least one, at most the timed count."""
@@ -380,8 +399,22 @@ def run_ours(args, rank: int, world: int):
         for _ in range(T):
             s.step()
 
+    # One bench step = `unit` denoising steps: a whole decode, or one
+    # semi-autoregressive block of it (decodes then run back to back).
+    unit = bench_unit_steps(args, setup)
+    cursor = [0]                 # next denoising step of the running decode
+
+    def run_unit():
+        for _ in range(unit):
+            if cursor[0] == 0:
+                s.start(d_prompts)
+            s.step()
+            cursor[0] = (cursor[0] + 1) % T
+
     for _ in range(args.warmup):
-        decode()
+        run_unit()
+    while cursor[0] != 0:        # untimed: the timed region starts with a decode
+        run_unit()
     torch.cuda.synchronize()
     clocks = ClockSampler(gpu_id_for(dev), os.path.join(args.out_dir, f"clocks_rank{rank}.csv")) \
         if rank == 0 else None
@@ -394,17 +427,19 @@ def run_ours(args, rank: int, world: int):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record()
     for _ in range(args.steps):
-        decode()
+        run_unit()
     ev1.record()
     torch.cuda.synchronize()
     ms_local = ev0.elapsed_time(ev1)
+    while cursor[0] != 0:        # finish the running decode (untimed)
+        run_unit()
     clk = clocks.stop() if clocks else None
     kernels_timed = model.timing_read(reset=True)["kernels"]
     barrier()
     ms = max_over_ranks(ms_local)
-    # the instrumented and end-to-end passes run `aux` decodes (about 20 s of
-    # decoding each, at most K): the timed region above is never shortened
-    aux = aux_decodes(args.steps, ms / args.steps)
+    # the instrumented and end-to-end passes run `aux` whole decodes (about 20 s
+    # of decoding each): the timed region above is never shortened
+    aux = aux_decodes(max(1, args.steps * unit // T), ms / args.steps * T / unit)
 
     # Per-kernel CUDA events around every GEMM / attention / lock launch.  An
     # event between two kernels also removes the programmatic-launch overlap at
@@ -457,16 +492,19 @@ def run_ours(args, rank: int, world: int):
     result = None
     if rank == 0:
         peaks = load_peaks()
-        value = aggregate_rate(world, args.steps * T, ms)
+        timed_steps = args.steps * unit
+        value = aggregate_rate(world, timed_steps, ms)
         e2e_value = aggregate_rate(world, aux * T, e2e_ms)
-        gen_tokens = world * args.steps * setup.batch * setup.gen_len
-        # per-step roofline over the trajectory, burst peaks
+        gen_tokens = world * timed_steps * setup.batch * setup.tokens_per_step
+        # per-step roofline over the timed steps' own M_t (the timed region
+        # starts at step 0 of a decode), burst peaks
         pf = peaks["bf16_tflops"] * 1e12
         pb = peaks["hbm_gbs"] * 1e9
-        roof = [max(fl / pf, by / pb) for fl, by in
-                (step_work(shape, int(m), setup.batch, setup.n_ctx) for m in traj)]
-        decode_ms = ms_local / args.steps
-        step_frac = (sum(roof) * 1e3) / decode_ms
+        roof_t = [max(fl / pf, by / pb) for fl, by in
+                  (step_work(shape, int(m), setup.batch, setup.n_ctx) for m in traj)]
+        roof = [roof_t[i % T] for i in range(timed_steps)]
+        decode_ms = ms_local / timed_steps * T
+        step_frac = (sum(roof) * 1e3) / ms_local
         flops_traj = sum(step_work(shape, int(m), setup.batch, setup.n_ctx)[0] for m in traj)
         flops_dense = T * step_work(shape, setup.batch * setup.n_ctx, setup.batch, setup.n_ctx)[0]
         # dominant kernel: the tensor-core GEMM
@@ -508,7 +546,8 @@ def run_ours(args, rank: int, world: int):
             "config": workload_config(args, setup, world),
             "gen_tok_s": round(gen_tokens / (ms / 1e3), 3),
             "e2e": {"value": round(e2e_value, 3), "unit": "denoise steps/s",
-                    "gen_tok_s": round(gen_tokens * aux / args.steps / (e2e_ms / 1e3), 3),
+                    "gen_tok_s": round(world * aux * setup.batch * setup.gen_len
+                                       / (e2e_ms / 1e3), 3),
                     "decodes": aux,
                     "h2d_bytes_per_step": int(prompts.nbytes),
                     "d2h_bytes_per_step": int(setup.batch * setup.n_ctx * 4)},
@@ -521,8 +560,9 @@ def run_ours(args, rank: int, world: int):
                          "measured_in": f"instrumented pass of {aux} more decode(s) "
                                         f"({ms_instr / aux:.1f} ms/decode with events)"},
             "step_roofline": {"frac": round(step_frac, 4), "roofline_ms_per_decode":
-                              round(sum(roof) * 1e3, 3), "measured_ms_per_decode":
-                              round(decode_ms, 3), "peaks": "burst (bf16_tflops, hbm_gbs)"},
+                              round(sum(roof_t) * 1e3, 3), "measured_ms_per_decode":
+                              round(decode_ms, 3), "timed_steps": timed_steps,
+                              "peaks": "burst (bf16_tflops, hbm_gbs)"},
             "algorithmic_flops_reduction": round(1.0 - flops_traj / flops_dense, 4),
             "kernel_time_ms": {k: round(tim[k]["ms"], 3) for k in ("gemm", "attn", "lock")},
             "curve": curve,
@@ -584,7 +624,12 @@ def main():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="full8b")
+    ap.add_argument("--workload", default="long8b",
+                    help="long8b: LLaDA-8B shape, batch 4, N = 2048, 512 steps (the default); "
+                         "full8b: batch 1, N = 384, 256 steps")
+    ap.add_argument("--bench-step", default="auto", choices=["auto", "decode", "block"],
+                    help="denoising steps per bench step: a whole decode, or one "
+                         "semi-autoregressive block (auto: block for long8b)")
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--scripted", action="store_true")
     ap.add_argument("--batch", type=int, default=None,

@@ -160,3 +160,25 @@ def test_trajectory_from_lock_steps():
     lock_t = np.array([-1, 0, 0, 2, -1, 1, 2, 2], dtype=np.int32)
     # all 8 rows active at step 0; 2 locked at step 0, 1 at step 1, 3 at step 2
     assert bench.trajectory_from_lock_t(lock_t, 4).tolist() == [8, 6, 5, 2]
+
+
+def test_bench_step_unit():
+    """The long decode's bench step is one semi-autoregressive block (16 per
+    decode), the short decode's a whole decode; --bench-step overrides."""
+    import types
+    sys.path.insert(0, ROOT)
+    import bench
+    long_ = bench.make_setup("long8b", None, False)
+    short = bench.make_setup("full8b", None, False)
+    a = types.SimpleNamespace(workload="long8b", bench_step="auto")
+    assert bench.bench_unit_steps(a, long_) == 32 == long_.steps // 16
+    assert "block" in bench.workload_config(a, long_, 1)["bench_step"]
+    a = types.SimpleNamespace(workload="full8b", bench_step="auto")
+    assert bench.bench_unit_steps(a, short) == 256
+    assert "full decode" in bench.workload_config(a, short, 1)["bench_step"]
+    a = types.SimpleNamespace(workload="long8b", bench_step="decode")
+    assert bench.bench_unit_steps(a, long_) == 512
+    # instrumented / end-to-end passes: about 20 s of decodes, at least one
+    assert bench.aux_decodes(20, 19600.0) == 1
+    assert bench.aux_decodes(20, 1250.0) == 16
+    assert bench.aux_decodes(2, 100.0) == 2

@@ -1,8 +1,8 @@
 """Attention of the active queries over every cached key (sl_attention, bf16
 path) against the oracle's attention in fp64, for both kernels: the tensor-core
-kernel (128 queries per CTA, tcgen05 + TMEM, TMA-fed K/V; the library's
-default) with its key range whole or split across CTAs (merged by per-row
-tickets), and the mma.sync kernel in each warp layout (16, 32 or 64 queries per
+kernel (tcgen05 + TMEM, TMA-fed K/V; the library's default) with one or two
+128-query tiles per CTA and its key range whole or split across CTAs (merged by
+per-row tickets), and the mma.sync kernel in each warp layout (16, 32 or 64 queries per
 CTA, the key tile shared by 4, 2 or 1 warps); ragged query counts (several
 128-query tiles, partial last tiles), empty sequences and key counts off the
 tile grids.  Every layout is pinned in turn (sl_model_set_attention) as well as
@@ -33,14 +33,15 @@ CASES = [
     ([0, 40, 0], 260),      # empty sequences
     ([300], 700),           # three 128-query tiles, the last one partial
     ([129, 128, 1], 384),   # tile boundaries one row either side
+    ([257, 384, 130], 640), # two-tile CTAs with a lone third tile, full pairs, one ragged
 ]
 
 
 # (queries per CTA, cross-CTA key split); 0 = the library's cost model.
-# 128 queries per CTA = the tensor-core kernel (the default), 16/32/64 the
-# mma.sync kernel.
-LAYOUTS = [(0, 0), (128, 1), (128, 2), (128, 3), (128, 16), (16, 1), (32, 1), (64, 1), (16, 4),
-           (32, 2), (64, 3)]
+# 128 or 256 queries per CTA = the tensor-core kernel (one or two 128-query
+# tiles sharing each K/V tile; the default), 16/32/64 the mma.sync kernel.
+LAYOUTS = [(0, 0), (128, 1), (128, 2), (128, 3), (128, 16), (256, 1), (256, 2), (256, 5),
+           (16, 1), (32, 1), (64, 1), (16, 4), (32, 2), (64, 3)]
 
 
 @pytest.mark.parametrize("layout", LAYOUTS)
@@ -104,7 +105,8 @@ NOKV_CASES = [
     # active rows only at the end of the range
     ([9, 20], 3000, "tail"),
 ]
-NOKV_LAYOUTS = [(0, 0), (128, 1), (128, 4), (16, 1), (32, 2), (64, 3), (16, 4)]
+NOKV_LAYOUTS = [(0, 0), (128, 1), (128, 4), (256, 1), (256, 3), (16, 1), (32, 2), (64, 3),
+                (16, 4)]
 
 
 def _positions(rng, counts, n_ctx, where):

@@ -131,6 +131,7 @@ struct sl_kv_cache {
   int attn_max_splits = 16;
   unsigned int *attn_tickets = nullptr;   // [max_rows][H] per-row split tickets, kept zero
   std::vector<TmaMat> k_maps, v_maps;     // per layer, 128-row boxes (tensor-core attention)
+  std::vector<TmaMat> k_maps64, v_maps64; // per layer, 64-row boxes (two query tiles per CTA)
   TmaMat map_q;                           // q workspace [M][d], 128-row boxes
   TmaMat map_qx{};                        // a caller's q (sl_attention), by pointer and M
   unsigned int *fix_ctr = nullptr;        // split-K fix-up tickets [max_rows/32 + 8][384]
@@ -421,9 +422,13 @@ extern "C" sl_status sl_kv_cache_create(const sl_model *m, int batch, int n_ctx,
          alloc((void **)&c->fix_ctr, fix_ctr_bytes(c->max_rows, cfg));
     c->k_maps.resize(cfg.n_layers);
     c->v_maps.resize(cfg.n_layers);
+    c->k_maps64.resize(cfg.n_layers);
+    c->v_maps64.resize(cfg.n_layers);
     for (int l = 0; l < cfg.n_layers && ok; ++l)
       ok = tma_encode(&c->k_maps[l], c->k[l], c->max_rows, d, 128) &&
-           tma_encode(&c->v_maps[l], c->v[l], c->max_rows, d, 128);
+           tma_encode(&c->v_maps[l], c->v[l], c->max_rows, d, 128) &&
+           tma_encode(&c->k_maps64[l], c->k[l], c->max_rows, d, 64) &&
+           tma_encode(&c->v_maps64[l], c->v[l], c->max_rows, d, 64);
   }
   if (ok) {
     // rotary table in double precision: angle = pos * theta^(-2i/dh)
@@ -907,11 +912,13 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
   Timed t(m, SL_K_ATTN, 2.0 * (2.0 * M * d + 2.0 * seqs.batch * c->n_ctx * d),
           4.0 * (double)M * c->n_ctx * d, s);
   // the output projection's weights follow; the attention leaves HBM idle
-  if (m->attn_q == 0 || m->attn_q == 128) {
-    SL_CUDA(launch_attn_tc(q_map, c->k_maps[l], c->v_maps[l], seqs, M, c->n_ctx, m->cfg.n_heads,
-                           o, c->attn_ws, c->attn_tickets, c->attn_max_splits, m->num_sms, m->err,
-                           g_wait_limit_ns.load(std::memory_order_relaxed), s, m->attn_splits,
-                           m->layers[l].wo, (size_t)d * d * 2, ks.stamp, ks.gen));
+  if (m->attn_q == 0 || m->attn_q >= 128) {
+    SL_CUDA(launch_attn_tc(q_map, c->k_maps[l], c->v_maps[l], c->k_maps64[l], c->v_maps64[l],
+                           seqs, M, c->n_ctx, m->cfg.n_heads, o, c->attn_ws, c->attn_tickets,
+                           c->attn_max_splits, m->num_sms, m->err,
+                           g_wait_limit_ns.load(std::memory_order_relaxed), s, m->attn_q,
+                           m->attn_splits, m->layers[l].wo, (size_t)d * d * 2, ks.stamp,
+                           ks.gen));
     return SL_OK;
   }
   SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
@@ -1472,10 +1479,10 @@ extern "C" sl_status sl_model_set_ablation(sl_model *m, int flags) {
 
 extern "C" sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits) {
   if (!m || (queries_per_cta != 0 && queries_per_cta != 16 && queries_per_cta != 32 &&
-             queries_per_cta != 64 && queries_per_cta != 128) ||
+             queries_per_cta != 64 && queries_per_cta != 128 && queries_per_cta != 256) ||
       splits < 0 || splits > 16)
     return fail(SL_ERR_INVALID,
-                "sl_model_set_attention: queries_per_cta 0/16/32/64/128, splits 0..16");
+                "sl_model_set_attention: queries_per_cta 0/16/32/64/128/256, splits 0..16");
   m->attn_q = queries_per_cta;
   m->attn_splits = splits;
   return SL_OK;

@@ -381,7 +381,7 @@ def main():
                     help="decode: profile --steps steps at each of these step indices")
     ap.add_argument("--n-ctx", default="384,2048", help="attn: key counts")
     ap.add_argument("--batch", type=int, default=1, help="attn: sequences")
-    ap.add_argument("--layouts", default="0:0,128:1,128:2,128:4,16:1,32:1,64:1,16:2,16:4,64:4",
+    ap.add_argument("--layouts", default="0:0,128:1,128:2,128:4,256:1,256:2,16:1,32:1,64:1,16:2,16:4,64:4",
                     help="attn: queries-per-CTA:splits list (0:0 = the library's choice)")
     ap.add_argument("--tuning-out", default=None, help="decode: save the autotuned GEMM tilings")
     ap.add_argument("--tuning-in", default=None,
