@@ -781,17 +781,6 @@ static sl_status layer_f32(sl_model *m, sl_kv_cache *c, sl_active *a, int l, flo
 static std::atomic<unsigned long long> g_wait_limit_ns{0};
 static std::atomic<int> g_lost_load{0};
 
-// K-blocks of weight tiles a GEMM prefetches into L2 while it waits for its
-// predecessor (SL_GEMM_L2_PREFETCH overrides the default; read once).
-static int gemm_l2_prefetch_kblocks() {
-  static int v = -1;
-  if (v < 0) {
-    const char *e = getenv("SL_GEMM_L2_PREFETCH");
-    v = e ? std::max(0, std::min(256, atoi(e))) : 0;
-  }
-  return v;
-}
-
 // Split-K tile fix-up in the GEMM epilogue instead of a finalize kernel
 // (SL_GEMM_FIXUP=0 turns it off; read once).
 static bool gemm_fixup_enabled() {
@@ -806,7 +795,6 @@ static bool gemm_fixup_enabled() {
 static cudaError_t launch_gemm_hooked(TcGemmArgs g, int num_sms, int *err, cudaStream_t s) {
   g.wait_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   g.lost_load = g_lost_load.exchange(0, std::memory_order_relaxed);
-  g.l2_pf = gemm_l2_prefetch_kblocks();
   return launch_gemm_tc(g, num_sms, err, s);
 }
 

@@ -159,8 +159,6 @@ struct TcParams {
   int fixup;               // ACCUM: the split-K tile fix-up (see accum_fixup)
   unsigned int *fix_ctr;   // [ceil(M / 32)][n_tiles] arrival tickets, zero between uses
   bf16 *fix_act;           // gate/up fix-up output [M][ffn]
-  int l2_pf;               // K-blocks of the first unit's weights prefetched into L2
-                           // beyond the ring while waiting on the previous kernel
   // QKV epilogue: rotary table [n_ctx][64] (cos, sin), q out [M][d], cache k/v
   const float2 *rope;
   int n_ctx, dmodel;
@@ -269,21 +267,6 @@ __device__ __forceinline__ void load_b(const TcParams &p, uint32_t sb, int nt, i
     if (c0 < p.seg0) tma_load_2d(sb, &p.b[0], kb * 64, c0, bar);
     else if (c0 < p.seg1) tma_load_2d(sb, &p.b[1], kb * 64, c0 - p.seg0, bar);
     else tma_load_2d(sb, &p.b[2], kb * 64, c0 - p.seg1, bar);
-  }
-}
-
-// L2 prefetch of the same B tile (no shared memory involved).
-template <int BN>
-__device__ __forceinline__ void prefetch_b(const TcParams &p, int nt, int kb) {
-  if (p.b_swiglu) {
-    const int f0 = nt * (BN / 2);
-    tma_prefetch_l2_2d(&p.b[0], kb * 64, f0);
-    tma_prefetch_l2_2d(&p.b[1], kb * 64, f0);
-  } else {
-    const int c0 = nt * BN;
-    if (c0 < p.seg0) tma_prefetch_l2_2d(&p.b[0], kb * 64, c0);
-    else if (c0 < p.seg1) tma_prefetch_l2_2d(&p.b[1], kb * 64, c0 - p.seg0);
-    else tma_prefetch_l2_2d(&p.b[2], kb * 64, c0 - p.seg1);
   }
 }
 
@@ -689,10 +672,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
           mbar_expect_tx(full_bar(i), L::STAGE_BYTES);
           load_b<BN>(p, sb, nt, kb0 + i, full_bar(i));
         }
-        // while the previous kernel drains, keep HBM busy with the weight
-        // tiles that follow the ring: they wait in L2 for the main loop
-        const int npf = min(p.l2_pf, kb1 - kb0 - npre);
-        for (int i = 0; i < npf; ++i) prefetch_b<BN>(p, nt, kb0 + npre + i);
       }
       pdl_wait();
       int stage = 0;
@@ -913,18 +892,6 @@ __global__ void __launch_bounds__(192, 1) gemm_tc2_kernel(const __grid_constant_
         for (int i = 0; i < npre; ++i) {
           if (leader) mbar_expect_tx(full_bar(i), 2 * STAGE_BYTES);
           load_b_half(sbase + i * STAGE_BYTES + A_BYTES, nt, kb0 + i, map_to_rank(full_bar(i), 0));
-        }
-        const int npf = min(p.l2_pf, kb1 - kb0 - npre);
-        for (int i = 0; i < npf; ++i) {
-          const int kb = kb0 + npre + i;
-          if (p.b_swiglu) {
-            tma_prefetch_l2_2d(&p.b[rank], kb * 64, nt * (BN / 2));
-          } else {
-            const int c0 = nt * BN + (int)rank * (BN / 2);
-            if (c0 < p.seg0) tma_prefetch_l2_2d(&p.b[0], kb * 64, c0);
-            else if (c0 < p.seg1) tma_prefetch_l2_2d(&p.b[1], kb * 64, c0 - p.seg0);
-            else tma_prefetch_l2_2d(&p.b[2], kb * 64, c0 - p.seg1);
-          }
         }
       }
       pdl_wait();
@@ -1167,7 +1134,6 @@ cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStrea
   p.err = err;
   p.wait_ns = a.wait_ns ? a.wait_ns : WAIT_LIMIT_NS;
   p.lost_load = a.lost_load && !pair_mma ? 1 : 0;
-  p.l2_pf = a.l2_pf > 0 ? a.l2_pf : 0;
   if (a.epi == EPI_ACCUM && a.fix_ctr) {
     // the fix-up needs whole heads per Q|K|V tile and the gate/up output
     if (!swiglu_b && (bn % 128 != 0 || !a.row_map || !a.rope || !a.q_out || !a.ck || !a.cv ||

@@ -192,9 +192,6 @@ struct TcGemmArgs {
   // q_out, ck, cv; gate/up writes SiLU(gate) * up to fix_act [M][N / 2]
   unsigned int *fix_ctr;
   void *fix_act;
-  // K-blocks of the first unit's weight tiles that follow the shared-memory
-  // ring, prefetched into L2 before waiting on the previous kernel (0 = none)
-  int l2_pf;
 };
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s);
 
