@@ -8,8 +8,11 @@
 // CTA pair needs tiles of at least 128 columns; the LM head writes logits rows
 // and takes no K split; stream-K runs only where partial sums can be added.
 // This program sweeps model shapes, row counts and SM counts and checks that
-// every plan the planner returns satisfies them.  It includes the runtime's
-// source so that it sees the planner as the library compiles it.
+// every plan the planner returns satisfies them, and does the same for the
+// layout and key split the tensor-core attention plans (a plan must exist for
+// any launch with queries, and every split must hold key tiles).  It includes
+// the runtime's source so that it sees the planners as the library compiles
+// them.
 #include "api.cu"
 
 #include <cstdio>
@@ -92,6 +95,53 @@ int main() {
         for (int kind = 0; kind < G_KINDS; ++kind) check_plan(sh, kind, M, ns, plan_kind(&m, kind, M, ns));
       }
     }
+  }
+  // the tensor-core attention's layout and key split: a plan exists whenever
+  // some sequence has queries; one or two query tiles per CTA as pinned; every
+  // split holds at least one key tile and together they cover all of them
+  {
+    const int counts_set[][4] = {{1, 0, 0, 0}, {5, 0, 0, 0}, {128, 1, 0, 0}, {129, 128, 1, 0},
+                                 {300, 0, 0, 0}, {2048, 2048, 2048, 2048}, {0, 40, 0, 0},
+                                 {257, 384, 130, 7}};
+    const int nctx_set[] = {64, 130, 384, 640, 2048, 2500, 4000};
+    for (const auto &cs : counts_set)
+      for (int batch = 1; batch <= 4; ++batch)
+        for (int n_ctx : nctx_set)
+          for (int ns : sms)
+            for (int fq : {0, 128, 256})
+              for (int fs = 0; fs <= 17; ++fs) {
+                AttnSeqs seqs{};
+                seqs.batch = batch;
+                int tiles = 0, off = 0;
+                for (int b = 0; b < batch; ++b) {
+                  const int c = cs[b] > n_ctx ? n_ctx : cs[b];
+                  seqs.seq_start[b] = off;
+                  seqs.seq_count[b] = c;
+                  off += c;
+                  tiles += (c + 127) / 128;
+                }
+                const AttnTcPlan pl = attn_tc_plan(seqs, 32, n_ctx, ns, 16, fq, fs);
+                ++g_checked;
+#define ACTX "attn batch=%d n_ctx=%d sms=%d fq=%d fs=%d -> qt=%d splits=%d per=%d kt=%d units=%d",              batch, n_ctx, ns, fq, fs, pl.qt, pl.splits, pl.kt_per_split, pl.ktiles, pl.units
+                if (tiles == 0) {
+                  CHECK(pl.units == 0, ACTX);
+                  continue;
+                }
+                CHECK(pl.units > 0, ACTX);
+                if (pl.units <= 0) continue;
+                CHECK(pl.qt == 1 || pl.qt == 2, ACTX);
+                CHECK(fq == 0 || fq == 128 * pl.qt, ACTX);
+                const int bn = pl.qt == 2 ? 64 : 128;
+                CHECK(pl.ktiles == (n_ctx + bn - 1) / bn, ACTX);
+                CHECK(pl.splits >= 1 && pl.splits <= 16, ACTX);
+                CHECK(pl.kt_per_split * pl.splits >= pl.ktiles, ACTX);
+                CHECK(pl.kt_per_split * (pl.splits - 1) < pl.ktiles, ACTX);   // no empty split
+                int units = 0;
+                for (int b = 0; b < batch; ++b)
+                  units += ((seqs.seq_count[b] + 127) / 128 + pl.qt - 1) / pl.qt;
+                CHECK(units == pl.units, ACTX);
+#undef ACTX
+              }
   }
   // row-count buckets of the autotuner: every M maps to the smallest bound >= M
   for (int M = 1; M <= 131072; M = M < 512 ? M + 1 : M + 97) {

@@ -3,9 +3,10 @@ epilogue of the LM-head GEMM stores the bf16 logits and takes per-tile
 statistics of the stored values; a per-row merge writes lse, D, u, conf and
 argmax.  Checked against
 
-* sl_step on the same state: the stored logits are the same bits;
-* sl_kl_lock (a separate pass over the stored logits): same argmax, and lse,
-  D, u, conf within fp32 summation-order rounding;
+* sl_kl_lock, the separate pass, over the same stored logits: same argmax,
+  and lse, D, u, conf within fp32 summation-order rounding;
+* sl_step on the same state: the same logits up to the order in which split-K
+  partial sums are added;
 * the oracle's log_softmax / kl_rows / uncertainty / prediction on the stored
   logits (fp64): argmax exact, the rest within the lock-test tolerances;
 * sl_lock_decide on the fused statistics: the same lock flags as sl_kl_lock;
@@ -57,14 +58,16 @@ def _run(model, shape, cache, act, tokens, dev, has_prev, eps=0.05, gate_q=0.5, 
                   f["argmax"], has_prev=has_prev)
     lock_f = torch.zeros(R, device=dev, dtype=torch.uint8)
     rt.lock_decide(act, masked, f["kl"], f["unc"], lock_f, eps, gate_q, has_prev)
-    # unfused: sl_step, then the separate statistics pass and decisions
-    z_u = torch.zeros_like(z_f)
-    rt.step(model, cache, act, tokens, z_u)
+    # the separate statistics pass and decisions over the same stored logits
     u = {k: torch.zeros(R, device=dev) for k in ("lse", "kl", "unc", "conf")}
     u["argmax"] = torch.zeros(R, device=dev, dtype=torch.int32)
     lock_u = torch.zeros(R, device=dev, dtype=torch.uint8)
-    rt.kl_lock(act, V, shape.mask_id, z_u, prev, lse_prev, u["lse"], masked, u["kl"], u["unc"],
+    rt.kl_lock(act, V, shape.mask_id, z_f, prev, lse_prev, u["lse"], masked, u["kl"], u["unc"],
                u["conf"], u["argmax"], lock_u, eps=eps, gate_q=gate_q, has_prev=has_prev)
+    # and sl_step on the same state: the same logits (split-K GEMMs may add their
+    # partial sums in another order, so within bf16 rounding rather than bitwise)
+    z_u = torch.zeros_like(z_f)
+    rt.step(model, cache, act, tokens, z_u)
     torch.cuda.synchronize()
     rt.device_check()
     return z_f, f, lock_f, z_u, u, lock_u, prev, masked
@@ -73,7 +76,8 @@ def _run(model, shape, cache, act, tokens, dev, has_prev, eps=0.05, gate_q=0.5, 
 def _compare(shape, act, z_f, f, lock_f, z_u, u, lock_u, prev, has_prev, n_oracle_rows=12):
     rows = np.concatenate([p + b * act.n_ctx for b, p in enumerate(act.positions())])
     M = len(rows)
-    assert torch.equal(z_f[rows], z_u[rows]), "fused and unfused logits differ"
+    zd = (z_f[rows].float() - z_u[rows].float()).abs().max().item()
+    assert zd <= 2e-2, f"sl_step_stats and sl_step logits differ by {zd}"
     F = {k: v.cpu().numpy() for k, v in f.items()}
     U = {k: v.cpu().numpy() for k, v in u.items()}
     np.testing.assert_array_equal(F["argmax"][:M], U["argmax"][:M])

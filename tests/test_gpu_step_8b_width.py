@@ -8,11 +8,15 @@ all M active rows, writes layer 2's fresh k, v of all M rows into its copy of
 the cache (two projections per row), and finishes layer 2, the final norm and
 the LM head on 16 sampled rows.  The oracle computes in fp32 on the device's
 bf16 weights (an 8B-width layer in fp64 would take minutes on the host)."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
 
 import workloads as wl
+from parity_util import LOGIT_TOL
 from oracle import model as om
 from token_locking_b200 import runtime as rt
 
@@ -82,9 +86,14 @@ def test_step_8b_width_full_vocab(step8, cuda_dev, M):
     z_gpu = logits.float().cpu().numpy()[pos[S]]
     err = np.abs(z_gpu - z_ref).max()
     print(f"M={M}: logits max err {err:.4g} (|z| max {np.abs(z_ref).max():.3g})")
+    path = os.environ.get("SL_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"test": "width8b-2layers", "M": M, "logits_max_abs_err": float(err),
+                                "z_max_abs": float(np.abs(z_ref).max())}) + "\n")
     # bf16 activations, GEMM outputs and logits around fp32 residuals over two
-    # 8B-width layers: a few 1e-2 expected; 5% of the largest logit as the bound
-    assert err <= 5e-2 * max(1.0, np.abs(z_ref).max()), f"M={M}: logits max err {err}"
+    # 8B-width layers: the stated bf16 bound, max abs 5e-2
+    assert err <= LOGIT_TOL["bf16"], f"M={M}: logits max err {err}"
     frozen = np.ones(N_CTX, dtype=bool)
     frozen[pos] = False
     for l in range(2):

@@ -520,10 +520,13 @@ AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sm
     const double fill = (double)tiles / ((double)units * qt);   // query tiles present per slot
     const double c_unit = qt == 2 ? 0.42 : 0.6;                 // us per 128 x 128 of work
     const int max_sp = std::min(ktiles, std::min(max_splits, 16));
-    for (int sp = 1; sp <= max_sp; ++sp) {
-      const int per = (ktiles + sp - 1) / sp;
-      if ((ktiles + per - 1) / per != sp) continue;
-      if (force_splits && sp != std::min(force_splits, max_sp)) continue;
+    for (int req = 1; req <= max_sp; ++req) {
+      // a requested split rounds to the count that covers the key tiles evenly
+      // (no empty split); a pinned request is taken as that count
+      if (force_splits && req != std::min(force_splits, max_sp)) continue;
+      const int per = (ktiles + req - 1) / req;
+      const int sp = (ktiles + per - 1) / per;
+      if (!force_splits && sp != req) continue;
       const long ctas = (long)units * n_heads * sp;
       const long waves = (ctas + num_sms - 1) / num_sms;
       const double work = (double)per * bn / 128.0 * qt * fill;
@@ -553,10 +556,13 @@ cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map128, const Tm
                            int force_splits, const void *pf, size_t pf_bytes,
                            const int32_t *stamp, int gen) {
   if (M <= 0) return cudaSuccess;
+  if (force_q != 0 && force_q != 128 && force_q != 256) return cudaErrorInvalidValue;
+  int q_tiles = 0;
+  for (int b = 0; b < seqs.batch; ++b) q_tiles += (seqs.seq_count[b] + TA_BM - 1) / TA_BM;
+  if (q_tiles == 0) return cudaSuccess;
   const AttnTcPlan pl = attn_tc_plan(seqs, n_heads, n_ctx, num_sms, max_splits, force_q,
                                      force_splits);
-  if (pl.units == 0) return force_q && force_q != 128 && force_q != 256 ? cudaErrorInvalidValue
-                                                                         : cudaSuccess;
+  if (pl.units == 0) return cudaErrorInvalidConfiguration;     // never silently skip work
   TaParams p;
   memset(&p, 0, sizeof(p));
   p.q_map = q_map.map;

@@ -13,8 +13,9 @@ captures).
       (row max + 8) on a random half of the rows, previous logits perturbed by
       N(0,0.05); KL test eps in {0.01, 0.05} with the 0.5-quantile confidence
       gate, then compaction.
-  python -m token_locking_b200.microbench decode [--steps S]
-      The first S denoising steps of the LLaDA-8B-shaped decode (N=384).
+  python -m token_locking_b200.microbench decode [--steps S] [--skip T] [--workload W]
+      S denoising steps (after T untimed ones) of the LLaDA-8B-shaped decode:
+      batch 1, N=384 (full8b, the default) or batch 4, N=2048 (long8b).
   python -m token_locking_b200.microbench gemm [--m 8,64,...]
       Sweep of the tensor-core GEMM tilings (tile width, 128/256-row tiles,
       K splits) on the LLaDA-8B projection shapes; one JSON line per tiling.
@@ -180,13 +181,13 @@ def bench_lock(args, dev):
 
 
 def bench_decode(args, dev):
-    setup = wl.cfg_full8b(eps=0.05)
+    setup = wl.cfg_long8b() if args.workload == "long8b" else wl.cfg_full8b(eps=0.05)
     shape = setup.shape
     w = wl.torch_weights(shape, dev)
     model = rt.Model(shape, w, "bf16")
-    s = rt.Sampler(model, 1, setup.prompt_len, setup.gen_len, setup.steps, setup.block_len,
-                   setup.tokens_per_step, setup.eps)
-    max_rows = setup.prompt_len + setup.gen_len
+    s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, setup.steps,
+                   setup.block_len, setup.tokens_per_step, setup.eps, setup.gate_q)
+    max_rows = setup.batch * (setup.prompt_len + setup.gen_len)
     if args.tuning_in:
         for kind, M, bn, sp, var in json.load(open(args.tuning_in)):
             model.set_tuning(kind, M, bn, sp, var)
@@ -195,7 +196,8 @@ def bench_decode(args, dev):
     if args.tuning_out:
         json.dump([[kind, M, *model.tuning(kind, M)] for kind in range(5)
                    for M in range(1, max_rows + 1)], open(args.tuning_out, "w"))
-    prompts = torch.from_numpy(wl.np_prompts(1, setup.prompt_len, shape.vocab, shape.mask_id)).to(dev)
+    prompts = torch.from_numpy(wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab,
+                                             shape.mask_id)).to(dev)
     s.start(prompts)
     if args.windows:
         # profiled windows of --steps steps starting at the given step indices;
@@ -381,6 +383,8 @@ def main():
                     help="decode: profile --steps steps at each of these step indices")
     ap.add_argument("--n-ctx", default="384,2048", help="attn: key counts")
     ap.add_argument("--batch", type=int, default=1, help="attn: sequences")
+    ap.add_argument("--workload", default="full8b", choices=["full8b", "long8b"],
+                    help="decode: batch 1 x 384 positions, or batch 4 x 2048")
     ap.add_argument("--layouts", default="0:0,128:1,128:2,128:4,256:1,256:2,16:1,32:1,64:1,16:2,16:4,64:4",
                     help="attn: queries-per-CTA:splits list (0:0 = the library's choice)")
     ap.add_argument("--tuning-out", default=None, help="decode: save the autotuned GEMM tilings")
