@@ -512,11 +512,20 @@ def run_ours(args, rank: int, world: int):
         t_f = g["flops"] / pf
         t_b = g["bytes"] / pb
         traffic = gemm_traffic()
+        # the GEMM is timed inside a long decode: a tensor-bound kernel runs at
+        # the power-capped clock, so its peak is the sustained bf16 figure
         if t_b >= t_f:
             bound, ach, peak, unit = "hbm", g["bytes"] / (g["ms"] / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
+            peak_kind = "HBM copy"
         else:
             bound, ach, peak, unit = ("tensor", g["flops"] / (g["ms"] / 1e3) / 1e12,
-                                      peaks["bf16_tflops"], "TFLOP/s")
+                                      peaks["bf16_tflops_sustained"], "TFLOP/s")
+            peak_kind = "bf16 sustained (kernel timed inside the decode)"
+        pfs = peaks["bf16_tflops_sustained"] * 1e12
+        roof_s = [max(fl / pfs, by / pb) for fl, by in
+                  (step_work(shape, int(traj[i % T]), setup.batch, setup.n_ctx)
+                   for i in range(timed_steps))]
+        step_frac_sustained = (sum(roof_s) * 1e3) / ms_local
         idx = list(range(0, T, 16)) + [T - 1]
         def roof_ms(m):
             fl, by = step_work(shape, int(m), setup.batch, setup.n_ctx)
@@ -556,13 +565,16 @@ def run_ours(args, rank: int, world: int):
                          "algorithmic_bytes_per_launch": round(g["bytes"] / max(1, g["launches"])),
                          "kernel": "gemm_tc_kernel (tcgen05)",
                          "launches": g["launches"], "kernel_ms": round(g["ms"], 3),
-                         "peak_source": peaks["source"],
+                         "peak_source": peaks["source"], "peak_kind": peak_kind,
                          "measured_in": f"instrumented pass of {aux} more decode(s) "
                                         f"({ms_instr / aux:.1f} ms/decode with events)"},
-            "step_roofline": {"frac": round(step_frac, 4), "roofline_ms_per_decode":
-                              round(sum(roof_t) * 1e3, 3), "measured_ms_per_decode":
-                              round(decode_ms, 3), "timed_steps": timed_steps,
-                              "peaks": "burst (bf16_tflops, hbm_gbs)"},
+            "step_roofline": {"frac": round(step_frac, 4),
+                              "frac_sustained": round(step_frac_sustained, 4),
+                              "roofline_ms_per_decode": round(sum(roof_t) * 1e3, 3),
+                              "measured_ms_per_decode": round(decode_ms, 3),
+                              "timed_steps": timed_steps,
+                              "peaks": "frac: burst (bf16_tflops, hbm_gbs); frac_sustained: "
+                                       "bf16_tflops_sustained, hbm_gbs"},
             "algorithmic_flops_reduction": round(1.0 - flops_traj / flops_dense, 4),
             "kernel_time_ms": {k: round(tim[k]["ms"], 3) for k in ("gemm", "attn", "lock")},
             "curve": curve,

@@ -430,9 +430,10 @@ sl_status sl_device_check(int clear);
  * fault: they only make a wait run out, after which the kernel records
  * SL_ERR_TIMEOUT in the device error word, drains its copies, frees its TMEM
  * and returns, and the context stays usable.
- *   sl_debug_set_wait_limit: every later tensor-core GEMM launch (sl_step,
- *     sl_layer_forward, sl_gemm_bf16, autotuning) gives up a barrier wait after
- *     `ns` nanoseconds instead of the default 2 s; 0 restores the default.
+ *   sl_debug_set_wait_limit: every later tensor-core GEMM and attention launch
+ *     (sl_step, sl_step_stats, sl_layer_forward, sl_attention, sl_gemm_bf16,
+ *     autotuning) gives up a barrier wait after `ns` nanoseconds instead of
+ *     the default 2 s; 0 restores the default.
  *     SL_ERR_INVALID outside [1 ms, 2 s].  Process-wide.
  *   sl_debug_inject_lost_load: the next tensor-core GEMM launch on the 1-SM
  *     kernels has its first CTA leave out the operand copies of its first
