@@ -15,12 +15,11 @@ configuration the bench times (autotuned GEMM tilings, the default attention):
   active row's fresh K/V, so the oracle's work scales with the sample).
 
 At each checked step: logits and log-probs within the bf16 tolerance of a
-32-layer model (max abs 5e-2 per two layers, growing as the square root of
-the depth because the layers' bf16 roundings are independent: 0.2; see
-parity_util.deep_logit_tol), the fresh K/V the step wrote within 3e-2
-relative, and the sure test, gate, unmasking and compaction decided by the
-oracle on the GPU's own logits equal to the GPU's outside the rounding bands.
-The observed errors are appended to the JSON-lines file named by
+whole step at this width (8 bf16 ulps of the largest logit, 0.25 for |z| in
+[4, 8); see parity_util.wide_logit_tol), the fresh K/V the step wrote within
+3e-2 relative, and the sure test, gate, unmasking and compaction decided by
+the oracle on the GPU's own logits equal to the GPU's outside the rounding
+bands.  The observed errors are appended to the JSON-lines file named by
 SL_PARITY_LOG when that variable is set.
 """
 import json
@@ -33,7 +32,7 @@ import torch
 
 import parity_8b as p8
 import workloads as wl
-from parity_util import deep_logit_tol
+from parity_util import wide_logit_tol
 from token_locking_b200 import runtime as rt
 
 pytestmark = pytest.mark.gpu
@@ -43,8 +42,6 @@ CHECK5_FULL = (255, 510, 511)
 CHECK5_SAMPLED = (1,)
 SAMPLE5 = 32
 KV_TOL = 3e-2
-# bf16 rounding noise of 32 layers adds in quadrature (parity_util.deep_logit_tol)
-DEEP_TOL = deep_logit_tol(wl.LLADA8B.n_layers)
 
 
 @pytest.fixture(scope="module")
@@ -128,9 +125,10 @@ def _decode(llada8b, dev, setup, full_steps, sampled_steps, name):
             _log({"test": name, "t": t, "b": b, "M": m, "rows_checked": n_rows,
                   "logits_max_abs_err": zerr, "logp_max_abs_err": lperr, "kv_max_rel_err": kv,
                   "z_max_abs": float(np.abs(z).max()), "oracle_s": round(time.time() - t0, 1)})
-            assert zerr <= DEEP_TOL, f"{name} t={t} b={b}: logits err {zerr}"
+            tol = wide_logit_tol(float(np.abs(z).max()))
+            assert zerr <= tol, f"{name} t={t} b={b}: logits err {zerr} > {tol}"
             assert kv <= KV_TOL, f"{name} t={t} b={b}: fresh K/V rel err {kv}"
-            assert lperr <= DEEP_TOL, f"{name} t={t} b={b}: log-prob err {lperr}"
+            assert lperr <= tol, f"{name} t={t} b={b}: log-prob err {lperr} > {tol}"
             p8.check_decisions(setup, t, b, A, snap, g, j0, stats)
             j0 += m            # per-row outputs run over all sequences in order
     final = s.state()

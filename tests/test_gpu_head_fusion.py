@@ -77,7 +77,7 @@ def _compare(shape, act, z_f, f, lock_f, z_u, u, lock_u, prev, has_prev, n_oracl
     rows = np.concatenate([p + b * act.n_ctx for b, p in enumerate(act.positions())])
     M = len(rows)
     zd = (z_f[rows].float() - z_u[rows].float()).abs().max().item()
-    assert zd <= 2e-2, f"sl_step_stats and sl_step logits differ by {zd}"
+    assert zd <= 5e-2, f"sl_step_stats and sl_step logits differ by {zd}"
     F = {k: v.cpu().numpy() for k, v in f.items()}
     U = {k: v.cpu().numpy() for k, v in u.items()}
     np.testing.assert_array_equal(F["argmax"][:M], U["argmax"][:M])
