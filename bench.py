@@ -128,17 +128,21 @@ def workload_config(args, setup: wl.SamplerSetup, world: int) -> dict:
             "l2": "inputs larger than L2 (15 GB of weights streamed per step)"}
 
 
-def gemm_traffic():
-    """DRAM bytes per GEMM launch from the committed ncu capture, or None when
-    the kernel source changed since the counters were taken."""
+def gemm_traffic(alg_bytes_per_launch: float):
+    """DRAM bytes per GEMM launch of this run: the committed ncu capture's ratio
+    of measured DRAM bytes (read + write) to the library's algorithmic bytes
+    over the same launches, applied to this run's algorithmic bytes per launch
+    (the GEMM's traffic grows with the units it processes); None when the
+    kernel source changed since the counters were taken."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")) as f:
             rec = json.load(f)
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-                return None
-        return float(rec["dram_bytes_per_launch"])
+        for src, sha in rec["sources"].items():
+            with open(os.path.join(ROOT, src), "rb") as f:
+                if hashlib.sha256(f.read()).hexdigest() != sha:
+                    return None
+        return float(rec["dram_bytes"]) / float(rec["algorithmic_bytes"]) * alg_bytes_per_launch
     except Exception:
         return None
 
@@ -511,7 +515,7 @@ def run_ours(args, rank: int, world: int):
         g = tim["gemm"]
         t_f = g["flops"] / pf
         t_b = g["bytes"] / pb
-        traffic = gemm_traffic()
+        traffic = gemm_traffic(g["bytes"] / max(1, g["launches"]))
         # the GEMM is timed inside a long decode: a tensor-bound kernel runs at
         # the power-capped clock, so its peak is the sustained bf16 figure
         if t_b >= t_f:
@@ -561,7 +565,8 @@ def run_ours(args, rank: int, world: int):
                     "h2d_bytes_per_step": int(prompts.nbytes),
                     "d2h_bytes_per_step": int(setup.batch * setup.n_ctx * 4)},
             "roofline": {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": unit,
-                         "frac": round(ach / peak, 4), "traffic": traffic,
+                         "frac": round(ach / peak, 4),
+                         "traffic": round(traffic) if traffic else None,
                          "algorithmic_bytes_per_launch": round(g["bytes"] / max(1, g["launches"])),
                          "kernel": "gemm_tc_kernel (tcgen05)",
                          "launches": g["launches"], "kernel_ms": round(g["ms"], 3),
