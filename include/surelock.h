@@ -317,11 +317,18 @@ sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows, void *str
  * sl_gemm_bf16. */
 sl_status sl_model_tuning(const sl_model *m, int kind, int M, int *bn, int *splits, int *variant);
 /* Pin the attention layout of sl_step / sl_attention on this model:
- * queries_per_cta 16, 32 or 64 (the four warps of a CTA then split every
- * 64-key tile 4, 2 or 1 ways) and the split of the key range across CTAs
- * (1..16, capped so every split keeps >= 4 tiles); 0 leaves either to the
- * library's cost model.  SL_ERR_INVALID for other values. */
+ * queries_per_cta 128 or 256 (the tensor-core kernel with one or two 128-query
+ * tiles per CTA), or 16, 32 or 64 (the mma.sync kernel; its four warps then
+ * split every 64-key tile 4, 2 or 1 ways), and the split of the key range
+ * across CTAs (1..16, rounded so that every split holds key tiles); 0 leaves
+ * either to the library's cost model (the tensor-core kernel).
+ * SL_ERR_INVALID for other values. */
 sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, int splits);
+/* Pin the key tile of the tensor-core attention (queries_per_cta 0, 128 or
+ * 256): 64 or 128 keys per tile (128 with one query tile per CTA only; a pin
+ * that no layout satisfies makes the step fail with SL_ERR_CUDA), 0 = cost
+ * model.  SL_ERR_INVALID for other values. */
+sl_status sl_model_set_attention_keys(sl_model *m, int key_tile);
 /* Pin the tiling of GEMM `kind` for the row-count bucket that holds M (the
  * buckets of sl_model_autotune); arguments as for sl_gemm_bf16.  Returns
  * SL_ERR_INVALID for a tiling the GEMM cannot use (the LM head takes no K

@@ -109,6 +109,7 @@ int main() {
         for (int n_ctx : nctx_set)
           for (int ns : sms)
             for (int fq : {0, 128, 256})
+              for (int fb : {0, 64, 128})
               for (int fs = 0; fs <= 17; ++fs) {
                 AttnSeqs seqs{};
                 seqs.batch = batch;
@@ -120,9 +121,13 @@ int main() {
                   off += c;
                   tiles += (c + 127) / 128;
                 }
-                const AttnTcPlan pl = attn_tc_plan(seqs, 32, n_ctx, ns, 16, fq, fs);
+                const AttnTcPlan pl = attn_tc_plan(seqs, 32, n_ctx, ns, 16, fq, fs, fb);
                 ++g_checked;
-#define ACTX "attn batch=%d n_ctx=%d sms=%d fq=%d fs=%d -> qt=%d splits=%d per=%d kt=%d units=%d",              batch, n_ctx, ns, fq, fs, pl.qt, pl.splits, pl.kt_per_split, pl.ktiles, pl.units
+#define ACTX "attn batch=%d n_ctx=%d sms=%d fq=%d fb=%d fs=%d -> qt=%d bn=%d splits=%d per=%d kt=%d units=%d",              batch, n_ctx, ns, fq, fb, fs, pl.qt, pl.bn, pl.splits, pl.kt_per_split, pl.ktiles, pl.units
+                if (fq == 256 && fb == 128) {          // no such layout: no plan
+                  CHECK(pl.units == 0, ACTX);
+                  continue;
+                }
                 if (tiles == 0) {
                   CHECK(pl.units == 0, ACTX);
                   continue;
@@ -131,8 +136,9 @@ int main() {
                 if (pl.units <= 0) continue;
                 CHECK(pl.qt == 1 || pl.qt == 2, ACTX);
                 CHECK(fq == 0 || fq == 128 * pl.qt, ACTX);
-                const int bn = pl.qt == 2 ? 64 : 128;
-                CHECK(pl.ktiles == (n_ctx + bn - 1) / bn, ACTX);
+                CHECK(fb == 0 || fb == pl.bn, ACTX);
+                CHECK(pl.bn == 64 || (pl.bn == 128 && pl.qt == 1), ACTX);
+                CHECK(pl.ktiles == (n_ctx + pl.bn - 1) / pl.bn, ACTX);
                 CHECK(pl.splits >= 1 && pl.splits <= 16, ACTX);
                 CHECK(pl.kt_per_split * pl.splits >= pl.ktiles, ACTX);
                 CHECK(pl.kt_per_split * (pl.splits - 1) < pl.ktiles, ACTX);   // no empty split

@@ -46,6 +46,32 @@ def wide_logit_tol(z_abs_max: float) -> float:
     several ulps of the largest logit (observed 2.0-2.7 ulps with two layers,
     3.5-6.4 with 32).  5e-2 is 1.6 ulps at |z| ~ 7."""
     return max(LOGIT_TOL["bf16"], WIDE_LOGIT_ULPS * bf16_ulp(z_abs_max))
+
+
+# bf16 ulps of the largest logit allowed after all 32 blocks (reading: bf16
+# tolerance through the full depth)
+DEEP_LOGIT_ULPS = 16
+
+
+def deep_logit_tol(z_abs_max: float) -> float:
+    """Logit (and log-prob) tolerance of a whole 32-block bf16 step against the
+    float32 oracle: DEEP_LOGIT_ULPS bf16 ulps of the largest logit (0.5 for |z|
+    in [4, 8)).  Every block, fed the oracle's own block input, differs from
+    the oracle's block by the same small amount whatever the step (rms 0.3 %
+    of the block's update, tested separately); what grows is the chained
+    difference, because the random-init network amplifies a block's rounding
+    through the blocks after it, and by how much depends on the tokens: from
+    1.6 % of the residual stream's rms after 32 blocks at the first step of a
+    batch-1 x 384 decode to 4.1 % at its step 254, for logit errors of 4.1 and
+    11 ulps."""
+    return max(LOGIT_TOL["bf16"], DEEP_LOGIT_ULPS * bf16_ulp(z_abs_max))
+
+
+# a block fed the oracle's block input: its output within this many bf16 ulps
+# of the largest entry of the block's update, and within this fraction of the
+# update's rms
+BLOCK_ULPS = 4
+BLOCK_RMS_FRAC = 0.02
 BAND_D = 1e-4
 BAND_U = 1e-4
 BAND_CONF_REL = 1e-5

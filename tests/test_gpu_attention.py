@@ -37,10 +37,12 @@ CASES = [
 ]
 
 
-# (queries per CTA, cross-CTA key split); 0 = the library's cost model.
-# 128 or 256 queries per CTA = the tensor-core kernel (one or two 128-query
-# tiles sharing each K/V tile; the default), 16/32/64 the mma.sync kernel.
-LAYOUTS = [(0, 0), (128, 1), (128, 2), (128, 3), (128, 16), (256, 1), (256, 2), (256, 5),
+# (queries per CTA, cross-CTA key split[, key tile]); 0 = the library's cost
+# model.  128 or 256 queries per CTA = the tensor-core kernel (one or two
+# 128-query tiles sharing each K/V tile; the default) with 64- or 128-key
+# tiles, 16/32/64 the mma.sync kernel.
+LAYOUTS = [(0, 0), (128, 1, 64), (128, 2, 64), (128, 16, 64), (128, 1, 128), (128, 3, 128),
+           (128, 16, 128), (256, 1), (256, 2), (256, 5),
            (16, 1), (32, 1), (64, 1), (16, 4), (32, 2), (64, 3)]
 
 
@@ -105,8 +107,8 @@ NOKV_CASES = [
     # active rows only at the end of the range
     ([9, 20], 3000, "tail"),
 ]
-NOKV_LAYOUTS = [(0, 0), (128, 1), (128, 4), (256, 1), (256, 3), (16, 1), (32, 2), (64, 3),
-                (16, 4)]
+NOKV_LAYOUTS = [(0, 0), (128, 1, 64), (128, 4, 64), (128, 1, 128), (128, 4, 128), (256, 1),
+                (256, 3), (16, 1), (32, 2), (64, 3), (16, 4)]
 
 
 def _positions(rng, counts, n_ctx, where):

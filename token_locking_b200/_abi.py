@@ -104,6 +104,7 @@ SIGNATURES = {
     "sl_model_tuning": (_I, [_P, _I, _I, C.POINTER(_I), C.POINTER(_I), C.POINTER(_I)]),
     "sl_model_set_tuning": (_I, [_P, _I, _I, _I, _I, _I]),
     "sl_model_set_attention": (_I, [_P, _I, _I]),
+    "sl_model_set_attention_keys": (_I, [_P, _I]),
     "sl_timing_enable": (_I, [_P, _I]),
     "sl_timing_read": (_I, [_P, C.POINTER(Timing), _I]),
     "sl_device_check": (_I, [_I]),

@@ -99,7 +99,7 @@ struct sl_model {
   const void *tok_emb, *final_norm, *lm_head;
   std::vector<sl_layer_weights> layers;
   std::vector<std::array<WMaps, W_COUNT>> maps;
-  int attn_q = 0, attn_splits = 0;   // pinned attention layout (0 = cost model)
+  int attn_q = 0, attn_splits = 0, attn_bn = 0;   // pinned attention layout (0 = cost model)
   bool head_fusion = true;           // samplers take the sure-test statistics from the
                                      // LM head's epilogue (bf16 models)
   int ablation = 0;                  // SL_ABLATE_* bits (0: the method itself)
@@ -905,8 +905,8 @@ static sl_status attn_bf16(sl_model *m, sl_kv_cache *c, const AttnSeqs &seqs, in
                            seqs, M, c->n_ctx, m->cfg.n_heads, o, c->attn_ws, c->attn_tickets,
                            c->attn_max_splits, m->num_sms, m->err,
                            g_wait_limit_ns.load(std::memory_order_relaxed), s, m->attn_q,
-                           m->attn_splits, m->layers[l].wo, (size_t)d * d * 2, ks.stamp,
-                           ks.gen));
+                           m->attn_splits, m->attn_bn, m->layers[l].wo, (size_t)d * d * 2,
+                           ks.stamp, ks.gen));
     return SL_OK;
   }
   SL_CUDA(launch_attn_bf16(q, c->k[l], c->v[l], seqs, M, c->n_ctx, m->cfg.n_heads, o,
@@ -1473,6 +1473,13 @@ extern "C" sl_status sl_model_set_attention(sl_model *m, int queries_per_cta, in
                 "sl_model_set_attention: queries_per_cta 0/16/32/64/128/256, splits 0..16");
   m->attn_q = queries_per_cta;
   m->attn_splits = splits;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_model_set_attention_keys(sl_model *m, int key_tile) {
+  if (!m || (key_tile != 0 && key_tile != 64 && key_tile != 128))
+    return fail(SL_ERR_INVALID, "sl_model_set_attention_keys: key_tile 0, 64 or 128");
+  m->attn_bn = key_tile;
   return SL_OK;
 }
 

@@ -25,11 +25,16 @@
 //               lazily (only when a tile's max exceeds it by more than 2^8,
 //               rescaling O in TMEM); the bf16 probabilities go to shared
 //               memory for the P V product.
-// Two query tiles per CTA (QT = 2, 64-key tiles) share every K/V tile, halving
-// the K/V traffic per multiply-add, and the two softmax warpgroups take turns
-// with the tensor cores: while one computes its exponentials the MMA warp
-// runs the other's products.  QT = 1 with 128-key tiles serves launches with
-// few query tiles.
+// Two query tiles per CTA (QT = 2) share every K/V tile, halving the K/V
+// traffic per multiply-add, and the two softmax warpgroups take turns with the
+// tensor cores: while one computes its exponentials the MMA warp runs the
+// other's products.  A K/V stage is released only when the P V product of its
+// tile has completed, so the copy of tile t + ST starts then and must land
+// before the scores of that tile can be issued: the ring has to be deep enough
+// to cover the TMA latency (about a microsecond) with the work of the tiles in
+// between.  Layouts: one query tile with 64-key tiles in a 5-deep ring or
+// 128-key tiles in a 2-deep ring, two query tiles with 64-key tiles in a
+// 4-deep ring; all fit the 227 KB of shared memory of a CTA.
 // A split key range leaves unnormalised partial rows and (max, sum) in a
 // workspace; the thread that completes a row's last split (atomic ticket per
 // row and head) merges them, so no second kernel is needed.
@@ -499,16 +504,24 @@ static cudaError_t run_attn_tc(const TaParams &p, dim3 grid, cudaStream_t s) {
 
 // Layout and key split of the tensor-core attention from a small cost model:
 // CTAs run in waves (one per SM, bound by shared memory); a CTA costs a fixed
-// set-up and drain plus a time per (128-query tile x 128 keys) of work, lower
-// for the two-tile CTA whose softmax warpgroups take turns with the tensor
-// cores; a split adds the merge.
+// set-up and drain plus a time per (128-query tile x 128 keys) of work that
+// depends on the layout; a split adds the merge.
+namespace {
+struct TaLayout {
+  int qt, bn;
+  double c_unit;   // us per 128 x 128 block of work at the power-capped clock
+};
+constexpr TaLayout kTaLayouts[] = {{1, 64, 1.4}, {1, 128, 2.0}, {2, 64, 1.4}};
+}  // namespace
+
 AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sms,
-                        int max_splits, int force_q, int force_splits) {
+                        int max_splits, int force_q, int force_splits, int force_bn) {
   AttnTcPlan best{};
   double best_t = 1e30;
-  for (int qt = 1; qt <= 2; ++qt) {
+  for (const TaLayout &ly : kTaLayouts) {
+    const int qt = ly.qt, bn = ly.bn;
     if (force_q && force_q != 128 * qt) continue;
-    const int bn = qt == 2 ? 64 : 128;
+    if (force_bn && force_bn != bn) continue;
     const int ktiles = (n_ctx + bn - 1) / bn;
     int units = 0, tiles = 0;
     for (int b = 0; b < seqs.batch; ++b) {
@@ -518,9 +531,6 @@ AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sm
     }
     if (units == 0) return best;
     const double fill = (double)tiles / ((double)units * qt);   // query tiles present per slot
-    // us per 128 x 128 of work: measured the same for both layouts (~2 us at
-    // the power-capped clock), so two-tile CTAs win only by packing waves
-    const double c_unit = 2.0;
     const int max_sp = std::min(ktiles, std::min(max_splits, 16));
     for (int req = 1; req <= max_sp; ++req) {
       // a requested split rounds to the count that covers the key tiles evenly
@@ -532,10 +542,11 @@ AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sm
       const long ctas = (long)units * n_heads * sp;
       const long waves = (ctas + num_sms - 1) / num_sms;
       const double work = (double)per * bn / 128.0 * qt * fill;
-      const double t = waves * (2.0 + c_unit * work) + (sp > 1 ? 3.0 : 0.0);
+      const double t = waves * (2.0 + ly.c_unit * work) + (sp > 1 ? 3.0 : 0.0);
       if (t < best_t * 0.97) {                 // a clear gain, else the earlier layout
         best_t = t;
         best.qt = qt;
+        best.bn = bn;
         best.splits = sp;
         best.kt_per_split = per;
         best.ktiles = ktiles;
@@ -555,21 +566,22 @@ cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map128, const Tm
                            int M, int n_ctx, int n_heads, void *o, float *ws,
                            unsigned int *tickets, int max_splits, int num_sms, int *err,
                            unsigned long long wait_ns, cudaStream_t s, int force_q,
-                           int force_splits, const void *pf, size_t pf_bytes,
+                           int force_splits, int force_bn, const void *pf, size_t pf_bytes,
                            const int32_t *stamp, int gen) {
   if (M <= 0) return cudaSuccess;
   if (force_q != 0 && force_q != 128 && force_q != 256) return cudaErrorInvalidValue;
+  if (force_bn != 0 && force_bn != 64 && force_bn != 128) return cudaErrorInvalidValue;
   int q_tiles = 0;
   for (int b = 0; b < seqs.batch; ++b) q_tiles += (seqs.seq_count[b] + TA_BM - 1) / TA_BM;
   if (q_tiles == 0) return cudaSuccess;
   const AttnTcPlan pl = attn_tc_plan(seqs, n_heads, n_ctx, num_sms, max_splits, force_q,
-                                     force_splits);
+                                     force_splits, force_bn);
   if (pl.units == 0) return cudaErrorInvalidConfiguration;     // never silently skip work
   TaParams p;
   memset(&p, 0, sizeof(p));
   p.q_map = q_map.map;
-  p.k_map = pl.qt == 2 ? k_map64.map : k_map128.map;
-  p.v_map = pl.qt == 2 ? v_map64.map : v_map128.map;
+  p.k_map = pl.bn == 64 ? k_map64.map : k_map128.map;
+  p.v_map = pl.bn == 64 ? v_map64.map : v_map128.map;
   p.o = (bf16 *)o;
   p.ws_o = ws;
   p.ws_ml = ws + (size_t)pl.splits * M * n_heads * TA_D;
@@ -589,7 +601,9 @@ cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map128, const Tm
   p.wait_ns = wait_ns ? wait_ns : WAIT_LIMIT_NS;
   const dim3 grid(pl.units, n_heads, pl.splits);
   if (pl.qt == 2)
-    return stamp ? run_attn_tc<2, 64, 3, true>(p, grid, s) : run_attn_tc<2, 64, 3, false>(p, grid, s);
+    return stamp ? run_attn_tc<2, 64, 4, true>(p, grid, s) : run_attn_tc<2, 64, 4, false>(p, grid, s);
+  if (pl.bn == 64)
+    return stamp ? run_attn_tc<1, 64, 5, true>(p, grid, s) : run_attn_tc<1, 64, 5, false>(p, grid, s);
   return stamp ? run_attn_tc<1, 128, 2, true>(p, grid, s) : run_attn_tc<1, 128, 2, false>(p, grid, s);
 }
 

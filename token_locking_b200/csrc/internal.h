@@ -125,25 +125,26 @@ cudaError_t launch_attn_bf16(const void *q, const void *ck, const void *cv, cons
 
 // ----------------------------------------------------------------- attn_tc.cu
 // Tensor-core attention (head_dim 128, bf16): q_map over q [M][d] with
-// 128-row boxes, the layer's cache k/v [B*n_ctx][d] with 128-row boxes (one
-// query tile per CTA, 128-key tiles) and 64-row boxes (two query tiles per
-// CTA, 64-key tiles); ws as for launch_attn_bf16; tickets [M][n_heads] zero
-// between calls.  force_q 128 or 256 pins one or two query tiles per CTA and
+// 128-row boxes, the layer's cache k/v [B*n_ctx][d] with 128-row boxes (for
+// 128-key tiles) and 64-row boxes (for 64-key tiles); ws as for
+// launch_attn_bf16; tickets [M][n_heads] zero
+// between calls.  force_q 128 or 256 pins one or two query tiles per CTA,
+// force_bn 64 or 128 the key tile (128 with one query tile only) and
 // force_splits >= 1 the key split (0 = cost model).
 struct TmaMat;
 struct AttnTcPlan {
-  int qt = 0, splits = 0, kt_per_split = 0, ktiles = 0, units = 0;
+  int qt = 0, bn = 0, splits = 0, kt_per_split = 0, ktiles = 0, units = 0;
 };
 AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sms,
-                        int max_splits, int force_q, int force_splits);
+                        int max_splits, int force_q, int force_splits, int force_bn = 0);
 size_t attn_tc_tickets_bytes(int max_rows, int n_heads);
 cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map128, const TmaMat &v_map128,
                            const TmaMat &k_map64, const TmaMat &v_map64, const AttnSeqs &seqs,
                            int M, int n_ctx, int n_heads, void *o, float *ws,
                            unsigned int *tickets, int max_splits, int num_sms, int *err,
                            unsigned long long wait_ns, cudaStream_t s, int force_q = 0,
-                           int force_splits = 0, const void *pf = nullptr, size_t pf_bytes = 0,
-                           const int32_t *stamp = nullptr, int gen = 0);
+                           int force_splits = 0, int force_bn = 0, const void *pf = nullptr,
+                           size_t pf_bytes = 0, const int32_t *stamp = nullptr, int gen = 0);
 
 // ----------------------------------------------------------------- gemm_tc.cu
 // A bf16 K-major operand in global memory with its TMA descriptor.

@@ -264,8 +264,10 @@ def bench_attn(args, dev):
                       for b in range(B)])
             q = torch.randn((B * M, d), device=dev, generator=g).to(torch.bfloat16)
             o = torch.empty((B * M, d), device=dev, dtype=torch.bfloat16)
-            for qpc, sp in args.attn_layouts:
-                model.set_attention(qpc, sp)
+            for lay in args.attn_layouts:
+                qpc, sp = lay[0], lay[1]
+                kt = lay[2] if len(lay) > 2 else 0
+                model.set_attention(qpc, sp, kt)
 
                 def fn():
                     rt.attention(model, cache, act, 0, q, o)
@@ -282,7 +284,7 @@ def bench_attn(args, dev):
                 us = e0.elapsed_time(e1) * 1e3 / args.iters
                 fl = 4.0 * B * M * n_ctx * d
                 print(json.dumps({"case": "attn", "batch": B, "M": M, "n_ctx": n_ctx,
-                                  "q_per_cta": qpc,
+                                  "q_per_cta": qpc, "key_tile": kt,
                                   "splits": sp, "us": round(us, 2),
                                   "TFLOPs": round(fl / us / 1e6, 1)}), flush=True)
         cache.close()
@@ -385,8 +387,9 @@ def main():
     ap.add_argument("--batch", type=int, default=1, help="attn: sequences")
     ap.add_argument("--workload", default="full8b", choices=["full8b", "long8b"],
                     help="decode: batch 1 x 384 positions, or batch 4 x 2048")
-    ap.add_argument("--layouts", default="0:0,128:1,128:2,128:4,256:1,256:2,16:1,32:1,64:1,16:2,16:4,64:4",
-                    help="attn: queries-per-CTA:splits list (0:0 = the library's choice)")
+    ap.add_argument("--layouts", default="0:0,128:1:64,128:1:128,128:2:64,128:4:64,256:1,256:2,"
+                    "16:1,32:1,64:1,16:2,16:4,64:4",
+                    help="attn: queries-per-CTA:splits[:key tile] list (0:0 = the library's choice)")
     ap.add_argument("--tuning-out", default=None, help="decode: save the autotuned GEMM tilings")
     ap.add_argument("--tuning-in", default=None,
                     help="decode: load GEMM tilings instead of autotuning (e.g. under a profiler)")

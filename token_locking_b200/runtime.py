@@ -108,10 +108,12 @@ class Model:
                                         C.byref(var)), "sl_model_tuning")
         return bn.value, sp.value, var.value
 
-    def set_attention(self, queries_per_cta: int = 0, splits: int = 0):
+    def set_attention(self, queries_per_cta: int = 0, splits: int = 0, key_tile: int = 0):
         """Pin the attention layout (0 = the library's cost model)."""
         A.check(A.lib().sl_model_set_attention(self.handle, queries_per_cta, splits),
                 "sl_model_set_attention")
+        A.check(A.lib().sl_model_set_attention_keys(self.handle, key_tile),
+                "sl_model_set_attention_keys")
 
     def set_ablation(self, no_kv_cache: bool = False, gate_only: bool = False):
         """Ablations of the method: attention without the locked rows' cached
