@@ -23,8 +23,12 @@
 //               i (its TMEM lane), so the row max and sum need no shuffles.
 //               Scores are scaled into base 2; the running max is raised
 //               lazily (only when a tile's max exceeds it by more than 2^8,
-//               rescaling O in TMEM); the bf16 probabilities go to shared
-//               memory for the P V product.
+//               rescaling O in TMEM); the bf16 probabilities go back to TMEM
+//               (one query tile per CTA: two P buffers, so the P V product of
+//               tile t runs while the exponentials of tile t + 1 are taken, and
+//               the product reads P from TMEM, sparing shared memory the P
+//               traffic) or to shared memory (two query tiles, which use all
+//               of TMEM for scores and outputs).
 // Two query tiles per CTA (QT = 2) share every K/V tile, halving the K/V
 // traffic per multiply-add, and the two softmax warpgroups take turns with the
 // tensor cores: while one computes its exponentials the MMA warp runs the
@@ -32,8 +36,8 @@
 // tile has completed, so the copy of tile t + ST starts then and must land
 // before the scores of that tile can be issued: the ring has to be deep enough
 // to cover the TMA latency (about a microsecond) with the work of the tiles in
-// between.  Layouts: one query tile with 64-key tiles in a 5-deep ring or
-// 128-key tiles in a 2-deep ring, two query tiles with 64-key tiles in a
+// between.  Layouts: one query tile with 64-key tiles in a 6-deep ring or
+// 128-key tiles in a 3-deep ring, two query tiles with 64-key tiles in a
 // 4-deep ring; all fit the 227 KB of shared memory of a CTA.
 // A split key range leaves unnormalised partial rows and (max, sum) in a
 // workspace; the thread that completes a row's last split (atomic ticket per
@@ -54,26 +58,29 @@ constexpr int TA_D = 128;                     // head dim
 constexpr int TA_HBOX = 128 * 128;            // [128 rows][64 bf16] swizzled box, bytes
 constexpr float TA_RESCALE = 8.f;             // raise the running max when exceeded by 2^8
 
-template <int QT, int BN, int ST>
+template <int QT, int BN, int ST, bool TP>
 struct TaCfg {
   static constexpr int KBOX = BN * 128;                  // [BN rows][64 dims] box of K or V
   static constexpr int STAGE = 4 * KBOX;                 // K box 0, K box 1, V box 0, V box 1
-  static constexpr int P_TILE = (BN / 64) * TA_HBOX;     // P of one query tile: [128][BN] bf16
+  // P of one query tile in shared memory ([128][BN] bf16), unless it lives in TMEM
+  static constexpr int P_TILE = TP ? 0 : (BN / 64) * TA_HBOX;
   static constexpr int Q_OFF = 0;                        // per query tile two dims boxes
   static constexpr int KV_OFF = QT * 2 * TA_HBOX;
   static constexpr int P_OFF = KV_OFF + ST * STAGE;
   static constexpr int BAR_OFF = P_OFF + QT * P_TILE;
   // barriers: Q, kv_full[ST], kv_empty[ST], per query tile (s_full[2],
-  // s_free[2], p_full, o_ready), drain
+  // s_free[2], p_full[2], pv_done[2]; index u = key tile & 1), drain
   static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + ST, B_TILE = 1 + 2 * ST;
-  static constexpr int B_DRAIN = B_TILE + 6 * QT, B_COUNT = B_DRAIN + 1;
+  static constexpr int B_DRAIN = B_TILE + 8 * QT, B_COUNT = B_DRAIN + 1;
   static constexpr int SMEM = BAR_OFF + 8 * B_COUNT + 16 + 1024;   // + slot/flag + alignment
   static constexpr int THREADS = 64 + 128 * QT;
   // TMEM: S buffers of tile j at j * 2 BN (+ BN for the second), O of tile j
-  // at O_COL + 128 j
+  // at O_COL + 128 j, and with TP the two bf16 P buffers of tile j (BN / 2
+  // columns each, two keys per column) at P_COL + (2 j + u) BN / 2
   static constexpr uint32_t O_COL = QT * 2 * BN;
+  static constexpr uint32_t P_COL = O_COL + QT * 128;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(O_COL + QT * 128 <= TMEM_COLS, "TMEM columns");
+  static_assert(P_COL + (TP ? QT * BN : 0) <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory of a CTA");
   static_assert(BN % 64 == 0 && BN <= 256, "key tile");
 };
@@ -119,17 +126,17 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float *s) {
   tmem_wait_ld();
 }
 
-template <int QT, int BN, int ST, bool MASK>
-__global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
+template <int QT, int BN, int ST, bool TP, bool MASK>
+__global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
     attn_tc_kernel(const __grid_constant__ TaParams p) {
-  using C = TaCfg<QT, BN, ST>;
+  using C = TaCfg<QT, BN, ST, TP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s_addr(smem);
   const uint32_t bar0 = sbase + C::BAR_OFF;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-  auto tbar = [&](int j, int k) { return bar0 + 8u * (uint32_t)(C::B_TILE + 6 * j + k); };
-  // per query tile: 0,1 s_full[u]; 2,3 s_free[u]; 4 p_full; 5 o_ready
+  auto tbar = [&](int j, int k) { return bar0 + 8u * (uint32_t)(C::B_TILE + 8 * j + k); };
+  // per query tile: 0,1 s_full[u]; 2,3 s_free[u]; 4,5 p_full[u]; 6,7 pv_done[u]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + 8 * C::B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -157,14 +164,13 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
       mbar_init(bar(C::B_KVF + s), 1);
       mbar_init(bar(C::B_KVE + s), 1);
     }
-    for (int j = 0; j < QT; ++j) {
-      mbar_init(tbar(j, 0), 1);
-      mbar_init(tbar(j, 1), 1);
-      mbar_init(tbar(j, 2), 4);              // the tile's four softmax warps
-      mbar_init(tbar(j, 3), 4);
-      mbar_init(tbar(j, 4), 4);
-      mbar_init(tbar(j, 5), 1);
-    }
+    for (int j = 0; j < QT; ++j)
+      for (int u = 0; u < 2; ++u) {
+        mbar_init(tbar(j, u), 1);            // MMA commit
+        mbar_init(tbar(j, 2 + u), 4);        // the tile's four softmax warps
+        mbar_init(tbar(j, 4 + u), 4);
+        mbar_init(tbar(j, 6 + u), 1);
+      }
     mbar_init(bar(C::B_DRAIN), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -242,14 +248,22 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t sv = sbase + C::KV_OFF + (t % ST) * C::STAGE + 2 * C::KBOX;
-        const uint32_t sp = sbase + C::P_OFF + j * C::P_TILE;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(sp + (kk >> 2) * TA_HBOX) + 2 * (kk & 3);
           const uint64_t bd = smem_desc_sw128_mn(sv + kk * 2048, C::KBOX, 1024);
-          tc_mma(tmem_base + C::O_COL + 128 * j, a, bd, id_o, (t > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          if constexpr (TP) {
+            // P of key tile t from its TMEM buffer: 16 keys = 8 columns per step
+            const uint32_t pa =
+                tmem_base + C::P_COL + (uint32_t)((2 * j + (t & 1)) * (BN / 2) + kk * 8);
+            tc_mma_ts(tmem_base + C::O_COL + 128 * j, pa, bd, id_o, acc);
+          } else {
+            const uint32_t sp = sbase + C::P_OFF + j * C::P_TILE;
+            const uint64_t a = smem_desc_sw128(sp + (kk >> 2) * TA_HBOX) + 2 * (kk & 3);
+            tc_mma(tmem_base + C::O_COL + 128 * j, a, bd, id_o, acc);
+          }
         }
-        tc_commit(tbar(j, 5));
+        tc_commit(tbar(j, 6 + (t & 1)));
       };
       bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, lim);
       if (ok && T > 0) ok = mbar_wait(bar(C::B_KVF), 0, abort_flag, lim);
@@ -277,7 +291,10 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
           if (!ok) break;
         }
         for (int j = 0; ok && j < nj; ++j) {
-          if (!mbar_wait(tbar(j, 4), (uint32_t)t & 1u, abort_flag, lim)) { ok = false; break; }
+          if (!mbar_wait(tbar(j, 4 + (t & 1)), (uint32_t)(t >> 1) & 1u, abort_flag, lim)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           issue_pv(t, j);
         }
@@ -315,50 +332,54 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(tbar(j, 2 + u));
         const int key0 = (kt0 + t) * BN;
-        // eight independent partial maxima (and sums below): a single running
-        // value would chain BN dependent instructions per row
+        // row max of the raw scores (the scale is positive) as eight independent
+        // partials: a single running value would chain BN dependent instructions
         float mx[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
         if (key0 + BN <= p.n_ctx && !MASK) {
 #pragma unroll
-          for (int i = 0; i < BN; ++i) {
-            s[i] *= sl2;
-            mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-          }
+          for (int i = 0; i < BN; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
         } else {
 #pragma unroll
           for (int i = 0; i < BN; ++i) {
             const int key = key0 + i;
             bool live = key < p.n_ctx;
             if constexpr (MASK) live = live && p.stamp[(size_t)b * p.n_ctx + key] == p.gen;
-            s[i] = live ? s[i] * sl2 : -INFINITY;
+            s[i] = live ? s[i] : -INFINITY;
             mx[i & 7] = fmaxf(mx[i & 7], s[i]);
           }
         }
-        const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mt = sl2 * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const float m_new = fmaxf(m, mt);
         const bool resc = t > 0 && m_new > m + TA_RESCALE;
         const float m_use = (t == 0 || resc) ? m_new : m;
         const float alpha = resc ? ((m == -INFINITY) ? 0.f : ex2_approx(m - m_new)) : 1.f;
         float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;   // all scores -inf: p = 0
+        // p = 2^(s log2(e) / sqrt(dh) - m): the scale and the shift in one FMA
 #pragma unroll
         for (int i = 0; i < BN; ++i) {
-          const float pv = ex2_approx(s[i] - m_sub);
+          const float pv = ex2_approx(fmaf(s[i], sl2, -m_sub));
           s[i] = pv;
           sm[i & 7] += pv;
         }
         const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
-        if (t > 0) {
-          // P V of the previous key tile done: P may be overwritten, O is current
-          if (!warp_wait(tbar(j, 5), (uint32_t)(t - 1) & 1u, abort_flag, lim)) {
+        // O must be current before a rescale, and the P buffer about to be
+        // written must have been read: with P in TMEM the buffer of tile t was
+        // last read by the P V product of tile t - 2; in shared memory there is
+        // one buffer, read by the product of tile t - 1
+        const bool any_resc = __any_sync(0xffffffffu, resc);
+        const int t_prev = (TP && !any_resc) ? t - 2 : t - 1;
+        if (t_prev >= 0) {
+          const int ub = t_prev & 1;
+          if (!warp_wait(tbar(j, 6 + ub), (uint32_t)(t_prev >> 1) & 1u, abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, resc)) {
+          if (any_resc) {
 #pragma unroll 1
             for (int c = 0; c < TA_D; c += 32) {
               float o[32];
@@ -373,21 +394,35 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
         }
         l = l * alpha + rs;
         m = m_use;
-        // P row -> shared memory, K-major with the 128-byte swizzle of a TMA tile
-        const uint32_t prow = sbase + C::P_OFF + j * C::P_TILE + (uint32_t)r * 128u;
+        if constexpr (TP) {
+          // P row -> this lane of the tile's P buffer u, two bf16 keys per column
+          const uint32_t tp = tmem_base + lane_off + C::P_COL + (uint32_t)((2 * j + u) * (BN / 2));
 #pragma unroll
-        for (int c = 0; c < BN / 8; ++c) {
-          st_shared_v4(prow + (c >> 3) * TA_HBOX + ((uint32_t)((c & 7) ^ (r & 7)) << 4),
-                       pack2_bf16(s[8 * c], s[8 * c + 1]), pack2_bf16(s[8 * c + 2], s[8 * c + 3]),
-                       pack2_bf16(s[8 * c + 4], s[8 * c + 5]),
-                       pack2_bf16(s[8 * c + 6], s[8 * c + 7]));
+          for (int c = 0; c < BN / 64; ++c) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = pack2_bf16(s[64 * c + 2 * e], s[64 * c + 2 * e + 1]);
+            tmem_st32_u(tp + 32 * c, pk);
+          }
+          tmem_wait_st();
+        } else {
+          // P row -> shared memory, K-major with the 128-byte swizzle of a TMA tile
+          const uint32_t prow = sbase + C::P_OFF + j * C::P_TILE + (uint32_t)r * 128u;
+#pragma unroll
+          for (int c = 0; c < BN / 8; ++c) {
+            st_shared_v4(prow + (c >> 3) * TA_HBOX + ((uint32_t)((c & 7) ^ (r & 7)) << 4),
+                         pack2_bf16(s[8 * c], s[8 * c + 1]), pack2_bf16(s[8 * c + 2], s[8 * c + 3]),
+                         pack2_bf16(s[8 * c + 4], s[8 * c + 5]),
+                         pack2_bf16(s[8 * c + 6], s[8 * c + 7]));
+          }
+          fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tbar(j, 4));
+        if (lane == 0) mbar_arrive(tbar(j, 4 + u));
       }
-      if (ok && T > 0) ok = warp_wait(tbar(j, 5), (uint32_t)(T - 1) & 1u, abort_flag, lim);
+      if (ok && T > 0)
+        ok = warp_wait(tbar(j, 6 + ((T - 1) & 1)), (uint32_t)((T - 1) >> 1) & 1u, abort_flag, lim);
       if (ok && T > 0) {
         tc_fence_after();
         const int jr = q0 + j * TA_BM + r;     // active-row index of this query
@@ -489,17 +524,17 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST>::THREADS, 1)
   }
 }
 
-template <int QT, int BN, int ST, bool MASK>
+template <int QT, int BN, int ST, bool TP, bool MASK>
 static cudaError_t run_attn_tc(const TaParams &p, dim3 grid, cudaStream_t s) {
-  using C = TaCfg<QT, BN, ST>;
+  using C = TaCfg<QT, BN, ST, TP>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, BN, ST, MASK>,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, BN, ST, TP, MASK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_k(attn_tc_kernel<QT, BN, ST, MASK>, grid, C::THREADS, C::SMEM, s, p);
+  return launch_k(attn_tc_kernel<QT, BN, ST, TP, MASK>, grid, C::THREADS, C::SMEM, s, p);
 }
 
 // Layout and key split of the tensor-core attention from a small cost model:
@@ -511,7 +546,7 @@ struct TaLayout {
   int qt, bn;
   double c_unit;   // us per 128 x 128 block of work at the power-capped clock
 };
-constexpr TaLayout kTaLayouts[] = {{1, 64, 1.4}, {1, 128, 2.0}, {2, 64, 1.4}};
+constexpr TaLayout kTaLayouts[] = {{1, 128, 1.5}, {1, 64, 2.1}, {2, 64, 2.0}};
 }  // namespace
 
 AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sms,
@@ -601,10 +636,13 @@ cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map128, const Tm
   p.wait_ns = wait_ns ? wait_ns : WAIT_LIMIT_NS;
   const dim3 grid(pl.units, n_heads, pl.splits);
   if (pl.qt == 2)
-    return stamp ? run_attn_tc<2, 64, 4, true>(p, grid, s) : run_attn_tc<2, 64, 4, false>(p, grid, s);
+    return stamp ? run_attn_tc<2, 64, 4, false, true>(p, grid, s)
+                 : run_attn_tc<2, 64, 4, false, false>(p, grid, s);
   if (pl.bn == 64)
-    return stamp ? run_attn_tc<1, 64, 5, true>(p, grid, s) : run_attn_tc<1, 64, 5, false>(p, grid, s);
-  return stamp ? run_attn_tc<1, 128, 2, true>(p, grid, s) : run_attn_tc<1, 128, 2, false>(p, grid, s);
+    return stamp ? run_attn_tc<1, 64, 6, true, true>(p, grid, s)
+                 : run_attn_tc<1, 64, 6, true, false>(p, grid, s);
+  return stamp ? run_attn_tc<1, 128, 3, true, true>(p, grid, s)
+               : run_attn_tc<1, 128, 3, true, false>(p, grid, s);
 }
 
 }  // namespace sl
