@@ -14,31 +14,36 @@
 //               ST-stage ring (64-column boxes, 128-byte swizzle)
 //   warp 1      TMEM owner and single-thread MMA issue, per key tile t and
 //               query tile j:
-//                 S_j = Q_j K_t^T  (M=128, N=BN keys, K=128 dims; both K-major)
-//                 into one of two TMEM score buffers of tile j, one key tile
-//                 ahead, then
-//                 O_j += P_j V_t   (M=128, N=128 dims, K=BN keys; P K-major from
-//                 shared memory, V MN-major straight from its TMA tile)
+//                 S_j = Q_j K_t^T  (M=128, N=BN keys, K=128 dims; both K-major
+//                 from shared memory) into a TMEM score buffer of tile j, one
+//                 key tile ahead, then
+//                 O_j += P_j V_t   (M=128, N=128 dims, K=BN keys; P K-major
+//                 from TMEM, V MN-major straight from its TMA tile)
 //   warps 2..   one softmax warpgroup per query tile: thread i owns query row
 //               i (its TMEM lane), so the row max and sum need no shuffles.
 //               Scores are scaled into base 2; the running max is raised
 //               lazily (only when a tile's max exceeds it by more than 2^8,
 //               rescaling O in TMEM); the bf16 probabilities go back to TMEM
-//               (one query tile per CTA: two P buffers, so the P V product of
-//               tile t runs while the exponentials of tile t + 1 are taken, and
-//               the product reads P from TMEM, sparing shared memory the P
-//               traffic) or to shared memory (two query tiles, which use all
-//               of TMEM for scores and outputs).
-// Two query tiles per CTA (QT = 2) share every K/V tile, halving the K/V
-// traffic per multiply-add, and the two softmax warpgroups take turns with the
-// tensor cores: while one computes its exponentials the MMA warp runs the
-// other's products.  A K/V stage is released only when the P V product of its
-// tile has completed, so the copy of tile t + ST starts then and must land
-// before the scores of that tile can be issued: the ring has to be deep enough
-// to cover the TMA latency (about a microsecond) with the work of the tiles in
-// between.  Layouts: one query tile with 64-key tiles in a 6-deep ring or
-// 128-key tiles in a 3-deep ring, two query tiles with 64-key tiles in a
-// 4-deep ring; all fit the 227 KB of shared memory of a CTA.
+//               into one of two P buffers, so the P V product of tile t runs
+//               while the exponentials of tile t + 1 are taken, and the
+//               product reads P from TMEM, sparing shared memory the P traffic.
+// What bounds the kernel is the K/V feed: a CTA reads BN keys and values of
+// 256 bytes each per BN x 128 x QT x 128 x 4 FLOP, and with one query tile per
+// CTA the 148 SMs together pull about 7 TB/s from L2 at half the tensor peak.
+// Two query tiles per CTA (QT = 2) share every K/V tile, halving those bytes
+// per FLOP, and the two softmax warpgroups take turns with the tensor cores:
+// while one computes its exponentials the MMA warp runs the other's products.
+// TMEM then holds one score buffer per query tile (64-key tiles): the scores of
+// tile t + 1 are issued as soon as the softmax has loaded those of tile t.
+// A K/V stage is released only when the P V products of its tile have
+// completed, so the copy of tile t + ST starts then and must land before the
+// scores of that tile can be issued: the ring is deep enough to cover the TMA
+// latency (about a microsecond) with the work of the tiles in between.
+// Layouts (query tiles / key tile / ring depth / score buffers): 1 / 128 / 3 /
+// 2 and 2 / 64 / 5 / 1 use most of an SM's shared memory and all 512 TMEM
+// columns (one CTA per SM); 1 / 64 / 2 / 1 needs 97 KB and 256 columns, so two
+// CTAs share an SM and each hides the other's barrier handoffs, start-up and
+// drain.
 // A split key range leaves unnormalised partial rows and (max, sum) in a
 // workspace; the thread that completes a row's last split (atomic ticket per
 // row and head) merges them, so no second kernel is needed.
@@ -58,31 +63,34 @@ constexpr int TA_D = 128;                     // head dim
 constexpr int TA_HBOX = 128 * 128;            // [128 rows][64 bf16] swizzled box, bytes
 constexpr float TA_RESCALE = 8.f;             // raise the running max when exceeded by 2^8
 
-template <int QT, int BN, int ST, bool TP>
+template <int QT, int BN, int ST, int SB>
 struct TaCfg {
   static constexpr int KBOX = BN * 128;                  // [BN rows][64 dims] box of K or V
   static constexpr int STAGE = 4 * KBOX;                 // K box 0, K box 1, V box 0, V box 1
-  // P of one query tile in shared memory ([128][BN] bf16), unless it lives in TMEM
-  static constexpr int P_TILE = TP ? 0 : (BN / 64) * TA_HBOX;
   static constexpr int Q_OFF = 0;                        // per query tile two dims boxes
   static constexpr int KV_OFF = QT * 2 * TA_HBOX;
-  static constexpr int P_OFF = KV_OFF + ST * STAGE;
-  static constexpr int BAR_OFF = P_OFF + QT * P_TILE;
-  // barriers: Q, kv_full[ST], kv_empty[ST], per query tile (s_full[2],
-  // s_free[2], p_full[2], pv_done[2]; index u = key tile & 1), drain
-  static constexpr int B_Q = 0, B_KVF = 1, B_KVE = 1 + ST, B_TILE = 1 + 2 * ST;
+  static constexpr int BAR_OFF = KV_OFF + ST * STAGE;
+  // barriers: Q, k_full[ST], k_empty[ST], v_full[ST], v_empty[ST] (a stage's
+  // K half is released when the scores of its tile are done, its V half when
+  // the P V products are), per query tile (s_full[2], s_free[2], p_full[2],
+  // pv_done[2]), drain
+  static constexpr int B_Q = 0, B_KF = 1, B_KE = 1 + ST, B_VF = 1 + 2 * ST, B_VE = 1 + 3 * ST;
+  static constexpr int B_TILE = 1 + 4 * ST;
   static constexpr int B_DRAIN = B_TILE + 8 * QT, B_COUNT = B_DRAIN + 1;
   static constexpr int SMEM = BAR_OFF + 8 * B_COUNT + 16 + 1024;   // + slot/flag + alignment
   static constexpr int THREADS = 64 + 128 * QT;
-  // TMEM: S buffers of tile j at j * 2 BN (+ BN for the second), O of tile j
-  // at O_COL + 128 j, and with TP the two bf16 P buffers of tile j (BN / 2
-  // columns each, two keys per column) at P_COL + (2 j + u) BN / 2
-  static constexpr uint32_t O_COL = QT * 2 * BN;
+  // TMEM: SB score buffers of tile j at (SB j + b) BN, O of tile j at
+  // O_COL + 128 j, the two bf16 P buffers of tile j (BN / 2 columns each, two
+  // keys per column) at P_COL + (2 j + u) BN / 2
+  static constexpr uint32_t O_COL = QT * SB * BN;
   static constexpr uint32_t P_COL = O_COL + QT * 128;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(P_COL + (TP ? QT * BN : 0) <= TMEM_COLS, "TMEM columns");
+  // two CTAs per SM when both fit: half of TMEM and of shared memory each
+  static constexpr int CTAS_PER_SM = (P_COL + QT * BN <= 256 && SMEM <= 232448 / 2 - 1024) ? 2 : 1;
+  static constexpr uint32_t TMEM_COLS = CTAS_PER_SM == 2 ? 256 : 512;
+  static_assert(P_COL + QT * BN <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM <= 232448, "shared memory of a CTA");
   static_assert(BN % 64 == 0 && BN <= 256, "key tile");
+  static_assert(SB == 1 || SB == 2, "score buffers");
 };
 }  // namespace
 
@@ -126,17 +134,22 @@ __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float *s) {
   tmem_wait_ld();
 }
 
-template <int QT, int BN, int ST, bool TP, bool MASK>
-__global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
+template <int QT, int BN, int ST, int SB, bool MASK>
+__global__ void __launch_bounds__(TaCfg<QT, BN, ST, SB>::THREADS, TaCfg<QT, BN, ST, SB>::CTAS_PER_SM)
     attn_tc_kernel(const __grid_constant__ TaParams p) {
-  using C = TaCfg<QT, BN, ST, TP>;
+  using C = TaCfg<QT, BN, ST, SB>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = s_addr(smem);
   const uint32_t bar0 = sbase + C::BAR_OFF;
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   auto tbar = [&](int j, int k) { return bar0 + 8u * (uint32_t)(C::B_TILE + 8 * j + k); };
-  // per query tile: 0,1 s_full[u]; 2,3 s_free[u]; 4,5 p_full[u]; 6,7 pv_done[u]
+  // per query tile: 0,1 s_full[b]; 2,3 s_free[b]; 4,5 p_full[u]; 6,7 pv_done[u]
+  // (b = score buffer of key tile t, u = t & 1).  With two score buffers each
+  // completes once every other key tile; with one, s_full[0] and s_free[0]
+  // complete once per key tile.
+  auto sbuf = [](int t) { return SB == 2 ? (t & 1) : 0; };
+  auto spar = [](int t) { return (uint32_t)(SB == 2 ? (t >> 1) : t) & 1u; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::BAR_OFF + 8 * C::B_COUNT);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -161,8 +174,10 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(C::B_Q), 1);
     for (int s = 0; s < ST; ++s) {
-      mbar_init(bar(C::B_KVF + s), 1);
-      mbar_init(bar(C::B_KVE + s), 1);
+      mbar_init(bar(C::B_KF + s), 1);
+      mbar_init(bar(C::B_KE + s), 1);
+      mbar_init(bar(C::B_VF + s), 1);
+      mbar_init(bar(C::B_VE + s), 1);
     }
     for (int j = 0; j < QT; ++j)
       for (int u = 0; u < 2; ++u) {
@@ -203,31 +218,44 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
         tma_load_2d(sq, &p.q_map, h * TA_D, q0 + j * TA_BM, bar(C::B_Q));
         tma_load_2d(sq + TA_HBOX, &p.q_map, h * TA_D + 64, q0 + j * TA_BM, bar(C::B_Q));
       }
-      int last_st = -1;
-      uint32_t last_ph = 0;
+      // K of tile t + ST goes into stage t % ST once the scores of tile t are
+      // done, V once its P V products are: K runs ahead of V
+      int nk = 0, nv = 0;                    // K and V copies issued
       for (int t = 0; t < T; ++t) {
         const int st = t % ST;
         const uint32_t ph = (uint32_t)(t / ST) & 1u;
-        if (!mbar_wait(bar(C::B_KVE + st), ph ^ 1u, abort_flag, lim)) { ok = false; break; }
-        mbar_expect_tx(bar(C::B_KVF + st), C::STAGE);
         const int y = b * p.n_ctx + (kt0 + t) * BN;
         const uint32_t sk = sbase + C::KV_OFF + st * C::STAGE;
-        tma_load_2d(sk, &p.k_map, h * TA_D, y, bar(C::B_KVF + st));
-        tma_load_2d(sk + C::KBOX, &p.k_map, h * TA_D + 64, y, bar(C::B_KVF + st));
-        tma_load_2d(sk + 2 * C::KBOX, &p.v_map, h * TA_D, y, bar(C::B_KVF + st));
-        tma_load_2d(sk + 3 * C::KBOX, &p.v_map, h * TA_D + 64, y, bar(C::B_KVF + st));
-        last_st = st;
-        last_ph = ph;
+        if (!mbar_wait(bar(C::B_KE + st), ph ^ 1u, abort_flag, lim)) { ok = false; break; }
+        mbar_expect_tx(bar(C::B_KF + st), 2 * C::KBOX);
+        tma_load_2d(sk, &p.k_map, h * TA_D, y, bar(C::B_KF + st));
+        tma_load_2d(sk + C::KBOX, &p.k_map, h * TA_D + 64, y, bar(C::B_KF + st));
+        ++nk;
+        if (!mbar_wait(bar(C::B_VE + st), ph ^ 1u, abort_flag, lim)) { ok = false; break; }
+        mbar_expect_tx(bar(C::B_VF + st), 2 * C::KBOX);
+        tma_load_2d(sk + 2 * C::KBOX, &p.v_map, h * TA_D, y, bar(C::B_VF + st));
+        tma_load_2d(sk + 3 * C::KBOX, &p.v_map, h * TA_D + 64, y, bar(C::B_VF + st));
+        ++nv;
       }
       pdl_trigger();
       if (!ok) {
         atomicExch(p.err, DEV_TIMEOUT_PRODUCER);
         *abort_flag = 1;
       }
-      // every issued copy lands before the CTA can exit
+      // every issued copy lands before the CTA can exit: the last copy into
+      // each stage of each ring (copies complete in any order)
       volatile int never = 0;
       mbar_wait(bar(C::B_Q), 0, &never, lim);
-      if (last_st >= 0) mbar_wait(bar(C::B_KVF + last_st), last_ph, &never, lim);
+      for (int st = 0; st < ST; ++st) {
+        if (st < nk) {
+          const int tl = st + ((nk - 1 - st) / ST) * ST;   // last tile copied into stage st
+          mbar_wait(bar(C::B_KF + st), (uint32_t)(tl / ST) & 1u, &never, lim);
+        }
+        if (st < nv) {
+          const int tl = st + ((nv - 1 - st) / ST) * ST;
+          mbar_wait(bar(C::B_VF + st), (uint32_t)(tl / ST) & 1u, &never, lim);
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA
@@ -237,51 +265,45 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
       auto issue_s = [&](int t, int j) {
         const uint32_t sq = sbase + C::Q_OFF + j * 2 * TA_HBOX;
         const uint32_t sk = sbase + C::KV_OFF + (t % ST) * C::STAGE;
-        const uint32_t dt = tmem_base + (uint32_t)(j * 2 * BN + (t & 1) * BN);
+        const uint32_t dt = tmem_base + (uint32_t)((j * SB + sbuf(t)) * BN);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = smem_desc_sw128(sq + (kk >> 2) * TA_HBOX) + 2 * (kk & 3);
           const uint64_t bd = smem_desc_sw128(sk + (kk >> 2) * C::KBOX) + 2 * (kk & 3);
           tc_mma(dt, a, bd, id_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(tbar(j, t & 1));
+        tc_commit(tbar(j, sbuf(t)));
       };
       auto issue_pv = [&](int t, int j) {
         const uint32_t sv = sbase + C::KV_OFF + (t % ST) * C::STAGE + 2 * C::KBOX;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
+          // P of key tile t from its TMEM buffer: 16 keys = 8 columns per step
           const uint64_t bd = smem_desc_sw128_mn(sv + kk * 2048, C::KBOX, 1024);
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          if constexpr (TP) {
-            // P of key tile t from its TMEM buffer: 16 keys = 8 columns per step
-            const uint32_t pa =
-                tmem_base + C::P_COL + (uint32_t)((2 * j + (t & 1)) * (BN / 2) + kk * 8);
-            tc_mma_ts(tmem_base + C::O_COL + 128 * j, pa, bd, id_o, acc);
-          } else {
-            const uint32_t sp = sbase + C::P_OFF + j * C::P_TILE;
-            const uint64_t a = smem_desc_sw128(sp + (kk >> 2) * TA_HBOX) + 2 * (kk & 3);
-            tc_mma(tmem_base + C::O_COL + 128 * j, a, bd, id_o, acc);
-          }
+          const uint32_t pa =
+              tmem_base + C::P_COL + (uint32_t)((2 * j + (t & 1)) * (BN / 2) + kk * 8);
+          tc_mma_ts(tmem_base + C::O_COL + 128 * j, pa, bd, id_o, (t > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(tbar(j, 6 + (t & 1)));
       };
       bool ok = mbar_wait(bar(C::B_Q), 0, abort_flag, lim);
-      if (ok && T > 0) ok = mbar_wait(bar(C::B_KVF), 0, abort_flag, lim);
+      if (ok && T > 0) ok = mbar_wait(bar(C::B_KF), 0, abort_flag, lim);
       if (ok && T > 0) {
         tc_fence_after();
         for (int j = 0; j < nj; ++j) issue_s(0, j);
+        tc_commit(bar(C::B_KE));             // K_0 free once these scores are done
       }
       for (int t = 0; ok && t < T; ++t) {
         if (t + 1 < T) {
           const int st = (t + 1) % ST;
-          if (!mbar_wait(bar(C::B_KVF + st), (uint32_t)((t + 1) / ST) & 1u, abort_flag, lim)) {
+          if (!mbar_wait(bar(C::B_KF + st), (uint32_t)((t + 1) / ST) & 1u, abort_flag, lim)) {
             ok = false;
             break;
           }
           for (int j = 0; ok && j < nj; ++j) {
-            // score buffer (t+1) & 1 of tile j was last read at key tile t - 1
-            if (!mbar_wait(tbar(j, 2 + ((t + 1) & 1)), ((uint32_t)((t + 1) >> 1) & 1u) ^ 1u,
-                           abort_flag, lim)) {
+            // the score buffer of key tile t + 1 was last read at key tile
+            // t + 1 - SB (its s_free phase before the current one)
+            if (!mbar_wait(tbar(j, 2 + sbuf(t + 1)), spar(t + 1) ^ 1u, abort_flag, lim)) {
               ok = false;
               break;
             }
@@ -289,6 +311,11 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
             issue_s(t + 1, j);
           }
           if (!ok) break;
+          tc_commit(bar(C::B_KE + st));      // K_{t+1} consumed by every tile
+        }
+        if (!mbar_wait(bar(C::B_VF + t % ST), (uint32_t)(t / ST) & 1u, abort_flag, lim)) {
+          ok = false;
+          break;
         }
         for (int j = 0; ok && j < nj; ++j) {
           if (!mbar_wait(tbar(j, 4 + (t & 1)), (uint32_t)(t >> 1) & 1u, abort_flag, lim)) {
@@ -299,7 +326,7 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
           issue_pv(t, j);
         }
         if (!ok) break;
-        tc_commit(bar(C::B_KVE + t % ST));   // K_t and V_t consumed by every tile
+        tc_commit(bar(C::B_VE + t % ST));    // V_t consumed by every tile
       }
       if (!ok) {
         atomicExch(p.err, DEV_TIMEOUT_MMA);
@@ -325,12 +352,12 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
       float s[BN];
       for (int t = 0; t < T; ++t) {
         const int u = t & 1;
-        if (!warp_wait(tbar(j, u), (uint32_t)(t >> 1) & 1u, abort_flag, lim)) { ok = false; break; }
+        if (!warp_wait(tbar(j, sbuf(t)), spar(t), abort_flag, lim)) { ok = false; break; }
         tc_fence_after();
-        tmem_ld_row<BN>(tmem_base + lane_off + (uint32_t)(j * 2 * BN + u * BN), s);
+        tmem_ld_row<BN>(tmem_base + lane_off + (uint32_t)((j * SB + sbuf(t)) * BN), s);
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tbar(j, 2 + u));
+        if (lane == 0) mbar_arrive(tbar(j, 2 + sbuf(t)));
         const int key0 = (kt0 + t) * BN;
         // row max of the raw scores (the scale is positive) as eight independent
         // partials: a single running value would chain BN dependent instructions
@@ -367,11 +394,9 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
         }
         const float rs = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
         // O must be current before a rescale, and the P buffer about to be
-        // written must have been read: with P in TMEM the buffer of tile t was
-        // last read by the P V product of tile t - 2; in shared memory there is
-        // one buffer, read by the product of tile t - 1
+        // written must have been read, last by the P V product of tile t - 2
         const bool any_resc = __any_sync(0xffffffffu, resc);
-        const int t_prev = (TP && !any_resc) ? t - 2 : t - 1;
+        const int t_prev = any_resc ? t - 1 : t - 2;
         if (t_prev >= 0) {
           const int ub = t_prev & 1;
           if (!warp_wait(tbar(j, 6 + ub), (uint32_t)(t_prev >> 1) & 1u, abort_flag, lim)) {
@@ -394,8 +419,8 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
         }
         l = l * alpha + rs;
         m = m_use;
-        if constexpr (TP) {
-          // P row -> this lane of the tile's P buffer u, two bf16 keys per column
+        // P row -> this lane of the tile's P buffer u, two bf16 keys per column
+        {
           const uint32_t tp = tmem_base + lane_off + C::P_COL + (uint32_t)((2 * j + u) * (BN / 2));
 #pragma unroll
           for (int c = 0; c < BN / 64; ++c) {
@@ -405,17 +430,6 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
             tmem_st32_u(tp + 32 * c, pk);
           }
           tmem_wait_st();
-        } else {
-          // P row -> shared memory, K-major with the 128-byte swizzle of a TMA tile
-          const uint32_t prow = sbase + C::P_OFF + j * C::P_TILE + (uint32_t)r * 128u;
-#pragma unroll
-          for (int c = 0; c < BN / 8; ++c) {
-            st_shared_v4(prow + (c >> 3) * TA_HBOX + ((uint32_t)((c & 7) ^ (r & 7)) << 4),
-                         pack2_bf16(s[8 * c], s[8 * c + 1]), pack2_bf16(s[8 * c + 2], s[8 * c + 3]),
-                         pack2_bf16(s[8 * c + 4], s[8 * c + 5]),
-                         pack2_bf16(s[8 * c + 6], s[8 * c + 7]));
-          }
-          fence_proxy_async_smem();
         }
         tc_fence_before();
         __syncwarp();
@@ -524,29 +538,38 @@ __global__ void __launch_bounds__(TaCfg<QT, BN, ST, TP>::THREADS, 1)
   }
 }
 
-template <int QT, int BN, int ST, bool TP, bool MASK>
+template <int QT, int BN, int ST, int SB, bool MASK>
 static cudaError_t run_attn_tc(const TaParams &p, dim3 grid, cudaStream_t s) {
-  using C = TaCfg<QT, BN, ST, TP>;
+  using C = TaCfg<QT, BN, ST, SB>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, BN, ST, TP, MASK>,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<QT, BN, ST, SB, MASK>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    // all of the SM's unified L1 as shared memory, so that two CTAs fit
+    e = cudaFuncSetAttribute(attn_tc_kernel<QT, BN, ST, SB, MASK>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  return launch_k(attn_tc_kernel<QT, BN, ST, TP, MASK>, grid, C::THREADS, C::SMEM, s, p);
+  return launch_k(attn_tc_kernel<QT, BN, ST, SB, MASK>, grid, C::THREADS, C::SMEM, s, p);
 }
 
 // Layout and key split of the tensor-core attention from a small cost model:
-// CTAs run in waves (one per SM, bound by shared memory); a CTA costs a fixed
-// set-up and drain plus a time per (128-query tile x 128 keys) of work that
-// depends on the layout; a split adds the merge.
+// CTAs run in waves (one or two per SM, bound by shared memory and TMEM); a
+// CTA costs a fixed set-up and drain plus a time per (128-query tile x 128
+// keys) of work that depends on the layout; a split adds the merge.
 namespace {
 struct TaLayout {
-  int qt, bn;
-  double c_unit;   // us per 128 x 128 block of work at the power-capped clock
+  int qt, bn, per_sm;   // query tiles and key tile of a CTA, CTAs resident per SM
+  double c_unit;        // us per 128 x 128 block of work of one CTA at the power-capped clock
 };
-constexpr TaLayout kTaLayouts[] = {{1, 128, 1.5}, {1, 64, 2.1}, {2, 64, 2.0}};
+// measured on batch 4 x 512 and 2048 queries over 2048 keys; a CTA's start-up
+// (first Q/K/V copies, TMEM allocation) and drain (O out) cost ~6 us, and a key
+// split as much again (partial rows out and back, the merge)
+constexpr TaLayout kTaLayouts[] = {{1, 128, 1, 1.3}, {1, 64, 2, 2.2}, {2, 64, 1, 1.9}};
+constexpr double kTaCtaFixed = 6.0, kTaSplitCost = 6.0;
 }  // namespace
 
 AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sms,
@@ -575,9 +598,9 @@ AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sm
       const int sp = (ktiles + per - 1) / per;
       if (!force_splits && sp != req) continue;
       const long ctas = (long)units * n_heads * sp;
-      const long waves = (ctas + num_sms - 1) / num_sms;
+      const long waves = (ctas + (long)num_sms * ly.per_sm - 1) / ((long)num_sms * ly.per_sm);
       const double work = (double)per * bn / 128.0 * qt * fill;
-      const double t = waves * (2.0 + ly.c_unit * work) + (sp > 1 ? 3.0 : 0.0);
+      const double t = waves * (kTaCtaFixed + ly.c_unit * work) + (sp > 1 ? kTaSplitCost : 0.0);
       if (t < best_t * 0.97) {                 // a clear gain, else the earlier layout
         best_t = t;
         best.qt = qt;
@@ -636,13 +659,13 @@ cudaError_t launch_attn_tc(const TmaMat &q_map, const TmaMat &k_map128, const Tm
   p.wait_ns = wait_ns ? wait_ns : WAIT_LIMIT_NS;
   const dim3 grid(pl.units, n_heads, pl.splits);
   if (pl.qt == 2)
-    return stamp ? run_attn_tc<2, 64, 4, false, true>(p, grid, s)
-                 : run_attn_tc<2, 64, 4, false, false>(p, grid, s);
+    return stamp ? run_attn_tc<2, 64, 5, 1, true>(p, grid, s)
+                 : run_attn_tc<2, 64, 5, 1, false>(p, grid, s);
   if (pl.bn == 64)
-    return stamp ? run_attn_tc<1, 64, 6, true, true>(p, grid, s)
-                 : run_attn_tc<1, 64, 6, true, false>(p, grid, s);
-  return stamp ? run_attn_tc<1, 128, 3, true, true>(p, grid, s)
-               : run_attn_tc<1, 128, 3, true, false>(p, grid, s);
+    return stamp ? run_attn_tc<1, 64, 2, 1, true>(p, grid, s)
+                 : run_attn_tc<1, 64, 2, 1, false>(p, grid, s);
+  return stamp ? run_attn_tc<1, 128, 3, 2, true>(p, grid, s)
+               : run_attn_tc<1, 128, 3, 2, false>(p, grid, s);
 }
 
 }  // namespace sl
