@@ -29,7 +29,7 @@ region is bracketed by barriers and the max over ranks is taken.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload full8b|long8b] [--eps E] [--scripted] [--batch B]
-                  [--gate-q Q] [--ablation none|no_kv_cache|gate_only]
+                  [--gate-q Q] [--ablation none|no_kv_cache|gate_only] [--head-fusion on|off]
 """
 from __future__ import annotations
 
@@ -117,7 +117,9 @@ def workload_config(args, setup: wl.SamplerSetup, world: int) -> dict:
                         + (", scripted lock schedule" if setup.scripted else "")
                         + (", ablation: no KV cache (active rows' keys only)"
                            if setup.no_kv_cache else "")
-                        + (", ablation: confidence gate only" if setup.gate_only else ""),
+                        + (", ablation: confidence gate only" if setup.gate_only else "")
+                        + (", sure-test statistics in a separate pass after the LM head"
+                           if getattr(args, "head_fusion", "on") == "off" else ""),
             "bench_step": (f"one full decode ({T} denoising steps)"
                            if bench_unit_steps(args, setup) == T else
                            f"one semi-autoregressive block ({setup.steps_per_block} denoising "
@@ -347,11 +349,15 @@ class Ranks:
 
 
 def bench_unit_steps(args, setup: wl.SamplerSetup) -> int:
-    """Denoising steps per bench step: one semi-autoregressive block for the
-    long decode (512 steps, ~20 s), a whole decode otherwise."""
+    """Denoising steps per bench step: a whole decode (the default), so that
+    any K timed steps weigh the decode's early, heavy steps (every row active)
+    and its late, light ones as the decode itself does; or, for quick looks,
+    one semi-autoregressive block (timed from a decode's first step, so a K
+    that is not a multiple of the blocks per decode over-weights the first
+    blocks)."""
     mode = getattr(args, "bench_step", "auto")
     if mode == "auto":
-        mode = "block" if args.workload == "long8b" else "decode"
+        mode = "decode"
     return setup.steps_per_block if mode == "block" else setup.steps
 
 
@@ -389,6 +395,7 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     model = rt.Model(shape, weights, "bf16")
     model.set_ablation(no_kv_cache=setup.no_kv_cache, gate_only=setup.gate_only)
+    model.set_head_fusion(args.head_fusion == "on")
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, T, setup.block_len,
                    setup.tokens_per_step, setup.eps, setup.gate_q, setup.scripted)
     prompts = wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab, shape.mask_id,
@@ -638,15 +645,16 @@ def run_reference(args, rank: int, world: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long8b",
                     help="long8b: LLaDA-8B shape, batch 4, N = 2048, 512 steps (the default); "
                          "full8b: batch 1, N = 384, 256 steps")
     ap.add_argument("--bench-step", default="auto", choices=["auto", "decode", "block"],
-                    help="denoising steps per bench step: a whole decode, or one "
-                         "semi-autoregressive block (auto: block for long8b)")
+                    help="denoising steps per bench step: a whole decode (auto), or one "
+                         "semi-autoregressive block (a quick look; biased towards the "
+                         "first blocks unless K is a multiple of the blocks per decode)")
     ap.add_argument("--eps", type=float, default=None)
     ap.add_argument("--scripted", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
@@ -655,6 +663,9 @@ def main():
                     help="confidence-gate quantile (default: the workload's; < 0 = off)")
     ap.add_argument("--ablation", default="none", choices=["none", "no_kv_cache", "gate_only"],
                     help="run one of the pages' ablations instead of the method")
+    ap.add_argument("--head-fusion", default="on", choices=["on", "off"],
+                    help="sure-test statistics in the LM head's epilogue (on) or in a "
+                         "separate pass over the stored logits (off)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "surelock_bench"),
                     help="where the per-rank clock samples (CSV) are written")

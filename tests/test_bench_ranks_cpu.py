@@ -163,14 +163,17 @@ def test_trajectory_from_lock_steps():
 
 
 def test_bench_step_unit():
-    """The long decode's bench step is one semi-autoregressive block (16 per
-    decode), the short decode's a whole decode; --bench-step overrides."""
+    """A bench step is a whole decode for both workloads (unbiased for any K);
+    --bench-step block takes one semi-autoregressive block (16 per long decode)."""
     import types
     sys.path.insert(0, ROOT)
     import bench
     long_ = bench.make_setup("long8b", None, False)
     short = bench.make_setup("full8b", None, False)
     a = types.SimpleNamespace(workload="long8b", bench_step="auto")
+    assert bench.bench_unit_steps(a, long_) == 512
+    assert "full decode" in bench.workload_config(a, long_, 1)["bench_step"]
+    a = types.SimpleNamespace(workload="long8b", bench_step="block")
     assert bench.bench_unit_steps(a, long_) == 32 == long_.steps // 16
     assert "block" in bench.workload_config(a, long_, 1)["bench_step"]
     a = types.SimpleNamespace(workload="full8b", bench_step="auto")

@@ -39,8 +39,9 @@ CASES = [
 
 # (queries per CTA, cross-CTA key split[, key tile]); 0 = the library's cost
 # model.  128 or 256 queries per CTA = the tensor-core kernel (one or two
-# 128-query tiles sharing each K/V tile; the default) with 64- or 128-key
-# tiles, 16/32/64 the mma.sync kernel.
+# 128-query tiles sharing each K/V tile; the default): one tile with 64-key
+# tiles runs two CTAs per SM, one tile with 128-key tiles and two tiles (64-key)
+# one CTA per SM; 16/32/64 the mma.sync kernel.
 LAYOUTS = [(0, 0), (128, 1, 64), (128, 2, 64), (128, 16, 64), (128, 1, 128), (128, 3, 128),
            (128, 16, 128), (256, 1), (256, 2), (256, 5),
            (16, 1), (32, 1), (64, 1), (16, 4), (32, 2), (64, 3)]
