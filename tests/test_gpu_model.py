@@ -125,6 +125,8 @@ def test_layer_forward_bf16_matches_oracle(cuda_dev):
     cvb = cv[1].astype(np.float64).copy()
     ref = om.layer_forward(shape, w64["layers"][1], h_np.astype(np.float64), positions[0], ckb, cvb)
     err = np.abs(h.double().cpu().numpy() - ref).max()
+    print(f"block output max abs err {err:.4g} (|ref| max {np.abs(ref).max():.3g}, "
+          f"update max {np.abs(ref - h_np).max():.3g})")
     assert err <= 5e-2 * max(1.0, np.abs(ref).max()), err
     model.close()
 
