@@ -8,7 +8,7 @@ import torch
 import workloads as wl
 from oracle import model as om
 from token_locking_b200 import runtime as rt
-from parity_util import LOGIT_TOL, to64, weights_for_oracle, weights_to_device
+from parity_util import BLOCK_ULPS, LOGIT_TOL, bf16_ulp, to64, weights_for_oracle, weights_to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -125,9 +125,10 @@ def test_layer_forward_bf16_matches_oracle(cuda_dev):
     cvb = cv[1].astype(np.float64).copy()
     ref = om.layer_forward(shape, w64["layers"][1], h_np.astype(np.float64), positions[0], ckb, cvb)
     err = np.abs(h.double().cpu().numpy() - ref).max()
-    print(f"block output max abs err {err:.4g} (|ref| max {np.abs(ref).max():.3g}, "
-          f"update max {np.abs(ref - h_np).max():.3g})")
-    assert err <= 5e-2 * max(1.0, np.abs(ref).max()), err
+    # one block: within BLOCK_ULPS bf16 ulps of the largest entry of the block's
+    # update (observed 0.0053 for an update of max 2.28: bound 0.0625)
+    upd = np.abs(ref - h_np).max()
+    assert err <= BLOCK_ULPS * bf16_ulp(upd), (err, upd)
     model.close()
 
 

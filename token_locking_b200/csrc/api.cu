@@ -1366,15 +1366,48 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
   const int Ns[G_KINDS] = {3 * d, d, 2 * f, d, V};
   const int Ks[G_KINDS] = {d, d, d, f, d};
   const int split_opts[] = {1, 2, 3, 4, 6, 8, 9, 12, 16, -1};   // -1: stream-K
+  // one candidate's time at M rows: three blocks of three back-to-back
+  // repetitions, the median block (a stray slow block does not decide); each
+  // repetition is followed by a small kernel (an RMSNorm, as in the layer) so
+  // that successive GEMMs cannot overlap each other through programmatic launch
+  // and flatter tilings with few CTAs
+  auto time_plan = [&](int kind, const Plan &pl, int M, float *ms_out) -> sl_status {
+    auto launch = [&]() {
+      sl_status r = run_gemm(m, c, rows, 0, kind, pl, M, c->h, logits, s);
+      if (r != SL_OK) return r;
+      cudaError_t e = launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, M, c->a, s);
+      return e == cudaSuccess ? SL_OK : cuda_fail(e, "sl_model_autotune: spacer");
+    };
+    sl_status r = launch();
+    if (r != SL_OK) return r;
+    float blocks[3] = {0.f, 0.f, 0.f};
+    for (int blk = 0; blk < 3; ++blk) {
+      cudaEventRecord(e0, s);
+      for (int it = 0; it < 3; ++it)
+        if ((r = launch()) != SL_OK) return r;
+      cudaEventRecord(e1, s);
+      if (cudaEventSynchronize(e1) != cudaSuccess)
+        return cuda_fail(cudaGetLastError(), "sl_model_autotune: timing");
+      cudaEventElapsedTime(&blocks[blk], e0, e1);
+    }
+    std::sort(blocks, blocks + 3);
+    *ms_out = blocks[1];
+    return SL_OK;
+  };
   for (int b = 0; b < kTuneCount && st == SL_OK; ++b) {
     if (b > 0 && kTuneBounds[b - 1] >= max_rows) break;
     const int Mb = std::min(kTuneBounds[b], max_rows);
-    if ((st = ensure_maps(c, Mb)) != SL_OK) break;
-    for (int kind = 0; kind < G_KINDS && st == SL_OK; ++kind) {
+    // a bucket's tiling serves every row count in it: from 1024 rows up (where
+    // a 256-row tile more or less is a large share of the work) it is timed at
+    // both ends of the bucket and the tiling with the least summed slowdown
+    // against each end's fastest is kept; below, at the bucket's upper end
+    std::vector<int> pts = {Mb};
+    if (b > 0 && Mb >= 1024 && kTuneBounds[b - 1] + 1 < Mb) pts.push_back(kTuneBounds[b - 1] + 1);
+    // candidates of every GEMM kind, filtered at the upper end
+    std::vector<std::array<int, 3>> cands[G_KINDS];
+    for (int kind = 0; kind < G_KINDS; ++kind) {
       if (kind == G_HD && Mb > head_rows) continue;
       const int N = Ns[kind], K = Ks[kind], kblocks = K / 64;
-      double best_ms = 1e30;
-      std::array<int, 3> best = {0, 1, 1};
       for (int variant = 0; variant <= 2; ++variant) {
         const int msub = variant >= 1 ? 2 : 1;
         if (variant >= 1 && Mb <= 128) continue;
@@ -1396,44 +1429,39 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
               const long units = (long)((Mb + 128 * msub - 1) / (128 * msub)) * (N / bn) * ss;
               if (units > 24L * m->num_sms) continue;
             }
-            Plan pl{bn, ss, msub, 0.0};
-            plan_set_variant(pl, variant);
-            // each repetition is followed by a small kernel (an RMSNorm, as in
-            // the layer) so that successive GEMMs cannot overlap each other
-            // through programmatic launch and flatter tilings with few CTAs
-            auto launch = [&]() {
-              sl_status r = run_gemm(m, c, rows, 0, kind, pl, Mb, c->h, logits, s);
-              if (r != SL_OK) return r;
-              cudaError_t e = launch_rmsnorm(SL_BF16, c->h, m->final_norm, d, cfg.rms_eps, Mb,
-                                             c->a, s);
-              return e == cudaSuccess ? SL_OK : cuda_fail(e, "sl_model_autotune: spacer");
-            };
-            // three blocks of three back-to-back repetitions; the candidate's
-            // time is the median block (a stray slow block does not decide)
-            if ((st = launch()) != SL_OK) break;
-            float blocks[3] = {0.f, 0.f, 0.f};
-            for (int blk = 0; blk < 3 && st == SL_OK; ++blk) {
-              cudaEventRecord(e0, s);
-              for (int it = 0; it < 3 && st == SL_OK; ++it) st = launch();
-              cudaEventRecord(e1, s);
-              if (st != SL_OK) break;
-              if (cudaEventSynchronize(e1) != cudaSuccess) {
-                st = cuda_fail(cudaGetLastError(), "sl_model_autotune: timing");
-                break;
-              }
-              cudaEventElapsedTime(&blocks[blk], e0, e1);
-            }
-            if (st != SL_OK) break;
-            std::sort(blocks, blocks + 3);
-            const float ms = blocks[1];
-            if (ms < best_ms) {
-              best_ms = ms;
-              best = {bn, ss, variant};
-            }
+            cands[kind].push_back({bn, ss, variant});
           }
-          if (st != SL_OK) break;
         }
-        if (st != SL_OK) break;
+      }
+    }
+    std::vector<std::vector<float>> times[G_KINDS];
+    for (int kind = 0; kind < G_KINDS; ++kind)
+      times[kind].assign(cands[kind].size(), std::vector<float>(pts.size(), 0.f));
+    for (size_t pi = 0; pi < pts.size() && st == SL_OK; ++pi) {
+      if ((st = ensure_maps(c, pts[pi])) != SL_OK) break;
+      for (int kind = 0; kind < G_KINDS && st == SL_OK; ++kind)
+        for (size_t ci = 0; ci < cands[kind].size() && st == SL_OK; ++ci) {
+          Plan pl{cands[kind][ci][0], cands[kind][ci][1], cands[kind][ci][2] >= 1 ? 2 : 1, 0.0};
+          plan_set_variant(pl, cands[kind][ci][2]);
+          st = time_plan(kind, pl, pts[pi], &times[kind][ci][pi]);
+        }
+    }
+    if (st != SL_OK) break;
+    for (int kind = 0; kind < G_KINDS; ++kind) {
+      if (cands[kind].empty()) continue;
+      std::vector<float> fastest(pts.size(), 1e30f);
+      for (const auto &tc : times[kind])
+        for (size_t pi = 0; pi < pts.size(); ++pi) fastest[pi] = std::min(fastest[pi], tc[pi]);
+      double best_score = 1e30;
+      std::array<int, 3> best = {0, 1, 1};
+      for (size_t ci = 0; ci < cands[kind].size(); ++ci) {
+        double score = 0.0;
+        for (size_t pi = 0; pi < pts.size(); ++pi)
+          score += times[kind][ci][pi] / std::max(fastest[pi], 1e-6f);
+        if (score < best_score) {
+          best_score = score;
+          best = cands[kind][ci];
+        }
       }
       m->tuned[kind][b] = best;
     }
