@@ -270,8 +270,11 @@ sl_status sl_attention(sl_model *m, sl_kv_cache *c, sl_active *a, int layer, con
  * its partial tiles atomically) pick the tiling; variant
  * picks the kernel: 0 = one CTA per 128 x bn tile, 1 = one CTA per 256 x bn
  * tile (two accumulators share each weight tile), 2 = a CTA pair per 256 x bn
- * tile with 2-SM tensor-core instructions (bn 128, 192 or 256).  bn = 0 lets the
- * library choose everything.  K % 64 == 0, N % bn == 0, pointers 16-byte
+ * tile with 2-SM tensor-core instructions (bn 128, 192 or 256), 3 = swapped
+ * operands for few rows (M <= 256, bn 128, splits >= 1, RESID or ACCUM): each
+ * CTA multiplies 128 weight rows by all M rows (C^T = B A^T, the tensor-core
+ * work following M rounded up to 32 instead of a padded 256-row tile) and adds
+ * the transposed tile into out.  bn = 0 lets the library choose everything.  K % 64 == 0, N % bn == 0, pointers 16-byte
  * aligned, ldo >= the output columns (N, or F for SWIGLU) with 16-byte rows
  * (ldo % 4 == 0 for fp32 outputs, % 8 for bf16); SL_ERR_INVALID otherwise. */
 enum { SL_GEMM_STORE = 0, SL_GEMM_RESID = 1, SL_GEMM_SWIGLU = 2, SL_GEMM_ACCUM = 3 };
@@ -332,7 +335,8 @@ sl_status sl_model_set_attention_keys(sl_model *m, int key_tile);
 /* Pin the tiling of GEMM `kind` for the row-count bucket that holds M (the
  * buckets of sl_model_autotune); arguments as for sl_gemm_bf16.  Returns
  * SL_ERR_INVALID for a tiling the GEMM cannot use (the LM head takes no K
- * split).  bf16 models only. */
+ * split and no swapped operands; swapped operands need a bucket of at most 256
+ * rows).  bf16 models only. */
 sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits, int variant);
 
 /* Ablations of the method (Paper-Notes, ablation table), a bit set; 0 (the

@@ -54,7 +54,9 @@ static void check_plan(const Shape &sh, int kind, int M, int ns, const Plan &pl)
   const int v = plan_variant(pl);
   Plan back{pl.bn, pl.splits, 1, 0.0};
   plan_set_variant(back, v);
-  CHECK(back.msub == pl.msub && back.pair == pl.pair, CTX);
+  CHECK(back.msub == pl.msub && back.pair == pl.pair && back.swap == pl.swap, CTX);
+  // swapped operands: projections of at most 256 rows, 128 weight rows per tile
+  CHECK(!pl.swap || (pl.bn == 128 && M <= 256 && kind != G_HD && pl.splits >= 1), CTX);
   switch (kind) {
     case G_QKV:
       CHECK(d % pl.bn == 0, CTX);                           // one of Wq, Wk, Wv per tile

@@ -148,3 +148,54 @@ def test_resid_strided_output(cuda_dev, variant, splits):
     _close(buf[:, :N] - 3.0, _ref(a, b), K, False)
     assert torch.all(buf[:, N:] == 3.0)
     rt.device_check()
+
+
+# Swapped operands (variant 3): the weight tile is the MMA's 128-row operand
+# and the M rows its N dimension (rounded up to 32), for M <= 256.
+@pytest.mark.parametrize("splits", [1, 2, 5])
+@pytest.mark.parametrize("M", [1, 5, 31, 33, 128, 130, 200, 255, 256])
+def test_swap_resid(cuda_dev, splits, M):
+    K, N = 1024, 768
+    a, b = _mk((M, K), 21, cuda_dev), _mk((N, K), 22, cuda_dev)
+    h0 = torch.randn((M, N), generator=torch.Generator().manual_seed(23)).to(cuda_dev)
+    h = h0.clone()
+    rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=128, splits=splits, variant=3)
+    torch.cuda.synchronize()
+    _close(h - h0, _ref(a, b), K, False)
+    rt.device_check()
+
+
+@pytest.mark.parametrize("swiglu", [False, True])
+@pytest.mark.parametrize("splits", [1, 3])
+@pytest.mark.parametrize("M", [7, 129, 256])
+def test_swap_accum(cuda_dev, swiglu, splits, M):
+    """ACCUM into a zeroed fp32 buffer; gate/up halves into columns [0, F) and
+    [F, 2F), as the gate/up finishing pass reads them."""
+    K, F = 2048, 384
+    a = _mk((M, K), 24, cuda_dev)
+    if swiglu:
+        wg, wu = _mk((F, K), 25, cuda_dev), _mk((F, K), 26, cuda_dev)
+        out = torch.zeros((M, 2 * F), device=cuda_dev, dtype=torch.float32)
+        rt.gemm_bf16(A.GEMM_ACCUM, a, wg, out, b2=wu, bn=128, splits=splits, variant=3)
+        torch.cuda.synchronize()
+        _close(out[:, :F], _ref(a, wg), K, False)
+        _close(out[:, F:], _ref(a, wu), K, False)
+    else:
+        b = _mk((3 * F, K), 27, cuda_dev)
+        out = torch.zeros((M, 3 * F), device=cuda_dev, dtype=torch.float32)
+        rt.gemm_bf16(A.GEMM_ACCUM, a, b, out, bn=128, splits=splits, variant=3)
+        torch.cuda.synchronize()
+        _close(out, _ref(a, b), K, False)
+    rt.device_check()
+
+
+def test_swap_rejects_what_it_cannot_do(cuda_dev):
+    a, b = _mk((300, 256), 28, cuda_dev), _mk((256, 256), 29, cuda_dev)
+    h = torch.zeros((300, 256), device=cuda_dev)
+    with pytest.raises(Exception):            # more than 256 rows
+        rt.gemm_bf16(A.GEMM_RESID, a, b, h, bn=128, splits=1, variant=3)
+    out = torch.zeros((200, 256), device=cuda_dev, dtype=torch.bfloat16)
+    with pytest.raises(Exception):            # a bf16 store epilogue
+        rt.gemm_bf16(A.GEMM_STORE, a[:200], b, out, bn=128, splits=1, variant=3)
+    with pytest.raises(Exception):            # another tile width
+        rt.gemm_bf16(A.GEMM_RESID, a[:200], b, h[:200], bn=256, splits=1, variant=3)

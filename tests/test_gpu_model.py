@@ -146,7 +146,9 @@ def test_autotuned_step_matches_oracle(cuda_dev):
     for kind in range(5):
         for M in (1, 100, 257, 400):
             bn, sp, var = model.tuning(kind, M)
-            assert bn in (64, 128, 192, 256) and (sp >= 1 or sp == -1) and var in (0, 1, 2)
+            assert bn in (64, 128, 192, 256) and (sp >= 1 or sp == -1) and var in (0, 1, 2, 3)
+            # swapped operands only for projections in buckets of at most 256 rows
+            assert var != 3 or (kind != 4 and M <= 256 and bn == 128 and sp >= 1)
     act = rt.Active(B, n_ctx)
     tokens, positions, ck, cv = _state(shape, B, n_ctx, [160, 130], seed=11, dev=cuda_dev,
                                        dtype="bf16")
@@ -187,6 +189,45 @@ def test_pinned_tilings_step_matches_oracle(cuda_dev, tiling):
         model.set_tuning(4, M, 128, -1, 0)            # the LM head takes no K split
     act = rt.Active(B, n_ctx)
     tokens, positions, ck, cv = _state(shape, B, n_ctx, counts, seed=12, dev=cuda_dev, dtype="bf16")
+    act.load(positions)
+    _load_cache(cache, ck, cv, torch.bfloat16)
+    tok = torch.from_numpy(tokens).to(cuda_dev)
+    logits = torch.zeros((B * n_ctx, shape.vocab), device=cuda_dev, dtype=torch.bfloat16)
+    rt.step(model, cache, act, tok, logits)
+    torch.cuda.synchronize()
+    rt.device_check()
+    zs, ck2, cv2 = _oracle_step(shape, w64, tokens, positions, ck, cv, n_ctx)
+    lg = to64(logits)
+    for b in range(B):
+        err = np.abs(lg[positions[b] + b * n_ctx] - zs[b]).max()
+        assert err <= LOGIT_TOL["bf16"], err
+    model.close()
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+def test_swapped_operand_tilings_step_matches_oracle(cuda_dev, splits):
+    """Every projection GEMM pinned to the swapped-operand kernel (the weight
+    tile as the 128-row MMA operand, the 220 active rows as its N): Q|K|V and
+    gate/up through the fp32 workspace and their finishing kernels, the output
+    and down projections by reduce-add into the residual stream."""
+    shape = MINI_BF16
+    B, n_ctx = 2, 200
+    w_np = wl.np_weights(shape, seed=2, std=0.05, gain_jitter=0.1)
+    w_dev = weights_to_device(w_np, "bf16", cuda_dev)
+    w64 = weights_for_oracle(w_dev)
+    model = rt.Model(shape, w_dev, "bf16")
+    cache = rt.KVCache(model, B, n_ctx)
+    counts = [130, 90]
+    M = sum(counts)
+    for kind in range(4):
+        model.set_tuning(kind, M, 128, splits, 3)
+        assert model.tuning(kind, M) == (128, splits, 3)
+    with pytest.raises(RuntimeError):
+        model.set_tuning(4, M, 128, 1, 3)             # not for the LM head
+    with pytest.raises(RuntimeError):
+        model.set_tuning(0, 300, 128, 1, 3)           # a bucket above 256 rows
+    act = rt.Active(B, n_ctx)
+    tokens, positions, ck, cv = _state(shape, B, n_ctx, counts, seed=13, dev=cuda_dev, dtype="bf16")
     act.load(positions)
     _load_cache(cache, ck, cv, torch.bfloat16)
     tok = torch.from_numpy(tokens).to(cuda_dev)

@@ -576,14 +576,19 @@ struct Plan {
   int bn, splits, msub;
   double cost;
   int pair = 0;     // 1: CTA-pair kernel (2-SM MMA)
+  int swap = 0;     // 1: swapped operands (weights as the 128-row MMA operand, M <= 256)
 };
 
 // Kernel variant codes (sl_gemm_bf16, tuning tables): 0 = 1-SM 128-row units,
-// 1 = 1-SM 256-row units, 2 = CTA pair.
-static int plan_variant(const Plan &p) { return p.pair ? 2 : (p.msub == 2 ? 1 : 0); }
+// 1 = 1-SM 256-row units, 2 = CTA pair, 3 = swapped operands (bn 128, at most
+// 256 rows, fp32 reduce epilogues).
+static int plan_variant(const Plan &p) {
+  return p.swap ? 3 : p.pair ? 2 : (p.msub == 2 ? 1 : 0);
+}
 static void plan_set_variant(Plan &p, int v) {
   p.msub = v >= 1 ? 2 : 1;
   p.pair = v == 2 ? 1 : 0;
+  p.swap = v == 3 ? 1 : 0;
 }
 
 // Choose the tile shape (BN, 128 or 256 rows per unit) and K split of one
@@ -939,13 +944,18 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
   const sl_config &cfg = m->cfg;
   const int d = cfg.d_model, f = cfg.d_ffn, V = cfg.vocab, H = cfg.n_heads;
   const double Md = (double)M;
-  const bool split = pl.splits != 1;      // split K or stream-K: partial sums
+  // split K, stream-K or swapped operands: fp32 partial sums (the swapped
+  // kernel always leaves its tiles by reduce-add)
+  const bool split = pl.splits != 1 || pl.swap;
+  if (pl.swap && (kind == G_HD || M > 256 || pl.bn != 128))
+    return fail(SL_ERR_INVALID, "swapped-operand GEMM: projections of at most 256 rows, bn 128");
   TcGemmArgs g{};
   g.M = M;
   g.bn = pl.bn;
   g.splits = pl.splits;
   g.msub = pl.msub;
   g.pair = pl.pair;
+  g.swap = pl.swap;
   const int bbox = pl.pair ? pl.bn / 2 : pl.bn;    // weight rows per TMA box
   double bytes = 0, flops = 0;
   switch (kind) {
@@ -967,7 +977,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
         g.out = c->ws;
         g.ldo = 3 * d;
         g.OUT = &c->out_ws3;
-        if (gemm_fixup_enabled() && pl.bn % 128 == 0) {
+        if (gemm_fixup_enabled() && pl.bn % 128 == 0 && !pl.swap) {
           g.fix_ctr = c->fix_ctr;
           g.row_map = rows;
           g.rope = c->rope;
@@ -1026,7 +1036,7 @@ static sl_status run_gemm(sl_model *m, sl_kv_cache *c, const int32_t *rows, int 
       g.out = split ? (void *)c->ws : c->act;
       g.ldo = split ? 2 * f : f;
       g.OUT = split ? &c->out_ws2 : &c->out_act;
-      if (split && gemm_fixup_enabled()) {
+      if (split && gemm_fixup_enabled() && !pl.swap) {
         g.fix_ctr = c->fix_ctr;
         g.fix_act = c->act;
       }
@@ -1260,10 +1270,15 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   }
   if (M == 0) return SL_OK;
   const int ns = sm_count();
-  if (variant < 0 || variant > 2)
-    return fail(SL_ERR_INVALID, "sl_gemm_bf16: variant must be 0, 1 or 2");
+  if (variant < 0 || variant > 3)
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: variant must be 0, 1, 2 or 3");
   int msub = variant >= 1 ? 2 : 1;
   int pair = variant == 2 ? 1 : 0;
+  const int swap = variant == 3 ? 1 : 0;
+  if (swap && (M > 256 || bn != 128 || splits < 1 ||
+               (epi != SL_GEMM_RESID && epi != SL_GEMM_ACCUM)))
+    return fail(SL_ERR_INVALID, "sl_gemm_bf16: the swapped-operand kernel takes M <= 256, bn 128, "
+                                "splits >= 1 and the RESID or ACCUM epilogue");
   if (bn == 0) {
     Plan p = plan_gemm(M, N, K, epi == SL_GEMM_RESID ? SPLIT_RESID
                                 : epi == SL_GEMM_ACCUM ? SPLIT_ACCUM : SPLIT_NONE, ns, swiglu);
@@ -1305,6 +1320,7 @@ extern "C" sl_status sl_gemm_bf16(int epi, const void *d_a, int M, int K, const 
   g.row_map = d_row_map;
   g.msub = msub;
   g.pair = pair;
+  g.swap = swap;
   // TMA epilogue when the output rows qualify (16-byte row pitch)
   TmaMat mo;
   if (epi == SL_GEMM_RESID || epi == SL_GEMM_ACCUM) {
@@ -1433,6 +1449,19 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
           }
         }
       }
+      // swapped operands for buckets of at most 256 rows (projections only)
+      if (kind != G_HD && Mb <= 256 && N % 128 == 0 && (kind != G_GU || (N / 2) % 64 == 0)) {
+        int last_ss = 0;
+        for (int sp : split_opts) {
+          if (sp < 1 || sp > std::max(1, kblocks / 2)) continue;
+          const int kbp = (kblocks + sp - 1) / sp;
+          const int ss = (kblocks + kbp - 1) / kbp;
+          if (ss == last_ss) continue;
+          last_ss = ss;
+          if ((long)(N / 128) * ss > 24L * m->num_sms) continue;
+          cands[kind].push_back({128, ss, 3});
+        }
+      }
     }
     std::vector<std::vector<float>> times[G_KINDS];
     for (int kind = 0; kind < G_KINDS; ++kind)
@@ -1441,7 +1470,7 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
       if ((st = ensure_maps(c, pts[pi])) != SL_OK) break;
       for (int kind = 0; kind < G_KINDS && st == SL_OK; ++kind)
         for (size_t ci = 0; ci < cands[kind].size() && st == SL_OK; ++ci) {
-          Plan pl{cands[kind][ci][0], cands[kind][ci][1], cands[kind][ci][2] >= 1 ? 2 : 1, 0.0};
+          Plan pl{cands[kind][ci][0], cands[kind][ci][1], 1, 0.0};
           plan_set_variant(pl, cands[kind][ci][2]);
           st = time_plan(kind, pl, pts[pi], &times[kind][ci][pi]);
         }
@@ -1513,7 +1542,7 @@ extern "C" sl_status sl_model_set_attention_keys(sl_model *m, int key_tile) {
 
 extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, int splits,
                                          int variant) {
-  if (!m || kind < 0 || kind >= G_KINDS || M <= 0)
+  if (!m || kind < 0 || kind >= G_KINDS || M <= 0 || tune_bucket(M) < 0)
     return fail(SL_ERR_INVALID, "sl_model_set_tuning: bad argument");
   if (m->cfg.dtype != SL_BF16) return fail(SL_ERR_INVALID, "sl_model_set_tuning: bf16 models only");
   const int d = m->cfg.d_model, f = m->cfg.d_ffn, V = m->cfg.vocab;
@@ -1521,7 +1550,9 @@ extern "C" sl_status sl_model_set_tuning(sl_model *m, int kind, int M, int bn, i
   const int N = Ns[kind];
   if ((bn != 64 && bn != 128 && bn != 192 && bn != 256) || N % bn || (kind == G_GU && f % (bn / 2)) ||
       (kind == G_QKV && (bn < 128 || d % bn || (bn % 128 != 0 && splits == 1))) || variant < 0 ||
-      variant > 2 || (variant == 2 && bn < 128) ||
+      variant > 3 || (variant == 2 && bn < 128) ||
+      (variant == 3 && (bn != 128 || kind == G_HD || splits < 1 ||
+                        kTuneBounds[tune_bucket(M)] > 256)) ||
       (splits < 1 && splits != -1) || (kind == G_HD && splits != 1))
     return fail(SL_ERR_INVALID, "sl_model_set_tuning: tiling not valid for this GEMM");
   if (m->tuned[kind].empty())

@@ -810,6 +810,234 @@ __global__ void __launch_bounds__(192, 1) gemm_tc_kernel(const __grid_constant__
   }
 }
 
+// ------------------------------------------------ swapped-operand kernel ---
+// D^T = W X^T for few rows (M <= 256): the weight tile is the MMA's 128-row A
+// operand and the M active rows are its N dimension (rounded up to 32), so the
+// tensor-core work follows M instead of a 256-row padded tile.  TMEM then holds
+// output features on its lanes and rows on its columns; the epilogue reads 32
+// rows of a lane's feature at a time, writes them transposed into the warp's
+// 32-row x 128-byte staging box (same 128-byte swizzle as the other fp32
+// epilogues) and adds the box into the fp32 destination with a TMA reduce:
+// the residual stream (RESID) or a zeroed workspace whose finishing pass
+// (RoPE + cache scatter, SiLU(gate) * up) runs as its own kernel (ACCUM).
+// A stage holds the unit's two 128-row activation boxes (rows past M read as
+// zeros) and 128 weight rows (64 gate + 64 up rows for the gate/up GEMM).
+template <int STAGES>
+struct SwSmem {
+  static constexpr int A_BYTES = 2 * 128 * 64 * 2;     // 256 activation rows
+  static constexpr int B_BYTES = 128 * 64 * 2;         // 128 weight rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_OFF = STAGES * STAGE_BYTES;
+  static constexpr int BAR_OFF = EPI_OFF + EPI_STAGING_BYTES;
+  static constexpr int TOTAL = BAR_OFF + 256 + 1024;
+};
+
+template <int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1) gemm_swap_kernel(const __grid_constant__ TcParams p) {
+  using L = SwSmem<STAGES>;
+  constexpr int ACC_COLS = 256;                        // up to 256 rows per accumulator
+  constexpr uint32_t TMEM_COLS = 512;                  // two accumulators
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s_addr(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
+  const uint32_t bar0 = s_addr(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::BAR_OFF + 8 * (2 * STAGES + 5));
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int np = min(256, (p.M + 31) & ~31);           // MMA N: rows rounded up to 32
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    tma_prefetch_desc(&p.a);
+    tma_prefetch_desc(&p.b[0]);
+  }
+  __syncthreads();
+  uint32_t tmem_base = 0;
+  if (warp >= 1) {
+    if (warp == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       s_addr(tmem_slot)),
+                   "r"(TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    named_bar_sync(1, 160);
+    tc_fence_after();
+    tmem_base = *tmem_slot;
+  }
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      // the first unit's weight tiles before the wait on the previous kernel
+      int npre = 0;
+      WorkIter first_it(p, blockIdx.x, gridDim.x);
+      int mt, nt, kb0, kb1;
+      if (first_it.next(p, mt, nt, kb0, kb1)) {
+        npre = min(STAGES, kb1 - kb0);
+        for (int i = 0; i < npre; ++i) {
+          mbar_expect_tx(full_bar(i), L::STAGE_BYTES);
+          load_b<128>(p, sbase + i * L::STAGE_BYTES + L::A_BYTES, nt, kb0 + i, full_bar(i));
+        }
+      }
+      pdl_wait();
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_stage = -1;
+      uint32_t last_phase = 0;
+      bool ok = true, first = true;
+      WorkIter it(p, blockIdx.x, gridDim.x);
+      while (ok && it.next(p, mt, nt, kb0, kb1)) {
+        for (int kb = kb0; kb < kb1; ++kb) {
+          const bool pre = first && (kb - kb0) < npre;
+          if (!pre) {
+            if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(full_bar(stage), L::STAGE_BYTES);
+          }
+          const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          tma_load_2d(sa, &p.a, kb * 64, 0, full_bar(stage));
+          tma_load_2d(sa + 16384, &p.a, kb * 64, 128, full_bar(stage));
+          if (!pre) load_b<128>(p, sa + L::A_BYTES, nt, kb, full_bar(stage));
+          last_stage = stage;
+          last_phase = phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        first = false;
+      }
+      pdl_trigger();
+      if (!ok) {
+        atomicExch(p.err, DEV_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+      }
+      if (last_stage >= 0) {
+        volatile int never = 0;
+        mbar_wait(full_bar(last_stage), last_phase, &never, p.wait_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------------------------- MMA
+    if (lane == 0) {
+      // M = 128 weight rows, N = np activation rows (a multiple of 32 <= 256)
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(np >> 3) << 17) |
+                             ((uint32_t)(128 >> 4) << 24);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      WorkIter it(p, blockIdx.x, gridDim.x);
+      int mt, nt, kb0, kb1;
+      while (ok && it.next(p, mt, nt, kb0, kb1)) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = sbase + stage * L::STAGE_BYTES;
+          const uint64_t wdesc = smem_desc_sw128(sa + L::A_BYTES);   // weights: the A operand
+          const uint64_t xdesc = smem_desc_sw128(sa);                // rows: the B operand
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc_mma(d_tmem, wdesc + 2 * k, xdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) {
+        atomicExch(p.err, DEV_TIMEOUT_MMA);
+        *abort_flag = 1;
+      }
+      tc_commit(drain_bar);
+      volatile int never = 0;
+      mbar_wait(drain_bar, 0, &never, p.wait_ns);
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    pdl_wait();
+    const int q = warp & 3;                 // TMEM lane quarter: features q*32 .. q*32+31
+    const uint32_t stg = sbase + L::EPI_OFF + q * 4096;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    WorkIter it(p, blockIdx.x, gridDim.x);
+    int mt, nt, kb0, kb1;
+    while (it.next(p, mt, nt, kb0, kb1)) {
+      if (!mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.wait_ns)) { ok = false; break; }
+      tc_fence_after();
+      // destination column of this warp's 32 features
+      int col = nt * 128 + q * 32;
+      if (p.b_swiglu) {                     // gate features into [0, F), up into [F, 2F)
+        const int f0 = nt * 64;
+        col = q < 2 ? f0 + q * 32 : p.ffn + f0 + (q - 2) * 32;
+      }
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * ACC_COLS) + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int r0 = 0; r0 < np && r0 < p.M; r0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + r0, v);            // rows r0 .. r0+31 of this lane's feature
+        stage_wait(lane);
+        // element (row i, feature lane) of the 32 x 32 fp32 box: 16-byte chunk
+        // lane / 4 of row i, swizzled by row i % 8
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          asm volatile("st.shared.f32 [%0], %1;" ::"r"(stg + i * 128 +
+                                                         ((((uint32_t)lane >> 2) ^ (i & 7)) << 4) +
+                                                         ((lane & 3) << 2)),
+                       "f"(v[i])
+                       : "memory");
+        stage_done();
+        if (lane == 0) {
+          tma_reduce_add_2d(&p.out_map, col, r0, stg);
+          bulk_commit();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (lane == 0) bulk_wait0();
+    if (!ok && lane == 0) {
+      atomicExch(p.err, DEV_TIMEOUT_EPI);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------ CTA-pair kernel ---
 // The same GEMM with 2-SM tensor-core instructions: a cluster of two CTAs
 // computes a 256 x BN tile; each CTA stages its own 128 rows of A and its half
@@ -1053,6 +1281,19 @@ static cudaError_t run_tc2(const TcParams &p, int pairs, cudaStream_t s) {
   return launch_k_cluster2(gemm_tc2_kernel<BN, STAGES, EPI>, 2 * pairs, 192, SMEM, s, p);
 }
 
+template <int STAGES, int EPI>
+static cudaError_t run_swap(const TcParams &p, int grid, cudaStream_t s) {
+  using L = SwSmem<STAGES>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_swap_kernel<STAGES, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::TOTAL);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  return launch_k(gemm_swap_kernel<STAGES, EPI>, grid, 192, L::TOTAL, s, p);
+}
+
 template <int BN, int STAGES>
 static cudaError_t run_epi2(int epi, const TcParams &p, int pairs, cudaStream_t s) {
   switch (epi) {
@@ -1082,6 +1323,44 @@ static cudaError_t run_epi(int epi, const TcParams &p, int grid, cudaStream_t s)
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
   const int bn = a.bn;
+  if (a.swap) {
+    // swapped operands: 128 weight rows per tile, at most 256 rows, the fp32
+    // reduce epilogues only (no fix-up, no stream-K)
+    if (bn != 128 || a.M > 256 || a.K % 64 != 0 || a.N % 128 != 0 || a.pair || a.fix_ctr ||
+        (a.epi != EPI_RESID && a.epi != EPI_ACCUM) || !a.OUT || a.splits < 1)
+      return cudaErrorInvalidValue;
+    if (a.b_swiglu && (a.N % 2 != 0 || (a.N / 2) % 64 != 0)) return cudaErrorInvalidValue;
+    TcParams p;
+    memset(&p, 0, sizeof(p));
+    p.a = a.A->map;
+    for (int i = 0; i < 3; ++i)
+      if (a.B[i]) p.b[i] = a.B[i]->map;
+    p.b_swiglu = a.b_swiglu ? 1 : 0;
+    p.seg0 = a.n_seg[0];
+    p.seg1 = a.n_seg[0] + a.n_seg[1];
+    if (!a.b_swiglu && p.seg0 == 0) p.seg0 = a.N;
+    if (p.seg1 < p.seg0) p.seg1 = p.seg0;
+    p.M = a.M;
+    p.N = a.N;
+    p.K = a.K;
+    p.m_tiles = 1;
+    p.n_tiles = a.N / 128;
+    p.kblocks = a.K / 64;
+    int splits = a.splits > p.kblocks ? p.kblocks : a.splits;
+    p.kb_per_split = (p.kblocks + splits - 1) / splits;
+    p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
+    p.units = p.n_tiles * p.splits;
+    p.out_map = a.OUT->map;
+    p.tma_out = 1;
+    p.out = a.out;
+    p.ldo = a.ldo;
+    p.ffn = a.N / 2;
+    p.err = err;
+    p.wait_ns = a.wait_ns ? a.wait_ns : WAIT_LIMIT_NS;
+    const int grid = p.units < num_sms ? p.units : num_sms;
+    return a.epi == EPI_RESID ? run_swap<4, EPI_RESID>(p, grid, s)
+                              : run_swap<4, EPI_ACCUM>(p, grid, s);
+  }
   if ((bn != 64 && bn != 128 && bn != 192 && bn != 256) || a.K % 64 != 0 || a.N % bn != 0)
     return cudaErrorInvalidValue;
   const bool swiglu_b = a.b_swiglu != 0;

@@ -193,6 +193,9 @@ struct TcGemmArgs {
   // q_out, ck, cv; gate/up writes SiLU(gate) * up to fix_act [M][N / 2]
   unsigned int *fix_ctr;
   void *fix_act;
+  // swapped operands (M <= 256, bn = 128, RESID / ACCUM): the weight tile is the
+  // MMA's 128-row operand and the M rows its N dimension (gemm_swap_kernel)
+  int swap;
 };
 cudaError_t launch_gemm_tc(const TcGemmArgs &a, int num_sms, int *err, cudaStream_t s);
 

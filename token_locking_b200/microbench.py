@@ -328,15 +328,18 @@ def bench_gemm(args, dev):
                     continue
                 if sp != 1 and name == "head":
                     continue
+                if variant == 3 and (M > 256 or bn != 128 or sp < 1 or name == "head"):
+                    continue                     # swapped operands: few rows, 128 weight rows
                 if True:
+                    acc = sp != 1 or variant == 3  # fp32 partial sums (split K, swapped operands)
                     if name == "gu":
-                        epi, b, b2, out = ((A.GEMM_SWIGLU, wg, wu, outa) if sp == 1 else
-                                           (A.GEMM_ACCUM, wg, wu, outf))
+                        epi, b, b2, out = ((A.GEMM_ACCUM, wg, wu, outf) if acc else
+                                           (A.GEMM_SWIGLU, wg, wu, outa))
                     elif name in ("o", "down"):
                         epi, b, b2, out = A.GEMM_RESID, weights[name], None, outf
                     else:
-                        epi, b, b2, out = ((A.GEMM_STORE, weights[name], None, outb) if sp == 1
-                                           else (A.GEMM_ACCUM, weights[name], None, outf))
+                        epi, b, b2, out = ((A.GEMM_ACCUM, weights[name], None, outf) if acc
+                                           else (A.GEMM_STORE, weights[name], None, outb))
 
                     def fn():
                         rt.gemm_bf16(epi, a, b, out, b2=b2, bn=bn, splits=sp, variant=variant)
