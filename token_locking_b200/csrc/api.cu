@@ -1449,8 +1449,12 @@ extern "C" sl_status sl_model_autotune(sl_model *m, sl_kv_cache *c, int max_rows
           }
         }
       }
-      // swapped operands for buckets of at most 256 rows (projections only)
-      if (kind != G_HD && Mb <= 256 && N % 128 == 0 && (kind != G_GU || (N / 2) % 64 == 0)) {
+      // swapped operands for buckets of at most 256 rows, for the projections
+      // that add into the residual stream (output, down): Q|K|V and gate/up
+      // would need their finishing pass as a kernel of its own, whose launch
+      // boundary costs more in the decode than the swap saves (sl_gemm_bf16
+      // and sl_model_set_tuning still take them)
+      if ((kind == G_O || kind == G_DN) && Mb <= 256 && N % 128 == 0) {
         int last_ss = 0;
         for (int sp : split_opts) {
           if (sp < 1 || sp > std::max(1, kblocks / 2)) continue;
