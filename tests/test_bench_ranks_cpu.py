@@ -185,3 +185,47 @@ def test_bench_step_unit():
     assert bench.aux_decodes(20, 19600.0) == 1
     assert bench.aux_decodes(20, 1250.0) == 16
     assert bench.aux_decodes(2, 100.0) == 2
+
+
+def _bench_args(**kw):
+    import types
+    base = dict(gpus=1, steps=1, warmup=0, impl="reference", workload="long8b", bench_step="auto",
+                eps=None, scripted=False, batch=None, gate_q=None, ablation="none",
+                head_fusion="on", no_cpu_baseline=False)
+    base.update(kw)
+    return types.SimpleNamespace(**base)
+
+
+def test_reference_arm_finds_the_stored_trajectory():
+    """The reference arm weighs its oracle samples by the M_t trajectory a GPU
+    run of the same workload recorded (profiles/trajectory_*.json): one per
+    stored workload, as long as the decode, starting from every row active and
+    never growing."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import numpy as np
+    for kw in ({}, {"workload": "full8b", "eps": 0.05}, {"workload": "full8b", "eps": 0.0},
+               {"workload": "full8b", "eps": 0.01}, {"workload": "full8b", "eps": 0.05,
+                                                      "scripted": True}):
+        a = _bench_args(**kw)
+        setup = bench.setup_from_args(a)
+        got = bench.stored_trajectory(bench.workload_config(a, setup, 1)["workload"])
+        assert got is not None, kw
+        traj, name = got
+        assert len(traj) == setup.steps, (kw, name)
+        assert traj[0] == setup.batch * setup.n_ctx
+        assert np.all(np.diff(traj) <= 0) and traj[-1] >= 1
+    # a workload no GPU run recorded has none
+    a = _bench_args(workload="full8b", eps=0.2)
+    setup = bench.setup_from_args(a)
+    assert bench.stored_trajectory(bench.workload_config(a, setup, 1)["workload"]) is None
+
+
+def test_head_fusion_arm_is_named_in_the_workload():
+    sys.path.insert(0, ROOT)
+    import bench
+    on, off = _bench_args(), _bench_args(head_fusion="off")
+    setup = bench.setup_from_args(on)
+    w_on = bench.workload_config(on, setup, 1)["workload"]
+    w_off = bench.workload_config(off, setup, 1)["workload"]
+    assert w_on != w_off and "separate pass" in w_off and "separate pass" not in w_on

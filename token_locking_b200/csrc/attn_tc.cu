@@ -27,14 +27,16 @@
 //               into one of two P buffers, so the P V product of tile t runs
 //               while the exponentials of tile t + 1 are taken, and the
 //               product reads P from TMEM, sparing shared memory the P traffic.
-// What bounds the kernel is the K/V feed: a CTA reads BN keys and values of
-// 256 bytes each per BN x 128 x QT x 128 x 4 FLOP, and with one query tile per
-// CTA the 148 SMs together pull about 7 TB/s from L2 at half the tensor peak.
-// Two query tiles per CTA (QT = 2) share every K/V tile, halving those bytes
-// per FLOP, and the two softmax warpgroups take turns with the tensor cores:
-// while one computes its exponentials the MMA warp runs the other's products.
-// TMEM then holds one score buffer per query tile (64-key tiles): the scores of
-// tile t + 1 are issued as soon as the softmax has loaded those of tile t.
+// What bounds one CTA is latency, not a pipe or a memory path: every key tile
+// passes from the TMA producer to the MMA warp (scores), to the softmax
+// warpgroup (P), and back to the MMA warp (P V), about a microsecond of
+// handoffs per tile whatever the work in it; a CTA also spends ~6 us starting
+// (TMEM, first copies) and draining (O out).  So the default layout is small
+// enough for two CTAs per SM, which then run two independent tile chains that
+// hide each other's handoffs, start-up and drain.  Two query tiles per CTA
+// (QT = 2) share every K/V tile instead, halving the K/V bytes per FLOP, with
+// one score buffer per query tile (64-key tiles): the scores of tile t + 1 are
+// issued as soon as the softmax has loaded those of tile t.
 // A K/V stage is released only when the P V products of its tile have
 // completed, so the copy of tile t + ST starts then and must land before the
 // scores of that tile can be issued: the ring is deep enough to cover the TMA
