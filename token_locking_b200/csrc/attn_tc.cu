@@ -568,10 +568,13 @@ struct TaLayout {
   double c_unit;        // us per 128 x 128 block of work of one CTA at the power-capped clock
 };
 // measured on batch 4 x 512 and 2048 queries over 2048 keys; a CTA's start-up
-// (first Q/K/V copies, TMEM allocation) and drain (O out) cost ~6 us, and a key
-// split as much again (partial rows out and back, the merge)
+// (first Q/K/V copies, TMEM allocation) and drain (O out) cost ~6 us; a key
+// split costs as much again plus its partial rows: every split of every query
+// row and head writes 128 fp32 values and the merge reads them back, at an
+// effective ~1.8 TB/s (measured: two splits take 91 / 134 / 245 us at batch 4 x
+// 256 / 384 / 768 queries against 46 / 85 / 126 us unsplit)
 constexpr TaLayout kTaLayouts[] = {{1, 128, 1, 1.3}, {1, 64, 2, 2.2}, {2, 64, 1, 1.9}};
-constexpr double kTaCtaFixed = 6.0, kTaSplitCost = 6.0;
+constexpr double kTaCtaFixed = 6.0, kTaSplitCost = 6.0, kTaSplitBytesPerUs = 1.8e6;
 }  // namespace
 
 AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sms,
@@ -591,6 +594,8 @@ AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sm
     }
     if (units == 0) return best;
     const double fill = (double)tiles / ((double)units * qt);   // query tiles present per slot
+    long rows = 0;                                              // query rows of the launch
+    for (int b = 0; b < seqs.batch; ++b) rows += seqs.seq_count[b];
     const int max_sp = std::min(ktiles, std::min(max_splits, 16));
     for (int req = 1; req <= max_sp; ++req) {
       // a requested split rounds to the count that covers the key tiles evenly
@@ -602,7 +607,9 @@ AttnTcPlan attn_tc_plan(const AttnSeqs &seqs, int n_heads, int n_ctx, int num_sm
       const long ctas = (long)units * n_heads * sp;
       const long waves = (ctas + (long)num_sms * ly.per_sm - 1) / ((long)num_sms * ly.per_sm);
       const double work = (double)per * bn / 128.0 * qt * fill;
-      const double t = waves * (kTaCtaFixed + ly.c_unit * work) + (sp > 1 ? kTaSplitCost : 0.0);
+      const double split_bytes = sp > 1 ? (double)rows * n_heads * sp * TA_D * 4.0 * 2.0 : 0.0;
+      const double t = waves * (kTaCtaFixed + ly.c_unit * work) +
+                       (sp > 1 ? kTaSplitCost + split_bytes / kTaSplitBytesPerUs : 0.0);
       if (t < best_t * 0.97) {                 // a clear gain, else the earlier layout
         best_t = t;
         best.qt = qt;
