@@ -159,11 +159,15 @@ class State:
     ck: np.ndarray            # [B, L, N, d]
     cv: np.ndarray            # [B, L, N, d]
     lp_prev: np.ndarray       # [B, N, V]  last posterior (frozen p_hat for locked rows)
+    # mask flags at the start of the previous step (K/V reuse: a row unmasked
+    # during that step is computed once more before it can be reused)
+    masked_before: Optional[np.ndarray] = None
 
     def copy(self) -> "State":
         return State(self.tokens.copy(), self.masked.copy(), [a.copy() for a in self.act],
                      self.locked.copy(), self.lock_t.copy(), self.has_prev.copy(),
-                     self.ck.copy(), self.cv.copy(), self.lp_prev.copy())
+                     self.ck.copy(), self.cv.copy(), self.lp_prev.copy(),
+                     None if self.masked_before is None else self.masked_before.copy())
 
 
 def init_state(shape, tokens: np.ndarray, masked: np.ndarray, dtype=np.float64) -> State:
@@ -177,7 +181,8 @@ def init_state(shape, tokens: np.ndarray, masked: np.ndarray, dtype=np.float64) 
                  lock_t=np.full((B, N), -1, dtype=np.int32),
                  has_prev=np.zeros((B, N), dtype=bool),
                  ck=np.zeros((B, L, N, d), dtype=dtype), cv=np.zeros((B, L, N, d), dtype=dtype),
-                 lp_prev=np.zeros((B, N, V), dtype=dtype))
+                 lp_prev=np.zeros((B, N, V), dtype=dtype),
+                 masked_before=masked.astype(bool).copy())
 
 
 def lock_test(lp: np.ndarray, lp_prev: np.ndarray, has_prev: np.ndarray,
@@ -210,29 +215,52 @@ def step(shape, w: dict, st: State, setup, t: int, record_block_inputs: bool = F
     current block -> record p_t for the active rows (frozen for those that lock)
     -> remove the locked rows from A_t.  Returns one record per sequence.
     Paper-Notes, "Method: overall framework" (compute A_t, serve L_t from the
-    cache) and "permanent locking" (a locked row's posterior is frozen)."""
+    cache) and "permanent locking" (a locked row's posterior is frozen).
+
+    With setup.kv_reuse = R > 1 (the pages' composition with cross-step K/V
+    reuse, Paper-Notes "loss / training strategy" and "key results": orthogonal
+    and stackable; the scheme itself is this restatement's reading) the forward
+    runs on all of A_t only when t mod R = 0.  Between those refresh steps it
+    runs on the active rows that are masked or were masked at the start of the
+    previous step; the other active rows keep their cached K/V and their last
+    posterior, are not tested, and stay active."""
     out = []
     lo, hi = setup.block_bounds(t)
+    R = getattr(setup, "kv_reuse", 1)
+    if R > 1 and (setup.scripted or setup.no_kv_cache):
+        # the scripted lock count is defined over the whole active set, and the
+        # no-cache ablation has no stale K/V to reuse
+        raise ValueError("K/V reuse composes with the sure test on the full cache only")
+    refresh = R <= 1 or t % R == 0
+    if st.masked_before is None:
+        st.masked_before = st.masked.copy()
+    masked_start = st.masked.copy()
     for b in range(st.tokens.shape[0]):
         A = st.act[b]
+        # the rows computed this step: all of A_t, or, between refresh steps of
+        # the K/V reuse, its masked rows and the rows unmasked during the
+        # previous step (reading: composition with K/V reuse for active rows)
+        C = A if refresh else A[st.masked[b, A] | st.masked_before[b, A]]
         blk = [] if record_block_inputs else None
-        z = om.forward_active(shape, w, st.tokens[b], A, st.ck[b], st.cv[b], blk,
+        z = om.forward_active(shape, w, st.tokens[b], C, st.ck[b], st.cv[b], blk,
                               setup.no_kv_cache)
         lp = log_softmax(z)
-        masked_rows = st.masked[b, A].copy()
-        rec = lock_test(lp, st.lp_prev[b, A], st.has_prev[b, A], masked_rows, A,
+        masked_rows = st.masked[b, C].copy()
+        rec = lock_test(lp, st.lp_prev[b, C], st.has_prev[b, C], masked_rows, C,
                         shape, setup, t)
-        sel = unmask_select(A, rec["conf"], masked_rows, lo, hi, setup.tokens_per_step)
-        st.tokens[b, A[sel]] = rec["pred"][sel]
-        st.masked[b, A[sel]] = False
-        st.lp_prev[b, A] = lp
-        st.has_prev[b, A] = True
+        sel = unmask_select(C, rec["conf"], masked_rows, lo, hi, setup.tokens_per_step)
+        st.tokens[b, C[sel]] = rec["pred"][sel]
+        st.masked[b, C[sel]] = False
+        st.lp_prev[b, C] = lp
+        st.has_prev[b, C] = True
         lk = rec["lock"]
-        st.locked[b, A[lk]] = True
-        st.lock_t[b, A[lk]] = t
-        st.act[b] = compact(A, lk)
-        rec.update({"z": z, "lp": lp, "pos": A, "unmasked": A[sel], "block_inputs": blk})
+        st.locked[b, C[lk]] = True
+        st.lock_t[b, C[lk]] = t
+        st.act[b] = compact(A, np.isin(A, C[lk]))
+        rec.update({"z": z, "lp": lp, "pos": C, "active": A, "unmasked": C[sel],
+                    "block_inputs": blk})
         out.append(rec)
+    st.masked_before = masked_start
     return out
 
 

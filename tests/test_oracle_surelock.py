@@ -361,3 +361,113 @@ def test_no_kv_cache_sampler_departs_only_after_the_first_lock():
             break
         assert np.all(np.diff(st_b.act[0]) > 0)
     assert first_lock is not None
+
+
+# ---- composition with K/V reuse for the active rows (refresh interval R) ----
+
+def _reuse_state_trace(cfg, w, tok, msk):
+    """Run the decode step by step; per step the active set and mask flags at
+    its start, the record, and snapshots of the cache and posteriors."""
+    st = sl.init_state(cfg.shape, tok, msk)
+    out = []
+    for t in range(cfg.steps):
+        snap = (st.act[0].copy(), st.masked[0].copy(), st.locked[0].copy(),
+                st.ck.copy(), st.cv.copy(), st.lp_prev.copy())
+        rec = sl.step(cfg.shape, w, st, cfg, t, record_block_inputs=True)[0]
+        out.append((snap, rec))
+    return st, out
+
+
+@pytest.mark.parametrize("R", [2, 3])
+def test_kv_reuse_computed_rows_and_frozen_rows(R):
+    """Between refresh steps (t mod R != 0) only the active rows that are masked,
+    or were masked at the start of the previous step, are computed; every other
+    active row keeps its cached K/V and its last posterior bitwise, and only
+    computed rows can lock.  Refresh steps compute all of A_t."""
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    c = dataclasses.replace(cfg, kv_reuse=R)
+    st, trace = _reuse_state_trace(c, w, tok, msk)
+    prev_mask = msk[0].astype(bool)
+    n_reused = n_locks = 0
+    for t, ((A, mask0, locked0, ck0, cv0, lp0), rec) in enumerate(trace):
+        C = rec["pos"]
+        np.testing.assert_array_equal(rec["active"], A)
+        if t % R == 0:
+            np.testing.assert_array_equal(C, A)
+        else:
+            np.testing.assert_array_equal(C, A[mask0[A] | prev_mask[A]])
+            assert set(np.nonzero(mask0)[0].tolist()) <= set(C.tolist())
+        reused = np.setdiff1d(A, C)
+        n_reused += len(reused)
+        nxt = trace[t + 1][0] if t + 1 < len(trace) else (st.act[0], st.masked[0], st.locked[0],
+                                                             st.ck, st.cv, st.lp_prev)
+        for p in reused:
+            np.testing.assert_array_equal(nxt[3][0, :, p], ck0[0, :, p])
+            np.testing.assert_array_equal(nxt[4][0, :, p], cv0[0, :, p])
+            np.testing.assert_array_equal(nxt[5][0, p], lp0[0, p])
+        # the computed rows' cache entries are those of this step's block inputs
+        for l in range(c.shape.n_layers):
+            k, v = om.kv_of_block_input(c.shape, w["layers"][l], rec["block_inputs"][l], C)
+            np.testing.assert_array_equal(k, nxt[3][0, l, C])
+            np.testing.assert_array_equal(v, nxt[4][0, l, C])
+        # locks: among computed rows only, never on a row masked at the step's start
+        new_locks = np.nonzero(nxt[2] & ~locked0)[0]
+        np.testing.assert_array_equal(new_locks, C[rec["lock"]])
+        assert not np.any(mask0[new_locks])
+        np.testing.assert_array_equal(nxt[0], np.setdiff1d(A, new_locks))
+        n_locks += len(new_locks)
+        prev_mask = mask0
+    assert n_reused > 20 and n_locks > 10       # both mechanisms are exercised
+    assert not np.any(st.tokens == c.shape.mask_id)
+
+
+@pytest.mark.parametrize("R", [2, 3, 7])
+def test_kv_reuse_is_exact_for_a_single_block(R):
+    """With one block a row's K/V depend on its own token and position only, and
+    an unmasked token never changes, so a row recomputed once after its
+    unmasking has exact K/V from then on.  Reuse (like locking) then changes no
+    decision: the decode's tokens are those of the sampler without locking.
+    A computed set that missed the rows unmasked in the previous step would
+    leave their mask-token K/V in the cache and change the tokens."""
+    import dataclasses
+    shape1 = dataclasses.replace(wl.TINY, n_layers=1)
+    c = dataclasses.replace(wl.CFG_TINY, shape=shape1, kv_reuse=R, eps=0.05)
+    w = om.cast_weights(wl.np_weights(shape1, seed=0, std=0.2), np.float64)
+    pr = wl.np_prompts(c.batch, c.prompt_len, shape1.vocab, shape1.mask_id)
+    tok, msk = wl.initial_tokens(pr, c.gen_len, shape1.mask_id)
+    t_reuse = sl.surelock_sampler(shape1, w, tok, msk, c)[0]
+    t_plain = sl.plain_sampler(shape1, w, tok, msk, c)[0]
+    np.testing.assert_array_equal(t_reuse, t_plain)
+
+
+def test_kv_reuse_is_an_approximation_with_two_blocks():
+    """With two blocks the second block's K/V of a reused row depend on the
+    other rows, so the first step between refreshes already departs from the
+    recomputing sampler on the rows it does compute; R = 1 is SureLock."""
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    st1 = sl.init_state(cfg.shape, tok, msk)
+    st2 = sl.init_state(cfg.shape, tok, msk)
+    st3 = sl.init_state(cfg.shape, tok, msk)
+    c2 = dataclasses.replace(cfg, kv_reuse=2)
+    c1 = dataclasses.replace(cfg, kv_reuse=1)
+    for t in range(2):
+        r1 = sl.step(cfg.shape, w, st1, cfg, t)[0]
+        r2 = sl.step(cfg.shape, w, st2, c2, t)[0]
+        r3 = sl.step(cfg.shape, w, st3, c1, t)[0]
+        np.testing.assert_array_equal(r1["lp"], r3["lp"])
+    C = r2["pos"]
+    assert len(C) < len(r1["pos"])
+    j = np.searchsorted(r1["pos"], C)
+    assert np.abs(r1["lp"][j] - r2["lp"]).max() > 1e-6
+
+
+def test_kv_reuse_rejects_the_scripted_schedule_and_the_no_cache_ablation():
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    for kw in ({"scripted": True}, {"no_kv_cache": True}):
+        c = dataclasses.replace(cfg, kv_reuse=2, **kw)
+        st = sl.init_state(cfg.shape, tok, msk)
+        with pytest.raises(ValueError):
+            sl.step(cfg.shape, w, st, c, 0)

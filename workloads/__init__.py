@@ -76,6 +76,10 @@ class SamplerSetup:
     # see the active rows' keys only (locked rows' cached K/V unused)
     gate_only: bool = False
     no_kv_cache: bool = False
+    # K/V reuse for active rows, refresh interval R (1 = off): between refresh
+    # steps the active rows that are neither masked nor just unmasked are not
+    # recomputed; their cached K/V and last posterior stand in for them
+    kv_reuse: int = 1
 
     @property
     def n_ctx(self) -> int:
