@@ -30,6 +30,7 @@ region is bracketed by barriers and the max over ranks is taken.
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload full8b|long8b] [--eps E] [--scripted] [--batch B]
                   [--gate-q Q] [--ablation none|no_kv_cache|gate_only] [--head-fusion on|off]
+                  [--kv-reuse R]
 """
 from __future__ import annotations
 
@@ -66,10 +67,12 @@ def load_peaks():
 
 # ------------------------------------------------------------- workload ---
 def make_setup(name: str, eps, scripted: bool, batch=None, gate_q=None,
-               ablation: str = "none") -> wl.SamplerSetup:
+               ablation: str = "none", kv_reuse: int = 1) -> wl.SamplerSetup:
     """The workload's decode; `batch` (1..64 sequences per GPU) overrides its batch,
     `gate_q` its confidence gate, and `ablation` selects one of the pages'
-    ablations (no_kv_cache, gate_only) instead of the method itself."""
+    ablations (no_kv_cache, gate_only) instead of the method itself; `kv_reuse`
+    R > 1 composes the method with K/V reuse for the active rows (all active
+    rows recomputed every R steps)."""
     if name == "full8b":
         s = wl.cfg_full8b(eps=0.05 if eps is None else eps, scripted=scripted)
     elif name == "long8b":
@@ -94,13 +97,19 @@ def make_setup(name: str, eps, scripted: bool, batch=None, gate_q=None,
         raise SystemExit("--ablation gate_only needs the confidence gate (--gate-q in [0, 1])")
     s = dataclasses.replace(s, no_kv_cache=ablation == "no_kv_cache",
                             gate_only=ablation == "gate_only")
+    if kv_reuse < 1:
+        raise SystemExit(f"--kv-reuse must be >= 1, got {kv_reuse}")
+    if kv_reuse > 1 and (s.scripted or s.no_kv_cache):
+        raise SystemExit("--kv-reuse composes with the sure test on the full cache only "
+                         "(not with --scripted or --ablation no_kv_cache)")
+    s = dataclasses.replace(s, kv_reuse=kv_reuse)
     s.validate()
     return s
 
 
 def setup_from_args(args) -> wl.SamplerSetup:
     return make_setup(args.workload, args.eps, args.scripted, args.batch, args.gate_q,
-                      args.ablation)
+                      args.ablation, getattr(args, "kv_reuse", 1))
 
 
 DATA_DESC = "synthetic (random-init N(0,0.02) weights, uniform random prompt ids)"
@@ -119,7 +128,9 @@ def workload_config(args, setup: wl.SamplerSetup, world: int) -> dict:
                            if setup.no_kv_cache else "")
                         + (", ablation: confidence gate only" if setup.gate_only else "")
                         + (", sure-test statistics in a separate pass after the LM head"
-                           if getattr(args, "head_fusion", "on") == "off" else ""),
+                           if getattr(args, "head_fusion", "on") == "off" else "")
+                        + (f", K/V reuse for active rows (all recomputed every "
+                           f"{setup.kv_reuse} steps)" if setup.kv_reuse > 1 else ""),
             "bench_step": (f"one full decode ({T} denoising steps)"
                            if bench_unit_steps(args, setup) == T else
                            f"one semi-autoregressive block ({setup.steps_per_block} denoising "
@@ -398,6 +409,8 @@ def run_ours(args, rank: int, world: int):
     model.set_head_fusion(args.head_fusion == "on")
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, T, setup.block_len,
                    setup.tokens_per_step, setup.eps, setup.gate_q, setup.scripted)
+    if setup.kv_reuse > 1:
+        s.set_kv_reuse(setup.kv_reuse)
     prompts = wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab, shape.mask_id,
                             seed=replica_prompt_seed(rank))
     d_prompts = torch.from_numpy(prompts).to(dev)
@@ -484,6 +497,17 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     step_ms = np.array([evs[t].elapsed_time(evs[t + 1]) for t in range(T)])
     traj2 = trajectory_from_lock_t(s.state()["lock_t"].cpu().numpy(), T)
+    # the rows each step's forward runs on: M_t, or with K/V reuse the computed
+    # rows between refreshes (read per step from one more untimed decode)
+    rows_t, rows_t2 = traj, traj2
+    if setup.kv_reuse > 1:
+        s.start(d_prompts)
+        got = []
+        for t in range(T):
+            m_act = sum(s.state()["active"].counts())
+            s.step()
+            got.append(m_act if t % setup.kv_reuse == 0 else sum(s.state()["computed"].counts()))
+        rows_t = rows_t2 = np.array(got)
 
     # end to end: host prompts -> host tokens through the public call
     h_prompts = torch.from_numpy(prompts).pin_memory()
@@ -507,16 +531,17 @@ def run_ours(args, rank: int, world: int):
         value = aggregate_rate(world, timed_steps, ms)
         e2e_value = aggregate_rate(world, aux * T, e2e_ms)
         gen_tokens = world * timed_steps * setup.batch * setup.tokens_per_step
-        # per-step roofline over the timed steps' own M_t (the timed region
-        # starts at step 0 of a decode), burst peaks
+        # per-step roofline over the rows the timed steps compute (M_t, or the
+        # computed rows under K/V reuse; the timed region starts at step 0 of a
+        # decode), burst peaks
         pf = peaks["bf16_tflops"] * 1e12
         pb = peaks["hbm_gbs"] * 1e9
         roof_t = [max(fl / pf, by / pb) for fl, by in
-                  (step_work(shape, int(m), setup.batch, setup.n_ctx) for m in traj)]
+                  (step_work(shape, int(m), setup.batch, setup.n_ctx) for m in rows_t)]
         roof = [roof_t[i % T] for i in range(timed_steps)]
         decode_ms = ms_local / timed_steps * T
         step_frac = (sum(roof) * 1e3) / ms_local
-        flops_traj = sum(step_work(shape, int(m), setup.batch, setup.n_ctx)[0] for m in traj)
+        flops_traj = sum(step_work(shape, int(m), setup.batch, setup.n_ctx)[0] for m in rows_t)
         flops_dense = T * step_work(shape, setup.batch * setup.n_ctx, setup.batch, setup.n_ctx)[0]
         # dominant kernel: the tensor-core GEMM
         g = tim["gemm"]
@@ -534,7 +559,7 @@ def run_ours(args, rank: int, world: int):
             peak_kind = "bf16 sustained (kernel timed inside the decode)"
         pfs = peaks["bf16_tflops_sustained"] * 1e12
         roof_s = [max(fl / pfs, by / pb) for fl, by in
-                  (step_work(shape, int(traj[i % T]), setup.batch, setup.n_ctx)
+                  (step_work(shape, int(rows_t[i % T]), setup.batch, setup.n_ctx)
                    for i in range(timed_steps))]
         step_frac_sustained = (sum(roof_s) * 1e3) / ms_local
         idx = list(range(0, T, 16)) + [T - 1]
@@ -544,10 +569,12 @@ def run_ours(args, rank: int, world: int):
 
         curve = {"t": idx, "M_t": [int(traj2[i]) for i in idx],
                  "ms": [round(float(step_ms[i]), 3) for i in idx],
-                 "roofline_frac": [round(roof_ms(traj2[i]) / float(step_ms[i]), 3) for i in idx]}
+                 "roofline_frac": [round(roof_ms(rows_t2[i]) / float(step_ms[i]), 3) for i in idx]}
+        if setup.kv_reuse > 1:
+            curve["computed_rows"] = [int(rows_t2[i]) for i in idx]
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            v, desc, thr = oracle_sample(setup, traj)
+            v, desc, thr = oracle_sample(setup, rows_t)
             cpu = {"value": v, "unit": "denoise steps/s", "cores": thr, "kind": "oracle",
                    "sample": desc}
         result = {
@@ -591,6 +618,7 @@ def run_ours(args, rank: int, world: int):
             "kernel_time_ms": {k: round(tim[k]["ms"], 3) for k in ("gemm", "attn", "lock")},
             "curve": curve,
             "trajectory": [int(m) for m in traj],
+            **({"computed_rows": [int(m) for m in rows_t]} if setup.kv_reuse > 1 else {}),
             "cpu_baseline": cpu,
             "clocks": clk,
             "gpu_launches": int(kernels_timed),
@@ -666,6 +694,10 @@ def main():
     ap.add_argument("--head-fusion", default="on", choices=["on", "off"],
                     help="sure-test statistics in the LM head's epilogue (on) or in a "
                          "separate pass over the stored logits (off)")
+    ap.add_argument("--kv-reuse", type=int, default=1,
+                    help="compose the method with K/V reuse for the active rows: all active "
+                         "rows are recomputed every R steps, between them only the masked and "
+                         "just-unmasked ones (1 = off)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--out-dir", default=os.path.join(tempfile.gettempdir(), "surelock_bench"),
                     help="where the per-rank clock samples (CSV) are written")

@@ -382,13 +382,16 @@ typedef struct sl_sampler_state {
   int32_t *lock_t;       /* [B][N], -1 if unlocked */
   void *logits[2];       /* [B][N][V] ping-pong, step t writes logits[t % 2] */
   float *lse[2];         /* [B][N] */
-  float *kl, *unc, *conf;/* [B*N] by active-row index */
+  float *kl, *unc, *conf;/* [B*N] by the index of the rows the step computed */
   int32_t *argmax;       /* [B*N] */
   uint8_t *lock;         /* [B*N] */
   sl_kv_cache *cache;
   sl_active *active;
   int t;                 /* next step to run */
   int batch, n_ctx;
+  sl_active *computed;   /* K/V reuse on: the rows the last step between refreshes
+                            computed (refresh steps compute `active` and leave it
+                            as it was); NULL if reuse was never switched on */
 } sl_sampler_state;
 
 /* Creates a sampler for `batch` sequences (1..SL_MAX_BATCH) of n_ctx =
@@ -400,8 +403,26 @@ typedef struct sl_sampler_state {
 sl_status sl_sampler_create(sl_model *m, int batch, const sl_sampler_params *p, sl_sampler **out);
 /* Reset state for a new decode from device prompts [batch][prompt_len]. */
 sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, void *stream);
+/* SureLock composed with cross-step K/V reuse for the active rows, which the
+ * pages call orthogonal to locking and stackable with it (Paper-Notes, "loss /
+ * training strategy" and "key results"); the scheme is this library's reading:
+ * period R = 1 (the default) is SureLock alone.  With R > 1, step t computes
+ * all active rows when t mod R = 0 (a refresh step).  Between refreshes it
+ * computes the active rows that are masked, or were masked at the start of the
+ * previous step (so a row is computed once more after its unmasking); each
+ * other active row keeps its cached K/V, its last logits and lse (carried into
+ * the step's logit buffer), is not tested and stays active.  The sure test,
+ * the confidence gate's quantile and the unmasking run over the computed rows;
+ * kl, unc, conf, argmax and lock are indexed by them.  The first call with
+ * R > 1 allocates a second active list and 3 bytes per position.
+ * SL_ERR_INVALID: R < 1, or R > 1 on a scripted sampler (its lock count is
+ * defined over the whole active set); SL_ERR_STATE while a decode is in
+ * progress (started and t < steps); SL_ERR_OOM.  sl_sampler_step returns
+ * SL_ERR_INVALID if R > 1 and the model has the no-KV-cache ablation. */
+sl_status sl_sampler_set_kv_reuse(sl_sampler *s, int period);
 /* One denoising step t: sl_step_stats and sl_lock_decide (or sl_step and
- * sl_kl_lock, see sl_model_set_head_fusion), sl_unmask_topk, sl_compact_active. */
+ * sl_kl_lock, see sl_model_set_head_fusion), sl_unmask_topk, sl_compact_active
+ * (with K/V reuse, on the computed rows; see sl_sampler_set_kv_reuse). */
 sl_status sl_sampler_step(sl_sampler *s, void *stream);
 /* Whole decode from host prompts [batch][prompt_len] to host tokens
  * [batch][n_ctx]; both copies are inside the call. */

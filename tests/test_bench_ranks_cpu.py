@@ -8,6 +8,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -229,3 +230,18 @@ def test_head_fusion_arm_is_named_in_the_workload():
     w_on = bench.workload_config(on, setup, 1)["workload"]
     w_off = bench.workload_config(off, setup, 1)["workload"]
     assert w_on != w_off and "separate pass" in w_off and "separate pass" not in w_on
+
+
+def test_kv_reuse_arm_is_named_and_checked():
+    sys.path.insert(0, ROOT)
+    import bench
+    plain, reuse = _bench_args(), _bench_args(kv_reuse=4)
+    s0, s4 = bench.setup_from_args(plain), bench.setup_from_args(reuse)
+    assert s0.kv_reuse == 1 and s4.kv_reuse == 4
+    w0 = bench.workload_config(plain, s0, 1)["workload"]
+    w4 = bench.workload_config(reuse, s4, 1)["workload"]
+    assert "K/V reuse" in w4 and "every 4 steps" in w4 and "K/V reuse" not in w0
+    for bad in (dict(kv_reuse=0), dict(kv_reuse=2, scripted=True, workload="full8b"),
+                dict(kv_reuse=2, ablation="no_kv_cache")):
+        with pytest.raises(SystemExit):
+            bench.setup_from_args(_bench_args(**bad))

@@ -32,6 +32,8 @@ def _sampler(setup, dev, std=0.02, seed_w=0, head_fusion=True):
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, setup.steps,
                    setup.block_len, setup.tokens_per_step, setup.eps, setup.gate_q,
                    setup.scripted)
+    if setup.kv_reuse > 1:
+        s.set_kv_reuse(setup.kv_reuse)
     prompts = wl.np_prompts(setup.batch, setup.prompt_len, shape.vocab, shape.mask_id)
     return model, s, weights_for_oracle(w_dev), prompts
 
@@ -63,10 +65,15 @@ def _teacher_forced(setup, dev, steps, std=0.02, head_fusion=True):
     shape = setup.shape
     B, N = setup.batch, setup.n_ctx
     s.start(torch.from_numpy(prompts).to(dev))
-    stats = {"mismatch": 0, "ambiguous": 0, "locks": 0, "unmask_amb": 0}
+    stats = {"mismatch": 0, "ambiguous": 0, "locks": 0, "unmask_amb": 0, "reused": 0}
+    R = setup.kv_reuse
+    mask_prev = None          # mask flags at the start of the previous step
     for t in range(steps):
         snap = _snapshot(s, setup)
         assert snap["t"] == t
+        if mask_prev is None:
+            mask_prev = snap["masked"]
+        refresh = R <= 1 or t % R == 0
         s.step()
         torch.cuda.synchronize()
         rt.device_check()
@@ -79,10 +86,26 @@ def _teacher_forced(setup, dev, steps, std=0.02, head_fusion=True):
         new_act = st["active"].positions()
         tok_after = st["tokens"].cpu().numpy()
         msk_after = st["masked"].cpu().numpy().astype(bool)
+        if not refresh:
+            comp_gpu = st["computed"].positions()
+            after = _snapshot(s, setup)
+            lse_c = st["lse"][cur].cpu().numpy().reshape(B, N)
+            lse_p = st["lse"][cur ^ 1].cpu().numpy().reshape(B, N)
         j0 = 0
         for b in range(B):
-            A = snap["act"][b]
+            A_all = snap["act"][b]
+            # the rows this step computes (K/V reuse between refresh steps)
+            A = A_all if refresh else A_all[snap["masked"][b, A_all] | mask_prev[b, A_all]]
             m = len(A)
+            if not refresh:
+                np.testing.assert_array_equal(comp_gpu[b], A)
+                reused = np.setdiff1d(A_all, A)
+                stats["reused"] += len(reused)
+                # reused rows: logits and lse carried forward, cache rows untouched
+                np.testing.assert_array_equal(z_gpu[b, reused], snap["z_prev"][b, reused])
+                np.testing.assert_array_equal(lse_c[b, reused], lse_p[b, reused])
+                np.testing.assert_array_equal(after["ck"][b][:, reused], snap["ck"][b][:, reused])
+                np.testing.assert_array_equal(after["cv"][b][:, reused], snap["cv"][b][:, reused])
             # forward: oracle on the GPU's state
             ck = np.ascontiguousarray(snap["ck"][b]); cv = np.ascontiguousarray(snap["cv"][b])
             z = om.forward_active(shape, w64, snap["tokens"][b], A, ck, cv,
@@ -132,9 +155,11 @@ def _teacher_forced(setup, dev, steps, std=0.02, head_fusion=True):
                 stats["unmask_amb"] += 1
             # masked rows never lock; compaction is the stable removal of GPU locks
             assert not np.any(lock_g[sl_] & snap["masked"][b, A])
-            np.testing.assert_array_equal(new_act[b], osl.compact(A, lock_g[sl_]))
+            np.testing.assert_array_equal(new_act[b],
+                                          osl.compact(A_all, np.isin(A_all, A[lock_g[sl_]])))
             assert np.array_equal(msk_after[b], tok_after[b] == shape.mask_id)
             j0 += m
+        mask_prev = snap["masked"]
     model_locked = s.state()["locked"].cpu().numpy().astype(bool)
     assert stats["mismatch"] == 0, stats
     return stats, model_locked
@@ -216,6 +241,61 @@ def test_tiny_free_running_ablations_match_oracle(cuda_dev):
         np.testing.assert_array_equal(out, tokT)
         assert list(s.state()["active"].counts()) == [counts[-1][0]]
         assert counts[-1][0] < setup.n_ctx
+
+
+# ------------------------------------------------ K/V reuse for active rows --
+
+@pytest.mark.parametrize("R", [2, 3])
+def test_tiny_decode_kv_reuse_teacher_forced(cuda_dev, R):
+    """Between refresh steps the step computes the masked and just-unmasked
+    active rows only: the computed list, their logits and sure test against the
+    oracle on the GPU's state; the reused rows' logits, lse and cache entries
+    unchanged; locks mapped back onto the active list."""
+    setup = dataclasses.replace(wl.CFG_TINY, kv_reuse=R)
+    stats, _ = _teacher_forced(setup, cuda_dev, setup.steps)
+    assert stats["locks"] > 5 and stats["reused"] > 10, stats
+
+
+@pytest.mark.parametrize("head_fusion", [True, False])
+def test_bf16_mini_decode_kv_reuse_teacher_forced(cuda_dev, head_fusion):
+    setup = wl.SamplerSetup(MINI_BF16, "bf16", batch=2, prompt_len=40, gen_len=160, steps=40,
+                            block_len=32, tokens_per_step=4, eps=0.01, gate_q=0.5, kv_reuse=3)
+    setup.validate()
+    stats, _ = _teacher_forced(setup, cuda_dev, 14, std=0.05, head_fusion=head_fusion)
+    assert stats["reused"] > 100, stats
+
+
+@pytest.mark.parametrize("R", [2, 4])
+def test_tiny_free_running_kv_reuse_matches_oracle(cuda_dev, R):
+    """Whole decode with reuse: final tokens and active counts as the oracle's."""
+    setup = dataclasses.replace(wl.CFG_TINY, kv_reuse=R)
+    model, s, w64, prompts = _sampler(setup, cuda_dev)
+    out = s.generate(prompts)
+    tok0, msk0 = wl.initial_tokens(prompts, setup.gen_len, setup.shape.mask_id)
+    tokT, _, counts, _, _ = osl.surelock_sampler(setup.shape, w64, tok0, msk0, setup)
+    np.testing.assert_array_equal(out, tokT)
+    assert list(s.state()["active"].counts()) == [counts[-1][0]]
+
+
+def test_kv_reuse_rejections(cuda_dev):
+    setup = dataclasses.replace(wl.CFG_TINY, scripted=True)
+    model, s, w64, prompts = _sampler(setup, cuda_dev)
+    with pytest.raises(RuntimeError):
+        s.set_kv_reuse(2)                                         # scripted schedule
+    with pytest.raises(RuntimeError):
+        s.set_kv_reuse(0)
+    model, s, w64, prompts = _sampler(wl.CFG_TINY, cuda_dev)
+    s.start(torch.from_numpy(prompts).to(cuda_dev))
+    with pytest.raises(RuntimeError):
+        s.set_kv_reuse(2)                                         # decode in progress
+    model.set_ablation(no_kv_cache=True)
+    s2 = rt.Sampler(model, 1, wl.CFG_TINY.prompt_len, wl.CFG_TINY.gen_len, wl.CFG_TINY.steps,
+                    wl.CFG_TINY.block_len, wl.CFG_TINY.tokens_per_step, wl.CFG_TINY.eps)
+    s2.set_kv_reuse(2)
+    s2.start(torch.from_numpy(prompts).to(cuda_dev))
+    with pytest.raises(RuntimeError):
+        s2.step()                                                 # no-KV-cache ablation
+    assert s2.state()["t"] == 0
 
 
 def test_gate_only_sampler_needs_the_gate(cuda_dev):

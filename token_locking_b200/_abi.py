@@ -54,7 +54,8 @@ class SamplerState(C.Structure):
                 ("lock_t", C.c_void_p), ("logits", C.c_void_p * 2), ("lse", C.c_void_p * 2),
                 ("kl", C.c_void_p), ("unc", C.c_void_p), ("conf", C.c_void_p),
                 ("argmax", C.c_void_p), ("lock", C.c_void_p), ("cache", C.c_void_p),
-                ("active", C.c_void_p), ("t", C.c_int), ("batch", C.c_int), ("n_ctx", C.c_int)]
+                ("active", C.c_void_p), ("t", C.c_int), ("batch", C.c_int), ("n_ctx", C.c_int),
+                ("computed", C.c_void_p)]
 
 
 class Timing(C.Structure):
@@ -93,6 +94,7 @@ SIGNATURES = {
     "sl_model_set_ablation": (_I, [_P, _I]),
     "sl_sampler_create": (_I, [_P, _I, C.POINTER(SamplerParams), C.POINTER(_P)]),
     "sl_sampler_start": (_I, [_P, _P, _P]),
+    "sl_sampler_set_kv_reuse": (_I, [_P, _I]),
     "sl_sampler_step": (_I, [_P, _P]),
     "sl_sampler_generate": (_I, [_P, _P, _P, _P]),
     "sl_sampler_get_state": (_I, [_P, C.POINTER(SamplerState)]),

@@ -173,6 +173,13 @@ struct sl_sampler {
   float *kl = nullptr, *unc = nullptr, *conf = nullptr;
   int t = 0;
   bool started = false;
+  // K/V reuse for active rows (refresh interval kv_reuse, 1 = off): the rows a
+  // step between refreshes computes, the mask flags at the start of the
+  // previous step, a per-position lock byte array (zero between steps) and the
+  // lock flags mapped onto the active list
+  int kv_reuse = 1;
+  sl_active *comp = nullptr;
+  uint8_t *masked_before = nullptr, *lock_by_pos = nullptr, *lock_act = nullptr;
 };
 
 // ----------------------------------------------------------------- timing --
@@ -1710,8 +1717,10 @@ extern "C" void sl_sampler_destroy(sl_sampler *s) {
   if (!s) return;
   sl_kv_cache_destroy(s->cache);
   sl_active_destroy(s->act);
+  sl_active_destroy(s->comp);
   void *ps[] = {s->tokens, s->masked, s->locked, s->lock, s->lock_t, s->argmax, s->d_prompts,
-                s->logits[0], s->logits[1], s->lse[0], s->lse[1], s->kl, s->unc, s->conf};
+                s->logits[0], s->logits[1], s->lse[0], s->lse[1], s->kl, s->unc, s->conf,
+                s->masked_before, s->lock_by_pos, s->lock_act};
   for (void *p : ps)
     if (p) cudaFree(p);
   delete s;
@@ -1794,8 +1803,40 @@ extern "C" sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, v
   if (r != SL_OK) return r;
   r = sl_active_reset(s->act, stream);
   if (r != SL_OK) return r;
+  if (s->lock_by_pos)
+    SL_CUDA(cudaMemsetAsync(s->lock_by_pos, 0, (size_t)rows, st));
   s->t = 0;
   s->started = true;
+  return SL_OK;
+}
+
+extern "C" sl_status sl_sampler_set_kv_reuse(sl_sampler *s, int period) {
+  if (!s) return fail(SL_ERR_INVALID, "sl_sampler_set_kv_reuse: null sampler");
+  if (period < 1) return fail(SL_ERR_INVALID, "sl_sampler_set_kv_reuse: period %d < 1", period);
+  if (period > 1 && s->p.scripted)
+    return fail(SL_ERR_INVALID, "sl_sampler_set_kv_reuse: the scripted schedule counts its "
+                                "locks over the whole active set");
+  if (s->started && s->t < s->p.steps)
+    return fail(SL_ERR_STATE, "sl_sampler_set_kv_reuse: a decode is in progress");
+  if (period > 1 && !s->comp) {
+    const size_t rows = (size_t)s->batch * s->n_ctx;
+    sl_status st = sl_active_create(s->batch, s->n_ctx, &s->comp);
+    if (st != SL_OK) return st;
+    bool ok = cudaMalloc(&s->masked_before, rows) == cudaSuccess &&
+              cudaMalloc(&s->lock_by_pos, rows) == cudaSuccess &&
+              cudaMalloc(&s->lock_act, rows) == cudaSuccess &&
+              cudaMemset(s->lock_by_pos, 0, rows) == cudaSuccess;
+    if (!ok) {
+      sl_active_destroy(s->comp);
+      for (uint8_t **q : {&s->masked_before, &s->lock_by_pos, &s->lock_act}) {
+        if (*q) cudaFree(*q);
+        *q = nullptr;
+      }
+      s->comp = nullptr;
+      return fail(SL_ERR_OOM, "sl_sampler_set_kv_reuse: device allocation failed");
+    }
+  }
+  s->kv_reuse = period;
   return SL_OK;
 }
 
@@ -1805,10 +1846,41 @@ extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
   if (s->t >= s->p.steps) return fail(SL_ERR_STATE, "sl_sampler_step: decode already finished");
   if ((s->m->ablation & SL_ABLATE_GATE_ONLY) && !s->p.scripted && !(s->p.gate_q >= 0.f))
     return fail(SL_ERR_INVALID, "sl_sampler_step: the gate-only ablation needs gate_q >= 0");
+  const bool reuse = s->kv_reuse > 1;
+  if (reuse && (s->m->ablation & SL_ABLATE_NO_KV_CACHE))
+    return fail(SL_ERR_INVALID, "sl_sampler_step: K/V reuse needs the cache of every row (the "
+                                "no-KV-cache ablation is on)");
   const int t = s->t;
   const int cur = t & 1, prv = cur ^ 1;
   const sl_config &cfg = s->m->cfg;
   sl_status st = SL_OK;
+  cudaStream_t cs = (cudaStream_t)stream;
+  // K/V reuse: all active rows at a refresh step (t mod R = 0), else the rows
+  // that are masked or were masked at the start of the previous step; the
+  // others carry their logits and lse into this step's buffers
+  const bool refresh = !reuse || t % s->kv_reuse == 0;
+  sl_active *run = refresh ? s->act : s->comp;
+  if (!refresh) {
+    SL_CUDA(launch_reuse_select(s->act->rows, s->act->seq_off, s->batch, s->masked,
+                                s->masked_before, s->comp->rows, s->comp->seq_off, cs));
+    if ((st = active_mirror(s->comp, cs)) != SL_OK) return st;
+    int32_t ca[SL_MAX_BATCH], cc[SL_MAX_BATCH];
+    if ((st = sl_active_counts(s->act, ca)) != SL_OK) return st;
+    if ((st = sl_active_counts(s->comp, cc)) != SL_OK) return st;
+    int ma = 0, mc = 0;
+    for (int b = 0; b < s->batch; ++b) {
+      ma += ca[b];
+      mc += cc[b];
+    }
+    const size_t row_bytes = (size_t)cfg.vocab * dsize(cfg.dtype);
+    Timed tm(s->m, SL_K_OTHER, 2.0 * (ma - mc) * ((double)row_bytes + 4.0), 0.0, cs);
+    SL_CUDA(launch_reuse_carry(s->act->rows, s->act->seq_off, s->batch, ma, s->masked,
+                               s->masked_before, s->logits[prv], s->logits[cur], s->lse[prv],
+                               s->lse[cur], row_bytes, cs));
+  }
+  if (reuse)
+    SL_CUDA(cudaMemcpyAsync(s->masked_before, s->masked, (size_t)s->batch * s->n_ctx,
+                            cudaMemcpyDeviceToDevice, cs));
   sl_lock_params lp;
   lp.eps = s->p.eps;
   lp.gate_q = s->p.gate_q;
@@ -1824,25 +1896,31 @@ extern "C" sl_status sl_sampler_step(sl_sampler *s, void *stream) {
   }
   if (s->m->head_fusion && cfg.dtype == SL_BF16) {
     // the sure test's statistics come out of the LM head's epilogue
-    st = sl_step_stats(s->m, s->cache, s->act, s->tokens, s->logits[cur], s->logits[prv],
+    st = sl_step_stats(s->m, s->cache, run, s->tokens, s->logits[cur], s->logits[prv],
                        s->lse[prv], lp.has_prev, s->lse[cur], s->kl, s->unc, s->conf, s->argmax,
                        stream);
     if (st != SL_OK) return st;
-    st = lock_decide_impl(s->act, s->masked, &lp, s->kl, s->unc, s->lock, (cudaStream_t)stream);
+    st = lock_decide_impl(run, s->masked, &lp, s->kl, s->unc, s->lock, cs);
   } else {
-    st = sl_step(s->m, s->cache, s->act, s->tokens, s->logits[cur], stream);
+    st = sl_step(s->m, s->cache, run, s->tokens, s->logits[cur], stream);
     if (st != SL_OK) return st;
-    st = kl_lock_impl(s->m, s->act, cfg.vocab, cfg.mask_id, cfg.dtype, s->logits[cur],
+    st = kl_lock_impl(s->m, run, cfg.vocab, cfg.mask_id, cfg.dtype, s->logits[cur],
                       s->logits[prv], s->lse[prv], s->lse[cur], s->masked, &lp, s->kl, s->unc,
                       s->conf, s->argmax, s->lock, (cudaStream_t)stream);
   }
   if (st != SL_OK) return st;
   const int spb = s->p.steps / (s->p.gen_len / s->p.block_len);
   const int lo = s->p.prompt_len + (t / spb) * s->p.block_len;
-  st = sl_unmask_topk(s->act, s->conf, s->argmax, lo, lo + s->p.block_len, s->p.tokens_per_step,
+  st = sl_unmask_topk(run, s->conf, s->argmax, lo, lo + s->p.block_len, s->p.tokens_per_step,
                       s->tokens, s->masked, stream);
   if (st != SL_OK) return st;
-  st = sl_compact_active(s->act, s->lock, s->locked, s->lock_t, t, stream);
+  const uint8_t *lock_act = s->lock;
+  if (!refresh) {
+    SL_CUDA(launch_reuse_lock_map(s->comp->rows, s->comp->seq_off, s->lock, s->act->rows,
+                                  s->act->seq_off, s->batch, s->lock_by_pos, s->lock_act, cs));
+    lock_act = s->lock_act;
+  }
+  st = sl_compact_active(s->act, lock_act, s->locked, s->lock_t, t, stream);
   if (st != SL_OK) return st;
   s->t = t + 1;
   return SL_OK;
@@ -1890,6 +1968,7 @@ extern "C" sl_status sl_sampler_get_state(const sl_sampler *s, sl_sampler_state 
   o->lock = s->lock;
   o->cache = s->cache;
   o->active = s->act;
+  o->computed = s->comp;
   o->t = s->t;
   o->batch = s->batch;
   o->n_ctx = s->n_ctx;

@@ -233,5 +233,20 @@ cudaError_t launch_head_stats_merge(const float4 *stat, const int *stat_idx, int
                                     float *conf, int32_t *argmax, cudaStream_t s);
 cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n_ctx,
                                cudaStream_t s);
+// K/V reuse for active rows: the computed list of a step between refreshes,
+// the reused rows' logits and lse carried forward, and the computed rows' lock
+// flags mapped onto the active list.
+cudaError_t launch_reuse_select(const int32_t *rows, const int32_t *seq_off, int batch,
+                                const uint8_t *masked, const uint8_t *masked_before,
+                                int32_t *out_rows, int32_t *out_off, cudaStream_t s);
+cudaError_t launch_reuse_carry(const int32_t *rows, const int32_t *seq_off, int batch,
+                               int m_active, const uint8_t *masked,
+                               const uint8_t *masked_before, const void *prev, void *cur,
+                               const float *lse_prev, float *lse_cur, size_t row_bytes,
+                               cudaStream_t s);
+cudaError_t launch_reuse_lock_map(const int32_t *c_rows, const int32_t *c_off,
+                                  const uint8_t *c_lock, const int32_t *a_rows,
+                                  const int32_t *a_off, int batch, uint8_t *by_pos,
+                                  uint8_t *a_lock, cudaStream_t s);
 
 }  // namespace sl

@@ -560,6 +560,154 @@ cudaError_t launch_active_fill(int32_t *rows, int32_t *seq_off, int batch, int n
   return err;
 }
 
+// ----------------------------------------------- K/V reuse for active rows --
+// Between the refresh steps of the reuse, a step computes the active rows that
+// are masked now or were masked at the start of the previous step (a row is
+// computed once more after its unmasking, so that its cached K/V carry its
+// token).  The other active rows keep their cache entries and last posterior.
+
+__device__ __forceinline__ bool reuse_computed(const uint8_t *masked,
+                                               const uint8_t *masked_before, int p) {
+  return (masked[p] | masked_before[p]) != 0;
+}
+
+// C_t = [rows_j : computed(rows_j)], stable, into a second list; one CTA walks
+// the sequences in order, as the compaction does.
+__global__ void __launch_bounds__(DEC_THREADS) reuse_select_kernel(
+    const int32_t *__restrict__ rows, const int32_t *__restrict__ seq_off, int batch,
+    const uint8_t *__restrict__ masked, const uint8_t *__restrict__ masked_before,
+    int32_t *__restrict__ out_rows, int32_t *__restrict__ out_off) {
+  __shared__ int wsum[DEC_THREADS / 32];
+  __shared__ int total;
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int out = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int s0 = seq_off[b], s1 = seq_off[b + 1];
+    if (threadIdx.x == 0) out_off[b] = out;
+    for (int c0 = s0; c0 < s1; c0 += blockDim.x) {
+      const int j = c0 + threadIdx.x;
+      int p = 0;
+      bool keep = false;
+      if (j < s1) {
+        p = rows[j];
+        keep = reuse_computed(masked, masked_before, p);
+      }
+      const unsigned int bal = __ballot_sync(0xffffffffu, keep);
+      const int wpre = __popc(bal & ((1u << lane) - 1u));
+      if (lane == 0) wsum[warp] = __popc(bal);
+      __syncthreads();
+      if (warp == 0) {
+        const int v = lane < (int)(blockDim.x >> 5) ? wsum[lane] : 0;
+        int inc = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        wsum[lane] = inc - v;
+        if (lane == 31) total = inc;
+      }
+      __syncthreads();
+      if (keep) out_rows[out + wsum[warp] + wpre] = p;
+      out += total;
+      __syncthreads();
+    }
+  }
+  if (threadIdx.x == 0) out_off[batch] = out;
+}
+
+// The reused rows' logits and lse carried from the previous step's buffers to
+// this step's, so that the ping-pong pair always holds every row's last
+// posterior (bandwidth-bound copy of 16-byte vectors; blockIdx.y strides over
+// the active rows, blockIdx.x over one row's vectors).
+constexpr int REUSE_CARRY_THREADS = 256;
+constexpr int REUSE_CARRY_VEC = 4;   // 16-byte vectors per thread per pass
+
+__global__ void __launch_bounds__(REUSE_CARRY_THREADS) reuse_carry_kernel(
+    const int32_t *__restrict__ rows, const int32_t *__restrict__ seq_off, int batch,
+    const uint8_t *__restrict__ masked, const uint8_t *__restrict__ masked_before,
+    const uint4 *__restrict__ prev, uint4 *__restrict__ cur, const float *__restrict__ lse_prev,
+    float *__restrict__ lse_cur, int row_vecs) {
+  pdl_wait();
+  pdl_trigger();
+  const int M = seq_off[batch];
+  for (int j = blockIdx.y; j < M; j += gridDim.y) {
+    const int p = rows[j];
+    if (reuse_computed(masked, masked_before, p)) continue;
+    const uint4 *src = prev + (size_t)p * row_vecs;
+    uint4 *dst = cur + (size_t)p * row_vecs;
+    const int span = REUSE_CARRY_THREADS * REUSE_CARRY_VEC;
+    for (int i0 = blockIdx.x * span; i0 < row_vecs; i0 += gridDim.x * span) {
+      uint4 v[REUSE_CARRY_VEC];
+#pragma unroll
+      for (int u = 0; u < REUSE_CARRY_VEC; ++u) {
+        const int i = i0 + u * REUSE_CARRY_THREADS + threadIdx.x;
+        if (i < row_vecs) v[u] = src[i];
+      }
+#pragma unroll
+      for (int u = 0; u < REUSE_CARRY_VEC; ++u) {
+        const int i = i0 + u * REUSE_CARRY_THREADS + threadIdx.x;
+        if (i < row_vecs) dst[i] = v[u];
+      }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) lse_cur[p] = lse_prev[p];
+  }
+}
+
+// Lock flags of the computed rows (by computed-row index) onto the active list
+// (by active-row index) through a per-position byte array that is zero
+// between calls: scatter, then gather and clear.  One CTA, so the barrier
+// between the two passes is __syncthreads.
+__global__ void __launch_bounds__(DEC_THREADS) reuse_lock_map_kernel(
+    const int32_t *__restrict__ c_rows, const int32_t *__restrict__ c_off,
+    const uint8_t *__restrict__ c_lock, const int32_t *__restrict__ a_rows,
+    const int32_t *__restrict__ a_off, int batch, uint8_t *__restrict__ by_pos,
+    uint8_t *__restrict__ a_lock) {
+  pdl_wait();
+  pdl_trigger();
+  const int mc = c_off[batch], ma = a_off[batch];
+  for (int j = threadIdx.x; j < mc; j += blockDim.x) by_pos[c_rows[j]] = c_lock[j];
+  __syncthreads();
+  for (int j = threadIdx.x; j < ma; j += blockDim.x) {
+    const int p = a_rows[j];
+    a_lock[j] = by_pos[p];
+    by_pos[p] = 0;
+  }
+}
+
+cudaError_t launch_reuse_select(const int32_t *rows, const int32_t *seq_off, int batch,
+                                const uint8_t *masked, const uint8_t *masked_before,
+                                int32_t *out_rows, int32_t *out_off, cudaStream_t s) {
+  return launch_k(reuse_select_kernel, 1, DEC_THREADS, 0, s, rows, seq_off, batch, masked,
+                  masked_before, out_rows, out_off);
+}
+
+cudaError_t launch_reuse_carry(const int32_t *rows, const int32_t *seq_off, int batch,
+                               int m_active, const uint8_t *masked,
+                               const uint8_t *masked_before, const void *prev, void *cur,
+                               const float *lse_prev, float *lse_cur, size_t row_bytes,
+                               cudaStream_t s) {
+  if (m_active <= 0) return cudaSuccess;
+  if (row_bytes % 16 != 0 || ((uintptr_t)prev & 15) || ((uintptr_t)cur & 15))
+    return cudaErrorInvalidValue;
+  const int row_vecs = (int)(row_bytes / 16);
+  const int span = REUSE_CARRY_THREADS * REUSE_CARRY_VEC;
+  dim3 grid((row_vecs + span - 1) / span, m_active < 65535 ? m_active : 65535);
+  return launch_k(reuse_carry_kernel, grid, REUSE_CARRY_THREADS, 0, s, rows, seq_off, batch,
+                  masked, masked_before, static_cast<const uint4 *>(prev),
+                  static_cast<uint4 *>(cur), lse_prev, lse_cur, row_vecs);
+}
+
+cudaError_t launch_reuse_lock_map(const int32_t *c_rows, const int32_t *c_off,
+                                  const uint8_t *c_lock, const int32_t *a_rows,
+                                  const int32_t *a_off, int batch, uint8_t *by_pos,
+                                  uint8_t *a_lock, cudaStream_t s) {
+  return launch_k(reuse_lock_map_kernel, 1, DEC_THREADS, 0, s, c_rows, c_off, c_lock, a_rows,
+                  a_off, batch, by_pos, a_lock);
+}
+
 }  // namespace sl
 
 // ---------------------------------------------------- no-allocation variant --

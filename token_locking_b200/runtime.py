@@ -373,6 +373,12 @@ class Sampler:
         A.check(A.lib().sl_sampler_start(self.handle, _ptr(prompts), _stream(stream)),
                 "sl_sampler_start")
 
+    def set_kv_reuse(self, period: int):
+        """K/V reuse for the active rows with refresh interval `period` (1 = off);
+        between decodes only."""
+        A.check(A.lib().sl_sampler_set_kv_reuse(self.handle, int(period)),
+                "sl_sampler_set_kv_reuse")
+
     def step(self, stream=None):
         A.check(A.lib().sl_sampler_step(self.handle, _stream(stream)), "sl_sampler_step")
 
@@ -418,6 +424,7 @@ class Sampler:
             "lock": device_view(st.lock, (R,), torch.uint8),
             "cache": KVCache.wrap(st.cache, self.model, B, N),
             "active": Active.wrap(st.active, B, N),
+            "computed": Active.wrap(st.computed, B, N) if st.computed else None,
         }
 
     def close(self):
