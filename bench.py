@@ -563,6 +563,10 @@ def run_ours(args, rank: int, world: int):
                    for i in range(timed_steps))]
         step_frac_sustained = (sum(roof_s) * 1e3) / ms_local
         idx = list(range(0, T, 16)) + [T - 1]
+        if setup.kv_reuse > 1:
+            # every sampled step with its successor, so that steps between
+            # refreshes are in the curve too
+            idx = sorted({j for i in idx for j in (i, i + 1) if j < T})
         def roof_ms(m):
             fl, by = step_work(shape, int(m), setup.batch, setup.n_ctx)
             return max(fl / pf, by / pb) * 1e3
