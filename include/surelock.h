@@ -404,8 +404,10 @@ sl_status sl_sampler_create(sl_model *m, int batch, const sl_sampler_params *p, 
 /* Reset state for a new decode from device prompts [batch][prompt_len]. */
 sl_status sl_sampler_start(sl_sampler *s, const int32_t *d_prompts, void *stream);
 /* SureLock composed with cross-step K/V reuse for the active rows, which the
- * pages call orthogonal to locking and stackable with it (Paper-Notes, "loss /
- * training strategy" and "key results"); the scheme is this library's reading:
+ * pages call orthogonal to locking and stackable with it (Paper-Notes,
+ * "permanent locking" design motivation, where dLLM-Cache is the per-step
+ * selective counterpart, and "loss / training strategy"; gist.science/it
+ * section 4, "Ortogonalita"); the scheme is this library's reading:
  * period R = 1 (the default) is SureLock alone.  With R > 1, step t computes
  * all active rows when t mod R = 0 (a refresh step).  Between refreshes it
  * computes the active rows that are masked, or were masked at the start of the

@@ -217,9 +217,12 @@ def step(shape, w: dict, st: State, setup, t: int, record_block_inputs: bool = F
     Paper-Notes, "Method: overall framework" (compute A_t, serve L_t from the
     cache) and "permanent locking" (a locked row's posterior is frozen).
 
-    With setup.kv_reuse = R > 1 (the pages' composition with cross-step K/V
-    reuse, Paper-Notes "loss / training strategy" and "key results": orthogonal
-    and stackable; the scheme itself is this restatement's reading) the forward
+    With setup.kv_reuse = R > 1 (the pages' composition with cross-step reuse:
+    Paper-Notes, "permanent locking", design motivation, sets SureLock's
+    permanent removal against dLLM-Cache's per-step choice of what to compute;
+    "loss / training strategy" and gist.science/it section 4, "Ortogonalita",
+    call the two orthogonal and stackable; the scheme itself is this
+    restatement's reading) the forward
     runs on all of A_t only when t mod R = 0.  Between those refresh steps it
     runs on the active rows that are masked or were masked at the start of the
     previous step; the other active rows keep their cached K/V and their last
