@@ -378,6 +378,18 @@ def aux_decodes(k: int, decode_ms: float, budget_ms: float = 20000.0) -> int:
     return max(1, min(k, int(budget_ms // max(decode_ms, 1e-3))))
 
 
+def carry_line(rec: dict, decodes: int, peaks: dict) -> dict:
+    """The K/V reuse carry kernel over the instrumented decodes: its time per
+    decode and its bandwidth (the reused rows' logits and lse read and written
+    once) against the measured HBM copy peak."""
+    ms, by = rec["ms"], rec["bytes"]
+    gbs = by / (ms / 1e3) / 1e9 if ms > 0 else None
+    return {"ms_per_decode": round(ms / max(1, decodes), 3),
+            "launches_per_decode": rec["launches"] // max(1, decodes),
+            "achieved_gbs": round(gbs, 1) if gbs else None,
+            "frac_hbm": round(gbs / peaks["hbm_gbs"], 4) if gbs else None}
+
+
 def replica_prompt_seed(rank: int) -> int:
     """Each replica decodes its own prompts."""
     return wl.SEED_PROMPTS + rank
@@ -620,6 +632,7 @@ def run_ours(args, rank: int, world: int):
                                        "bf16_tflops_sustained, hbm_gbs"},
             "algorithmic_flops_reduction": round(1.0 - flops_traj / flops_dense, 4),
             "kernel_time_ms": {k: round(tim[k]["ms"], 3) for k in ("gemm", "attn", "lock")},
+            **({"reuse_carry": carry_line(tim["other"], aux, peaks)} if setup.kv_reuse > 1 else {}),
             "curve": curve,
             "trajectory": [int(m) for m in traj],
             **({"computed_rows": [int(m) for m in rows_t]} if setup.kv_reuse > 1 else {}),

@@ -245,3 +245,14 @@ def test_kv_reuse_arm_is_named_and_checked():
                 dict(kv_reuse=2, ablation="no_kv_cache")):
         with pytest.raises(SystemExit):
             bench.setup_from_args(_bench_args(**bad))
+
+
+def test_carry_line_arithmetic():
+    sys.path.insert(0, ROOT)
+    import bench
+    got = bench.carry_line({"ms": 20.0, "bytes": 100e9 * 0.02, "launches": 768}, 2,
+                           {"hbm_gbs": 6400.0})
+    assert got == {"ms_per_decode": 10.0, "launches_per_decode": 384, "achieved_gbs": 100.0,
+                   "frac_hbm": 0.0156}
+    assert bench.carry_line({"ms": 0.0, "bytes": 0.0, "launches": 0}, 1,
+                            {"hbm_gbs": 6400.0})["achieved_gbs"] is None
