@@ -135,9 +135,11 @@ def cache_rows(s, setup, b, rows) -> tuple:
     return np.stack(ks), np.stack(vs)
 
 
-def check_decisions(setup, t, b, A, snap, g, j0, stats):
+def check_decisions(setup, t, b, A, snap, g, j0, stats, A_all=None):
     """Sure test, gate, unmasking and compaction of sequence b at step t, taken
-    by the oracle on the GPU's logits; exact outside the rounding bands."""
+    by the oracle on the GPU's logits; exact outside the rounding bands.  A are
+    the rows the step computed; A_all the active rows when that is more (K/V
+    reuse between refresh steps), which the compaction runs over."""
     shape = setup.shape
     m = len(A)
     sl_ = slice(j0, j0 + m)
@@ -178,7 +180,10 @@ def check_decisions(setup, t, b, A, snap, g, j0, stats):
         assert conf_ambiguous(conf, sel, cands), f"t={t} b={b}: unmasking differs"
         stats["unmask_amb"] += 1
     assert not np.any(lock_g & snap["masked"][b, A]), "a masked row locked"
-    np.testing.assert_array_equal(g["act"][b], osl.compact(A, lock_g))
+    if A_all is None:
+        np.testing.assert_array_equal(g["act"][b], osl.compact(A, lock_g))
+    else:
+        np.testing.assert_array_equal(g["act"][b], osl.compact(A_all, np.isin(A_all, A[lock_g])))
     assert np.array_equal(g["masked"][b], g["tokens"][b] == shape.mask_id)
 
 

@@ -86,17 +86,27 @@ def _decode(llada8b, dev, setup, full_steps, sampled_steps, name, kv_tol=KV_TOL)
     model, _, w_or = llada8b
     shape = setup.shape
     B = setup.batch
+    R = setup.kv_reuse
     s = rt.Sampler(model, B, setup.prompt_len, setup.gen_len, setup.steps, setup.block_len,
                    setup.tokens_per_step, setup.eps, setup.gate_q, setup.scripted)
+    if R > 1:
+        s.set_kv_reuse(R)
     s.autotune()
     prompts = wl.np_prompts(B, setup.prompt_len, shape.vocab, shape.mask_id,
                             seed=wl.SEED_PROMPTS)
     s.start(torch.from_numpy(prompts).to(dev))
     stats = {"mismatch": 0, "ambiguous": 0, "locks": 0, "unmask_amb": 0}
     worst = {"logits": 0.0, "kv": 0.0, "lp": 0.0}
+    mask_prev = None          # K/V reuse: mask flags at the start of the previous step
     for t in range(setup.steps):
+        if R > 1:
+            mask_start = s.state()["masked"].cpu().numpy().astype(bool)
+            if mask_prev is None:
+                mask_prev = mask_start
         if t not in full_steps and t not in sampled_steps:
             s.step()
+            if R > 1:
+                mask_prev = mask_start
             continue
         full = t in full_steps
         snap = p8.snapshot(s, setup, want_cache=full)
@@ -105,9 +115,22 @@ def _decode(llada8b, dev, setup, full_steps, sampled_steps, name, kv_tol=KV_TOL)
         rt.device_check()
         g = p8.gpu_after(s, setup, t)
         t0 = time.time()
+        refresh = R <= 1 or t % R == 0
+        comp_gpu = None if refresh else s.state()["computed"].positions()
         j0 = 0
         for b in range(B):
-            A = snap["act"][b]
+            A_all = snap["act"][b]
+            # the rows the step computes (all active rows unless K/V reuse
+            # skips the unmasked ones between refreshes)
+            A = A_all if refresh else A_all[snap["masked"][b, A_all] | mask_prev[b, A_all]]
+            if not refresh:
+                np.testing.assert_array_equal(comp_gpu[b], A)
+                reused = np.setdiff1d(A_all, A)
+                if full and len(reused):
+                    kr, vr = p8.cache_rows(s, setup, b, reused)
+                    np.testing.assert_array_equal(kr, snap["ck"][b][:, reused])
+                    np.testing.assert_array_equal(vr, snap["cv"][b][:, reused])
+                    np.testing.assert_array_equal(g["z"][b, reused], snap["z_prev"][b, reused])
             m = len(A)
             if m == 0:
                 continue
@@ -138,8 +161,11 @@ def _decode(llada8b, dev, setup, full_steps, sampled_steps, name, kv_tol=KV_TOL)
             assert zerr <= tol, f"{name} t={t} b={b}: logits err {zerr} > {tol}"
             assert kv <= kv_tol, f"{name} t={t} b={b}: fresh K/V rel err {kv}"
             assert lperr <= tol, f"{name} t={t} b={b}: log-prob err {lperr} > {tol}"
-            p8.check_decisions(setup, t, b, A, snap, g, j0, stats)
+            p8.check_decisions(setup, t, b, A, snap, g, j0, stats,
+                               A_all=None if refresh else A_all)
             j0 += m            # per-row outputs run over all sequences in order
+        if R > 1:
+            mask_prev = mask_start
     final = s.state()
     assert int(final["masked"].sum().item()) == 0, "positions left masked at the end"
     _log({"test": name, "summary": stats, "worst": worst})
@@ -161,6 +187,17 @@ def test_llada8b_b1_n384_teacher_forced(llada8b, cuda_dev, arm):
         assert stats["locks"] == 0
     else:
         assert stats["locks"] > 0
+
+
+def test_llada8b_b1_n384_kv_reuse_teacher_forced(llada8b, cuda_dev):
+    """The composition with K/V reuse (all active rows recomputed every 4 steps)
+    at the batch-1 shape: steps 1, 2, 31, 254 and 255 fall between refreshes,
+    where the computed list, the computed rows' logits, K/V and decisions, and
+    the reused rows' unchanged cache entries and carried logits are checked."""
+    import dataclasses
+    setup = dataclasses.replace(wl.cfg_full8b(eps=0.05), kv_reuse=4)
+    stats, _ = _decode(llada8b, cuda_dev, setup, CHECK4, (), "cfg4-reuse4")
+    assert stats["locks"] > 0
 
 
 def test_llada8b_b4_n2048_teacher_forced(llada8b, cuda_dev):
