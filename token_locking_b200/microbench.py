@@ -187,6 +187,8 @@ def bench_decode(args, dev):
     model = rt.Model(shape, w, "bf16")
     s = rt.Sampler(model, setup.batch, setup.prompt_len, setup.gen_len, setup.steps,
                    setup.block_len, setup.tokens_per_step, setup.eps, setup.gate_q)
+    if args.kv_reuse > 1:
+        s.set_kv_reuse(args.kv_reuse)
     max_rows = setup.batch * (setup.prompt_len + setup.gen_len)
     if args.tuning_in:
         for kind, M, bn, sp, var in json.load(open(args.tuning_in)):
@@ -394,6 +396,8 @@ def main():
                     "16:1,32:1,64:1,16:2,16:4,64:4",
                     help="attn: queries-per-CTA:splits[:key tile] list (0:0 = the library's choice)")
     ap.add_argument("--tuning-out", default=None, help="decode: save the autotuned GEMM tilings")
+    ap.add_argument("--kv-reuse", type=int, default=1,
+                    help="decode: K/V reuse for the active rows, all recomputed every R steps")
     ap.add_argument("--tuning-in", default=None,
                     help="decode: load GEMM tilings instead of autotuning (e.g. under a profiler)")
     args = ap.parse_args()
