@@ -108,3 +108,37 @@ def test_header_is_plain_c_and_links(tmp_path):
     assert r.returncode == 0, r.stderr[-4000:]
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="gcc not on PATH")
+def test_struct_layouts_match_the_header(tmp_path):
+    """Every struct the binding passes through the boundary has the header's
+    size and field offsets (a field added to the header but not to the
+    binding, or in another order, shifts what the library reads)."""
+    from token_locking_b200 import _abi as A
+    pairs = [("sl_config", A.Config), ("sl_layer_weights", A.LayerWeights),
+             ("sl_weights", A.Weights), ("sl_lock_params", A.LockParams),
+             ("sl_sampler_params", A.SamplerParams), ("sl_sampler_state", A.SamplerState),
+             ("sl_timing", A.Timing)]
+    lines = []
+    for cname, py in pairs:
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    src = tmp_path / "layout.c"
+    src.write_text('#include "surelock.h"\n#include <stddef.h>\n#include <stdio.h>\n'
+                   "int main(void) {\n" + "\n".join(lines) + "\n  return 0;\n}\n")
+    exe = str(tmp_path / "layout")
+    r = subprocess.run(["gcc", "-std=c99", "-I" + os.path.join(ROOT, "include"), str(src),
+                        "-o", exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr[-4000:]
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0
+    got = {}
+    for line in r.stdout.splitlines():
+        *key, val = line.split()
+        got[tuple(key)] = int(val)
+    for cname, py in pairs:
+        assert got[(cname, "size")] == C.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
