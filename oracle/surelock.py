@@ -30,6 +30,11 @@ Readings where the pages are silent (the plainest reading consistent with them):
   R11 semi-autoregressive blocks over the generated region; each step unmasks
       the k highest-confidence masked positions of the current block, where
       confidence and prediction are taken over v != [MASK].
+  R22 composition with K/V reuse for the active rows (refresh interval R): all
+      of A_t computed when t mod R = 0, else the active rows masked now or at
+      the start of the previous step; the others keep their cached K/V and last
+      posterior and are not tested (step()); the gate quantile of R8 is then
+      taken over the computed rows.
   Scripted mode: instead of the KL test, lock the eligible (unmasked, with a
   previous posterior) active rows in ascending (D, position) order until the
   active count reaches a target.
