@@ -175,10 +175,11 @@ def step_work(shape: wl.ModelShape, m_rows: int, batch: int, n_ctx: int):
 
 
 def stored_trajectory(workload: str):
-    """The M_t trajectory a GPU run of this exact workload recorded
-    (profiles/trajectory_*.json, copied from the bench line's "trajectory"), or
-    None.  It only weights the CPU oracle's timed sample by the work of each
-    step; it is never an input or an expected value of a parity check."""
+    """The rows each step computes, as a GPU run of this exact workload
+    recorded them (profiles/trajectory_*.json, copied from the bench line's
+    "trajectory" = M_t, or its "computed_rows" under K/V reuse), or None.  It
+    only weights the CPU oracle's timed sample by the work of each step; it is
+    never an input or an expected value of a parity check."""
     import glob
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "trajectory_*.json"))):
         try:
@@ -187,7 +188,8 @@ def stored_trajectory(workload: str):
         except Exception:
             continue
         if rec.get("workload") == workload and rec.get("M_t"):
-            return np.asarray(rec["M_t"], dtype=np.int64), os.path.basename(path)
+            rows = rec.get("computed_rows") or rec["M_t"]
+            return np.asarray(rows, dtype=np.int64), os.path.basename(path)
     return None
 
 
@@ -660,7 +662,7 @@ def run_reference(args, rank: int, world: int):
     # GPU arm's cpu_baseline uses), else a linear decay from N as a stand-in
     got = stored_trajectory(cfg["workload"])
     if got is not None and len(got[0]) == T:
-        traj, traj_note = got[0], f"M_t trajectory from {got[1]}"
+        traj, traj_note = got[0], f"per-step rows from {got[1]}"
     else:
         traj = np.array([setup.batch * (setup.n_ctx - int(round(t * (setup.n_ctx - 1) / max(1, T))))
                          for t in range(T)])

@@ -256,3 +256,29 @@ def test_carry_line_arithmetic():
                    "frac_hbm": 0.0156}
     assert bench.carry_line({"ms": 0.0, "bytes": 0.0, "launches": 0}, 1,
                             {"hbm_gbs": 6400.0})["achieved_gbs"] is None
+
+
+def test_reference_arm_weighs_reuse_workloads_by_their_computed_rows():
+    """Under K/V reuse the reference arm's samples are weighted by the rows each
+    step computed: all rows at step 0 (a refresh step), and fewer than the
+    active rows in total (the two arrays come from two decodes of the run,
+    which may lock a few rows at different steps, so they are not compared
+    step by step)."""
+    sys.path.insert(0, ROOT)
+    import json as _json
+    import bench
+    import numpy as np
+    for kw in ({"kv_reuse": 2}, {"kv_reuse": 4}, {"kv_reuse": 4, "eps": 0.01},
+               {"kv_reuse": 4, "eps": 0.0}, {"kv_reuse": 4, "workload": "full8b", "eps": 0.05},
+               {"kv_reuse": 4, "workload": "full8b", "eps": 0.0}):
+        a = _bench_args(**kw)
+        setup = bench.setup_from_args(a)
+        got = bench.stored_trajectory(bench.workload_config(a, setup, 1)["workload"])
+        assert got is not None, kw
+        rows, name = got
+        rec = _json.load(open(os.path.join(ROOT, "profiles", name)))
+        m_t = np.asarray(rec["M_t"])
+        assert len(rows) == len(m_t) == setup.steps, (kw, name)
+        assert rows[0] == m_t[0] == setup.batch * setup.n_ctx
+        assert np.all((rows >= 0) & (rows <= setup.batch * setup.n_ctx))
+        assert rows.sum() < m_t.sum()
