@@ -48,7 +48,7 @@ typedef enum sl_status {
   SL_ERR_INVALID = 1,     /* bad argument: null pointer, size out of range, unsupported shape */
   SL_ERR_CUDA = 2,        /* a CUDA runtime call or launch failed */
   SL_ERR_OOM = 3,         /* device or pinned allocation failed */
-  SL_ERR_UNSUPPORTED = 4, /* valid request this build does not implement */
+  SL_ERR_UNSUPPORTED = 4, /* valid request the library does not implement */
   SL_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait and flagged it */
   SL_ERR_STATE = 6        /* call out of order (e.g. stepping a finished sampler) */
 } sl_status;
