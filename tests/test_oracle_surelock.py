@@ -471,3 +471,43 @@ def test_kv_reuse_rejects_the_scripted_schedule_and_the_no_cache_ablation():
         st = sl.init_state(cfg.shape, tok, msk)
         with pytest.raises(ValueError):
             sl.step(cfg.shape, w, st, c, 0)
+
+
+def test_semi_ar_blocks_fill_in_order():
+    """The semi-autoregressive schedule: each step unmasks exactly k positions,
+    all inside the current block; a block has no masked position left after its
+    steps, and no later block is touched before it is current (two blocks of 24
+    positions, 8 steps each, 3 per step)."""
+    import dataclasses
+    cfg, w, tok, msk = _tiny()
+    c = dataclasses.replace(cfg, block_len=24, steps=16, tokens_per_step=3)
+    c.validate()
+    st = sl.init_state(c.shape, tok, msk)
+    for t in range(c.steps):
+        lo, hi = c.block_bounds(t)
+        before = st.masked[0].copy()
+        sl.step(c.shape, w, st, c, t)
+        newly = np.nonzero(before & ~st.masked[0])[0]
+        assert len(newly) == c.tokens_per_step
+        assert np.all((newly >= lo) & (newly < hi))
+        if (t + 1) % c.steps_per_block == 0:
+            assert not st.masked[0, lo:hi].any()
+        assert st.masked[0, hi:].all()
+    assert not st.masked.any()
+
+
+def test_sequences_of_a_batch_are_independent():
+    """Two sequences stepped together give, bitwise, what each gives alone: the
+    gate quantile, the unmasking and the compaction are per sequence."""
+    import dataclasses
+    cfg, w, _, _ = _tiny()
+    c2 = dataclasses.replace(cfg, batch=2, gate_q=0.5, eps=0.05)
+    pr = wl.np_prompts(2, c2.prompt_len, c2.shape.vocab, c2.shape.mask_id, seed=11)
+    tok, msk = wl.initial_tokens(pr, c2.gen_len, c2.shape.mask_id)
+    both = sl.surelock_sampler(c2.shape, w, tok, msk, c2)
+    c1 = dataclasses.replace(c2, batch=1)
+    for b in range(2):
+        one = sl.surelock_sampler(c1.shape, w, tok[b:b + 1], msk[b:b + 1], c1)
+        np.testing.assert_array_equal(both[0][b], one[0][0])
+        np.testing.assert_array_equal(both[1][b], one[1][0])
+        np.testing.assert_array_equal(both[2][:, b], one[2][:, 0])
