@@ -265,6 +265,17 @@ def test_bf16_mini_decode_kv_reuse_teacher_forced(cuda_dev, head_fusion):
     assert stats["reused"] > 100, stats
 
 
+def test_bf16_mini_decode_kv_reuse_batch8_gate_only(cuda_dev):
+    """Reuse with eight sequences (per-sequence computed lists, gate quantiles
+    over each sequence's computed rows) and the gate-only ablation."""
+    setup = wl.SamplerSetup(MINI_BF16, "bf16", batch=8, prompt_len=40, gen_len=160, steps=40,
+                            block_len=32, tokens_per_step=4, eps=0.01, gate_q=0.5,
+                            gate_only=True, kv_reuse=2)
+    setup.validate()
+    stats, _ = _teacher_forced(setup, cuda_dev, 8, std=0.05)
+    assert stats["reused"] > 100 and stats["locks"] > 0, stats
+
+
 @pytest.mark.parametrize("R", [2, 4])
 def test_tiny_free_running_kv_reuse_matches_oracle(cuda_dev, R):
     """Whole decode with reuse: final tokens and active counts as the oracle's."""
